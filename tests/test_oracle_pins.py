@@ -1,0 +1,409 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Nothing here compares the oracle with itself: every check uses an independent
+fact -- a hand-built vector from the pages, a closed form, an invariant that a
+plausible mistake (dropped term, wrong sign, wrong index, transposed operand)
+breaks, a special case that reduces to a library routine, or an exact finite
+difference of a bilinear function.
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from qlora_quantized_linear_b200 import synthetic as syn
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bf16(x: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 bits (round to nearest even), via torch."""
+    return syn.bits_u16(torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16))
+
+
+# --------------------------------------------------------------------------
+# number formats
+# --------------------------------------------------------------------------
+def test_f16_conversion_matches_numpy_rne():
+    rng = np.random.default_rng(1)
+    xs = np.concatenate([
+        rng.standard_normal(4000).astype(np.float32) * 10.0 ** rng.integers(-9, 5, 4000),
+        np.array([65504.0, 65520.0, 65519.996, 2.0 ** -24, 2.0 ** -25, 3 * 2.0 ** -26,
+                  1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, -0.0, 0.0], np.float32),
+    ]).astype(np.float32)
+    with np.errstate(over="ignore"):
+        _f16_loop(xs)
+
+
+def _f16_loop(xs):
+    for x in xs:
+        assert oracle.f32_to_f16(float(x)) == int(np.float16(x).view(np.uint16)), x
+        h = np.float16(x).view(np.uint16)
+        if np.isfinite(np.float16(x)):
+            assert oracle.f16_to_f32(int(h)) == float(np.float16(x))
+
+
+def test_bf16_widening_matches_torch():
+    x = torch.randn(1000, dtype=torch.float32).to(torch.bfloat16)
+    assert np.array_equal(oracle.bf16_to_f32(syn.bits_u16(x)), x.float().numpy())
+
+
+# --------------------------------------------------------------------------
+# packing -- hand-built vectors from the bitsandbytes guide's packing rule
+# --------------------------------------------------------------------------
+def _golden_packing():
+    rows = []
+    with open(os.path.join(GOLDEN, "packing.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            b, codes, packed = [p.strip() for p in line.split(";")]
+            rows.append((int(b), [int(c) for c in codes.split()], bytes.fromhex(packed.replace(" ", ""))))
+    return rows
+
+
+@pytest.mark.parametrize("bits,codes,packed", _golden_packing())
+def test_pack_golden(bits, codes, packed):
+    c = np.array([codes], np.uint8)
+    got = oracle.pack(c, bits)
+    assert bytes(got.ravel()) == packed
+    assert np.array_equal(oracle.unpack(got, len(codes), bits), c)
+
+
+def test_pack_roundtrip_random():
+    rng = np.random.default_rng(2)
+    for bits in (2, 4):
+        c = rng.integers(0, 1 << bits, (7, 256), dtype=np.uint8)
+        assert np.array_equal(oracle.unpack(oracle.pack(c, bits), 256, bits), c)
+
+
+# --------------------------------------------------------------------------
+# storage accounting -- closed forms from the pages
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("bits,group,expect", [(4, 128, 4.25), (2, 64, 2.5)])
+def test_minmax_bits_per_param(bits, group, expect):
+    # GreenBit article, 模型量化 (1): INT4 g128 and INT2 g64 with a 16-bit scale
+    # and a 16-bit zero per group -> b + 32/g bits per parameter.
+    n, k = 4, 512
+    W = syn.bits_u16(syn.normal_bf16((n, k), 0.02, 0))
+    codes, scale, zero = oracle.minmax_quantize(W, bits, group)
+    packed = oracle.pack(codes, bits)
+    total_bits = 8 * (packed.nbytes + scale.nbytes + zero.nbytes)
+    assert total_bits / (n * k) == expect
+    # 4x compression of the 16-bit weight before the group overhead (GreenBit
+    # article, 模型量化: 4-bit vs FP16), 16/4.25 with it.
+    assert 16 * n * k / (8 * packed.nbytes) == 16 / bits
+
+
+def test_double_quant_saves_0_373_bits():
+    # QLoRA explainer, 关键技术细节 2 / 结论: double quantization saves about
+    # 0.37 bit per parameter.  fp32 absmax per 64 weights -> 8-bit per 64 plus
+    # an fp32 scale per 256 absmax values.
+    n, k = 64, 256 * 64  # 256 absmax blocks per row
+    nb = n * k // 64
+    absmax = np.abs(np.random.default_rng(3).standard_normal(nb)).astype(np.float32) + 0.1
+    q8, s2, off, exact = oracle.double_quant(absmax)
+    before = 32 * absmax.size
+    after = 8 * q8.size + 32 * s2.size
+    saved = (before - after) / (n * k)
+    assert saved == 32 / 64 - 8 / 64 - 32 / (64 * 256) == 0.373046875
+    assert round(saved, 2) == 0.37
+
+
+# --------------------------------------------------------------------------
+# MinMax quantizer
+# --------------------------------------------------------------------------
+def _mixed_weight(n, k, seed):
+    w = syn.weight_bf16(n, k, 0.02, seed, outlier_frac=0.01, outlier_scale=20.0).float()
+    # rows with all-positive and all-negative groups, a constant group and a
+    # zero row, so that zero points outside [0, Q] and degenerate groups occur
+    w[1] = w[1].abs() + 0.05
+    w[2] = -w[2].abs() - 0.05
+    w[3, :128] = 0.3
+    w[4] = 0.0
+    return syn.bits_u16(w.to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("bits,group", [(4, 128), (2, 64)])
+def test_minmax_roundtrip_bound(bits, group):
+    n, k = 16, 512
+    Q = (1 << bits) - 1
+    W = _mixed_weight(n, k, 5)
+    codes, scale, zero = oracle.minmax_quantize(W, bits, group)
+    assert codes.max() <= Q
+    What = oracle.minmax_dequantize(oracle.pack(codes, bits), scale, zero, k, bits, group)
+    w = oracle.bf16_to_f32(W).reshape(n, k // group, group).astype(np.float64)
+    sf = np.array([oracle.f16_to_f32(int(h)) for h in scale.ravel()]).reshape(n, k // group, 1)
+    err = np.abs(w - What.reshape(n, k // group, group))
+    # |w - w_hat| <= scale/2 inside [min, max]; the fp16 rounding of the scale
+    # can shorten the top of the grid by at most Q * scale * 2^-11, and the fp32
+    # division adds a relative 2^-24.
+    bound = sf * (0.5 + Q * 2.0 ** -11) + 2.0 ** -23 * np.abs(w) + 1e-30
+    assert np.all(err <= bound), float((err - bound).max())
+    # the group minimum maps to code 0 and the maximum to Q (or within one
+    # step when the fp16 scale shortened the grid)
+    cg = codes.reshape(n, k // group, group)
+    for i in range(n):
+        for g in range(k // group):
+            if w[i, g].max() == w[i, g].min():
+                continue
+            assert cg[i, g][w[i, g].argmin()] == 0
+            assert cg[i, g][w[i, g].argmax()] >= Q - 1
+
+
+def test_minmax_scale_zero_exact_rational_crosscheck():
+    """Scale and zero of every group, recomputed with exact rationals and
+    numpy's float16: pins which elements form a group (along k) and the order
+    fp32 range -> /Q -> fp16 -> zero = rint(-min/scale)."""
+    n, k, bits, group = 6, 256, 4, 128
+    W = _mixed_weight(n, k, 11)
+    codes, scale, zero = oracle.minmax_quantize(W, bits, group)
+    w = oracle.bf16_to_f32(W).reshape(n, k // group, group)
+    for i in range(n):
+        for g in range(k // group):
+            mn, mx = float(w[i, g].min()), float(w[i, g].max())
+            r = np.float32(Fraction(mx) - Fraction(mn))   # exact difference fits fp64
+            s32 = np.float32(r) / np.float32(15)          # IEEE fp32 division
+            s16 = np.float16(s32)
+            if r == 0 or s16 == 0:
+                s16 = np.float16(1.0)
+            assert int(s16.view(np.uint16)) == int(scale[i, g])
+            # IEEE fp32 negation and division (numpy float32), keeping the
+            # sign of zero: -(+0)/s = -0 is stored as fp16 -0
+            z = np.float32(-(np.float32(mn) + np.float32(0.0))) / np.float32(s16)
+            zr = np.float16(np.rint(z))
+            assert int(zr.view(np.uint16)) == int(zero[i, g]), (i, g)
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_minmax_grid_values_roundtrip_exactly(bits):
+    """Every representable grid value (q - z) * s re-quantizes to q, with the
+    same scale and zero recovered (GreenBit article, 模型量化 (1))."""
+    Q = (1 << bits) - 1
+    group = 128 if bits == 4 else 64
+    rng = np.random.default_rng(7)
+    n, k = 8, 4 * group
+    q = rng.integers(0, Q + 1, (n, k)).astype(np.int64)
+    qg = q.reshape(n, k // group, group)
+    qg[:, :, 0] = 0
+    qg[:, :, 1] = Q
+    z = rng.integers(0, Q + 1, (n, k // group))
+    sf = (rng.integers(1, 8, (n, k // group)) * 2.0 ** rng.integers(-10, -4, (n, k // group)))
+    w = (qg - z[:, :, None]) * sf[:, :, None]          # exact in bf16 (<= 7 bits)
+    W = _bf16(w.reshape(n, k).astype(np.float32))
+    assert np.array_equal(oracle.bf16_to_f32(W).astype(np.float64), w.reshape(n, k))
+    codes, scale, zero = oracle.minmax_quantize(W, bits, group)
+    assert np.array_equal(codes.astype(np.int64), q)
+    assert np.array_equal(np.array([oracle.f16_to_f32(int(h)) for h in scale.ravel()]), sf.ravel())
+    assert np.array_equal(np.array([oracle.f16_to_f32(int(h)) for h in zero.ravel()]), z.ravel())
+    What = oracle.minmax_dequantize(oracle.pack(codes, bits), scale, zero, k, bits, group)
+    assert np.array_equal(What.astype(np.float64), w.reshape(n, k))
+
+
+def test_minmax_constant_and_zero_groups():
+    n, k = 2, 128
+    w = np.zeros((n, k), np.float32)
+    w[0] = 3.0
+    W = _bf16(w)
+    codes, scale, zero = oracle.minmax_quantize(W, 4, 128)
+    assert oracle.f16_to_f32(int(scale[0, 0])) == 1.0 and oracle.f16_to_f32(int(scale[1, 0])) == 1.0
+    What = oracle.minmax_dequantize(oracle.pack(codes, 4), scale, zero, k, 4, 128)
+    assert np.all(What[0] == 3.0) and np.all(What[1] == 0.0)
+
+
+def test_minmax_signed_zero_independent_of_order():
+    w = np.zeros((2, 128), np.float32)
+    w[0, 0] = -0.0
+    w[1, 5] = -0.0
+    w[:, 64] = 1.0
+    W = _bf16(w)
+    _, scale, zero = oracle.minmax_quantize(W, 4, 128)
+    assert scale[0, 0] == scale[1, 0] and zero[0, 0] == zero[1, 0]
+
+
+def test_minmax_rejects_nonfinite():
+    w = np.zeros((1, 128), np.float32)
+    w[0, 3] = np.inf
+    with pytest.raises(ValueError):
+        oracle.minmax_quantize(_bf16(w), 4, 128)
+
+
+# --------------------------------------------------------------------------
+# codebook quantizer
+# --------------------------------------------------------------------------
+def test_codebook_uniform_grid_reduces_to_round_to_nearest():
+    """With the uniform table c_j = (j - 8)/8, the nearest-entry rule is
+    round-to-nearest on x*8 with ties to the lower entry, clamped."""
+    cb = ((np.arange(16) - 8) / 8).astype(np.float32)
+    n, k = 16, 256
+    W = syn.bits_u16(syn.normal_bf16((n, k), 0.02, 13))
+    codes, absmax = oracle.codebook_quantize(W, cb)
+    w = oracle.bf16_to_f32(W).reshape(-1, 64)
+    a = np.abs(w).max(axis=1)
+    assert np.array_equal(absmax, a)
+    x = (w / a[:, None]).astype(np.float32)          # fp32 division, as defined
+    d = x.astype(np.float64) * 8                      # exact
+    expect = np.clip(np.ceil(d - 0.5) + 8, 0, 15)     # tie -> lower index
+    assert np.array_equal(codes.reshape(-1, 64), expect.astype(np.uint8))
+
+
+def test_codebook_entries_map_to_themselves():
+    """Idempotence: w = c_j * a is quantized to code j (a = block absmax)."""
+    cb = np.array([-1, -0.75, -0.5, -0.375, -0.25, -0.125, -0.0625, 0,
+                   0.0625, 0.125, 0.1875, 0.25, 0.375, 0.5, 0.75, 1], np.float32)
+    rng = np.random.default_rng(17)
+    n, k = 8, 128
+    j = rng.integers(0, 16, (n * k // 64, 64))
+    j[:, 0] = 15  # |c| = 1 in every block, so absmax = a
+    a = 2.0 ** rng.integers(-8, -2, (n * k // 64, 1))
+    w = (cb[j] * a).astype(np.float32).reshape(n, k)
+    W = _bf16(w)
+    codes, absmax = oracle.codebook_quantize(W, cb)
+    assert np.array_equal(codes.reshape(-1, 64), j.astype(np.uint8))
+    assert np.array_equal(absmax, a.ravel().astype(np.float32))
+
+
+def test_codebook_error_bound_and_zero_block():
+    cb = syn.codebook_normal16()
+    n, k = 32, 256
+    wt = syn.weight_bf16(n, k, 0.015, 19).float()
+    wt[3, :64] = 0.0
+    W = syn.bits_u16(wt.to(torch.bfloat16))
+    codes, absmax = oracle.codebook_quantize(W, cb)
+    zero_idx = int(np.where(cb == 0)[0][0])
+    assert np.all(codes[3, :64] == zero_idx) and absmax[3 * (k // 64)] == 0
+    What = oracle.codebook_dequantize(oracle.pack(codes, 4), absmax, cb, n, k)
+    w = oracle.bf16_to_f32(W).astype(np.float64)
+    maxgap = np.diff(cb.astype(np.float64)).max()
+    a = np.repeat(absmax.astype(np.float64), 64).reshape(n, k)
+    assert np.all(np.abs(w - What) <= a * (maxgap / 2) * (1 + 1e-6) + 1e-30)
+
+
+def test_codebook_rejects_bad_tables():
+    W = syn.bits_u16(syn.normal_bf16((1, 64), 1.0, 0))
+    cb = syn.codebook_normal16()
+    with pytest.raises(ValueError):
+        oracle.codebook_quantize(W, cb[::-1].copy())          # not sorted
+    bad = cb.copy()
+    bad[7] = 1e-3                                             # no exact zero
+    with pytest.raises(ValueError):
+        oracle.codebook_quantize(W, bad)
+
+
+# --------------------------------------------------------------------------
+# double quantization
+# --------------------------------------------------------------------------
+def test_double_quant_properties():
+    rng = np.random.default_rng(23)
+    nb = 256 * 5 + 77                               # ragged last block
+    absmax = _bf16((np.abs(rng.standard_normal(nb)) * 0.03 + 0.01).astype(np.float32))
+    absmax = oracle.bf16_to_f32(absmax)             # absmax values are bf16 values
+    q8, s2, off, exact = oracle.double_quant(absmax)
+    assert exact
+    # offset = mean, rounded once from fp64 (the fp64 sum is exact here)
+    mean = Fraction(math.fsum(float(a) for a in absmax)) / nb
+    assert np.float32(off) == np.float32(float(np.float64(float(mean))))
+    ah = oracle.double_dequant(q8, s2, off)
+    for b in range(len(s2)):
+        lo, hi = 256 * b, min(256 * b + 256, nb)
+        c = (absmax[lo:hi] - off).astype(np.float32)
+        assert s2[b] == np.abs(c).max()
+        assert np.abs(q8[lo:hi]).max() == 127          # the block extreme
+        err = np.abs(ah[lo:hi].astype(np.float64) - absmax[lo:hi])
+        assert np.all(err <= s2[b] / 254 + 4 * np.spacing(np.float32(abs(off) + s2[b])))
+    assert q8.dtype == np.int8 and np.abs(q8.astype(int)).max() <= 127
+
+
+def test_double_quant_flags_inexact_sum():
+    absmax = np.array([1.0, 2.0 ** -60, 3.0], np.float32)
+    *_, exact = oracle.double_quant(absmax, allow_inexact=True)
+    assert not exact
+
+
+# --------------------------------------------------------------------------
+# quantized linear layer with LoRA
+# --------------------------------------------------------------------------
+def _tiny_problem(m=5, n=24, k=256, r=4, seed=29):
+    X = syn.bits_u16(syn.normal_bf16((m, k), 1.0, seed))
+    Wb = syn.bits_u16(syn.normal_bf16((n, k), 0.02, seed + 1))
+    codes, scale, zero = oracle.minmax_quantize(Wb, 4, 128)
+    What = oracle.minmax_dequantize(oracle.pack(codes, 4), scale, zero, k, 4, 128)
+    A = syn.bits_u16(syn.normal_bf16((r, k), 0.01, seed + 2))
+    B = syn.bits_u16(syn.normal_bf16((n, r), 0.01, seed + 3))
+    dY = syn.bits_u16(syn.normal_bf16((m, n), 0.1, seed + 4))
+    return X, What, A, B, dY, (codes, scale, zero)
+
+
+def test_rank0_reduces_to_matmul():
+    X, What, *_ = _tiny_problem()
+    Y, T, Yb = oracle.linear_fwd(X, What)
+    ref = oracle.bf16_to_f32(X).astype(np.float64) @ What.astype(np.float64).T
+    np.testing.assert_allclose(Y, ref, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(Yb, np.abs(oracle.bf16_to_f32(X)).astype(np.float64)
+                               @ np.abs(What.astype(np.float64)).T, rtol=1e-12)
+
+
+def test_zero_weight_leaves_only_adapter_term():
+    X, What, A, B, _, _ = _tiny_problem()
+    s = 2.0
+    Y, T, _ = oracle.linear_fwd(X, np.zeros_like(What), A, B, s)
+    x = oracle.bf16_to_f32(X).astype(np.float64)
+    a = oracle.bf16_to_f32(A).astype(np.float64)
+    b = oracle.bf16_to_f32(B).astype(np.float64)
+    np.testing.assert_allclose(T, x @ a.T, rtol=1e-12, atol=1e-18)
+    np.testing.assert_allclose(Y, s * (x @ a.T) @ b.T, rtol=1e-12, atol=1e-18)
+
+
+def test_sampled_forward_matches_full():
+    X, What, A, B, _, (codes, scale, zero) = _tiny_problem()
+    s = 2.0
+    Y, _, Yb = oracle.linear_fwd(X, What, A, B, s)
+    rows = np.array([0, 4, 2, 3]); cols = np.array([0, 23, 7, 11])
+    Ys, Ybs = oracle.linear_fwd_sampled_minmax(X, oracle.pack(codes, 4), scale, zero, What.shape[0],
+                                               What.shape[1], 4, 128, rows, cols, A, B, s)
+    np.testing.assert_allclose(Ys, Y[rows, cols], rtol=1e-13, atol=1e-16)
+    np.testing.assert_allclose(Ybs, Yb[rows, cols], rtol=1e-13)
+
+
+def _loss(X, What, A, B, s, dY):
+    Y, _, _ = oracle.linear_fwd(X, What, A, B, s)
+    return float(np.sum(oracle.bf16_to_f32(dY).astype(np.float64) * Y))
+
+
+def _bump(bits_arr, idx, new_val):
+    out = bits_arr.copy()
+    out[idx] = _bf16(np.array([new_val], np.float32))[0]
+    return out
+
+
+def test_backward_products_by_exact_finite_differences():
+    """L = sum(dY * Y) is linear in each of X, A and B separately, so a finite
+    difference over one element is exact (up to fp64 rounding).  This pins
+    dX = dY W + s (dY B) A, dA = s (dY B)^T X and dB = s dY^T (X A^T) against
+    the forward definition Y = X W^T + s (X A^T) B^T."""
+    X, What, A, B, dY, _ = _tiny_problem()
+    s = 2.0
+    dX, U, _ = oracle.linear_bwd(dY, What, A, B, s)
+    dA, dB, _, _ = oracle.lora_grads(X, dY, A, B, s)
+    L0 = _loss(X, What, A, B, s, dY)
+    checks = 0
+    for arr_name, idx in [("X", (0, 3)), ("X", (4, 200)), ("X", (2, 129)),
+                          ("A", (0, 5)), ("A", (3, 255)), ("B", (0, 0)), ("B", (23, 3)), ("B", (11, 2))]:
+        arr = {"X": X, "A": A, "B": B}[arr_name]
+        old = float(oracle.bf16_to_f32(arr[idx]))
+        new = float(oracle.bf16_to_f32(_bf16(np.array([old * 1.5 + 0.25], np.float32)))[0])
+        h = new - old
+        args = dict(X=X, A=A, B=B)
+        args[arr_name] = _bump(arr, idx, new)
+        fd = (_loss(args["X"], What, args["A"], args["B"], s, dY) - L0) / h
+        grad = {"X": dX, "A": dA, "B": dB}[arr_name][idx]
+        assert abs(fd - grad) <= 1e-9 * (abs(grad) + 1e-6), (arr_name, idx, fd, grad)
+        checks += 1
+    assert checks == 8
+    # U = dY B (shared by dX and dA)
+    np.testing.assert_allclose(U, oracle.bf16_to_f32(dY).astype(np.float64)
+                               @ oracle.bf16_to_f32(B).astype(np.float64), rtol=1e-12, atol=1e-18)
