@@ -1,0 +1,204 @@
+/*
+ * lbq.h -- C ABI of the low-bit quantized linear layer library for B200
+ * (sm_100a).  All entry points are `extern "C"`, take plain pointers and sizes,
+ * and launch asynchronously on the caller's CUDA stream.
+ *
+ * Sources (web pages, cited by title and section):
+ *  - GreenBit.AI article "只需单卡RTX 3090，低比特量化训练就能实现LLaMA-3 8B全参微调",
+ *    section 模型量化, step (1): group-wise MinMax quantizer; INT4 with group
+ *    size 128 and INT2 with group size 64; layer-mix and channel-mix layouts.
+ *  - bitsandbytes FSDP-QLoRA guide, section 量化数据的存储 (quant_storage):
+ *    two 4-bit codes per byte with the first code in the high nibble; NF4/FP4
+ *    codebooks; nested quantization of absmax; weights are dequantized to the
+ *    compute dtype (bf16) inside the kernels.
+ *  - QLoRA explainer, sections QLoRA技术原理 / 关键技术细节 / 结论: 4-bit
+ *    NormalFloat codebook, double quantization of the scale factors and their
+ *    offset (about 0.37 bit per parameter saved), and backpropagation through
+ *    the frozen 4-bit weight into the low-rank adapters.
+ *
+ * Conventions
+ *  - W is [n out, k in] row-major; quantization groups run along k.
+ *  - bf16 and fp16 data are passed as their 16-bit patterns (uint16_t / void*).
+ *  - Every pointer in lbq_qweight and every data pointer argument is DEVICE
+ *    memory owned by the caller.  The library allocates nothing; it never
+ *    frees, retains or reallocates caller memory.
+ *  - Device pointers must be 16-byte aligned (LBQ_EALIGN otherwise); sizes
+ *    must satisfy the per-function constraints (LBQ_EINVAL otherwise).
+ *  - Arguments are validated on the host before anything is launched; a
+ *    rejected call launches nothing.  Launch failures are reported as
+ *    LBQ_ECUDA.  Kernels that wait on a device-side condition give up after a
+ *    bounded number of polls and record LBQ_ETIMEOUT in the device status word,
+ *    read with lbq_device_status().  Nothing aborts the process.
+ *  - Results are deterministic: the same inputs give the same bits.
+ */
+#ifndef LBQ_H
+#define LBQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Compatible with cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* lbq_stream_t;
+
+typedef enum {
+    LBQ_OK = 0,
+    LBQ_EINVAL = 1,        /* bad shape, bit width, group, scheme or NULL pointer */
+    LBQ_EALIGN = 2,        /* a device pointer is not 16-byte aligned */
+    LBQ_EUNSUPPORTED = 3,  /* valid request that this build does not implement */
+    LBQ_ECUDA = 4,         /* a CUDA runtime call or launch failed */
+    LBQ_ETIMEOUT = 5,      /* a device-side wait gave up (see lbq_device_status) */
+    LBQ_EWORKSPACE = 6     /* workspace missing or smaller than the query said */
+} lbq_status;
+
+typedef enum {
+    LBQ_MINMAX_ASYM = 0,   /* group-wise asymmetric MinMax, INT4 g128 / INT2 g64 */
+    LBQ_CODEBOOK4 = 1      /* 4-bit codebook with per-64 absmax (NF4-style) */
+} lbq_scheme;
+
+/*
+ * A quantized weight.  All pointers are caller-owned DEVICE memory.
+ *
+ * LBQ_MINMAX_ASYM (GreenBit article, 模型量化 (1)):
+ *   bits in {4, 2}, group in {128 (bits 4), 64 (bits 2)}, k % group == 0,
+ *   k % 64 == 0.  For each row and group of `group` consecutive k:
+ *     scale = fp16(fp32(max - min) / Q), Q = 2^bits - 1 (1.0 if that is 0),
+ *     zero  = fp16(rint(-min / scale)),
+ *     code  = clamp(rint(w / scale) + zero, 0, Q)            (rint: half-even)
+ *   packed [n, k*bits/8] u8: codes in order, first code in the high bits.
+ *   scale, zero [n, k/group] fp16 bit patterns.
+ *   Dequantized value: (code - zero) * scale.
+ *
+ * LBQ_CODEBOOK4 (QLoRA explainer, 关键技术细节 1; bitsandbytes guide, nf4/fp4):
+ *   bits 4, group 64 (blocks of 64 consecutive elements of the row-major W),
+ *   k % 64 == 0.  codebook: 16 sorted fp32 values in [-1, 1] that include an
+ *   exact 0 (device memory, read only).  absmax [n*k/64] fp32 = max |w| per
+ *   block; code = index of the entry nearest to fp32(w / absmax) (the lower
+ *   index on a tie; the 0 entry when absmax is 0).  packed [n, k/2] u8 as above.
+ *   Dequantized value: codebook[code] * absmax.
+ *   With double_quant != 0 (QLoRA explainer, 结论; bitsandbytes guide, nested
+ *   absmax): offset = fp32(fp64 sum of absmax / (n*k/64)); per block of 256
+ *   absmax values s2 = max |absmax - offset| and
+ *   q8 = clamp(rint(fp32(fp32((absmax - offset) / s2) * 127)), -127, 127);
+ *   absmax' = fp32(fp32(fp32(q8 / 127) * s2) + offset) replaces absmax in the
+ *   dequantized value.  absmax_q8 [n*k/64] i8, absmax_s2 [ceil(n*k/64/256)]
+ *   fp32, absmax_offset [1] fp32.  absmax is still required: lbq_quantize
+ *   writes the first-level values there.  The offset is reproducible bit for
+ *   bit whenever the fp64 sum of the absmax values is exact, which holds when
+ *   they span less than 2^(45 - log2(n*k/64)) in magnitude.
+ */
+typedef struct {
+    int32_t n, k;
+    int32_t bits, group;
+    int32_t scheme;         /* lbq_scheme */
+    int32_t double_quant;   /* CODEBOOK4 only */
+    uint8_t* packed;
+    uint16_t* scale;        /* MINMAX */
+    uint16_t* zero;         /* MINMAX */
+    float* absmax;          /* CODEBOOK4 */
+    int8_t* absmax_q8;      /* CODEBOOK4 + double_quant */
+    float* absmax_s2;       /* CODEBOOK4 + double_quant */
+    float* absmax_offset;   /* CODEBOOK4 + double_quant */
+    const float* codebook;  /* CODEBOOK4 */
+} lbq_qweight;
+
+/*
+ * Channel-mix layout (GreenBit article, 模型量化 (1)): inside one matrix some
+ * output channels are INT4 g128 and the rest INT2 g64.  The rows are stored as
+ * two contiguous MinMax matrices, `hi` (INT4) then `lo` (INT2), with the same
+ * k; perm[i] (0 <= i < hi.n + lo.n) is the original output channel of stored
+ * row i (rows of `hi` first).  Y is produced in the original channel order.
+ * hi.n and lo.n must be multiples of 128.
+ */
+typedef struct {
+    lbq_qweight hi;
+    lbq_qweight lo;
+    const int32_t* perm;    /* device, hi.n + lo.n entries, a permutation */
+} lbq_qweight_mix;
+
+/* Human-readable name of a status code (static string). */
+const char* lbq_status_string(lbq_status s);
+
+/*
+ * Quantize and pack W (bf16 [q->n, q->k], device) into q.  Fills packed and
+ * scale/zero (MINMAX) or absmax (+ q8, s2, offset with double_quant)
+ * (CODEBOOK4).  CODEBOOK4 with double_quant needs a workspace of
+ * lbq_quantize_workspace_size(q) bytes (device, any contents); every other
+ * case needs none (workspace may be NULL).
+ */
+size_t lbq_quantize_workspace_size(const lbq_qweight* q);
+lbq_status lbq_quantize(const void* W_bf16, lbq_qweight* q, void* workspace,
+                        size_t workspace_bytes, lbq_stream_t stream);
+
+/*
+ * Dequantize q into W_f32 [q->n, q->k] fp32 (device).  MINMAX values are exact
+ * ((code - zero) * scale is one fp32 product); CODEBOOK4 values are
+ * fp32(codebook[code] * absmax) with absmax' when double_quant is set.
+ */
+lbq_status lbq_dequantize(const lbq_qweight* q, float* W_f32,
+                          lbq_stream_t stream);
+
+/*
+ * Forward of the quantized linear layer with a low-rank adapter (QLoRA
+ * explainer, QLoRA技术原理):
+ *   T = X A^T  [m, rank]                         (fp32, written to T_save)
+ *   Y = X W^T + s T B^T  [m, n]                  (fp32)
+ * X bf16 [m, k], A bf16 [rank, k], B bf16 [n, rank], all row-major device.
+ * rank == 0 (A, B, T_save may be NULL) is the plain dequantize-GEMM.
+ * 1 <= rank <= 64 needs T_save.  m >= 1.  The weight is dequantized to bf16
+ * (the compute dtype) inside the kernel and products accumulate in fp32.
+ * workspace: lbq_linear_fwd_workspace_size(m, q, rank) bytes of device memory
+ * (contents ignored); NULL is accepted when that size is 0.
+ */
+size_t lbq_linear_fwd_workspace_size(int m, const lbq_qweight* q, int rank);
+lbq_status lbq_linear_fwd(const void* X, int m, const lbq_qweight* q,
+                          const void* A, const void* B, int rank, float s,
+                          float* Y, float* T_save, void* workspace,
+                          size_t workspace_bytes, lbq_stream_t stream);
+
+/* The same forward for a channel-mix weight; Y columns in original order. */
+size_t lbq_linear_fwd_mix_workspace_size(int m, const lbq_qweight_mix* q,
+                                         int rank);
+lbq_status lbq_linear_fwd_mix(const void* X, int m, const lbq_qweight_mix* q,
+                              const void* A, const void* B, int rank, float s,
+                              float* Y, float* T_save, void* workspace,
+                              size_t workspace_bytes, lbq_stream_t stream);
+
+/*
+ * Input gradient (QLoRA explainer, QLoRA技术原理: gradients pass through the
+ * frozen quantized weight):
+ *   U  = dY B  [m, rank]                         (fp32, written to U_save)
+ *   dX = dY W + s U A  [m, k]                    (fp32)
+ * dY bf16 [m, n].  Same rank, workspace and layout rules as lbq_linear_fwd.
+ */
+size_t lbq_linear_bwd_workspace_size(int m, const lbq_qweight* q, int rank);
+lbq_status lbq_linear_bwd(const void* dY, int m, const lbq_qweight* q,
+                          const void* A, const void* B, int rank, float s,
+                          float* dX, float* U_save, void* workspace,
+                          size_t workspace_bytes, lbq_stream_t stream);
+
+/*
+ * Adapter gradients (the only trainable parameters; QLoRA explainer,
+ * QLoRA技术原理):
+ *   dA = s U^T X  [rank, k]       dB = s dY^T T  [n, rank]      (fp32)
+ * X bf16 [m, k], dY bf16 [m, n], T = X A^T and U = dY B fp32 [m, rank] as
+ * saved by lbq_linear_fwd / lbq_linear_bwd.  1 <= rank <= 64.
+ */
+lbq_status lbq_lora_grads(const void* X, const void* dY, int m, int n, int k,
+                          const float* T, const float* U, int rank, float s,
+                          float* dA, float* dB, lbq_stream_t stream);
+
+/*
+ * Device status word: the OR of the LBQ_ETIMEOUT-style flags recorded by
+ * kernels since the last call (0 when none).  Synchronizes the current device,
+ * then clears the word.  Returns LBQ_ECUDA if the read itself fails.
+ */
+lbq_status lbq_device_status(uint32_t* flags);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LBQ_H */

@@ -1,0 +1,478 @@
+// lbq.cu -- the C ABI (include/lbq.h): argument validation, tensor-map setup,
+// tile and split selection, and kernel launches.  One translation unit holds
+// every kernel so that the device status word is a single object.
+#include <mutex>
+
+#include "dqgemm.cuh"
+#include "dqgemm_bwd.cuh"
+#include "lora.cuh"
+#include "quantize.cuh"
+
+using namespace lbq;
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// small host helpers
+// ---------------------------------------------------------------------------
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+
+lbq_status last_launch() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? LBQ_OK : LBQ_ECUDA;
+}
+
+int sm_count() {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms > 0 ? sms : 148;
+}
+
+// cuTensorMapEncodeTiled, fetched from the driver through the runtime so that
+// the library needs no link-time dependency on libcuda.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D row-major tensor [rows, cols] of `esize`-byte elements, box [brows, bcols].
+bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esize, uint64_t rows,
+                 uint64_t cols, uint32_t brows, uint32_t bcols, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * static_cast<uint64_t>(esize)};
+    cuuint32_t box[2] = {bcols, brows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// weight descriptor checks
+// ---------------------------------------------------------------------------
+lbq_status check_qweight(const lbq_qweight* q, bool need_data) {
+    if (!q) return LBQ_EINVAL;
+    if (q->n < 1 || q->k < 64 || q->k % 64 != 0) return LBQ_EINVAL;
+    if (q->scheme == LBQ_MINMAX_ASYM) {
+        if (!((q->bits == 4 && q->group == 128) || (q->bits == 2 && q->group == 64))) return LBQ_EUNSUPPORTED;
+        if (q->k % q->group != 0) return LBQ_EINVAL;
+        if (need_data && (!q->packed || !q->scale || !q->zero)) return LBQ_EINVAL;
+        if (need_data && (!aligned16(q->packed) || !aligned16(q->scale) || !aligned16(q->zero))) return LBQ_EALIGN;
+    } else if (q->scheme == LBQ_CODEBOOK4) {
+        if (q->bits != 4 || q->group != 64) return LBQ_EUNSUPPORTED;
+        if (need_data && (!q->packed || !q->absmax || !q->codebook)) return LBQ_EINVAL;
+        if (need_data && (!aligned16(q->packed) || !aligned16(q->absmax) || !aligned16(q->codebook)))
+            return LBQ_EALIGN;
+        if (q->double_quant) {
+            if (need_data && (!q->absmax_q8 || !q->absmax_s2 || !q->absmax_offset)) return LBQ_EINVAL;
+            if (need_data && (!aligned16(q->absmax_q8) || !aligned16(q->absmax_s2) || !aligned16(q->absmax_offset)))
+                return LBQ_EALIGN;
+        }
+    } else {
+        return LBQ_EUNSUPPORTED;
+    }
+    return LBQ_OK;
+}
+
+int kind_of(const lbq_qweight* q) {
+    if (q->scheme == LBQ_CODEBOOK4) return kCode4;
+    return q->bits == 4 ? kInt4 : kInt2;
+}
+
+// ---------------------------------------------------------------------------
+// forward GEMM planning
+// ---------------------------------------------------------------------------
+constexpr int kCodebookQuantizeMaxCtas = 4096;
+
+int token_tile(int m) { return m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : 128; }
+
+struct Plan {
+    int nt;          // token tile
+    int tiles;       // output tiles (rows x token tiles)
+    int nsplit;      // K splits
+    int per_split;   // reduction blocks per split
+    size_t partial_bytes, counter_bytes;
+    size_t workspace() const { return nsplit > 1 ? partial_bytes + counter_bytes : 0; }
+};
+
+Plan plan_gemm(int m, int64_t out_rows, int64_t red_blocks, int sms) {
+    Plan pl;
+    pl.nt = token_tile(m);
+    pl.tiles = static_cast<int>(cdiv(out_rows, 128) * cdiv(m, pl.nt));
+    const int target = 2 * sms;
+    pl.nsplit = 1;
+    if (pl.tiles < target) pl.nsplit = static_cast<int>(std::min<int64_t>(red_blocks, cdiv(target, pl.tiles)));
+    pl.per_split = static_cast<int>(cdiv(red_blocks, pl.nsplit));
+    pl.nsplit = static_cast<int>(cdiv(red_blocks, pl.per_split));
+    pl.partial_bytes = round_up(static_cast<size_t>(pl.nsplit) * m * out_rows * sizeof(float), 256);
+    pl.counter_bytes = round_up(static_cast<size_t>(pl.tiles) * sizeof(uint32_t), 256);
+    return pl;
+}
+
+template <int NT>
+struct FwdCfg {
+    static constexpr int kStages = NT <= 32 ? 8 : NT <= 64 ? 6 : 4;
+    static constexpr int kAStages = 2;
+};
+
+template <int NT, int KIND>
+lbq_status launch_fwd_nt(const FwdParams& p, const void* X, int m, int64_t k, const uint8_t* packed, int nrows,
+                         int nsplit, cudaStream_t st) {
+    constexpr int S = FwdCfg<NT>::kStages, AS = FwdCfg<NT>::kAStages;
+    constexpr int WB = WeightTile<KIND>::kRowBytes;
+    using L = GemmSmem<NT, S, AS, 128 * WB>;
+    auto kern = dqgemm_fwd_kernel<NT, KIND, S, AS>;
+    const size_t smem = L::total(p.rank_pad);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+        return LBQ_ECUDA;
+    CUtensorMap tmX, tmW;
+    if (!make_map_2d(&tmX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, m, k, NT, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return LBQ_ECUDA;
+    if (!make_map_2d(&tmW, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, nrows, k * (KIND == kInt2 ? 2 : 4) / 8, 128, WB,
+                     WB == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE))
+        return LBQ_ECUDA;
+    dim3 grid(static_cast<unsigned>(cdiv(nrows, 128)), static_cast<unsigned>(cdiv(m, NT)), static_cast<unsigned>(nsplit));
+    kern<<<grid, 192, smem, st>>>(tmX, tmW, p);
+    return last_launch();
+}
+
+template <int KIND>
+lbq_status launch_fwd_kind(int nt, const FwdParams& p, const void* X, int m, int64_t k, const uint8_t* packed,
+                           int nrows, int nsplit, cudaStream_t st) {
+    switch (nt) {
+        case 16: return launch_fwd_nt<16, KIND>(p, X, m, k, packed, nrows, nsplit, st);
+        case 32: return launch_fwd_nt<32, KIND>(p, X, m, k, packed, nrows, nsplit, st);
+        case 64: return launch_fwd_nt<64, KIND>(p, X, m, k, packed, nrows, nsplit, st);
+        default: return launch_fwd_nt<128, KIND>(p, X, m, k, packed, nrows, nsplit, st);
+    }
+}
+
+// One fused dequantize-GEMM over one stored weight (or one half of a
+// channel-mix weight).  `perm` maps its stored rows to output columns.
+lbq_status run_fwd_gemm(const void* X, int m, const lbq_qweight* q, const void* B, int rank, float s,
+                        const float* T, float* Y, int64_t ldy, const int32_t* perm, void* ws, int sms,
+                        cudaStream_t st) {
+    const Plan pl = plan_gemm(m, q->n, q->k / 64, sms);
+    FwdParams p{};
+    p.m = m;
+    p.n = q->n;
+    p.k = q->k;
+    p.ngroups = q->scheme == LBQ_MINMAX_ASYM ? q->k / q->group : 0;
+    p.scale = q->scale;
+    p.zero = q->zero;
+    p.absmax = q->absmax;
+    p.q8 = (q->scheme == LBQ_CODEBOOK4 && q->double_quant) ? q->absmax_q8 : nullptr;
+    p.s2 = q->absmax_s2;
+    p.offset = q->absmax_offset;
+    p.codebook = q->codebook;
+    p.rank = rank;
+    p.rank_pad = rank > 0 ? (rank + 15) / 16 * 16 : 16;
+    p.s = s;
+    p.T = T;
+    p.B = static_cast<const uint16_t*>(B);
+    p.Y = Y;
+    p.ldy = ldy;
+    p.perm = perm;
+    p.kb_per_split = pl.per_split;
+    p.nsplit = pl.nsplit;
+    if (pl.nsplit > 1) {
+        if (!ws) return LBQ_EWORKSPACE;
+        p.partial = static_cast<float*>(ws);
+        p.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + pl.partial_bytes);
+        if (cudaMemsetAsync(p.counters, 0, pl.counter_bytes, st) != cudaSuccess) return LBQ_ECUDA;
+    }
+    switch (kind_of(q)) {
+        case kInt4: return launch_fwd_kind<kInt4>(pl.nt, p, X, m, q->k, q->packed, q->n, pl.nsplit, st);
+        case kInt2: return launch_fwd_kind<kInt2>(pl.nt, p, X, m, q->k, q->packed, q->n, pl.nsplit, st);
+        default: return launch_fwd_kind<kCode4>(pl.nt, p, X, m, q->k, q->packed, q->n, pl.nsplit, st);
+    }
+}
+
+lbq_status check_lora(int rank, const void* A, const void* B, const void* saved) {
+    if (rank < 0 || rank > kLoraMaxRank) return LBQ_EINVAL;
+    if (rank == 0) return LBQ_OK;
+    if (!A || !B || !saved) return LBQ_EINVAL;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(saved)) return LBQ_EALIGN;
+    return LBQ_OK;
+}
+
+// ---------------------------------------------------------------------------
+// backward GEMM
+// ---------------------------------------------------------------------------
+template <int NT, int BITS>
+lbq_status launch_bwd_nt(const BwdParams& p, const void* dY, const uint8_t* packed, cudaStream_t st) {
+    constexpr int S = FwdCfg<NT>::kStages, AS = FwdCfg<NT>::kAStages;
+    constexpr int KTB = 128 * BITS / 8;
+    using L = GemmSmem<NT, S, AS, 64 * KTB>;
+    auto kern = dqgemm_bwd_kernel<NT, BITS, S, AS>;
+    const size_t smem = L::total(p.rank_pad);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+        return LBQ_ECUDA;
+    CUtensorMap tmDY, tmW;
+    if (!make_map_2d(&tmDY, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.m, p.n, NT, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return LBQ_ECUDA;
+    if (!make_map_2d(&tmW, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.n, static_cast<int64_t>(p.k) * BITS / 8, 64,
+                     KTB, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return LBQ_ECUDA;
+    dim3 grid(static_cast<unsigned>(cdiv(p.k, 128)), static_cast<unsigned>(cdiv(p.m, NT)),
+              static_cast<unsigned>(p.nsplit));
+    kern<<<grid, 192, smem, st>>>(tmDY, tmW, p);
+    return last_launch();
+}
+
+template <int BITS>
+lbq_status launch_bwd_bits(int nt, const BwdParams& p, const void* dY, const uint8_t* packed, cudaStream_t st) {
+    switch (nt) {
+        case 16: return launch_bwd_nt<16, BITS>(p, dY, packed, st);
+        case 32: return launch_bwd_nt<32, BITS>(p, dY, packed, st);
+        case 64: return launch_bwd_nt<64, BITS>(p, dY, packed, st);
+        default: return launch_bwd_nt<128, BITS>(p, dY, packed, st);
+    }
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* lbq_status_string(lbq_status s) {
+    switch (s) {
+        case LBQ_OK: return "ok";
+        case LBQ_EINVAL: return "invalid argument";
+        case LBQ_EALIGN: return "device pointer not 16-byte aligned";
+        case LBQ_EUNSUPPORTED: return "unsupported configuration";
+        case LBQ_ECUDA: return "CUDA error";
+        case LBQ_ETIMEOUT: return "device-side wait timed out";
+        case LBQ_EWORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+size_t lbq_quantize_workspace_size(const lbq_qweight* q) {
+    if (q && q->scheme == LBQ_CODEBOOK4 && q->double_quant) return kCodebookQuantizeMaxCtas * sizeof(double);
+    return 0;
+}
+
+lbq_status lbq_quantize(const void* W_bf16, lbq_qweight* q, void* workspace, size_t workspace_bytes,
+                        lbq_stream_t stream) {
+    lbq_status st = check_qweight(q, true);
+    if (st != LBQ_OK) return st;
+    if (!W_bf16) return LBQ_EINVAL;
+    if (!aligned16(W_bf16)) return LBQ_EALIGN;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t nchunks = static_cast<int64_t>(q->n) * q->k / 8;
+    const int sms = sm_count();
+    if (q->scheme == LBQ_MINMAX_ASYM) {
+        const int grid = static_cast<int>(std::min<int64_t>(cdiv(nchunks, 256), 16LL * sms));
+        if (q->bits == 4)
+            minmax_quantize_kernel<4><<<grid, 256, 0, s>>>(static_cast<const uint4*>(W_bf16), nchunks, q->packed,
+                                                            q->scale, q->zero);
+        else
+            minmax_quantize_kernel<2><<<grid, 256, 0, s>>>(static_cast<const uint4*>(W_bf16), nchunks, q->packed,
+                                                            q->scale, q->zero);
+        return last_launch();
+    }
+    const int grid = static_cast<int>(std::min<int64_t>(cdiv(nchunks, 256), std::min(16 * sms, kCodebookQuantizeMaxCtas)));
+    double* sums = nullptr;
+    if (q->double_quant) {
+        if (!workspace || workspace_bytes < lbq_quantize_workspace_size(q)) return LBQ_EWORKSPACE;
+        if (!aligned16(workspace)) return LBQ_EALIGN;
+        sums = static_cast<double*>(workspace);
+    }
+    codebook_quantize_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(W_bf16), nchunks, q->codebook, q->packed,
+                                                  q->absmax, sums);
+    if ((st = last_launch()) != LBQ_OK) return st;
+    if (q->double_quant) {
+        const int64_t nb = static_cast<int64_t>(q->n) * q->k / 64;
+        absmax_offset_kernel<<<1, 256, 0, s>>>(sums, grid, nb, q->absmax_offset);
+        if ((st = last_launch()) != LBQ_OK) return st;
+        double_quant_kernel<<<static_cast<unsigned>(cdiv(nb, 256)), 256, 0, s>>>(q->absmax, nb, q->absmax_offset,
+                                                                                q->absmax_q8, q->absmax_s2);
+        return last_launch();
+    }
+    return LBQ_OK;
+}
+
+lbq_status lbq_dequantize(const lbq_qweight* q, float* W_f32, lbq_stream_t stream) {
+    lbq_status st = check_qweight(q, true);
+    if (st != LBQ_OK) return st;
+    if (!W_f32) return LBQ_EINVAL;
+    if (!aligned16(W_f32)) return LBQ_EALIGN;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t nchunks = static_cast<int64_t>(q->n) * q->k / 8;
+    const int grid = static_cast<int>(std::min<int64_t>(cdiv(nchunks, 256), 16LL * sm_count()));
+    float4* out = reinterpret_cast<float4*>(W_f32);
+    if (q->scheme == LBQ_MINMAX_ASYM) {
+        if (q->bits == 4)
+            minmax_dequantize_kernel<4><<<grid, 256, 0, s>>>(q->packed, q->scale, q->zero, nchunks, out);
+        else
+            minmax_dequantize_kernel<2><<<grid, 256, 0, s>>>(q->packed, q->scale, q->zero, nchunks, out);
+    } else {
+        codebook_dequantize_kernel<<<grid, 256, 0, s>>>(q->packed, q->absmax, q->double_quant ? q->absmax_q8 : nullptr,
+                                                        q->absmax_s2, q->absmax_offset, q->codebook, nchunks, out);
+    }
+    return last_launch();
+}
+
+size_t lbq_linear_fwd_workspace_size(int m, const lbq_qweight* q, int rank) {
+    (void)rank;
+    if (m < 1 || check_qweight(q, false) != LBQ_OK) return 0;
+    return plan_gemm(m, q->n, q->k / 64, sm_count()).workspace();
+}
+
+lbq_status lbq_linear_fwd(const void* X, int m, const lbq_qweight* q, const void* A, const void* B, int rank,
+                          float s, float* Y, float* T_save, void* workspace, size_t workspace_bytes,
+                          lbq_stream_t stream) {
+    lbq_status st = check_qweight(q, true);
+    if (st != LBQ_OK) return st;
+    if (m < 1 || !X || !Y) return LBQ_EINVAL;
+    if (!aligned16(X) || !aligned16(Y)) return LBQ_EALIGN;
+    if ((st = check_lora(rank, A, B, T_save)) != LBQ_OK) return st;
+    const int sms = sm_count();
+    const size_t need = plan_gemm(m, q->n, q->k / 64, sms).workspace();
+    if (need > 0 && (!workspace || workspace_bytes < need)) return LBQ_EWORKSPACE;
+    if (need > 0 && !aligned16(workspace)) return LBQ_EALIGN;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    if (rank > 0) {
+        lora_rowdot_kernel<false><<<m, 256, 0, cs>>>(static_cast<const uint16_t*>(X), q->k,
+                                                     static_cast<const uint16_t*>(A), rank, T_save);
+        if ((st = last_launch()) != LBQ_OK) return st;
+    }
+    return run_fwd_gemm(X, m, q, B, rank, s, T_save, Y, q->n, nullptr, workspace, sms, cs);
+}
+
+size_t lbq_linear_fwd_mix_workspace_size(int m, const lbq_qweight_mix* q, int rank) {
+    (void)rank;
+    if (!q || m < 1) return 0;
+    if (check_qweight(&q->hi, false) != LBQ_OK || check_qweight(&q->lo, false) != LBQ_OK) return 0;
+    const int sms = sm_count();
+    return round_up(plan_gemm(m, q->hi.n, q->hi.k / 64, sms).workspace(), 256) +
+           plan_gemm(m, q->lo.n, q->lo.k / 64, sms).workspace();
+}
+
+lbq_status lbq_linear_fwd_mix(const void* X, int m, const lbq_qweight_mix* q, const void* A, const void* B, int rank,
+                              float s, float* Y, float* T_save, void* workspace, size_t workspace_bytes,
+                              lbq_stream_t stream) {
+    if (!q || !q->perm) return LBQ_EINVAL;
+    lbq_status st;
+    if ((st = check_qweight(&q->hi, true)) != LBQ_OK) return st;
+    if ((st = check_qweight(&q->lo, true)) != LBQ_OK) return st;
+    if (q->hi.scheme != LBQ_MINMAX_ASYM || q->lo.scheme != LBQ_MINMAX_ASYM || q->hi.k != q->lo.k)
+        return LBQ_EINVAL;
+    if (m < 1 || !X || !Y) return LBQ_EINVAL;
+    if (!aligned16(X) || !aligned16(Y) || !aligned16(q->perm)) return LBQ_EALIGN;
+    if ((st = check_lora(rank, A, B, T_save)) != LBQ_OK) return st;
+    const int sms = sm_count();
+    const size_t need_hi = round_up(plan_gemm(m, q->hi.n, q->hi.k / 64, sms).workspace(), 256);
+    const size_t need = need_hi + plan_gemm(m, q->lo.n, q->lo.k / 64, sms).workspace();
+    if (need > 0 && (!workspace || workspace_bytes < need)) return LBQ_EWORKSPACE;
+    if (need > 0 && !aligned16(workspace)) return LBQ_EALIGN;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t n_total = static_cast<int64_t>(q->hi.n) + q->lo.n;
+    if (rank > 0) {
+        lora_rowdot_kernel<false><<<m, 256, 0, cs>>>(static_cast<const uint16_t*>(X), q->hi.k,
+                                                     static_cast<const uint16_t*>(A), rank, T_save);
+        if ((st = last_launch()) != LBQ_OK) return st;
+    }
+    if ((st = run_fwd_gemm(X, m, &q->hi, B, rank, s, T_save, Y, n_total, q->perm, workspace, sms, cs)) != LBQ_OK)
+        return st;
+    void* ws_lo = workspace ? static_cast<uint8_t*>(workspace) + need_hi : nullptr;
+    return run_fwd_gemm(X, m, &q->lo, B, rank, s, T_save, Y, n_total, q->perm + q->hi.n, ws_lo, sms, cs);
+}
+
+size_t lbq_linear_bwd_workspace_size(int m, const lbq_qweight* q, int rank) {
+    (void)rank;
+    if (m < 1 || check_qweight(q, false) != LBQ_OK) return 0;
+    return plan_gemm(m, q->k, cdiv(q->n, 64), sm_count()).workspace();
+}
+
+lbq_status lbq_linear_bwd(const void* dY, int m, const lbq_qweight* q, const void* A, const void* B, int rank,
+                          float s, float* dX, float* U_save, void* workspace, size_t workspace_bytes,
+                          lbq_stream_t stream) {
+    lbq_status st = check_qweight(q, true);
+    if (st != LBQ_OK) return st;
+    if (q->scheme != LBQ_MINMAX_ASYM) return LBQ_EUNSUPPORTED;
+    if (m < 1 || !dY || !dX || q->n % 8 != 0) return LBQ_EINVAL;
+    if (!aligned16(dY) || !aligned16(dX)) return LBQ_EALIGN;
+    if ((st = check_lora(rank, A, B, U_save)) != LBQ_OK) return st;
+    const int sms = sm_count();
+    const Plan pl = plan_gemm(m, q->k, cdiv(q->n, 64), sms);
+    if (pl.workspace() > 0 && (!workspace || workspace_bytes < pl.workspace())) return LBQ_EWORKSPACE;
+    if (pl.workspace() > 0 && !aligned16(workspace)) return LBQ_EALIGN;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    if (rank > 0) {
+        lora_rowdot_kernel<true><<<m, 256, 0, cs>>>(static_cast<const uint16_t*>(dY), q->n,
+                                                    static_cast<const uint16_t*>(B), rank, U_save);
+        if ((st = last_launch()) != LBQ_OK) return st;
+    }
+    BwdParams p{};
+    p.m = m;
+    p.n = q->n;
+    p.k = q->k;
+    p.bits = q->bits;
+    p.ngroups = q->k / q->group;
+    p.scale = q->scale;
+    p.zero = q->zero;
+    p.rank = rank;
+    p.rank_pad = rank > 0 ? (rank + 15) / 16 * 16 : 16;
+    p.s = s;
+    p.U = U_save;
+    p.A = static_cast<const uint16_t*>(A);
+    p.dX = dX;
+    p.cb_per_split = pl.per_split;
+    p.nsplit = pl.nsplit;
+    if (pl.nsplit > 1) {
+        p.partial = static_cast<float*>(workspace);
+        p.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + pl.partial_bytes);
+        if (cudaMemsetAsync(p.counters, 0, pl.counter_bytes, cs) != cudaSuccess) return LBQ_ECUDA;
+    }
+    if (q->bits == 4) return launch_bwd_bits<4>(pl.nt, p, dY, q->packed, cs);
+    return launch_bwd_bits<2>(pl.nt, p, dY, q->packed, cs);
+}
+
+lbq_status lbq_lora_grads(const void* X, const void* dY, int m, int n, int k, const float* T, const float* U,
+                          int rank, float s, float* dA, float* dB, lbq_stream_t stream) {
+    if (m < 1 || n < 1 || k < 64 || k % 64 != 0 || n % 8 != 0) return LBQ_EINVAL;
+    if (rank < 1 || rank > kLoraMaxRank) return LBQ_EINVAL;
+    if (!X || !dY || !T || !U || !dA || !dB) return LBQ_EINVAL;
+    if (!aligned16(X) || !aligned16(dY) || !aligned16(T) || !aligned16(U) || !aligned16(dA) || !aligned16(dB))
+        return LBQ_EALIGN;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    lora_colgrad_kernel<<<static_cast<unsigned>(cdiv(k, 32)), 256, 0, cs>>>(
+        static_cast<const uint16_t*>(X), m, k, U, rank, s, dA, 1, k);
+    lbq_status st = last_launch();
+    if (st != LBQ_OK) return st;
+    lora_colgrad_kernel<<<static_cast<unsigned>(cdiv(n, 32)), 256, 0, cs>>>(
+        static_cast<const uint16_t*>(dY), m, n, T, rank, s, dB, rank, 1);
+    return last_launch();
+}
+
+lbq_status lbq_device_status(uint32_t* flags) {
+    if (!flags) return LBQ_EINVAL;
+    if (cudaDeviceSynchronize() != cudaSuccess) return LBQ_ECUDA;
+    uint32_t v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return LBQ_ECUDA;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return LBQ_ECUDA;
+    *flags = v;
+    return LBQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,266 @@
+"""Python binding of the lbq C ABI (include/lbq.h).
+
+Argument marshalling only: every computation runs in the CUDA kernels of
+liblbq.so.  The low-level functions (`lbq_quantize`, `lbq_linear_fwd`, ...)
+have the C names and take raw integers (device pointers, sizes, stream
+handles) and `lbq_qweight` structures.  The helpers below them accept torch
+tensors, allocate outputs and workspaces with torch (device memory is the one
+thing PyTorch supplies) and pass pointers through.
+
+There is no fallback: importing this module fails when liblbq.so is missing,
+and every call raises `LbqError` when the library returns a non-OK status.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "liblbq.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "lbq.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m qlora_quantized_linear_b200.build`")
+_L = ctypes.CDLL(LIB_PATH)
+
+LBQ_OK, LBQ_EINVAL, LBQ_EALIGN, LBQ_EUNSUPPORTED, LBQ_ECUDA, LBQ_ETIMEOUT, LBQ_EWORKSPACE = range(7)
+LBQ_MINMAX_ASYM, LBQ_CODEBOOK4 = 0, 1
+STATUS_TIMEOUT, STATUS_BAD_TABLE = 1, 2
+
+
+class lbq_qweight(ctypes.Structure):
+    _fields_ = [
+        ("n", ctypes.c_int32), ("k", ctypes.c_int32),
+        ("bits", ctypes.c_int32), ("group", ctypes.c_int32),
+        ("scheme", ctypes.c_int32), ("double_quant", ctypes.c_int32),
+        ("packed", ctypes.c_void_p),
+        ("scale", ctypes.c_void_p), ("zero", ctypes.c_void_p),
+        ("absmax", ctypes.c_void_p),
+        ("absmax_q8", ctypes.c_void_p), ("absmax_s2", ctypes.c_void_p), ("absmax_offset", ctypes.c_void_p),
+        ("codebook", ctypes.c_void_p),
+    ]
+
+
+class lbq_qweight_mix(ctypes.Structure):
+    _fields_ = [("hi", lbq_qweight), ("lo", lbq_qweight), ("perm", ctypes.c_void_p)]
+
+
+_vp, _int, _f32, _sz, _u32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.POINTER(ctypes.c_uint32)
+_QP, _MP = ctypes.POINTER(lbq_qweight), ctypes.POINTER(lbq_qweight_mix)
+_SIGS = {
+    "lbq_status_string": (ctypes.c_char_p, [_int]),
+    "lbq_quantize_workspace_size": (_sz, [_QP]),
+    "lbq_quantize": (_int, [_vp, _QP, _vp, _sz, _vp]),
+    "lbq_dequantize": (_int, [_QP, _vp, _vp]),
+    "lbq_linear_fwd_workspace_size": (_sz, [_int, _QP, _int]),
+    "lbq_linear_fwd": (_int, [_vp, _int, _QP, _vp, _vp, _int, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "lbq_linear_fwd_mix_workspace_size": (_sz, [_int, _MP, _int]),
+    "lbq_linear_fwd_mix": (_int, [_vp, _int, _MP, _vp, _vp, _int, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "lbq_linear_bwd_workspace_size": (_sz, [_int, _QP, _int]),
+    "lbq_linear_bwd": (_int, [_vp, _int, _QP, _vp, _vp, _int, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "lbq_lora_grads": (_int, [_vp, _vp, _int, _int, _int, _vp, _vp, _int, _f32, _vp, _vp, _vp]),
+    "lbq_device_status": (_int, [_u32p]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_L, _name)
+    _f.restype, _f.argtypes = _res, _args
+
+
+def header_functions():
+    """Names of the functions that include/lbq.h declares."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(lbq_\w+)\(", text, re.M)))
+
+
+# --------------------------------------------------------------------------- C names
+lbq_status_string = _L.lbq_status_string
+lbq_quantize_workspace_size = _L.lbq_quantize_workspace_size
+lbq_quantize = _L.lbq_quantize
+lbq_dequantize = _L.lbq_dequantize
+lbq_linear_fwd_workspace_size = _L.lbq_linear_fwd_workspace_size
+lbq_linear_fwd = _L.lbq_linear_fwd
+lbq_linear_fwd_mix_workspace_size = _L.lbq_linear_fwd_mix_workspace_size
+lbq_linear_fwd_mix = _L.lbq_linear_fwd_mix
+lbq_linear_bwd_workspace_size = _L.lbq_linear_bwd_workspace_size
+lbq_linear_bwd = _L.lbq_linear_bwd
+lbq_lora_grads = _L.lbq_lora_grads
+lbq_device_status = _L.lbq_device_status
+
+
+class LbqError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {lbq_status_string(code).decode()} (status {code})")
+
+
+def _check(code: int, what: str) -> None:
+    if code != LBQ_OK:
+        raise LbqError(code, what)
+
+
+# --------------------------------------------------------------------------- torch helpers
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _bf16_2d(t, name):
+    torch = _torch()
+    if t.dtype != torch.bfloat16 or t.dim() != 2 or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous 2-D bf16 CUDA tensor")
+    return t
+
+
+class QuantizedWeight:
+    """Device buffers of one quantized weight plus its `lbq_qweight` view.
+
+    scheme "minmax": bits 4 (group 128) or 2 (group 64).
+    scheme "codebook": 4-bit codes, absmax per 64, optional double quantization;
+    `codebook` is 16 sorted floats in [-1, 1] with an exact 0.
+    """
+
+    def __init__(self, n: int, k: int, scheme: str = "minmax", bits: int = 4, group: Optional[int] = None,
+                 double_quant: bool = False, codebook=None, device="cuda"):
+        torch = _torch()
+        self.n, self.k, self.scheme, self.bits = int(n), int(k), scheme, int(bits)
+        self.double_quant = bool(double_quant)
+        u8, f32 = torch.uint8, torch.float32
+        if scheme == "minmax":
+            self.group = int(group or (128 if bits == 4 else 64))
+            self.packed = torch.empty((n, k * bits // 8), dtype=u8, device=device)
+            self.scale = torch.empty((n, k // self.group), dtype=torch.float16, device=device)
+            self.zero = torch.empty((n, k // self.group), dtype=torch.float16, device=device)
+            self.absmax = self.q8 = self.s2 = self.offset = self.codebook = None
+        elif scheme == "codebook":
+            self.group, self.bits = 64, 4
+            nb = n * k // 64
+            self.packed = torch.empty((n, k // 2), dtype=u8, device=device)
+            self.scale = self.zero = None
+            self.absmax = torch.empty(nb, dtype=f32, device=device)
+            self.codebook = torch.as_tensor(codebook, dtype=f32).to(device).contiguous()
+            if self.double_quant:
+                self.q8 = torch.empty(nb, dtype=torch.int8, device=device)
+                self.s2 = torch.empty((nb + 255) // 256, dtype=f32, device=device)
+                self.offset = torch.empty(4, dtype=f32, device=device)  # 1 used; 16-byte buffer
+            else:
+                self.q8 = self.s2 = self.offset = None
+        else:
+            raise ValueError(f"unknown scheme {scheme!r}")
+        self.struct = self._make_struct()
+
+    def _make_struct(self) -> lbq_qweight:
+        return lbq_qweight(
+            n=self.n, k=self.k, bits=self.bits, group=self.group,
+            scheme=LBQ_MINMAX_ASYM if self.scheme == "minmax" else LBQ_CODEBOOK4,
+            double_quant=int(self.double_quant),
+            packed=_ptr(self.packed), scale=_ptr(self.scale), zero=_ptr(self.zero), absmax=_ptr(self.absmax),
+            absmax_q8=_ptr(self.q8), absmax_s2=_ptr(self.s2), absmax_offset=_ptr(self.offset),
+            codebook=_ptr(self.codebook))
+
+    def quantize(self, W, stream=None) -> "QuantizedWeight":
+        torch = _torch()
+        W = _bf16_2d(W, "W")
+        assert tuple(W.shape) == (self.n, self.k)
+        nws = lbq_quantize_workspace_size(ctypes.byref(self.struct))
+        ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=W.device) if nws else None
+        _check(lbq_quantize(W.data_ptr(), ctypes.byref(self.struct), _ptr(ws), nws, _stream(stream)), "lbq_quantize")
+        self._keep = ws
+        return self
+
+    def dequantize(self, stream=None):
+        torch = _torch()
+        out = torch.empty((self.n, self.k), dtype=torch.float32, device=self.packed.device)
+        _check(lbq_dequantize(ctypes.byref(self.struct), out.data_ptr(), _stream(stream)), "lbq_dequantize")
+        return out
+
+
+class ChannelMixWeight:
+    """Channel-mix weight: INT4 g128 rows `hi`, INT2 g64 rows `lo`, and perm
+    (stored row -> original output channel; rows of hi first)."""
+
+    def __init__(self, hi: QuantizedWeight, lo: QuantizedWeight, perm):
+        torch = _torch()
+        self.hi, self.lo = hi, lo
+        self.perm = torch.as_tensor(perm, dtype=torch.int32).to(hi.packed.device).contiguous()
+        self.n, self.k = hi.n + lo.n, hi.k
+        self.struct = lbq_qweight_mix(hi=hi.struct, lo=lo.struct, perm=self.perm.data_ptr())
+
+
+def _workspace(nbytes: int, device):
+    torch = _torch()
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device) if nbytes else None
+
+
+def linear_fwd(X, qw, A=None, B=None, s: float = 0.0, Y=None, T=None, workspace=None, stream=None):
+    """Y = X W^T + s (X A^T) B^T; returns (Y fp32 [m, n], T fp32 [m, rank] or None)."""
+    torch = _torch()
+    X = _bf16_2d(X, "X")
+    m = X.shape[0]
+    rank = 0 if A is None else int(A.shape[0])
+    if Y is None:
+        Y = torch.empty((m, qw.n), dtype=torch.float32, device=X.device)
+    if rank > 0 and T is None:
+        T = torch.empty((m, rank), dtype=torch.float32, device=X.device)
+    mix = isinstance(qw, ChannelMixWeight)
+    size_fn = lbq_linear_fwd_mix_workspace_size if mix else lbq_linear_fwd_workspace_size
+    nws = size_fn(m, ctypes.byref(qw.struct), rank)
+    if workspace is None:
+        workspace = _workspace(nws, X.device)
+    fn = lbq_linear_fwd_mix if mix else lbq_linear_fwd
+    _check(fn(X.data_ptr(), m, ctypes.byref(qw.struct), _ptr(A), _ptr(B), rank, float(s), Y.data_ptr(), _ptr(T),
+              _ptr(workspace), nws, _stream(stream)), fn.__name__)
+    return Y, T
+
+
+def linear_bwd(dY, qw, A=None, B=None, s: float = 0.0, dX=None, U=None, workspace=None, stream=None):
+    """dX = dY W + s (dY B) A; returns (dX fp32 [m, k], U fp32 [m, rank] or None)."""
+    torch = _torch()
+    dY = _bf16_2d(dY, "dY")
+    m = dY.shape[0]
+    rank = 0 if A is None else int(A.shape[0])
+    if dX is None:
+        dX = torch.empty((m, qw.k), dtype=torch.float32, device=dY.device)
+    if rank > 0 and U is None:
+        U = torch.empty((m, rank), dtype=torch.float32, device=dY.device)
+    nws = lbq_linear_bwd_workspace_size(m, ctypes.byref(qw.struct), rank)
+    if workspace is None:
+        workspace = _workspace(nws, dY.device)
+    _check(lbq_linear_bwd(dY.data_ptr(), m, ctypes.byref(qw.struct), _ptr(A), _ptr(B), rank, float(s), dX.data_ptr(),
+                          _ptr(U), _ptr(workspace), nws, _stream(stream)), "lbq_linear_bwd")
+    return dX, U
+
+
+def lora_grads(X, dY, T, U, s: float, dA=None, dB=None, stream=None):
+    """dA = s U^T X [rank, k], dB = s dY^T T [n, rank] (fp32)."""
+    torch = _torch()
+    X, dY = _bf16_2d(X, "X"), _bf16_2d(dY, "dY")
+    m, k = X.shape
+    n = dY.shape[1]
+    rank = int(T.shape[1])
+    if dA is None:
+        dA = torch.empty((rank, k), dtype=torch.float32, device=X.device)
+    if dB is None:
+        dB = torch.empty((n, rank), dtype=torch.float32, device=X.device)
+    _check(lbq_lora_grads(X.data_ptr(), dY.data_ptr(), m, n, k, T.data_ptr(), U.data_ptr(), rank, float(s),
+                          dA.data_ptr(), dB.data_ptr(), _stream(stream)), "lbq_lora_grads")
+    return dA, dB
+
+
+def device_status() -> int:
+    """The device status word (timeouts, bad codebooks) since the last read."""
+    v = ctypes.c_uint32(0)
+    _check(lbq_device_status(ctypes.byref(v)), "lbq_device_status")
+    return int(v.value)

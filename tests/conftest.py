@@ -25,3 +25,13 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _built_libraries():
+    """Build the oracle (gcc) and the CUDA library (nvcc, sm_100a) when stale."""
+    from oracle.build import build as build_oracle
+    from qlora_quantized_linear_b200.build import build as build_lbq
+    build_oracle()
+    build_lbq()
+    yield

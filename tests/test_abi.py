@@ -1,0 +1,76 @@
+"""The C ABI library loads on a machine without a GPU, exports every entry
+point that include/lbq.h declares, and rejects bad arguments on the host
+before touching the device."""
+import ctypes
+
+import pytest
+
+from qlora_quantized_linear_b200 import lbq
+
+
+def test_exports_every_declared_function():
+    names = lbq.header_functions()
+    assert len(names) >= 12
+    for name in names:
+        assert hasattr(lbq._L, name), f"{name} declared in include/lbq.h but not exported"
+
+
+def test_status_strings():
+    for code in range(7):
+        assert lbq.lbq_status_string(code)
+    assert lbq.lbq_status_string(99) == b"unknown status"
+
+
+def _qw(**kw):
+    q = lbq.lbq_qweight(n=256, k=512, bits=4, group=128, scheme=lbq.LBQ_MINMAX_ASYM, double_quant=0,
+                        packed=0x1000, scale=0x2000, zero=0x3000)
+    for key, v in kw.items():
+        setattr(q, key, v)
+    return q
+
+
+@pytest.mark.parametrize("change,expect", [
+    (dict(bits=3), lbq.LBQ_EUNSUPPORTED),
+    (dict(bits=4, group=64), lbq.LBQ_EUNSUPPORTED),
+    (dict(k=100), lbq.LBQ_EINVAL),
+    (dict(n=0), lbq.LBQ_EINVAL),
+    (dict(packed=None), lbq.LBQ_EINVAL),
+    (dict(packed=0x1008), lbq.LBQ_EALIGN),
+    (dict(scheme=7), lbq.LBQ_EUNSUPPORTED),
+])
+def test_quantize_rejects_bad_descriptors(change, expect):
+    q = _qw(**change)
+    assert lbq.lbq_quantize(0x4000, ctypes.byref(q), None, 0, None) == expect
+
+
+def test_linear_fwd_rejects_bad_arguments():
+    q = _qw()
+    fwd = lbq.lbq_linear_fwd
+    assert fwd(0x4000, 0, ctypes.byref(q), None, None, 0, 0.0, 0x5000, None, None, 0, None) == lbq.LBQ_EINVAL
+    assert fwd(None, 4, ctypes.byref(q), None, None, 0, 0.0, 0x5000, None, None, 0, None) == lbq.LBQ_EINVAL
+    assert fwd(0x4004, 4, ctypes.byref(q), None, None, 0, 0.0, 0x5000, None, None, 0, None) == lbq.LBQ_EALIGN
+    # rank > 0 needs A, B and T_save; rank above 64 is rejected
+    assert fwd(0x4000, 4, ctypes.byref(q), None, None, 8, 1.0, 0x5000, None, None, 0, None) == lbq.LBQ_EINVAL
+    assert fwd(0x4000, 4, ctypes.byref(q), 0x6000, 0x7000, 65, 1.0, 0x5000, 0x8000, None, 0, None) == lbq.LBQ_EINVAL
+    assert fwd(0x4000, 4, None, None, None, 0, 0.0, 0x5000, None, None, 0, None) == lbq.LBQ_EINVAL
+
+
+def test_bwd_and_grads_reject_bad_arguments():
+    q = _qw()
+    bwd = lbq.lbq_linear_bwd
+    cb = _qw(scheme=lbq.LBQ_CODEBOOK4, group=64, absmax=0x9000, codebook=0xA000)
+    assert bwd(0x4000, 4, ctypes.byref(cb), None, None, 0, 0.0, 0x5000, None, None, 0, None) == lbq.LBQ_EUNSUPPORTED
+    q2 = _qw(n=250)
+    assert bwd(0x4000, 4, ctypes.byref(q2), None, None, 0, 0.0, 0x5000, None, None, 0, None) == lbq.LBQ_EINVAL
+    g = lbq.lbq_lora_grads
+    assert g(0x4000, 0x5000, 4, 256, 512, 0x6000, 0x7000, 0, 1.0, 0x8000, 0x9000, None) == lbq.LBQ_EINVAL
+    assert g(0x4000, 0x5000, 4, 255, 512, 0x6000, 0x7000, 8, 1.0, 0x8000, 0x9000, None) == lbq.LBQ_EINVAL
+    assert g(0x4002, 0x5000, 4, 256, 512, 0x6000, 0x7000, 8, 1.0, 0x8000, 0x9000, None) == lbq.LBQ_EALIGN
+
+
+def test_workspace_queries_are_host_only():
+    q = _qw()
+    assert lbq.lbq_linear_fwd_workspace_size(0, ctypes.byref(q), 0) == 0
+    assert lbq.lbq_quantize_workspace_size(ctypes.byref(q)) == 0
+    cb = _qw(scheme=lbq.LBQ_CODEBOOK4, group=64, double_quant=1)
+    assert lbq.lbq_quantize_workspace_size(ctypes.byref(cb)) > 0

@@ -1,0 +1,250 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI.
+
+Bit-exact: packed codes, scales, zeros, absmax, q8, s2, offset and the fp32
+dequantized weights.  GEMM outputs: within the stated bound
+|dY| <= 2^-7 * sum_k |x_k| |w_eff,k| + 1e-6 (w_eff = W_hat plus the adapter
+term), computed by the oracle for every element.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from qlora_quantized_linear_b200 import synthetic as syn
+
+pytestmark = pytest.mark.gpu
+
+TOL_REL = 2.0 ** -7
+TOL_ABS = 1e-6
+
+
+@pytest.fixture(scope="module")
+def lbq():
+    from qlora_quantized_linear_b200 import lbq as m
+    return m
+
+
+def u16(t: torch.Tensor) -> np.ndarray:
+    """Bits of a bf16/fp16 tensor (any device) as uint16 numpy."""
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def assert_status_clean(lbq):
+    assert lbq.device_status() == 0
+
+
+def assert_within(got, ref, bound, what):
+    got = np.asarray(got, np.float64)
+    err = np.abs(got - ref)
+    lim = TOL_REL * bound + TOL_ABS
+    bad = err > lim
+    assert not bad.any(), (f"{what}: {int(bad.sum())}/{bad.size} elements outside the bound; "
+                           f"worst excess {float((err - lim).max()):.3e} at {np.unravel_index(np.argmax(err - lim), err.shape)}")
+
+
+def mixed_weight(n, k, seed, std=0.02):
+    """Weights with outlier columns, all-positive / all-negative rows, a
+    constant group and a zero row (edge cases of the MinMax quantizer)."""
+    w = syn.weight_bf16(n, k, std, seed, outlier_frac=0.01, outlier_scale=20.0).float()
+    if n > 5:
+        w[1] = w[1].abs() + 0.05
+        w[2] = -w[2].abs() - 0.05
+        w[3, :128] = 0.3
+        w[4] = 0.0
+        w[5, 7] = -0.0
+    return w.to(torch.bfloat16)
+
+
+# --------------------------------------------------------------------------- quantize / dequantize
+@pytest.mark.parametrize("bits", [4, 2])
+@pytest.mark.parametrize("shape", [(256, 512), (300, 1024), (1, 128), (4096, 256)])
+def test_minmax_quantize_bit_exact(lbq, bits, shape):
+    n, k = shape
+    W = mixed_weight(n, k, seed=n + k + bits)
+    qw = lbq.QuantizedWeight(n, k, "minmax", bits).quantize(W.cuda())
+    torch.cuda.synchronize()
+    codes, scale, zero = oracle.minmax_quantize(syn.bits_u16(W), bits, qw.group)
+    assert np.array_equal(qw.packed.cpu().numpy(), oracle.pack(codes, bits)), "packed codes differ"
+    assert np.array_equal(u16(qw.scale), scale), "scales differ"
+    assert np.array_equal(u16(qw.zero), zero), "zeros differ"
+    What = qw.dequantize().cpu().numpy()
+    ref = oracle.minmax_dequantize(oracle.pack(codes, bits), scale, zero, k, bits, qw.group)
+    assert np.array_equal(What.view(np.uint32), ref.view(np.uint32)), "dequantized weights differ"
+    assert_status_clean(lbq)
+
+
+def test_minmax_quantize_grid_values(lbq):
+    """Exact grid values re-quantize to themselves on the GPU as well."""
+    n, k, bits, group = 64, 512, 4, 128
+    rng = np.random.default_rng(5)
+    q = rng.integers(0, 16, (n, k))
+    qg = q.reshape(n, k // group, group)
+    qg[:, :, 0], qg[:, :, 1] = 0, 15
+    z = rng.integers(0, 16, (n, k // group))
+    sf = rng.integers(1, 8, (n, k // group)) * 2.0 ** rng.integers(-10, -4, (n, k // group))
+    w = ((qg - z[:, :, None]) * sf[:, :, None]).reshape(n, k).astype(np.float32)
+    W = torch.from_numpy(w).to(torch.bfloat16)
+    qw = lbq.QuantizedWeight(n, k, "minmax", bits).quantize(W.cuda())
+    got = oracle.unpack(qw.packed.cpu().numpy(), k, bits)
+    assert np.array_equal(got.astype(np.int64), q)
+
+
+@pytest.mark.parametrize("double_quant", [False, True])
+@pytest.mark.parametrize("shape", [(256, 512), (1000, 1024), (128, 64 * 300)])
+def test_codebook_quantize_bit_exact(lbq, double_quant, shape):
+    n, k = shape
+    cb = syn.codebook_normal16()
+    Wt = syn.weight_bf16(n, k, 0.015, seed=n * 7 + k).float()
+    Wt[0, :64] = 0.0
+    W = Wt.to(torch.bfloat16)
+    qw = lbq.QuantizedWeight(n, k, "codebook", double_quant=double_quant, codebook=cb).quantize(W.cuda())
+    torch.cuda.synchronize()
+    codes, absmax = oracle.codebook_quantize(syn.bits_u16(W), cb)
+    packed = oracle.pack(codes, 4)
+    assert np.array_equal(qw.packed.cpu().numpy(), packed)
+    assert np.array_equal(qw.absmax.cpu().numpy().view(np.uint32), absmax.view(np.uint32))
+    a_used = absmax
+    if double_quant:
+        q8, s2, off, exact = oracle.double_quant(absmax)
+        assert exact
+        assert np.float32(qw.offset[0].item()).view(np.uint32) == np.float32(off).view(np.uint32)
+        assert np.array_equal(qw.q8.cpu().numpy(), q8)
+        assert np.array_equal(qw.s2.cpu().numpy().view(np.uint32), s2.view(np.uint32))
+        a_used = oracle.double_dequant(q8, s2, off)
+    What = qw.dequantize().cpu().numpy()
+    ref = oracle.codebook_dequantize(packed, a_used, cb, n, k)
+    assert np.array_equal(What.view(np.uint32), ref.view(np.uint32))
+    assert_status_clean(lbq)
+
+
+# --------------------------------------------------------------------------- forward
+def fwd_problem(m, n, k, rank, seed, scheme="minmax", bits=4, double_quant=False):
+    X = syn.normal_bf16((m, k), 1.0, seed)
+    W = mixed_weight(n, k, seed + 1) if scheme == "minmax" else syn.weight_bf16(n, k, 0.015, seed + 1)
+    A = syn.normal_bf16((rank, k), 0.01, seed + 2) if rank else None
+    B = syn.normal_bf16((n, rank), 0.01, seed + 3) if rank else None
+    return X, W, A, B
+
+
+def oracle_weight(W, scheme, bits, double_quant, cb):
+    n, k = W.shape
+    if scheme == "minmax":
+        group = 128 if bits == 4 else 64
+        codes, scale, zero = oracle.minmax_quantize(syn.bits_u16(W), bits, group)
+        return oracle.minmax_dequantize(oracle.pack(codes, bits), scale, zero, k, bits, group)
+    codes, absmax = oracle.codebook_quantize(syn.bits_u16(W), cb)
+    if double_quant:
+        q8, s2, off, _ = oracle.double_quant(absmax)
+        absmax = oracle.double_dequant(q8, s2, off)
+    return oracle.codebook_dequantize(oracle.pack(codes, 4), absmax, cb, n, k)
+
+
+FWD_CASES = [
+    # m, n, k, rank, scheme, bits, dq
+    (8, 256, 512, 8, "minmax", 4, False),       # tiny single linear
+    (1, 256, 512, 0, "minmax", 4, False),
+    (15, 384, 1024, 16, "minmax", 4, False),
+    (16, 200, 640, 16, "minmax", 4, False),     # ragged n
+    (17, 256, 512, 0, "minmax", 4, False),
+    (63, 128, 512, 8, "minmax", 4, False),
+    (64, 256, 512, 16, "minmax", 4, False),
+    (65, 256, 512, 64, "minmax", 4, False),
+    (130, 384, 768, 16, "minmax", 4, False),    # two token tiles, ragged
+    (16, 256, 512, 8, "minmax", 2, False),
+    (200, 256, 512, 0, "minmax", 2, False),
+    (1, 256, 1024, 0, "codebook", 4, False),
+    (16, 256, 512, 16, "codebook", 4, True),
+    (140, 256, 512, 0, "codebook", 4, True),
+]
+
+
+@pytest.mark.parametrize("m,n,k,rank,scheme,bits,dq", FWD_CASES)
+def test_linear_fwd_parity(lbq, m, n, k, rank, scheme, bits, dq):
+    cb = syn.codebook_normal16()
+    X, W, A, B = fwd_problem(m, n, k, rank, seed=m * 131 + n + k + rank, scheme=scheme, bits=bits)
+    qw = lbq.QuantizedWeight(n, k, scheme, bits, double_quant=dq, codebook=cb).quantize(W.cuda())
+    s = 2.0
+    Y, T = lbq.linear_fwd(X.cuda(), qw, None if A is None else A.cuda(), None if B is None else B.cuda(), s)
+    torch.cuda.synchronize()
+    What = oracle_weight(W, scheme, bits, dq, cb)
+    Yr, Tr, Yb = oracle.linear_fwd(syn.bits_u16(X), What, None if A is None else syn.bits_u16(A),
+                                   None if B is None else syn.bits_u16(B), s)
+    assert_within(Y.cpu().numpy(), Yr, Yb, "Y")
+    if rank:
+        Tb = np.abs(oracle.bf16_to_f32(syn.bits_u16(X))).astype(np.float64) @ \
+            np.abs(oracle.bf16_to_f32(syn.bits_u16(A))).astype(np.float64).T
+        assert_within(T.cpu().numpy(), Tr, Tb, "T")
+    assert_status_clean(lbq)
+
+
+def test_linear_fwd_repeatable(lbq):
+    """Same inputs, same bits (split-K partials are summed in a fixed order)."""
+    X, W, A, B = fwd_problem(4, 512, 2048, 16, seed=3)
+    qw = lbq.QuantizedWeight(512, 2048, "minmax", 4).quantize(W.cuda())
+    Y1, _ = lbq.linear_fwd(X.cuda(), qw, A.cuda(), B.cuda(), 2.0)
+    Y2, _ = lbq.linear_fwd(X.cuda(), qw, A.cuda(), B.cuda(), 2.0)
+    assert torch.equal(Y1, Y2)
+
+
+def test_channel_mix_fwd(lbq):
+    m, n, k = 16, 512, 1024
+    X, W, A, B = fwd_problem(m, n, k, 16, seed=77)
+    perm, n4 = syn.channel_mix_perm(n, 0.25, seed=1)
+    Wp = W[torch.from_numpy(perm.astype(np.int64))]
+    hi = lbq.QuantizedWeight(n4, k, "minmax", 4).quantize(Wp[:n4].contiguous().cuda())
+    lo = lbq.QuantizedWeight(n - n4, k, "minmax", 2).quantize(Wp[n4:].contiguous().cuda())
+    mix = lbq.ChannelMixWeight(hi, lo, perm)
+    Y, _ = lbq.linear_fwd(X.cuda(), mix, A.cuda(), B.cuda(), 2.0)
+    torch.cuda.synchronize()
+    What = np.zeros((n, k), np.float32)
+    What[perm[:n4]] = oracle_weight(Wp[:n4].contiguous(), "minmax", 4, False, None)
+    What[perm[n4:]] = oracle_weight(Wp[n4:].contiguous(), "minmax", 2, False, None)
+    Yr, _, Yb = oracle.linear_fwd(syn.bits_u16(X), What, syn.bits_u16(A), syn.bits_u16(B), 2.0)
+    assert_within(Y.cpu().numpy(), Yr, Yb, "Y (channel-mix)")
+
+
+# --------------------------------------------------------------------------- backward
+BWD_CASES = [
+    (8, 256, 512, 8, 4),
+    (1, 256, 512, 0, 4),
+    (16, 384, 1024, 16, 4),
+    (70, 200, 640, 16, 4),
+    (130, 256, 512, 64, 4),
+    (16, 256, 512, 8, 2),
+    (100, 256, 512, 0, 2),
+]
+
+
+@pytest.mark.parametrize("m,n,k,rank,bits", BWD_CASES)
+def test_linear_bwd_parity(lbq, m, n, k, rank, bits):
+    s = 2.0
+    X, W, A, B = fwd_problem(m, n, k, rank, seed=m + 7 * n + k + rank)
+    dY = syn.normal_bf16((m, n), 0.1, seed=m + n + 99)
+    qw = lbq.QuantizedWeight(n, k, "minmax", bits).quantize(W.cuda())
+    dX, U = lbq.linear_bwd(dY.cuda(), qw, None if A is None else A.cuda(), None if B is None else B.cuda(), s)
+    torch.cuda.synchronize()
+    What = oracle_weight(W, "minmax", bits, False, None)
+    dXr, Ur, dXb = oracle.linear_bwd(syn.bits_u16(dY), What, None if A is None else syn.bits_u16(A),
+                                     None if B is None else syn.bits_u16(B), s)
+    assert_within(dX.cpu().numpy(), dXr, dXb, "dX")
+    if rank:
+        Ub = np.abs(oracle.bf16_to_f32(syn.bits_u16(dY))).astype(np.float64) @ \
+            np.abs(oracle.bf16_to_f32(syn.bits_u16(B))).astype(np.float64)
+        assert_within(U.cpu().numpy(), Ur, Ub, "U")
+    assert_status_clean(lbq)
+
+
+@pytest.mark.parametrize("m,n,k,rank", [(8, 256, 512, 8), (130, 384, 768, 16), (64, 200, 512, 64)])
+def test_lora_grads_parity(lbq, m, n, k, rank):
+    s = 2.0
+    X, W, A, B = fwd_problem(m, n, k, rank, seed=m + n + k)
+    dY = syn.normal_bf16((m, n), 0.1, seed=m * 3 + 1)
+    qw = lbq.QuantizedWeight(n, k, "minmax", 4).quantize(W.cuda())
+    _, T = lbq.linear_fwd(X.cuda(), qw, A.cuda(), B.cuda(), s)
+    _, U = lbq.linear_bwd(dY.cuda(), qw, A.cuda(), B.cuda(), s)
+    dA, dB = lbq.lora_grads(X.cuda(), dY.cuda(), T, U, s)
+    torch.cuda.synchronize()
+    dAr, dBr, dAb, dBb = oracle.lora_grads(syn.bits_u16(X), syn.bits_u16(dY), syn.bits_u16(A), syn.bits_u16(B), s)
+    assert_within(dA.cpu().numpy(), dAr, dAb, "dA")
+    assert_within(dB.cpu().numpy(), dBr, dBb, "dB")
+    assert_status_clean(lbq)
