@@ -34,7 +34,7 @@ __global__ void __launch_bounds__(256) minmax_quantize_kernel(const uint4* __res
     constexpr float Q = static_cast<float>((1 << BITS) - 1);
     const int lane = threadIdx.x & 31;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t base = (static_cast<int64_t>(blockIdx.x) * blockDim.x) & ~int64_t(31); base < nchunks;
+    for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31u); base < nchunks;
          base += stride) {
         const int64_t chunk = base + lane;
         const bool valid = chunk < nchunks;
@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(256) codebook_quantize_kernel(const uint4* __r
     const int lane = threadIdx.x & 31;
     double my_sum = 0.0;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t base = (static_cast<int64_t>(blockIdx.x) * blockDim.x) & ~int64_t(31); base < nchunks;
+    for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31u); base < nchunks;
          base += stride) {
         const int64_t chunk = base + lane;
         const bool valid = chunk < nchunks;

@@ -126,6 +126,29 @@ def fwd_problem(m, n, k, rank, seed, scheme="minmax", bits=4, double_quant=False
     return X, W, A, B
 
 
+def device_qweight(lbq, W, scheme, bits, double_quant, cb):
+    """A QuantizedWeight whose buffers hold the ORACLE's quantization of W, so
+    that the GEMM tests do not depend on the GPU quantizer."""
+    n, k = W.shape
+    qw = lbq.QuantizedWeight(n, k, scheme, bits, double_quant=double_quant, codebook=cb)
+    if scheme == "minmax":
+        codes, scale, zero = oracle.minmax_quantize(syn.bits_u16(W), bits, qw.group)
+        qw.packed.copy_(torch.from_numpy(oracle.pack(codes, bits)))
+        qw.scale.copy_(torch.from_numpy(scale.view(np.float16)))
+        qw.zero.copy_(torch.from_numpy(zero.view(np.float16)))
+    else:
+        codes, absmax = oracle.codebook_quantize(syn.bits_u16(W), cb)
+        qw.packed.copy_(torch.from_numpy(oracle.pack(codes, 4)))
+        qw.absmax.copy_(torch.from_numpy(absmax))
+        if double_quant:
+            q8, s2, off, _ = oracle.double_quant(absmax)
+            qw.q8.copy_(torch.from_numpy(q8))
+            qw.s2.copy_(torch.from_numpy(s2))
+            qw.offset.fill_(float(off))
+    torch.cuda.synchronize()
+    return qw
+
+
 def oracle_weight(W, scheme, bits, double_quant, cb):
     n, k = W.shape
     if scheme == "minmax":
@@ -162,7 +185,7 @@ FWD_CASES = [
 def test_linear_fwd_parity(lbq, m, n, k, rank, scheme, bits, dq):
     cb = syn.codebook_normal16()
     X, W, A, B = fwd_problem(m, n, k, rank, seed=m * 131 + n + k + rank, scheme=scheme, bits=bits)
-    qw = lbq.QuantizedWeight(n, k, scheme, bits, double_quant=dq, codebook=cb).quantize(W.cuda())
+    qw = device_qweight(lbq, W, scheme, bits, dq, cb)
     s = 2.0
     Y, T = lbq.linear_fwd(X.cuda(), qw, None if A is None else A.cuda(), None if B is None else B.cuda(), s)
     torch.cuda.synchronize()
@@ -180,7 +203,7 @@ def test_linear_fwd_parity(lbq, m, n, k, rank, scheme, bits, dq):
 def test_linear_fwd_repeatable(lbq):
     """Same inputs, same bits (split-K partials are summed in a fixed order)."""
     X, W, A, B = fwd_problem(4, 512, 2048, 16, seed=3)
-    qw = lbq.QuantizedWeight(512, 2048, "minmax", 4).quantize(W.cuda())
+    qw = device_qweight(lbq, W, "minmax", 4, False, None)
     Y1, _ = lbq.linear_fwd(X.cuda(), qw, A.cuda(), B.cuda(), 2.0)
     Y2, _ = lbq.linear_fwd(X.cuda(), qw, A.cuda(), B.cuda(), 2.0)
     assert torch.equal(Y1, Y2)
@@ -191,8 +214,8 @@ def test_channel_mix_fwd(lbq):
     X, W, A, B = fwd_problem(m, n, k, 16, seed=77)
     perm, n4 = syn.channel_mix_perm(n, 0.25, seed=1)
     Wp = W[torch.from_numpy(perm.astype(np.int64))]
-    hi = lbq.QuantizedWeight(n4, k, "minmax", 4).quantize(Wp[:n4].contiguous().cuda())
-    lo = lbq.QuantizedWeight(n - n4, k, "minmax", 2).quantize(Wp[n4:].contiguous().cuda())
+    hi = device_qweight(lbq, Wp[:n4].contiguous(), "minmax", 4, False, None)
+    lo = device_qweight(lbq, Wp[n4:].contiguous(), "minmax", 2, False, None)
     mix = lbq.ChannelMixWeight(hi, lo, perm)
     Y, _ = lbq.linear_fwd(X.cuda(), mix, A.cuda(), B.cuda(), 2.0)
     torch.cuda.synchronize()
@@ -220,7 +243,7 @@ def test_linear_bwd_parity(lbq, m, n, k, rank, bits):
     s = 2.0
     X, W, A, B = fwd_problem(m, n, k, rank, seed=m + 7 * n + k + rank)
     dY = syn.normal_bf16((m, n), 0.1, seed=m + n + 99)
-    qw = lbq.QuantizedWeight(n, k, "minmax", bits).quantize(W.cuda())
+    qw = device_qweight(lbq, W, "minmax", bits, False, None)
     dX, U = lbq.linear_bwd(dY.cuda(), qw, None if A is None else A.cuda(), None if B is None else B.cuda(), s)
     torch.cuda.synchronize()
     What = oracle_weight(W, "minmax", bits, False, None)
@@ -239,7 +262,7 @@ def test_lora_grads_parity(lbq, m, n, k, rank):
     s = 2.0
     X, W, A, B = fwd_problem(m, n, k, rank, seed=m + n + k)
     dY = syn.normal_bf16((m, n), 0.1, seed=m * 3 + 1)
-    qw = lbq.QuantizedWeight(n, k, "minmax", 4).quantize(W.cuda())
+    qw = device_qweight(lbq, W, "minmax", 4, False, None)
     _, T = lbq.linear_fwd(X.cuda(), qw, A.cuda(), B.cuda(), s)
     _, U = lbq.linear_bwd(dY.cuda(), qw, A.cuda(), B.cuda(), s)
     dA, dB = lbq.lora_grads(X.cuda(), dY.cuda(), T, U, s)
