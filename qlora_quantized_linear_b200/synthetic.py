@@ -40,15 +40,18 @@ LLAMA3_70B_SHAPES = {
 }
 
 
-def _gen(seed: int) -> torch.Generator:
-    g = torch.Generator(device="cpu")
+def _gen(seed: int, device="cpu") -> torch.Generator:
+    g = torch.Generator(device=device)
     g.manual_seed(int(seed))
     return g
 
 
-def normal_bf16(shape, std: float, seed: int) -> torch.Tensor:
-    """bf16 tensor of N(0, std^2) samples (drawn in fp32, rounded once)."""
-    x = torch.randn(tuple(shape), generator=_gen(seed), dtype=torch.float32)
+def normal_bf16(shape, std: float, seed: int, device="cpu") -> torch.Tensor:
+    """bf16 tensor of N(0, std^2) samples (drawn in fp32, rounded once).
+    device="cuda" draws with the device generator (a different stream of
+    numbers than the CPU one for the same seed; used for large benchmark
+    inputs that never meet the oracle)."""
+    x = torch.randn(tuple(shape), generator=_gen(seed, device), dtype=torch.float32, device=device)
     if std != 1.0:
         x.mul_(std)
     return x.to(torch.bfloat16)
@@ -64,13 +67,13 @@ def outlier_columns(k: int, frac: float, seed: int) -> torch.Tensor:
 
 
 def weight_bf16(n: int, k: int, std: float, seed: int,
-                outlier_frac: float = 0.0, outlier_scale: float = 20.0) -> torch.Tensor:
+                outlier_frac: float = 0.0, outlier_scale: float = 20.0, device="cpu") -> torch.Tensor:
     """Weight [n, k] ~ N(0, std^2), with `outlier_frac` of its input channels
     (columns) multiplied by `outlier_scale` before the bf16 rounding."""
-    x = torch.randn((n, k), generator=_gen(seed), dtype=torch.float32)
+    x = torch.randn((n, k), generator=_gen(seed, device), dtype=torch.float32, device=device)
     x.mul_(std)
     if outlier_frac > 0:
-        cols = outlier_columns(k, outlier_frac, seed)
+        cols = outlier_columns(k, outlier_frac, seed).to(device)
         x[:, cols] *= outlier_scale
     return x.to(torch.bfloat16)
 
