@@ -159,6 +159,35 @@ lbq_status lbq_linear_fwd(const void* X, int m, const lbq_qweight* q,
                           float* Y, float* T_save, void* workspace,
                           size_t workspace_bytes, lbq_stream_t stream);
 
+/*
+ * lbq_linear_fwd_noalloc -- the same forward as lbq_linear_fwd for callers
+ * that cannot allocate device memory: code whose device memory is all handed
+ * out up front by another runtime's pool, real-time or embedded loops that
+ * must not allocate after start-up, and callers for whom a cudaMalloc (which
+ * can synchronize the device) is not allowed at the point of the call.  It
+ * takes no workspace: the split-K scratch of the decode-sized path lives in
+ * a fixed array of 8 MiB (8388608 bytes) that the library declares once per
+ * device and every device that loads the library keeps until the process
+ * exits.  (The source pages have no
+ * counterpart of this entry point.)
+ *
+ * Arguments, layouts, results and errors are those of lbq_linear_fwd, plus:
+ *  - LBQ_EWORKSPACE when this call's scratch (lbq_linear_fwd_workspace_size)
+ *    is larger than the 8 MiB array; nothing is launched then.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current); make that first call before any stream capture.
+ *  - All calls share the one array: calls that can run at the same time on
+ *    the GPU (different streams, overlapping graphs) race on it and must be
+ *    ordered by the caller.  The per-tile counters in it are cleared by every
+ *    call (an asynchronous memset on `stream`), so leftover contents do not
+ *    matter.
+ *  - It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+lbq_status lbq_linear_fwd_noalloc(const void* X, int m, const lbq_qweight* q,
+                                  const void* A, const void* B, int rank,
+                                  float s, float* Y, float* T_save,
+                                  lbq_stream_t stream);
+
 /* The same forward for a channel-mix weight; Y columns in original order. */
 size_t lbq_linear_fwd_mix_workspace_size(int m, const lbq_qweight_mix* q,
                                          int rank);

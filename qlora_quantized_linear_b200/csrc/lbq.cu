@@ -248,6 +248,36 @@ lbq_status launch_bwd_bits(int nt, const BwdParams& p, const void* dY, const uin
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Fixed scratch of lbq_linear_fwd_noalloc.  Every device that loads this
+// library holds one copy until the process exits.  In host code the name
+// below is only a stand-in for the symbol; the device address of each
+// device's copy comes from cudaGetSymbolAddress, taken once per device with
+// that device current, on the first call made on it.
+// ---------------------------------------------------------------------------
+static constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+lbq_status noalloc_scratch_address(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LBQ_ECUDA;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return LBQ_EUNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return LBQ_ECUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return LBQ_OK;
+}
+}  // namespace
+
 // ===========================================================================
 // C ABI
 // ===========================================================================
@@ -357,6 +387,27 @@ lbq_status lbq_linear_fwd(const void* X, int m, const lbq_qweight* q, const void
         if ((st = last_launch()) != LBQ_OK) return st;
     }
     return run_fwd_gemm(X, m, q, B, rank, s, T_save, Y, q->n, nullptr, workspace, sms, cs);
+}
+
+lbq_status lbq_linear_fwd_noalloc(const void* X, int m, const lbq_qweight* q, const void* A, const void* B, int rank,
+                                  float s, float* Y, float* T_save, lbq_stream_t stream) {
+    lbq_status st = check_qweight(q, true);
+    if (st != LBQ_OK) return st;
+    if (m < 1 || !X || !Y) return LBQ_EINVAL;
+    if (!aligned16(X) || !aligned16(Y)) return LBQ_EALIGN;
+    if ((st = check_lora(rank, A, B, T_save)) != LBQ_OK) return st;
+    const int sms = sm_count();
+    const size_t need = plan_gemm(m, q->n, q->k / 64, sms).workspace();
+    if (need > kNoAllocScratchBytes) return LBQ_EWORKSPACE;  // this call's scratch does not fit
+    void* scratch = nullptr;
+    if (need > 0 && (st = noalloc_scratch_address(&scratch)) != LBQ_OK) return st;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    if (rank > 0) {
+        lora_rowdot_kernel<false><<<m, 256, 0, cs>>>(static_cast<const uint16_t*>(X), q->k,
+                                                     static_cast<const uint16_t*>(A), rank, T_save);
+        if ((st = last_launch()) != LBQ_OK) return st;
+    }
+    return run_fwd_gemm(X, m, q, B, rank, s, T_save, Y, q->n, nullptr, scratch, sms, cs);
 }
 
 size_t lbq_linear_fwd_mix_workspace_size(int m, const lbq_qweight_mix* q, int rank) {

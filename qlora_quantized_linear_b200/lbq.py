@@ -56,6 +56,7 @@ _SIGS = {
     "lbq_dequantize": (_int, [_QP, _vp, _vp]),
     "lbq_linear_fwd_workspace_size": (_sz, [_int, _QP, _int]),
     "lbq_linear_fwd": (_int, [_vp, _int, _QP, _vp, _vp, _int, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "lbq_linear_fwd_noalloc": (_int, [_vp, _int, _QP, _vp, _vp, _int, _f32, _vp, _vp, _vp]),
     "lbq_linear_fwd_mix_workspace_size": (_sz, [_int, _MP, _int]),
     "lbq_linear_fwd_mix": (_int, [_vp, _int, _MP, _vp, _vp, _int, _f32, _vp, _vp, _vp, _sz, _vp]),
     "lbq_linear_bwd_workspace_size": (_sz, [_int, _QP, _int]),
@@ -81,6 +82,7 @@ lbq_quantize = _L.lbq_quantize
 lbq_dequantize = _L.lbq_dequantize
 lbq_linear_fwd_workspace_size = _L.lbq_linear_fwd_workspace_size
 lbq_linear_fwd = _L.lbq_linear_fwd
+lbq_linear_fwd_noalloc = _L.lbq_linear_fwd_noalloc
 lbq_linear_fwd_mix_workspace_size = _L.lbq_linear_fwd_mix_workspace_size
 lbq_linear_fwd_mix = _L.lbq_linear_fwd_mix
 lbq_linear_bwd_workspace_size = _L.lbq_linear_bwd_workspace_size
