@@ -47,6 +47,11 @@ def parse_args():
     ap.add_argument("--rows", choices=["all", "none"], default="all",
                     help="also measure the other workloads (training step, 70B codebook, mixed, quantize)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default=None,
+                    help="run one kernel configuration `reps` times and exit (for ncu captures): "
+                         "decode_<matrix>_m<M> | train_<matrix>_{fwd,bwd,grads} | codebook70b_<matrix>_m<M> | "
+                         "quantize_<matrix>")
+    ap.add_argument("--reps", type=int, default=3)
     return ap.parse_args()
 
 
@@ -571,9 +576,70 @@ def run_reference(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- single cases (ncu)
+def run_case(args):
+    """One kernel configuration, `reps` times, on fresh inputs; prints the
+    CUDA-event time of the last call.  Inputs of the 8B/70B shapes exceed no
+    more than a few hundred MB on the device."""
+    import torch
+    from qlora_quantized_linear_b200 import lbq, synthetic as syn
+    torch.cuda.set_device(0)
+    kind, rest = args.case.split("_", 1)
+    name, arg = rest.rsplit("_", 1)
+    stream = torch.cuda.current_stream()
+    if kind == "decode" or kind == "train":
+        n, k = syn.LLAMA3_8B_SHAPES[name]
+        W = syn.weight_bf16(n, k, 0.02, seed=1, outlier_frac=0.001, device="cuda")
+        qw = lbq.QuantizedWeight(n, k, "minmax", 4).quantize(W)
+        del W
+        if kind == "decode":
+            m = int(arg[1:])
+            X = syn.normal_bf16((m, k), 1.0, seed=2, device="cuda")
+            fn = lambda: lbq.linear_fwd(X, qw)
+        else:
+            m, r, s = 4096, 16, 2.0
+            X = syn.normal_bf16((m, k), 1.0, seed=2, device="cuda")
+            A = syn.normal_bf16((r, k), 0.01, seed=3, device="cuda")
+            B = syn.normal_bf16((n, r), 0.01, seed=4, device="cuda")
+            dY = syn.normal_bf16((m, n), 0.1, seed=5, device="cuda")
+            _, T = lbq.linear_fwd(X, qw, A, B, s)
+            _, U = lbq.linear_bwd(dY, qw, A, B, s)
+            fn = {"fwd": lambda: lbq.linear_fwd(X, qw, A, B, s),
+                  "bwd": lambda: lbq.linear_bwd(dY, qw, A, B, s),
+                  "grads": lambda: lbq.lora_grads(X, dY, T, U, s)}[arg]
+    elif kind == "codebook70b":
+        n, k = syn.LLAMA3_70B_SHAPES[name]
+        W = syn.weight_bf16(n, k, 0.015, seed=1, device="cuda")
+        qw = lbq.QuantizedWeight(n, k, "codebook", double_quant=True, codebook=syn.codebook_normal16()).quantize(W)
+        del W
+        m = int(arg[1:])
+        X = syn.normal_bf16((m, k), 1.0, seed=2, device="cuda")
+        fn = lambda: lbq.linear_fwd(X, qw)
+    elif kind == "quantize":
+        n, k = (syn.LLAMA3_8B_SHAPES.get(name) or syn.LLAMA3_70B_SHAPES[name])
+        W = syn.weight_bf16(n, k, 0.02, seed=1, device="cuda")
+        qw = lbq.QuantizedWeight(n, k, "minmax", 4) if arg == "int4" else \
+            lbq.QuantizedWeight(n, k, "codebook", double_quant=True, codebook=syn.codebook_normal16())
+        fn = lambda: qw.quantize(W)
+    else:
+        raise SystemExit(f"unknown case {args.case}")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(args.reps - 1):
+        fn()
+    e0.record(stream)
+    fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    print(json.dumps({"case": args.case, "ms_last_call": round(e0.elapsed_time(e1), 4),
+                      "device_status": lbq.device_status()}))
+    return 0
+
+
 # ----------------------------------------------------------------------------- main
 def main():
     args = parse_args()
+    if args.case:
+        return run_case(args)
     if args.impl == "reference":
         return run_reference(args)
     # CPU baseline first (before any CUDA work; OpenMP threads of the oracle)
