@@ -150,8 +150,13 @@ lbq_status lbq_dequantize(const lbq_qweight* q, float* W_f32,
  * rank == 0 (A, B, T_save may be NULL) is the plain dequantize-GEMM.
  * 1 <= rank <= 64 needs T_save.  m >= 1.  The weight is dequantized to bf16
  * (the compute dtype) inside the kernel and products accumulate in fp32.
- * workspace: lbq_linear_fwd_workspace_size(m, q, rank) bytes of device memory
- * (contents ignored); NULL is accepted when that size is 0.
+ * workspace: lbq_linear_fwd_workspace_size(m, q, rank) bytes of device memory,
+ * zero-filled before the first call that uses it; NULL is accepted when that
+ * size is 0.  It holds split-K partial sums and per-tile arrival counters;
+ * every call leaves the counters at zero again, so one zero-fill at
+ * allocation serves any number of later calls of any shape.  After a call
+ * whose kernels timed out (LBQ_ETIMEOUT from lbq_device_status), zero it
+ * again.  Calls that may run at the same time need separate workspaces.
  */
 size_t lbq_linear_fwd_workspace_size(int m, const lbq_qweight* q, int rank);
 lbq_status lbq_linear_fwd(const void* X, int m, const lbq_qweight* q,
@@ -178,9 +183,11 @@ lbq_status lbq_linear_fwd(const void* X, int m, const lbq_qweight* q,
  *    that device current); make that first call before any stream capture.
  *  - All calls share the one array: calls that can run at the same time on
  *    the GPU (different streams, overlapping graphs) race on it and must be
- *    ordered by the caller.  The per-tile counters in it are cleared by every
- *    call (an asynchronous memset on `stream`), so leftover contents do not
- *    matter.
+ *    ordered by the caller.  The array starts zero-filled (static storage)
+ *    and every call leaves its per-tile counters at zero again; after a call
+ *    whose kernels timed out (LBQ_ETIMEOUT from lbq_device_status) the
+ *    counters may not be zero and later results of this entry point are
+ *    undefined.
  *  - It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  */
 lbq_status lbq_linear_fwd_noalloc(const void* X, int m, const lbq_qweight* q,

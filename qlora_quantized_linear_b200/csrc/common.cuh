@@ -32,6 +32,22 @@ __device__ uint32_t g_status;
 
 __device__ __forceinline__ void record_status(uint32_t flag) { atomicOr(&g_status, flag); }
 
+// Optional pipeline trace (built only with -DLBQ_TRACE): SM clock stamps of
+// the pipeline events of CTA (0, 0, 0), read back with lbq_trace_read().
+#ifdef LBQ_TRACE
+constexpr int kTraceKinds = 8, kTraceLen = 256;
+__device__ long long g_trace[kTraceKinds][kTraceLen];
+#define LBQ_TRACE_EVENT(kind, idx)                                                                   \
+    do {                                                                                             \
+        if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (idx) < kTraceLen && (idx) >= 0) \
+            g_trace[(kind)][(idx)] = clock64();                                                      \
+    } while (0)
+#else
+#define LBQ_TRACE_EVENT(kind, idx) \
+    do {                           \
+    } while (0)
+#endif
+
 // Upper bound for every spin-wait: about two seconds of device time.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint32_t kWaitLimitIters = 1u << 30;
@@ -118,6 +134,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
+                                            int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
 

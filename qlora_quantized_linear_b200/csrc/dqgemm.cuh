@@ -7,17 +7,21 @@
 // dequantized to the bf16 compute dtype inside the kernel).  One CTA computes
 // a tile of 128 output channels x NT tokens:
 //
-//   warp 0      TMA producer: per k-block of 64, the X tile [NT x 64] bf16
-//               (128-byte swizzle, the MMA's B operand) and the packed weight
-//               tile [128 rows x 64 codes] into a STAGES-deep smem ring.
+//   warp 0      TMA producer: X tiles [NT x 64] bf16 (128-byte swizzle, the
+//               MMA's B operand), several k-blocks per 3-D box, into one ring;
+//               the packed weights in chunks of 128 rows x 128 bytes (256
+//               INT4 or 512 INT2 codes per row, 128-byte swizzle) into a
+//               second ring -- wide boxes keep the TMA engine efficient.
 //   warp 1      allocates tensor memory; lane 0 issues tcgen05.mma.
-//   warps 2..5  dequantize: thread i owns output channel i, which is TMEM
-//               lane i.  It unpacks its row's codes from smem, forms bf16
-//               W_hat values and stores them with tcgen05.st straight into
-//               the MMA's A operand in tensor memory (an ASTAGES-deep ring),
-//               so dequantized weights never touch shared memory.  After the
-//               last k-block the same threads drain the fp32 accumulator from
-//               tensor memory, add the adapter term and write Y.
+//   warps 2..9  dequantize: output channel i is TMEM lane i; the two warps
+//               of a lane quarter each take half of a k-block.  A thread
+//               unpacks its row's codes from smem, forms bf16 W_hat values and
+//               stores them with tcgen05.st straight into the MMA's A operand
+//               in tensor memory (an ASTAGES-deep ring), so dequantized
+//               weights never touch shared memory.  Per-row scale/zero are
+//               loaded one k-block ahead.  After the last k-block the same
+//               threads drain the fp32 accumulator from tensor memory, add
+//               the adapter term and write Y.
 //
 // Decode-sized problems (few tokens) split K across CTAs; each CTA writes an
 // fp32 partial tile to the workspace and the last CTA of a tile (found with a
@@ -58,11 +62,33 @@ struct FwdParams {
 template <int KIND>
 struct WeightTile {
     static constexpr int kRowBytes = (KIND == kInt2) ? 16 : 32;  // packed bytes per row per k-block
+    // The forward kernel loads weights in chunks of 128 bytes per row (a
+    // 128-row x 128-byte box, 128-byte swizzle): kSub k-blocks per chunk.
+    static constexpr int kSub = 128 / kRowBytes;
+};
+
+// Shared-memory layout of the forward kernel: a ring of XS activation slots
+// (XB k-blocks of NT x 64 bf16 each, fetched by one 3-D TMA box), a ring of
+// WS packed-weight chunks (128 rows x 128 B), the mbarriers and the adapter T
+// tile [NT, rank_pad].  Few, large TMA boxes: each box costs the TMA engine
+// a fixed issue-to-completion slot, so small boxes waste its throughput.
+template <int NT, int XS, int XB, int WS, int AS>
+struct FwdSmem {
+    static constexpr int kXTile = NT * 128;              // one k-block of X
+    static constexpr int kXBytes = XB * kXTile;          // one X slot
+    static constexpr int kWBytes = 128 * 128;
+    static constexpr size_t kX = 0;
+    static constexpr size_t kW = kX + size_t(XS) * kXBytes;
+    static constexpr size_t kBar = kW + size_t(WS) * kWBytes;
+    static constexpr int kNumBars = 2 * XS + 2 * WS + 2 * AS + 1;
+    static constexpr size_t kMisc = kBar + kNumBars * 8;
+    static constexpr size_t kLoraT = (kMisc + 128 + 15) / 16 * 16;
+    static size_t total(int rank_pad) { return kLoraT + size_t(NT) * rank_pad * 4 + 1024; }
 };
 
 // Shared-memory layout of one CTA: a ring of STAGES (activation tile, packed
 // weight tile) pairs, the mbarriers, and the adapter T tile [NT, rank_pad].
-template <int NT, int STAGES, int ASTAGES, int WTILE>
+template <int NT, int STAGES, int ASTAGES, int WTILE, int TABBYTES = 0>
 struct GemmSmem {
     static constexpr int kXBytes = NT * 128;   // NT rows x 64 bf16
     static constexpr int kWBytes = WTILE;      // packed weight tile
@@ -71,9 +97,8 @@ struct GemmSmem {
     static constexpr size_t kBar = (kW + size_t(STAGES) * kWBytes + 7) / 8 * 8;
     static constexpr int kNumBars = 2 * STAGES + 2 * ASTAGES + 1;
     static constexpr size_t kMisc = kBar + kNumBars * 8;
-    static constexpr size_t kTab = (kMisc + 128 + 15) / 16 * 16;   // per-stage dequant tables (backward)
-    static constexpr size_t kTabBytes = 64 * 2 * 16;
-    static constexpr size_t kLoraT = kTab + size_t(STAGES) * kTabBytes;
+    static constexpr size_t kTab = (kMisc + 128 + 15) / 16 * 16;   // dequant tables (backward only)
+    static constexpr size_t kLoraT = kTab + size_t(TABBYTES);
     static size_t total(int rank_pad) { return kLoraT + size_t(NT) * rank_pad * 4 + 1024; }
 };
 
@@ -122,6 +147,13 @@ __device__ __forceinline__ uint32_t hsub_hmul_bf16x2(uint32_t v, uint32_t sub, u
     return *reinterpret_cast<uint32_t*>(&a);
 }
 
+__device__ __forceinline__ uint32_t hsub_bf16x2(uint32_t v, uint32_t sub) {
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&v);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&sub);
+    a = __hsub2(a, b);
+    return *reinterpret_cast<uint32_t*>(&a);
+}
+
 // Per-row, per-group dequantization constants of the MinMax format.
 struct MinMaxConst {
     uint32_t sub2;   // bf16x2 (128 + zero) in both halves
@@ -147,22 +179,49 @@ __device__ __forceinline__ uint32_t minmax_pair_exact(uint32_t q0, uint32_t q1, 
     return pack_bf16x2_rn(w0, w1);
 }
 
-// Dequantize this thread's row of one k-block (64 codes) into 32 bf16x2 words.
+// Raw per-(row, k-block) constants, loaded one k-block ahead of their use so
+// that the load latency hides behind the previous block's dequantization.
+struct PreConst {
+    uint32_t a, b;   // MinMax: scale bits, zero bits; codebook: absmax bits or (q8, s2 bits)
+};
+
 template <int KIND>
-__device__ __forceinline__ void dequant_row_kblock(const uint8_t* wrow_smem, int row, int kb, int64_t grow,
-                                                   const FwdParams& p, const float* s_cb, uint32_t (&out)[32]) {
+__device__ __forceinline__ PreConst preload_const(const FwdParams& p, int64_t grow, int kb, bool ok) {
+    PreConst c{0u, 0u};
+    if (!ok) return c;
+    if (KIND != kCode4) {
+        const int g = (KIND == kInt4) ? (kb >> 1) : kb;
+        c.a = __ldg(p.scale + grow * p.ngroups + g);
+        c.b = __ldg(p.zero + grow * p.ngroups + g);
+    } else {
+        const int64_t b = grow * (p.k / 64) + kb;
+        if (p.q8 != nullptr) {
+            c.a = static_cast<uint32_t>(static_cast<int32_t>(__ldg(p.q8 + b)));
+            c.b = __float_as_uint(__ldg(p.s2 + (b >> 8)));
+        } else {
+            c.a = __float_as_uint(__ldg(p.absmax + b));
+        }
+    }
+    return c;
+}
+
+// Dequantize half of this thread's row of one k-block (32 codes) into 16
+// bf16x2 words (first code of each pair in the low half).  `wrow` is the row's
+// 128-byte line of the weight chunk, stored by TMA with the 128-byte swizzle
+// (16-byte unit u of row r sits at unit u ^ (r & 7)); `byte0` is the offset of
+// this half k-block's codes within the line.
+template <int KIND>
+__device__ __forceinline__ void dequant_half_kblock(const uint8_t* wrow, int row, int byte0, PreConst pc,
+                                                    float dq_offset, bool has_dq, const float* s_cb,
+                                                    uint32_t (&out)[16]) {
+    const int unit = (byte0 >> 4) ^ (row & 7);
     if (KIND == kInt4) {
-        // 32 bytes, stored by TMA with the 32-byte swizzle: 16-byte chunk c of
-        // row r sits at chunk c ^ ((r >> 2) & 1).
-        const int sw = (row >> 2) & 1;
-        const uint4 c0 = *reinterpret_cast<const uint4*>(wrow_smem + 16 * (0 ^ sw));
-        const uint4 c1 = *reinterpret_cast<const uint4*>(wrow_smem + 16 * (1 ^ sw));
-        const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        const int g = (kb * 64) / 128;
-        const MinMaxConst c = minmax_const(__ldg(p.scale + grow * p.ngroups + g), __ldg(p.zero + grow * p.ngroups + g));
+        const uint4 c4 = *reinterpret_cast<const uint4*>(wrow + 16 * unit);
+        const uint32_t w[4] = {c4.x, c4.y, c4.z, c4.w};
+        const MinMaxConst c = minmax_const(static_cast<uint16_t>(pc.a), static_cast<uint16_t>(pc.b));
         if (c.fast) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < 4; ++i) {
                 uint32_t o[4];
                 unpack_int4_word(w[i], o);
 #pragma unroll
@@ -170,19 +229,18 @@ __device__ __forceinline__ void dequant_row_kblock(const uint8_t* wrow_smem, int
             }
         } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     out[4 * i + j] = minmax_pair_exact((w[i] >> (8 * j + 4)) & 15u, (w[i] >> (8 * j)) & 15u, c);
         }
     } else if (KIND == kInt2) {
-        const uint4 c0 = *reinterpret_cast<const uint4*>(wrow_smem);
-        const uint32_t w[4] = {c0.x, c0.y, c0.z, c0.w};
-        const int g = kb;  // group 64 == k-block
-        const MinMaxConst c = minmax_const(__ldg(p.scale + grow * p.ngroups + g), __ldg(p.zero + grow * p.ngroups + g));
+        const uint2 c2 = *reinterpret_cast<const uint2*>(wrow + 16 * unit + (byte0 & 15));
+        const uint32_t w[2] = {c2.x, c2.y};
+        const MinMaxConst c = minmax_const(static_cast<uint16_t>(pc.a), static_cast<uint16_t>(pc.b));
         if (c.fast) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < 2; ++i) {
                 uint32_t o[8];
                 unpack_int2_word(w[i], o);
 #pragma unroll
@@ -190,7 +248,7 @@ __device__ __forceinline__ void dequant_row_kblock(const uint8_t* wrow_smem, int
             }
         } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 2; ++i)
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -199,21 +257,15 @@ __device__ __forceinline__ void dequant_row_kblock(const uint8_t* wrow_smem, int
                                                                    (w[i] >> (8 * j + 4 - 4 * h)) & 3u, c);
         }
     } else {
-        // codebook: W_hat = bf16(fp32(codebook[code] * absmax)), absmax per 64
-        const int sw = (row >> 2) & 1;
-        const uint4 c0 = *reinterpret_cast<const uint4*>(wrow_smem + 16 * (0 ^ sw));
-        const uint4 c1 = *reinterpret_cast<const uint4*>(wrow_smem + 16 * (1 ^ sw));
-        const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        const int64_t b = grow * (p.k / 64) + kb;
-        float a;
-        if (p.q8 != nullptr) {
-            a = __fadd_rn(__fmul_rn(__fdiv_rn(static_cast<float>(__ldg(p.q8 + b)), 127.0f), __ldg(p.s2 + (b >> 8))),
-                          __ldg(p.offset));
-        } else {
-            a = __ldg(p.absmax + b);
-        }
+        // codebook: W_hat = bf16(fp32(codebook[code] * absmax')), absmax per 64
+        const uint4 c4 = *reinterpret_cast<const uint4*>(wrow + 16 * unit);
+        const uint32_t w[4] = {c4.x, c4.y, c4.z, c4.w};
+        const float a = has_dq ? __fadd_rn(__fmul_rn(__fdiv_rn(static_cast<float>(static_cast<int32_t>(pc.a)), 127.0f),
+                                                     __uint_as_float(pc.b)),
+                                           dq_offset)
+                               : __uint_as_float(pc.a);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int j = 0; j < 4; ++j)
                 out[4 * i + j] = pack_bf16x2_rn(__fmul_rn(s_cb[(w[i] >> (8 * j + 4)) & 15u], a),
@@ -226,9 +278,6 @@ __device__ __forceinline__ void dequant_row_kblock(const uint8_t* wrow_smem, int
 // (bf16): B[out_col, :] in the forward pass, A[:, k] in the backward pass.
 __device__ __forceinline__ void lora_add16(float (&acc)[16], const float* sT, int rp, int rank,
                                            const uint16_t* brow, float s, int64_t bstride = 1) {
-    float d[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) d[j] = 0.0f;
     for (int u0 = 0; u0 < rp; u0 += 16) {
         float b[16];
 #pragma unroll
@@ -236,31 +285,57 @@ __device__ __forceinline__ void lora_add16(float (&acc)[16], const float* sT, in
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             const float4* t4 = reinterpret_cast<const float4*>(sT + j * rp + u0);
+            float d = 0.0f;
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
                 const float4 t = t4[v];
-                d[j] = fmaf(t.x, b[4 * v], d[j]);
-                d[j] = fmaf(t.y, b[4 * v + 1], d[j]);
-                d[j] = fmaf(t.z, b[4 * v + 2], d[j]);
-                d[j] = fmaf(t.w, b[4 * v + 3], d[j]);
+                d = fmaf(t.x, b[4 * v], d);
+                d = fmaf(t.y, b[4 * v + 1], d);
+                d = fmaf(t.z, b[4 * v + 2], d);
+                d = fmaf(t.w, b[4 * v + 3], d);
             }
+            acc[j] = fmaf(s, d, acc[j]);
         }
     }
-#pragma unroll
-    for (int j = 0; j < 16; ++j) acc[j] = fmaf(s, d[j], acc[j]);
 }
 
-template <int NT, int KIND, int STAGES, int ASTAGES>
-__global__ void __launch_bounds__(192, 2)
+// Launch shape of the forward kernel: warp 0 = TMA producer, warp 1 = TMEM
+// allocator + MMA issuer, warps 2..9 = dequantize + epilogue.  Two dequant
+// warps share each TMEM lane quarter (warp & 3); warp group h = (warp-2)/4
+// takes half h of every k-block and, in the epilogue, half h of the tokens.
+constexpr int kFwdThreads = 320;
+constexpr int kDqWarps = 8;
+
+template <int NT>
+struct FwdCfg {
+    static constexpr int kXBlocks = NT <= 16 ? 8 : NT <= 32 ? 4 : NT <= 64 ? 2 : 1;   // k-blocks per X box
+    static constexpr int kXStages = NT <= 32 ? 2 : NT <= 64 ? 3 : 4;
+    static constexpr int kWStages = NT <= 32 ? 4 : NT <= 64 ? 3 : 2;
+    static constexpr int kAStages = NT <= 32 ? 6 : 4;
+    static constexpr int kMinBlocks = NT >= 256 ? 1 : 2;   // CTAs per SM
+};
+
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+template <int NT, int KIND, int XS, int XB, int WS, int AS, int MINB>
+__global__ void __launch_bounds__(kFwdThreads, MINB)
 dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                   const FwdParams p) {
     constexpr int WB = WeightTile<KIND>::kRowBytes;
-    using L = GemmSmem<NT, STAGES, ASTAGES, 128 * WB>;
-    constexpr uint32_t kTxBytes = L::kXBytes + 128 * WB;
+    constexpr int SUB = WeightTile<KIND>::kSub;        // k-blocks per weight chunk
+    using L = FwdSmem<NT, XS, XB, WS, AS>;
     constexpr int kACols = 32;                         // one k-block of 64 bf16 = 32 columns
     constexpr int kDCol = 0;                           // fp32 accumulator: NT columns
     constexpr int kACol0 = (NT + 31) / 32 * 32;        // A ring after the accumulator
-    constexpr uint32_t kTmemCols = tmem_cols_for(kACol0 + kACols * ASTAGES);
+    constexpr uint32_t kTmemCols = tmem_cols_for(kACol0 + kACols * AS);
+    static_assert(kACol0 + kACols * AS <= 512, "tensor memory over-subscribed");
     constexpr uint32_t kIdesc = idesc_bf16_f32(128, NT);
 
     extern __shared__ uint8_t smem_raw[];
@@ -268,11 +343,13 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     uint8_t* sX = smem + L::kX;
     uint8_t* sW = smem + L::kW;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-    uint64_t* full = bars;
-    uint64_t* empty = bars + STAGES;
-    uint64_t* afull = bars + 2 * STAGES;
-    uint64_t* aempty = afull + ASTAGES;
-    uint64_t* dfull = aempty + ASTAGES;
+    uint64_t* fullX = bars;
+    uint64_t* emptyX = fullX + XS;
+    uint64_t* fullW = emptyX + XS;
+    uint64_t* emptyW = fullW + WS;
+    uint64_t* afull = emptyW + WS;
+    uint64_t* aempty = afull + AS;
+    uint64_t* dfull = aempty + AS;
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
     int* s_last = reinterpret_cast<int*>(smem + L::kMisc + 8);
@@ -284,16 +361,21 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     const int t0 = blockIdx.y * NT;
     const int split = blockIdx.z;
     const int kb_total = p.k / 64;
-    const int kb0 = split * p.kb_per_split;
+    const int kb0 = split * p.kb_per_split;            // a multiple of SUB
     const int nkb = min(p.kb_per_split, kb_total - kb0);
+    const int nch = (nkb + SUB - 1) / SUB;              // weight chunks of this CTA
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < STAGES; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1 + 4);
+        for (int i = 0; i < XS; ++i) {
+            mbar_init(&fullX[i], 1);
+            mbar_init(&emptyX[i], 1);
         }
-        for (int i = 0; i < ASTAGES; ++i) {
-            mbar_init(&afull[i], 4);
+        for (int i = 0; i < WS; ++i) {
+            mbar_init(&fullW[i], 1);
+            mbar_init(&emptyW[i], kDqWarps);
+        }
+        for (int i = 0; i < AS; ++i) {
+            mbar_init(&afull[i], kDqWarps);
             mbar_init(&aempty[i], 1);
         }
         mbar_init(dfull, 1);
@@ -313,39 +395,55 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
+    if (threadIdx.x == 0) LBQ_TRACE_EVENT(0, 0);  // kinds: see lbq_trace_read
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
+        // Weight chunks run ahead of the activation tiles: chunk c is issued
+        // before the first k-block that needs it.
         if (lane == 0) {
-            int issued = 0;
-            for (int i = 0; i < nkb; ++i) {
-                const int s = i % STAGES;
-                if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) - 1) & 1, s_abort)) break;
-                mbar_arrive_expect_tx(&full[s], kTxBytes);
-                const int kb = kb0 + i;
-                tma_load_2d(sX + s * L::kXBytes, &tmX, &full[s], kb * 64, t0);
-                tma_load_2d(sW + s * L::kWBytes, &tmW, &full[s], kb * WB, n0);
-                issued = i + 1;
+            int xi = 0, wi = 0;
+            bool ok = true;
+            for (int i = 0; i < nkb && ok; ++i) {
+                if (i % SUB == 0) {
+                    const int c = i / SUB, w = c % WS;
+                    if (c >= WS && !mbar_wait(&emptyW[w], ((c / WS) - 1) & 1, s_abort)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&fullW[w], L::kWBytes);
+                    tma_load_2d(sW + w * L::kWBytes, &tmW, &fullW[w], (kb0 + i) * WB, n0);
+                    wi = c + 1;
+                }
+                if (i % XB == 0) {
+                    const int j = i / XB, x = j % XS;
+                    if (j >= XS && !mbar_wait(&emptyX[x], ((j / XS) - 1) & 1, s_abort)) { ok = false; break; }
+                    LBQ_TRACE_EVENT(6, i);
+                    mbar_arrive_expect_tx(&fullX[x], L::kXBytes);
+                    tma_load_3d(sX + x * L::kXBytes, &tmX, &fullX[x], 0, t0, kb0 + i);
+                    LBQ_TRACE_EVENT(1, i);
+                    xi = j + 1;
+                }
             }
             // never leave with a copy in flight (matters only after an abort)
-            for (int i = max(0, issued - STAGES); i < issued; ++i) mbar_wait_drain(&full[i % STAGES], (i / STAGES) & 1);
+            for (int j = max(0, xi - XS); j < xi; ++j) mbar_wait_drain(&fullX[j % XS], (j / XS) & 1);
+            for (int c = max(0, wi - WS); c < wi; ++c) mbar_wait_drain(&fullW[c % WS], (c / WS) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             bool ok = true;
             for (int i = 0; i < nkb && ok; ++i) {
-                const int s = i % STAGES, a = i % ASTAGES;
-                ok = mbar_wait(&full[s], (i / STAGES) & 1, s_abort) &&
-                     mbar_wait(&afull[a], (i / ASTAGES) & 1, s_abort);
+                const int xj = i / XB, xsub = i - xj * XB, x = xj % XS, a = i % AS;
+                if (xsub == 0) ok = mbar_wait(&fullX[x], (xj / XS) & 1, s_abort);
+                LBQ_TRACE_EVENT(4, i);
+                ok = ok && mbar_wait(&afull[a], (i / AS) & 1, s_abort);
                 if (!ok) break;
                 tc_fence_after();
-                const uint64_t bdesc = smem_desc_k_sw128(smem_u32(sX + s * L::kXBytes));
+                LBQ_TRACE_EVENT(5, i);
+                const uint64_t bdesc = smem_desc_k_sw128(smem_u32(sX + x * L::kXBytes + xsub * L::kXTile));
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     mma_ts(tmem + kDCol, tmem + kACol0 + a * kACols + 8 * j, bdesc + static_cast<uint64_t>(2 * j), kIdesc,
                            (i > 0 || j > 0) ? 1u : 0u);
-                mma_commit(&empty[s]);
+                if (xsub == XB - 1 || i == nkb - 1) mma_commit(&emptyX[x]);
                 mma_commit(&aempty[a]);
             }
             mma_commit(dfull);  // also completes when nothing was issued
@@ -353,51 +451,65 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         }
     } else {
         // ------------------------------------------------------------ dequantize
-        const int q = warp & 3;            // TMEM lane quarter of this warp
-        const int row = q * 32 + lane;     // output channel within the tile
-        const int64_t grow = n0 + row;     // stored weight row
+        const int q = warp & 3;              // TMEM lane quarter of this warp
+        const int half = (warp - 2) >> 2;    // k-block half (and token half in the epilogue)
+        const int row = q * 32 + lane;       // output channel within the tile
+        const int64_t grow = n0 + row;       // stored weight row
         const bool row_ok = grow < p.n;
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        const bool has_dq = (KIND == kCode4) && (p.q8 != nullptr);
+        const float dq_offset = has_dq ? __ldg(p.offset) : 0.0f;
+        PreConst nxt = preload_const<KIND>(p, grow, kb0, row_ok && nkb > 0);
         for (int i = 0; i < nkb; ++i) {
-            const int s = i % STAGES, a = i % ASTAGES;
-            if (!mbar_wait(&full[s], (i / STAGES) & 1, s_abort)) break;
-            if (i >= ASTAGES && !mbar_wait(&aempty[a], ((i / ASTAGES) - 1) & 1, s_abort)) break;
+            const int c = i / SUB, sub = i - c * SUB, w = c % WS, a = i % AS;
+            const PreConst cur = nxt;
+            if (i + 1 < nkb) nxt = preload_const<KIND>(p, grow, kb0 + i + 1, row_ok);
+            if (sub == 0 && !mbar_wait(&fullW[w], (c / WS) & 1, s_abort)) break;
+            if (i >= AS && !mbar_wait(&aempty[a], ((i / AS) - 1) & 1, s_abort)) break;
             tc_fence_after();
-            uint32_t vals[32];
+            if (lane == 0) LBQ_TRACE_EVENT(2, i * 8 + (warp - 2));
+            uint32_t vals[16];
             if (row_ok) {
-                dequant_row_kblock<KIND>(sW + s * L::kWBytes + row * WB, row, kb0 + i, grow, p, s_cb, vals);
+                dequant_half_kblock<KIND>(sW + w * L::kWBytes + row * 128, row, sub * WB + half * (WB / 2), cur,
+                                          dq_offset, has_dq, s_cb, vals);
             } else {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) vals[j] = 0u;
+                for (int j = 0; j < 16; ++j) vals[j] = 0u;
             }
-            tmem_st_32x32b_x32(tmem + lane_base + kACol0 + a * kACols, vals);
+            tmem_st_32x32b_x16(tmem + lane_base + kACol0 + a * kACols + 16 * half, vals);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&afull[a]);
-                mbar_arrive(&empty[s]);
+                if (sub == SUB - 1 || i == nkb - 1) mbar_arrive(&emptyW[w]);
             }
+            if (lane == 0) LBQ_TRACE_EVENT(3, i * 8 + (warp - 2));
         }
+        (void)nch;
 
         // ------------------------------------------------------------ epilogue
         const int mt = min(NT, p.m - t0);  // tokens in this tile
         const bool lora = p.rank > 0;
-        // stage T[t0 : t0 + mt, :rank] (fp32) in smem for the adapter term
+        const int tid = threadIdx.x - 64;  // 0..255
         if (lora) {
-            const int tid = threadIdx.x - 64;
-            for (int e = tid; e < NT * p.rank_pad; e += 128) {
+            // stage T[t0 : t0 + mt, :rank] (fp32, zero-padded) for the adapter term
+            for (int e = tid; e < NT * p.rank_pad; e += 32 * kDqWarps) {
                 const int tt = e / p.rank_pad, u = e - tt * p.rank_pad;
                 sT[e] = (tt < mt && u < p.rank) ? p.T[static_cast<int64_t>(t0 + tt) * p.rank + u] : 0.0f;
             }
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("bar.sync 1, 256;" ::: "memory");
         const bool got = mbar_wait(dfull, 0, s_abort);
         tc_fence_after();
+        if (threadIdx.x == 64) LBQ_TRACE_EVENT(0, 1);
         const int out_col = row_ok ? (p.perm ? p.perm[grow] : static_cast<int>(grow)) : 0;
         const int rp = p.rank_pad;
         const bool splitk = p.nsplit > 1;
-        for (int jj = 0; jj < NT; jj += 16) {
+        constexpr int kHalfCols = NT >= 32 ? NT / 2 : 16;  // token columns per warp group
+        const int c_begin = half * kHalfCols;
+        const int c_end = min(NT, c_begin + kHalfCols);
+        for (int jj = c_begin; jj < c_end; jj += 16) {
             uint32_t raw[16];
             tmem_ld_32x32b_x16(tmem + lane_base + kDCol + jj, raw);
             tmem_ld_wait();
@@ -419,7 +531,7 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         if (splitk) {
             // the last CTA of this output tile sums the partials in split order
             __threadfence();
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            asm volatile("bar.sync 1, 256;" ::: "memory");
             if (threadIdx.x == 64) {
                 const uint32_t tile = blockIdx.y * gridDim.x + blockIdx.x;
                 const uint32_t prev = atomicAdd(p.counters + tile, 1u);
@@ -427,17 +539,20 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 if (last) p.counters[tile] = 0u;
                 *s_last = last;
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            asm volatile("bar.sync 1, 256;" ::: "memory");
             if (*s_last && row_ok && got) {
                 __threadfence();
-                for (int jj = 0; jj < mt; jj += 16) {
+                for (int jj = c_begin; jj < min(c_end, mt); jj += 16) {
                     float acc[16];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        acc[j] = 0.0f;
-                        if (jj + j < mt)
-                            for (int sp = 0; sp < p.nsplit; ++sp)
-                                acc[j] += __ldcg(p.partial + (static_cast<int64_t>(sp) * p.m + t0 + jj + j) * p.n + grow);
+                    for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
+                    for (int sp = 0; sp < p.nsplit; ++sp) {
+                        const float* src = p.partial + (static_cast<int64_t>(sp) * p.m + t0 + jj) * p.n + grow;
+                        float part[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) part[j] = (jj + j < mt) ? __ldcg(src + static_cast<int64_t>(j) * p.n) : 0.0f;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) acc[j] += part[j];
                     }
                     if (lora) lora_add16(acc, sT + jj * rp, rp, p.rank, p.B + static_cast<int64_t>(out_col) * p.rank, p.s);
 #pragma unroll
@@ -450,6 +565,7 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 
     tc_fence_before();
     __syncthreads();
+    if (threadIdx.x == 64) LBQ_TRACE_EVENT(0, 2);
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);

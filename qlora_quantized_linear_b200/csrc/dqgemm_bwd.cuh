@@ -35,6 +35,9 @@ struct BwdParams {
     uint32_t* counters;
 };
 
+// Two table buffers of 2048 bytes: G*32 PairConst + G*64 float2 each.
+constexpr int kBwdTabBytes = 4096;
+
 // Dequantization constants of one channel pair for one group (bf16x2 fast
 // path) and of single channels (fp32 exact path).
 struct PairConst {
@@ -48,15 +51,14 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
                   const BwdParams p) {
     constexpr int KTB = 128 * BITS / 8;       // packed bytes of one row across the 128-feature tile
     constexpr int G = (BITS == 4) ? 1 : 2;    // groups covered by the 128-feature tile
-    using L = GemmSmem<NT, STAGES, ASTAGES, 64 * KTB>;
+    using L = GemmSmem<NT, STAGES, ASTAGES, 64 * KTB, kBwdTabBytes>;
     constexpr uint32_t kTxBytes = L::kXBytes + 64 * KTB;
     constexpr int kACols = 32;
     constexpr int kDCol = 0;
     constexpr int kACol0 = (NT + 31) / 32 * 32;
     constexpr uint32_t kTmemCols = tmem_cols_for(kACol0 + kACols * ASTAGES);
     constexpr uint32_t kIdesc = idesc_bf16_f32(128, NT);
-    constexpr int kTabBuf = 2048;  // one table buffer: G*32 PairConst + G*64 float2
-    static_assert(2 * kTabBuf <= STAGES * L::kTabBytes, "table buffers do not fit");
+    constexpr int kTabBuf = kBwdTabBytes / 2;  // one table buffer: G*32 PairConst + G*64 float2
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));

@@ -1,0 +1,613 @@
+// dqgemv.cuh -- bandwidth-bound dequantize-GEMV for decode-sized batches
+// (M <= 16 tokens), stream-K over (row tile, k-block) work.
+//
+//   Y[t, c] = sum_k X[t, k] * W_hat[c, k]  (+ s * sum_u T[t, u] B[c, u])
+//
+// At decode sizes the packed weight is the whole cost (0.53 B/param for INT4
+// g128), so the kernel is built to stream it once at HBM speed:
+//
+//  * one producer lane streams the CTA's weight rows through a ring of
+//    128-row x 128-byte TMA boxes (128-byte swizzle); large boxes keep the TMA
+//    engine efficient and the ring keeps ~64 KB per CTA in flight without any
+//    load instruction in the compute warps;
+//  * eight compute warps own 16 rows each; a thread owns two rows (r, r+8)
+//    and, per 64-wide k-block, a quarter of each row's bytes.  Products run on
+//    register-resident tensor-core MMAs (mma.sync m16n8k16, bf16 in, fp32
+//    accumulate): rows are the M dimension, tokens (padded to 8 or 16) the N
+//    dimension;
+//  * codes become bf16 with one mask-and-or per two codes (the bf16 number
+//    128 + code), pairing codes that sit 2 bytes apart; the k order inside an
+//    MMA step is whatever pairing the codes have, and the activations staged in
+//    shared memory are permuted the same way, so each activation fragment is
+//    one 8-byte load;
+//  * dequantization is exact: A = bf16(code - zero) (exact for |zero| <= 128;
+//    otherwise bf16(code) with -zero * sum(x) added per group) and the
+//    per-group scale multiplies the fp32 group partial after the group's MMAs
+//    (GreenBit.AI article, 模型量化 (1): a scale and a zero per group).  The
+//    codebook format uses bf16(codebook[code]) times the fp32 per-64 absmax
+//    (QLoRA explainer, 关键技术细节 1).  Each (row, group) constant is
+//    converted once per CTA into a shared-memory table at the start, not by
+//    every lane that uses it;
+//  * stream-K: the grid is a whole number of waves and every CTA gets an equal
+//    contiguous share of the (row tile, k-block) work, spanning at most two
+//    row tiles.  A tile covered by several CTAs is finished by the last of them
+//    (per-tile counter), which sums the partials in CTA order, so the result
+//    does not depend on scheduling.
+#pragma once
+
+#include "dqgemm.cuh"
+
+namespace lbq {
+
+constexpr int kGemvComputeWarps = 8;                            // 16 rows each: 128 rows per tile
+constexpr int kGemvThreads = 32 * (kGemvComputeWarps + 1);      // + one producer warp
+constexpr int kGemvWStages = 4;                                 // 16 KB weight boxes in flight
+
+struct GemvParams {
+    int m, n, k;                      // tokens, stored rows, input features
+    int ngroups;                      // k / group (MinMax)
+    const uint16_t* scale;            // [n, ngroups] fp16 (MinMax)
+    const uint16_t* zero;             // [n, ngroups] fp16 (MinMax)
+    const float* absmax;              // codebook, no double quant
+    const int8_t* q8;                 // codebook, double quant
+    const float* s2;
+    const float* offset;
+    const float* codebook;
+    const uint16_t* X;                // [m, k] bf16
+    int rank;
+    float s;
+    const float* T;                   // [m, rank]
+    const uint16_t* B;                // [n_out, rank]
+    float* Y;
+    int64_t ldy;
+    const int32_t* perm;
+    int kbt;                          // k-blocks per row (k / 64)
+    int tiles;                        // row tiles of 128
+    int share;                        // k-blocks per CTA (<= kbt; a multiple of the scale group)
+    int64_t total;                    // tiles * kbt
+    float* partial;                   // [grid + tiles][m][128]
+    uint32_t* counters;               // [tiles], zero at launch
+};
+
+// D = A B + C (C = D on entry), one m16n8k16 bf16 MMA with fp32 accumulation.
+__device__ __forceinline__ void mma_m16n8k16_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                  uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D = A B (zero accumulator in).
+__device__ __forceinline__ void mma_m16n8k16_bf16_first(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                                        uint32_t a3, uint32_t b0, uint32_t b1) {
+    const float z = 0.0f;
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%10, %10, %10, %10};"
+        : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
+}
+
+template <int KIND>
+struct GemvTile {
+    static constexpr int kRowBytes = (KIND == kInt2) ? 16 : 32;        // per row per k-block
+    static constexpr int kThreadBytes = kRowBytes / 4;                 // a quarter row
+    static constexpr int kSub = 128 / kRowBytes;                       // k-blocks per weight box
+    static constexpr int kGroupBlocks = (KIND == kInt4) ? 2 : 1;       // k-blocks per scale group
+    // shared table of per-(group, row) constants: MinMax {subtrahend, scale},
+    // codebook the fp32 absmax of each (k-block, row)
+    static constexpr int kTabEntry = (KIND == kCode4) ? 4 : 8;
+};
+
+// Order of the 16 activations of a 16-wide k group as the MMA steps consume
+// them: step tau reads four consecutive entries (two code pairs).  4-bit
+// MinMax codes pair nibbles two bytes apart (k and k+4 in the group); 2-bit
+// codes pair crumbs two bytes apart (k and k+8); codebook codes pair the two
+// nibbles of one byte (k and k+1, the natural order).
+__device__ __forceinline__ int gemv_xperm(int kind, int p) {
+    constexpr int kPerm4[16] = {1, 5, 0, 4, 3, 7, 2, 6, 9, 13, 8, 12, 11, 15, 10, 14};
+    constexpr int kPerm2[16] = {0, 8, 1, 9, 2, 10, 3, 11, 4, 12, 5, 13, 6, 14, 7, 15};
+    return kind == kInt2 ? kPerm2[p] : kind == kInt4 ? kPerm4[p] : p;
+}
+
+// (a & MASK) | c in one logic op.
+template <uint32_t MASK>
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "n"(MASK), "r"(c));
+    return d;
+}
+
+// Code pairs of one 32-bit word of 4-bit codes (bytes b0..b3 = codes 0..7):
+// P0 = (1, 5), P1 = (0, 4), P2 = (3, 7), P3 = (2, 6), each half the bf16
+// number 128 + code (mg = 0x43004300 is passed in a register).
+__device__ __forceinline__ void int4_pairs(uint32_t w, uint32_t mg, uint32_t* o) {
+    o[0] = and_or<0x000F000Fu>(w, mg);
+    o[1] = and_or<0x000F000Fu>(w >> 4, mg);
+    o[2] = and_or<0x000F000Fu>(w >> 8, mg);
+    o[3] = and_or<0x000F000Fu>(w >> 12, mg);
+}
+
+// Code pairs of one 32-bit word of 2-bit codes (bytes b0..b3 = codes 0..15,
+// first code in the top bits): pair t = (t, t + 8), t = 0..7.
+__device__ __forceinline__ void int2_pairs(uint32_t w, uint32_t mg, uint32_t* o) {
+    o[0] = and_or<0x00030003u>(w >> 6, mg);
+    o[1] = and_or<0x00030003u>(w >> 4, mg);
+    o[2] = and_or<0x00030003u>(w >> 2, mg);
+    o[3] = and_or<0x00030003u>(w, mg);
+    o[4] = and_or<0x00030003u>(w >> 14, mg);
+    o[5] = and_or<0x00030003u>(w >> 12, mg);
+    o[6] = and_or<0x00030003u>(w >> 10, mg);
+    o[7] = and_or<0x00030003u>(w >> 8, mg);
+}
+
+// a - b on both bf16 halves (exact here: integers of at most 9 bits).
+__device__ __forceinline__ uint32_t sub_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint2 gemv_lds64(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t gemv_lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+template <int KIND, int NTOK>
+__global__ void __launch_bounds__(kGemvThreads, 2)
+dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
+    constexpr int NT8 = NTOK / 8;
+    constexpr int GB = GemvTile<KIND>::kGroupBlocks;
+    constexpr int SUB = GemvTile<KIND>::kSub;
+    constexpr int RB = GemvTile<KIND>::kRowBytes;
+    constexpr int TB = GemvTile<KIND>::kThreadBytes;
+    constexpr int TE = GemvTile<KIND>::kTabEntry;
+    constexpr int TW = TB / 4;                                    // code words per row, k-block and thread
+    constexpr int WS = kGemvWStages;
+    constexpr int kWBox = 128 * 128;
+    constexpr int kCompute = 32 * kGemvComputeWarps;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == kCompute) tma_prefetch_desc(&tmW);
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte alignment for the swizzled boxes, by pointer arithmetic on the
+    // shared array so that every access below stays a shared-memory access
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t* sW = smem;                                           // WS x 16 KB
+    const int xstride = p.share * 64 + 4;                         // bf16 per token row (+8 bytes)
+    uint16_t* sX = reinterpret_cast<uint16_t*>(smem + WS * kWBox);          // [m][xstride]
+    uint8_t* sTab = reinterpret_cast<uint8_t*>(sX + p.m * xstride);        // [groups][128] entries
+    const int tab_groups = p.share / GB;
+    uint32_t* s_lut = reinterpret_cast<uint32_t*>(sTab + tab_groups * 128 * TE);   // codebook pairs [256]
+    uint64_t* full = reinterpret_cast<uint64_t*>(s_lut + (KIND == kCode4 ? 256 : 0));
+    uint64_t* empty = full + WS;
+    int* s_last = reinterpret_cast<int*>(empty + WS);
+    volatile int* s_abort = s_last + 1;
+    int* s_far = s_last + 2;
+
+    // this CTA's work: up to two (tile, first k-block, k-blocks) segments
+    // (tiles * kbt < 2^31, checked by the host)
+    int t0 = 0, a0 = 0, n0 = 0, n1 = 0;
+    {
+        const uint32_t u0 = blockIdx.x * static_cast<uint32_t>(p.share);
+        const uint32_t tot = static_cast<uint32_t>(p.total);
+        const uint32_t u1 = u0 + p.share < tot ? u0 + p.share : tot;
+        if (u0 < u1) {
+            t0 = static_cast<int>(u0 / static_cast<uint32_t>(p.kbt));
+            a0 = static_cast<int>(u0 - static_cast<uint32_t>(t0) * p.kbt);
+            n0 = min(static_cast<int>(u1 - u0), p.kbt - a0);
+            n1 = static_cast<int>(u1 - u0) - n0;
+        }
+    }
+    const int nseg = n0 == 0 ? 0 : (n1 == 0 ? 1 : 2);
+    const int nk = n0 + n1;
+    const int nbox0 = (n0 + SUB - 1) / SUB;
+    const int nbox = nbox0 + (n1 + SUB - 1) / SUB;
+
+    if (tid == 0) {
+        for (int i = 0; i < WS; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kGemvComputeWarps);
+        }
+        *s_abort = 0;
+        *s_far = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == kGemvComputeWarps) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0 && nbox > 0) {
+            int issued = 0;
+            for (int c = 0; c < nbox; ++c) {
+                const int w = c % WS;
+                if (c >= WS && !mbar_wait(&empty[w], ((c / WS) - 1) & 1, s_abort)) break;
+                mbar_arrive_expect_tx(&full[w], kWBox);
+                const int x = c < nbox0 ? (a0 + c * SUB) * RB : (c - nbox0) * SUB * RB;
+                const int y = (c < nbox0 ? t0 : t0 + 1) * 128;
+                tma_load_2d(sW + w * kWBox, &tmW, &full[w], x, y);
+                issued = c + 1;
+            }
+            for (int c = max(0, issued - WS); c < issued; ++c) mbar_wait_drain(&full[c % WS], (c / WS) & 1);
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------- compute warps
+    // prologue: the table of this CTA's constants, then its activation slices
+    {
+        // table entry (local group lg, row rl); groups of segment 1 follow those of segment 0
+        const int G = nk / GB, G0 = n0 / GB;
+        const int total = G * 128;
+        for (int e0 = tid; e0 < total; e0 += 8 * kCompute) {
+            uint32_t raw[8][2];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int e = e0 + u * kCompute;
+                raw[u][0] = 0u;
+                raw[u][1] = 0u;
+                if (e < total) {
+                    const int rl = e / G, lg = e - rl * G;
+                    const int tile = lg < G0 ? t0 : t0 + 1;
+                    const int gl = lg < G0 ? a0 / GB + lg : lg - G0;      // group (codebook: k-block) in the row
+                    const int64_t r = static_cast<int64_t>(tile) * 128 + rl;
+                    if (r < p.n) {
+                        if (KIND != kCode4) {
+                            raw[u][0] = __ldg(p.scale + r * p.ngroups + gl);
+                            raw[u][1] = __ldg(p.zero + r * p.ngroups + gl);
+                        } else if (p.q8 != nullptr) {
+                            const int64_t b = r * p.kbt + gl;
+                            raw[u][0] = static_cast<uint32_t>(static_cast<int32_t>(__ldg(p.q8 + b)));
+                            raw[u][1] = __float_as_uint(__ldg(p.s2 + (b >> 8)));
+                        } else {
+                            raw[u][0] = __float_as_uint(__ldg(p.absmax + r * p.kbt + gl));
+                        }
+                    }
+                }
+            }
+            const float dq_off = (KIND == kCode4 && p.q8 != nullptr) ? __ldg(p.offset) : 0.0f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int e = e0 + u * kCompute;
+                if (e < total) {
+                    const int rl = e / G, lg = e - rl * G;
+                    if (KIND != kCode4) {
+                        const uint16_t s16 = static_cast<uint16_t>(raw[u][0]), z16 = static_cast<uint16_t>(raw[u][1]);
+                        const float zf = f16_bits_to_f32(z16);
+                        uint32_t word;
+                        if (fabsf(zf) <= 128.0f) {
+                            // (128 + q) - (128 + z) = q - z exactly
+                            word = pack_bf16x2_rn(128.0f + zf, 0.0f) & 0xFFFFu;
+                        } else {
+                            // (128 + q) - 128 = q, and -z (fp16 bits) in the high half
+                            word = 0x4300u | (static_cast<uint32_t>(z16 ^ 0x8000u) << 16);
+                            *s_far = 1;
+                        }
+                        const float sf = f16_bits_to_f32(s16);
+                        *reinterpret_cast<uint2*>(sTab + (lg * 128 + rl) * 8) = make_uint2(word, __float_as_uint(sf));
+                    } else {
+                        float am = __uint_as_float(raw[u][0]);
+                        if (p.q8 != nullptr)
+                            am = __fadd_rn(__fmul_rn(__fdiv_rn(static_cast<float>(static_cast<int32_t>(raw[u][0])), 127.0f),
+                                                     __uint_as_float(raw[u][1])),
+                                           dq_off);
+                        *reinterpret_cast<float*>(sTab + (lg * 128 + rl) * 4) = am;
+                    }
+                }
+            }
+        }
+        // activations of the m real tokens, permuted to the MMA step order
+        const int ngr16 = nk * 4;                                  // 16-wide k groups
+        const int xtotal = p.m * ngr16;
+        for (int e0 = tid; e0 < xtotal; e0 += 4 * kCompute) {
+            uint4 v[4][2];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + u * kCompute;
+                if (e < xtotal) {
+                    const int t = e / ngr16, g16 = e - t * ngr16;
+                    const int lk = g16 >> 2;
+                    const int kb = lk < n0 ? a0 + lk : lk - n0;
+                    const uint4* src = reinterpret_cast<const uint4*>(p.X + static_cast<int64_t>(t) * p.k + kb * 64 +
+                                                                      (g16 & 3) * 16);
+                    v[u][0] = __ldg(src);
+                    v[u][1] = __ldg(src + 1);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + u * kCompute;
+                if (e < xtotal) {
+                    const int t = e / ngr16, g16 = e - t * ngr16;
+                    const uint32_t w8[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
+                                            v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+                    uint16_t in[16];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        in[2 * q] = static_cast<uint16_t>(w8[q] & 0xFFFFu);
+                        in[2 * q + 1] = static_cast<uint16_t>(w8[q] >> 16);
+                    }
+                    // rows are 8-byte aligned (stride 128 * share + 8 bytes)
+                    uint2* d2 = reinterpret_cast<uint2*>(sX + t * xstride + g16 * 16);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        d2[q] = make_uint2(static_cast<uint32_t>(in[gemv_xperm(KIND, 4 * q)]) |
+                                               (static_cast<uint32_t>(in[gemv_xperm(KIND, 4 * q + 1)]) << 16),
+                                           static_cast<uint32_t>(in[gemv_xperm(KIND, 4 * q + 2)]) |
+                                               (static_cast<uint32_t>(in[gemv_xperm(KIND, 4 * q + 3)]) << 16));
+                }
+            }
+        }
+        if (KIND == kCode4) {
+            for (int e = tid; e < 256; e += kCompute) {
+                // byte e = (first code << 4) | second code -> (codebook[first], codebook[second])
+                s_lut[e] = pack_bf16x2_rn(p.codebook[e >> 4], p.codebook[e & 15]);
+            }
+        }
+    }
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+
+    const int j = lane & 3;                            // quarter of the row's bytes
+    const int g = lane >> 2;                           // MMA row in the 8-row half, token in the n8 tile
+    // MMA row g is weight row pi(g) of the warp's first 8 (pi interleaves even
+    // rows into lanes 0-15 and odd rows into lanes 16-31, so that each half
+    // warp's 8-byte reads of the 128-byte-swizzled lines hit 32 distinct banks)
+    const int rl0 = warp * 16 + (g & 3) * 2 + (g >> 2); // local rows rl0, rl0 + 8
+    const int sw = rl0 & 7;                            // swizzle of both rows' lines
+    uint32_t offs[SUB];                                // this thread's bytes of sub-block s in the line
+#pragma unroll
+    for (int s = 0; s < SUB; ++s) {
+        const int off = s * RB + TB * j;
+        offs[s] = static_cast<uint32_t>((((off >> 4) ^ sw) << 4) | (off & 15));
+    }
+    const uint32_t wrow = smem_u32(sW) + rl0 * 128;
+    const uint32_t trow = smem_u32(sTab) + rl0 * TE;   // table entries of row rl0 (row rl0 + 8: + 8 TE)
+    // B fragments: token nt * 8 + g (lanes of tokens >= m read nothing and use 0)
+    bool tok_ok[NT8];
+    uint32_t xthr[NT8];
+#pragma unroll
+    for (int nt = 0; nt < NT8; ++nt) {
+        tok_ok[nt] = nt * 8 + g < p.m;
+        xthr[nt] = smem_u32(sX) + static_cast<uint32_t>((tok_ok[nt] ? nt * 8 + g : 0) * xstride + 16 * j) * 2;
+    }
+    const bool far = *s_far != 0;                      // some group of this CTA has |zero| > 128
+    uint32_t mg = 0x43004300u;
+    asm volatile("" : "+r"(mg));                       // keep the magic in a register
+
+    uint32_t c = 0;                                    // weight boxes consumed (matches the producer)
+    int lk0 = 0;                                       // first local k-block of the segment
+    // (after a timed-out wait every warp still runs both segments' barriers)
+    for (int sgi = 0; sgi < nseg; ++sgi) {
+        const int tile = sgi == 0 ? t0 : t0 + 1;
+        const int kb0 = sgi == 0 ? a0 : 0;
+        const int nkb = sgi == 0 ? n0 : n1;
+        const int64_t gr0 = static_cast<int64_t>(tile) * 128 + rl0, gr1 = gr0 + 8;
+        const bool ok0 = gr0 < p.n, ok1 = gr1 < p.n;
+        // group partials in two chains (even and odd MMA steps), folded per group
+        float acc[NT8][4], cg[2][NT8][4];
+#pragma unroll
+        for (int nt = 0; nt < NT8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[nt][e] = cg[0][nt][e] = cg[1][nt][e] = 0.0f;
+        uint32_t sub0 = 0x43004300u, sub1 = 0x43004300u;
+        float sf0 = 1.0f, sf1 = 1.0f, corr0 = 0.0f, corr1 = 0.0f;
+
+        const int nbx = (nkb + SUB - 1) / SUB;
+        for (int bx = 0; bx < nbx; ++bx, ++c) {
+            const uint32_t w = c % WS;
+            if (!mbar_wait(&full[w], (c / WS) & 1u, s_abort)) break;
+            // the whole box's codes of this thread's two rows
+            const uint32_t base = wrow + w * kWBox;
+            uint32_t r0[SUB * TW], r1[SUB * TW];
+#pragma unroll
+            for (int s = 0; s < SUB; ++s) {
+                if (TW == 2) {
+                    const uint2 v0 = gemv_lds64(base + offs[s]);
+                    const uint2 v1 = gemv_lds64(base + 1024 + offs[s]);
+                    r0[2 * s] = v0.x;
+                    r0[2 * s + 1] = v0.y;
+                    r1[2 * s] = v1.x;
+                    r1[2 * s + 1] = v1.y;
+                } else {
+                    r0[s] = gemv_lds32(base + offs[s]);
+                    r1[s] = gemv_lds32(base + 1024 + offs[s]);
+                }
+            }
+
+#pragma unroll
+            for (int s = 0; s < SUB; ++s) {
+                const int i = bx * SUB + s;                 // k-block within the segment
+                if (i < nkb) {
+                    const int lk = lk0 + i;                 // k-block within the CTA's slice
+                    if (s % GB == 0) {
+                        // this group's constants from the table
+                        const uint32_t ta = trow + static_cast<uint32_t>(lk / GB) * (128 * TE);
+                        if (KIND != kCode4) {
+                            const uint2 e0 = gemv_lds64(ta), e1 = gemv_lds64(ta + 8 * TE);
+                            sub0 = __byte_perm(e0.x, 0u, 0x1010);
+                            sub1 = __byte_perm(e1.x, 0u, 0x1010);
+                            sf0 = __uint_as_float(e0.y);
+                            sf1 = __uint_as_float(e1.y);
+                            if (far) {
+                                corr0 = f16_bits_to_f32(static_cast<uint16_t>(e0.x >> 16));
+                                corr1 = f16_bits_to_f32(static_cast<uint16_t>(e1.x >> 16));
+                            }
+                        } else {
+                            sf0 = __uint_as_float(gemv_lds32(ta));
+                            sf1 = __uint_as_float(gemv_lds32(ta + 8 * TE));
+                        }
+                    }
+                    // A fragments: 8 code pairs of each row as bf16x2
+                    uint32_t f0[8], f1[8];
+                    if (KIND == kInt4) {
+                        int4_pairs(r0[2 * s], mg, f0);
+                        int4_pairs(r0[2 * s + 1], mg, f0 + 4);
+                        int4_pairs(r1[2 * s], mg, f1);
+                        int4_pairs(r1[2 * s + 1], mg, f1 + 4);
+                    } else if (KIND == kInt2) {
+                        int2_pairs(r0[s], mg, f0);
+                        int2_pairs(r1[s], mg, f1);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            f0[q] = s_lut[__byte_perm(r0[2 * s], 0u, 0x4440 + q)];
+                            f0[4 + q] = s_lut[__byte_perm(r0[2 * s + 1], 0u, 0x4440 + q)];
+                            f1[q] = s_lut[__byte_perm(r1[2 * s], 0u, 0x4440 + q)];
+                            f1[4 + q] = s_lut[__byte_perm(r1[2 * s + 1], 0u, 0x4440 + q)];
+                        }
+                    }
+                    if (KIND != kCode4) {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            f0[q] = sub_bf16x2(f0[q], sub0);
+                            f1[q] = sub_bf16x2(f1[q], sub1);
+                        }
+                    }
+                    // B fragments (permuted activations) and four MMA steps
+                    const uint32_t xoff = static_cast<uint32_t>(lk) * 128;
+                    uint2 bxf[4][NT8];
+#pragma unroll
+                    for (int tau = 0; tau < 4; ++tau)
+#pragma unroll
+                        for (int nt = 0; nt < NT8; ++nt)
+                            bxf[tau][nt] = tok_ok[nt] ? gemv_lds64(xthr[nt] + xoff + 8 * tau) : make_uint2(0u, 0u);
+#pragma unroll
+                    for (int tau = 0; tau < 4; ++tau)
+#pragma unroll
+                        for (int nt = 0; nt < NT8; ++nt) {
+                            if (s % GB == 0 && tau < 2)
+                                mma_m16n8k16_bf16_first(cg[tau & 1][nt], f0[2 * tau], f1[2 * tau], f0[2 * tau + 1],
+                                                        f1[2 * tau + 1], bxf[tau][nt].x, bxf[tau][nt].y);
+                            else
+                                mma_m16n8k16_bf16(cg[tau & 1][nt], f0[2 * tau], f1[2 * tau], f0[2 * tau + 1],
+                                                  f1[2 * tau + 1], bxf[tau][nt].x, bxf[tau][nt].y);
+                        }
+                    // end of a scale group: fold the group partial
+                    if (s % GB == GB - 1) {
+#pragma unroll
+                        for (int nt = 0; nt < NT8; ++nt) {
+                            float gs[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) gs[e] = cg[0][nt][e] + cg[1][nt][e];
+                            if (KIND != kCode4 && far) {
+                                // -zero * (sum of x over the group) for groups with |zero| > 128
+                                const int tA = nt * 8 + 2 * j;
+                                float sx0 = 0.0f, sx1 = 0.0f;
+                                for (int kk = (lk + 1 - GB) * 64; kk < (lk + 1) * 64; ++kk) {
+                                    if (tA < p.m) sx0 += bf16_bits_to_f32(sX[tA * xstride + kk]);
+                                    if (tA + 1 < p.m) sx1 += bf16_bits_to_f32(sX[(tA + 1) * xstride + kk]);
+                                }
+                                gs[0] = fmaf(corr0, sx0, gs[0]);
+                                gs[1] = fmaf(corr0, sx1, gs[1]);
+                                gs[2] = fmaf(corr1, sx0, gs[2]);
+                                gs[3] = fmaf(corr1, sx1, gs[3]);
+                            }
+                            acc[nt][0] = fmaf(sf0, gs[0], acc[nt][0]);
+                            acc[nt][1] = fmaf(sf0, gs[1], acc[nt][1]);
+                            acc[nt][2] = fmaf(sf1, gs[2], acc[nt][2]);
+                            acc[nt][3] = fmaf(sf1, gs[3], acc[nt][3]);
+                        }
+                    }
+                }
+            }
+            // release the slot only after every loaded word has been used: an
+            // arrive issued right behind the shared loads let the next TMA
+            // write land before some of those loads had read the slot
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[w]);
+        }
+        lk0 += nkb;
+        // -------------------------------------------------------------- segment epilogue
+        auto lora = [&](int t, int oc) -> float {
+            if (p.rank == 0) return 0.0f;
+            float d = 0.0f;
+            for (int u = 0; u < p.rank; ++u)
+                d = fmaf(p.T[static_cast<int64_t>(t) * p.rank + u],
+                         bf16_bits_to_f32(__ldg(p.B + static_cast<int64_t>(oc) * p.rank + u)), d);
+            return p.s * d;
+        };
+        if (kb0 == 0 && nkb == p.kbt) {
+            // this CTA covered the whole tile
+#pragma unroll
+            for (int nt = 0; nt < NT8; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int t = nt * 8 + 2 * j + (e & 1);
+                    const bool ok = (e < 2) ? ok0 : ok1;
+                    const int64_t r = (e < 2) ? gr0 : gr1;
+                    if (ok && t < p.m) {
+                        const int oc = p.perm ? p.perm[r] : static_cast<int>(r);
+                        p.Y[static_cast<int64_t>(t) * p.ldy + oc] = acc[nt][e] + lora(t, oc);
+                    }
+                }
+            continue;
+        }
+        // partial slot of (CTA b, tile t) is b + t: CTAs cover the work in
+        // order, so no two (CTA, tile) pairs share a slot
+        float* slot = p.partial + (static_cast<int64_t>(blockIdx.x) + tile) * p.m * 128;
+#pragma unroll
+        for (int nt = 0; nt < NT8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int t = nt * 8 + 2 * j + (e & 1);
+                if (t < p.m) slot[t * 128 + rl0 + ((e < 2) ? 0 : 8)] = acc[nt][e];
+            }
+        __threadfence();
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        const int cta_lo = static_cast<int>((static_cast<int64_t>(tile) * p.kbt) / p.share);
+        const int cta_hi = static_cast<int>((static_cast<int64_t>(tile + 1) * p.kbt - 1) / p.share);
+        if (tid == 0) {
+            const uint32_t prev = atomicAdd(p.counters + tile, 1u);
+            const int last = (prev == static_cast<uint32_t>(cta_hi - cta_lo)) ? 1 : 0;
+            // the last contributor leaves the counter at zero for the next call
+            if (last) p.counters[tile] = 0u;
+            *s_last = last;
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (*s_last) {
+            __threadfence();
+            // sum the partials of every CTA that touched this tile, in CTA order,
+            // four rows per thread, all partials' loads in flight together
+            const float4* part4 = reinterpret_cast<const float4*>(p.partial);
+            for (int e = tid; e < 32 * p.m; e += kCompute) {
+                const int t = e >> 5, rq = (e & 31) * 4;
+                float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                for (int b0 = cta_lo; b0 <= cta_hi; b0 += 8) {
+                    float4 part[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        part[q] = (b0 + q <= cta_hi)
+                                      ? __ldcg(part4 + ((static_cast<int64_t>(b0 + q) + tile) * p.m + t) * 32 + (e & 31))
+                                      : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        v.x += part[q].x;
+                        v.y += part[q].y;
+                        v.z += part[q].z;
+                        v.w += part[q].w;
+                    }
+                }
+                const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int64_t r = static_cast<int64_t>(tile) * 128 + rq + q;
+                    if (r < p.n) {
+                        const int oc = p.perm ? p.perm[r] : static_cast<int>(r);
+                        p.Y[static_cast<int64_t>(t) * p.ldy + oc] = vv[q] + lora(t, oc);
+                    }
+                }
+            }
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+    }
+}
+
+}  // namespace lbq

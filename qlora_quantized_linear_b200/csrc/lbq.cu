@@ -5,6 +5,7 @@
 
 #include "dqgemm.cuh"
 #include "dqgemm_bwd.cuh"
+#include "dqgemv.cuh"
 #include "lora.cuh"
 #include "quantize.cuh"
 
@@ -63,6 +64,23 @@ bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Activation view for the forward kernel: bf16 [rows, cols] seen as 3-D
+// (64 elements, rows, cols / 64 blocks), box (64, brows, bblocks): one box
+// brings `bblocks` consecutive k-blocks of `brows` rows, each k-block landing
+// as its own [brows x 128 B] tile (128-byte swizzle).
+bool make_map_x3d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t brows,
+                  uint32_t bblocks) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {64, rows, cols / 64};
+    cuuint64_t strides[2] = {cols * 2, 128};
+    cuuint32_t box[3] = {64, brows, bblocks};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------------------
 // weight descriptor checks
 // ---------------------------------------------------------------------------
@@ -100,33 +118,104 @@ int kind_of(const lbq_qweight* q) {
 // ---------------------------------------------------------------------------
 constexpr int kCodebookQuantizeMaxCtas = 4096;
 
-int token_tile(int m) { return m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : 128; }
+int token_tile(int m) { return m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256; }
+
+// Split-K workspace layout, the same for every plan: a fixed header of
+// per-tile arrival counters at offset 0, then the fp32 partial sums.  The
+// last CTA of a tile sets its counter back to zero, so the header stays zero
+// between calls whatever shapes share the workspace (partials never land on
+// it).
+constexpr size_t kCounterHeader = 64 * 1024;
+constexpr int kMaxSplitTiles = static_cast<int>(kCounterHeader / sizeof(uint32_t));
+
+inline uint32_t* ws_counters(void* ws) { return static_cast<uint32_t*>(ws); }
+inline float* ws_partials(void* ws) { return reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kCounterHeader); }
 
 struct Plan {
     int nt;          // token tile
     int tiles;       // output tiles (rows x token tiles)
     int nsplit;      // K splits
     int per_split;   // reduction blocks per split
-    size_t partial_bytes, counter_bytes;
-    size_t workspace() const { return nsplit > 1 ? partial_bytes + counter_bytes : 0; }
+    size_t partial_bytes;
+    size_t workspace() const { return nsplit > 1 ? kCounterHeader + partial_bytes : 0; }
 };
 
-Plan plan_gemm(int m, int64_t out_rows, int64_t red_blocks, int sms) {
+// Token tile, output tiles and K splits of one GEMM.  When the output tiles
+// alone cannot fill the CTA slots of the machine (decode sizes), the
+// reduction is split so that all CTAs fit in one wave.
+Plan plan_gemm(int m, int64_t out_rows, int64_t red_blocks, int sms, int max_nt = 256, int align = 1) {
     Plan pl;
-    pl.nt = token_tile(m);
+    pl.nt = std::min(token_tile(m), max_nt);
     pl.tiles = static_cast<int>(cdiv(out_rows, 128) * cdiv(m, pl.nt));
-    const int target = 2 * sms;
+    const int slots = (pl.nt >= 256 ? 1 : 2) * sms;
     pl.nsplit = 1;
-    if (pl.tiles < target) pl.nsplit = static_cast<int>(std::min<int64_t>(red_blocks, cdiv(target, pl.tiles)));
-    pl.per_split = static_cast<int>(cdiv(red_blocks, pl.nsplit));
+    if (pl.tiles < slots) pl.nsplit = static_cast<int>(std::min<int64_t>(red_blocks, std::max(1, slots / pl.tiles)));
+    pl.per_split = static_cast<int>(cdiv(cdiv(red_blocks, pl.nsplit), align) * align);
     pl.nsplit = static_cast<int>(cdiv(red_blocks, pl.per_split));
     pl.partial_bytes = round_up(static_cast<size_t>(pl.nsplit) * m * out_rows * sizeof(float), 256);
-    pl.counter_bytes = round_up(static_cast<size_t>(pl.tiles) * sizeof(uint32_t), 256);
     return pl;
 }
 
+// Decode-sized batches (m <= 16) run the stream-K GEMV: every CTA gets an
+// equal share of the (row tile, k-block) work, a whole number of scale
+// groups and as many k-blocks as its shared memory holds (weight ring,
+// activation slice, constant table) with two CTAs per SM, and the grid fills
+// whole waves of two CTAs per SM.
+constexpr int kGemvMaxM = 16;
+constexpr size_t kGemvSmemBudget = 113 * 1024;     // two CTAs per SM
+
+size_t gemv_smem_bytes(int m, int share, int kind) {
+    const int gb = kind == kInt4 ? 2 : 1;
+    const size_t entry = kind == kCode4 ? 4 : 8;
+    return 1024 + static_cast<size_t>(kGemvWStages) * 128 * 128 + static_cast<size_t>(m) * (share * 64 + 4) * 2 +
+           static_cast<size_t>(share / gb) * 128 * entry + (kind == kCode4 ? 1024 : 0) + 2 * kGemvWStages * 8 + 16;
+}
+
+Plan plan_gemv(int m, const lbq_qweight* q, int sms) {
+    Plan pl;
+    pl.nt = m <= 8 ? 8 : 16;
+    const int kind = kind_of(q);
+    const int64_t kbt = q->k / 64;
+    const int gb = kind == kInt4 ? 2 : 1;
+    pl.tiles = static_cast<int>(cdiv(q->n, 128));
+    const int64_t total = static_cast<int64_t>(pl.tiles) * kbt;
+    const int64_t slots = 2LL * sms;
+    int64_t smax = gb;
+    while (smax + gb <= kbt && gemv_smem_bytes(m, static_cast<int>(smax + gb), kind) <= kGemvSmemBudget) smax += gb;
+    const int64_t waves = cdiv(total, slots * smax);
+    int64_t share = cdiv(cdiv(total, waves * slots), gb) * gb;
+    // at least an eighth of a row per CTA, so that the CTA finishing a tile
+    // sums a handful of partials (small layers then use fewer CTAs)
+    share = std::max(share, std::min(cdiv(cdiv(kbt, 8), gb) * gb, smax));
+    share = std::max<int64_t>(gb, std::min(share, smax));
+    pl.per_split = static_cast<int>(share);                      // k-blocks per CTA
+    pl.nsplit = static_cast<int>(cdiv(total, share));            // CTAs
+    pl.partial_bytes = round_up(static_cast<size_t>(pl.nsplit + pl.tiles) * m * 128 * sizeof(float), 256);
+    return pl;
+}
+
+template <int KIND, int NTOK>
+lbq_status launch_gemv_kind(const GemvParams& p, const uint8_t* packed, int grid, cudaStream_t st) {
+    auto kern = dqgemv_kernel<KIND, NTOK>;
+    const size_t smem = gemv_smem_bytes(p.m, p.share, KIND);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+        return LBQ_ECUDA;
+    CUtensorMap tmW;
+    if (!make_map_2d(&tmW, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.n, static_cast<int64_t>(p.k) * (KIND == kInt2 ? 2 : 4) / 8,
+                     128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+        return LBQ_ECUDA;
+    kern<<<grid, kGemvThreads, smem, st>>>(tmW, p);
+    return last_launch();
+}
+
+// Forward plan: splits start on a whole weight chunk (128 bytes of a row).
+Plan plan_fwd(int m, const lbq_qweight* q, int sms) {
+    if (m <= kGemvMaxM) return plan_gemv(m, q, sms);
+    return plan_gemm(m, q->n, q->k / 64, sms, 256, q->bits == 2 ? 8 : 4);
+}
+
 template <int NT>
-struct FwdCfg {
+struct BwdCfg {
     static constexpr int kStages = NT <= 32 ? 8 : NT <= 64 ? 6 : 4;
     static constexpr int kAStages = 2;
 };
@@ -134,21 +223,19 @@ struct FwdCfg {
 template <int NT, int KIND>
 lbq_status launch_fwd_nt(const FwdParams& p, const void* X, int m, int64_t k, const uint8_t* packed, int nrows,
                          int nsplit, cudaStream_t st) {
-    constexpr int S = FwdCfg<NT>::kStages, AS = FwdCfg<NT>::kAStages;
-    constexpr int WB = WeightTile<KIND>::kRowBytes;
-    using L = GemmSmem<NT, S, AS, 128 * WB>;
-    auto kern = dqgemm_fwd_kernel<NT, KIND, S, AS>;
+    using C = FwdCfg<NT>;
+    using L = FwdSmem<NT, C::kXStages, C::kXBlocks, C::kWStages, C::kAStages>;
+    auto kern = dqgemm_fwd_kernel<NT, KIND, C::kXStages, C::kXBlocks, C::kWStages, C::kAStages, C::kMinBlocks>;
     const size_t smem = L::total(p.rank_pad);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
         return LBQ_ECUDA;
     CUtensorMap tmX, tmW;
-    if (!make_map_2d(&tmX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, m, k, NT, 64, CU_TENSOR_MAP_SWIZZLE_128B))
-        return LBQ_ECUDA;
-    if (!make_map_2d(&tmW, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, nrows, k * (KIND == kInt2 ? 2 : 4) / 8, 128, WB,
-                     WB == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!make_map_x3d(&tmX, X, m, k, NT, C::kXBlocks)) return LBQ_ECUDA;
+    if (!make_map_2d(&tmW, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, nrows, k * (KIND == kInt2 ? 2 : 4) / 8, 128, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
         return LBQ_ECUDA;
     dim3 grid(static_cast<unsigned>(cdiv(nrows, 128)), static_cast<unsigned>(cdiv(m, NT)), static_cast<unsigned>(nsplit));
-    kern<<<grid, 192, smem, st>>>(tmX, tmW, p);
+    kern<<<grid, kFwdThreads, smem, st>>>(tmX, tmW, p);
     return last_launch();
 }
 
@@ -159,16 +246,63 @@ lbq_status launch_fwd_kind(int nt, const FwdParams& p, const void* X, int m, int
         case 16: return launch_fwd_nt<16, KIND>(p, X, m, k, packed, nrows, nsplit, st);
         case 32: return launch_fwd_nt<32, KIND>(p, X, m, k, packed, nrows, nsplit, st);
         case 64: return launch_fwd_nt<64, KIND>(p, X, m, k, packed, nrows, nsplit, st);
-        default: return launch_fwd_nt<128, KIND>(p, X, m, k, packed, nrows, nsplit, st);
+        case 128: return launch_fwd_nt<128, KIND>(p, X, m, k, packed, nrows, nsplit, st);
+        default: return launch_fwd_nt<256, KIND>(p, X, m, k, packed, nrows, nsplit, st);
     }
 }
 
 // One fused dequantize-GEMM over one stored weight (or one half of a
 // channel-mix weight).  `perm` maps its stored rows to output columns.
+lbq_status run_gemv(const void* X, int m, const lbq_qweight* q, const void* B, int rank, float s, const float* T,
+                    float* Y, int64_t ldy, const int32_t* perm, void* ws, int sms, cudaStream_t st) {
+    const Plan pl = plan_gemv(m, q, sms);
+    GemvParams p{};
+    p.m = m;
+    p.n = q->n;
+    p.k = q->k;
+    p.ngroups = q->scheme == LBQ_MINMAX_ASYM ? q->k / q->group : 0;
+    p.scale = q->scale;
+    p.zero = q->zero;
+    p.absmax = q->absmax;
+    p.q8 = (q->scheme == LBQ_CODEBOOK4 && q->double_quant) ? q->absmax_q8 : nullptr;
+    p.s2 = q->absmax_s2;
+    p.offset = q->absmax_offset;
+    p.codebook = q->codebook;
+    p.X = static_cast<const uint16_t*>(X);
+    p.rank = rank;
+    p.s = s;
+    p.T = T;
+    p.B = static_cast<const uint16_t*>(B);
+    p.Y = Y;
+    p.ldy = ldy;
+    p.perm = perm;
+    p.kbt = q->k / 64;
+    p.tiles = pl.tiles;
+    p.share = pl.per_split;
+    p.total = static_cast<int64_t>(pl.tiles) * p.kbt;
+    if (p.total >= (int64_t(1) << 31)) return LBQ_EUNSUPPORTED;
+    if (pl.workspace() > 0) {
+        if (!ws) return LBQ_EWORKSPACE;
+        if (pl.tiles > kMaxSplitTiles) return LBQ_EUNSUPPORTED;
+        p.partial = ws_partials(ws);
+        p.counters = ws_counters(ws);
+    }
+    const bool n8 = pl.nt == 8;
+    switch (kind_of(q)) {
+        case kInt4: return n8 ? launch_gemv_kind<kInt4, 8>(p, q->packed, pl.nsplit, st)
+                              : launch_gemv_kind<kInt4, 16>(p, q->packed, pl.nsplit, st);
+        case kInt2: return n8 ? launch_gemv_kind<kInt2, 8>(p, q->packed, pl.nsplit, st)
+                              : launch_gemv_kind<kInt2, 16>(p, q->packed, pl.nsplit, st);
+        default: return n8 ? launch_gemv_kind<kCode4, 8>(p, q->packed, pl.nsplit, st)
+                           : launch_gemv_kind<kCode4, 16>(p, q->packed, pl.nsplit, st);
+    }
+}
+
 lbq_status run_fwd_gemm(const void* X, int m, const lbq_qweight* q, const void* B, int rank, float s,
                         const float* T, float* Y, int64_t ldy, const int32_t* perm, void* ws, int sms,
                         cudaStream_t st) {
-    const Plan pl = plan_gemm(m, q->n, q->k / 64, sms);
+    if (m <= kGemvMaxM) return run_gemv(X, m, q, B, rank, s, T, Y, ldy, perm, ws, sms, st);
+    const Plan pl = plan_fwd(m, q, sms);
     FwdParams p{};
     p.m = m;
     p.n = q->n;
@@ -193,9 +327,9 @@ lbq_status run_fwd_gemm(const void* X, int m, const lbq_qweight* q, const void* 
     p.nsplit = pl.nsplit;
     if (pl.nsplit > 1) {
         if (!ws) return LBQ_EWORKSPACE;
-        p.partial = static_cast<float*>(ws);
-        p.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + pl.partial_bytes);
-        if (cudaMemsetAsync(p.counters, 0, pl.counter_bytes, st) != cudaSuccess) return LBQ_ECUDA;
+        if (pl.tiles > kMaxSplitTiles) return LBQ_EUNSUPPORTED;
+        p.partial = ws_partials(ws);
+        p.counters = ws_counters(ws);
     }
     switch (kind_of(q)) {
         case kInt4: return launch_fwd_kind<kInt4>(pl.nt, p, X, m, q->k, q->packed, q->n, pl.nsplit, st);
@@ -217,9 +351,9 @@ lbq_status check_lora(int rank, const void* A, const void* B, const void* saved)
 // ---------------------------------------------------------------------------
 template <int NT, int BITS>
 lbq_status launch_bwd_nt(const BwdParams& p, const void* dY, const uint8_t* packed, cudaStream_t st) {
-    constexpr int S = FwdCfg<NT>::kStages, AS = FwdCfg<NT>::kAStages;
+    constexpr int S = BwdCfg<NT>::kStages, AS = BwdCfg<NT>::kAStages;
     constexpr int KTB = 128 * BITS / 8;
-    using L = GemmSmem<NT, S, AS, 64 * KTB>;
+    using L = GemmSmem<NT, S, AS, 64 * KTB, kBwdTabBytes>;
     auto kern = dqgemm_bwd_kernel<NT, BITS, S, AS>;
     const size_t smem = L::total(p.rank_pad);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
@@ -365,7 +499,7 @@ lbq_status lbq_dequantize(const lbq_qweight* q, float* W_f32, lbq_stream_t strea
 size_t lbq_linear_fwd_workspace_size(int m, const lbq_qweight* q, int rank) {
     (void)rank;
     if (m < 1 || check_qweight(q, false) != LBQ_OK) return 0;
-    return plan_gemm(m, q->n, q->k / 64, sm_count()).workspace();
+    return plan_fwd(m, q, sm_count()).workspace();
 }
 
 lbq_status lbq_linear_fwd(const void* X, int m, const lbq_qweight* q, const void* A, const void* B, int rank,
@@ -377,7 +511,7 @@ lbq_status lbq_linear_fwd(const void* X, int m, const lbq_qweight* q, const void
     if (!aligned16(X) || !aligned16(Y)) return LBQ_EALIGN;
     if ((st = check_lora(rank, A, B, T_save)) != LBQ_OK) return st;
     const int sms = sm_count();
-    const size_t need = plan_gemm(m, q->n, q->k / 64, sms).workspace();
+    const size_t need = plan_fwd(m, q, sms).workspace();
     if (need > 0 && (!workspace || workspace_bytes < need)) return LBQ_EWORKSPACE;
     if (need > 0 && !aligned16(workspace)) return LBQ_EALIGN;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
@@ -397,7 +531,7 @@ lbq_status lbq_linear_fwd_noalloc(const void* X, int m, const lbq_qweight* q, co
     if (!aligned16(X) || !aligned16(Y)) return LBQ_EALIGN;
     if ((st = check_lora(rank, A, B, T_save)) != LBQ_OK) return st;
     const int sms = sm_count();
-    const size_t need = plan_gemm(m, q->n, q->k / 64, sms).workspace();
+    const size_t need = plan_fwd(m, q, sms).workspace();
     if (need > kNoAllocScratchBytes) return LBQ_EWORKSPACE;  // this call's scratch does not fit
     void* scratch = nullptr;
     if (need > 0 && (st = noalloc_scratch_address(&scratch)) != LBQ_OK) return st;
@@ -415,8 +549,7 @@ size_t lbq_linear_fwd_mix_workspace_size(int m, const lbq_qweight_mix* q, int ra
     if (!q || m < 1) return 0;
     if (check_qweight(&q->hi, false) != LBQ_OK || check_qweight(&q->lo, false) != LBQ_OK) return 0;
     const int sms = sm_count();
-    return round_up(plan_gemm(m, q->hi.n, q->hi.k / 64, sms).workspace(), 256) +
-           plan_gemm(m, q->lo.n, q->lo.k / 64, sms).workspace();
+    return std::max(plan_fwd(m, &q->hi, sms).workspace(), plan_fwd(m, &q->lo, sms).workspace());
 }
 
 lbq_status lbq_linear_fwd_mix(const void* X, int m, const lbq_qweight_mix* q, const void* A, const void* B, int rank,
@@ -432,8 +565,8 @@ lbq_status lbq_linear_fwd_mix(const void* X, int m, const lbq_qweight_mix* q, co
     if (!aligned16(X) || !aligned16(Y) || !aligned16(q->perm)) return LBQ_EALIGN;
     if ((st = check_lora(rank, A, B, T_save)) != LBQ_OK) return st;
     const int sms = sm_count();
-    const size_t need_hi = round_up(plan_gemm(m, q->hi.n, q->hi.k / 64, sms).workspace(), 256);
-    const size_t need = need_hi + plan_gemm(m, q->lo.n, q->lo.k / 64, sms).workspace();
+    // the two halves run one after the other on `stream` and share the workspace
+    const size_t need = std::max(plan_fwd(m, &q->hi, sms).workspace(), plan_fwd(m, &q->lo, sms).workspace());
     if (need > 0 && (!workspace || workspace_bytes < need)) return LBQ_EWORKSPACE;
     if (need > 0 && !aligned16(workspace)) return LBQ_EALIGN;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
@@ -445,14 +578,13 @@ lbq_status lbq_linear_fwd_mix(const void* X, int m, const lbq_qweight_mix* q, co
     }
     if ((st = run_fwd_gemm(X, m, &q->hi, B, rank, s, T_save, Y, n_total, q->perm, workspace, sms, cs)) != LBQ_OK)
         return st;
-    void* ws_lo = workspace ? static_cast<uint8_t*>(workspace) + need_hi : nullptr;
-    return run_fwd_gemm(X, m, &q->lo, B, rank, s, T_save, Y, n_total, q->perm + q->hi.n, ws_lo, sms, cs);
+    return run_fwd_gemm(X, m, &q->lo, B, rank, s, T_save, Y, n_total, q->perm + q->hi.n, workspace, sms, cs);
 }
 
 size_t lbq_linear_bwd_workspace_size(int m, const lbq_qweight* q, int rank) {
     (void)rank;
     if (m < 1 || check_qweight(q, false) != LBQ_OK) return 0;
-    return plan_gemm(m, q->k, cdiv(q->n, 64), sm_count()).workspace();
+    return plan_gemm(m, q->k, cdiv(q->n, 64), sm_count(), 128).workspace();
 }
 
 lbq_status lbq_linear_bwd(const void* dY, int m, const lbq_qweight* q, const void* A, const void* B, int rank,
@@ -465,7 +597,7 @@ lbq_status lbq_linear_bwd(const void* dY, int m, const lbq_qweight* q, const voi
     if (!aligned16(dY) || !aligned16(dX)) return LBQ_EALIGN;
     if ((st = check_lora(rank, A, B, U_save)) != LBQ_OK) return st;
     const int sms = sm_count();
-    const Plan pl = plan_gemm(m, q->k, cdiv(q->n, 64), sms);
+    const Plan pl = plan_gemm(m, q->k, cdiv(q->n, 64), sms, 128);
     if (pl.workspace() > 0 && (!workspace || workspace_bytes < pl.workspace())) return LBQ_EWORKSPACE;
     if (pl.workspace() > 0 && !aligned16(workspace)) return LBQ_EALIGN;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
@@ -491,9 +623,9 @@ lbq_status lbq_linear_bwd(const void* dY, int m, const lbq_qweight* q, const voi
     p.cb_per_split = pl.per_split;
     p.nsplit = pl.nsplit;
     if (pl.nsplit > 1) {
-        p.partial = static_cast<float*>(workspace);
-        p.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + pl.partial_bytes);
-        if (cudaMemsetAsync(p.counters, 0, pl.counter_bytes, cs) != cudaSuccess) return LBQ_ECUDA;
+        if (pl.tiles > kMaxSplitTiles) return LBQ_EUNSUPPORTED;
+        p.partial = ws_partials(workspace);
+        p.counters = ws_counters(workspace);
     }
     if (q->bits == 4) return launch_bwd_bits<4>(pl.nt, p, dY, q->packed, cs);
     return launch_bwd_bits<2>(pl.nt, p, dY, q->packed, cs);
@@ -515,6 +647,16 @@ lbq_status lbq_lora_grads(const void* X, const void* dY, int m, int n, int k, co
         static_cast<const uint16_t*>(dY), m, n, T, rank, s, dB, rank, 1);
     return last_launch();
 }
+
+#ifdef LBQ_TRACE
+// Trace builds only: copy the pipeline trace (kinds x 256 clock stamps).
+int lbq_trace_read(long long* host, int n) {
+    const int total = kTraceKinds * kTraceLen;
+    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+    if (cudaMemcpyFromSymbol(host, g_trace, sizeof(long long) * (n < total ? n : total)) != cudaSuccess) return -1;
+    return total;
+}
+#endif
 
 lbq_status lbq_device_status(uint32_t* flags) {
     if (!flags) return LBQ_EINVAL;

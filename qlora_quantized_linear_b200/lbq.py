@@ -203,7 +203,8 @@ class ChannelMixWeight:
 
 def _workspace(nbytes: int, device):
     torch = _torch()
-    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device) if nbytes else None
+    # zero-filled once: the library leaves its counters at zero after every call
+    return torch.zeros(max(int(nbytes), 16), dtype=torch.uint8, device=device) if nbytes else None
 
 
 def linear_fwd(X, qw, A=None, B=None, s: float = 0.0, Y=None, T=None, workspace=None, stream=None):

@@ -44,7 +44,8 @@ def assert_within(got, ref, bound, what):
 
 def mixed_weight(n, k, seed, std=0.02):
     """Weights with outlier columns, all-positive / all-negative rows, a
-    constant group and a zero row (edge cases of the MinMax quantizer)."""
+    constant group, a zero row and a row far from zero relative to its
+    spread (its zero point is far outside the code range: |zero| > 128)."""
     w = syn.weight_bf16(n, k, std, seed, outlier_frac=0.01, outlier_scale=20.0).float()
     if n > 5:
         w[1] = w[1].abs() + 0.05
@@ -52,6 +53,8 @@ def mixed_weight(n, k, seed, std=0.02):
         w[3, :128] = 0.3
         w[4] = 0.0
         w[5, 7] = -0.0
+    if n > 6:
+        w[6] = 2.0 + w[6] * 0.2
     return w.to(torch.bfloat16)
 
 
@@ -178,6 +181,11 @@ FWD_CASES = [
     (1, 256, 1024, 0, "codebook", 4, False),
     (16, 256, 512, 16, "codebook", 4, True),
     (140, 256, 512, 0, "codebook", 4, True),
+    # decode sizes at full layer shapes: CTA shares of the k-blocks straddle row tiles
+    (1, 14336, 4096, 16, "minmax", 4, False),
+    (8, 4096, 4096, 8, "minmax", 2, False),
+    (12, 2000, 3200, 0, "codebook", 4, True),   # ragged n
+    (16, 4096, 14336, 16, "minmax", 4, False),
 ]
 
 
@@ -207,6 +215,25 @@ def test_linear_fwd_repeatable(lbq):
     Y1, _ = lbq.linear_fwd(X.cuda(), qw, A.cuda(), B.cuda(), 2.0)
     Y2, _ = lbq.linear_fwd(X.cuda(), qw, A.cuda(), B.cuda(), 2.0)
     assert torch.equal(Y1, Y2)
+
+
+def test_workspace_reused_across_shapes(lbq):
+    """One zero-filled workspace serves calls of different shapes and sizes in
+    any order: each call leaves the split-K arrival counters at zero."""
+    import ctypes
+    probs = []
+    for (m, n, k) in [(1, 1024, 4096), (16, 896, 2048), (64, 512, 4096), (3, 1024, 4096)]:
+        X, W, _, _ = fwd_problem(m, n, k, 0, seed=m + n)
+        qw = device_qweight(lbq, W, "minmax", 4, False, None)
+        probs.append((X.cuda(), qw, lbq.lbq_linear_fwd_workspace_size(m, ctypes.byref(qw.struct), 0)))
+    ws = lbq._workspace(max(p[2] for p in probs), "cuda")
+    ref = [lbq.linear_fwd(X, qw)[0] for X, qw, _ in probs]    # each with a fresh workspace
+    for order in ([0, 1, 2, 3], [3, 2, 1, 0, 0, 2]):
+        for i in order:
+            X, qw, _ = probs[i]
+            Y, _ = lbq.linear_fwd(X, qw, workspace=ws)
+            assert torch.equal(Y, ref[i]), f"case {i}"
+    assert_status_clean(lbq)
 
 
 def test_channel_mix_fwd(lbq):
