@@ -97,11 +97,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait until the barrier's phase with the given parity has completed.  Gives
 // up after kWaitLimitNs (or kWaitLimitIters polls), records kStatusTimeout,
 // sets *abort so the other roles of the CTA stop too, and returns false.
+// try_wait that may suspend the thread until the phase completes or about
+// 20 us pass, so that a waiting warp does not spin on the issue slots that the
+// working warps of its SM need.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 0; it < kWaitLimitIters; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity)) return true;
         if (*abort) return false;
         if ((it & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) break;
     }
@@ -116,7 +131,7 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 0; it < kWaitLimitIters; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity)) return true;
         if ((it & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) break;
     }
     record_status(kStatusTimeout);

@@ -35,6 +35,8 @@
 //    does not depend on scheduling.
 #pragma once
 
+#include <type_traits>
+
 #include "dqgemm.cuh"
 
 namespace lbq {
@@ -42,6 +44,8 @@ namespace lbq {
 constexpr int kGemvComputeWarps = 8;                            // 16 rows each: 128 rows per tile
 constexpr int kGemvThreads = 32 * (kGemvComputeWarps + 1);      // + one producer warp
 constexpr int kGemvWStages = 4;                                 // 16 KB weight boxes in flight
+constexpr int kGemvTabPerThread = 16;                           // constant-table entries per thread
+constexpr int kGemvMaxTabGroups = 2 * kGemvTabPerThread;        // groups (codebook: k-blocks) per CTA
 
 struct GemvParams {
     int m, n, k;                      // tokens, stored rows, input features
@@ -183,10 +187,12 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* sW = smem;                                           // WS x 16 KB
     const int xstride = p.share * 64 + 4;                         // bf16 per token row (+8 bytes)
-    uint16_t* sX = reinterpret_cast<uint16_t*>(smem + WS * kWBox);          // [m][xstride]
-    uint8_t* sTab = reinterpret_cast<uint8_t*>(sX + p.m * xstride);        // [groups][128] entries
-    const int tab_groups = p.share / GB;
-    uint32_t* s_lut = reinterpret_cast<uint32_t*>(sTab + tab_groups * 128 * TE);   // codebook pairs [256]
+    uint16_t* sX = reinterpret_cast<uint16_t*>(smem + WS * kWBox);          // [m + 1][xstride], row m zero
+    // constant table [128 rows][tstride]: an odd row stride keeps the eight
+    // rows that a warp reads at once in distinct banks
+    const int tstride = (p.share / GB) | 1;
+    uint8_t* sTab = reinterpret_cast<uint8_t*>(sX + (p.m + 1) * xstride);
+    uint32_t* s_lut = reinterpret_cast<uint32_t*>(sTab + 128 * tstride * TE);     // codebook pairs [256]
     uint64_t* full = reinterpret_cast<uint64_t*>(s_lut + (KIND == kCode4 ? 256 : 0));
     uint64_t* empty = full + WS;
     int* s_last = reinterpret_cast<int*>(empty + WS);
@@ -212,7 +218,69 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
     const int nbox0 = (n0 + SUB - 1) / SUB;
     const int nbox = nbox0 + (n1 + SUB - 1) / SUB;
 
-    if (tid == 0) {
+    // prologue, first half (compute threads): issue the global loads of this
+    // CTA's constants and of its first activation round before anything else,
+    // so that they reach memory ahead of the weight stream
+    const int ngr16 = nk * 4;                                      // 16-wide k groups of the slice
+    const int xtotal = p.m * ngr16;
+    constexpr int XU = (KIND == kCode4) ? 2 : 4;                  // activation loads in flight per round
+    const int G = nk / GB, G0 = n0 / GB;                           // table groups (codebook: k-blocks)
+    // table entry (row rl, group lg) of thread (warp w, lane) and slot u = 2 it + ch:
+    // rl = 16 w + 2 it + lane / 16, lg = lane % 16 + 16 ch (coalesced along the row)
+    uint32_t raw[kGemvTabPerThread], raw2[kGemvTabPerThread];
+    uint4 v[XU][2];
+    if (tid < kCompute) {
+#pragma unroll
+        for (int u = 0; u < kGemvTabPerThread; ++u) {
+            const int rl = 16 * warp + 2 * (u >> 1) + (lane >> 4), lg = (lane & 15) + 16 * (u & 1);
+            raw[u] = 0u;
+            raw2[u] = 0u;
+            if (lg < G) {
+                const bool sb = lg >= G0;
+                const int64_t r = static_cast<int64_t>(sb ? t0 + 1 : t0) * 128 + rl;
+                const int gl = sb ? lg - G0 : a0 / GB + lg;            // group (codebook: k-block) in the row
+                // plain loads only: no arithmetic on a loaded value before the
+                // barrier below, or the thread would wait for the data there
+                if (r < p.n) {
+                    if (KIND != kCode4) {
+                        raw[u] = __ldg(p.scale + r * p.ngroups + gl);
+                        raw2[u] = __ldg(p.zero + r * p.ngroups + gl);
+                    } else if (p.q8 != nullptr) {
+                        const int64_t bi = r * p.kbt + gl;
+                        raw[u] = __ldg(reinterpret_cast<const uint8_t*>(p.q8) + bi);
+                        raw2[u] = __float_as_uint(__ldg(p.s2 + (bi >> 8)));
+                    } else {
+                        raw[u] = __float_as_uint(__ldg(p.absmax + r * p.kbt + gl));
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < XU; ++u) {
+            const int e = tid + u * kCompute;
+            if (e < xtotal) {
+                const int t = e / ngr16, g16 = e - t * ngr16;
+                const int lk = g16 >> 2;
+                const int kb = lk < n0 ? a0 + lk : lk - n0;
+                const uint4* src = reinterpret_cast<const uint4*>(p.X + static_cast<int64_t>(t) * p.k + kb * 64 +
+                                                                  (g16 & 3) * 16);
+                v[u][0] = __ldg(src);
+                v[u][1] = __ldg(src + 1);
+            }
+        }
+    }
+
+    // the weight stream starts only once the compute threads have issued the
+    // loads above: small scattered loads queued behind megabytes of weight
+    // boxes come back microseconds late
+    auto issue_box = [&](int c) {
+        const int w = c % WS;
+        mbar_arrive_expect_tx(&full[w], kWBox);
+        const int x = c < nbox0 ? (a0 + c * SUB) * RB : (c - nbox0) * SUB * RB;
+        const int y = (c < nbox0 ? t0 : t0 + 1) * 128;
+        tma_load_2d(sW + w * kWBox, &tmW, &full[w], x, y);
+    };
+    if (tid == kCompute) {
         for (int i = 0; i < WS; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], kGemvComputeWarps);
@@ -228,12 +296,8 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
         if (lane == 0 && nbox > 0) {
             int issued = 0;
             for (int c = 0; c < nbox; ++c) {
-                const int w = c % WS;
-                if (c >= WS && !mbar_wait(&empty[w], ((c / WS) - 1) & 1, s_abort)) break;
-                mbar_arrive_expect_tx(&full[w], kWBox);
-                const int x = c < nbox0 ? (a0 + c * SUB) * RB : (c - nbox0) * SUB * RB;
-                const int y = (c < nbox0 ? t0 : t0 + 1) * 128;
-                tma_load_2d(sW + w * kWBox, &tmW, &full[w], x, y);
+                if (c >= WS && !mbar_wait(&empty[c % WS], ((c / WS) - 1) & 1, s_abort)) break;
+                issue_box(c);
                 issued = c + 1;
             }
             for (int c = max(0, issued - WS); c < issued; ++c) mbar_wait_drain(&full[c % WS], (c / WS) & 1);
@@ -242,88 +306,34 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
     }
 
     // ---------------------------------------------------------------- compute warps
-    // prologue: the table of this CTA's constants, then its activation slices
+    // prologue, second half: store the activations, convert the constants
+    // (the empty asm keeps every use of the loaded values after the barrier)
+#pragma unroll
+    for (int u = 0; u < kGemvTabPerThread; ++u) asm volatile("" : "+r"(raw[u]), "+r"(raw2[u]));
+#pragma unroll
+    for (int u = 0; u < XU; ++u)
+        asm volatile("" : "+r"(v[u][0].x), "+r"(v[u][0].y), "+r"(v[u][0].z), "+r"(v[u][0].w), "+r"(v[u][1].x),
+                     "+r"(v[u][1].y), "+r"(v[u][1].z), "+r"(v[u][1].w));
     {
-        // table entry (local group lg, row rl); groups of segment 1 follow those of segment 0
-        const int G = nk / GB, G0 = n0 / GB;
-        const int total = G * 128;
-        for (int e0 = tid; e0 < total; e0 += 8 * kCompute) {
-            uint32_t raw[8][2];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int e = e0 + u * kCompute;
-                raw[u][0] = 0u;
-                raw[u][1] = 0u;
-                if (e < total) {
-                    const int rl = e / G, lg = e - rl * G;
-                    const int tile = lg < G0 ? t0 : t0 + 1;
-                    const int gl = lg < G0 ? a0 / GB + lg : lg - G0;      // group (codebook: k-block) in the row
-                    const int64_t r = static_cast<int64_t>(tile) * 128 + rl;
-                    if (r < p.n) {
-                        if (KIND != kCode4) {
-                            raw[u][0] = __ldg(p.scale + r * p.ngroups + gl);
-                            raw[u][1] = __ldg(p.zero + r * p.ngroups + gl);
-                        } else if (p.q8 != nullptr) {
-                            const int64_t b = r * p.kbt + gl;
-                            raw[u][0] = static_cast<uint32_t>(static_cast<int32_t>(__ldg(p.q8 + b)));
-                            raw[u][1] = __float_as_uint(__ldg(p.s2 + (b >> 8)));
-                        } else {
-                            raw[u][0] = __float_as_uint(__ldg(p.absmax + r * p.kbt + gl));
-                        }
-                    }
-                }
-            }
-            const float dq_off = (KIND == kCode4 && p.q8 != nullptr) ? __ldg(p.offset) : 0.0f;
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int e = e0 + u * kCompute;
-                if (e < total) {
-                    const int rl = e / G, lg = e - rl * G;
-                    if (KIND != kCode4) {
-                        const uint16_t s16 = static_cast<uint16_t>(raw[u][0]), z16 = static_cast<uint16_t>(raw[u][1]);
-                        const float zf = f16_bits_to_f32(z16);
-                        uint32_t word;
-                        if (fabsf(zf) <= 128.0f) {
-                            // (128 + q) - (128 + z) = q - z exactly
-                            word = pack_bf16x2_rn(128.0f + zf, 0.0f) & 0xFFFFu;
-                        } else {
-                            // (128 + q) - 128 = q, and -z (fp16 bits) in the high half
-                            word = 0x4300u | (static_cast<uint32_t>(z16 ^ 0x8000u) << 16);
-                            *s_far = 1;
-                        }
-                        const float sf = f16_bits_to_f32(s16);
-                        *reinterpret_cast<uint2*>(sTab + (lg * 128 + rl) * 8) = make_uint2(word, __float_as_uint(sf));
-                    } else {
-                        float am = __uint_as_float(raw[u][0]);
-                        if (p.q8 != nullptr)
-                            am = __fadd_rn(__fmul_rn(__fdiv_rn(static_cast<float>(static_cast<int32_t>(raw[u][0])), 127.0f),
-                                                     __uint_as_float(raw[u][1])),
-                                           dq_off);
-                        *reinterpret_cast<float*>(sTab + (lg * 128 + rl) * 4) = am;
-                    }
-                }
-            }
-        }
         // activations of the m real tokens, permuted to the MMA step order
-        const int ngr16 = nk * 4;                                  // 16-wide k groups
-        const int xtotal = p.m * ngr16;
-        for (int e0 = tid; e0 < xtotal; e0 += 4 * kCompute) {
-            uint4 v[4][2];
+        for (int e0 = tid; e0 < xtotal; e0 += XU * kCompute) {
+            if (e0 != tid) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int e = e0 + u * kCompute;
-                if (e < xtotal) {
-                    const int t = e / ngr16, g16 = e - t * ngr16;
-                    const int lk = g16 >> 2;
-                    const int kb = lk < n0 ? a0 + lk : lk - n0;
-                    const uint4* src = reinterpret_cast<const uint4*>(p.X + static_cast<int64_t>(t) * p.k + kb * 64 +
-                                                                      (g16 & 3) * 16);
-                    v[u][0] = __ldg(src);
-                    v[u][1] = __ldg(src + 1);
+                for (int u = 0; u < XU; ++u) {
+                    const int e = e0 + u * kCompute;
+                    if (e < xtotal) {
+                        const int t = e / ngr16, g16 = e - t * ngr16;
+                        const int lk = g16 >> 2;
+                        const int kb = lk < n0 ? a0 + lk : lk - n0;
+                        const uint4* src = reinterpret_cast<const uint4*>(p.X + static_cast<int64_t>(t) * p.k +
+                                                                          kb * 64 + (g16 & 3) * 16);
+                        v[u][0] = __ldg(src);
+                        v[u][1] = __ldg(src + 1);
+                    }
                 }
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < XU; ++u) {
                 const int e = e0 + u * kCompute;
                 if (e < xtotal) {
                     const int t = e / ngr16, g16 = e - t * ngr16;
@@ -346,6 +356,39 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
                 }
             }
         }
+        // convert the constants into the table
+        const float dq_off = (KIND == kCode4 && p.q8 != nullptr) ? __ldg(p.offset) : 0.0f;
+#pragma unroll
+        for (int u = 0; u < kGemvTabPerThread; ++u) {
+            const int rl = 16 * warp + 2 * (u >> 1) + (lane >> 4), lg = (lane & 15) + 16 * (u & 1);
+            if (lg < G) {
+                if (KIND != kCode4) {
+                    const uint16_t s16 = static_cast<uint16_t>(raw[u]), z16 = static_cast<uint16_t>(raw2[u]);
+                    const float zf = f16_bits_to_f32(z16);
+                    uint32_t word;
+                    if (fabsf(zf) <= 128.0f) {
+                        // (128 + q) - (128 + z) = q - z exactly
+                        word = pack_bf16x2_rn(128.0f + zf, 0.0f) & 0xFFFFu;
+                    } else {
+                        // (128 + q) - 128 = q, and -z (fp16 bits) in the high half
+                        word = 0x4300u | (static_cast<uint32_t>(z16 ^ 0x8000u) << 16);
+                        *s_far = 1;
+                    }
+                    *reinterpret_cast<uint2*>(sTab + (rl * tstride + lg) * 8) =
+                        make_uint2(word, __float_as_uint(f16_bits_to_f32(s16)));
+                } else {
+                    float am = __uint_as_float(raw[u]);
+                    if (p.q8 != nullptr)
+                        am = __fadd_rn(__fmul_rn(__fdiv_rn(static_cast<float>(static_cast<int8_t>(static_cast<uint8_t>(raw[u]))), 127.0f),
+                                                 __uint_as_float(raw2[u])),
+                                       dq_off);
+                    *reinterpret_cast<float*>(sTab + (rl * tstride + lg) * 4) = am;
+                }
+            }
+        }
+        // row m: zeros, read by the lanes of tokens >= m
+        for (int e = tid; e < xstride / 2; e += kCompute)
+            reinterpret_cast<uint32_t*>(sX + p.m * xstride)[e] = 0u;
         if (KIND == kCode4) {
             for (int e = tid; e < 256; e += kCompute) {
                 // byte e = (first code << 4) | second code -> (codebook[first], codebook[second])
@@ -369,14 +412,14 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
         offs[s] = static_cast<uint32_t>((((off >> 4) ^ sw) << 4) | (off & 15));
     }
     const uint32_t wrow = smem_u32(sW) + rl0 * 128;
-    const uint32_t trow = smem_u32(sTab) + rl0 * TE;   // table entries of row rl0 (row rl0 + 8: + 8 TE)
-    // B fragments: token nt * 8 + g (lanes of tokens >= m read nothing and use 0)
-    bool tok_ok[NT8];
+    const uint32_t trow = smem_u32(sTab) + rl0 * tstride * TE;   // table row rl0 (row rl0 + 8: + 8 tstride TE)
+    // B fragments: token nt * 8 + g; lanes of tokens >= m read the zero row
+    // (a select per load would cost more than the loads themselves)
     uint32_t xthr[NT8];
 #pragma unroll
     for (int nt = 0; nt < NT8; ++nt) {
-        tok_ok[nt] = nt * 8 + g < p.m;
-        xthr[nt] = smem_u32(sX) + static_cast<uint32_t>((tok_ok[nt] ? nt * 8 + g : 0) * xstride + 16 * j) * 2;
+        const int tok = nt * 8 + g < p.m ? nt * 8 + g : p.m;
+        xthr[nt] = smem_u32(sX) + static_cast<uint32_t>(tok * xstride + 16 * j) * 2;
     }
     const bool far = *s_far != 0;                      // some group of this CTA has |zero| > 128
     uint32_t mg = 0x43004300u;
@@ -398,12 +441,14 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[nt][e] = cg[0][nt][e] = cg[1][nt][e] = 0.0f;
         uint32_t sub0 = 0x43004300u, sub1 = 0x43004300u;
-        float sf0 = 1.0f, sf1 = 1.0f, corr0 = 0.0f, corr1 = 0.0f;
+        float sf0 = 1.0f, sf1 = 1.0f;
 
         const int nbx = (nkb + SUB - 1) / SUB;
-        for (int bx = 0; bx < nbx; ++bx, ++c) {
-            const uint32_t w = c % WS;
-            if (!mbar_wait(&full[w], (c / WS) & 1u, s_abort)) break;
+        const int nfull = nkb / SUB;                      // boxes whose SUB k-blocks all belong to the segment
+        // one box of k-blocks; the per-k-block bounds test is compiled only
+        // into the copy used for a partial last box (it costs ~15% of the loop)
+        auto run_box = [&](auto partial_tag, int bx, uint32_t w) {
+            constexpr bool kPartial = decltype(partial_tag)::value;
             // the whole box's codes of this thread's two rows
             const uint32_t base = wrow + w * kWBox;
             uint32_t r0[SUB * TW], r1[SUB * TW];
@@ -421,28 +466,23 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
                     r1[s] = gemv_lds32(base + 1024 + offs[s]);
                 }
             }
-
 #pragma unroll
             for (int s = 0; s < SUB; ++s) {
                 const int i = bx * SUB + s;                 // k-block within the segment
-                if (i < nkb) {
-                    const int lk = lk0 + i;                 // k-block within the CTA's slice
+                if (!kPartial || i < nkb) {
+                    const int lk = lk0 + i;                 // k-block within the CTA's slice (>= 0)
                     if (s % GB == 0) {
                         // this group's constants from the table
-                        const uint32_t ta = trow + static_cast<uint32_t>(lk / GB) * (128 * TE);
+                        const uint32_t ta = trow + static_cast<uint32_t>(lk) / GB * TE;
                         if (KIND != kCode4) {
-                            const uint2 e0 = gemv_lds64(ta), e1 = gemv_lds64(ta + 8 * TE);
+                            const uint2 e0 = gemv_lds64(ta), e1 = gemv_lds64(ta + 8 * tstride * TE);
                             sub0 = __byte_perm(e0.x, 0u, 0x1010);
                             sub1 = __byte_perm(e1.x, 0u, 0x1010);
                             sf0 = __uint_as_float(e0.y);
                             sf1 = __uint_as_float(e1.y);
-                            if (far) {
-                                corr0 = f16_bits_to_f32(static_cast<uint16_t>(e0.x >> 16));
-                                corr1 = f16_bits_to_f32(static_cast<uint16_t>(e1.x >> 16));
-                            }
                         } else {
                             sf0 = __uint_as_float(gemv_lds32(ta));
-                            sf1 = __uint_as_float(gemv_lds32(ta + 8 * TE));
+                            sf1 = __uint_as_float(gemv_lds32(ta + 8 * tstride * TE));
                         }
                     }
                     // A fragments: 8 code pairs of each row as bf16x2
@@ -478,7 +518,7 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
                     for (int tau = 0; tau < 4; ++tau)
 #pragma unroll
                         for (int nt = 0; nt < NT8; ++nt)
-                            bxf[tau][nt] = tok_ok[nt] ? gemv_lds64(xthr[nt] + xoff + 8 * tau) : make_uint2(0u, 0u);
+                            bxf[tau][nt] = gemv_lds64(xthr[nt] + xoff + 8 * tau);
 #pragma unroll
                     for (int tau = 0; tau < 4; ++tau)
 #pragma unroll
@@ -494,35 +534,52 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
                     if (s % GB == GB - 1) {
 #pragma unroll
                         for (int nt = 0; nt < NT8; ++nt) {
-                            float gs[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) gs[e] = cg[0][nt][e] + cg[1][nt][e];
-                            if (KIND != kCode4 && far) {
-                                // -zero * (sum of x over the group) for groups with |zero| > 128
-                                const int tA = nt * 8 + 2 * j;
-                                float sx0 = 0.0f, sx1 = 0.0f;
-                                for (int kk = (lk + 1 - GB) * 64; kk < (lk + 1) * 64; ++kk) {
-                                    if (tA < p.m) sx0 += bf16_bits_to_f32(sX[tA * xstride + kk]);
-                                    if (tA + 1 < p.m) sx1 += bf16_bits_to_f32(sX[(tA + 1) * xstride + kk]);
-                                }
-                                gs[0] = fmaf(corr0, sx0, gs[0]);
-                                gs[1] = fmaf(corr0, sx1, gs[1]);
-                                gs[2] = fmaf(corr1, sx0, gs[2]);
-                                gs[3] = fmaf(corr1, sx1, gs[3]);
-                            }
-                            acc[nt][0] = fmaf(sf0, gs[0], acc[nt][0]);
-                            acc[nt][1] = fmaf(sf0, gs[1], acc[nt][1]);
-                            acc[nt][2] = fmaf(sf1, gs[2], acc[nt][2]);
-                            acc[nt][3] = fmaf(sf1, gs[3], acc[nt][3]);
+                            acc[nt][0] = fmaf(sf0, cg[0][nt][0] + cg[1][nt][0], acc[nt][0]);
+                            acc[nt][1] = fmaf(sf0, cg[0][nt][1] + cg[1][nt][1], acc[nt][1]);
+                            acc[nt][2] = fmaf(sf1, cg[0][nt][2] + cg[1][nt][2], acc[nt][2]);
+                            acc[nt][3] = fmaf(sf1, cg[0][nt][3] + cg[1][nt][3], acc[nt][3]);
                         }
                     }
                 }
             }
+        };
+        for (int bx = 0; bx < nbx; ++bx, ++c) {
+            const uint32_t w = c % WS;
+            if (!mbar_wait(&full[w], (c / WS) & 1u, s_abort)) break;
+            if (bx < nfull)
+                run_box(std::false_type{}, bx, w);
+            else
+                run_box(std::true_type{}, bx, w);
             // release the slot only after every loaded word has been used: an
             // arrive issued right behind the shared loads let the next TMA
             // write land before some of those loads had read the slot
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[w]);
+        }
+        if (KIND != kCode4 && far) {
+            // groups stored with |zero| > 128 ran as (q - 0); add their
+            // scale * (-zero) * (sum of x over the group) here
+            for (int lg = lk0 / GB; lg < (lk0 + nkb) / GB; ++lg) {
+                const uint32_t ta = trow + static_cast<uint32_t>(lg) * TE;
+                const uint2 e0 = gemv_lds64(ta), e1 = gemv_lds64(ta + 8 * tstride * TE);
+                const float z0 = f16_bits_to_f32(static_cast<uint16_t>(e0.x >> 16));
+                const float z1 = f16_bits_to_f32(static_cast<uint16_t>(e1.x >> 16));
+                if (z0 == 0.0f && z1 == 0.0f) continue;
+                const float k0 = __uint_as_float(e0.y) * z0, k1 = __uint_as_float(e1.y) * z1;
+#pragma unroll
+                for (int nt = 0; nt < NT8; ++nt) {
+                    const int tA = nt * 8 + 2 * j;
+                    float sx0 = 0.0f, sx1 = 0.0f;
+                    for (int kk = lg * GB * 64; kk < (lg + 1) * GB * 64; ++kk) {
+                        if (tA < p.m) sx0 += bf16_bits_to_f32(sX[tA * xstride + kk]);
+                        if (tA + 1 < p.m) sx1 += bf16_bits_to_f32(sX[(tA + 1) * xstride + kk]);
+                    }
+                    acc[nt][0] = fmaf(k0, sx0, acc[nt][0]);
+                    acc[nt][1] = fmaf(k0, sx1, acc[nt][1]);
+                    acc[nt][2] = fmaf(k1, sx0, acc[nt][2]);
+                    acc[nt][3] = fmaf(k1, sx1, acc[nt][3]);
+                }
+            }
         }
         lk0 += nkb;
         // -------------------------------------------------------------- segment epilogue

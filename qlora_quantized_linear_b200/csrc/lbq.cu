@@ -167,8 +167,8 @@ constexpr size_t kGemvSmemBudget = 113 * 1024;     // two CTAs per SM
 size_t gemv_smem_bytes(int m, int share, int kind) {
     const int gb = kind == kInt4 ? 2 : 1;
     const size_t entry = kind == kCode4 ? 4 : 8;
-    return 1024 + static_cast<size_t>(kGemvWStages) * 128 * 128 + static_cast<size_t>(m) * (share * 64 + 4) * 2 +
-           static_cast<size_t>(share / gb) * 128 * entry + (kind == kCode4 ? 1024 : 0) + 2 * kGemvWStages * 8 + 16;
+    return 1024 + static_cast<size_t>(kGemvWStages) * 128 * 128 + static_cast<size_t>(m + 1) * (share * 64 + 4) * 2 +
+           static_cast<size_t>((share / gb) | 1) * 128 * entry + (kind == kCode4 ? 1024 : 0) + 2 * kGemvWStages * 8 + 16;
 }
 
 Plan plan_gemv(int m, const lbq_qweight* q, int sms) {
@@ -181,7 +181,9 @@ Plan plan_gemv(int m, const lbq_qweight* q, int sms) {
     const int64_t total = static_cast<int64_t>(pl.tiles) * kbt;
     const int64_t slots = 2LL * sms;
     int64_t smax = gb;
-    while (smax + gb <= kbt && gemv_smem_bytes(m, static_cast<int>(smax + gb), kind) <= kGemvSmemBudget) smax += gb;
+    while (smax + gb <= kbt && (smax + gb) / gb <= kGemvMaxTabGroups &&
+           gemv_smem_bytes(m, static_cast<int>(smax + gb), kind) <= kGemvSmemBudget)
+        smax += gb;
     const int64_t waves = cdiv(total, slots * smax);
     int64_t share = cdiv(cdiv(total, waves * slots), gb) * gb;
     // at least an eighth of a row per CTA, so that the CTA finishing a tile
