@@ -311,8 +311,8 @@ def run_decode(args, dist, lbq, syn, torch, peaks):
     per_matrix = {f"M{m}/{name}": {"us": round(1e3 * statistics.median(v), 2),
                                      "GB/s": round(gemm_bytes(m, *wl.shapes[name]) / (statistics.median(v) / 1e3) / 1e9, 1)}
                   for (m, name), v in per.items()}
-    traffic = profiled_traffic("dqgemm_fwd_decode")
-    roofline = {"kernel": "dqgemm_fwd_kernel (decode, NT=16)", "bound": "hbm", "achieved": round(achieved, 1),
+    traffic = profiled_traffic("dqgemv_decode_8b")
+    roofline = {"kernel": "dqgemv_kernel (decode stream-K GEMV, all 14 calls of the step)", "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "peak_source": peaks["source"], "traffic": traffic,
                 "per_launch_bytes_avg": int(tot_bytes / max(1, sum(len(v) for v in per.values()))),
