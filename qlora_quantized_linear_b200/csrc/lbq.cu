@@ -417,6 +417,80 @@ lbq_status noalloc_scratch_address(void** out) {
 // ===========================================================================
 // C ABI
 // ===========================================================================
+// T = X A^T (row layout) or U = dY B (col layout), [m, rank] fp32.  Decode
+// sizes use one CTA per row; larger batches the tensor-core kernel.
+template <bool kCol, int R8>
+void launch_lora_rows_r8(const uint16_t* in, int64_t m, int64_t len, const uint16_t* wt, int r, float* out,
+                         cudaStream_t st) {
+    lora_rows_mma_kernel<kCol, R8><<<static_cast<unsigned>(cdiv(m, 16)), 256, 0, st>>>(in, m, len, wt, r, out);
+}
+
+template <bool kCol>
+lbq_status launch_lora_rows(const void* in, int64_t m, int64_t len, const void* wt, int r, float* out,
+                            cudaStream_t st) {
+    const uint16_t* a = static_cast<const uint16_t*>(in);
+    const uint16_t* w = static_cast<const uint16_t*>(wt);
+    if (m < 32) {
+        lora_rowdot_kernel<kCol><<<static_cast<unsigned>(m), 256, 0, st>>>(a, len, w, r, out);
+        return last_launch();
+    }
+    switch ((r + 7) / 8) {
+        case 1: launch_lora_rows_r8<kCol, 1>(a, m, len, w, r, out, st); break;
+        case 2: launch_lora_rows_r8<kCol, 2>(a, m, len, w, r, out, st); break;
+        case 3: launch_lora_rows_r8<kCol, 3>(a, m, len, w, r, out, st); break;
+        case 4: launch_lora_rows_r8<kCol, 4>(a, m, len, w, r, out, st); break;
+        case 5: launch_lora_rows_r8<kCol, 5>(a, m, len, w, r, out, st); break;
+        case 6: launch_lora_rows_r8<kCol, 6>(a, m, len, w, r, out, st); break;
+        case 7: launch_lora_rows_r8<kCol, 7>(a, m, len, w, r, out, st); break;
+        default: launch_lora_rows_r8<kCol, 8>(a, m, len, w, r, out, st); break;
+    }
+    return last_launch();
+}
+
+template <int R8>
+void launch_lora_colgrad_r8(const uint16_t* in, int64_t m, int64_t ncols, const float* coef, int r, float s,
+                            float* grad, int64_t ocs, int64_t ots, cudaStream_t st) {
+    auto kern = lora_colgrad_mma_kernel<R8>;
+    const int smem = ColGradSmem<R8>::kBytes;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(cdiv(ncols, 32)), kLoraSplit, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = kLoraSplit;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kern, in, m, ncols, coef, r, s, grad, ocs, ots);
+}
+
+lbq_status launch_lora_colgrad(const void* in, int64_t m, int64_t ncols, const float* coef, int r, float s,
+                               float* grad, int64_t ocs, int64_t ots, cudaStream_t st) {
+    const uint16_t* a = static_cast<const uint16_t*>(in);
+    if (r % 4 != 0) {
+        // coefficient rows are copied in 16-byte pieces: ranks that are not a
+        // multiple of 4 take the plain kernel
+        lora_colgrad_kernel<<<static_cast<unsigned>(cdiv(ncols, 32)), 256, 0, st>>>(a, m, ncols, coef, r, s, grad,
+                                                                                    ocs, ots);
+        return last_launch();
+    }
+    switch ((r + 7) / 8) {
+        case 1: launch_lora_colgrad_r8<1>(a, m, ncols, coef, r, s, grad, ocs, ots, st); break;
+        case 2: launch_lora_colgrad_r8<2>(a, m, ncols, coef, r, s, grad, ocs, ots, st); break;
+        case 3: launch_lora_colgrad_r8<3>(a, m, ncols, coef, r, s, grad, ocs, ots, st); break;
+        case 4: launch_lora_colgrad_r8<4>(a, m, ncols, coef, r, s, grad, ocs, ots, st); break;
+        case 5: launch_lora_colgrad_r8<5>(a, m, ncols, coef, r, s, grad, ocs, ots, st); break;
+        case 6: launch_lora_colgrad_r8<6>(a, m, ncols, coef, r, s, grad, ocs, ots, st); break;
+        case 7: launch_lora_colgrad_r8<7>(a, m, ncols, coef, r, s, grad, ocs, ots, st); break;
+        default: launch_lora_colgrad_r8<8>(a, m, ncols, coef, r, s, grad, ocs, ots, st); break;
+    }
+    return last_launch();
+}
+
 extern "C" {
 
 const char* lbq_status_string(lbq_status s) {
@@ -518,9 +592,7 @@ lbq_status lbq_linear_fwd(const void* X, int m, const lbq_qweight* q, const void
     if (need > 0 && !aligned16(workspace)) return LBQ_EALIGN;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     if (rank > 0) {
-        lora_rowdot_kernel<false><<<m, 256, 0, cs>>>(static_cast<const uint16_t*>(X), q->k,
-                                                     static_cast<const uint16_t*>(A), rank, T_save);
-        if ((st = last_launch()) != LBQ_OK) return st;
+        if ((st = launch_lora_rows<false>(X, m, q->k, A, rank, T_save, cs)) != LBQ_OK) return st;
     }
     return run_fwd_gemm(X, m, q, B, rank, s, T_save, Y, q->n, nullptr, workspace, sms, cs);
 }
@@ -539,9 +611,7 @@ lbq_status lbq_linear_fwd_noalloc(const void* X, int m, const lbq_qweight* q, co
     if (need > 0 && (st = noalloc_scratch_address(&scratch)) != LBQ_OK) return st;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     if (rank > 0) {
-        lora_rowdot_kernel<false><<<m, 256, 0, cs>>>(static_cast<const uint16_t*>(X), q->k,
-                                                     static_cast<const uint16_t*>(A), rank, T_save);
-        if ((st = last_launch()) != LBQ_OK) return st;
+        if ((st = launch_lora_rows<false>(X, m, q->k, A, rank, T_save, cs)) != LBQ_OK) return st;
     }
     return run_fwd_gemm(X, m, q, B, rank, s, T_save, Y, q->n, nullptr, scratch, sms, cs);
 }
@@ -574,9 +644,7 @@ lbq_status lbq_linear_fwd_mix(const void* X, int m, const lbq_qweight_mix* q, co
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     const int64_t n_total = static_cast<int64_t>(q->hi.n) + q->lo.n;
     if (rank > 0) {
-        lora_rowdot_kernel<false><<<m, 256, 0, cs>>>(static_cast<const uint16_t*>(X), q->hi.k,
-                                                     static_cast<const uint16_t*>(A), rank, T_save);
-        if ((st = last_launch()) != LBQ_OK) return st;
+        if ((st = launch_lora_rows<false>(X, m, q->hi.k, A, rank, T_save, cs)) != LBQ_OK) return st;
     }
     if ((st = run_fwd_gemm(X, m, &q->hi, B, rank, s, T_save, Y, n_total, q->perm, workspace, sms, cs)) != LBQ_OK)
         return st;
@@ -604,9 +672,7 @@ lbq_status lbq_linear_bwd(const void* dY, int m, const lbq_qweight* q, const voi
     if (pl.workspace() > 0 && !aligned16(workspace)) return LBQ_EALIGN;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     if (rank > 0) {
-        lora_rowdot_kernel<true><<<m, 256, 0, cs>>>(static_cast<const uint16_t*>(dY), q->n,
-                                                    static_cast<const uint16_t*>(B), rank, U_save);
-        if ((st = last_launch()) != LBQ_OK) return st;
+        if ((st = launch_lora_rows<true>(dY, m, q->n, B, rank, U_save, cs)) != LBQ_OK) return st;
     }
     BwdParams p{};
     p.m = m;
@@ -641,13 +707,9 @@ lbq_status lbq_lora_grads(const void* X, const void* dY, int m, int n, int k, co
     if (!aligned16(X) || !aligned16(dY) || !aligned16(T) || !aligned16(U) || !aligned16(dA) || !aligned16(dB))
         return LBQ_EALIGN;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    lora_colgrad_kernel<<<static_cast<unsigned>(cdiv(k, 32)), 256, 0, cs>>>(
-        static_cast<const uint16_t*>(X), m, k, U, rank, s, dA, 1, k);
-    lbq_status st = last_launch();
+    lbq_status st = launch_lora_colgrad(X, m, k, U, rank, s, dA, 1, k, cs);
     if (st != LBQ_OK) return st;
-    lora_colgrad_kernel<<<static_cast<unsigned>(cdiv(n, 32)), 256, 0, cs>>>(
-        static_cast<const uint16_t*>(dY), m, n, T, rank, s, dB, rank, 1);
-    return last_launch();
+    return launch_lora_colgrad(dY, m, n, T, rank, s, dB, rank, 1, cs);
 }
 
 #ifdef LBQ_TRACE

@@ -284,7 +284,8 @@ def test_linear_bwd_parity(lbq, m, n, k, rank, bits):
     assert_status_clean(lbq)
 
 
-@pytest.mark.parametrize("m,n,k,rank", [(8, 256, 512, 8), (130, 384, 768, 16), (64, 200, 512, 64)])
+@pytest.mark.parametrize("m,n,k,rank", [(8, 256, 512, 8), (130, 384, 768, 16), (64, 200, 512, 64), (300, 264, 640, 6),
+                                         (1000, 512, 1024, 12)])
 def test_lora_grads_parity(lbq, m, n, k, rank):
     s = 2.0
     X, W, A, B = fwd_problem(m, n, k, rank, seed=m + n + k)
