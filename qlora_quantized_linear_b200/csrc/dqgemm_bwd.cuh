@@ -4,24 +4,35 @@
 //
 //   dX[t, k] = sum_c dY[t, c] * W_hat[c, k]  (+ s * sum_u U[t, u] A[u, k])
 //
-// The weight is read in its stored [n, k] packed layout -- no transposed copy
-// exists.  One CTA computes a tile of 128 input features x NT tokens: thread i
-// of the dequantize warps owns input feature k0 + i (TMEM lane i) and, for each
-// block of 64 output channels c, gathers its column of codes from the staged
-// packed tile, so the MMA's A operand in tensor memory is W_hat^T with the
-// reduction over c along the columns.  dY tiles [NT x 64 c] arrive by TMA as
-// the B operand.  Per-channel scale/zero constants of each block are built
-// once per block into a shared-memory table.  Roles, rings, bounded waits and
-// the split-K reduction mirror the forward kernel.
+// computed as dX^T = W_hat^T dY^T: one CTA owns 128 input features x NT tokens
+// and runs over the output channels c in blocks of 64.
+//
+//  * The weight is read in its stored [n, k] packed layout.  Each block's
+//    64 channel rows x 128 features are dequantized row-wise -- the same cheap
+//    per-word unpacking as the forward -- into a bf16 tile in shared memory
+//    laid out as the MMA's A operand in MN-major form (features contiguous,
+//    128-byte swizzle).  No column gathers, no transposed copy.
+//  * dY tiles [NT tokens x 64 channels] arrive by TMA as the K-major B operand.
+//  * tcgen05.mma (A and B from shared memory, fp32 accumulator in tensor
+//    memory) computes D[feature, token].
+//  * Codes are paired as in the forward (two codes of a 32-bit word that sit
+//    two bytes apart), so within every 8 (INT4) or 16 (INT2) features the A
+//    tile holds the features in a fixed permuted order; the epilogue writes
+//    each tensor-memory lane back to its own feature.
+//  * Roles: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, warps 2..9
+//    dequantize and run the epilogue.  Rings, bounded waits and the split-K
+//    reduction (the last CTA of a tile sums the partials in split order) follow
+//    the forward kernel.
 #pragma once
 
 #include "dqgemm.cuh"
+#include "dqgemv.cuh"
 
 namespace lbq {
 
 struct BwdParams {
     int m, n, k;                 // tokens, weight rows (output channels), input features
-    int bits, ngroups;           // MinMax bit width, k / group
+    int bits, ngroups, group;    // MinMax bit width, k / group, group
     const uint16_t* scale;       // [n, ngroups]
     const uint16_t* zero;        // [n, ngroups]
     int rank, rank_pad;
@@ -35,46 +46,98 @@ struct BwdParams {
     uint32_t* counters;
 };
 
-// Two table buffers of 2048 bytes: G*32 PairConst + G*64 float2 each.
-constexpr int kBwdTabBytes = 4096;
+constexpr int kBwdThreads = 320;
+constexpr int kBwdDqWarps = 8;
 
-// Dequantization constants of one channel pair for one group (bf16x2 fast
-// path) and of single channels (fp32 exact path).
-struct PairConst {
-    uint32_t sub2, mul2;
-    uint32_t fast, pad;
+template <int NT>
+struct BwdCfg {
+    static constexpr int kXStages = NT <= 64 ? 4 : 2;
+    static constexpr int kWStages = 4;
+    static constexpr int kAStages = NT <= 64 ? 3 : 2;
+    static constexpr int kMinBlocks = 2;
 };
 
-template <int NT, int BITS, int STAGES, int ASTAGES>
-__global__ void __launch_bounds__(192, 2)
+template <int NT, int BITS, int XS, int WS, int AS>
+struct BwdSmem {
+    static constexpr int kKTB = 128 * BITS / 8;      // packed bytes of one channel row across the tile
+    static constexpr int kXBytes = NT * 128;         // dY tile: NT tokens x 64 channels, bf16
+    static constexpr int kWBytes = 64 * kKTB;        // packed weight tile: 64 channels
+    static constexpr int kABytes = 64 * 128 * 2;     // A tile: 64 channels x 128 features, bf16
+    static constexpr size_t kX = 0;                  // all SW128 tiles 1024-byte aligned
+    static constexpr size_t kA = kX + size_t(XS) * kXBytes;
+    static constexpr size_t kW = kA + size_t(AS) * kABytes;
+    static constexpr size_t kBar = kW + size_t(WS) * kWBytes;
+    static constexpr int kNumBars = 2 * XS + 2 * WS + 2 * AS + 1;
+    static constexpr size_t kMisc = kBar + kNumBars * 8;
+    static constexpr size_t kLoraT = (kMisc + 128 + 15) / 16 * 16;
+    static size_t total(int rank_pad) { return kLoraT + size_t(NT) * rank_pad * 4 + 1024; }
+};
+
+// Shared-memory descriptor of an MN-major operand with the 128-byte swizzle:
+// atoms of 8 K-rows x 128 bytes, `lbo` bytes between atoms along M (or N),
+// `sbo` bytes between groups of 8 K-rows.
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;
+    d |= static_cast<uint64_t>(2u) << 61;
+    return d;
+}
+
+// D (tensor memory) [+]= A (shared, descriptor) * B (shared, descriptor).
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Byte offset of 16-byte unit `fu` (features 8 fu .. 8 fu + 7) of channel row
+// c (0..63) in the MN-major A tile [64 channels][128 features]: groups of 8
+// channels 2048 bytes apart, the two 64-feature halves 1024 bytes apart,
+// rows 128 bytes apart, units swizzled with the row.
+__device__ __forceinline__ uint32_t bwd_a_offset(int c, int fu) {
+    const int row = c & 7, uu = fu & 7;
+    return static_cast<uint32_t>((c >> 3) * 2048 + (fu >> 3) * 1024 + row * 128 + ((uu ^ row) << 4));
+}
+
+template <int NT, int BITS, int XS, int WS, int AS, int MINB>
+__global__ void __launch_bounds__(kBwdThreads, MINB)
 dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constant__ CUtensorMap tmW,
                   const BwdParams p) {
-    constexpr int KTB = 128 * BITS / 8;       // packed bytes of one row across the 128-feature tile
-    constexpr int G = (BITS == 4) ? 1 : 2;    // groups covered by the 128-feature tile
-    using L = GemmSmem<NT, STAGES, ASTAGES, 64 * KTB, kBwdTabBytes>;
-    constexpr uint32_t kTxBytes = L::kXBytes + 64 * KTB;
-    constexpr int kACols = 32;
-    constexpr int kDCol = 0;
-    constexpr int kACol0 = (NT + 31) / 32 * 32;
-    constexpr uint32_t kTmemCols = tmem_cols_for(kACol0 + kACols * ASTAGES);
-    constexpr uint32_t kIdesc = idesc_bf16_f32(128, NT);
-    constexpr int kTabBuf = kBwdTabBytes / 2;  // one table buffer: G*32 PairConst + G*64 float2
+    using L = BwdSmem<NT, BITS, XS, WS, AS>;
+    constexpr int KTB = L::kKTB;
+    constexpr int KIND = BITS == 4 ? kInt4 : kInt2;
+    constexpr int PG = BITS == 4 ? 8 : 16;                 // features per pairing group
+    constexpr int SLOTS = BITS == 4 ? 4 : 2;               // (channel, word) units per thread and block
+    constexpr uint32_t kTmemCols = tmem_cols_for(NT);
+    constexpr uint32_t kIdesc = idesc_bf16_f32(128, NT) | (1u << 15);   // A is MN-major
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* sX = smem + L::kX;
+    uint8_t* sA = smem + L::kA;
     uint8_t* sW = smem + L::kW;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-    uint64_t* full = bars;
-    uint64_t* empty = bars + STAGES;
-    uint64_t* afull = bars + 2 * STAGES;
-    uint64_t* aempty = afull + ASTAGES;
-    uint64_t* dfull = aempty + ASTAGES;
+    uint64_t* fullX = bars;
+    uint64_t* emptyX = fullX + XS;
+    uint64_t* fullW = emptyX + XS;
+    uint64_t* emptyW = fullW + WS;
+    uint64_t* afull = emptyW + WS;
+    uint64_t* aempty = afull + AS;
+    uint64_t* dfull = aempty + AS;
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
     int* s_last = reinterpret_cast<int*>(smem + L::kMisc + 8);
-    // two table buffers: [G][32 pairs] PairConst, then [G][64 channels] float2 (sf, zf)
-    uint8_t* s_tab = smem + L::kTab;
     float* sT = reinterpret_cast<float*>(smem + L::kLoraT);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -86,12 +149,16 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
     const int ncb = min(p.cb_per_split, cb_total - cb0);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < STAGES; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1 + 4);
+        for (int i = 0; i < XS; ++i) {
+            mbar_init(&fullX[i], 1);
+            mbar_init(&emptyX[i], 1);
         }
-        for (int i = 0; i < ASTAGES; ++i) {
-            mbar_init(&afull[i], 4);
+        for (int i = 0; i < WS; ++i) {
+            mbar_init(&fullW[i], 1);
+            mbar_init(&emptyW[i], kBwdDqWarps);
+        }
+        for (int i = 0; i < AS; ++i) {
+            mbar_init(&afull[i], kBwdDqWarps);
             mbar_init(&aempty[i], 1);
         }
         mbar_init(dfull, 1);
@@ -112,129 +179,142 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
     const uint32_t tmem = *s_tmem;
 
     if (warp == 0) {
+        // ------------------------------------------------------------ producer
         if (lane == 0) {
-            int issued = 0;
+            int wi = 0, xi = 0;
             for (int i = 0; i < ncb; ++i) {
-                const int s = i % STAGES;
-                if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) - 1) & 1, s_abort)) break;
-                mbar_arrive_expect_tx(&full[s], kTxBytes);
+                const int w = i % WS, x = i % XS;
                 const int c0 = (cb0 + i) * 64;
-                tma_load_2d(sX + s * L::kXBytes, &tmDY, &full[s], c0, t0);
-                tma_load_2d(sW + s * L::kWBytes, &tmW, &full[s], k0 * BITS / 8, c0);
-                issued = i + 1;
+                if (i >= WS && !mbar_wait(&emptyW[w], ((i / WS) - 1) & 1, s_abort)) break;
+                mbar_arrive_expect_tx(&fullW[w], L::kWBytes);
+                tma_load_2d(sW + w * L::kWBytes, &tmW, &fullW[w], k0 * BITS / 8, c0);
+                wi = i + 1;
+                if (i >= XS && !mbar_wait(&emptyX[x], ((i / XS) - 1) & 1, s_abort)) break;
+                mbar_arrive_expect_tx(&fullX[x], L::kXBytes);
+                tma_load_2d(sX + x * L::kXBytes, &tmDY, &fullX[x], c0, t0);
+                xi = i + 1;
             }
-            for (int i = max(0, issued - STAGES); i < issued; ++i) mbar_wait_drain(&full[i % STAGES], (i / STAGES) & 1);
+            for (int i = max(0, xi - XS); i < xi; ++i) mbar_wait_drain(&fullX[i % XS], (i / XS) & 1);
+            for (int i = max(0, wi - WS); i < wi; ++i) mbar_wait_drain(&fullW[i % WS], (i / WS) & 1);
         }
     } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             bool ok = true;
             for (int i = 0; i < ncb && ok; ++i) {
-                const int s = i % STAGES, a = i % ASTAGES;
-                ok = mbar_wait(&full[s], (i / STAGES) & 1, s_abort) &&
-                     mbar_wait(&afull[a], (i / ASTAGES) & 1, s_abort);
+                const int x = i % XS, a = i % AS;
+                ok = mbar_wait(&fullX[x], (i / XS) & 1, s_abort) && mbar_wait(&afull[a], (i / AS) & 1, s_abort);
                 if (!ok) break;
                 tc_fence_after();
-                const uint64_t bdesc = smem_desc_k_sw128(smem_u32(sX + s * L::kXBytes));
+                const uint32_t abase = smem_u32(sA + a * L::kABytes);
+                const uint64_t bdesc = smem_desc_k_sw128(smem_u32(sX + x * L::kXBytes));
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    mma_ts(tmem + kDCol, tmem + kACol0 + a * kACols + 8 * j, bdesc + static_cast<uint64_t>(2 * j), kIdesc,
-                           (i > 0 || j > 0) ? 1u : 0u);
-                mma_commit(&empty[s]);
+                    mma_ss(tmem, smem_desc_mn_sw128(abase + j * 4096, 1024, 2048), bdesc + static_cast<uint64_t>(2 * j),
+                           kIdesc, (i > 0 || j > 0) ? 1u : 0u);
+                mma_commit(&emptyX[x]);
                 mma_commit(&aempty[a]);
             }
-            mma_commit(dfull);
-            mbar_wait_drain(dfull, 0);
+            mma_commit(dfull);          // also completes when nothing was issued
+            mbar_wait_drain(dfull, 0);  // MMAs done before tensor memory is freed
         }
     } else {
-        const int q = warp & 3;
-        const int r = q * 32 + lane;            // feature within the tile = TMEM lane
-        const int64_t kcol = k0 + r;
-        const bool col_ok = kcol < p.k;
-        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-        const int tid = threadIdx.x - 64;       // 0..127
-        const int bytecol = (BITS == 4) ? (r >> 1) : (r >> 2);
-        const int sh = (BITS == 4) ? ((r & 1) ? 0 : 4) : (6 - 2 * (r & 3));
-        const uint32_t msk = (BITS == 4) ? 0x000F000Fu : 0x00030003u;
-        const int gi = (G == 1) ? 0 : (r >> 6);
-        bool dead = false;  // after an abort: keep meeting the named barriers, skip the work
-        for (int i = 0; i < ncb; ++i) {
-            const int s = i % STAGES, a = i % ASTAGES;
-            const int c0 = (cb0 + i) * 64;
-            // --- constants of this block's 64 channels, built by the 128 threads
-            PairConst* tabp = reinterpret_cast<PairConst*>(s_tab + (i & 1) * kTabBuf);
-            float2* tabs = reinterpret_cast<float2*>(s_tab + (i & 1) * kTabBuf + G * 32 * sizeof(PairConst));
-            if (tid < 64 * G) {
-                const int cl = tid & 63, g = tid >> 6;
-                const int64_t c = c0 + cl;
-                float sf = 0.0f, zf = 0.0f;
-                if (c < p.n) {
-                    const int gg = (k0 / (BITS == 4 ? 128 : 64)) + g;
-                    sf = f16_bits_to_f32(__ldg(p.scale + c * p.ngroups + gg));
-                    zf = f16_bits_to_f32(__ldg(p.zero + c * p.ngroups + gg));
-                }
-                tabs[g * 64 + cl] = make_float2(sf, zf);
-            }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (tid < 32 * G) {
-                const int pp = tid & 31, g = tid >> 5;
-                const float2 e0 = tabs[g * 64 + 2 * pp], e1 = tabs[g * 64 + 2 * pp + 1];
-                PairConst pc;
-                pc.sub2 = pack_bf16x2_rn(128.0f + e0.y, 128.0f + e1.y);
-                pc.mul2 = pack_bf16x2_rn(e0.x, e1.x);
-                pc.fast = (fabsf(e0.y) <= 128.0f && fabsf(e1.y) <= 128.0f) ? 1u : 0u;
-                pc.pad = 0;
-                tabp[g * 32 + pp] = pc;
-            }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            dead = dead || !mbar_wait(&full[s], (i / STAGES) & 1, s_abort);
-            dead = dead || (i >= ASTAGES && !mbar_wait(&aempty[a], ((i / ASTAGES) - 1) & 1, s_abort));
-            if (dead) continue;
-            tc_fence_after();
-            uint32_t vals[32];
-            const uint8_t* wt = sW + s * L::kWBytes + bytecol;
+        // ------------------------------------------------------------ dequantize
+        const int tid = threadIdx.x - 64;                  // 0..255
+        // unit slot u: channel row cl(u) of the block and word fw of that row
+        const int fw = BITS == 4 ? (tid & 15) : (tid & 7);
+        const int crow0 = BITS == 4 ? (tid >> 4) : (tid >> 3);
+        const int cstep = BITS == 4 ? 16 : 32;
+        const int gsub = BITS == 4 ? 0 : (fw >> 2);        // 64-feature group of this word (INT2 g64)
+        const int gcol = k0 / p.group + gsub;
+        uint32_t mg = 0x43004300u;
+        asm volatile("" : "+r"(mg));
+        // constants of the next block's channels, loaded one block ahead
+        uint32_t ns[SLOTS], nz[SLOTS];
+        auto load_const = [&](int i) {
 #pragma unroll
-            for (int pp = 0; pp < 32; ++pp) {
-                const uint32_t b0 = wt[(2 * pp) * KTB];
-                const uint32_t b1 = wt[(2 * pp + 1) * KTB];
-                const uint32_t t = __byte_perm(b0, b1, 0x5410);
-                const PairConst pc = tabp[gi * 32 + pp];
-                if (pc.fast) {
-                    const uint32_t v = ((t >> sh) & msk) | 0x43004300u;
-                    vals[pp] = hsub_hmul_bf16x2(v, pc.sub2, pc.mul2);
-                } else {
-                    const float2 e0 = tabs[gi * 64 + 2 * pp], e1 = tabs[gi * 64 + 2 * pp + 1];
-                    const float w0 = __fmul_rn(__fsub_rn(static_cast<float>((t >> sh) & (msk & 0xFFFFu)), e0.y), e0.x);
-                    const float w1 = __fmul_rn(__fsub_rn(static_cast<float>((t >> (sh + 16)) & (msk & 0xFFFFu)), e1.y), e1.x);
-                    vals[pp] = pack_bf16x2_rn(w0, w1);
-                }
+            for (int u = 0; u < SLOTS; ++u) {
+                const int64_t c = static_cast<int64_t>(cb0 + i) * 64 + crow0 + u * cstep;
+                ns[u] = c < p.n ? __ldg(p.scale + c * p.ngroups + gcol) : 0u;
+                nz[u] = c < p.n ? __ldg(p.zero + c * p.ngroups + gcol) : 0u;
             }
-            tmem_st_32x32b_x32(tmem + lane_base + kACol0 + a * kACols, vals);
-            tmem_st_wait();
-            tc_fence_before();
+        };
+        if (ncb > 0) load_const(0);
+        for (int i = 0; i < ncb; ++i) {
+            const int w = i % WS, a = i % AS;
+            uint32_t cs[SLOTS], cz[SLOTS];
+#pragma unroll
+            for (int u = 0; u < SLOTS; ++u) {
+                cs[u] = ns[u];
+                cz[u] = nz[u];
+            }
+            if (i + 1 < ncb) load_const(i + 1);
+            if (!mbar_wait(&fullW[w], (i / WS) & 1, s_abort)) break;
+            if (i >= AS && !mbar_wait(&aempty[a], ((i / AS) - 1) & 1, s_abort)) break;
+            uint32_t words[SLOTS];
+#pragma unroll
+            for (int u = 0; u < SLOTS; ++u)
+                words[u] = *reinterpret_cast<const uint32_t*>(sW + w * L::kWBytes + (crow0 + u * cstep) * KTB + 4 * fw);
+            uint8_t* atile = sA + a * L::kABytes;
+#pragma unroll
+            for (int u = 0; u < SLOTS; ++u) {
+                const int c = crow0 + u * cstep;
+                const MinMaxConst mc = minmax_const(static_cast<uint16_t>(cs[u]), static_cast<uint16_t>(cz[u]));
+                uint32_t o[PG / 2];
+                if (BITS == 4)
+                    int4_pairs(words[u], mg, o);
+                else
+                    int2_pairs(words[u], mg, o);
+                if (mc.fast) {
+#pragma unroll
+                    for (int q = 0; q < PG / 2; ++q) o[q] = hsub_hmul_bf16x2(o[q], mc.sub2, mc.mul2);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < PG / 2; ++q)
+                        o[q] = minmax_pair_exact((o[q] & 0xFFu), (o[q] >> 16) & 0xFFu, mc);
+                }
+#pragma unroll
+                for (int h = 0; h < PG / 8; ++h)
+                    *reinterpret_cast<uint4*>(atile + bwd_a_offset(c, (PG / 8) * fw + h)) =
+                        make_uint4(o[4 * h], o[4 * h + 1], o[4 * h + 2], o[4 * h + 3]);
+            }
+            // the tile was written through the generic proxy; the tensor core reads it through the async one
+            fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&afull[a]);
-                mbar_arrive(&empty[s]);
+                mbar_arrive(&emptyW[w]);
             }
         }
 
         // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;                            // TMEM lane quarter of this warp
+        const int half = (warp - 2) >> 2;                  // token half
+        const int lrow = q * 32 + lane;                    // A-tile row = TMEM lane
+        // feature of this lane: the pairing order of its group of PG features
+        const int feat = (lrow & ~(PG - 1)) + gemv_xperm(KIND, lrow & (PG - 1));
+        const int64_t kcol = k0 + feat;
+        const bool col_ok = kcol < p.k;
+        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         const int mt = min(NT, p.m - t0);
         const bool lora = p.rank > 0;
         if (lora) {
-            for (int e = tid; e < NT * p.rank_pad; e += 128) {
+            for (int e = tid; e < NT * p.rank_pad; e += 32 * kBwdDqWarps) {
                 const int tt = e / p.rank_pad, u = e - tt * p.rank_pad;
                 sT[e] = (tt < mt && u < p.rank) ? p.U[static_cast<int64_t>(t0 + tt) * p.rank + u] : 0.0f;
             }
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("bar.sync 1, 256;" ::: "memory");
         const bool got = mbar_wait(dfull, 0, s_abort);
         tc_fence_after();
         const int rp = p.rank_pad;
         const bool splitk = p.nsplit > 1;
-        for (int jj = 0; jj < NT; jj += 16) {
+        constexpr int kHalfCols = NT >= 32 ? NT / 2 : 16;
+        const int c_begin = half * kHalfCols;
+        const int c_end = min(NT, c_begin + kHalfCols);
+        for (int jj = c_begin; jj < c_end; jj += 16) {
             uint32_t raw[16];
-            tmem_ld_32x32b_x16(tmem + lane_base + kDCol + jj, raw);
+            tmem_ld_32x32b_x16(tmem + lane_base + jj, raw);
             tmem_ld_wait();
             if (!col_ok || !got || jj >= mt) continue;
             float acc[16];
@@ -253,25 +333,30 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
         }
         if (splitk) {
             __threadfence();
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            asm volatile("bar.sync 1, 256;" ::: "memory");
             if (threadIdx.x == 64) {
                 const uint32_t tile = blockIdx.y * gridDim.x + blockIdx.x;
                 const uint32_t prev = atomicAdd(p.counters + tile, 1u);
                 const int last = (prev == static_cast<uint32_t>(p.nsplit - 1)) ? 1 : 0;
-                if (last) p.counters[tile] = 0u;
+                if (last) p.counters[tile] = 0u;   // left at zero for the next call
                 *s_last = last;
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            asm volatile("bar.sync 1, 256;" ::: "memory");
             if (*s_last && col_ok && got) {
                 __threadfence();
-                for (int jj = 0; jj < mt; jj += 16) {
+                for (int jj = c_begin; jj < min(c_end, mt); jj += 16) {
                     float acc[16];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        acc[j] = 0.0f;
-                        if (jj + j < mt)
-                            for (int sp = 0; sp < p.nsplit; ++sp)
-                                acc[j] += __ldcg(p.partial + (static_cast<int64_t>(sp) * p.m + t0 + jj + j) * p.k + kcol);
+                    for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
+                    for (int sp = 0; sp < p.nsplit; ++sp) {
+                        float part[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            part[j] = (jj + j < mt)
+                                          ? __ldcg(p.partial + (static_cast<int64_t>(sp) * p.m + t0 + jj + j) * p.k + kcol)
+                                          : 0.0f;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) acc[j] += part[j];
                     }
                     if (lora) lora_add16(acc, sT + jj * rp, rp, p.rank, p.A + kcol, p.s, p.k);
 #pragma unroll

@@ -216,12 +216,6 @@ Plan plan_fwd(int m, const lbq_qweight* q, int sms) {
     return plan_gemm(m, q->n, q->k / 64, sms, 256, q->bits == 2 ? 8 : 4);
 }
 
-template <int NT>
-struct BwdCfg {
-    static constexpr int kStages = NT <= 32 ? 8 : NT <= 64 ? 6 : 4;
-    static constexpr int kAStages = 2;
-};
-
 template <int NT, int KIND>
 lbq_status launch_fwd_nt(const FwdParams& p, const void* X, int m, int64_t k, const uint8_t* packed, int nrows,
                          int nsplit, cudaStream_t st) {
@@ -353,10 +347,9 @@ lbq_status check_lora(int rank, const void* A, const void* B, const void* saved)
 // ---------------------------------------------------------------------------
 template <int NT, int BITS>
 lbq_status launch_bwd_nt(const BwdParams& p, const void* dY, const uint8_t* packed, cudaStream_t st) {
-    constexpr int S = BwdCfg<NT>::kStages, AS = BwdCfg<NT>::kAStages;
-    constexpr int KTB = 128 * BITS / 8;
-    using L = GemmSmem<NT, S, AS, 64 * KTB, kBwdTabBytes>;
-    auto kern = dqgemm_bwd_kernel<NT, BITS, S, AS>;
+    using C = BwdCfg<NT>;
+    using L = BwdSmem<NT, BITS, C::kXStages, C::kWStages, C::kAStages>;
+    auto kern = dqgemm_bwd_kernel<NT, BITS, C::kXStages, C::kWStages, C::kAStages, C::kMinBlocks>;
     const size_t smem = L::total(p.rank_pad);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
         return LBQ_ECUDA;
@@ -364,11 +357,11 @@ lbq_status launch_bwd_nt(const BwdParams& p, const void* dY, const uint8_t* pack
     if (!make_map_2d(&tmDY, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.m, p.n, NT, 64, CU_TENSOR_MAP_SWIZZLE_128B))
         return LBQ_ECUDA;
     if (!make_map_2d(&tmW, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.n, static_cast<int64_t>(p.k) * BITS / 8, 64,
-                     KTB, CU_TENSOR_MAP_SWIZZLE_NONE))
+                     L::kKTB, CU_TENSOR_MAP_SWIZZLE_NONE))
         return LBQ_ECUDA;
     dim3 grid(static_cast<unsigned>(cdiv(p.k, 128)), static_cast<unsigned>(cdiv(p.m, NT)),
               static_cast<unsigned>(p.nsplit));
-    kern<<<grid, 192, smem, st>>>(tmDY, tmW, p);
+    kern<<<grid, kBwdThreads, smem, st>>>(tmDY, tmW, p);
     return last_launch();
 }
 
@@ -680,6 +673,7 @@ lbq_status lbq_linear_bwd(const void* dY, int m, const lbq_qweight* q, const voi
     p.k = q->k;
     p.bits = q->bits;
     p.ngroups = q->k / q->group;
+    p.group = q->group;
     p.scale = q->scale;
     p.zero = q->zero;
     p.rank = rank;
