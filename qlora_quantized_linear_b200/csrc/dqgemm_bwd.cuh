@@ -51,10 +51,10 @@ constexpr int kBwdDqWarps = 8;
 
 template <int NT>
 struct BwdCfg {
-    static constexpr int kXStages = NT <= 64 ? 4 : 2;
+    static constexpr int kXStages = NT <= 64 ? 4 : NT <= 128 ? 2 : 3;
     static constexpr int kWStages = 4;
     static constexpr int kAStages = NT <= 64 ? 3 : 2;
-    static constexpr int kMinBlocks = 2;
+    static constexpr int kMinBlocks = NT >= 256 ? 1 : 2;   // CTAs per SM
 };
 
 template <int NT, int BITS, int XS, int WS, int AS>

@@ -371,7 +371,8 @@ lbq_status launch_bwd_bits(int nt, const BwdParams& p, const void* dY, const uin
         case 16: return launch_bwd_nt<16, BITS>(p, dY, packed, st);
         case 32: return launch_bwd_nt<32, BITS>(p, dY, packed, st);
         case 64: return launch_bwd_nt<64, BITS>(p, dY, packed, st);
-        default: return launch_bwd_nt<128, BITS>(p, dY, packed, st);
+        case 128: return launch_bwd_nt<128, BITS>(p, dY, packed, st);
+        default: return launch_bwd_nt<256, BITS>(p, dY, packed, st);
     }
 }
 
@@ -647,7 +648,7 @@ lbq_status lbq_linear_fwd_mix(const void* X, int m, const lbq_qweight_mix* q, co
 size_t lbq_linear_bwd_workspace_size(int m, const lbq_qweight* q, int rank) {
     (void)rank;
     if (m < 1 || check_qweight(q, false) != LBQ_OK) return 0;
-    return plan_gemm(m, q->k, cdiv(q->n, 64), sm_count(), 128).workspace();
+    return plan_gemm(m, q->k, cdiv(q->n, 64), sm_count(), 256).workspace();
 }
 
 lbq_status lbq_linear_bwd(const void* dY, int m, const lbq_qweight* q, const void* A, const void* B, int rank,
@@ -660,7 +661,7 @@ lbq_status lbq_linear_bwd(const void* dY, int m, const lbq_qweight* q, const voi
     if (!aligned16(dY) || !aligned16(dX)) return LBQ_EALIGN;
     if ((st = check_lora(rank, A, B, U_save)) != LBQ_OK) return st;
     const int sms = sm_count();
-    const Plan pl = plan_gemm(m, q->k, cdiv(q->n, 64), sms, 128);
+    const Plan pl = plan_gemm(m, q->k, cdiv(q->n, 64), sms, 256);
     if (pl.workspace() > 0 && (!workspace || workspace_bytes < pl.workspace())) return LBQ_EWORKSPACE;
     if (pl.workspace() > 0 && !aligned16(workspace)) return LBQ_EALIGN;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
