@@ -218,9 +218,30 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
     const int nbox0 = (n0 + SUB - 1) / SUB;
     const int nbox = nbox0 + (n1 + SUB - 1) / SUB;
 
+    // the producer lane issues the first weight box at once; the rest of the
+    // ring fills only after the compute threads have issued their loads
+    // (small scattered loads queued behind megabytes of weight boxes come
+    // back microseconds late)
+    auto issue_box = [&](int c) {
+        const int w = c % WS;
+        mbar_arrive_expect_tx(&full[w], kWBox);
+        const int x = c < nbox0 ? (a0 + c * SUB) * RB : (c - nbox0) * SUB * RB;
+        const int y = (c < nbox0 ? t0 : t0 + 1) * 128;
+        tma_load_2d(sW + w * kWBox, &tmW, &full[w], x, y);
+    };
+    if (tid == kCompute) {
+        for (int i = 0; i < WS; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kGemvComputeWarps);
+        }
+        *s_abort = 0;
+        *s_far = 0;
+        fence_mbar_init();
+        if (nbox > 0) issue_box(0);
+    }
     // prologue, first half (compute threads): issue the global loads of this
-    // CTA's constants and of its first activation round before anything else,
-    // so that they reach memory ahead of the weight stream
+    // CTA's constants and of its first activation round, so that they reach
+    // memory ahead of all but the first weight box
     const int ngr16 = nk * 4;                                      // 16-wide k groups of the slice
     const int xtotal = p.m * ngr16;
     constexpr int XU = (KIND == kCode4) ? 2 : 4;                  // activation loads in flight per round
@@ -270,32 +291,13 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
         }
     }
 
-    // the weight stream starts only once the compute threads have issued the
-    // loads above: small scattered loads queued behind megabytes of weight
-    // boxes come back microseconds late
-    auto issue_box = [&](int c) {
-        const int w = c % WS;
-        mbar_arrive_expect_tx(&full[w], kWBox);
-        const int x = c < nbox0 ? (a0 + c * SUB) * RB : (c - nbox0) * SUB * RB;
-        const int y = (c < nbox0 ? t0 : t0 + 1) * 128;
-        tma_load_2d(sW + w * kWBox, &tmW, &full[w], x, y);
-    };
-    if (tid == kCompute) {
-        for (int i = 0; i < WS; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], kGemvComputeWarps);
-        }
-        *s_abort = 0;
-        *s_far = 0;
-        fence_mbar_init();
-    }
     __syncthreads();
 
     if (warp == kGemvComputeWarps) {
         // ------------------------------------------------------------ producer
         if (lane == 0 && nbox > 0) {
-            int issued = 0;
-            for (int c = 0; c < nbox; ++c) {
+            int issued = 1;
+            for (int c = 1; c < nbox; ++c) {
                 if (c >= WS && !mbar_wait(&empty[c % WS], ((c / WS) - 1) & 1, s_abort)) break;
                 issue_box(c);
                 issued = c + 1;
