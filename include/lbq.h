@@ -157,6 +157,16 @@ lbq_status lbq_dequantize(const lbq_qweight* q, float* W_f32,
  * allocation serves any number of later calls of any shape.  After a call
  * whose kernels timed out (LBQ_ETIMEOUT from lbq_device_status), zero it
  * again.  Calls that may run at the same time need separate workspaces.
+ *
+ * Overlap with the previous kernel: for m <= 16 the kernel is launched with
+ * programmatic stream serialisation and may start streaming the packed
+ * weight and its scales/zeros while the kernel before it on `stream` is
+ * still running (X, the workspace, Y and T_save are touched only after that
+ * kernel has finished).  When the previous library call on `stream` was
+ * lbq_quantize, the forward waits instead.  A caller's own kernel that
+ * writes the packed weight or its constants must not directly precede the
+ * forward on the same stream (record an event or launch through another
+ * stream in between).
  */
 size_t lbq_linear_fwd_workspace_size(int m, const lbq_qweight* q, int rank);
 lbq_status lbq_linear_fwd(const void* X, int m, const lbq_qweight* q,

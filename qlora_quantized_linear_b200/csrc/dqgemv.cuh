@@ -71,6 +71,8 @@ struct GemvParams {
     int64_t total;                    // tiles * kbt
     float* partial;                   // [grid + tiles][m][128]
     uint32_t* counters;               // [tiles], zero at launch
+    int w_early;                      // the packed weight and its constants may be read before the
+                                      // previous kernel on the stream has finished
 };
 
 // D = A B + C (C = D on entry), one m16n8k16 bf16 MMA with fp32 accumulation.
@@ -179,6 +181,8 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
     constexpr int kCompute = 32 * kGemvComputeWarps;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // let the next kernel on the stream be scheduled as soon as our CTAs leave
+    griddep_launch_dependents();
     if (tid == kCompute) tma_prefetch_desc(&tmW);
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -237,6 +241,7 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
         *s_abort = 0;
         *s_far = 0;
         fence_mbar_init();
+        if (!p.w_early) griddep_wait();
         if (nbox > 0) issue_box(0);
     }
     // prologue, first half (compute threads): issue the global loads of this
@@ -251,6 +256,9 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
     uint32_t raw[kGemvTabPerThread], raw2[kGemvTabPerThread];
     uint4 v[XU][2];
     if (tid < kCompute) {
+        // the weight's constants may be read early; the activations (and the
+        // workspace, Y, T) only after the previous kernel has finished
+        if (!p.w_early) griddep_wait();
 #pragma unroll
         for (int u = 0; u < kGemvTabPerThread; ++u) {
             const int rl = 16 * warp + 2 * (u >> 1) + (lane >> 4), lg = (lane & 15) + 16 * (u & 1);
@@ -276,6 +284,7 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
                 }
             }
         }
+        if (p.w_early) griddep_wait();
 #pragma unroll
         for (int u = 0; u < XU; ++u) {
             const int e = tid + u * kCompute;

@@ -2,6 +2,7 @@
 // tile and split selection, and kernel launches.  One translation unit holds
 // every kernel so that the device status word is a single object.
 #include <mutex>
+#include <unordered_set>
 
 #include "dqgemm.cuh"
 #include "dqgemm_bwd.cuh"
@@ -156,6 +157,23 @@ Plan plan_gemm(int m, int64_t out_rows, int64_t red_blocks, int sms, int max_nt 
     return pl;
 }
 
+// Streams on which the last library call was a quantization: the forward
+// that follows on such a stream reads the weight only after that kernel has
+// finished.  Any other forward may stream the packed weight while the kernel
+// before it on the stream is still running.
+std::mutex g_wq_mu;
+std::unordered_set<cudaStream_t> g_weights_written;
+
+void note_weights_written(cudaStream_t st) {
+    std::lock_guard<std::mutex> lock(g_wq_mu);
+    g_weights_written.insert(st);
+}
+
+bool weights_stable(cudaStream_t st) {
+    std::lock_guard<std::mutex> lock(g_wq_mu);
+    return g_weights_written.erase(st) == 0;
+}
+
 // Decode-sized batches (m <= 16) run the stream-K GEMV: every CTA gets an
 // equal share of the (row tile, k-block) work, a whole number of scale
 // groups and as many k-blocks as its shared memory holds (weight ring,
@@ -206,7 +224,20 @@ lbq_status launch_gemv_kind(const GemvParams& p, const uint8_t* packed, int grid
     if (!make_map_2d(&tmW, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.n, static_cast<int64_t>(p.k) * (KIND == kInt2 ? 2 : 4) / 8,
                      128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
         return LBQ_ECUDA;
-    kern<<<grid, kGemvThreads, smem, st>>>(tmW, p);
+    // programmatic dependent launch: the kernel may start during the previous
+    // kernel's tail and waits for it (griddepcontrol.wait) before reading
+    // anything that kernel can have written
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(kGemvThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tmW, p) != cudaSuccess) return LBQ_ECUDA;
     return last_launch();
 }
 
@@ -276,6 +307,7 @@ lbq_status run_gemv(const void* X, int m, const lbq_qweight* q, const void* B, i
     p.tiles = pl.tiles;
     p.share = pl.per_split;
     p.total = static_cast<int64_t>(pl.tiles) * p.kbt;
+    p.w_early = weights_stable(st) ? 1 : 0;
     if (p.total >= (int64_t(1) << 31)) return LBQ_EUNSUPPORTED;
     if (pl.workspace() > 0) {
         if (!ws) return LBQ_EWORKSPACE;
@@ -512,6 +544,7 @@ lbq_status lbq_quantize(const void* W_bf16, lbq_qweight* q, void* workspace, siz
     if (!W_bf16) return LBQ_EINVAL;
     if (!aligned16(W_bf16)) return LBQ_EALIGN;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    note_weights_written(s);
     const int64_t nchunks = static_cast<int64_t>(q->n) * q->k / 8;
     const int sms = sm_count();
     if (q->scheme == LBQ_MINMAX_ASYM) {
