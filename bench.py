@@ -222,9 +222,12 @@ class Decode8B:
         self.lbq.linear_fwd(self.X[(m, k)], self.qw[copy][name], Y=self.Y[(m, name)], workspace=self.ws[(m, name)],
                             stream=stream)
 
-    def capture(self, phase: int, stream):
+    def capture(self, phase: int, stream, probe: bool = False):
         """CUDA graph of one step: both decode sizes over the layer set, each
-        size on its own weight copy; timing events around every call."""
+        size on its own weight copy.  The timed graphs hold the 14 calls back
+        to back (each call may overlap the tail of the one before it); the
+        probe graphs put timing events around every call, which serialises
+        them, to give the per-call durations."""
         torch = self.torch
         g = torch.cuda.CUDAGraph()
         evs = []
@@ -232,12 +235,14 @@ class Decode8B:
             for j, m in enumerate(DECODE_M):
                 copy = (2 * phase + j) % COPIES
                 for name, (n, k) in self.shapes.items():
-                    e0 = torch.cuda.Event(enable_timing=True, external=True)
-                    e1 = torch.cuda.Event(enable_timing=True, external=True)
-                    e0.record()
+                    if probe:
+                        e0 = torch.cuda.Event(enable_timing=True, external=True)
+                        e1 = torch.cuda.Event(enable_timing=True, external=True)
+                        e0.record()
                     self.call(m, name, copy)
-                    e1.record()
-                    evs.append((m, name, e0, e1))
+                    if probe:
+                        e1.record()
+                        evs.append((m, name, e0, e1))
         return g, evs
 
 
@@ -295,28 +300,37 @@ def run_decode(args, dist, lbq, syn, torch, peaks):
     units = args.steps * wl.step_bytes * dist.world
     value = units / (ms_max / 1e3) / 1e9
 
-    # per-launch durations of the dominant kernel (the fused dequant-GEMM),
-    # from the events of the last replay of each graph inside the timed region
+    # The timed region launches nothing but the dominant kernel (the decode
+    # GEMV), back to back: its average launch duration is the region's
+    # device time over the launches in it.
+    launches = args.steps * wl.calls_per_step
+    avg_launch_ms = ms / launches
+    per_launch_bytes = wl.step_bytes / wl.calls_per_step
+    achieved = per_launch_bytes / (avg_launch_ms / 1e3) / 1e9
+    traffic = profiled_traffic("dqgemv_decode_8b")
+    roofline = {"kernel": "dqgemv_kernel (decode stream-K GEMV, all 14 calls of the step)", "bound": "hbm",
+                "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "peak_source": peaks["source"], "traffic": traffic,
+                "per_launch_bytes_avg": int(per_launch_bytes), "avg_launch_us": round(1e3 * avg_launch_ms, 3),
+                "launches_timed": launches}
+
+    # per-call durations, from probe graphs with an event pair around every
+    # call (the events keep consecutive calls from overlapping), after the
+    # timed region
+    probes = [wl.capture(ph, stream, probe=True) for ph in range(COPIES)]
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            for g, _evs in probes:
+                g.replay()
+    torch.cuda.synchronize()
     per = {}
-    tot_bytes = tot_ms = 0.0
-    for g, evs in graphs:
+    for g, evs in probes:
         for (m, name, e0, e1) in evs:
-            d = e0.elapsed_time(e1)
-            n, k = wl.shapes[name]
-            b = gemm_bytes(m, n, k)
-            per.setdefault((m, name), []).append(d)
-            tot_bytes += b
-            tot_ms += d
-    achieved = tot_bytes / (tot_ms / 1e3) / 1e9
+            per.setdefault((m, name), []).append(e0.elapsed_time(e1))
     per_matrix = {f"M{m}/{name}": {"us": round(1e3 * statistics.median(v), 2),
                                      "GB/s": round(gemm_bytes(m, *wl.shapes[name]) / (statistics.median(v) / 1e3) / 1e9, 1)}
                   for (m, name), v in per.items()}
-    traffic = profiled_traffic("dqgemv_decode_8b")
-    roofline = {"kernel": "dqgemv_kernel (decode stream-K GEMV, all 14 calls of the step)", "bound": "hbm", "achieved": round(achieved, 1),
-                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "peak_source": peaks["source"], "traffic": traffic,
-                "per_launch_bytes_avg": int(tot_bytes / max(1, sum(len(v) for v in per.values()))),
-                "launches_sampled": sum(len(v) for v in per.values())}
+    del probes
 
     # end to end through the public API: pinned host X in, Y out, every call
     e2e = run_decode_e2e(args, wl, lbq, torch, stream)
@@ -675,7 +689,7 @@ def main():
                                "INT4 g128 MinMax, forward dequant-GEMM at M=1 and M=16 per step",
                    "weights": "N(0, 0.02^2) bf16, 0.1% input channels x20, 7 seeded copies",
                    "l2": "7 rotating weight copies (116 MB per pass > one pass of L2 reuse; a copy returns every 7th pass)",
-                   "launch": "one CUDA graph per step (14 fused dequant-GEMM launches)",
+                   "launch": "one CUDA graph per step: 14 decode GEMV launches back to back (programmatic dependent launch); per_matrix from separate probe graphs with events between calls",
                    "parallelism": f"replicas x{dist.world}"},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": args.steps * wl_calls(),
