@@ -20,6 +20,20 @@
 
 namespace lbq {
 
+// rint(fl(w / d)), the IEEE quotient rounded half-to-even to an integer, for
+// finite w and a positive normal d with rs = fl(1 / d).  t = fl(w * rs) is
+// within 2 ulp of w / d and fl(w / d) within half an ulp, so rint(t) is the
+// answer whenever t is more than 3 ulp away from the nearest half-integer;
+// only those rare elements pay for the correctly rounded division.
+__device__ __forceinline__ float rint_div(float w, float d, float rs) {
+    const float t = __fmul_rn(w, rs);
+    const float n = rintf(t);
+    const float gap = 0.5f - fabsf(__fsub_rn(t, n));                 // distance to the half-integer
+    const float ulp3 = fmaxf(fabsf(t), 1.0f) * 3.5762786865234375e-07f;  // 3 * 2^-23 * max(|t|, 1)
+    if (gap > ulp3) return n;
+    return rintf(__fdiv_rn(w, d));
+}
+
 // ---------------------------------------------------------------------------
 // MinMax quantize + pack.  Group = 128 (4 bit) or 64 (2 bit); one group is
 // covered by GROUP/8 consecutive lanes.
@@ -68,9 +82,11 @@ __global__ void __launch_bounds__(256) minmax_quantize_kernel(const uint4* __res
         const uint16_t z16 = f32_to_f16_bits(rintf(__fdiv_rn(-mn, sf)));
         const float zf = f16_bits_to_f32(z16);
         uint32_t q[8];
+        const float rs = __frcp_rn(sf);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            float t = __fadd_rn(rintf(__fdiv_rn(v[i], sf)), zf);
+            float t = rint_div(v[i], sf, rs);
+            t = __fadd_rn(t, zf);
             t = fminf(fmaxf(t, 0.0f), Q);
             q[i] = static_cast<uint32_t>(t);
         }
