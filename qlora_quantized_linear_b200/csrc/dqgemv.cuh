@@ -460,28 +460,25 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
         // into the copy used for a partial last box (it costs ~15% of the loop)
         auto run_box = [&](auto partial_tag, int bx, uint32_t w) {
             constexpr bool kPartial = decltype(partial_tag)::value;
-            // the whole box's codes of this thread's two rows
             const uint32_t base = wrow + w * kWBox;
-            uint32_t r0[SUB * TW], r1[SUB * TW];
-#pragma unroll
-            for (int s = 0; s < SUB; ++s) {
-                if (TW == 2) {
-                    const uint2 v0 = gemv_lds64(base + offs[s]);
-                    const uint2 v1 = gemv_lds64(base + 1024 + offs[s]);
-                    r0[2 * s] = v0.x;
-                    r0[2 * s + 1] = v0.y;
-                    r1[2 * s] = v1.x;
-                    r1[2 * s + 1] = v1.y;
-                } else {
-                    r0[s] = gemv_lds32(base + offs[s]);
-                    r1[s] = gemv_lds32(base + 1024 + offs[s]);
-                }
-            }
 #pragma unroll
             for (int s = 0; s < SUB; ++s) {
                 const int i = bx * SUB + s;                 // k-block within the segment
                 if (!kPartial || i < nkb) {
                     const int lk = lk0 + i;                 // k-block within the CTA's slice (>= 0)
+                    // this k-block's codes of the thread's two rows
+                    uint32_t r0[2 * TW], r1[2 * TW];
+                    if (TW == 2) {
+                        const uint2 v0 = gemv_lds64(base + offs[s]);
+                        const uint2 v1 = gemv_lds64(base + 1024 + offs[s]);
+                        r0[0] = v0.x;
+                        r0[1] = v0.y;
+                        r1[0] = v1.x;
+                        r1[1] = v1.y;
+                    } else {
+                        r0[0] = gemv_lds32(base + offs[s]);
+                        r1[0] = gemv_lds32(base + 1024 + offs[s]);
+                    }
                     if (s % GB == 0) {
                         // this group's constants from the table
                         const uint32_t ta = trow + static_cast<uint32_t>(lk) / GB * TE;
@@ -499,20 +496,20 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
                     // A fragments: 8 code pairs of each row as bf16x2
                     uint32_t f0[8], f1[8];
                     if (KIND == kInt4) {
-                        int4_pairs(r0[2 * s], mg, f0);
-                        int4_pairs(r0[2 * s + 1], mg, f0 + 4);
-                        int4_pairs(r1[2 * s], mg, f1);
-                        int4_pairs(r1[2 * s + 1], mg, f1 + 4);
+                        int4_pairs(r0[0], mg, f0);
+                        int4_pairs(r0[TW - 1], mg, f0 + 4);
+                        int4_pairs(r1[0], mg, f1);
+                        int4_pairs(r1[TW - 1], mg, f1 + 4);
                     } else if (KIND == kInt2) {
-                        int2_pairs(r0[s], mg, f0);
-                        int2_pairs(r1[s], mg, f1);
+                        int2_pairs(r0[0], mg, f0);
+                        int2_pairs(r1[0], mg, f1);
                     } else {
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
-                            f0[q] = s_lut[__byte_perm(r0[2 * s], 0u, 0x4440 + q)];
-                            f0[4 + q] = s_lut[__byte_perm(r0[2 * s + 1], 0u, 0x4440 + q)];
-                            f1[q] = s_lut[__byte_perm(r1[2 * s], 0u, 0x4440 + q)];
-                            f1[4 + q] = s_lut[__byte_perm(r1[2 * s + 1], 0u, 0x4440 + q)];
+                            f0[q] = s_lut[__byte_perm(r0[0], 0u, 0x4440 + q)];
+                            f0[4 + q] = s_lut[__byte_perm(r0[TW - 1], 0u, 0x4440 + q)];
+                            f1[q] = s_lut[__byte_perm(r1[0], 0u, 0x4440 + q)];
+                            f1[4 + q] = s_lut[__byte_perm(r1[TW - 1], 0u, 0x4440 + q)];
                         }
                     }
                     if (KIND != kCode4) {
