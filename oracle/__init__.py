@@ -65,6 +65,8 @@ def _declare(L) -> None:
         "oracle_lora_grads": (_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _int, _dbl, _vp, _vp, _vp, _vp]),
         "oracle_linear_fwd_sampled_minmax": (_int, [_vp, _i64, _vp, _vp, _vp, _i64, _i64, _int, _int,
                                                     _vp, _vp, _int, _dbl, _i64, _vp, _vp, _vp, _vp]),
+        "oracle_linear_bwd_sampled_minmax": (_int, [_vp, _i64, _vp, _vp, _vp, _i64, _i64, _int, _int,
+                                                    _vp, _vp, _int, _dbl, _i64, _vp, _vp, _vp, _vp]),
         "oracle_set_threads": (None, [_int]),
         "oracle_get_threads": (_int, []),
     }
@@ -266,3 +268,23 @@ def linear_fwd_sampled_minmax(X, packed, scale, zero, n: int, k: int, bits: int,
         _p(X), m, _p(packed), _p(scale), _p(zero), n, k, bits, group, _p(A), _p(B), r, float(s),
         rows.shape[0], _p(rows), _p(cols), _p(Y), _p(Yb)), "linear_fwd_sampled_minmax")
     return Y, Yb
+
+
+def linear_bwd_sampled_minmax(dY, packed, scale, zero, n: int, k: int, bits: int, group: int,
+                              rows, cols, A=None, B=None, s: float = 0.0):
+    """dX and its bound at the (rows[i] = token, cols[i] = feature) pairs, from the packed weight."""
+    dY = _u16(dY)
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    scale, zero = _u16(scale), _u16(zero)
+    m = dY.shape[0]
+    r = 0 if A is None else A.shape[0]
+    A = None if A is None else _u16(A)
+    B = None if B is None else _u16(B)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    cols = np.ascontiguousarray(cols, dtype=np.int64)
+    dX = np.zeros(rows.shape[0], np.float64)
+    dXb = np.zeros(rows.shape[0], np.float64)
+    _check(lib().oracle_linear_bwd_sampled_minmax(
+        _p(dY), m, _p(packed), _p(scale), _p(zero), n, k, bits, group, _p(A), _p(B), r, float(s),
+        rows.shape[0], _p(rows), _p(cols), _p(dX), _p(dXb)), "linear_bwd_sampled_minmax")
+    return dX, dXb

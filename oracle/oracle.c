@@ -508,3 +508,47 @@ int oracle_linear_fwd_sampled_minmax(const uint16_t* X, int64_t m,
     }
     return 0;
 }
+
+/* dX (and its bound) at a list of (token, feature) pairs, for sampled parity
+ * at full size ([QL] QLoRA技术原理: dX = dY W_hat + s (dY B) A).  Each pair
+ * is computed on its own from the packed MinMax weight, one column of W_hat
+ * at a time, with U = dY B recomputed for its token. */
+int oracle_linear_bwd_sampled_minmax(const uint16_t* dY, int64_t m,
+                                     const uint8_t* packed,
+                                     const uint16_t* scale,
+                                     const uint16_t* zero, int64_t n,
+                                     int64_t k, int bits, int group,
+                                     const uint16_t* A, const uint16_t* B,
+                                     int r, double s, int64_t npairs,
+                                     const int64_t* rows, const int64_t* cols,
+                                     double* dX, double* dXbound) {
+    if (!(bits == 2 || bits == 4) || k % group != 0 || r < 0) return -1;
+#pragma omp parallel for schedule(dynamic, 8)
+    for (int64_t p = 0; p < npairs; ++p) {
+        int64_t t = rows[p], col = cols[p];
+        if (t < 0 || t >= m || col < 0 || col >= k) continue;
+        double acc = 0.0, bnd = 0.0;
+        for (int64_t c = 0; c < n; ++c) {
+            double g = oracle_bf16_to_f32(dY[t * n + c]);
+            double w = minmax_element(packed, scale, zero, k, bits, group, c, col);
+            acc += g * w;
+            bnd += fabs(g) * fabs(w);
+        }
+        double lora = 0.0, lbnd = 0.0;
+        for (int u = 0; u < r; ++u) {
+            double uu = 0.0, ub = 0.0;
+            for (int64_t c = 0; c < n; ++c) {
+                double g = oracle_bf16_to_f32(dY[t * n + c]);
+                double b = oracle_bf16_to_f32(B[c * r + u]);
+                uu += g * b;
+                ub += fabs(g) * fabs(b);
+            }
+            double a = oracle_bf16_to_f32(A[u * k + col]);
+            lora += uu * a;
+            lbnd += ub * fabs(a);
+        }
+        dX[p] = acc + s * lora;
+        dXbound[p] = bnd + fabs(s) * lbnd;
+    }
+    return 0;
+}

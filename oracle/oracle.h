@@ -122,6 +122,18 @@ int  oracle_linear_fwd_sampled_minmax(const uint16_t* X, int64_t m,
                                       const int64_t* rows, const int64_t* cols,
                                       double* Y, double* Ybound);
 
+/* dX (and its bound) at a list of (token, feature) pairs only, from the
+ * packed MinMax weight (no full fp32 matrix); U = dY B per sampled token. */
+int  oracle_linear_bwd_sampled_minmax(const uint16_t* dY, int64_t m,
+                                      const uint8_t* packed,
+                                      const uint16_t* scale,
+                                      const uint16_t* zero, int64_t n,
+                                      int64_t k, int bits, int group,
+                                      const uint16_t* A, const uint16_t* B,
+                                      int r, double s, int64_t npairs,
+                                      const int64_t* rows, const int64_t* cols,
+                                      double* dX, double* dXbound);
+
 /* Threads used by the loops over rows (OpenMP); 0 keeps the default. */
 void oracle_set_threads(int nthreads);
 int  oracle_get_threads(void);

@@ -369,6 +369,20 @@ def test_sampled_forward_matches_full():
     np.testing.assert_allclose(Ybs, Yb[rows, cols], rtol=1e-13)
 
 
+def test_sampled_backward_matches_full():
+    X, What, A, B, _, (codes, scale, zero) = _tiny_problem()
+    s = 2.0
+    n, k = What.shape
+    m = X.shape[0]
+    dY = _bf16(np.random.default_rng(9).standard_normal((m, n)).astype(np.float32) * 0.1)
+    dX, _, dXb = oracle.linear_bwd(dY, What, A, B, s)
+    rows = np.array([0, 2, 1, 3, 0]); cols = np.array([0, 100, 7, 255, 129])
+    dXs, dXbs = oracle.linear_bwd_sampled_minmax(dY, oracle.pack(codes, 4), scale, zero, n, k, 4, 128,
+                                                 rows, cols, A, B, s)
+    np.testing.assert_allclose(dXs, dX[rows, cols], rtol=1e-12, atol=1e-16)
+    np.testing.assert_allclose(dXbs, dXb[rows, cols], rtol=1e-12)
+
+
 def _loss(X, What, A, B, s, dY):
     Y, _, _ = oracle.linear_fwd(X, What, A, B, s)
     return float(np.sum(oracle.bf16_to_f32(dY).astype(np.float64) * Y))
