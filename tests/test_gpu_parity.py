@@ -299,3 +299,66 @@ def test_lora_grads_parity(lbq, m, n, k, rank):
     assert_within(dA.cpu().numpy(), dAr, dAb, "dA")
     assert_within(dB.cpu().numpy(), dBr, dBb, "dB")
     assert_status_clean(lbq)
+
+
+# --------------------------------------------------------------------------- full-size training step
+@pytest.fixture(scope="module")
+def train_problem(lbq):
+    """The 8B MLP gate layer of the QLoRA step at full size: W 14336 x 4096
+    INT4 g128, M = 4096 tokens, rank 16, s = 2 (the benchmark's training row)."""
+    m, n, k, r, s = 4096, 14336, 4096, 16, 2.0
+    W = syn.weight_bf16(n, k, 0.02, seed=41, outlier_frac=0.001)
+    X = syn.normal_bf16((m, k), 1.0, seed=42)
+    A = syn.normal_bf16((r, k), 0.01, seed=43)
+    B = syn.normal_bf16((n, r), 0.01, seed=44)
+    dY = syn.normal_bf16((m, n), 0.1, seed=45)
+    codes, scale, zero = oracle.minmax_quantize(syn.bits_u16(W), 4, 128)
+    packed = oracle.pack(codes, 4)
+    qw = lbq.QuantizedWeight(n, k, "minmax", 4)
+    qw.packed.copy_(torch.from_numpy(packed))
+    qw.scale.copy_(torch.from_numpy(scale.view(np.float16)))
+    qw.zero.copy_(torch.from_numpy(zero.view(np.float16)))
+    Xd, Ad, Bd, dYd = X.cuda(), A.cuda(), B.cuda(), dY.cuda()
+    Y, T = lbq.linear_fwd(Xd, qw, Ad, Bd, s)
+    dX, U = lbq.linear_bwd(dYd, qw, Ad, Bd, s)
+    dA, dB = lbq.lora_grads(Xd, dYd, T, U, s)
+    torch.cuda.synchronize()
+    return dict(m=m, n=n, k=k, r=r, s=s, X=X, A=A, B=B, dY=dY, packed=packed, scale=scale, zero=zero,
+                Y=Y.cpu().numpy(), dX=dX.cpu().numpy(), dA=dA.cpu().numpy(), dB=dB.cpu().numpy())
+
+
+def _sample_pairs(nr, nc, count, seed):
+    """`count` seeded (row, col) pairs plus one full row and one full column."""
+    rng = np.random.default_rng(seed)
+    r = rng.integers(0, nr, count)
+    c = rng.integers(0, nc, count)
+    fr, fc = int(rng.integers(0, nr)), int(rng.integers(0, nc))
+    rows = np.concatenate([r, np.full(nc, fr), np.arange(nr)])
+    cols = np.concatenate([c, np.arange(nc), np.full(nr, fc)])
+    return rows, cols
+
+
+def test_training_forward_full_size_sampled(lbq, train_problem):
+    P = train_problem
+    rows, cols = _sample_pairs(P["m"], P["n"], 4096, seed=5)
+    ref, bound = oracle.linear_fwd_sampled_minmax(syn.bits_u16(P["X"]), P["packed"], P["scale"], P["zero"],
+                                                  P["n"], P["k"], 4, 128, rows, cols, syn.bits_u16(P["A"]),
+                                                  syn.bits_u16(P["B"]), P["s"])
+    assert_within(P["Y"][rows, cols], ref, bound, "Y")
+
+
+def test_training_backward_full_size_sampled(lbq, train_problem):
+    P = train_problem
+    rows, cols = _sample_pairs(P["m"], P["k"], 2048, seed=6)
+    ref, bound = oracle.linear_bwd_sampled_minmax(syn.bits_u16(P["dY"]), P["packed"], P["scale"], P["zero"],
+                                                  P["n"], P["k"], 4, 128, rows, cols, syn.bits_u16(P["A"]),
+                                                  syn.bits_u16(P["B"]), P["s"])
+    assert_within(P["dX"][rows, cols], ref, bound, "dX")
+
+
+def test_training_lora_grads_full_size(lbq, train_problem):
+    P = train_problem
+    dA, dB, dAb, dBb = oracle.lora_grads(syn.bits_u16(P["X"]), syn.bits_u16(P["dY"]), syn.bits_u16(P["A"]),
+                                         syn.bits_u16(P["B"]), P["s"])
+    assert_within(P["dA"], dA, dAb, "dA")
+    assert_within(P["dB"], dB, dBb, "dB")
