@@ -139,18 +139,25 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- distributed plumbing
 class Dist:
+    """One process per GPU (torchrun env).  NCCL on GPUs; gloo when there is
+    no GPU (or LBQ_DIST_BACKEND=gloo), which the CPU tests use."""
+
     def __init__(self):
         import torch
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.torch = torch
+        self.backend = os.environ.get("LBQ_DIST_BACKEND") or ("nccl" if torch.cuda.is_available() else "gloo")
         if self.world > 1:
             import datetime
-            torch.cuda.set_device(self.local)
-            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                                 device_id=torch.device("cuda", self.local))
-        else:
+            if self.backend == "nccl":
+                torch.cuda.set_device(self.local)
+                torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                                     device_id=torch.device("cuda", self.local))
+            else:
+                torch.distributed.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+        elif torch.cuda.is_available():
             torch.cuda.set_device(0)
 
     def barrier(self):
@@ -160,13 +167,20 @@ class Dist:
     def max(self, x: float) -> float:
         if self.world == 1:
             return x
-        t = self.torch.tensor([x], dtype=self.torch.float64, device="cuda")
+        dev = "cuda" if self.backend == "nccl" else "cpu"
+        t = self.torch.tensor([x], dtype=self.torch.float64, device=dev)
         self.torch.distributed.all_reduce(t, op=self.torch.distributed.ReduceOp.MAX)
         return float(t.item())
 
     def close(self):
         if self.world > 1:
             self.torch.distributed.destroy_process_group()
+
+
+def replica_value(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job throughput of N independent replicas (weak scaling): the
+    units all ranks processed over the slowest rank's device time, in G/s."""
+    return units_per_rank * world / (ms_max / 1e3) / 1e9
 
 
 # ----------------------------------------------------------------------------- byte / flop accounting
@@ -297,8 +311,7 @@ def run_decode(args, dist, lbq, syn, torch, peaks):
     clocks["timed_s"] = round(host1 - host0, 3)
 
     ms_max = dist.max(ms)
-    units = args.steps * wl.step_bytes * dist.world
-    value = units / (ms_max / 1e3) / 1e9
+    value = replica_value(args.steps * wl.step_bytes, dist.world, ms_max)
 
     # The timed region launches nothing but the dominant kernel (the decode
     # GEMV), back to back: its average launch duration is the region's
