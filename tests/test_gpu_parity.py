@@ -362,3 +362,60 @@ def test_training_lora_grads_full_size(lbq, train_problem):
                                          syn.bits_u16(P["B"]), P["s"])
     assert_within(P["dA"], dA, dAb, "dA")
     assert_within(P["dB"], dB, dBb, "dB")
+
+
+# --------------------------------------------------------------------------- full-size 70B codebook layer
+@pytest.fixture(scope="module")
+def codebook70b(lbq):
+    """The 70B attention projection (8192 x 8192) in the 4-bit codebook
+    format with double quantization, quantized on the GPU, at the benchmark's
+    sizes."""
+    n = k = 8192
+    cb = syn.codebook_normal16()
+    W = syn.weight_bf16(n, k, 0.015, seed=71)
+    qw = lbq.QuantizedWeight(n, k, "codebook", double_quant=True, codebook=cb).quantize(W.cuda())
+    torch.cuda.synchronize()
+    codes, absmax = oracle.codebook_quantize(syn.bits_u16(W), cb)
+    packed = oracle.pack(codes, 4)
+    q8, s2, off, exact = oracle.double_quant(absmax)
+    What = oracle.codebook_dequantize(packed, oracle.double_dequant(q8, s2, off), cb, n, k)
+    return dict(n=n, k=k, qw=qw, packed=packed, q8=q8, s2=s2, off=off, exact=exact, What=What)
+
+
+def test_codebook70b_quantize_full_size(lbq, codebook70b):
+    C = codebook70b
+    assert C["exact"]
+    assert np.array_equal(C["qw"].packed.cpu().numpy(), C["packed"])
+    assert np.array_equal(C["qw"].q8.cpu().numpy(), C["q8"])
+    assert np.array_equal(C["qw"].s2.cpu().numpy().view(np.uint32), C["s2"].view(np.uint32))
+    assert np.float32(C["qw"].offset[0].item()).view(np.uint32) == np.float32(C["off"]).view(np.uint32)
+    assert_status_clean(lbq)
+
+
+def test_codebook70b_decode_full_size(lbq, codebook70b):
+    C = codebook70b
+    X = syn.normal_bf16((1, C["k"]), 1.0, seed=72)
+    Y, _ = lbq.linear_fwd(X.cuda(), C["qw"])
+    torch.cuda.synchronize()
+    Yr, _, Yb = oracle.linear_fwd(syn.bits_u16(X), C["What"])
+    assert_within(Y.cpu().numpy(), Yr, Yb, "Y")
+
+
+def test_codebook70b_prefill_full_size_sampled(lbq, codebook70b):
+    C = codebook70b
+    m = 2048
+    X = syn.normal_bf16((m, C["k"]), 1.0, seed=73)
+    Y, _ = lbq.linear_fwd(X.cuda(), C["qw"])
+    torch.cuda.synchronize()
+    rows, cols = _sample_pairs(m, C["n"], 2048, seed=7)
+    x = oracle.bf16_to_f32(syn.bits_u16(X))
+    w = C["What"]
+    ref = np.empty(rows.size)
+    bound = np.empty(rows.size)
+    for i in range(0, rows.size, 1024):          # sampled dot products, a chunk at a time
+        xr = x[rows[i:i + 1024]].astype(np.float64)
+        wc = w[cols[i:i + 1024]].astype(np.float64)
+        ref[i:i + 1024] = np.einsum("ij,ij->i", xr, wc)
+        bound[i:i + 1024] = np.einsum("ij,ij->i", np.abs(xr), np.abs(wc))
+    assert_within(Y.cpu().numpy()[rows, cols], ref, bound, "Y")
+    assert_status_clean(lbq)
