@@ -30,9 +30,12 @@
 //    every lane that uses it;
 //  * stream-K: the grid is a whole number of waves and every CTA gets an equal
 //    contiguous share of the (row tile, k-block) work, spanning at most two
-//    row tiles.  A tile covered by several CTAs is finished by the last of them
-//    (per-tile counter), which sums the partials in CTA order, so the result
-//    does not depend on scheduling.
+//    row tiles.  A tile covered by several CTAs is finished by the one that
+//    covers its last k-block (the highest CTA index among them): the others
+//    store their partial sums, count themselves on a per-tile flag and leave
+//    without waiting; the finishing CTA waits for the count (CTAs start in
+//    index order, so its contributors are running or done) and adds the
+//    partials in CTA order, so the result does not depend on scheduling.
 #pragma once
 
 #include <type_traits>
@@ -43,7 +46,7 @@ namespace lbq {
 
 constexpr int kGemvComputeWarps = 8;                            // 16 rows each: 128 rows per tile
 constexpr int kGemvThreads = 32 * (kGemvComputeWarps + 1);      // + one producer warp
-constexpr int kGemvWStages = 4;                                 // 16 KB weight boxes in flight
+constexpr int kGemvMaxWStages = 4;                              // 16 KB weight boxes in flight (3 or 4)
 constexpr int kGemvTabPerThread = 16;                           // constant-table entries per thread
 constexpr int kGemvMaxTabGroups = 2 * kGemvTabPerThread;        // groups (codebook: k-blocks) per CTA
 
@@ -70,7 +73,7 @@ struct GemvParams {
     int share;                        // k-blocks per CTA (<= kbt; a multiple of the scale group)
     int64_t total;                    // tiles * kbt
     float* partial;                   // [grid + tiles][m][128]
-    uint32_t* counters;               // [tiles], zero at launch
+    uint32_t* counters;               // [tiles] arrival flags, zero at launch and left at zero
     int w_early;                      // the packed weight and its constants may be read before the
                                       // previous kernel on the stream has finished
 };
@@ -100,9 +103,10 @@ struct GemvTile {
     static constexpr int kThreadBytes = kRowBytes / 4;                 // a quarter row
     static constexpr int kSub = 128 / kRowBytes;                       // k-blocks per weight box
     static constexpr int kGroupBlocks = (KIND == kInt4) ? 2 : 1;       // k-blocks per scale group
-    // shared table of per-(group, row) constants: MinMax {subtrahend, scale},
+    // shared table of per-(group, row) constants, 4 bytes each: MinMax the
+    // bf16 subtrahend 128 + zero (low half) and the fp16 scale (high half);
     // codebook the fp32 absmax of each (k-block, row)
-    static constexpr int kTabEntry = (KIND == kCode4) ? 4 : 8;
+    static constexpr int kTabEntry = 4;
 };
 
 // Order of the 16 activations of a 16-wide k group as the MMA steps consume
@@ -166,7 +170,34 @@ __device__ __forceinline__ uint32_t gemv_lds32(uint32_t addr) {
     return v;
 }
 
-template <int KIND, int NTOK>
+// Split-tile flags: a contributor publishes its partial sums (stored by all
+// threads of the CTA before the barrier that precedes this call) and counts
+// itself; the finishing CTA waits for the count with acquire semantics.
+__device__ __forceinline__ void flag_publish(uint32_t* f) {
+    asm volatile("fence.acq_rel.gpu;\n\tred.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(f) : "memory");
+}
+
+__device__ __forceinline__ uint32_t flag_load_acquire(const uint32_t* f) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    return v;
+}
+
+// Bounded wait for *f >= want; records kStatusTimeout and returns false when
+// it gives up.
+__device__ __forceinline__ bool flag_wait_geq(const uint32_t* f, uint32_t want) {
+    if (flag_load_acquire(f) >= want) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 0; it < kWaitLimitIters; ++it) {
+        __nanosleep(64);
+        if (flag_load_acquire(f) >= want) return true;
+        if ((it & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) break;
+    }
+    record_status(kStatusTimeout);
+    return false;
+}
+
+template <int KIND, int NTOK, int WS>
 __global__ void __launch_bounds__(kGemvThreads, 2)
 dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
     constexpr int NT8 = NTOK / 8;
@@ -176,7 +207,7 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
     constexpr int TB = GemvTile<KIND>::kThreadBytes;
     constexpr int TE = GemvTile<KIND>::kTabEntry;
     constexpr int TW = TB / 4;                                    // code words per row, k-block and thread
-    constexpr int WS = kGemvWStages;
+    static_assert(WS >= 2 && WS <= kGemvMaxWStages, "weight ring depth");
     constexpr int kWBox = 128 * 128;
     constexpr int kCompute = 32 * kGemvComputeWarps;
 
@@ -191,17 +222,19 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* sW = smem;                                           // WS x 16 KB
     const int xstride = p.share * 64 + 4;                         // bf16 per token row (+8 bytes)
-    uint16_t* sX = reinterpret_cast<uint16_t*>(smem + WS * kWBox);          // [m + 1][xstride], row m zero
+    // token rows, plus a zero row m when the token tile has padding lanes
+    const int xrows = p.m < NTOK ? p.m + 1 : p.m;
+    uint16_t* sX = reinterpret_cast<uint16_t*>(smem + WS * kWBox);          // [xrows][xstride]
     // constant table [128 rows][tstride]: an odd row stride keeps the eight
     // rows that a warp reads at once in distinct banks
     const int tstride = (p.share / GB) | 1;
-    uint8_t* sTab = reinterpret_cast<uint8_t*>(sX + (p.m + 1) * xstride);
+    uint8_t* sTab = reinterpret_cast<uint8_t*>(sX + xrows * xstride);
     uint32_t* s_lut = reinterpret_cast<uint32_t*>(sTab + 128 * tstride * TE);     // codebook pairs [256]
     uint64_t* full = reinterpret_cast<uint64_t*>(s_lut + (KIND == kCode4 ? 256 : 0));
     uint64_t* empty = full + WS;
-    int* s_last = reinterpret_cast<int*>(empty + WS);
-    volatile int* s_abort = s_last + 1;
-    int* s_far = s_last + 2;
+    int* s_misc = reinterpret_cast<int*>(empty + WS);
+    volatile int* s_abort = s_misc;
+    int* s_far = s_misc + 1;
 
     // this CTA's work: up to two (tile, first k-block, k-blocks) segments
     // (tiles * kbt < 2^31, checked by the host)
@@ -219,8 +252,11 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
     }
     const int nseg = n0 == 0 ? 0 : (n1 == 0 ? 1 : 2);
     const int nk = n0 + n1;
-    const int nbox0 = (n0 + SUB - 1) / SUB;
-    const int nbox = nbox0 + (n1 + SUB - 1) / SUB;
+    // the second segment (the start of tile t0 + 1) is processed first: its
+    // partial sums are published before this CTA waits on anything, so the
+    // CTAs that finish tiles never wait on each other in a chain
+    const int nbox1 = (n1 + SUB - 1) / SUB;
+    const int nbox = nbox1 + (n0 + SUB - 1) / SUB;
 
     // the producer lane issues the first weight box at once; the rest of the
     // ring fills only after the compute threads have issued their loads
@@ -229,8 +265,8 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
     auto issue_box = [&](int c) {
         const int w = c % WS;
         mbar_arrive_expect_tx(&full[w], kWBox);
-        const int x = c < nbox0 ? (a0 + c * SUB) * RB : (c - nbox0) * SUB * RB;
-        const int y = (c < nbox0 ? t0 : t0 + 1) * 128;
+        const int x = c < nbox1 ? c * SUB * RB : (a0 + (c - nbox1) * SUB) * RB;
+        const int y = (c < nbox1 ? t0 + 1 : t0) * 128;
         tma_load_2d(sW + w * kWBox, &tmW, &full[w], x, y);
     };
     if (tid == kCompute) {
@@ -381,12 +417,12 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
                         // (128 + q) - (128 + z) = q - z exactly
                         word = pack_bf16x2_rn(128.0f + zf, 0.0f) & 0xFFFFu;
                     } else {
-                        // (128 + q) - 128 = q, and -z (fp16 bits) in the high half
-                        word = 0x4300u | (static_cast<uint32_t>(z16 ^ 0x8000u) << 16);
+                        // (128 + q) - 128 = q; the zero is added after the loop
+                        word = 0x4300u;
                         *s_far = 1;
                     }
-                    *reinterpret_cast<uint2*>(sTab + (rl * tstride + lg) * 8) =
-                        make_uint2(word, __float_as_uint(f16_bits_to_f32(s16)));
+                    *reinterpret_cast<uint32_t*>(sTab + (rl * tstride + lg) * 4) =
+                        word | (static_cast<uint32_t>(s16) << 16);
                 } else {
                     float am = __uint_as_float(raw[u]);
                     if (p.q8 != nullptr)
@@ -398,8 +434,9 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
             }
         }
         // row m: zeros, read by the lanes of tokens >= m
-        for (int e = tid; e < xstride / 2; e += kCompute)
-            reinterpret_cast<uint32_t*>(sX + p.m * xstride)[e] = 0u;
+        if (p.m < NTOK)
+            for (int e = tid; e < xstride / 2; e += kCompute)
+                reinterpret_cast<uint32_t*>(sX + p.m * xstride)[e] = 0u;
         if (KIND == kCode4) {
             for (int e = tid; e < 256; e += kCompute) {
                 // byte e = (first code << 4) | second code -> (codebook[first], codebook[second])
@@ -437,12 +474,13 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
     asm volatile("" : "+r"(mg));                       // keep the magic in a register
 
     uint32_t c = 0;                                    // weight boxes consumed (matches the producer)
-    int lk0 = 0;                                       // first local k-block of the segment
     // (after a timed-out wait every warp still runs both segments' barriers)
-    for (int sgi = 0; sgi < nseg; ++sgi) {
+    for (int si = 0; si < nseg; ++si) {
+        const int sgi = nseg - 1 - si;                 // segment 1 (if any) first, then segment 0
         const int tile = sgi == 0 ? t0 : t0 + 1;
         const int kb0 = sgi == 0 ? a0 : 0;
         const int nkb = sgi == 0 ? n0 : n1;
+        const int lk0 = sgi == 0 ? 0 : n0;             // first local k-block of the segment
         const int64_t gr0 = static_cast<int64_t>(tile) * 128 + rl0, gr1 = gr0 + 8;
         const bool ok0 = gr0 < p.n, ok1 = gr1 < p.n;
         // group partials in two chains (even and odd MMA steps), folded per group
@@ -482,15 +520,15 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
                     if (s % GB == 0) {
                         // this group's constants from the table
                         const uint32_t ta = trow + static_cast<uint32_t>(lk) / GB * TE;
+                        const uint32_t e0 = gemv_lds32(ta), e1 = gemv_lds32(ta + 8 * tstride * TE);
                         if (KIND != kCode4) {
-                            const uint2 e0 = gemv_lds64(ta), e1 = gemv_lds64(ta + 8 * tstride * TE);
-                            sub0 = __byte_perm(e0.x, 0u, 0x1010);
-                            sub1 = __byte_perm(e1.x, 0u, 0x1010);
-                            sf0 = __uint_as_float(e0.y);
-                            sf1 = __uint_as_float(e1.y);
+                            sub0 = __byte_perm(e0, 0u, 0x1010);
+                            sub1 = __byte_perm(e1, 0u, 0x1010);
+                            sf0 = f16_bits_to_f32(static_cast<uint16_t>(e0 >> 16));
+                            sf1 = f16_bits_to_f32(static_cast<uint16_t>(e1 >> 16));
                         } else {
-                            sf0 = __uint_as_float(gemv_lds32(ta));
-                            sf1 = __uint_as_float(gemv_lds32(ta + 8 * tstride * TE));
+                            sf0 = __uint_as_float(e0);
+                            sf1 = __uint_as_float(e1);
                         }
                     }
                     // A fragments: 8 code pairs of each row as bf16x2
@@ -568,12 +606,17 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
             // groups stored with |zero| > 128 ran as (q - 0); add their
             // scale * (-zero) * (sum of x over the group) here
             for (int lg = lk0 / GB; lg < (lk0 + nkb) / GB; ++lg) {
-                const uint32_t ta = trow + static_cast<uint32_t>(lg) * TE;
-                const uint2 e0 = gemv_lds64(ta), e1 = gemv_lds64(ta + 8 * tstride * TE);
-                const float z0 = f16_bits_to_f32(static_cast<uint16_t>(e0.x >> 16));
-                const float z1 = f16_bits_to_f32(static_cast<uint16_t>(e1.x >> 16));
-                if (z0 == 0.0f && z1 == 0.0f) continue;
-                const float k0 = __uint_as_float(e0.y) * z0, k1 = __uint_as_float(e1.y) * z1;
+                const int64_t gi = kb0 / GB + (lg - lk0 / GB);      // group within the row
+                float k0 = 0.0f, k1 = 0.0f;
+                if (ok0) {
+                    const float z = f16_bits_to_f32(__ldg(p.zero + gr0 * p.ngroups + gi));
+                    if (fabsf(z) > 128.0f) k0 = f16_bits_to_f32(__ldg(p.scale + gr0 * p.ngroups + gi)) * -z;
+                }
+                if (ok1) {
+                    const float z = f16_bits_to_f32(__ldg(p.zero + gr1 * p.ngroups + gi));
+                    if (fabsf(z) > 128.0f) k1 = f16_bits_to_f32(__ldg(p.scale + gr1 * p.ngroups + gi)) * -z;
+                }
+                if (k0 == 0.0f && k1 == 0.0f) continue;
 #pragma unroll
                 for (int nt = 0; nt < NT8; ++nt) {
                     const int tA = nt * 8 + 2 * j;
@@ -589,7 +632,6 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
                 }
             }
         }
-        lk0 += nkb;
         // -------------------------------------------------------------- segment epilogue
         auto lora = [&](int t, int oc) -> float {
             if (p.rank == 0) return 0.0f;
@@ -615,63 +657,71 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
                 }
             continue;
         }
-        // partial slot of (CTA b, tile t) is b + t: CTAs cover the work in
-        // order, so no two (CTA, tile) pairs share a slot
-        float* slot = p.partial + (static_cast<int64_t>(blockIdx.x) + tile) * p.m * 128;
+        // split tile.  Partial slot of (CTA b, tile t) is b + t: CTAs cover the
+        // work in order, so no two (CTA, tile) pairs share a slot.
+        const int cta_lo = static_cast<int>((static_cast<int64_t>(tile) * p.kbt) / p.share);
+        const int cta_hi = static_cast<int>((static_cast<int64_t>(tile + 1) * p.kbt - 1) / p.share);
+        if (kb0 + nkb < p.kbt) {
+            // contributor (the tile's last k-block belongs to a later CTA)
+            float* slot = p.partial + (static_cast<int64_t>(blockIdx.x) + tile) * p.m * 128;
+#pragma unroll
+            for (int nt = 0; nt < NT8; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int t = nt * 8 + 2 * j + (e & 1);
+                    if (t < p.m) slot[t * 128 + rl0 + ((e < 2) ? 0 : 8)] = acc[nt][e];
+                }
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (tid == 0) flag_publish(p.counters + tile);
+            continue;
+        }
+        // this CTA finishes the tile: wait for the cta_hi - cta_lo contributors
+        if (tid == 0) {
+            if (!flag_wait_geq(p.counters + tile, static_cast<uint32_t>(cta_hi - cta_lo))) *s_abort = 1;
+            p.counters[tile] = 0u;                     // left at zero for the next call
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        // the contributors' partials in CTA order (QB CTAs' loads in flight
+        // together), then this CTA's own sums
+        constexpr int QB = NT8 == 1 ? 8 : 2;
+        float v[NT8][4];
+#pragma unroll
+        for (int nt = 0; nt < NT8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[nt][e] = 0.0f;
+        for (int b0 = cta_lo; b0 < cta_hi; b0 += QB) {
+            float part[QB][NT8][4];
+#pragma unroll
+            for (int q = 0; q < QB; ++q)
+#pragma unroll
+                for (int nt = 0; nt < NT8; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int t = nt * 8 + 2 * j + (e & 1);
+                        part[q][nt][e] = (b0 + q < cta_hi && t < p.m)
+                                             ? __ldcg(p.partial + ((static_cast<int64_t>(b0 + q) + tile) * p.m + t) * 128 +
+                                                      rl0 + ((e < 2) ? 0 : 8))
+                                             : 0.0f;
+                    }
+#pragma unroll
+            for (int q = 0; q < QB; ++q)
+#pragma unroll
+                for (int nt = 0; nt < NT8; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) v[nt][e] += part[q][nt][e];
+        }
 #pragma unroll
         for (int nt = 0; nt < NT8; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int t = nt * 8 + 2 * j + (e & 1);
-                if (t < p.m) slot[t * 128 + rl0 + ((e < 2) ? 0 : 8)] = acc[nt][e];
-            }
-        __threadfence();
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        const int cta_lo = static_cast<int>((static_cast<int64_t>(tile) * p.kbt) / p.share);
-        const int cta_hi = static_cast<int>((static_cast<int64_t>(tile + 1) * p.kbt - 1) / p.share);
-        if (tid == 0) {
-            const uint32_t prev = atomicAdd(p.counters + tile, 1u);
-            const int last = (prev == static_cast<uint32_t>(cta_hi - cta_lo)) ? 1 : 0;
-            // the last contributor leaves the counter at zero for the next call
-            if (last) p.counters[tile] = 0u;
-            *s_last = last;
-        }
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        if (*s_last) {
-            __threadfence();
-            // sum the partials of every CTA that touched this tile, in CTA order,
-            // four rows per thread, all partials' loads in flight together
-            const float4* part4 = reinterpret_cast<const float4*>(p.partial);
-            for (int e = tid; e < 32 * p.m; e += kCompute) {
-                const int t = e >> 5, rq = (e & 31) * 4;
-                float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                for (int b0 = cta_lo; b0 <= cta_hi; b0 += 8) {
-                    float4 part[8];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        part[q] = (b0 + q <= cta_hi)
-                                      ? __ldcg(part4 + ((static_cast<int64_t>(b0 + q) + tile) * p.m + t) * 32 + (e & 31))
-                                      : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        v.x += part[q].x;
-                        v.y += part[q].y;
-                        v.z += part[q].z;
-                        v.w += part[q].w;
-                    }
-                }
-                const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int64_t r = static_cast<int64_t>(tile) * 128 + rq + q;
-                    if (r < p.n) {
-                        const int oc = p.perm ? p.perm[r] : static_cast<int>(r);
-                        p.Y[static_cast<int64_t>(t) * p.ldy + oc] = vv[q] + lora(t, oc);
-                    }
+                const bool ok = (e < 2) ? ok0 : ok1;
+                const int64_t r = (e < 2) ? gr0 : gr1;
+                if (ok && t < p.m) {
+                    const int oc = p.perm ? p.perm[r] : static_cast<int>(r);
+                    p.Y[static_cast<int64_t>(t) * p.ldy + oc] = (v[nt][e] + acc[nt][e]) + lora(t, oc);
                 }
             }
-        }
-        asm volatile("bar.sync 1, 256;" ::: "memory");
     }
 }
 

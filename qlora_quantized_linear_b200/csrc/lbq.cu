@@ -123,9 +123,9 @@ int token_tile(int m) { return m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <=
 
 // Split-K workspace layout, the same for every plan: a fixed header of
 // per-tile arrival counters at offset 0, then the fp32 partial sums.  The
-// last CTA of a tile sets its counter back to zero, so the header stays zero
-// between calls whatever shapes share the workspace (partials never land on
-// it).
+// CTA that finishes a tile sets its counter back to zero, so the header stays
+// zero between calls whatever shapes share the workspace (partials never land
+// on it).
 constexpr size_t kCounterHeader = 64 * 1024;
 constexpr int kMaxSplitTiles = static_cast<int>(kCounterHeader / sizeof(uint32_t));
 
@@ -137,6 +137,7 @@ struct Plan {
     int tiles;       // output tiles (rows x token tiles)
     int nsplit;      // K splits
     int per_split;   // reduction blocks per split
+    int stages = 4;  // decode GEMV: weight boxes in flight
     size_t partial_bytes;
     size_t workspace() const { return nsplit > 1 ? kCounterHeader + partial_bytes : 0; }
 };
@@ -178,15 +179,18 @@ bool weights_stable(cudaStream_t st) {
 // equal share of the (row tile, k-block) work, a whole number of scale
 // groups and as many k-blocks as its shared memory holds (weight ring,
 // activation slice, constant table) with two CTAs per SM, and the grid fills
-// whole waves of two CTAs per SM.
+// whole waves of two CTAs per SM.  The weight ring holds four boxes, or
+// three when that lets the whole grid run in one wave (wide token tiles,
+// whose activation slice takes most of the shared memory).
 constexpr int kGemvMaxM = 16;
 constexpr size_t kGemvSmemBudget = 113 * 1024;     // two CTAs per SM
 
-size_t gemv_smem_bytes(int m, int share, int kind) {
+size_t gemv_smem_bytes(int m, int share, int kind, int stages) {
     const int gb = kind == kInt4 ? 2 : 1;
-    const size_t entry = kind == kCode4 ? 4 : 8;
-    return 1024 + static_cast<size_t>(kGemvWStages) * 128 * 128 + static_cast<size_t>(m + 1) * (share * 64 + 4) * 2 +
-           static_cast<size_t>((share / gb) | 1) * 128 * entry + (kind == kCode4 ? 1024 : 0) + 2 * kGemvWStages * 8 + 16;
+    const int nt = m <= 8 ? 8 : 16;
+    const size_t xrows = static_cast<size_t>(m < nt ? m + 1 : m);      // + a zero row for padded lanes
+    return 1024 + static_cast<size_t>(stages) * 128 * 128 + xrows * (share * 64 + 4) * 2 +
+           static_cast<size_t>((share / gb) | 1) * 128 * 4 + (kind == kCode4 ? 1024 : 0) + 2 * stages * 8 + 16;
 }
 
 Plan plan_gemv(int m, const lbq_qweight* q, int sms) {
@@ -198,11 +202,24 @@ Plan plan_gemv(int m, const lbq_qweight* q, int sms) {
     pl.tiles = static_cast<int>(cdiv(q->n, 128));
     const int64_t total = static_cast<int64_t>(pl.tiles) * kbt;
     const int64_t slots = 2LL * sms;
-    int64_t smax = gb;
-    while (smax + gb <= kbt && (smax + gb) / gb <= kGemvMaxTabGroups &&
-           gemv_smem_bytes(m, static_cast<int>(smax + gb), kind) <= kGemvSmemBudget)
-        smax += gb;
-    const int64_t waves = cdiv(total, slots * smax);
+    auto max_share = [&](int stages) {
+        int64_t smax = gb;
+        while (smax + gb <= kbt && (smax + gb) / gb <= kGemvMaxTabGroups &&
+               gemv_smem_bytes(m, static_cast<int>(smax + gb), kind, stages) <= kGemvSmemBudget)
+            smax += gb;
+        return smax;
+    };
+    int64_t smax = max_share(kGemvMaxWStages);
+    int64_t waves = cdiv(total, slots * smax);
+    pl.stages = kGemvMaxWStages;
+    if (waves > 1) {
+        const int64_t smax3 = max_share(kGemvMaxWStages - 1);
+        if (cdiv(total, slots * smax3) < waves) {
+            smax = smax3;
+            waves = cdiv(total, slots * smax3);
+            pl.stages = kGemvMaxWStages - 1;
+        }
+    }
     int64_t share = cdiv(cdiv(total, waves * slots), gb) * gb;
     // at least an eighth of a row per CTA, so that the CTA finishing a tile
     // sums a handful of partials (small layers then use fewer CTAs)
@@ -214,10 +231,10 @@ Plan plan_gemv(int m, const lbq_qweight* q, int sms) {
     return pl;
 }
 
-template <int KIND, int NTOK>
+template <int KIND, int NTOK, int WS>
 lbq_status launch_gemv_kind(const GemvParams& p, const uint8_t* packed, int grid, cudaStream_t st) {
-    auto kern = dqgemv_kernel<KIND, NTOK>;
-    const size_t smem = gemv_smem_bytes(p.m, p.share, KIND);
+    auto kern = dqgemv_kernel<KIND, NTOK, WS>;
+    const size_t smem = gemv_smem_bytes(p.m, p.share, KIND, WS);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
         return LBQ_ECUDA;
     CUtensorMap tmW;
@@ -278,6 +295,23 @@ lbq_status launch_fwd_kind(int nt, const FwdParams& p, const void* X, int m, int
     }
 }
 
+template <int WS>
+lbq_status launch_gemv_tile(const GemvParams& p, const lbq_qweight* q, const Plan& pl, cudaStream_t st) {
+    if (WS != pl.stages) {
+        if constexpr (WS > kGemvMaxWStages - 1) return launch_gemv_tile<WS - 1>(p, q, pl, st);
+        return LBQ_EUNSUPPORTED;
+    }
+    const bool n8 = pl.nt == 8;
+    switch (kind_of(q)) {
+        case kInt4: return n8 ? launch_gemv_kind<kInt4, 8, WS>(p, q->packed, pl.nsplit, st)
+                              : launch_gemv_kind<kInt4, 16, WS>(p, q->packed, pl.nsplit, st);
+        case kInt2: return n8 ? launch_gemv_kind<kInt2, 8, WS>(p, q->packed, pl.nsplit, st)
+                              : launch_gemv_kind<kInt2, 16, WS>(p, q->packed, pl.nsplit, st);
+        default: return n8 ? launch_gemv_kind<kCode4, 8, WS>(p, q->packed, pl.nsplit, st)
+                           : launch_gemv_kind<kCode4, 16, WS>(p, q->packed, pl.nsplit, st);
+    }
+}
+
 // One fused dequantize-GEMM over one stored weight (or one half of a
 // channel-mix weight).  `perm` maps its stored rows to output columns.
 lbq_status run_gemv(const void* X, int m, const lbq_qweight* q, const void* B, int rank, float s, const float* T,
@@ -315,15 +349,7 @@ lbq_status run_gemv(const void* X, int m, const lbq_qweight* q, const void* B, i
         p.partial = ws_partials(ws);
         p.counters = ws_counters(ws);
     }
-    const bool n8 = pl.nt == 8;
-    switch (kind_of(q)) {
-        case kInt4: return n8 ? launch_gemv_kind<kInt4, 8>(p, q->packed, pl.nsplit, st)
-                              : launch_gemv_kind<kInt4, 16>(p, q->packed, pl.nsplit, st);
-        case kInt2: return n8 ? launch_gemv_kind<kInt2, 8>(p, q->packed, pl.nsplit, st)
-                              : launch_gemv_kind<kInt2, 16>(p, q->packed, pl.nsplit, st);
-        default: return n8 ? launch_gemv_kind<kCode4, 8>(p, q->packed, pl.nsplit, st)
-                           : launch_gemv_kind<kCode4, 16>(p, q->packed, pl.nsplit, st);
-    }
+    return launch_gemv_tile<4>(p, q, pl, st);
 }
 
 lbq_status run_fwd_gemm(const void* X, int m, const lbq_qweight* q, const void* B, int rank, float s,
