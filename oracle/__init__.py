@@ -67,6 +67,7 @@ def _declare(L) -> None:
                                                     _vp, _vp, _int, _dbl, _i64, _vp, _vp, _vp, _vp]),
         "oracle_linear_bwd_sampled_minmax": (_int, [_vp, _i64, _vp, _vp, _vp, _i64, _i64, _int, _int,
                                                     _vp, _vp, _int, _dbl, _i64, _vp, _vp, _vp, _vp]),
+        "oracle_lora_merge": (_int, [_vp, _i64, _i64, _vp, _vp, _int, ctypes.c_float, _int, _vp]),
         "oracle_set_threads": (None, [_int]),
         "oracle_get_threads": (_int, []),
     }
@@ -288,3 +289,19 @@ def linear_bwd_sampled_minmax(dY, packed, scale, zero, n: int, k: int, bits: int
         _p(dY), m, _p(packed), _p(scale), _p(zero), n, k, bits, group, _p(A), _p(B), r, float(s),
         rows.shape[0], _p(rows), _p(cols), _p(dX), _p(dXb)), "linear_bwd_sampled_minmax")
     return dX, dXb
+
+
+# ---------------------------------------------------------------- adapter merge
+def lora_merge(W_in, A, B, s: float, sign: int = 1) -> np.ndarray:
+    """bf16 bits [n, k] of W_in + sign * s * (B A), evaluated as oracle.h
+    states (fp32 fma over the rank in order, then * s, then +/-, then bf16).
+    W_in: fp32 [n, k] (a dequantized weight, or a bf16 weight widened)."""
+    W_in = np.ascontiguousarray(W_in, dtype=np.float32)
+    n, k = W_in.shape
+    r = 0 if A is None else A.shape[0]
+    A = None if A is None else _u16(A)
+    B = None if B is None else _u16(B)
+    out = np.zeros((n, k), np.uint16)
+    _check(lib().oracle_lora_merge(_p(W_in), n, k, _p(A), _p(B), r, ctypes.c_float(float(s)), int(sign), _p(out)),
+           "lora_merge")
+    return out

@@ -552,3 +552,40 @@ int oracle_linear_bwd_sampled_minmax(const uint16_t* dY, int64_t m,
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Merging the adapter into the weight                                       */
+/* [GB] introduction: after QLoRA fine-tuning the LoRA module is merged into */
+/* the full-precision model.  The merged weight is W_hat + s B A; removing   */
+/* the adapter again subtracts the same product.                             */
+/* ------------------------------------------------------------------------ */
+
+/* binary32 -> bf16, round to nearest, ties to even: keep the upper 16 bits
+ * and round up when the dropped half is above one half ulp, or exactly one
+ * half with an odd kept part (a carry into the exponent is the correct
+ * result).  NaN stays a quiet NaN. */
+static uint16_t f32_to_bf16_rne(float x) {
+    uint32_t u;
+    memcpy(&u, &x, 4);
+    if (isnan(x)) return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t hi = u >> 16, lo = u & 0xFFFFu;
+    if (lo > 0x8000u || (lo == 0x8000u && (hi & 1u))) hi += 1u;
+    return (uint16_t)hi;
+}
+
+int oracle_lora_merge(const float* W_in, int64_t n, int64_t k,
+                      const uint16_t* A, const uint16_t* B, int r, float s,
+                      int sign, uint16_t* W_out) {
+    if (r < 0 || (r > 0 && (!A || !B)) || !(sign == 1 || sign == -1)) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t row = 0; row < n; ++row)
+        for (int64_t col = 0; col < k; ++col) {
+            float d = 0.0f;
+            for (int u = 0; u < r; ++u)
+                d = fmaf(oracle_bf16_to_f32(B[row * r + u]), oracle_bf16_to_f32(A[(int64_t)u * k + col]), d);
+            float t = s * d;
+            float v = (sign > 0) ? W_in[row * k + col] + t : W_in[row * k + col] - t;
+            W_out[row * k + col] = f32_to_bf16_rne(v);
+        }
+    return 0;
+}

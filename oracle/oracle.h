@@ -134,6 +134,22 @@ int  oracle_linear_bwd_sampled_minmax(const uint16_t* dY, int64_t m,
                                       const int64_t* rows, const int64_t* cols,
                                       double* dX, double* dXbound);
 
+/* --- merging an adapter into the weight ([GB] introduction) ------------ */
+/* After fine-tuning, the low-rank module is merged into the full-precision
+ * weight.  W_in fp32 [n, k] (the dequantized weight for a merge, a bf16
+ * weight widened to fp32 for an unmerge), A bf16 [r, k], B bf16 [n, r],
+ * sign +1 (merge) or -1 (unmerge).  Every output element is evaluated in
+ * binary32 steps in this order (the pages fix no precision; this order is the
+ * definition, so that re-quantizing a merged weight is reproducible):
+ *   d = 0;  d = fma(B[i,u], A[u,j], d)  for u = 0 .. r-1
+ *   t = s * d
+ *   v = W_in[i,j] + t   (merge)   or   W_in[i,j] - t   (unmerge)
+ *   W_out[i,j] = bf16 round-to-nearest-even of v
+ * r may be 0 (A, B ignored).  W_out: bf16 bits [n, k]. */
+int  oracle_lora_merge(const float* W_in, int64_t n, int64_t k,
+                       const uint16_t* A, const uint16_t* B, int r, float s,
+                       int sign, uint16_t* W_out);
+
 /* Threads used by the loops over rows (OpenMP); 0 keeps the default. */
 void oracle_set_threads(int nthreads);
 int  oracle_get_threads(void);

@@ -37,6 +37,13 @@ MUTANTS = {
                              "double w = W_hat[(c % n) * k + j % k];\n                acc += g * w;"),
     "dA_uses_T": ("acc += U[i * r + t] * x;", "acc += T[i * r + t] * x;"),
     "dB_missing_s": ("if (dB) dB[j * r + t] = s * acc;", "if (dB) dB[j * r + t] = acc;"),
+    "merge_missing_s": ("float t = s * d;", "float t = d;"),
+    "merge_sign_ignored": ("float v = (sign > 0) ? W_in[row * k + col] + t : W_in[row * k + col] - t;",
+                           "float v = W_in[row * k + col] + t;"),
+    "merge_A_transposed": ("oracle_bf16_to_f32(A[(int64_t)u * k + col])", "oracle_bf16_to_f32(A[col * r + u])"),
+    "merge_truncates": ("if (lo > 0x8000u || (lo == 0x8000u && (hi & 1u))) hi += 1u;", "(void)lo;"),
+    "merge_ties_away": ("if (lo > 0x8000u || (lo == 0x8000u && (hi & 1u))) hi += 1u;", "if (lo >= 0x8000u) hi += 1u;"),
+    "merge_reordered_sum": ("for (int u = 0; u < r; ++u)\n                d = fmaf(", "for (int u = r - 1; u >= 0; --u)\n                d = fmaf("),
 }
 
 

@@ -421,3 +421,82 @@ def test_backward_products_by_exact_finite_differences():
     # U = dY B (shared by dX and dA)
     np.testing.assert_allclose(U, oracle.bf16_to_f32(dY).astype(np.float64)
                                @ oracle.bf16_to_f32(B).astype(np.float64), rtol=1e-12, atol=1e-18)
+
+
+# --------------------------------------------------------------------------
+# merging the adapter into the weight (GreenBit article, introduction: the
+# LoRA module is merged into the full-precision model after fine-tuning)
+# --------------------------------------------------------------------------
+def _bits(t: torch.Tensor) -> np.ndarray:
+    return syn.bits_u16(t.to(torch.bfloat16))
+
+
+def _as_f32(bits: np.ndarray) -> np.ndarray:
+    return oracle.bf16_to_f32(bits).astype(np.float32)
+
+
+def test_merge_hand_built():
+    # W = [1, 1], B = [[2]], A = [[0.5, -1]], s = 3: B A = [1, -2], s B A = [3, -6]
+    W = np.array([[1.0, 1.0]], np.float32)
+    A = _bits(torch.tensor([[0.5, -1.0]]))
+    B = _bits(torch.tensor([[2.0]]))
+    assert _as_f32(oracle.lora_merge(W, A, B, 3.0, 1)).tolist() == [[4.0, -5.0]]
+    assert _as_f32(oracle.lora_merge(W, A, B, 3.0, -1)).tolist() == [[-2.0, 7.0]]
+
+
+def test_merge_rank0_is_bf16_rounding_of_the_weight():
+    # no adapter: the merged weight is the weight rounded to bf16 (torch's
+    # fp32 -> bf16 conversion rounds to nearest even), ties included
+    rng = np.random.default_rng(11)
+    W = (rng.standard_normal((64, 96)) * 0.02).astype(np.float32)
+    W[0, :6] = [1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(1.0 + 2.0 ** -8), 2.0 ** -130, 0.0, 65504.0]
+    got = oracle.lora_merge(W, None, None, 2.0, 1)
+    assert np.array_equal(got, _bf16(W))
+    assert _as_f32(got[:1, :3]).tolist() == [[1.0, 1.0 + 2.0 ** -6, -1.0]]
+    # the one difference from plain rounding: -0 + (s * 0) is +0 in IEEE arithmetic
+    assert oracle.lora_merge(np.array([[-0.0]], np.float32), None, None, 2.0, 1).tolist() == [[0]]
+
+
+def test_merge_matches_fp64_product_within_rounding():
+    # against numpy's fp64 matmul: a dropped s, a wrong sign or a transposed
+    # operand would be off by far more than the binary32 and bf16 roundings
+    rng = np.random.default_rng(12)
+    n, k, r, s = 48, 80, 16, 2.0
+    W = (rng.standard_normal((n, k)) * 0.02).astype(np.float32)
+    A = _bits(torch.from_numpy(rng.standard_normal((r, k)).astype(np.float32) * 0.05))
+    B = _bits(torch.from_numpy(rng.standard_normal((n, r)).astype(np.float32) * 0.05))
+    Af, Bf = _as_f32(A).astype(np.float64), _as_f32(B).astype(np.float64)
+    for sign in (1, -1):
+        got = _as_f32(oracle.lora_merge(W, A, B, s, sign)).astype(np.float64)
+        exact = W.astype(np.float64) + sign * s * (Bf @ Af)
+        mag = np.abs(W) + abs(s) * (np.abs(Bf) @ np.abs(Af))
+        lim = np.abs(exact) * 2.0 ** -8 + (r + 3) * 2.0 ** -24 * mag
+        assert np.all(np.abs(got - exact) <= lim)
+        # and the adapter term really is there (not the rank-0 result)
+        assert np.mean(got != _as_f32(_bf16(W))) > 0.5
+
+
+def test_merge_accumulates_the_rank_in_order():
+    # products 1, 2^-30, -1 summed in binary32 in order: (1 + 2^-30) rounds to
+    # 1, so d = 0; an exact or reordered sum would leave 2^-30
+    W = np.zeros((1, 1), np.float32)
+    A = _bits(torch.tensor([[1.0], [2.0 ** -15], [1.0]]))
+    B = _bits(torch.tensor([[1.0, 2.0 ** -15, -1.0]]))
+    assert _as_f32(oracle.lora_merge(W, A, B, 1.0, 1)).tolist() == [[0.0]]
+    # the same products in the order 1, -1, 2^-30 keep the small one
+    A2 = _bits(torch.tensor([[1.0], [1.0], [2.0 ** -15]]))
+    B2 = _bits(torch.tensor([[1.0, -1.0, 2.0 ** -15]]))
+    assert _as_f32(oracle.lora_merge(W, A2, B2, 1.0, 1)).tolist() == [[2.0 ** -30]]
+
+
+def test_unmerge_inverts_an_exact_merge():
+    # small integers and a power-of-two scale: no step rounds, so removing the
+    # adapter gives the weight back bit for bit
+    rng = np.random.default_rng(13)
+    n, k, r = 16, 32, 4
+    W = rng.integers(-8, 8, (n, k)).astype(np.float32)
+    A = _bits(torch.from_numpy(rng.integers(-3, 4, (r, k)).astype(np.float32)))
+    B = _bits(torch.from_numpy(rng.integers(-3, 4, (n, r)).astype(np.float32)))
+    merged = oracle.lora_merge(W, A, B, 0.5, 1)
+    back = oracle.lora_merge(_as_f32(merged), A, B, 0.5, -1)
+    assert np.array_equal(_as_f32(back), W)
