@@ -532,6 +532,34 @@ def row_quantize8b(lbq, syn, torch, peaks, stream):
     return out
 
 
+def row_merge8b(lbq, syn, torch, peaks, stream):
+    """Merging a rank-16 adapter into each 8B MLP matrix (INT4 g128 -> bf16),
+    then re-quantizing the merged weight; algorithmic bytes: packed weight and
+    constants + A + B read, bf16 written (merge); bf16 read, packed weight and
+    constants written (re-quantize)."""
+    out = {}
+    r = 16
+    for i, name in enumerate(("gate", "down")):
+        n, k = syn.LLAMA3_8B_SHAPES[name]
+        W = syn.weight_bf16(n, k, 0.02, seed=1500 + i, outlier_frac=0.001, device="cuda")
+        qw = lbq.QuantizedWeight(n, k, "minmax", 4).quantize(W, stream=stream)
+        A = syn.normal_bf16((r, k), 0.01, seed=1510 + i, device="cuda")
+        B = syn.normal_bf16((n, r), 0.01, seed=1520 + i, device="cuda")
+        merged = torch.empty((n, k), dtype=torch.bfloat16, device="cuda")
+        q2 = lbq.QuantizedWeight(n, k, "minmax", 4)
+        ms_m = time_graph(torch, lambda: lbq.merge_lora(qw, A, B, 2.0, out=merged, stream=stream), stream, reps=10)
+        ms_q = time_graph(torch, lambda: q2.quantize(merged, stream=stream), stream, reps=10)
+        packed = n * k // 2 + 4 * (n * k // 128)
+        b_m = packed + 2 * r * (n + k) + 2 * n * k
+        b_q = 2 * n * k + packed
+        out[f"{name} {n}x{k}"] = {"merge_us": round(1e3 * ms_m, 1), "merge_GB/s": round(b_m / ms_m / 1e6, 1),
+                                  "merge_frac_hbm": round(b_m / ms_m / 1e6 / peaks["hbm_gbs"], 3),
+                                  "requantize_us": round(1e3 * ms_q, 1),
+                                  "requantize_GB/s": round(b_q / ms_q / 1e6, 1)}
+        del W, qw, A, B, merged, q2
+    return out
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 def oracle_sample(rows: int, threads: int = 0):
     """The oracle's forward on `rows` output rows of the gate matrix (K = 4096)
@@ -686,7 +714,8 @@ def main():
         del wl
         torch.cuda.empty_cache()
         for key, fn in (("train_8b_mlp_M4096_r16", row_training), ("codebook_70b_dq", row_codebook70b),
-                        ("mixed_8b", row_mixed), ("quantize_8b_int4", row_quantize8b)):
+                        ("mixed_8b", row_mixed), ("quantize_8b_int4", row_quantize8b),
+                        ("merge_8b_r16", row_merge8b)):
             try:
                 rows[key] = fn(lbq, syn, torch, peaks, stream)
             except Exception as e:  # report, do not hide, a failing row

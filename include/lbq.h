@@ -142,6 +142,34 @@ lbq_status lbq_dequantize(const lbq_qweight* q, float* W_f32,
                           lbq_stream_t stream);
 
 /*
+ * Merge the low-rank adapter into the weight (GreenBit article,
+ * introduction: after QLoRA fine-tuning the LoRA module is merged into the
+ * full-precision model):
+ *   W_out[i, j] = bf16( W_hat[i, j] + s * sum_u B[i, u] A[u, j] )
+ * W_hat is q dequantized exactly as lbq_dequantize does; A bf16 [rank, k] and
+ * B bf16 [q->n, rank] row-major; W_out bf16 [q->n, q->k] row-major.  All
+ * device pointers, caller-owned, 16-byte aligned.  Each element is evaluated
+ * in binary32 in this order: d = 0, then d = fma(B[i,u], A[u,j], d) for
+ * u = 0 .. rank-1; t = s * d; v = W_hat + t; W_out = v rounded to bf16
+ * (nearest, ties to even).  The order is part of the contract: the merged
+ * weight, and lbq_quantize of it (re-quantizing the merged model), are
+ * reproducible bit for bit.  rank == 0 (A, B may be NULL) writes bf16(W_hat).
+ * 0 <= rank <= 64.  Returns LBQ_EINVAL / LBQ_EALIGN on bad arguments before
+ * any launch.
+ */
+lbq_status lbq_merge_lora(const lbq_qweight* q, const void* A, const void* B,
+                          int rank, float s, void* W_out, lbq_stream_t stream);
+
+/*
+ * Remove a merged adapter: W_out = bf16(W - s * B A) for a bf16 weight W
+ * [n, k] (device, row-major), with the same binary32 order as lbq_merge_lora
+ * and v = W - t.  k must be a multiple of 8; W_out may be W (in place).
+ */
+lbq_status lbq_unmerge_lora(const void* W, int n, int k, const void* A,
+                            const void* B, int rank, float s, void* W_out,
+                            lbq_stream_t stream);
+
+/*
  * Forward of the quantized linear layer with a low-rank adapter (QLoRA
  * explainer, QLoRA技术原理):
  *   T = X A^T  [m, rank]                         (fp32, written to T_save)

@@ -8,6 +8,7 @@
 #include "dqgemm_bwd.cuh"
 #include "dqgemv.cuh"
 #include "lora.cuh"
+#include "merge.cuh"
 #include "quantize.cuh"
 
 using namespace lbq;
@@ -622,6 +623,63 @@ lbq_status lbq_dequantize(const lbq_qweight* q, float* W_f32, lbq_stream_t strea
         codebook_dequantize_kernel<<<grid, 256, 0, s>>>(q->packed, q->absmax, q->double_quant ? q->absmax_q8 : nullptr,
                                                         q->absmax_s2, q->absmax_offset, q->codebook, nchunks, out);
     }
+    return last_launch();
+}
+
+lbq_status lbq_merge_lora(const lbq_qweight* q, const void* A, const void* B, int rank, float s, void* W_out,
+                          lbq_stream_t stream) {
+    lbq_status st = check_qweight(q, true);
+    if (st != LBQ_OK) return st;
+    if (!W_out || rank < 0 || rank > kLoraMaxRank || (rank > 0 && (!A || !B))) return LBQ_EINVAL;
+    if (!aligned16(W_out) || (rank > 0 && (!aligned16(A) || !aligned16(B)))) return LBQ_EALIGN;
+    MergeParams p{};
+    p.n = q->n;
+    p.k = q->k;
+    p.ngroups = q->scheme == LBQ_MINMAX_ASYM ? q->k / q->group : 0;
+    p.packed = q->packed;
+    p.scale = q->scale;
+    p.zero = q->zero;
+    p.absmax = q->absmax;
+    p.q8 = (q->scheme == LBQ_CODEBOOK4 && q->double_quant) ? q->absmax_q8 : nullptr;
+    p.s2 = q->absmax_s2;
+    p.offset = q->absmax_offset;
+    p.codebook = q->codebook;
+    p.A = static_cast<const uint16_t*>(A);
+    p.B = static_cast<const uint16_t*>(B);
+    p.rank = rank;
+    p.s = s;
+    p.out = static_cast<uint16_t*>(W_out);
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    const dim3 grid(static_cast<unsigned>(cdiv(q->k, kMergeCols)), static_cast<unsigned>(cdiv(q->n, kMergeRows)));
+    if (grid.y > 65535u) return LBQ_EUNSUPPORTED;
+    if (q->scheme == LBQ_MINMAX_ASYM) {
+        if (q->bits == 4)
+            lora_merge_kernel<kMergeInt4><<<grid, kMergeThreads, 0, cs>>>(p);
+        else
+            lora_merge_kernel<kMergeInt2><<<grid, kMergeThreads, 0, cs>>>(p);
+    } else {
+        lora_merge_kernel<kMergeCode4><<<grid, kMergeThreads, 0, cs>>>(p);
+    }
+    return last_launch();
+}
+
+lbq_status lbq_unmerge_lora(const void* W, int n, int k, const void* A, const void* B, int rank, float s, void* W_out,
+                            lbq_stream_t stream) {
+    if (!W || !W_out || n < 1 || k < 8 || k % 8 != 0) return LBQ_EINVAL;
+    if (rank < 0 || rank > kLoraMaxRank || (rank > 0 && (!A || !B))) return LBQ_EINVAL;
+    if (!aligned16(W) || !aligned16(W_out) || (rank > 0 && (!aligned16(A) || !aligned16(B)))) return LBQ_EALIGN;
+    MergeParams p{};
+    p.n = n;
+    p.k = k;
+    p.W = static_cast<const uint16_t*>(W);
+    p.A = static_cast<const uint16_t*>(A);
+    p.B = static_cast<const uint16_t*>(B);
+    p.rank = rank;
+    p.s = s;
+    p.out = static_cast<uint16_t*>(W_out);
+    const dim3 grid(static_cast<unsigned>(cdiv(k, kMergeCols)), static_cast<unsigned>(cdiv(n, kMergeRows)));
+    if (grid.y > 65535u) return LBQ_EUNSUPPORTED;
+    lora_merge_kernel<kMergeBf16><<<grid, kMergeThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
     return last_launch();
 }
 

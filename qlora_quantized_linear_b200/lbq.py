@@ -63,6 +63,8 @@ _SIGS = {
     "lbq_linear_bwd": (_int, [_vp, _int, _QP, _vp, _vp, _int, _f32, _vp, _vp, _vp, _sz, _vp]),
     "lbq_lora_grads": (_int, [_vp, _vp, _int, _int, _int, _vp, _vp, _int, _f32, _vp, _vp, _vp]),
     "lbq_device_status": (_int, [_u32p]),
+    "lbq_merge_lora": (_int, [_QP, _vp, _vp, _int, _f32, _vp, _vp]),
+    "lbq_unmerge_lora": (_int, [_vp, _int, _int, _vp, _vp, _int, _f32, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_L, _name)
@@ -89,6 +91,8 @@ lbq_linear_bwd_workspace_size = _L.lbq_linear_bwd_workspace_size
 lbq_linear_bwd = _L.lbq_linear_bwd
 lbq_lora_grads = _L.lbq_lora_grads
 lbq_device_status = _L.lbq_device_status
+lbq_merge_lora = _L.lbq_merge_lora
+lbq_unmerge_lora = _L.lbq_unmerge_lora
 
 
 class LbqError(RuntimeError):
@@ -260,6 +264,34 @@ def lora_grads(X, dY, T, U, s: float, dA=None, dB=None, stream=None):
     _check(lbq_lora_grads(X.data_ptr(), dY.data_ptr(), m, n, k, T.data_ptr(), U.data_ptr(), rank, float(s),
                           dA.data_ptr(), dB.data_ptr(), _stream(stream)), "lbq_lora_grads")
     return dA, dB
+
+
+def merge_lora(qw, A=None, B=None, s: float = 0.0, out=None, stream=None):
+    """bf16 [n, k]: the dequantized weight plus s B A (the adapter merged in)."""
+    torch = _torch()
+    rank = 0 if A is None else int(A.shape[0])
+    if rank:
+        A, B = _bf16_2d(A, "A"), _bf16_2d(B, "B")
+    if out is None:
+        out = torch.empty((qw.n, qw.k), dtype=torch.bfloat16, device=qw.packed.device)
+    _check(lbq_merge_lora(ctypes.byref(qw.struct), _ptr(A) if rank else None, _ptr(B) if rank else None, rank,
+                          float(s), out.data_ptr(), _stream(stream)), "lbq_merge_lora")
+    return out
+
+
+def unmerge_lora(W, A=None, B=None, s: float = 0.0, out=None, stream=None):
+    """bf16 [n, k]: W minus s B A (a merged adapter removed); out may be W."""
+    torch = _torch()
+    W = _bf16_2d(W, "W")
+    n, k = W.shape
+    rank = 0 if A is None else int(A.shape[0])
+    if rank:
+        A, B = _bf16_2d(A, "A"), _bf16_2d(B, "B")
+    if out is None:
+        out = torch.empty_like(W)
+    _check(lbq_unmerge_lora(W.data_ptr(), n, k, _ptr(A) if rank else None, _ptr(B) if rank else None, rank,
+                            float(s), out.data_ptr(), _stream(stream)), "lbq_unmerge_lora")
+    return out
 
 
 def device_status() -> int:

@@ -74,3 +74,17 @@ def test_workspace_queries_are_host_only():
     assert lbq.lbq_quantize_workspace_size(ctypes.byref(q)) == 0
     cb = _qw(scheme=lbq.LBQ_CODEBOOK4, group=64, double_quant=1)
     assert lbq.lbq_quantize_workspace_size(ctypes.byref(cb)) > 0
+
+
+def test_merge_entry_points_reject_bad_arguments():
+    q = _qw()
+    merge, unmerge = lbq.lbq_merge_lora, lbq.lbq_unmerge_lora
+    assert merge(None, None, None, 0, 1.0, 0x5000, None) == lbq.LBQ_EINVAL
+    assert merge(ctypes.byref(q), None, None, 0, 1.0, None, None) == lbq.LBQ_EINVAL
+    assert merge(ctypes.byref(q), None, None, 8, 1.0, 0x5000, None) == lbq.LBQ_EINVAL      # rank > 0 needs A, B
+    assert merge(ctypes.byref(q), 0x6000, 0x7000, 65, 1.0, 0x5000, None) == lbq.LBQ_EINVAL  # rank above 64
+    assert merge(ctypes.byref(q), 0x6000, 0x7000, 8, 1.0, 0x5004, None) == lbq.LBQ_EALIGN
+    assert merge(ctypes.byref(q), 0x6008, 0x7000, 8, 1.0, 0x5000, None) == lbq.LBQ_EALIGN
+    assert unmerge(0x4000, 16, 12, None, None, 0, 1.0, 0x5000, None) == lbq.LBQ_EINVAL     # k % 8 != 0
+    assert unmerge(0x4000, 0, 16, None, None, 0, 1.0, 0x5000, None) == lbq.LBQ_EINVAL
+    assert unmerge(0x4002, 16, 16, None, None, 0, 1.0, 0x5000, None) == lbq.LBQ_EALIGN

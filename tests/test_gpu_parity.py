@@ -419,3 +419,112 @@ def test_codebook70b_prefill_full_size_sampled(lbq, codebook70b):
         bound[i:i + 1024] = np.einsum("ij,ij->i", np.abs(xr), np.abs(wc))
     assert_within(Y.cpu().numpy()[rows, cols], ref, bound, "Y")
     assert_status_clean(lbq)
+
+
+# --------------------------------------------------------------------------- adapter merge
+MERGE_CASES = [
+    # n, k, rank, scheme, bits, dq
+    (256, 512, 16, "minmax", 4, False),
+    (200, 640, 8, "minmax", 2, False),      # ragged rows (200 = 3 x 64 + 8)
+    (130, 1024, 64, "minmax", 4, False),    # rank 64: two staged chunks of the adapter
+    (96, 448, 40, "codebook", 4, True),     # codebook + double quant; rank 40 = 32 + 8; k = 3.5 column tiles
+    (64, 192, 5, "codebook", 4, False),
+    (128, 256, 0, "minmax", 4, False),      # no adapter: bf16 of the dequantized weight
+]
+
+
+def _merge_inputs(n, k, rank, seed):
+    A = syn.normal_bf16((rank, k), 0.05, seed + 2) if rank else None
+    B = syn.normal_bf16((n, rank), 0.05, seed + 3) if rank else None
+    return A, B
+
+
+@pytest.mark.parametrize("n,k,rank,scheme,bits,dq", MERGE_CASES)
+def test_merge_bit_exact(lbq, n, k, rank, scheme, bits, dq):
+    seed = n + k + rank
+    cb = syn.codebook_normal16() if scheme == "codebook" else None
+    W = mixed_weight(n, k, seed) if scheme == "minmax" else syn.weight_bf16(n, k, 0.015, seed)
+    qw = device_qweight(lbq, W, scheme, bits, dq, cb)
+    A, B = _merge_inputs(n, k, rank, seed)
+    s = 2.0
+    out = lbq.merge_lora(qw, A.cuda() if rank else None, B.cuda() if rank else None, s)
+    torch.cuda.synchronize()
+    ref = oracle.lora_merge(oracle_weight(W, scheme, bits, dq, cb), syn.bits_u16(A) if rank else None,
+                            syn.bits_u16(B) if rank else None, s, 1)
+    assert np.array_equal(u16(out), ref)
+    assert_status_clean(lbq)
+
+
+def test_merge_sums_the_rank_in_order(lbq):
+    # products 1, 2^-30, -1 in every element: summed in order they cancel to
+    # exactly 0, so the merged weight is bf16(W_hat) itself
+    n, k = 64, 128
+    W = mixed_weight(n, k, 3)
+    qw = device_qweight(lbq, W, "minmax", 4, False, None)
+    A = torch.tensor([[1.0], [2.0 ** -15], [1.0]]).repeat(1, k).to(torch.bfloat16)
+    B = torch.tensor([[1.0, 2.0 ** -15, -1.0]]).repeat(n, 1).to(torch.bfloat16)
+    out = lbq.merge_lora(qw, A.cuda(), B.cuda(), 1.0)
+    torch.cuda.synchronize()
+    What = oracle_weight(W, "minmax", 4, False, None)
+    ref = oracle.lora_merge(What, syn.bits_u16(A), syn.bits_u16(B), 1.0, 1)
+    assert np.array_equal(u16(out), ref)
+    assert np.array_equal(ref, oracle.lora_merge(What, None, None, 1.0, 1))
+
+
+@pytest.mark.parametrize("n,k,rank", [(192, 512, 16), (100, 200, 7)])
+def test_unmerge_bit_exact_in_place(lbq, n, k, rank):
+    W = syn.weight_bf16(n, k, 0.02, seed=n + k)
+    A, B = _merge_inputs(n, k, rank, n)
+    ref = oracle.lora_merge(oracle.bf16_to_f32(syn.bits_u16(W)).astype(np.float32), syn.bits_u16(A),
+                            syn.bits_u16(B), 1.5, -1)
+    Wd = W.cuda()
+    out = lbq.unmerge_lora(Wd, A.cuda(), B.cuda(), 1.5)
+    lbq.unmerge_lora(Wd, A.cuda(), B.cuda(), 1.5, out=Wd)
+    torch.cuda.synchronize()
+    assert np.array_equal(u16(out), ref)
+    assert np.array_equal(u16(Wd), ref)
+    assert_status_clean(lbq)
+
+
+@pytest.mark.parametrize("scheme,bits,dq", [("minmax", 4, False), ("minmax", 2, False), ("codebook", 4, True)])
+def test_merge_then_requantize_bit_exact(lbq, scheme, bits, dq):
+    # re-quantizing the merged model: the merged bf16 weight goes through the
+    # GPU quantizer and must give the oracle's codes and constants exactly
+    n, k, rank, s = 256, 1024, 16, 2.0
+    cb = syn.codebook_normal16() if scheme == "codebook" else None
+    W = syn.weight_bf16(n, k, 0.02, seed=77, outlier_frac=0.01)
+    qw = device_qweight(lbq, W, scheme, bits, dq, cb)
+    A, B = _merge_inputs(n, k, rank, 77)
+    merged = lbq.merge_lora(qw, A.cuda(), B.cuda(), s)
+    q2 = lbq.QuantizedWeight(n, k, scheme, bits, double_quant=dq, codebook=cb).quantize(merged)
+    torch.cuda.synchronize()
+    mref = oracle.lora_merge(oracle_weight(W, scheme, bits, dq, cb), syn.bits_u16(A), syn.bits_u16(B), s, 1)
+    if scheme == "minmax":
+        codes, scale, zero = oracle.minmax_quantize(mref, bits, 128 if bits == 4 else 64)
+        assert np.array_equal(q2.packed.cpu().numpy(), oracle.pack(codes, bits))
+        assert np.array_equal(u16(q2.scale), scale)
+        assert np.array_equal(u16(q2.zero), zero)
+    else:
+        codes, absmax = oracle.codebook_quantize(mref, cb)
+        q8, s2, off, exact = oracle.double_quant(absmax)
+        assert exact
+        assert np.array_equal(q2.packed.cpu().numpy(), oracle.pack(codes, 4))
+        assert np.array_equal(q2.q8.cpu().numpy(), q8)
+        assert np.array_equal(q2.s2.cpu().numpy().view(np.uint32), s2.view(np.uint32))
+    assert_status_clean(lbq)
+
+
+def test_merge_full_size_gate(lbq, train_problem):
+    # the 8B MLP gate matrix (14336 x 4096, INT4 g128) with its rank-16
+    # adapter, every element against the oracle
+    P = train_problem
+    qw = lbq.QuantizedWeight(P["n"], P["k"], "minmax", 4)
+    qw.packed.copy_(torch.from_numpy(P["packed"]))
+    qw.scale.copy_(torch.from_numpy(P["scale"].view(np.float16)))
+    qw.zero.copy_(torch.from_numpy(P["zero"].view(np.float16)))
+    out = lbq.merge_lora(qw, P["A"].cuda(), P["B"].cuda(), P["s"])
+    torch.cuda.synchronize()
+    What = oracle.minmax_dequantize(P["packed"], P["scale"], P["zero"], P["k"], 4, 128)
+    ref = oracle.lora_merge(What, syn.bits_u16(P["A"]), syn.bits_u16(P["B"]), P["s"], 1)
+    assert np.array_equal(u16(out), ref)
+    assert_status_clean(lbq)
