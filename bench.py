@@ -66,10 +66,15 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+# The sources that decide what the decode GEMV kernel does and how it is
+# launched: the kernel, the headers it includes and its host-side plan.
+GEMV_SOURCES = ("common.cuh", "dqgemm.cuh", "dqgemv.cuh", "dqgemv_host.cuh")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "qlora_quantized_linear_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in GEMV_SOURCES:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]

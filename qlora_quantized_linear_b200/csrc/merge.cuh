@@ -11,10 +11,12 @@
 // reproducible bit for bit.
 //
 // Bound by HBM (the bf16 output is 2 bytes per weight against 0.5 read for
-// INT4; the adapter stays in L2): a CTA owns a 64-row x 128-column tile, each
-// thread 8 rows x 4 consecutive columns.  The 32 partial sums stay in
-// registers; the adapter is staged in shared memory as fp32 in rank chunks of
-// 32, one 16-byte load of A and two broadcast loads of B feeding 32 FMAs.
+// INT4; the adapter stays in L2).  A CTA owns a 64-row x 128-column tile, a
+// thread 8 rows x 4 consecutive columns, with the 32 partial sums in
+// registers.  The thread's weight words go out first; meanwhile the adapter
+// is staged in shared memory as fp32 (A as 16-byte loads along the columns, B
+// as 16-byte loads along each row when the rank is a multiple of 8), so that
+// one 16-byte load of A and two broadcast loads of B feed 16 paired FMAs.
 #pragma once
 
 #include "quantize.cuh"
@@ -49,10 +51,55 @@ struct MergeParams {
 
 __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) { return pack_bf16x2_rn(lo, hi); }
 
-// MODE: the source of the weight (kMerge*); unmerge reads a bf16 weight and
+// (d0, d1) = fma((a0, a1), (b, b), (d0, d1)): two IEEE fused multiply-adds in
+// one instruction, each rounded once exactly as fmaf
+__device__ __forceinline__ void fma_x2(float& d0, float& d1, float a0, float a1, float b) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\tmov.b64 rd, {%0, %1};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rd;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a0), "f"(a1), "f"(b));
+}
+
+// The weight inputs of one thread for one row tile (loaded a tile ahead).
+struct MergeIn {
+    uint32_t raw[8];              // packed codes of the 8 rows (or bf16 pairs x)
+    uint32_t raw2[8];             // bf16 pairs y (removal)
+    uint32_t aux[8];              // MinMax: fp16 zero | fp16 scale << 16; codebook: fp32 absmax bits
+};
+
+template <int MODE>
+__device__ __forceinline__ void merge_load(const MergeParams& p, int64_t row0, int col0, MergeIn& in) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int64_t row = row0 + i;
+        in.raw[i] = in.raw2[i] = in.aux[i] = 0u;
+        if (row >= p.n || col0 >= p.k) continue;
+        const int64_t e0 = row * p.k + col0;                  // first element
+        if (MODE == kMergeInt4 || MODE == kMergeCode4) {
+            in.raw[i] = __ldg(reinterpret_cast<const uint16_t*>(p.packed) + e0 / 4);
+        } else if (MODE == kMergeInt2) {
+            in.raw[i] = __ldg(p.packed + e0 / 4);
+        } else {
+            const uint2 w = __ldg(reinterpret_cast<const uint2*>(p.W + e0));
+            in.raw[i] = w.x;
+            in.raw2[i] = w.y;
+        }
+        if (MODE == kMergeInt4 || MODE == kMergeInt2) {
+            const int64_t g = row * p.ngroups + col0 / (p.k / p.ngroups);
+            in.aux[i] = static_cast<uint32_t>(__ldg(p.zero + g)) | (static_cast<uint32_t>(__ldg(p.scale + g)) << 16);
+        } else if (MODE == kMergeCode4) {
+            const int64_t b = e0 / 64;
+            in.aux[i] = __float_as_uint((p.q8 != nullptr) ? double_dequant(p.q8[b], p.s2[b >> 8], *p.offset)
+                                                          : __ldg(p.absmax + b));
+        }
+    }
+}
+
+// MODE: the source of the weight (kMerge*); a removal reads a bf16 weight and
 // subtracts, every other mode dequantizes and adds.
 template <int MODE>
-__global__ void __launch_bounds__(kMergeThreads) lora_merge_kernel(const MergeParams p) {
+__global__ void __launch_bounds__(kMergeThreads, 3) lora_merge_kernel(const MergeParams p) {
     __shared__ __align__(16) float sA[kMergeRankChunk][kMergeCols];     // 16 KB
     __shared__ __align__(16) float sB[kMergeRankChunk][kMergeRows];     // 8 KB
     __shared__ float s_cb[16];
@@ -64,6 +111,10 @@ __global__ void __launch_bounds__(kMergeThreads) lora_merge_kernel(const MergePa
     const int64_t row0 = tile_row + warp * 8;                 // and 8 rows
     if (MODE == kMergeCode4 && tid < 16) s_cb[tid] = p.codebook[tid];
 
+    // the weight words of the thread's 8 rows go out first
+    MergeIn in;
+    merge_load<MODE>(p, row0, col0, in);
+
     float d[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
@@ -72,7 +123,7 @@ __global__ void __launch_bounds__(kMergeThreads) lora_merge_kernel(const MergePa
 
     for (int u0 = 0; u0 < p.rank; u0 += kMergeRankChunk) {
         const int ur = min(kMergeRankChunk, p.rank - u0);
-        __syncthreads();                                      // the previous chunk is consumed
+        if (u0 > 0) __syncthreads();                          // the previous chunk is consumed
         // A[u0 + u][tile columns] as fp32, 8 columns (16 bytes of bf16) per step
         for (int e = tid; e < ur * (kMergeCols / 8); e += kMergeThreads) {
             const int u = e / (kMergeCols / 8), c8 = e - u * (kMergeCols / 8);
@@ -85,61 +136,44 @@ __global__ void __launch_bounds__(kMergeThreads) lora_merge_kernel(const MergePa
             dst[1] = make_float4(bf16_bits_to_f32(v.z & 0xFFFFu), bf16_bits_to_f32(v.z >> 16),
                                  bf16_bits_to_f32(v.w & 0xFFFFu), bf16_bits_to_f32(v.w >> 16));
         }
-        // B[tile rows][u0 + u], transposed to [u][row] (consecutive lanes take
-        // consecutive rows, so the shared stores do not conflict)
-        for (int e = tid; e < ur * kMergeRows; e += kMergeThreads) {
-            const int u = e / kMergeRows, rr = e - u * kMergeRows;
-            const int64_t row = tile_row + rr;
-            sB[u][rr] = row < p.n ? bf16_bits_to_f32(__ldg(p.B + row * p.rank + u0 + u)) : 0.0f;
+        // B[tile rows][u0 + u] transposed to [u][row]
+        if ((p.rank & 7) == 0) {
+            // 8 rank terms of one row (16 bytes) per step: rows are contiguous in B
+            const int pieces = ur / 8;
+            for (int e = tid; e < kMergeRows * pieces; e += kMergeThreads) {
+                const int rr = e / pieces, pc = e - rr * pieces;
+                const int64_t row = tile_row + rr;
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (row < p.n) v = __ldg(reinterpret_cast<const uint4*>(p.B + row * p.rank + u0 + pc * 8));
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    sB[pc * 8 + 2 * h][rr] = bf16_bits_to_f32(w4[h] & 0xFFFFu);
+                    sB[pc * 8 + 2 * h + 1][rr] = bf16_bits_to_f32(w4[h] >> 16);
+                }
+            }
+        } else {
+            for (int e = tid; e < ur * kMergeRows; e += kMergeThreads) {
+                const int u = e / kMergeRows, rr = e - u * kMergeRows;
+                const int64_t row = tile_row + rr;
+                sB[u][rr] = row < p.n ? bf16_bits_to_f32(__ldg(p.B + row * p.rank + u0 + u)) : 0.0f;
+            }
         }
         __syncthreads();
         for (int u = 0; u < ur; ++u) {
             const float4 a = *reinterpret_cast<const float4*>(&sA[u][lane * 4]);
             const float4 b0 = *reinterpret_cast<const float4*>(&sB[u][warp * 8]);
             const float4 b1 = *reinterpret_cast<const float4*>(&sB[u][warp * 8 + 4]);
-            const float av[4] = {a.x, a.y, a.z, a.w};
             const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) d[i][c] = fmaf(bv[i], av[c], d[i][c]);
+            for (int i = 0; i < 8; ++i) {
+                fma_x2(d[i][0], d[i][1], a.x, a.y, bv[i]);
+                fma_x2(d[i][2], d[i][3], a.z, a.w, bv[i]);
+            }
         }
     }
-    if (MODE == kMergeCode4 && p.rank == 0) __syncthreads();  // the codebook copy (else done by the chunk barriers)
+    if (MODE == kMergeCode4 && p.rank == 0) __syncthreads();  // the codebook copy (else done by the chunk barrier)
     if (col0 >= p.k) return;                                  // k % 8 == 0: a thread's 4 columns are all in or out
-
-    // the weight: all eight rows' loads first, then the arithmetic
-    uint32_t raw[8];
-    float amax[8], zf[8], sf[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int64_t row = row0 + i;
-        raw[i] = 0u;
-        amax[i] = zf[i] = sf[i] = 0.0f;
-        if (row >= p.n) continue;
-        const int64_t e0 = row * p.k + col0;                  // first element
-        if (MODE == kMergeInt4 || MODE == kMergeCode4) {
-            raw[i] = __ldg(reinterpret_cast<const uint16_t*>(p.packed) + e0 / 4);
-        } else if (MODE == kMergeInt2) {
-            raw[i] = __ldg(p.packed + e0 / 4);
-        }
-        if (MODE == kMergeInt4 || MODE == kMergeInt2) {
-            const int64_t g = row * p.ngroups + col0 / (p.k / p.ngroups);
-            zf[i] = f16_bits_to_f32(__ldg(p.zero + g));
-            sf[i] = f16_bits_to_f32(__ldg(p.scale + g));
-        } else if (MODE == kMergeCode4) {
-            const int64_t b = e0 / 64;
-            amax[i] = (p.q8 != nullptr) ? double_dequant(p.q8[b], p.s2[b >> 8], *p.offset) : __ldg(p.absmax + b);
-        }
-    }
-    uint2 wb[8];
-    if (MODE == kMergeBf16) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int64_t row = row0 + i;
-            wb[i] = row < p.n ? __ldg(reinterpret_cast<const uint2*>(p.W + row * p.k + col0)) : make_uint2(0u, 0u);
-        }
-    }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int64_t row = row0 + i;
@@ -147,20 +181,25 @@ __global__ void __launch_bounds__(kMergeThreads) lora_merge_kernel(const MergePa
         float w[4];
         if (MODE == kMergeInt4 || MODE == kMergeCode4) {
             // bytes (c0 << 4 | c1), (c2 << 4 | c3): the first code in the high nibble
-            const uint32_t q[4] = {(raw[i] >> 4) & 15u, raw[i] & 15u, (raw[i] >> 12) & 15u, (raw[i] >> 8) & 15u};
+            const uint32_t r = in.raw[i];
+            const uint32_t q[4] = {(r >> 4) & 15u, r & 15u, (r >> 12) & 15u, (r >> 8) & 15u};
+            const float zf = f16_bits_to_f32(static_cast<uint16_t>(in.aux[i] & 0xFFFFu));
+            const float sf = f16_bits_to_f32(static_cast<uint16_t>(in.aux[i] >> 16));
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-                w[c] = (MODE == kMergeInt4) ? __fmul_rn(__fsub_rn(static_cast<float>(q[c]), zf[i]), sf[i])
-                                            : __fmul_rn(s_cb[q[c]], amax[i]);
+                w[c] = (MODE == kMergeInt4) ? __fmul_rn(__fsub_rn(static_cast<float>(q[c]), zf), sf)
+                                            : __fmul_rn(s_cb[q[c]], __uint_as_float(in.aux[i]));
         } else if (MODE == kMergeInt2) {
+            const float zf = f16_bits_to_f32(static_cast<uint16_t>(in.aux[i] & 0xFFFFu));
+            const float sf = f16_bits_to_f32(static_cast<uint16_t>(in.aux[i] >> 16));
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-                w[c] = __fmul_rn(__fsub_rn(static_cast<float>((raw[i] >> (6 - 2 * c)) & 3u), zf[i]), sf[i]);
+                w[c] = __fmul_rn(__fsub_rn(static_cast<float>((in.raw[i] >> (6 - 2 * c)) & 3u), zf), sf);
         } else {
-            w[0] = bf16_bits_to_f32(wb[i].x & 0xFFFFu);
-            w[1] = bf16_bits_to_f32(wb[i].x >> 16);
-            w[2] = bf16_bits_to_f32(wb[i].y & 0xFFFFu);
-            w[3] = bf16_bits_to_f32(wb[i].y >> 16);
+            w[0] = bf16_bits_to_f32(in.raw[i] & 0xFFFFu);
+            w[1] = bf16_bits_to_f32(in.raw[i] >> 16);
+            w[2] = bf16_bits_to_f32(in.raw2[i] & 0xFFFFu);
+            w[3] = bf16_bits_to_f32(in.raw2[i] >> 16);
         }
         float v[4];
 #pragma unroll
