@@ -186,6 +186,7 @@ FWD_CASES = [
     (8, 4096, 4096, 8, "minmax", 2, False),
     (12, 2000, 3200, 0, "codebook", 4, True),   # ragged n
     (16, 4096, 14336, 16, "minmax", 4, False),
+    (16, 14336, 4096, 16, "minmax", 4, False),  # three-box ring; shares span two row tiles
 ]
 
 
@@ -399,6 +400,18 @@ def test_codebook70b_decode_full_size(lbq, codebook70b):
     torch.cuda.synchronize()
     Yr, _, Yb = oracle.linear_fwd(syn.bits_u16(X), C["What"])
     assert_within(Y.cpu().numpy(), Yr, Yb, "Y")
+
+
+def test_codebook70b_decode_m16_full_size(lbq, codebook70b):
+    # 16 tokens: the grid takes two waves, so tile owners also wait on
+    # contributors of the earlier wave
+    C = codebook70b
+    X = syn.normal_bf16((16, C["k"]), 1.0, seed=74)
+    Y, _ = lbq.linear_fwd(X.cuda(), C["qw"])
+    torch.cuda.synchronize()
+    Yr, _, Yb = oracle.linear_fwd(syn.bits_u16(X), C["What"])
+    assert_within(Y.cpu().numpy(), Yr, Yb, "Y")
+    assert_status_clean(lbq)
 
 
 def test_codebook70b_prefill_full_size_sampled(lbq, codebook70b):
