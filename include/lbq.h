@@ -197,6 +197,19 @@ lbq_status lbq_unmerge_lora(const void* W, int n, int k, const void* A,
  * stream in between).
  */
 size_t lbq_linear_fwd_workspace_size(int m, const lbq_qweight* q, int rank);
+
+/*
+ * The decode plan that lbq_linear_fwd uses for 1 <= m <= 16 (host only: no
+ * device work, no GPU needed).  The units are (128-row tile, 64-column
+ * k-block) pairs, row tiles x k/64 of them, cut into equal contiguous CTA
+ * shares; a share spans at most two row tiles.  On success plan[0..5] =
+ * CTAs, k-blocks per CTA, row tiles, weight-ring boxes of 16 KB, dynamic
+ * shared memory per CTA in bytes, and the SM count the plan was made for
+ * (`sms`; when sms <= 0, the current device's, or 148 without one).
+ * Only n, k, bits, group and scheme of q are read.  Returns LBQ_EINVAL for m
+ * outside 1..16, a NULL plan or an invalid q.
+ */
+lbq_status lbq_gemv_plan(int m, const lbq_qweight* q, int sms, int64_t* plan);
 lbq_status lbq_linear_fwd(const void* X, int m, const lbq_qweight* q,
                           const void* A, const void* B, int rank, float s,
                           float* Y, float* T_save, void* workspace,

@@ -556,6 +556,19 @@ size_t lbq_linear_fwd_workspace_size(int m, const lbq_qweight* q, int rank) {
     return plan_fwd(m, q, sm_count()).workspace();
 }
 
+lbq_status lbq_gemv_plan(int m, const lbq_qweight* q, int sms, int64_t* plan) {
+    if (m < 1 || m > kGemvMaxM || !plan || check_qweight(q, false) != LBQ_OK) return LBQ_EINVAL;
+    if (sms <= 0) sms = sm_count();
+    const Plan pl = plan_gemv(m, q, sms);
+    plan[0] = pl.nsplit;
+    plan[1] = pl.per_split;
+    plan[2] = pl.tiles;
+    plan[3] = pl.stages;
+    plan[4] = static_cast<int64_t>(gemv_smem_bytes(m, pl.per_split, kind_of(q), pl.stages));
+    plan[5] = sms;
+    return LBQ_OK;
+}
+
 lbq_status lbq_linear_fwd(const void* X, int m, const lbq_qweight* q, const void* A, const void* B, int rank,
                           float s, float* Y, float* T_save, void* workspace, size_t workspace_bytes,
                           lbq_stream_t stream) {

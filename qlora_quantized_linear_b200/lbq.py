@@ -64,6 +64,7 @@ _SIGS = {
     "lbq_lora_grads": (_int, [_vp, _vp, _int, _int, _int, _vp, _vp, _int, _f32, _vp, _vp, _vp]),
     "lbq_device_status": (_int, [_u32p]),
     "lbq_merge_lora": (_int, [_QP, _vp, _vp, _int, _f32, _vp, _vp]),
+    "lbq_gemv_plan": (_int, [_int, _QP, _int, ctypes.POINTER(ctypes.c_int64)]),
     "lbq_unmerge_lora": (_int, [_vp, _int, _int, _vp, _vp, _int, _f32, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -92,6 +93,7 @@ lbq_linear_bwd = _L.lbq_linear_bwd
 lbq_lora_grads = _L.lbq_lora_grads
 lbq_device_status = _L.lbq_device_status
 lbq_merge_lora = _L.lbq_merge_lora
+lbq_gemv_plan = _L.lbq_gemv_plan
 lbq_unmerge_lora = _L.lbq_unmerge_lora
 
 
