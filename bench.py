@@ -351,17 +351,18 @@ def run_decode(args, dist, lbq, syn, torch, peaks):
     del probes
 
     # end to end through the public API: pinned host X in, Y out, every call
-    e2e = run_decode_e2e(args, wl, lbq, torch, stream)
+    e2e = run_decode_e2e(args, dist, wl, lbq, torch, stream)
     del graphs
     return wl, value, ms_max, clocks, roofline, per_matrix, e2e
 
 
-def run_decode_e2e(args, wl, lbq, torch, stream):
+def run_decode_e2e(args, dist, wl, lbq, torch, stream):
     """The decode step end to end through the C ABI: every step copies that
     step's activations from pinned host memory to the device (one copy of the
     four distinct X of the layer set), makes the 14 lbq_linear_fwd calls, and
     reads all 14 outputs back to pinned host memory (one copy).  Wall clock
-    from the host, synchronised at both ends."""
+    from the host, synchronised at both ends, between barriers; with several
+    ranks, the units of all ranks over the slowest rank's time."""
     import ctypes
     xkeys = sorted(wl.X)                                      # (m, k): the distinct activations
     ykeys = [(m, name) for m in DECODE_M for name in wl.shapes]
@@ -409,15 +410,19 @@ def run_decode_e2e(args, wl, lbq, torch, stream):
     for i in range(3):
         one_step(i)
     torch.cuda.synchronize()
+    dist.barrier()
     t0 = time.perf_counter()
     for i in range(steps):
         one_step(i)
     stream.synchronize()
     dt = time.perf_counter() - t0
-    return {"value": round(steps * wl.step_bytes / dt / 1e9, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+    dist.barrier()
+    dt_max = dist.max(dt)
+    return {"value": round(replica_value(steps * wl.step_bytes, dist.world, 1e3 * dt_max), 1), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps,
-            "note": "lbq_linear_fwd through the C ABI for the 14 calls of a step; per step one pinned host->device "
-                    "copy of the four distinct activations and one device->host copy of the 14 outputs"}
+            "note": "lbq_linear_fwd through the C ABI for the 14 calls of a step; per step and rank one pinned "
+                    "host->device copy of the four distinct activations and one device->host copy of the 14 outputs"}
 
 
 # ----------------------------------------------------------------------------- extra rows
