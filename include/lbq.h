@@ -7,6 +7,8 @@
  *  - GreenBit.AI article "只需单卡RTX 3090，低比特量化训练就能实现LLaMA-3 8B全参微调",
  *    section 模型量化, step (1): group-wise MinMax quantizer; INT4 with group
  *    size 128 and INT2 with group size 64; layer-mix and channel-mix layouts.
+ *    Its introduction: after QLoRA fine-tuning the low-rank module is merged
+ *    into the full-precision model (lbq_merge_lora, lbq_unmerge_lora).
  *  - bitsandbytes FSDP-QLoRA guide, section 量化数据的存储 (quant_storage):
  *    two 4-bit codes per byte with the first code in the high nibble; NF4/FP4
  *    codebooks; nested quantization of absmax; weights are dequantized to the
