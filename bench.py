@@ -49,8 +49,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", default=None,
                     help="run one kernel configuration `reps` times and exit (for ncu captures): "
-                         "decode_<matrix>_m<M> | train_<matrix>_{fwd,bwd,grads} | codebook70b_<matrix>_m<M> | "
-                         "quantize_<matrix>")
+                         "decode_<matrix>_m<M> | layerset_8b_m<M> | train_<matrix>_{fwd,bwd,grads} | "
+                         "codebook70b_<matrix>_m<M> | quantize_<matrix>")
     ap.add_argument("--reps", type=int, default=3)
     return ap.parse_args()
 
@@ -210,7 +210,12 @@ def gemm_flops(m, n, k, rank=0):
 
 # ----------------------------------------------------------------------------- the decode workload
 class Decode8B:
+    """The decode step: the seven layers at M = 1 and at M = 16, each size one
+    grouped forward call (one launch of the decode GEMV over the seven
+    weights), each size on its own rotating weight copy."""
+
     def __init__(self, lbq, syn, torch):
+        import ctypes
         self.lbq, self.torch = lbq, torch
         self.shapes = syn.LLAMA3_8B_SHAPES
         dev = "cuda"
@@ -226,42 +231,62 @@ class Decode8B:
                   for k in {kk for (_, kk) in self.shapes.values()}}
         self.Y = {(m, name): torch.empty((m, n), dtype=torch.float32, device=dev)
                   for m in DECODE_M for name, (n, _) in self.shapes.items()}
-        self.ws = {(m, name): lbq._workspace(self._ws_size(m, self.qw[0][name]), dev)
-                   for m in DECODE_M for name in self.shapes}
-        self.calls_per_step = len(DECODE_M) * len(self.shapes)
+        self.calls_per_step = len(DECODE_M)                  # grouped launches per step
         self.step_bytes = sum(gemm_bytes(m, n, k) for m in DECODE_M for (n, k) in self.shapes.values())
+        # the C arguments of every (size, copy): one lbq_fwd_problem array each
+        self.problems = {}
+        for m in DECODE_M:
+            for c in range(COPIES):
+                arr = (lbq.lbq_fwd_problem * len(self.shapes))()
+                for i, (name, (n, k)) in enumerate(self.shapes.items()):
+                    arr[i] = lbq.lbq_fwd_problem(X=self.X[(m, k)].data_ptr(), q=ctypes.pointer(self.qw[c][name].struct),
+                                                 A=None, B=None, rank=0, s=0.0, Y=self.Y[(m, name)].data_ptr(),
+                                                 T_save=None)
+                self.problems[(m, c)] = arr
+        self.ws_bytes = max(lbq.lbq_linear_fwd_grouped_workspace_size(m, self.problems[(m, 0)], len(self.shapes))
+                            for m in DECODE_M)
+        self.ws = lbq._workspace(self.ws_bytes, dev)
+        self.ws_single = {(m, name): lbq._workspace(self._ws_size(m, self.qw[0][name]), dev)
+                          for m in DECODE_M for name in self.shapes}
         torch.cuda.synchronize()
 
     def _ws_size(self, m, q):
         import ctypes
         return self.lbq.lbq_linear_fwd_workspace_size(m, ctypes.byref(q.struct), 0)
 
+    def call_group(self, m, copy, stream_handle):
+        rc = self.lbq.lbq_linear_fwd_grouped(m, self.problems[(m, copy)], len(self.shapes), self.ws.data_ptr(),
+                                             self.ws_bytes, stream_handle)
+        if rc != 0:
+            raise RuntimeError(f"lbq_linear_fwd_grouped returned {rc}")
+
     def call(self, m, name, copy, stream=None):
         k = self.shapes[name][1]
-        self.lbq.linear_fwd(self.X[(m, k)], self.qw[copy][name], Y=self.Y[(m, name)], workspace=self.ws[(m, name)],
-                            stream=stream)
+        self.lbq.linear_fwd(self.X[(m, k)], self.qw[copy][name], Y=self.Y[(m, name)],
+                            workspace=self.ws_single[(m, name)], stream=stream)
 
     def capture(self, phase: int, stream, probe: bool = False):
-        """CUDA graph of one step: both decode sizes over the layer set, each
-        size on its own weight copy.  The timed graphs hold the 14 calls back
-        to back (each call may overlap the tail of the one before it); the
-        probe graphs put timing events around every call, which serialises
-        them, to give the per-call durations."""
+        """CUDA graph of one step: both decode sizes, each one grouped launch
+        over the layer set on its own weight copy (back to back; each may
+        overlap the tail of the one before it).  The probe graphs instead make
+        the 14 per-matrix calls with timing events around every call, which
+        serialises them, to give per-matrix durations."""
         torch = self.torch
         g = torch.cuda.CUDAGraph()
         evs = []
         with torch.cuda.graph(g, stream=stream):
             for j, m in enumerate(DECODE_M):
                 copy = (2 * phase + j) % COPIES
-                for name, (n, k) in self.shapes.items():
-                    if probe:
-                        e0 = torch.cuda.Event(enable_timing=True, external=True)
-                        e1 = torch.cuda.Event(enable_timing=True, external=True)
-                        e0.record()
+                if not probe:
+                    self.call_group(m, copy, stream.cuda_stream)
+                    continue
+                for name in self.shapes:
+                    e0 = torch.cuda.Event(enable_timing=True, external=True)
+                    e1 = torch.cuda.Event(enable_timing=True, external=True)
+                    e0.record()
                     self.call(m, name, copy)
-                    if probe:
-                        e1.record()
-                        evs.append((m, name, e0, e1))
+                    e1.record()
+                    evs.append((m, name, e0, e1))
         return g, evs
 
 
@@ -272,6 +297,7 @@ def run_decode(args, dist, lbq, syn, torch, peaks):
     with torch.cuda.stream(stream):
         for c in range(2):
             for m in DECODE_M:
+                wl.call_group(m, c, stream.cuda_stream)
                 for name in wl.shapes:
                     wl.call(m, name, c)
     torch.cuda.synchronize()
@@ -318,23 +344,35 @@ def run_decode(args, dist, lbq, syn, torch, peaks):
     ms_max = dist.max(ms)
     value = replica_value(args.steps * wl.step_bytes, dist.world, ms_max)
 
-    # The timed region launches nothing but the dominant kernel (the decode
-    # GEMV), back to back: its average launch duration is the region's
-    # device time over the launches in it.
+    # The timed region launches nothing but the dominant kernel (the grouped
+    # decode GEMV, one launch per decode size), back to back: its average
+    # launch duration is the region's device time over the launches in it.
     launches = args.steps * wl.calls_per_step
     avg_launch_ms = ms / launches
     per_launch_bytes = wl.step_bytes / wl.calls_per_step
     achieved = per_launch_bytes / (avg_launch_ms / 1e3) / 1e9
     traffic = profiled_traffic("dqgemv_decode_8b")
-    roofline = {"kernel": "dqgemv_kernel (decode stream-K GEMV, all 14 calls of the step)", "bound": "hbm",
-                "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+    roofline = {"kernel": "dqgemv_grouped_kernel (one launch per decode size over the 7-matrix layer set)",
+                "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4), "peak_source": peaks["source"], "traffic": traffic,
                 "per_launch_bytes_avg": int(per_launch_bytes), "avg_launch_us": round(1e3 * avg_launch_ms, 3),
                 "launches_timed": launches}
 
-    # per-call durations, from probe graphs with an event pair around every
-    # call (the events keep consecutive calls from overlapping), after the
-    # timed region
+    # per-size launch durations (one grouped launch between events) and
+    # per-matrix durations (single calls between events), after the timed region
+    per_size = {}
+    for m in DECODE_M:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 50
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for r in range(reps):
+                wl.call_group(m, r % COPIES, stream.cuda_stream)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        us = 1e3 * e0.elapsed_time(e1) / reps
+        b = sum(gemm_bytes(m, n, k) for (n, k) in wl.shapes.values())
+        per_size[f"M{m}"] = {"us": round(us, 2), "GB/s": round(b / us / 1e3, 1)}
     probes = [wl.capture(ph, stream, probe=True) for ph in range(COPIES)]
     with torch.cuda.stream(stream):
         for _ in range(2):
@@ -348,6 +386,7 @@ def run_decode(args, dist, lbq, syn, torch, peaks):
     per_matrix = {f"M{m}/{name}": {"us": round(1e3 * statistics.median(v), 2),
                                      "GB/s": round(gemm_bytes(m, *wl.shapes[name]) / (statistics.median(v) / 1e3) / 1e9, 1)}
                   for (m, name), v in per.items()}
+    per_matrix["grouped_launch"] = per_size
     del probes
 
     # end to end through the public API: pinned host X in, Y out, every call
@@ -359,7 +398,8 @@ def run_decode(args, dist, lbq, syn, torch, peaks):
 def run_decode_e2e(args, dist, wl, lbq, torch, stream):
     """The decode step end to end through the C ABI: every step copies that
     step's activations from pinned host memory to the device (one copy of the
-    four distinct X of the layer set), makes the 14 lbq_linear_fwd calls, and
+    four distinct X of the layer set), makes the two grouped forward calls
+    (seven layers each), and
     reads all 14 outputs back to pinned host memory (one copy).  Wall clock
     from the host, synchronised at both ends, between barriers; with several
     ranks, the units of all ranks over the slowest rank's time."""
@@ -381,19 +421,20 @@ def run_decode_e2e(args, dist, wl, lbq, torch, stream):
     for key in ykeys:
         yview[key] = yd[off:off + yn[key]]
         off += yn[key]
-    fwd = lbq.lbq_linear_fwd
+    import ctypes
     sh = stream.cuda_stream
-    calls = []                                                # the C arguments of every call of a step phase
+    calls = []                                                # one grouped call per decode size and copy
     for phase in range(COPIES):
         row = []
         for j, m in enumerate(DECODE_M):
             copy = (2 * phase + j) % COPIES
-            for name, (n, k) in wl.shapes.items():
-                ws = wl.ws[(m, name)]
-                row.append((xview[(m, k)].data_ptr(), m, ctypes.byref(wl.qw[copy][name].struct), None, None, 0, 0.0,
-                            yview[(m, name)].data_ptr(), None, None if ws is None else ws.data_ptr(),
-                            0 if ws is None else ws.numel() * ws.element_size(), sh))
+            arr = (lbq.lbq_fwd_problem * len(wl.shapes))()
+            for i, (name, (n, k)) in enumerate(wl.shapes.items()):
+                arr[i] = lbq.lbq_fwd_problem(X=xview[(m, k)].data_ptr(), q=ctypes.pointer(wl.qw[copy][name].struct),
+                                             A=None, B=None, rank=0, s=0.0, Y=yview[(m, name)].data_ptr(), T_save=None)
+            row.append((m, arr, len(wl.shapes), wl.ws.data_ptr(), wl.ws_bytes, sh))
         calls.append(row)
+    fwd = lbq.lbq_linear_fwd_grouped
     h2d = xh.numel() * xh.element_size()
     d2h = yh.numel() * yh.element_size()
     steps = max(3, min(args.steps, 50))
@@ -404,7 +445,7 @@ def run_decode_e2e(args, dist, wl, lbq, torch, stream):
             for a in calls[i % COPIES]:
                 rc = fwd(*a)
                 if rc != 0:
-                    raise RuntimeError(f"lbq_linear_fwd returned {rc}")
+                    raise RuntimeError(f"lbq_linear_fwd_grouped returned {rc}")
             yh.copy_(yd, non_blocking=True)
 
     for i in range(3):
@@ -421,8 +462,9 @@ def run_decode_e2e(args, dist, wl, lbq, torch, stream):
     return {"value": round(replica_value(steps * wl.step_bytes, dist.world, 1e3 * dt_max), 1), "unit": "GB/s",
             "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps,
-            "note": "lbq_linear_fwd through the C ABI for the 14 calls of a step; per step and rank one pinned "
-                    "host->device copy of the four distinct activations and one device->host copy of the 14 outputs"}
+            "note": "lbq_linear_fwd_grouped through the C ABI, one call per decode size (7 layers each); per step "
+                    "and rank one pinned host->device copy of the four distinct activations and one device->host "
+                    "copy of the 14 outputs"}
 
 
 # ----------------------------------------------------------------------------- extra rows
@@ -536,18 +578,33 @@ def row_mixed(lbq, syn, torch, peaks, stream):
         lo = lbq.QuantizedWeight(n - n4, k, "minmax", 2).quantize(Wp[n4:].contiguous())
         mixw[name] = lbq.ChannelMixWeight(hi, lo, perm)
         del W, Wp
+    import ctypes
     for m in (16, 512):
         Xs = {k: syn.normal_bf16((m, k), 1.0, seed=1300 + k, device="cuda") for k in (4096, 14336)}
         Ys = {name: torch.empty((m, n), dtype=torch.float32, device="cuda") for name, (n, _) in shapes.items()}
-        for label, fn_weight, bytes_of in (
-                ("layer_mix", lambda nm: layer[nm],
+        # layer-mix: the seven layers in one grouped call (one launch at M = 16)
+        probs = (lbq.lbq_fwd_problem * len(shapes))()
+        for i, (nm, (n, k)) in enumerate(shapes.items()):
+            probs[i] = lbq.lbq_fwd_problem(X=Xs[k].data_ptr(), q=ctypes.pointer(layer[nm].struct), A=None, B=None,
+                                           rank=0, s=0.0, Y=Ys[nm].data_ptr(), T_save=None)
+        gws_bytes = lbq.lbq_linear_fwd_grouped_workspace_size(m, probs, len(shapes))
+        gws = lbq._workspace(gws_bytes, "cuda")
+
+        def layer_mix_step():
+            rc = lbq.lbq_linear_fwd_grouped(m, probs, len(shapes), None if gws is None else gws.data_ptr(), gws_bytes,
+                                            stream.cuda_stream)
+            if rc != 0:
+                raise RuntimeError(f"lbq_linear_fwd_grouped returned {rc}")
+
+        def channel_mix_step():
+            for nm, (n, k) in shapes.items():
+                lbq.linear_fwd(Xs[k], mixw[nm], Y=Ys[nm], stream=stream)
+        for label, step, bytes_of in (
+                ("layer_mix", layer_mix_step,
                  lambda nm, n, k: gemm_bytes(m, n, k, bits=bits[nm], group=128 if bits[nm] == 4 else 64)),
-                ("channel_mix", lambda nm: mixw[nm],
+                ("channel_mix", channel_mix_step,
                  lambda nm, n, k: gemm_bytes(m, mixw[nm].hi.n, k) + gemm_bytes(m, mixw[nm].lo.n, k, bits=2, group=64)
                  - 2 * m * k)):
-            def step():
-                for nm, (n, k) in shapes.items():
-                    lbq.linear_fwd(Xs[k], fn_weight(nm), Y=Ys[nm], stream=stream)
             ms = time_graph(torch, step, stream, reps=10)
             b = sum(bytes_of(nm, n, k) for nm, (n, k) in shapes.items())
             fl = sum(gemm_flops(m, n, k) for (n, k) in shapes.values())
@@ -600,6 +657,35 @@ def row_merge8b(lbq, syn, torch, peaks, stream):
                                   "requantize_us": round(1e3 * ms_q, 1),
                                   "requantize_GB/s": round(b_q / ms_q / 1e6, 1)}
         del W, qw, A, B, merged, q2
+    return out
+
+
+def row_channel_select(lbq, syn, torch, peaks, stream):
+    """Choosing the INT4 quarter of each 8B MLP matrix's output channels by
+    sensitivity (lbq_channel_mix_select, 128 calibration tokens); algorithmic
+    bytes: the bf16 weight and the calibration activations read, the
+    permutation written."""
+    out = {}
+    t = 128
+    for i, name in enumerate(("gate", "down")):
+        n, k = syn.LLAMA3_8B_SHAPES[name]
+        W = syn.weight_bf16(n, k, 0.02, seed=1600 + i, outlier_frac=0.001, device="cuda")
+        X = syn.normal_bf16((t, k), 1.0, seed=1610 + i, device="cuda")
+        n4 = n // 4
+        perm = torch.empty(n, dtype=torch.int32, device="cuda")
+        nws = lbq.lbq_channel_mix_select_workspace_size(n, k)
+        ws = torch.empty(nws, dtype=torch.uint8, device="cuda")
+
+        def fn():
+            rc = lbq.lbq_channel_mix_select(W.data_ptr(), n, k, X.data_ptr(), t, n4, None, perm.data_ptr(),
+                                            ws.data_ptr(), nws, stream.cuda_stream)
+            if rc != 0:
+                raise RuntimeError(f"lbq_channel_mix_select returned {rc}")
+        ms = time_graph(torch, fn, stream, reps=10)
+        b = 2 * n * k + 2 * t * k + 4 * n
+        out[f"{name} {n}x{k}"] = {"us": round(1e3 * ms, 1), "GB/s": round(b / ms / 1e6, 1),
+                                  "frac_hbm": round(b / ms / 1e6 / peaks["hbm_gbs"], 3)}
+        del W, X
     return out
 
 
@@ -685,7 +771,30 @@ def run_case(args):
     kind, rest = args.case.split("_", 1)
     name, arg = rest.rsplit("_", 1)
     stream = torch.cuda.current_stream()
-    if kind == "decode" or kind == "train":
+    if kind == "layerset":
+        # the 8B layer set in one grouped forward call at M = int(arg[1:])
+        import ctypes
+        m = int(arg[1:])
+        qws, Xs = [], {}
+        for i, (nm, (n, k)) in enumerate(syn.LLAMA3_8B_SHAPES.items()):
+            W = syn.weight_bf16(n, k, 0.02, seed=10 + i, outlier_frac=0.001, device="cuda")
+            qws.append(lbq.QuantizedWeight(n, k, "minmax", 4).quantize(W))
+            del W
+            if k not in Xs:
+                Xs[k] = syn.normal_bf16((m, k), 1.0, seed=2 + k, device="cuda")
+        Ys = [torch.empty((m, q.n), dtype=torch.float32, device="cuda") for q in qws]
+        probs = (lbq.lbq_fwd_problem * len(qws))()
+        for i, q in enumerate(qws):
+            probs[i] = lbq.lbq_fwd_problem(X=Xs[q.k].data_ptr(), q=ctypes.pointer(q.struct), A=None, B=None, rank=0,
+                                           s=0.0, Y=Ys[i].data_ptr(), T_save=None)
+        nws = lbq.lbq_linear_fwd_grouped_workspace_size(m, probs, len(qws))
+        ws = lbq._workspace(nws, "cuda")
+
+        def fn():
+            rc = lbq.lbq_linear_fwd_grouped(m, probs, len(qws), None if ws is None else ws.data_ptr(), nws,
+                                            stream.cuda_stream)
+            assert rc == 0, rc
+    elif kind == "decode" or kind == "train":
         n, k = syn.LLAMA3_8B_SHAPES[name]
         W = syn.weight_bf16(n, k, 0.02, seed=1, outlier_frac=0.001, device="cuda")
         qw = lbq.QuantizedWeight(n, k, "minmax", 4).quantize(W)
@@ -758,7 +867,7 @@ def main():
         torch.cuda.empty_cache()
         for key, fn in (("train_8b_mlp_M4096_r16", row_training), ("codebook_70b_dq", row_codebook70b),
                         ("mixed_8b", row_mixed), ("quantize_8b_int4", row_quantize8b),
-                        ("merge_8b_r16", row_merge8b)):
+                        ("merge_8b_r16", row_merge8b), ("channel_select_8b", row_channel_select)):
             try:
                 rows[key] = fn(lbq, syn, torch, peaks, stream)
             except Exception as e:  # report, do not hide, a failing row
@@ -774,7 +883,7 @@ def main():
                                "INT4 g128 MinMax, forward dequant-GEMM at M=1 and M=16 per step",
                    "weights": "N(0, 0.02^2) bf16, 0.1% input channels x20, 7 seeded copies",
                    "l2": "7 rotating weight copies (116 MB per pass > one pass of L2 reuse; a copy returns every 7th pass)",
-                   "launch": "one CUDA graph per step: 14 decode GEMV launches back to back (programmatic dependent launch); per_matrix from separate probe graphs with events between calls",
+                   "launch": "one CUDA graph per step: 2 grouped decode GEMV launches (M=1 and M=16, 7 layers each) back to back (programmatic dependent launch); per_matrix from separate probe graphs with events between single-matrix calls",
                    "parallelism": f"replicas x{dist.world}"},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": args.steps * wl_calls(),
@@ -787,7 +896,7 @@ def main():
 
 
 def wl_calls():
-    return len(DECODE_M) * 7
+    return len(DECODE_M)
 
 
 if __name__ == "__main__":

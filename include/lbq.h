@@ -76,10 +76,16 @@ typedef enum {
  *
  * LBQ_CODEBOOK4 (QLoRA explainer, 关键技术细节 1; bitsandbytes guide, nf4/fp4):
  *   bits 4, group 64 (blocks of 64 consecutive elements of the row-major W),
- *   k % 64 == 0.  codebook: 16 sorted fp32 values in [-1, 1] that include an
- *   exact 0 (device memory, read only).  absmax [n*k/64] fp32 = max |w| per
- *   block; code = index of the entry nearest to fp32(w / absmax) (the lower
- *   index on a tie; the 0 entry when absmax is 0).  packed [n, k/2] u8 as above.
+ *   k % 64 == 0.  codebook: 16 fp32 values in code order (device memory, read
+ *   only), all in [-1, 1], at least one of them a zero; they need not be
+ *   sorted or distinct (an NF4-style table is sorted; the FP4 E2M1 table,
+ *   bitsandbytes guide "nf4与fp4", holds +0 at code 0 and -0 at code 8), but
+ *   distinct values must be at least 2^-20 apart (otherwise lbq_quantize
+ *   sets LBQ_STATUS_BAD_TABLE in the device status word).
+ *   absmax [n*k/64] fp32 = max |w| per block; code = index of the entry
+ *   nearest to fp32(w / absmax) in fp32, the lower index on a tie (so of two
+ *   equal entries the lower code is the one produced; a zero goes to the
+ *   lowest zero code).  packed [n, k/2] u8 as above.
  *   Dequantized value: codebook[code] * absmax.
  *   With double_quant != 0 (QLoRA explainer, 结论; bitsandbytes guide, nested
  *   absmax): offset = fp32(fp64 sum of absmax / (n*k/64)); per block of 256
@@ -113,7 +119,7 @@ typedef struct {
  * two contiguous MinMax matrices, `hi` (INT4) then `lo` (INT2), with the same
  * k; perm[i] (0 <= i < hi.n + lo.n) is the original output channel of stored
  * row i (rows of `hi` first).  Y is produced in the original channel order.
- * hi.n and lo.n must be multiples of 128.
+ * hi.n and lo.n may be any sizes >= 1.
  */
 typedef struct {
     lbq_qweight hi;
@@ -201,17 +207,24 @@ lbq_status lbq_unmerge_lora(const void* W, int n, int k, const void* A,
 size_t lbq_linear_fwd_workspace_size(int m, const lbq_qweight* q, int rank);
 
 /*
- * The decode plan that lbq_linear_fwd uses for 1 <= m <= 16 (host only: no
- * device work, no GPU needed).  The units are (128-row tile, 64-column
- * k-block) pairs, row tiles x k/64 of them, cut into equal contiguous CTA
- * shares; a share spans at most two row tiles.  On success plan[0..5] =
- * CTAs, k-blocks per CTA, row tiles, weight-ring boxes of 16 KB, dynamic
- * shared memory per CTA in bytes, and the SM count the plan was made for
- * (`sms`; when sms <= 0, the current device's, or 148 without one).
- * Only n, k, bits, group and scheme of q are read.  Returns LBQ_EINVAL for m
- * outside 1..16, a NULL plan or an invalid q.
+ * The decode plan that the forward uses for 1 <= m <= 16 (host only: no
+ * device work, no GPU needed) for one launch over `count` weights
+ * (1 <= count <= 8; qs[i] are host pointers; only n, k, bits, group,
+ * scheme and double_quant are read).  The work of weight i is its
+ * (128-row tile, 64-column k-block) units, row tiles x k/64 of them in
+ * tile-major order, cut into equal contiguous CTA shares; every CTA of the
+ * launch gets about the same bytes and the launch is one wave of two CTAs per
+ * SM.  On success plan[0..7] = CTAs, ring stages, stage bytes, dynamic shared
+ * memory per CTA, workspace bytes, the SM count the plan was made for (`sms`;
+ * when sms <= 0, the current device's, or 148 without one), the bytes of the
+ * largest activation box of a stage and the row stride of the per-warp
+ * constant buffers; when per_problem is not
+ * NULL, per_problem[4i .. 4i+3] = k-blocks per CTA (share), CTAs, first CTA
+ * and row tiles of weight i.  Returns LBQ_EINVAL for m outside 1..16, count
+ * outside 1..8, a NULL plan or qs, or an invalid descriptor.
  */
-lbq_status lbq_gemv_plan(int m, const lbq_qweight* q, int sms, int64_t* plan);
+lbq_status lbq_gemv_plan(int m, const lbq_qweight* const* qs, int count, int sms,
+                         int64_t* plan, int64_t* per_problem);
 lbq_status lbq_linear_fwd(const void* X, int m, const lbq_qweight* q,
                           const void* A, const void* B, int rank, float s,
                           float* Y, float* T_save, void* workspace,
@@ -223,29 +236,72 @@ lbq_status lbq_linear_fwd(const void* X, int m, const lbq_qweight* q,
  * out up front by another runtime's pool, real-time or embedded loops that
  * must not allocate after start-up, and callers for whom a cudaMalloc (which
  * can synchronize the device) is not allowed at the point of the call.  It
- * takes no workspace: the split-K scratch of the decode-sized path lives in
- * a fixed array of 8 MiB (8388608 bytes) that the library declares once per
- * device and every device that loads the library keeps until the process
- * exits.  (The source pages have no
- * counterpart of this entry point.)
+ * takes no workspace: the split-K scratch of both forward paths (the decode
+ * GEMV for m <= 16 and the tensor-core GEMM when it splits K) lives in a fixed
+ * array of 8 MiB (8388608 bytes) that the library declares once per device
+ * and every device that loads the library keeps until the process exits.
+ * (The source pages have no counterpart of this entry point.)
  *
  * Arguments, layouts, results and errors are those of lbq_linear_fwd, plus:
  *  - LBQ_EWORKSPACE when this call's scratch (lbq_linear_fwd_workspace_size)
- *    is larger than the 8 MiB array; nothing is launched then.
- *  - The first call on a device looks up the array's device address (with
- *    that device current); make that first call before any stream capture.
+ *    is larger than the 8 MiB array; nothing is launched then.  Shapes whose
+ *    split-K scratch exceeds the array (large n or k with many token tiles)
+ *    are refused this way; lbq_linear_fwd_workspace_size tells in advance.
+ *  - Every call looks up the array's device address with the current device
+ *    current; the first call on a device may load the library's module, so
+ *    make it before any stream capture.
  *  - All calls share the one array: calls that can run at the same time on
  *    the GPU (different streams, overlapping graphs) race on it and must be
  *    ordered by the caller.  The array starts zero-filled (static storage)
  *    and every call leaves its per-tile counters at zero again; after a call
- *    whose kernels timed out (LBQ_ETIMEOUT from lbq_device_status) the
- *    counters may not be zero and later results of this entry point are
- *    undefined.
+ *    whose kernels timed out (LBQ_ETIMEOUT from lbq_device_status), call
+ *    lbq_linear_fwd_noalloc_reset before the next call.
  *  - It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  */
 lbq_status lbq_linear_fwd_noalloc(const void* X, int m, const lbq_qweight* q,
                                   const void* A, const void* B, int rank,
                                   float s, float* Y, float* T_save,
+                                  lbq_stream_t stream);
+
+/*
+ * Zero the per-tile counters of lbq_linear_fwd_noalloc's array (an
+ * asynchronous memset on `stream`; allocates nothing).  Needed only after a
+ * call whose kernels timed out.  (No counterpart in the source pages.)
+ */
+lbq_status lbq_linear_fwd_noalloc_reset(lbq_stream_t stream);
+
+/*
+ * Several forwards with the same token count m in one call (for example the
+ * seven linear layers of a transformer block at decode time, or q, k and v
+ * sharing X).  Each problem is one lbq_linear_fwd: Y_i = X_i W_i^T +
+ * s_i (X_i A_i^T) B_i^T with its own activations, weight, adapter and
+ * outputs (same layouts, rank and alignment rules; `q` is a host pointer to
+ * the descriptor).  For m <= 16 the problems run as one launch of the decode
+ * GEMV per group of up to 8 weights (after one adapter launch per problem with
+ * rank > 0), so the fixed costs of a launch are paid once per group; for
+ * larger m they run one after the other on `stream`.  The workspace
+ * (lbq_linear_fwd_grouped_workspace_size bytes, zero-filled before its first
+ * use, same reuse rules as lbq_linear_fwd's) serves all of them.  Results are
+ * bit for bit those of separate lbq_linear_fwd calls on the same inputs when
+ * the plan splits the matrices' work the same way; in every case each Y_i is
+ * within the forward's stated bound and deterministic.  (The pages' forward,
+ * QLoRA explainer, QLoRA技术原理, applied to a set of layers.)
+ */
+typedef struct {
+    const void* X;            /* bf16 [m, q->k], device */
+    const lbq_qweight* q;     /* host pointer to the weight descriptor */
+    const void* A;            /* bf16 [rank, q->k], device, or NULL when rank == 0 */
+    const void* B;            /* bf16 [q->n, rank], device, or NULL when rank == 0 */
+    int32_t rank;             /* 0 .. 64 */
+    float s;                  /* adapter scale */
+    float* Y;                 /* fp32 [m, q->n], device */
+    float* T_save;            /* fp32 [m, rank], device, or NULL when rank == 0 */
+} lbq_fwd_problem;
+
+size_t lbq_linear_fwd_grouped_workspace_size(int m, const lbq_fwd_problem* probs,
+                                             int count);
+lbq_status lbq_linear_fwd_grouped(int m, const lbq_fwd_problem* probs, int count,
+                                  void* workspace, size_t workspace_bytes,
                                   lbq_stream_t stream);
 
 /* The same forward for a channel-mix weight; Y columns in original order. */
@@ -262,6 +318,10 @@ lbq_status lbq_linear_fwd_mix(const void* X, int m, const lbq_qweight_mix* q,
  *   U  = dY B  [m, rank]                         (fp32, written to U_save)
  *   dX = dY W + s U A  [m, k]                    (fp32)
  * dY bf16 [m, n].  Same rank, workspace and layout rules as lbq_linear_fwd.
+ * Every weight format of lbq_qweight (MinMax INT4/INT2, the 4-bit codebook
+ * with or without double quantization) is accepted; n must be a multiple of
+ * 8.  The weight is dequantized to bf16 in the kernel: MinMax (code - zero)
+ * in bf16 times the scale, codebook bf16(fp32(codebook[code] * absmax')).
  */
 size_t lbq_linear_bwd_workspace_size(int m, const lbq_qweight* q, int rank);
 lbq_status lbq_linear_bwd(const void* dY, int m, const lbq_qweight* q,
@@ -281,10 +341,55 @@ lbq_status lbq_lora_grads(const void* X, const void* dY, int m, int n, int k,
                           float* dA, float* dB, lbq_stream_t stream);
 
 /*
- * Device status word: the OR of the LBQ_ETIMEOUT-style flags recorded by
- * kernels since the last call (0 when none).  Synchronizes the current device,
- * then clears the word.  Returns LBQ_ECUDA if the read itself fails.
+ * Channel-mix selection by sensitivity (GreenBit article, 模型量化 (1): the
+ * bit width of each output channel follows how much quantizing it to fewer
+ * bits costs).  W bf16 [n, k] (k % 128 == 0), calibration activations X bf16
+ * [t, k], all device, 16-byte aligned.
+ *   m2[j]    = (1/t) sum_i X[i,j]^2                       (fp64, i in order)
+ *   e4, e2   = W_hat - W of the MinMax INT4 g128 / INT2 g64 quantization
+ *              (lbq_quantize's arithmetic)
+ *   score[c] = sum_j m2[j] (e2[c,j]^2 - e4[c,j]^2)          (fp64)
+ * the rise of channel c's expected squared output error from INT4 to INT2.
+ * The n4 channels with the highest score (the lower index first among equal
+ * scores) are the INT4 channels: perm [n] (int32, device) lists them in
+ * ascending order, then the others in ascending order -- the permutation of
+ * lbq_qweight_mix.  score (fp64 [n], device) may be NULL.  workspace:
+ * lbq_channel_mix_select_workspace_size(n, k) bytes of device memory (any
+ * contents).  The per-channel sums run in an order of their own, so a score
+ * may differ from a sequential fp64 sum in its last bits.
  */
+size_t lbq_channel_mix_select_workspace_size(int n, int k);
+lbq_status lbq_channel_mix_select(const void* W_bf16, int n, int k,
+                                  const void* X_bf16, int t, int n4,
+                                  double* score, int32_t* perm, void* workspace,
+                                  size_t workspace_bytes, lbq_stream_t stream);
+
+/*
+ * out[i, :] = W[rows[i], :] for i < count: bf16 rows of W [n, k] (k % 8 ==
+ * 0), for example the INT4 and INT2 halves of a channel-mix weight in the
+ * order of its permutation.  rows: int32 device indices in [0, n).  (A data
+ * movement helper; the pages have no counterpart.)
+ */
+lbq_status lbq_gather_rows(const void* W_bf16, int n, int k, const int32_t* rows,
+                           int count, void* out, lbq_stream_t stream);
+
+/*
+ * Test hook for the bounded waits (no counterpart in the source pages): one
+ * kernel waits on an mbarrier phase that never completes and then on a
+ * device word that nothing sets, each for limit_us microseconds
+ * (1 <= limit_us <= 1000000), then returns.  Each wait that gives up records
+ * LBQ_ETIMEOUT in the device status word, exactly as the library's kernels do
+ * when a wait runs out; lbq_device_status reads it.  Nothing traps or faults.
+ */
+lbq_status lbq_selftest_wait_timeout(uint32_t limit_us, lbq_stream_t stream);
+
+/*
+ * Device status word: the OR of the flags below recorded by kernels since the
+ * last call (0 when none).  Synchronizes the current device, then clears the
+ * word.  Returns LBQ_ECUDA if the read itself fails.
+ */
+#define LBQ_STATUS_TIMEOUT 1u      /* a bounded device-side wait gave up (LBQ_ETIMEOUT) */
+#define LBQ_STATUS_BAD_TABLE 2u    /* a codebook broke the table preconditions */
 lbq_status lbq_device_status(uint32_t* flags);
 
 #ifdef __cplusplus

@@ -68,6 +68,8 @@ def _declare(L) -> None:
         "oracle_linear_bwd_sampled_minmax": (_int, [_vp, _i64, _vp, _vp, _vp, _i64, _i64, _int, _int,
                                                     _vp, _vp, _int, _dbl, _i64, _vp, _vp, _vp, _vp]),
         "oracle_lora_merge": (_int, [_vp, _i64, _i64, _vp, _vp, _int, ctypes.c_float, _int, _vp]),
+        "oracle_channel_score": (_int, [_vp, _i64, _i64, _vp, _i64, _vp, _vp]),
+        "oracle_channel_mix_select": (_int, [_vp, _i64, _i64, _vp]),
         "oracle_set_threads": (None, [_int]),
         "oracle_get_threads": (_int, []),
     }
@@ -305,3 +307,26 @@ def lora_merge(W_in, A, B, s: float, sign: int = 1) -> np.ndarray:
     _check(lib().oracle_lora_merge(_p(W_in), n, k, _p(A), _p(B), r, ctypes.c_float(float(s)), int(sign), _p(out)),
            "lora_merge")
     return out
+
+
+# ---------------------------------------------------------------- channel-mix selection
+def channel_score(W, X):
+    """(score [n] f64, bound [n] f64): the rise of channel c's expected
+    squared output error from INT4 g128 to INT2 g64, weighted by the
+    calibration activations' second moments (oracle.h)."""
+    W, X = _u16(W), _u16(X)
+    n, k = W.shape
+    t = X.shape[0]
+    assert X.shape[1] == k
+    score = np.zeros(n, np.float64)
+    bound = np.zeros(n, np.float64)
+    _check(lib().oracle_channel_score(_p(W), n, k, _p(X), t, _p(score), _p(bound)), "channel_score")
+    return score, bound
+
+
+def channel_mix_select(score, n4: int) -> np.ndarray:
+    """perm int32 [n]: the n4 highest-scoring channels ascending, then the rest."""
+    score = np.ascontiguousarray(score, dtype=np.float64)
+    perm = np.zeros(score.size, np.int32)
+    _check(lib().oracle_channel_mix_select(_p(score), score.size, int(n4), _p(perm)), "channel_mix_select")
+    return perm

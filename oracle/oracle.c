@@ -203,10 +203,12 @@ int oracle_codebook_quantize(const uint16_t* W, int64_t n, int64_t k,
                              const float* codebook, uint8_t* codes,
                              float* absmax) {
     if ((n * k) % 64 != 0) return -1;
+    /* any 16 entries in [-1, 1] that include a zero (+0 or -0), in any
+     * order: a table in code order, such as the FP4 (E2M1) one with its two
+     * zeros, is used as given */
     int has_zero = 0;
     for (int j = 0; j < 16; ++j) {
         if (codebook[j] == 0.0f) has_zero = 1;
-        if (j > 0 && !(codebook[j - 1] < codebook[j])) return -1;
         if (!(codebook[j] >= -1.0f && codebook[j] <= 1.0f)) return -1;
     }
     if (!has_zero) return -1;
@@ -588,4 +590,77 @@ int oracle_lora_merge(const float* W_in, int64_t n, int64_t k,
             W_out[row * k + col] = f32_to_bf16_rne(v);
         }
     return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* channel-mix selection by sensitivity ([GB] 模型量化 (1): the bit width of  */
+/* each output channel follows how sensitive it is to quantization)          */
+/*   m2[k]    = (1/T) sum_t x[t,k]^2               (second moment, fp64)      */
+/*   e4, e2   = W_hat - w for the MinMax INT4 g128 / INT2 g64 quantization    */
+/*   score[c] = sum_k m2[k] * (e2[c,k]^2 - e4[c,k]^2)                         */
+/*   bound[c] = sum_k m2[k] * (e2[c,k]^2 + e4[c,k]^2)                         */
+/* score is the rise of the expected squared output error of channel c when  */
+/* it goes from INT4 to INT2, with the calibration activations' second        */
+/* moments on the diagonal.  Selection: the n4 channels with the highest      */
+/* score (the lower channel index first among equal scores) are INT4.        */
+/* ------------------------------------------------------------------------ */
+int oracle_channel_score(const uint16_t* W, int64_t n, int64_t k, const uint16_t* X, int64_t t, double* score,
+                         double* bound) {
+    if (n < 1 || k < 128 || k % 128 != 0 || t < 1) return -1;
+    double* m2 = (double*)malloc(sizeof(double) * k);
+    uint8_t* c4 = (uint8_t*)malloc(n * k);
+    uint8_t* c2 = (uint8_t*)malloc(n * k);
+    uint16_t* s4 = (uint16_t*)malloc(sizeof(uint16_t) * n * (k / 128));
+    uint16_t* z4 = (uint16_t*)malloc(sizeof(uint16_t) * n * (k / 128));
+    uint16_t* s2 = (uint16_t*)malloc(sizeof(uint16_t) * n * (k / 64));
+    uint16_t* z2 = (uint16_t*)malloc(sizeof(uint16_t) * n * (k / 64));
+    int rc = (m2 && c4 && c2 && s4 && z4 && s2 && z2) ? 0 : -1;
+    if (rc == 0) {
+        for (int64_t j = 0; j < k; ++j) {
+            double acc = 0.0;
+            for (int64_t i = 0; i < t; ++i) {
+                double x = oracle_bf16_to_f32(X[i * k + j]);
+                acc += x * x;
+            }
+            m2[j] = acc / (double)t;
+        }
+        rc = oracle_minmax_quantize(W, n, k, 4, 128, c4, s4, z4);
+        if (rc == 0) rc = oracle_minmax_quantize(W, n, k, 2, 64, c2, s2, z2);
+    }
+    if (rc == 0) {
+#pragma omp parallel for schedule(static)
+        for (int64_t row = 0; row < n; ++row) {
+            double sc = 0.0, bd = 0.0;
+            for (int64_t j = 0; j < k; ++j) {
+                const double w = oracle_bf16_to_f32(W[row * k + j]);
+                /* the dequantized values, each one exact fp32 product */
+                const float w4 = ((float)c4[row * k + j] - oracle_f16_to_f32(z4[row * (k / 128) + j / 128])) *
+                                 oracle_f16_to_f32(s4[row * (k / 128) + j / 128]);
+                const float w2 = ((float)c2[row * k + j] - oracle_f16_to_f32(z2[row * (k / 64) + j / 64])) *
+                                 oracle_f16_to_f32(s2[row * (k / 64) + j / 64]);
+                const double e4 = (double)w4 - w, e2 = (double)w2 - w;
+                sc += m2[j] * (e2 * e2 - e4 * e4);
+                bd += m2[j] * (e2 * e2 + e4 * e4);
+            }
+            score[row] = sc;
+            if (bound) bound[row] = bd;
+        }
+    }
+    free(m2); free(c4); free(c2); free(s4); free(z4); free(s2); free(z2);
+    return rc;
+}
+
+int oracle_channel_mix_select(const double* score, int64_t n, int64_t n4, int32_t* perm) {
+    if (n < 1 || n4 < 0 || n4 > n) return -1;
+    /* rank of channel c: channels with a higher score, or an equal score and
+     * a lower index, come before it */
+    int64_t hi = 0, lo = n4;
+    for (int64_t c = 0; c < n; ++c) {
+        int64_t rank = 0;
+        for (int64_t d = 0; d < n; ++d)
+            if (score[d] > score[c] || (score[d] == score[c] && d < c)) ++rank;
+        if (rank < n4) perm[hi++] = (int32_t)c;
+        else perm[lo++] = (int32_t)c;
+    }
+    return (hi == n4 && lo == n) ? 0 : -1;
 }

@@ -63,8 +63,9 @@ int  oracle_minmax_dequantize(const uint8_t* packed, const uint16_t* scale,
                               int bits, int group, float* W_hat);
 
 /* --- 4-bit codebook quantizer with per-64 absmax ([QL], [BNB]) ---------- */
-/* codebook: 16 sorted fp32 entries in [-1, 1] containing an exact 0.
- * codes [n, k] (may be NULL), absmax fp32 [n*k/64]. */
+/* codebook: 16 fp32 entries in [-1, 1], in code order, containing a zero
+ * (+0 or -0); entries need not be sorted or distinct (the FP4 E2M1 table
+ * has both zeros).  codes [n, k] (may be NULL), absmax fp32 [n*k/64]. */
 int  oracle_codebook_quantize(const uint16_t* W, int64_t n, int64_t k,
                               const float* codebook, uint8_t* codes,
                               float* absmax);
@@ -151,6 +152,18 @@ int  oracle_lora_merge(const float* W_in, int64_t n, int64_t k,
                        int sign, uint16_t* W_out);
 
 /* Threads used by the loops over rows (OpenMP); 0 keeps the default. */
+/* --- channel-mix selection by sensitivity ([GB] 模型量化 (1)) -------------- */
+/* score[c] = sum_k m2[k] (e2^2 - e4^2), bound[c] = sum_k m2[k] (e2^2 + e4^2)
+ * with m2[k] = mean_t x[t,k]^2 over the calibration activations X [t, k]
+ * (bf16) and e4, e2 the errors of the MinMax INT4 g128 / INT2 g64
+ * dequantization of W [n, k] (bf16), all in fp64.  k % 128 == 0.
+ * bound may be NULL. */
+int  oracle_channel_score(const uint16_t* W, int64_t n, int64_t k, const uint16_t* X,
+                          int64_t t, double* score, double* bound);
+/* perm [n]: the n4 channels of highest score (ties: lower channel first) in
+ * ascending order, then the others in ascending order. */
+int  oracle_channel_mix_select(const double* score, int64_t n, int64_t n4, int32_t* perm);
+
 void oracle_set_threads(int nthreads);
 int  oracle_get_threads(void);
 

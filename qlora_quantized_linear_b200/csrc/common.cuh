@@ -112,13 +112,14 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
     return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 0; it < kWaitLimitIters; ++it) {
         if (mbar_try_wait_sleep(bar, parity)) return true;
         if (*abort) return false;
-        if ((it & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) break;
+        if ((it & 63u) == 63u && globaltimer_ns() - t0 > limit_ns) break;
     }
     *abort = 1;
     record_status(kStatusTimeout);
@@ -127,12 +128,39 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 
 // Bounded wait that ignores the abort flag: used to let this CTA's own
 // asynchronous copies and MMAs finish before it frees memory and exits.
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 0; it < kWaitLimitIters; ++it) {
         if (mbar_try_wait_sleep(bar, parity)) return true;
-        if ((it & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) break;
+        if ((it & 63u) == 63u && globaltimer_ns() - t0 > limit_ns) break;
+    }
+    record_status(kStatusTimeout);
+    return false;
+}
+
+// Split-tile flags: a contributor publishes its partial sums (stored by all
+// threads of the CTA before the barrier that precedes this call) and counts
+// itself; the finishing CTA waits for the count with acquire semantics.
+__device__ __forceinline__ void flag_publish(uint32_t* f) {
+    asm volatile("fence.acq_rel.gpu;\n\tred.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(f) : "memory");
+}
+
+__device__ __forceinline__ uint32_t flag_load_acquire(const uint32_t* f) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    return v;
+}
+
+// Bounded wait for *f >= want; records kStatusTimeout and returns false when
+// it gives up.
+__device__ __forceinline__ bool flag_wait_geq(const uint32_t* f, uint32_t want, uint64_t limit_ns = kWaitLimitNs) {
+    if (flag_load_acquire(f) >= want) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 0; it < kWaitLimitIters; ++it) {
+        __nanosleep(64);
+        if (flag_load_acquire(f) >= want) return true;
+        if ((it & 63u) == 63u && globaltimer_ns() - t0 > limit_ns) break;
     }
     record_status(kStatusTimeout);
     return false;
@@ -283,6 +311,37 @@ __device__ __forceinline__ uint16_t f32_to_f16_bits(float x) {
 __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// (a & MASK) | c in one logic op.
+template <uint32_t MASK>
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "n"(MASK), "r"(c));
+    return d;
+}
+
+// Code pairs of one 32-bit word of 4-bit codes (bytes b0..b3 = codes 0..7):
+// P0 = (1, 5), P1 = (0, 4), P2 = (3, 7), P3 = (2, 6), each half the bf16
+// number 128 + code (mg = 0x43004300 is passed in a register).
+__device__ __forceinline__ void int4_pairs(uint32_t w, uint32_t mg, uint32_t* o) {
+    o[0] = and_or<0x000F000Fu>(w, mg);
+    o[1] = and_or<0x000F000Fu>(w >> 4, mg);
+    o[2] = and_or<0x000F000Fu>(w >> 8, mg);
+    o[3] = and_or<0x000F000Fu>(w >> 12, mg);
+}
+
+// Code pairs of one 32-bit word of 2-bit codes (bytes b0..b3 = codes 0..15,
+// first code in the top bits): pair t = (t, t + 8), t = 0..7.
+__device__ __forceinline__ void int2_pairs(uint32_t w, uint32_t mg, uint32_t* o) {
+    o[0] = and_or<0x00030003u>(w >> 6, mg);
+    o[1] = and_or<0x00030003u>(w >> 4, mg);
+    o[2] = and_or<0x00030003u>(w >> 2, mg);
+    o[3] = and_or<0x00030003u>(w, mg);
+    o[4] = and_or<0x00030003u>(w >> 14, mg);
+    o[5] = and_or<0x00030003u>(w >> 12, mg);
+    o[6] = and_or<0x00030003u>(w >> 10, mg);
+    o[7] = and_or<0x00030003u>(w >> 8, mg);
 }
 
 }  // namespace lbq

@@ -69,9 +69,10 @@ struct WeightTile {
 
 // Shared-memory layout of the forward kernel: a ring of XS activation slots
 // (XB k-blocks of NT x 64 bf16 each, fetched by one 3-D TMA box), a ring of
-// WS packed-weight chunks (128 rows x 128 B), the mbarriers and the adapter T
-// tile [NT, rank_pad].  Few, large TMA boxes: each box costs the TMA engine
-// a fixed issue-to-completion slot, so small boxes waste its throughput.
+// WS packed-weight chunks (128 rows x 128 B), the mbarriers and, with an
+// adapter, the MMA operand tile of s*T [NT tokens x 64 rank] (bf16, K-major,
+// 128-byte swizzle).  Few, large TMA boxes: each box costs the TMA engine a
+// fixed issue-to-completion slot, so small boxes waste its throughput.
 template <int NT, int XS, int XB, int WS, int AS>
 struct FwdSmem {
     static constexpr int kXTile = NT * 128;              // one k-block of X
@@ -82,8 +83,8 @@ struct FwdSmem {
     static constexpr size_t kBar = kW + size_t(WS) * kWBytes;
     static constexpr int kNumBars = 2 * XS + 2 * WS + 2 * AS + 1;
     static constexpr size_t kMisc = kBar + kNumBars * 8;
-    static constexpr size_t kLoraT = (kMisc + 128 + 15) / 16 * 16;
-    static size_t total(int rank_pad) { return kLoraT + size_t(NT) * rank_pad * 4 + 1024; }
+    static constexpr size_t kLoraT = (kMisc + 128 + 1023) / 1024 * 1024;
+    static size_t total(int rank) { return kLoraT + (rank > 0 ? size_t(NT) * 128 : 0) + 1024; }
 };
 
 // Shared-memory layout of one CTA: a ring of STAGES (activation tile, packed
@@ -101,6 +102,10 @@ struct GemmSmem {
     static constexpr size_t kLoraT = kTab + size_t(TABBYTES);
     static size_t total(int rank_pad) { return kLoraT + size_t(NT) * rank_pad * 4 + 1024; }
 };
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 
 __host__ __device__ constexpr uint32_t tmem_cols_for(int ncols) {
     return ncols <= 32 ? 32 : ncols <= 64 ? 64 : ncols <= 128 ? 128 : ncols <= 256 ? 256 : 512;
@@ -309,7 +314,7 @@ constexpr int kDqWarps = 8;
 template <int NT>
 struct FwdCfg {
     static constexpr int kXBlocks = NT <= 16 ? 8 : NT <= 32 ? 4 : NT <= 64 ? 2 : 1;   // k-blocks per X box
-    static constexpr int kXStages = NT <= 32 ? 2 : NT <= 64 ? 3 : 4;
+    static constexpr int kXStages = NT <= 32 ? 2 : NT <= 128 ? 3 : 4;
     static constexpr int kWStages = NT <= 32 ? 4 : NT <= 64 ? 3 : 2;
     static constexpr int kAStages = NT <= 32 ? 6 : 4;
     static constexpr int kMinBlocks = NT >= 256 ? 1 : 2;   // CTAs per SM
@@ -354,7 +359,7 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
     int* s_last = reinterpret_cast<int*>(smem + L::kMisc + 8);
     float* s_cb = reinterpret_cast<float*>(smem + L::kMisc + 64);  // 16 floats
-    float* sT = reinterpret_cast<float*>(smem + L::kLoraT);
+    uint8_t* sTop = smem + L::kLoraT;                  // s*T operand tile [NT x 128 B]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * 128;
@@ -364,6 +369,11 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     const int kb0 = split * p.kb_per_split;            // a multiple of SUB
     const int nkb = min(p.kb_per_split, kb_total - kb0);
     const int nch = (nkb + SUB - 1) / SUB;              // weight chunks of this CTA
+    // the adapter term s * T B^T enters the accumulator through rank/16 MMAs
+    // before the main loop, in the first K split only: its A operand (the B
+    // rows) takes the first slot of the A ring, as a k-block before the first
+    const bool lora = p.rank > 0 && split == 0;
+    const int a_off = lora ? 1 : 0;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < XS; ++i) {
@@ -430,11 +440,21 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             bool ok = true;
+            if (lora) {
+                // D = (s T) B^T: A = the B rows (A ring slot 0), B operand = s T (shared)
+                ok = mbar_wait(&afull[0], 0, s_abort);
+                tc_fence_after();
+                const uint64_t tdesc = smem_desc_k_sw128(smem_u32(sTop));
+                for (int j = 0; ok && j < p.rank_pad / 16; ++j)
+                    mma_ts(tmem + kDCol, tmem + kACol0 + 8 * j, tdesc + static_cast<uint64_t>(2 * j), kIdesc,
+                           j > 0 ? 1u : 0u);
+                if (ok) mma_commit(&aempty[0]);
+            }
             for (int i = 0; i < nkb && ok; ++i) {
-                const int xj = i / XB, xsub = i - xj * XB, x = xj % XS, a = i % AS;
+                const int xj = i / XB, xsub = i - xj * XB, x = xj % XS, ia = i + a_off, a = ia % AS;
                 if (xsub == 0) ok = mbar_wait(&fullX[x], (xj / XS) & 1, s_abort);
                 LBQ_TRACE_EVENT(4, i);
-                ok = ok && mbar_wait(&afull[a], (i / AS) & 1, s_abort);
+                ok = ok && mbar_wait(&afull[a], (ia / AS) & 1, s_abort);
                 if (!ok) break;
                 tc_fence_after();
                 LBQ_TRACE_EVENT(5, i);
@@ -442,7 +462,7 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     mma_ts(tmem + kDCol, tmem + kACol0 + a * kACols + 8 * j, bdesc + static_cast<uint64_t>(2 * j), kIdesc,
-                           (i > 0 || j > 0) ? 1u : 0u);
+                           (lora || i > 0 || j > 0) ? 1u : 0u);
                 if (xsub == XB - 1 || i == nkb - 1) mma_commit(&emptyX[x]);
                 mma_commit(&aempty[a]);
             }
@@ -459,13 +479,47 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         const bool has_dq = (KIND == kCode4) && (p.q8 != nullptr);
         const float dq_offset = has_dq ? __ldg(p.offset) : 0.0f;
+        const int out_col = row_ok ? (p.perm ? p.perm[grow] : static_cast<int>(grow)) : 0;
+        const int mt = min(NT, p.m - t0);                  // tokens in this tile
+        if (lora) {
+            // A operand (ring slot 0): this row's adapter coefficients
+            // B[out_col, 32 half .. 32 half + 31] (bf16, zero beyond the rank)
+            uint32_t bv[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int u = 32 * half + 2 * i;
+                const uint32_t lo = (row_ok && u < p.rank) ? __ldg(p.B + static_cast<int64_t>(out_col) * p.rank + u) : 0u;
+                const uint32_t hi = (row_ok && u + 1 < p.rank) ? __ldg(p.B + static_cast<int64_t>(out_col) * p.rank + u + 1) : 0u;
+                bv[i] = lo | (hi << 16);
+            }
+            tmem_st_32x32b_x16(tmem + lane_base + kACol0 + 16 * half, bv);
+            // B operand: bf16(s * T[t0 + tt, u]) at row tt, 16-byte unit u / 8 of its
+            // 128-byte line, swizzled with the row (zero beyond the tokens and the rank)
+            const int tid = threadIdx.x - 64;
+            for (int e = tid; e < NT * 32; e += 32 * kDqWarps) {
+                const int tt = e >> 5, u = 2 * (e & 31);
+                float v0 = 0.0f, v1 = 0.0f;
+                if (tt < mt) {
+                    const float* trow = p.T + static_cast<int64_t>(t0 + tt) * p.rank;
+                    if (u < p.rank) v0 = __fmul_rn(p.s, trow[u]);
+                    if (u + 1 < p.rank) v1 = __fmul_rn(p.s, trow[u + 1]);
+                }
+                *reinterpret_cast<uint32_t*>(sTop + tt * 128 + (((u >> 3) ^ (tt & 7)) << 4) + (u & 7) * 2) =
+                    pack_bf16x2_rn(v0, v1);
+            }
+            fence_proxy_async_smem();
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&afull[0]);
+        }
         PreConst nxt = preload_const<KIND>(p, grow, kb0, row_ok && nkb > 0);
         for (int i = 0; i < nkb; ++i) {
-            const int c = i / SUB, sub = i - c * SUB, w = c % WS, a = i % AS;
+            const int c = i / SUB, sub = i - c * SUB, w = c % WS, ia = i + a_off, a = ia % AS;
             const PreConst cur = nxt;
             if (i + 1 < nkb) nxt = preload_const<KIND>(p, grow, kb0 + i + 1, row_ok);
             if (sub == 0 && !mbar_wait(&fullW[w], (c / WS) & 1, s_abort)) break;
-            if (i >= AS && !mbar_wait(&aempty[a], ((i / AS) - 1) & 1, s_abort)) break;
+            if (ia >= AS && !mbar_wait(&aempty[a], ((ia / AS) - 1) & 1, s_abort)) break;
             tc_fence_after();
             if (lane == 0) LBQ_TRACE_EVENT(2, i * 8 + (warp - 2));
             uint32_t vals[16];
@@ -489,22 +543,11 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         (void)nch;
 
         // ------------------------------------------------------------ epilogue
-        const int mt = min(NT, p.m - t0);  // tokens in this tile
-        const bool lora = p.rank > 0;
-        const int tid = threadIdx.x - 64;  // 0..255
-        if (lora) {
-            // stage T[t0 : t0 + mt, :rank] (fp32, zero-padded) for the adapter term
-            for (int e = tid; e < NT * p.rank_pad; e += 32 * kDqWarps) {
-                const int tt = e / p.rank_pad, u = e - tt * p.rank_pad;
-                sT[e] = (tt < mt && u < p.rank) ? p.T[static_cast<int64_t>(t0 + tt) * p.rank + u] : 0.0f;
-            }
-        }
+        // (the adapter term is already in the accumulator)
         asm volatile("bar.sync 1, 256;" ::: "memory");
         const bool got = mbar_wait(dfull, 0, s_abort);
         tc_fence_after();
         if (threadIdx.x == 64) LBQ_TRACE_EVENT(0, 1);
-        const int out_col = row_ok ? (p.perm ? p.perm[grow] : static_cast<int>(grow)) : 0;
-        const int rp = p.rank_pad;
         const bool splitk = p.nsplit > 1;
         constexpr int kHalfCols = NT >= 32 ? NT / 2 : 16;  // token columns per warp group
         const int c_begin = half * kHalfCols;
@@ -523,7 +566,6 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     if (jj + j < mt) p.partial[(static_cast<int64_t>(split) * p.m + t0 + jj + j) * p.n + grow] = acc[j];
                 continue;
             }
-            if (lora) lora_add16(acc, sT + jj * rp, rp, p.rank, p.B + static_cast<int64_t>(out_col) * p.rank, p.s);
 #pragma unroll
             for (int j = 0; j < 16; ++j)
                 if (jj + j < mt) p.Y[static_cast<int64_t>(t0 + jj + j) * p.ldy + out_col] = acc[j];
@@ -554,7 +596,6 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 #pragma unroll
                         for (int j = 0; j < 16; ++j) acc[j] += part[j];
                     }
-                    if (lora) lora_add16(acc, sT + jj * rp, rp, p.rank, p.B + static_cast<int64_t>(out_col) * p.rank, p.s);
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
                         if (jj + j < mt) p.Y[static_cast<int64_t>(t0 + jj + j) * p.ldy + out_col] = acc[j];

@@ -30,11 +30,26 @@
 
 namespace lbq {
 
+// Order of the 8 (4-bit) or 16 (2-bit) features of a pairing group as the
+// dequantized tile holds them: 4-bit codes pair nibbles two bytes apart
+// (features k and k+4 of a word), 2-bit codes pair crumbs two bytes apart
+// (k and k+8).  Entry p is the feature stored at position p.
+__device__ __forceinline__ int bwd_xperm(int kind, int p) {
+    constexpr int kPerm4[16] = {1, 5, 0, 4, 3, 7, 2, 6, 9, 13, 8, 12, 11, 15, 10, 14};
+    constexpr int kPerm2[16] = {0, 8, 1, 9, 2, 10, 3, 11, 4, 12, 5, 13, 6, 14, 7, 15};
+    return kind == kInt2 ? kPerm2[p] : kPerm4[p];
+}
+
 struct BwdParams {
     int m, n, k;                 // tokens, weight rows (output channels), input features
     int bits, ngroups, group;    // MinMax bit width, k / group, group
     const uint16_t* scale;       // [n, ngroups]
     const uint16_t* zero;        // [n, ngroups]
+    const float* absmax;         // [n * k / 64] (codebook, no double quant)
+    const int8_t* q8;            // [n * k / 64] (codebook, double quant)
+    const float* s2;             // [ceil(n * k / 64 / 256)]
+    const float* offset;         // [1]
+    const float* codebook;       // [16]
     int rank, rank_pad;
     float s;
     const float* U;              // [m, rank] fp32
@@ -69,8 +84,8 @@ struct BwdSmem {
     static constexpr size_t kBar = kW + size_t(WS) * kWBytes;
     static constexpr int kNumBars = 2 * XS + 2 * WS + 2 * AS + 1;
     static constexpr size_t kMisc = kBar + kNumBars * 8;
-    static constexpr size_t kLoraT = (kMisc + 128 + 15) / 16 * 16;
-    static size_t total(int rank_pad) { return kLoraT + size_t(NT) * rank_pad * 4 + 1024; }
+    static constexpr size_t kLoraT = (kMisc + 128 + 1023) / 1024 * 1024;   // s*U operand tile
+    static size_t total(int rank) { return kLoraT + (rank > 0 ? size_t(NT) * 128 : 0) + 1024; }
 };
 
 // Shared-memory descriptor of an MN-major operand with the 128-byte swizzle:
@@ -97,10 +112,6 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
         : "memory");
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // Byte offset of 16-byte unit `fu` (features 8 fu .. 8 fu + 7) of channel row
 // c (0..63) in the MN-major A tile [64 channels][128 features]: groups of 8
 // channels 2048 bytes apart, the two 64-feature halves 1024 bytes apart,
@@ -110,13 +121,13 @@ __device__ __forceinline__ uint32_t bwd_a_offset(int c, int fu) {
     return static_cast<uint32_t>((c >> 3) * 2048 + (fu >> 3) * 1024 + row * 128 + ((uu ^ row) << 4));
 }
 
-template <int NT, int BITS, int XS, int WS, int AS, int MINB>
+template <int NT, int KIND, int XS, int WS, int AS, int MINB>
 __global__ void __launch_bounds__(kBwdThreads, MINB)
 dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constant__ CUtensorMap tmW,
                   const BwdParams p) {
+    constexpr int BITS = KIND == kInt2 ? 2 : 4;
     using L = BwdSmem<NT, BITS, XS, WS, AS>;
     constexpr int KTB = L::kKTB;
-    constexpr int KIND = BITS == 4 ? kInt4 : kInt2;
     constexpr int PG = BITS == 4 ? 8 : 16;                 // features per pairing group
     constexpr int SLOTS = BITS == 4 ? 4 : 2;               // (channel, word) units per thread and block
     constexpr uint32_t kTmemCols = tmem_cols_for(NT);
@@ -138,7 +149,8 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
     int* s_last = reinterpret_cast<int*>(smem + L::kMisc + 8);
-    float* sT = reinterpret_cast<float*>(smem + L::kLoraT);
+    float* s_cb = reinterpret_cast<float*>(smem + L::kMisc + 64);   // codebook, 16 floats
+    uint8_t* sUop = smem + L::kLoraT;                  // s*U operand tile [NT x 128 B] (bf16, K-major, SW128)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int k0 = blockIdx.x * 128;
@@ -147,6 +159,11 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
     const int cb_total = (p.n + 63) / 64;
     const int cb0 = split * p.cb_per_split;
     const int ncb = min(p.cb_per_split, cb_total - cb0);
+    // the adapter term s * U A enters the accumulator through rank/16 MMAs
+    // before the main loop, in the first split only; its A operand (the rows
+    // of A) takes the first slot of the A ring, as a block before the first
+    const bool lora = p.rank > 0 && split == 0;
+    const int a_off = lora ? 1 : 0;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < XS; ++i) {
@@ -165,6 +182,7 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
         *s_abort = 0;
         fence_mbar_init();
     }
+    if (KIND == kCode4 && threadIdx.x < 16) s_cb[threadIdx.x] = p.codebook[threadIdx.x];
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmDY);
         tma_prefetch_desc(&tmW);
@@ -201,9 +219,20 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             bool ok = true;
+            if (lora) {
+                // D = A^T (s U)^T: A operand = the adapter's A rows (A ring slot 0), B operand = s U
+                ok = mbar_wait(&afull[0], 0, s_abort);
+                tc_fence_after();
+                const uint32_t abase = smem_u32(sA);
+                const uint64_t udesc = smem_desc_k_sw128(smem_u32(sUop));
+                for (int j = 0; ok && j < p.rank_pad / 16; ++j)
+                    mma_ss(tmem, smem_desc_mn_sw128(abase + j * 4096, 1024, 2048), udesc + static_cast<uint64_t>(2 * j),
+                           kIdesc, j > 0 ? 1u : 0u);
+                if (ok) mma_commit(&aempty[0]);
+            }
             for (int i = 0; i < ncb && ok; ++i) {
-                const int x = i % XS, a = i % AS;
-                ok = mbar_wait(&fullX[x], (i / XS) & 1, s_abort) && mbar_wait(&afull[a], (i / AS) & 1, s_abort);
+                const int x = i % XS, ia = i + a_off, a = ia % AS;
+                ok = mbar_wait(&fullX[x], (i / XS) & 1, s_abort) && mbar_wait(&afull[a], (ia / AS) & 1, s_abort);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t abase = smem_u32(sA + a * L::kABytes);
@@ -211,7 +240,7 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     mma_ss(tmem, smem_desc_mn_sw128(abase + j * 4096, 1024, 2048), bdesc + static_cast<uint64_t>(2 * j),
-                           kIdesc, (i > 0 || j > 0) ? 1u : 0u);
+                           kIdesc, (lora || i > 0 || j > 0) ? 1u : 0u);
                 mma_commit(&emptyX[x]);
                 mma_commit(&aempty[a]);
             }
@@ -226,22 +255,75 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
         const int crow0 = BITS == 4 ? (tid >> 4) : (tid >> 3);
         const int cstep = BITS == 4 ? 16 : 32;
         const int gsub = BITS == 4 ? 0 : (fw >> 2);        // 64-feature group of this word (INT2 g64)
-        const int gcol = k0 / p.group + gsub;
+        const int gcol = KIND == kCode4 ? 0 : k0 / p.group + gsub;
+        const int64_t kbt = p.k / 64;
+        const int kbc = k0 / 64 + (fw >> 3);               // codebook: the word's k-block
+        const bool has_dq = KIND == kCode4 && p.q8 != nullptr;
+        const float dq_off = has_dq ? __ldg(p.offset) : 0.0f;
         uint32_t mg = 0x43004300u;
         asm volatile("" : "+r"(mg));
-        // constants of the next block's channels, loaded one block ahead
+        // constants of the next block's channels, loaded one block ahead:
+        // MinMax scale and zero; codebook absmax, or q8 and s2
         uint32_t ns[SLOTS], nz[SLOTS];
         auto load_const = [&](int i) {
 #pragma unroll
             for (int u = 0; u < SLOTS; ++u) {
                 const int64_t c = static_cast<int64_t>(cb0 + i) * 64 + crow0 + u * cstep;
-                ns[u] = c < p.n ? __ldg(p.scale + c * p.ngroups + gcol) : 0u;
-                nz[u] = c < p.n ? __ldg(p.zero + c * p.ngroups + gcol) : 0u;
+                if (KIND != kCode4) {
+                    ns[u] = c < p.n ? __ldg(p.scale + c * p.ngroups + gcol) : 0u;
+                    nz[u] = c < p.n ? __ldg(p.zero + c * p.ngroups + gcol) : 0u;
+                } else if (has_dq) {
+                    const int64_t e = c * kbt + kbc;
+                    ns[u] = c < p.n ? static_cast<uint32_t>(static_cast<int32_t>(__ldg(p.q8 + e))) : 0u;
+                    nz[u] = c < p.n ? __float_as_uint(__ldg(p.s2 + (e >> 8))) : 0u;
+                } else {
+                    ns[u] = c < p.n ? __float_as_uint(__ldg(p.absmax + c * kbt + kbc)) : 0u;
+                    nz[u] = 0u;
+                }
             }
         };
         if (ncb > 0) load_const(0);
+        if (lora) {
+            // A operand (ring slot 0): K row u = A[u, k0 + feature], features in
+            // the tile's pairing order (zero beyond the rank and beyond k)
+            const int nunits = p.rank_pad * 16;            // 16-byte units: 8 features of one row
+            for (int e = tid; e < nunits; e += 32 * kBwdDqWarps) {
+                const int u = e >> 4, fu = e & 15;
+                uint32_t wv[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    uint32_t two[2];
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        const int pos = fu * 8 + 2 * h + t;
+                        const int f = (pos & ~(PG - 1)) + bwd_xperm(KIND, pos & (PG - 1));
+                        const int64_t kc = static_cast<int64_t>(k0) + f;
+                        two[t] = (u < p.rank && kc < p.k) ? __ldg(p.A + static_cast<int64_t>(u) * p.k + kc) : 0u;
+                    }
+                    wv[h] = two[0] | (two[1] << 16);
+                }
+                *reinterpret_cast<uint4*>(sA + bwd_a_offset(u, fu)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            }
+            // B operand: bf16(s * U[t0 + tt, u]) at row tt, 16-byte unit u / 8,
+            // swizzled with the row (zero beyond the tokens and the rank)
+            const int mt0 = min(NT, p.m - t0);
+            for (int e = tid; e < NT * 32; e += 32 * kBwdDqWarps) {
+                const int tt = e >> 5, u = 2 * (e & 31);
+                float v0 = 0.0f, v1 = 0.0f;
+                if (tt < mt0) {
+                    const float* urow = p.U + static_cast<int64_t>(t0 + tt) * p.rank;
+                    if (u < p.rank) v0 = __fmul_rn(p.s, urow[u]);
+                    if (u + 1 < p.rank) v1 = __fmul_rn(p.s, urow[u + 1]);
+                }
+                *reinterpret_cast<uint32_t*>(sUop + tt * 128 + (((u >> 3) ^ (tt & 7)) << 4) + (u & 7) * 2) =
+                    pack_bf16x2_rn(v0, v1);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&afull[0]);
+        }
         for (int i = 0; i < ncb; ++i) {
-            const int w = i % WS, a = i % AS;
+            const int w = i % WS, ia = i + a_off, a = ia % AS;
             uint32_t cs[SLOTS], cz[SLOTS];
 #pragma unroll
             for (int u = 0; u < SLOTS; ++u) {
@@ -250,7 +332,7 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
             }
             if (i + 1 < ncb) load_const(i + 1);
             if (!mbar_wait(&fullW[w], (i / WS) & 1, s_abort)) break;
-            if (i >= AS && !mbar_wait(&aempty[a], ((i / AS) - 1) & 1, s_abort)) break;
+            if (ia >= AS && !mbar_wait(&aempty[a], ((ia / AS) - 1) & 1, s_abort)) break;
             uint32_t words[SLOTS];
 #pragma unroll
             for (int u = 0; u < SLOTS; ++u)
@@ -259,8 +341,26 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
 #pragma unroll
             for (int u = 0; u < SLOTS; ++u) {
                 const int c = crow0 + u * cstep;
-                const MinMaxConst mc = minmax_const(static_cast<uint16_t>(cs[u]), static_cast<uint16_t>(cz[u]));
                 uint32_t o[PG / 2];
+                if (KIND == kCode4) {
+                    // W_hat = bf16(fp32(codebook[code] * absmax')), rounded once,
+                    // in the 4-bit pairing order (codes 1,5 / 0,4 / 3,7 / 2,6)
+                    const float a = has_dq ? __fadd_rn(__fmul_rn(__fdiv_rn(static_cast<float>(static_cast<int32_t>(cs[u])),
+                                                                           127.0f),
+                                                                 __uint_as_float(cz[u])),
+                                                       dq_off)
+                                           : __uint_as_float(cs[u]);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        o[q] = pack_bf16x2_rn(__fmul_rn(s_cb[(words[u] >> (4 * q)) & 15u], a),
+                                              __fmul_rn(s_cb[(words[u] >> (16 + 4 * q)) & 15u], a));
+#pragma unroll
+                    for (int h = 0; h < PG / 8; ++h)
+                        *reinterpret_cast<uint4*>(atile + bwd_a_offset(c, (PG / 8) * fw + h)) =
+                            make_uint4(o[4 * h], o[4 * h + 1], o[4 * h + 2], o[4 * h + 3]);
+                    continue;
+                }
+                const MinMaxConst mc = minmax_const(static_cast<uint16_t>(cs[u]), static_cast<uint16_t>(cz[u]));
                 if (BITS == 4)
                     int4_pairs(words[u], mg, o);
                 else
@@ -292,22 +392,15 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
         const int half = (warp - 2) >> 2;                  // token half
         const int lrow = q * 32 + lane;                    // A-tile row = TMEM lane
         // feature of this lane: the pairing order of its group of PG features
-        const int feat = (lrow & ~(PG - 1)) + gemv_xperm(KIND, lrow & (PG - 1));
+        const int feat = (lrow & ~(PG - 1)) + bwd_xperm(KIND, lrow & (PG - 1));
         const int64_t kcol = k0 + feat;
         const bool col_ok = kcol < p.k;
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         const int mt = min(NT, p.m - t0);
-        const bool lora = p.rank > 0;
-        if (lora) {
-            for (int e = tid; e < NT * p.rank_pad; e += 32 * kBwdDqWarps) {
-                const int tt = e / p.rank_pad, u = e - tt * p.rank_pad;
-                sT[e] = (tt < mt && u < p.rank) ? p.U[static_cast<int64_t>(t0 + tt) * p.rank + u] : 0.0f;
-            }
-        }
+        // (the adapter term is already in the accumulator)
         asm volatile("bar.sync 1, 256;" ::: "memory");
         const bool got = mbar_wait(dfull, 0, s_abort);
         tc_fence_after();
-        const int rp = p.rank_pad;
         const bool splitk = p.nsplit > 1;
         constexpr int kHalfCols = NT >= 32 ? NT / 2 : 16;
         const int c_begin = half * kHalfCols;
@@ -326,7 +419,6 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
                     if (jj + j < mt) p.partial[(static_cast<int64_t>(split) * p.m + t0 + jj + j) * p.k + kcol] = acc[j];
                 continue;
             }
-            if (lora) lora_add16(acc, sT + jj * rp, rp, p.rank, p.A + kcol, p.s, p.k);
 #pragma unroll
             for (int j = 0; j < 16; ++j)
                 if (jj + j < mt) p.dX[static_cast<int64_t>(t0 + jj + j) * p.k + kcol] = acc[j];
@@ -358,7 +450,6 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
 #pragma unroll
                         for (int j = 0; j < 16; ++j) acc[j] += part[j];
                     }
-                    if (lora) lora_add16(acc, sT + jj * rp, rp, p.rank, p.A + kcol, p.s, p.k);
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
                         if (jj + j < mt) p.dX[static_cast<int64_t>(t0 + jj + j) * p.k + kcol] = acc[j];

@@ -1,41 +1,54 @@
 // dqgemv.cuh -- bandwidth-bound dequantize-GEMV for decode-sized batches
-// (M <= 16 tokens), stream-K over (row tile, k-block) work.
+// (M <= 16 tokens) over a GROUP of weight matrices in one launch.
 //
-//   Y[t, c] = sum_k X[t, k] * W_hat[c, k]  (+ s * sum_u T[t, u] B[c, u])
+//   Y_i[t, c] = sum_k X_i[t, k] * W_hat_i[c, k]  (+ s_i * sum_u T_i[t, u] B_i[c, u])
 //
-// At decode sizes the packed weight is the whole cost (0.53 B/param for INT4
-// g128), so the kernel is built to stream it once at HBM speed:
+// At decode sizes the packed weights are the whole cost (0.53 B/param for INT4
+// g128), so the kernel is built to stream them once at HBM speed and to pay
+// the fixed costs of a launch (start-up, pipeline fill, the tail of split
+// tiles) once for a whole layer set instead of once per matrix:
 //
-//  * one producer lane streams the CTA's weight rows through a ring of
-//    128-row x 128-byte TMA boxes (128-byte swizzle); large boxes keep the TMA
-//    engine efficient and the ring keeps ~64 KB per CTA in flight without any
-//    load instruction in the compute warps;
+//  * persistent, one wave: two CTAs per SM; every CTA gets an equal share
+//    (in bytes) of the (128-row tile, 64-wide k-block) work of ONE matrix of
+//    the group, contiguous in (tile, k-block) order, so a share may span
+//    several tiles;
+//  * one producer lane fills a ring of stages, each with two TMA copies: one
+//    weight box (128 rows x 128 bytes, 128-byte swizzle) and the matching
+//    activation slice, a 3-D box of (64 k) x (tokens padded to 8 or 16) x
+//    (k-blocks of the weight box), 128-byte swizzle (rows beyond the real
+//    tokens read as zeros).  No prologue stages a CTA's whole slice first;
+//  * each compute warp fetches the per-row constants (scale and zero, or
+//    absmax) of its own 16 rows one weight box ahead, with a few cp.async
+//    into a small buffer of its own, so the constants never wait on memory
+//    and the producer stays a single lane;
 //  * eight compute warps own 16 rows each; a thread owns two rows (r, r+8)
-//    and, per 64-wide k-block, a quarter of each row's bytes.  Products run on
-//    register-resident tensor-core MMAs (mma.sync m16n8k16, bf16 in, fp32
-//    accumulate): rows are the M dimension, tokens (padded to 8 or 16) the N
-//    dimension;
-//  * codes become bf16 with one mask-and-or per two codes (the bf16 number
-//    128 + code), pairing codes that sit 2 bytes apart; the k order inside an
-//    MMA step is whatever pairing the codes have, and the activations staged in
-//    shared memory are permuted the same way, so each activation fragment is
-//    one 8-byte load;
-//  * dequantization is exact: A = bf16(code - zero) (exact for |zero| <= 128;
-//    otherwise bf16(code) with -zero * sum(x) added per group) and the
-//    per-group scale multiplies the fp32 group partial after the group's MMAs
-//    (GreenBit.AI article, 模型量化 (1): a scale and a zero per group).  The
-//    codebook format uses bf16(codebook[code]) times the fp32 per-64 absmax
-//    (QLoRA explainer, 关键技术细节 1).  Each (row, group) constant is
-//    converted once per CTA into a shared-memory table at the start, not by
-//    every lane that uses it;
-//  * stream-K: the grid is a whole number of waves and every CTA gets an equal
-//    contiguous share of the (row tile, k-block) work, spanning at most two
-//    row tiles.  A tile covered by several CTAs is finished by the one that
-//    covers its last k-block (the highest CTA index among them): the others
-//    store their partial sums, count themselves on a per-tile flag and leave
-//    without waiting; the finishing CTA waits for the count (CTAs start in
-//    index order, so its contributors are running or done) and adds the
-//    partials in CTA order, so the result does not depend on scheduling.
+//    and, per k-block, 16 consecutive codes of each.  Products run on
+//    register tensor-core MMAs (mma.sync m16n8k16, bf16 in, fp32 accumulate):
+//    rows are the M dimension, tokens (padded to 8 or 16) the N dimension;
+//  * codes become bf16 pairs in the cheapest order the packing allows: one
+//    logic op turns the two codes that sit two bytes apart in a 32-bit word
+//    into a bf16x2 (each half the number 128 + code): 4-bit codes k and k+4,
+//    2-bit codes k and k+8.  The producer warp's lanes permute each landed
+//    activation box in place to the same order (codebook codes pair
+//    naturally, through a 256-entry table, and their activations stay as
+//    loaded), then release the stage to the compute warps on a second barrier;
+//  * dequantization is exact and its scale comes last (GreenBit.AI article,
+//    模型量化 (1): one scale and one zero per group): with up to 8 tokens the
+//    MMA runs on A = 128 + code (exact in bf16) and, per group, the fold takes
+//    (128 + zero) * sum(x) off each token's fp32 partial before multiplying by
+//    the scale, the per-token sums coming from MMAs with an all-ones A (the
+//    tensor pipe has room for them at this size); with 9..16 tokens A =
+//    (128 + code) - (128 + zero) = code - zero in bf16 (exact for |zero| <=
+//    128; a group where some row's zero is farther out falls back to the
+//    folded form).  The codebook format uses bf16(codebook[code]) times the
+//    fp32 per-64 absmax (QLoRA explainer, 关键技术细节 1);
+//  * a tile covered by several CTAs is finished by the one that covers its
+//    last k-block (the highest CTA index among them): the others store their
+//    fp32 partial sums, count themselves on a per-tile flag and go on; the
+//    finishing CTA processes that tile last, waits for the count (CTAs start
+//    in index order, so its contributors are running or done, and each of
+//    them processes its contributing segment first) and adds the partials in
+//    CTA order, so the result does not depend on scheduling.
 #pragma once
 
 #include <type_traits>
@@ -44,38 +57,57 @@
 
 namespace lbq {
 
-constexpr int kGemvComputeWarps = 8;                            // 16 rows each: 128 rows per tile
-constexpr int kGemvThreads = 32 * (kGemvComputeWarps + 1);      // + one producer warp
-constexpr int kGemvMaxWStages = 4;                              // 16 KB weight boxes in flight (3 or 4)
-constexpr int kGemvTabPerThread = 16;                           // constant-table entries per thread
-constexpr int kGemvMaxTabGroups = 2 * kGemvTabPerThread;        // groups (codebook: k-blocks) per CTA
+constexpr int kGvComputeWarps = 8;                            // 16 rows each: 128 rows per tile
+constexpr int kGvThreads = 32 * (kGvComputeWarps + 1);        // + one producer warp
+constexpr int kGvMaxProblems = 8;                             // matrices per launch
+constexpr int kGvMaxStages = 4;
+constexpr int kGvWBox = 128 * 128;                            // weight box bytes
+constexpr int kGvExtraSmem = 3 * kGvMaxStages * 8 + 16 + 2 * 256 * 4;   // barriers, flags, codebook tables
+constexpr int kGvConstWords = 5;                              // 4-byte words per row and array a box needs (max)
 
-struct GemvParams {
-    int m, n, k;                      // tokens, stored rows, input features
-    int ngroups;                      // k / group (MinMax)
+// One matrix of a grouped launch (everything but its tensor maps).  Each CTA
+// copies its matrix's descriptor into shared memory once, so that the loops
+// read it from there.
+struct GvProblem {
+    const uint16_t* X;                // [m, k] bf16
+    float* Y;                         // Y[t * ldy + out_col]
+    const int32_t* perm;              // stored row -> output column (NULL = identity)
     const uint16_t* scale;            // [n, ngroups] fp16 (MinMax)
     const uint16_t* zero;             // [n, ngroups] fp16 (MinMax)
-    const float* absmax;              // codebook, no double quant
-    const int8_t* q8;                 // codebook, double quant
-    const float* s2;
-    const float* offset;
-    const float* codebook;
-    const uint16_t* X;                // [m, k] bf16
-    int rank;
-    float s;
-    const float* T;                   // [m, rank]
-    const uint16_t* B;                // [n_out, rank]
-    float* Y;
-    int64_t ldy;
-    const int32_t* perm;
-    int kbt;                          // k-blocks per row (k / 64)
-    int tiles;                        // row tiles of 128
-    int share;                        // k-blocks per CTA (<= kbt; a multiple of the scale group)
-    int64_t total;                    // tiles * kbt
-    float* partial;                   // [grid + tiles][m][128]
+    const float* absmax;              // [n * kbt] (codebook, no double quant)
+    const int8_t* q8;                 // [n * kbt] (codebook, double quant)
+    const float* s2;                  // [ceil(n * kbt / 256)]
+    const float* offset;              // [1]
+    const float* codebook;            // [16]
+    const float* T;                   // [m, rank] fp32
+    const uint16_t* B;                // [n_out, rank] bf16, by output column
+    float* partial;                   // [ctas + tiles][m][128] fp32 (split tiles)
     uint32_t* counters;               // [tiles] arrival flags, zero at launch and left at zero
-    int w_early;                      // the packed weight and its constants may be read before the
-                                      // previous kernel on the stream has finished
+    int64_t ldy;
+    int64_t total;                    // tiles * kbt  (< 2^31)
+    int n, k, kind, ngroups, kbt, tiles, share, cta0, rank;
+    int xbytes;                       // bytes of one activation box
+    float s;
+    int pad_;
+};
+
+struct GvParams {
+    CUtensorMap tmW[kGvMaxProblems];  // packed weights [n, k*bits/8] u8, box 128 x 128 B, 128-byte swizzle
+    CUtensorMap tmX[kGvMaxProblems];  // X as (64, m, k/64) bf16, box (64, 8 or 16, k-blocks per weight box)
+    GvProblem prob[kGvMaxProblems];
+    int nprob;
+    int m;                            // tokens, 1..16
+    int ws;                           // ring stages (2..4)
+    int stage_bytes;                  // a multiple of 1024: weight box, then the activation box
+    int cstride;                      // bytes per row of one constant array in a warp's buffer
+    int w_early;                      // weights and constants may be read before the previous kernel ends
+};
+
+template <int KIND>
+struct GvKind {
+    static constexpr int kRowBytes = (KIND == kInt2) ? 16 : 32;   // per row per k-block
+    static constexpr int kSub = 128 / kRowBytes;                  // k-blocks per weight box
+    static constexpr int kGroupBlocks = (KIND == kInt4) ? 2 : 1;  // k-blocks per scale group (codebook: absmax)
 };
 
 // D = A B + C (C = D on entry), one m16n8k16 bf16 MMA with fp32 accumulation.
@@ -97,60 +129,6 @@ __device__ __forceinline__ void mma_m16n8k16_bf16_first(float (&c)[4], uint32_t 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
 }
 
-template <int KIND>
-struct GemvTile {
-    static constexpr int kRowBytes = (KIND == kInt2) ? 16 : 32;        // per row per k-block
-    static constexpr int kThreadBytes = kRowBytes / 4;                 // a quarter row
-    static constexpr int kSub = 128 / kRowBytes;                       // k-blocks per weight box
-    static constexpr int kGroupBlocks = (KIND == kInt4) ? 2 : 1;       // k-blocks per scale group
-    // shared table of per-(group, row) constants, 4 bytes each: MinMax the
-    // bf16 subtrahend 128 + zero (low half) and the fp16 scale (high half);
-    // codebook the fp32 absmax of each (k-block, row)
-    static constexpr int kTabEntry = 4;
-};
-
-// Order of the 16 activations of a 16-wide k group as the MMA steps consume
-// them: step tau reads four consecutive entries (two code pairs).  4-bit
-// MinMax codes pair nibbles two bytes apart (k and k+4 in the group); 2-bit
-// codes pair crumbs two bytes apart (k and k+8); codebook codes pair the two
-// nibbles of one byte (k and k+1, the natural order).
-__device__ __forceinline__ int gemv_xperm(int kind, int p) {
-    constexpr int kPerm4[16] = {1, 5, 0, 4, 3, 7, 2, 6, 9, 13, 8, 12, 11, 15, 10, 14};
-    constexpr int kPerm2[16] = {0, 8, 1, 9, 2, 10, 3, 11, 4, 12, 5, 13, 6, 14, 7, 15};
-    return kind == kInt2 ? kPerm2[p] : kind == kInt4 ? kPerm4[p] : p;
-}
-
-// (a & MASK) | c in one logic op.
-template <uint32_t MASK>
-__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t c) {
-    uint32_t d;
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "n"(MASK), "r"(c));
-    return d;
-}
-
-// Code pairs of one 32-bit word of 4-bit codes (bytes b0..b3 = codes 0..7):
-// P0 = (1, 5), P1 = (0, 4), P2 = (3, 7), P3 = (2, 6), each half the bf16
-// number 128 + code (mg = 0x43004300 is passed in a register).
-__device__ __forceinline__ void int4_pairs(uint32_t w, uint32_t mg, uint32_t* o) {
-    o[0] = and_or<0x000F000Fu>(w, mg);
-    o[1] = and_or<0x000F000Fu>(w >> 4, mg);
-    o[2] = and_or<0x000F000Fu>(w >> 8, mg);
-    o[3] = and_or<0x000F000Fu>(w >> 12, mg);
-}
-
-// Code pairs of one 32-bit word of 2-bit codes (bytes b0..b3 = codes 0..15,
-// first code in the top bits): pair t = (t, t + 8), t = 0..7.
-__device__ __forceinline__ void int2_pairs(uint32_t w, uint32_t mg, uint32_t* o) {
-    o[0] = and_or<0x00030003u>(w >> 6, mg);
-    o[1] = and_or<0x00030003u>(w >> 4, mg);
-    o[2] = and_or<0x00030003u>(w >> 2, mg);
-    o[3] = and_or<0x00030003u>(w, mg);
-    o[4] = and_or<0x00030003u>(w >> 14, mg);
-    o[5] = and_or<0x00030003u>(w >> 12, mg);
-    o[6] = and_or<0x00030003u>(w >> 10, mg);
-    o[7] = and_or<0x00030003u>(w >> 8, mg);
-}
-
 // a - b on both bf16 halves (exact here: integers of at most 9 bits).
 __device__ __forceinline__ uint32_t sub_bf16x2(uint32_t a, uint32_t b) {
     uint32_t d;
@@ -158,490 +136,539 @@ __device__ __forceinline__ uint32_t sub_bf16x2(uint32_t a, uint32_t b) {
     return d;
 }
 
-__device__ __forceinline__ uint2 gemv_lds64(uint32_t addr) {
+__device__ __forceinline__ uint2 gv_lds64(uint32_t addr) {
     uint2 v;
     asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
     return v;
 }
 
-__device__ __forceinline__ uint32_t gemv_lds32(uint32_t addr) {
+__device__ __forceinline__ uint4 gv_lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t gv_lds32(uint32_t addr) {
     uint32_t v;
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
     return v;
 }
 
-// Split-tile flags: a contributor publishes its partial sums (stored by all
-// threads of the CTA before the barrier that precedes this call) and counts
-// itself; the finishing CTA waits for the count with acquire semantics.
-__device__ __forceinline__ void flag_publish(uint32_t* f) {
-    asm volatile("fence.acq_rel.gpu;\n\tred.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(f) : "memory");
-}
-
-__device__ __forceinline__ uint32_t flag_load_acquire(const uint32_t* f) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+__device__ __forceinline__ uint16_t gv_lds16(uint32_t addr) {
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
     return v;
 }
 
-// Bounded wait for *f >= want; records kStatusTimeout and returns false when
-// it gives up.
-__device__ __forceinline__ bool flag_wait_geq(const uint32_t* f, uint32_t want) {
-    if (flag_load_acquire(f) >= want) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 0; it < kWaitLimitIters; ++it) {
-        __nanosleep(64);
-        if (flag_load_acquire(f) >= want) return true;
-        if ((it & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) break;
-    }
-    record_status(kStatusTimeout);
-    return false;
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 
-template <int KIND, int NTOK, int WS>
-__global__ void __launch_bounds__(kGemvThreads, 2)
-dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
-    constexpr int NT8 = NTOK / 8;
-    constexpr int GB = GemvTile<KIND>::kGroupBlocks;
-    constexpr int SUB = GemvTile<KIND>::kSub;
-    constexpr int RB = GemvTile<KIND>::kRowBytes;
-    constexpr int TB = GemvTile<KIND>::kThreadBytes;
-    constexpr int TE = GemvTile<KIND>::kTabEntry;
-    constexpr int TW = TB / 4;                                    // code words per row, k-block and thread
-    static_assert(WS >= 2 && WS <= kGemvMaxWStages, "weight ring depth");
-    constexpr int kWBox = 128 * 128;
-    constexpr int kCompute = 32 * kGemvComputeWarps;
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
 
+// The mbarrier receives one arrival once every cp.async this thread issued so
+// far has landed (the arrival is one of the barrier's expected count).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// One segment of a CTA's share: k-blocks [ka, kb) of row tile `tile`.
+struct GvSeg {
+    int tile, ka, kb;
+};
+
+// A CTA's share: units [u0, u1) of (tile, k-block) in tile-major order, over
+// row tiles tA..tB.
+struct GvShare {
+    int64_t u0, u1;
+    int tA, tB, nseg, kbt;
+};
+
+// Segment si (0 .. nseg-1) in processing order: the share's last tile first
+// (where the CTA contributes to a tile that a later CTA finishes), then the
+// whole tiles, then the first tile (which this CTA finishes when it does not
+// start it).
+__device__ __forceinline__ GvSeg gv_segment(const GvShare& sh, int si) {
+    GvSeg s;
+    s.tile = sh.nseg == 1 ? sh.tA : (si == 0 ? sh.tB : (si == sh.nseg - 1 ? sh.tA : sh.tA + si));
+    s.ka = s.tile == sh.tA ? static_cast<int>(sh.u0 - static_cast<int64_t>(sh.tA) * sh.kbt) : 0;
+    s.kb = s.tile == sh.tB ? static_cast<int>(sh.u1 - static_cast<int64_t>(sh.tB) * sh.kbt) : sh.kbt;
+    return s;
+}
+
+// Calls fn(box index, tile, first k-block, k-blocks) for the CTA's weight
+// boxes in processing order until fn returns false.  The producer and the
+// compute warps walk the same sequence.
+template <int SUB, typename F>
+__device__ __forceinline__ void gv_for_each_box(const GvShare& sh, F&& fn) {
+    int c = 0;
+    for (int si = 0; si < sh.nseg; ++si) {
+        const GvSeg sg = gv_segment(sh, si);
+        for (int kbs = sg.ka; kbs < sg.kb; kbs += SUB, ++c)
+            if (!fn(c, sg.tile, kbs, min(SUB, sg.kb - kbs))) return;
+    }
+}
+
+// ----------------------------------------------------------------------------
+// producer lane
+// ----------------------------------------------------------------------------
+// One stage: the weight box and the activation box of k-blocks [kbs, kbs +
+// kSub) of row tile `tile`, both arriving on `full` (one expected arrival
+// plus their bytes).  The weights (and the arrival) may be issued before the
+// previous kernel on the stream has finished; the activations only after.
+template <int KIND>
+__device__ __forceinline__ void gv_issue_weights(const CUtensorMap* tmW, int xbytes, uint8_t* stage, uint64_t* full,
+                                                 int tile, int kbs) {
+    mbar_arrive_expect_tx(full, kGvWBox + xbytes);
+    tma_load_2d(stage, tmW, full, kbs * GvKind<KIND>::kRowBytes, tile * 128);
+}
+
+__device__ __forceinline__ void gv_issue_acts(const CUtensorMap* tmX, uint8_t* stage, uint64_t* full, int kbs) {
+    tma_load_3d(stage + kGvWBox, tmX, full, 0, 0, kbs);
+}
+
+// A walk over the CTA's weight boxes in processing order.
+struct GvBoxCursor {
+    const GvShare* sh;
+    int sub, si, kbs;
+    GvSeg sg;
+    bool valid;
+    __device__ __forceinline__ void start(const GvShare& s, int sub_) {
+        sh = &s;
+        sub = sub_;
+        si = 0;
+        valid = s.nseg > 0;
+        if (valid) {
+            sg = gv_segment(s, 0);
+            kbs = sg.ka;
+        }
+    }
+    __device__ __forceinline__ void next() {
+        kbs += sub;
+        if (kbs >= sg.kb) {
+            if (++si < sh->nseg) {
+                sg = gv_segment(*sh, si);
+                kbs = sg.ka;
+            } else {
+                valid = false;
+            }
+        }
+    }
+};
+
+// Puts the activations of a landed box (the m real token rows of its kSub
+// k-blocks) in the order of the weight-code pairs: within 8 consecutive k
+// (4-bit) the pairs (1,5) (0,4) (3,7) (2,6); within 16 (2-bit) the pairs
+// (t, t+8).  Rows are 128-byte lines swizzled with the token (kSub * 8 or
+// 16 rows per k-block, so the row's swizzle is the token's).
+template <int KIND>
+__device__ __forceinline__ void gv_permute_acts(uint8_t* xbox, int m, int mpad, int lane) {
+    constexpr int SUB = GvKind<KIND>::kSub;
+    const uint32_t base = smem_u32(xbox);
+    for (int s = 0; s < SUB; ++s) {
+        if (KIND == kInt4) {
+            for (int e = lane; e < m * 8; e += 32) {
+                const int t = e >> 3, u = e & 7;
+                const uint32_t a = base + (s * mpad + t) * 128 + ((u ^ (t & 7)) << 4);
+                const uint4 v = gv_lds128(a);
+                const uint4 o = make_uint4(__byte_perm(v.x, v.z, 0x7632), __byte_perm(v.x, v.z, 0x5410),
+                                           __byte_perm(v.y, v.w, 0x7632), __byte_perm(v.y, v.w, 0x5410));
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(o.x), "r"(o.y), "r"(o.z),
+                             "r"(o.w)
+                             : "memory");
+            }
+        } else {
+            for (int e = lane; e < m * 4; e += 32) {
+                const int t = e >> 2, up = e & 3;
+                const uint32_t row = base + (s * mpad + t) * 128;
+                const uint32_t a0 = row + (((2 * up) ^ (t & 7)) << 4), a1 = row + (((2 * up + 1) ^ (t & 7)) << 4);
+                const uint4 v = gv_lds128(a0), w = gv_lds128(a1);
+                const uint4 o0 = make_uint4(__byte_perm(v.x, w.x, 0x5410), __byte_perm(v.x, w.x, 0x7632),
+                                            __byte_perm(v.y, w.y, 0x5410), __byte_perm(v.y, w.y, 0x7632));
+                const uint4 o1 = make_uint4(__byte_perm(v.z, w.z, 0x5410), __byte_perm(v.z, w.z, 0x7632),
+                                            __byte_perm(v.w, w.w, 0x5410), __byte_perm(v.w, w.w, 0x7632));
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a0), "r"(o0.x), "r"(o0.y), "r"(o0.z),
+                             "r"(o0.w)
+                             : "memory");
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a1), "r"(o1.x), "r"(o1.y), "r"(o1.z),
+                             "r"(o1.w)
+                             : "memory");
+            }
+        }
+    }
+}
+
+// The producer warp: lane 0 issues the TMA copies, kept ws boxes ahead; the
+// warp permutes each box's activations once it has landed and releases the
+// stage on xready.  Box c's slot is refilled (with box c + ws) once the
+// compute warps have released it, after box c + 1 has been released to them.
+template <int KIND>
+__device__ __forceinline__ void gv_produce(const GvParams& p, const CUtensorMap* tmW, const CUtensorMap* tmX,
+                                           int xbytes, const GvShare& sh, uint8_t* ring, uint64_t* full,
+                                           uint64_t* xready, uint64_t* empty, volatile int* s_abort, int lane) {
+    constexpr int SUB = GvKind<KIND>::kSub;
+    const int ws = p.ws, mpad = p.m <= 8 ? 8 : 16;
+    GvBoxCursor ic;                                          // next box to issue
+    ic.start(sh, SUB);
+    int nissued = 0;
+    if (p.w_early) {
+        // the ring's weights before the previous kernel on the stream has
+        // finished; the activations only after it has
+        GvBoxCursor pre = ic;
+        for (int c = 0; pre.valid && c < ws; ++c, pre.next())
+            if (lane == 0) gv_issue_weights<KIND>(tmW, xbytes, ring + c * p.stage_bytes, &full[c], pre.sg.tile, pre.kbs);
+        griddep_wait();
+        for (; ic.valid && nissued < ws; ++nissued, ic.next())
+            if (lane == 0) gv_issue_acts(tmX, ring + nissued * p.stage_bytes, &full[nissued], ic.kbs);
+    } else {
+        griddep_wait();
+        for (; ic.valid && nissued < ws; ++nissued, ic.next()) {
+            if (lane == 0) {
+                gv_issue_weights<KIND>(tmW, xbytes, ring + nissued * p.stage_bytes, &full[nissued], ic.sg.tile, ic.kbs);
+                gv_issue_acts(tmX, ring + nissued * p.stage_bytes, &full[nissued], ic.kbs);
+            }
+        }
+    }
+    GvBoxCursor pc;                                          // next box to release
+    pc.start(sh, SUB);
+    for (int c = 0; pc.valid; ++c, pc.next()) {
+        const int w = c % ws;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[w], (c / ws) & 1, s_abort))) break;
+        uint8_t* stage = ring + w * p.stage_bytes;
+        if (KIND != kCode4) {
+            gv_permute_acts<KIND>(stage + kGvWBox, p.m, mpad, lane);
+            fence_proxy_async_smem();                        // before the next TMA write to this stage
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xready[w]);
+        if (c >= 1 && ic.valid) {
+            const int wp = (c - 1) % ws;
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[wp], ((c - 1) / ws) & 1, s_abort))) break;
+            if (lane == 0) {
+                gv_issue_weights<KIND>(tmW, xbytes, ring + wp * p.stage_bytes, &full[wp], ic.sg.tile, ic.kbs);
+                gv_issue_acts(tmX, ring + wp * p.stage_bytes, &full[wp], ic.kbs);
+            }
+            ic.next();
+            ++nissued;
+        }
+    }
+    // never leave with a copy in flight (matters only after an abort)
+    if (lane == 0)
+        for (int i = max(0, nissued - ws); i < nissued; ++i) mbar_wait_drain(&full[i % ws], (i / ws) & 1);
+    __syncwarp();
+}
+
+// ----------------------------------------------------------------------------
+// per-warp constants
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// The raw constants of one box for the warp's 16 rows into one of its two
+// buffer slots: lane (row lr = lane % 16, array lane / 16) copies the 4-byte
+// words that cover the row's entries (MinMax: scale, zero; codebook: absmax,
+// or q8 and s2).  A row's entries may start at an odd 2-byte (or 1-byte)
+// position in its first word; the readers account for it.
+template <int KIND>
+__device__ __forceinline__ void gv_fetch_consts(const GvProblem& P, uint32_t slot, int cstride, int tile, int kbs,
+                                                int nk, int warp, int lane) {
+    constexpr int GB = GvKind<KIND>::kGroupBlocks;
+    const int lr = lane & 15, arr = lane >> 4;
+    const int64_t grow = static_cast<int64_t>(tile) * 128 + warp * 16 + lr;
+    if (grow >= P.n) return;
+    const uint32_t d = slot + (arr * 16 + lr) * cstride;
+    if (KIND != kCode4) {
+        const int g0 = kbs / GB, ng = (nk + GB - 1) / GB;
+        const int64_t e0 = grow * P.ngroups + g0;
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(arr ? P.zero : P.scale);
+        const int64_t w0 = e0 >> 1, w1 = (e0 + ng - 1) >> 1;
+        for (int64_t w = w0; w <= w1; ++w) cp_async4(d + static_cast<uint32_t>(w - w0) * 4, src + w);
+    } else if (P.q8 == nullptr) {
+        if (arr == 0) {
+            const int64_t e0 = grow * P.kbt + kbs;
+            for (int i = 0; i < nk; ++i) cp_async4(d + 4 * i, P.absmax + e0 + i);
+        }
+    } else {
+        const int64_t e0 = grow * P.kbt + kbs, e1 = e0 + nk - 1;
+        if (arr == 0) {
+            const uint32_t* q32 = reinterpret_cast<const uint32_t*>(P.q8);
+            cp_async4(d, q32 + (e0 >> 2));
+            if ((e1 >> 2) != (e0 >> 2)) cp_async4(d + 4, q32 + (e1 >> 2));
+        } else {
+            cp_async4(d, P.s2 + (e0 >> 8));
+            if ((e1 >> 8) != (e0 >> 8)) cp_async4(d + 4, P.s2 + (e1 >> 8));
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------
+// compute warps
+// ----------------------------------------------------------------------------
+template <int KIND, int NT8>
+__device__ __forceinline__ void gv_compute(const GvParams& p, const GvProblem& P, const GvShare& sh, int b,
+                                           uint8_t* ring, uint64_t* xready, uint64_t* empty, volatile int* s_abort,
+                                           uint8_t* cbuf, const uint32_t* s_lut, const float* s_q8lut) {
+    using G = GvKind<KIND>;
+    constexpr int SUB = G::kSub, RB = G::kRowBytes, GB = G::kGroupBlocks;
+    constexpr int TB = RB / 4;                         // code bytes per thread, row and k-block
+    constexpr int MPAD = NT8 * 8;                      // token rows of an activation box
+    // MinMax with up to 8 tokens: A = 128 + code, the zero folded at the group's end
+    constexpr bool kFold = KIND != kCode4 && NT8 == 1;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // let the next kernel on the stream be scheduled as soon as our CTAs leave
-    griddep_launch_dependents();
-    if (tid == kCompute) tma_prefetch_desc(&tmW);
-
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    // 1024-byte alignment for the swizzled boxes, by pointer arithmetic on the
-    // shared array so that every access below stays a shared-memory access
-    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint8_t* sW = smem;                                           // WS x 16 KB
-    const int xstride = p.share * 64 + 4;                         // bf16 per token row (+8 bytes)
-    // token rows, plus a zero row m when the token tile has padding lanes
-    const int xrows = p.m < NTOK ? p.m + 1 : p.m;
-    uint16_t* sX = reinterpret_cast<uint16_t*>(smem + WS * kWBox);          // [xrows][xstride]
-    // constant table [128 rows][tstride]: an odd row stride keeps the eight
-    // rows that a warp reads at once in distinct banks
-    const int tstride = (p.share / GB) | 1;
-    uint8_t* sTab = reinterpret_cast<uint8_t*>(sX + xrows * xstride);
-    uint32_t* s_lut = reinterpret_cast<uint32_t*>(sTab + 128 * tstride * TE);     // codebook pairs [256]
-    uint64_t* full = reinterpret_cast<uint64_t*>(s_lut + (KIND == kCode4 ? 256 : 0));
-    uint64_t* empty = full + WS;
-    int* s_misc = reinterpret_cast<int*>(empty + WS);
-    volatile int* s_abort = s_misc;
-    int* s_far = s_misc + 1;
-
-    // this CTA's work: up to two (tile, first k-block, k-blocks) segments
-    // (tiles * kbt < 2^31, checked by the host)
-    int t0 = 0, a0 = 0, n0 = 0, n1 = 0;
-    {
-        const uint32_t u0 = blockIdx.x * static_cast<uint32_t>(p.share);
-        const uint32_t tot = static_cast<uint32_t>(p.total);
-        const uint32_t u1 = u0 + p.share < tot ? u0 + p.share : tot;
-        if (u0 < u1) {
-            t0 = static_cast<int>(u0 / static_cast<uint32_t>(p.kbt));
-            a0 = static_cast<int>(u0 - static_cast<uint32_t>(t0) * p.kbt);
-            n0 = min(static_cast<int>(u1 - u0), p.kbt - a0);
-            n1 = static_cast<int>(u1 - u0) - n0;
-        }
-    }
-    const int nseg = n0 == 0 ? 0 : (n1 == 0 ? 1 : 2);
-    const int nk = n0 + n1;
-    // the second segment (the start of tile t0 + 1) is processed first: its
-    // partial sums are published before this CTA waits on anything, so the
-    // CTAs that finish tiles never wait on each other in a chain
-    const int nbox1 = (n1 + SUB - 1) / SUB;
-    const int nbox = nbox1 + (n0 + SUB - 1) / SUB;
-
-    // the producer lane issues the first weight box at once; the rest of the
-    // ring fills only after the compute threads have issued their loads
-    // (small scattered loads queued behind megabytes of weight boxes come
-    // back microseconds late)
-    auto issue_box = [&](int c) {
-        const int w = c % WS;
-        mbar_arrive_expect_tx(&full[w], kWBox);
-        const int x = c < nbox1 ? c * SUB * RB : (a0 + (c - nbox1) * SUB) * RB;
-        const int y = (c < nbox1 ? t0 + 1 : t0) * 128;
-        tma_load_2d(sW + w * kWBox, &tmW, &full[w], x, y);
-    };
-    if (tid == kCompute) {
-        for (int i = 0; i < WS; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], kGemvComputeWarps);
-        }
-        *s_abort = 0;
-        *s_far = 0;
-        fence_mbar_init();
-        if (!p.w_early) griddep_wait();
-        if (nbox > 0) issue_box(0);
-    }
-    // prologue, first half (compute threads): issue the global loads of this
-    // CTA's constants and of its first activation round, so that they reach
-    // memory ahead of all but the first weight box
-    const int ngr16 = nk * 4;                                      // 16-wide k groups of the slice
-    const int xtotal = p.m * ngr16;
-    constexpr int XU = (KIND == kCode4) ? 2 : 4;                  // activation loads in flight per round
-    const int G = nk / GB, G0 = n0 / GB;                           // table groups (codebook: k-blocks)
-    // table entry (row rl, group lg) of thread (warp w, lane) and slot u = 2 it + ch:
-    // rl = 16 w + 2 it + lane / 16, lg = lane % 16 + 16 ch (coalesced along the row)
-    uint32_t raw[kGemvTabPerThread], raw2[kGemvTabPerThread];
-    uint4 v[XU][2];
-    if (tid < kCompute) {
-        // the weight's constants may be read early; the activations (and the
-        // workspace, Y, T) only after the previous kernel has finished
-        if (!p.w_early) griddep_wait();
-#pragma unroll
-        for (int u = 0; u < kGemvTabPerThread; ++u) {
-            const int rl = 16 * warp + 2 * (u >> 1) + (lane >> 4), lg = (lane & 15) + 16 * (u & 1);
-            raw[u] = 0u;
-            raw2[u] = 0u;
-            if (lg < G) {
-                const bool sb = lg >= G0;
-                const int64_t r = static_cast<int64_t>(sb ? t0 + 1 : t0) * 128 + rl;
-                const int gl = sb ? lg - G0 : a0 / GB + lg;            // group (codebook: k-block) in the row
-                // plain loads only: no arithmetic on a loaded value before the
-                // barrier below, or the thread would wait for the data there
-                if (r < p.n) {
-                    if (KIND != kCode4) {
-                        raw[u] = __ldg(p.scale + r * p.ngroups + gl);
-                        raw2[u] = __ldg(p.zero + r * p.ngroups + gl);
-                    } else if (p.q8 != nullptr) {
-                        const int64_t bi = r * p.kbt + gl;
-                        raw[u] = __ldg(reinterpret_cast<const uint8_t*>(p.q8) + bi);
-                        raw2[u] = __float_as_uint(__ldg(p.s2 + (bi >> 8)));
-                    } else {
-                        raw[u] = __float_as_uint(__ldg(p.absmax + r * p.kbt + gl));
-                    }
-                }
-            }
-        }
-        if (p.w_early) griddep_wait();
-#pragma unroll
-        for (int u = 0; u < XU; ++u) {
-            const int e = tid + u * kCompute;
-            if (e < xtotal) {
-                const int t = e / ngr16, g16 = e - t * ngr16;
-                const int lk = g16 >> 2;
-                const int kb = lk < n0 ? a0 + lk : lk - n0;
-                const uint4* src = reinterpret_cast<const uint4*>(p.X + static_cast<int64_t>(t) * p.k + kb * 64 +
-                                                                  (g16 & 3) * 16);
-                v[u][0] = __ldg(src);
-                v[u][1] = __ldg(src + 1);
-            }
-        }
-    }
-
-    __syncthreads();
-
-    if (warp == kGemvComputeWarps) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0 && nbox > 0) {
-            int issued = 1;
-            for (int c = 1; c < nbox; ++c) {
-                if (c >= WS && !mbar_wait(&empty[c % WS], ((c / WS) - 1) & 1, s_abort)) break;
-                issue_box(c);
-                issued = c + 1;
-            }
-            for (int c = max(0, issued - WS); c < issued; ++c) mbar_wait_drain(&full[c % WS], (c / WS) & 1);
-        }
-        return;
-    }
-
-    // ---------------------------------------------------------------- compute warps
-    // prologue, second half: store the activations, convert the constants
-    // (the empty asm keeps every use of the loaded values after the barrier)
-#pragma unroll
-    for (int u = 0; u < kGemvTabPerThread; ++u) asm volatile("" : "+r"(raw[u]), "+r"(raw2[u]));
-#pragma unroll
-    for (int u = 0; u < XU; ++u)
-        asm volatile("" : "+r"(v[u][0].x), "+r"(v[u][0].y), "+r"(v[u][0].z), "+r"(v[u][0].w), "+r"(v[u][1].x),
-                     "+r"(v[u][1].y), "+r"(v[u][1].z), "+r"(v[u][1].w));
-    {
-        // activations of the m real tokens, permuted to the MMA step order
-        for (int e0 = tid; e0 < xtotal; e0 += XU * kCompute) {
-            if (e0 != tid) {
-#pragma unroll
-                for (int u = 0; u < XU; ++u) {
-                    const int e = e0 + u * kCompute;
-                    if (e < xtotal) {
-                        const int t = e / ngr16, g16 = e - t * ngr16;
-                        const int lk = g16 >> 2;
-                        const int kb = lk < n0 ? a0 + lk : lk - n0;
-                        const uint4* src = reinterpret_cast<const uint4*>(p.X + static_cast<int64_t>(t) * p.k +
-                                                                          kb * 64 + (g16 & 3) * 16);
-                        v[u][0] = __ldg(src);
-                        v[u][1] = __ldg(src + 1);
-                    }
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < XU; ++u) {
-                const int e = e0 + u * kCompute;
-                if (e < xtotal) {
-                    const int t = e / ngr16, g16 = e - t * ngr16;
-                    const uint32_t w8[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
-                                            v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
-                    uint16_t in[16];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        in[2 * q] = static_cast<uint16_t>(w8[q] & 0xFFFFu);
-                        in[2 * q + 1] = static_cast<uint16_t>(w8[q] >> 16);
-                    }
-                    // rows are 8-byte aligned (stride 128 * share + 8 bytes)
-                    uint2* d2 = reinterpret_cast<uint2*>(sX + t * xstride + g16 * 16);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        d2[q] = make_uint2(static_cast<uint32_t>(in[gemv_xperm(KIND, 4 * q)]) |
-                                               (static_cast<uint32_t>(in[gemv_xperm(KIND, 4 * q + 1)]) << 16),
-                                           static_cast<uint32_t>(in[gemv_xperm(KIND, 4 * q + 2)]) |
-                                               (static_cast<uint32_t>(in[gemv_xperm(KIND, 4 * q + 3)]) << 16));
-                }
-            }
-        }
-        // convert the constants into the table
-        const float dq_off = (KIND == kCode4 && p.q8 != nullptr) ? __ldg(p.offset) : 0.0f;
-#pragma unroll
-        for (int u = 0; u < kGemvTabPerThread; ++u) {
-            const int rl = 16 * warp + 2 * (u >> 1) + (lane >> 4), lg = (lane & 15) + 16 * (u & 1);
-            if (lg < G) {
-                if (KIND != kCode4) {
-                    const uint16_t s16 = static_cast<uint16_t>(raw[u]), z16 = static_cast<uint16_t>(raw2[u]);
-                    const float zf = f16_bits_to_f32(z16);
-                    uint32_t word;
-                    if (fabsf(zf) <= 128.0f) {
-                        // (128 + q) - (128 + z) = q - z exactly
-                        word = pack_bf16x2_rn(128.0f + zf, 0.0f) & 0xFFFFu;
-                    } else {
-                        // (128 + q) - 128 = q; the zero is added after the loop
-                        word = 0x4300u;
-                        *s_far = 1;
-                    }
-                    *reinterpret_cast<uint32_t*>(sTab + (rl * tstride + lg) * 4) =
-                        word | (static_cast<uint32_t>(s16) << 16);
-                } else {
-                    float am = __uint_as_float(raw[u]);
-                    if (p.q8 != nullptr)
-                        am = __fadd_rn(__fmul_rn(__fdiv_rn(static_cast<float>(static_cast<int8_t>(static_cast<uint8_t>(raw[u]))), 127.0f),
-                                                 __uint_as_float(raw2[u])),
-                                       dq_off);
-                    *reinterpret_cast<float*>(sTab + (rl * tstride + lg) * 4) = am;
-                }
-            }
-        }
-        // row m: zeros, read by the lanes of tokens >= m
-        if (p.m < NTOK)
-            for (int e = tid; e < xstride / 2; e += kCompute)
-                reinterpret_cast<uint32_t*>(sX + p.m * xstride)[e] = 0u;
-        if (KIND == kCode4) {
-            for (int e = tid; e < 256; e += kCompute) {
-                // byte e = (first code << 4) | second code -> (codebook[first], codebook[second])
-                s_lut[e] = pack_bf16x2_rn(p.codebook[e >> 4], p.codebook[e & 15]);
-            }
-        }
-    }
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-
     const int j = lane & 3;                            // quarter of the row's bytes
     const int g = lane >> 2;                           // MMA row in the 8-row half, token in the n8 tile
+    const int m = p.m;
     // MMA row g is weight row pi(g) of the warp's first 8 (pi interleaves even
     // rows into lanes 0-15 and odd rows into lanes 16-31, so that each half
     // warp's 8-byte reads of the 128-byte-swizzled lines hit 32 distinct banks)
-    const int rl0 = warp * 16 + (g & 3) * 2 + (g >> 2); // local rows rl0, rl0 + 8
-    const int sw = rl0 & 7;                            // swizzle of both rows' lines
-    uint32_t offs[SUB];                                // this thread's bytes of sub-block s in the line
+    const int lr0 = (g & 3) * 2 + (g >> 2);                 // warp-local rows lr0, lr0 + 8
+    const int rl0 = warp * 16 + lr0;                        // tile rows rl0, rl0 + 8
+    const int sw = rl0 & 7;                                 // swizzle of both rows' lines
+    uint32_t offs[SUB];                                     // this thread's bytes of k-block s in the line
 #pragma unroll
     for (int s = 0; s < SUB; ++s) {
         const int off = s * RB + TB * j;
         offs[s] = static_cast<uint32_t>((((off >> 4) ^ sw) << 4) | (off & 15));
     }
-    const uint32_t wrow = smem_u32(sW) + rl0 * 128;
-    const uint32_t trow = smem_u32(sTab) + rl0 * tstride * TE;   // table row rl0 (row rl0 + 8: + 8 tstride TE)
-    // B fragments: token nt * 8 + g; lanes of tokens >= m read the zero row
-    // (a select per load would cost more than the loads themselves)
-    uint32_t xthr[NT8];
+    // B fragments of token nt * 8 + g (a zero row beyond the real tokens):
+    // row (s * MPAD + token) of the activation box, 16-byte units 2j and
+    // 2j + 1 of its 128-byte line, swizzled with the row (s * MPAD is a
+    // multiple of 8, so the swizzle is the token's)
+    uint32_t xoff[NT8];
 #pragma unroll
     for (int nt = 0; nt < NT8; ++nt) {
-        const int tok = nt * 8 + g < p.m ? nt * 8 + g : p.m;
-        xthr[nt] = smem_u32(sX) + static_cast<uint32_t>(tok * xstride + 16 * j) * 2;
+        const int tok = nt * 8 + g;
+        xoff[nt] = static_cast<uint32_t>(kGvWBox + tok * 128 + (((2 * j) ^ (tok & 7)) << 4));
     }
-    const bool far = *s_far != 0;                      // some group of this CTA has |zero| > 128
-    uint32_t mg = 0x43004300u;
-    asm volatile("" : "+r"(mg));                       // keep the magic in a register
+    const float dq_off = (KIND == kCode4 && P.q8 != nullptr) ? __ldg(P.offset) : 0.0f;
+    const uint32_t ones = 0x3F803F80u;                       // bf16x2 (1, 1)
+    uint32_t mg = 0x43004300u;                               // bf16x2 (128, 128), kept in a register
+    asm volatile("" : "+r"(mg));
+    // this warp's two constant slots; rows lr0 and lr0 + 8 of array 0 / 1
+    const uint32_t cslot0 = smem_u32(cbuf) + warp * (2 * 32 * p.cstride);
+    const uint32_t cslot_bytes = 32 * p.cstride;
+    const uint32_t zoff = 16 * p.cstride;
 
-    uint32_t c = 0;                                    // weight boxes consumed (matches the producer)
-    // (after a timed-out wait every warp still runs both segments' barriers)
-    for (int si = 0; si < nseg; ++si) {
-        const int sgi = nseg - 1 - si;                 // segment 1 (if any) first, then segment 0
-        const int tile = sgi == 0 ? t0 : t0 + 1;
-        const int kb0 = sgi == 0 ? a0 : 0;
-        const int nkb = sgi == 0 ? n0 : n1;
-        const int lk0 = sgi == 0 ? 0 : n0;             // first local k-block of the segment
+    // the first box's constants; nothing global is written before the
+    // previous kernel on the stream has finished
+    {
+        const GvSeg s0 = gv_segment(sh, 0);
+        if (!p.w_early) griddep_wait();
+        gv_fetch_consts<KIND>(P, cslot0, p.cstride, s0.tile, s0.ka, min(SUB, s0.kb - s0.ka), warp, lane);
+        cp_async_commit();
+        if (p.w_early) griddep_wait();
+    }
+
+    bool live = true;                                        // false after a timed-out wait
+    int c = 0;                                               // boxes consumed (matches the producer)
+    // (after a timed-out wait every warp still runs every segment's barriers)
+    for (int si = 0; si < sh.nseg; ++si) {
+        const GvSeg sg = gv_segment(sh, si);
+        const int tile = sg.tile;
         const int64_t gr0 = static_cast<int64_t>(tile) * 128 + rl0, gr1 = gr0 + 8;
-        const bool ok0 = gr0 < p.n, ok1 = gr1 < p.n;
-        // group partials in two chains (even and odd MMA steps), folded per group
-        float acc[NT8][4], cg[2][NT8][4];
+        const bool ok0 = gr0 < P.n, ok1 = gr1 < P.n;
+        // per-token activation sums sx; with the folded zero they are kept in
+        // the same two chains as the group partials cg, so that (128 + zero)
+        // * sum(x) cancels the code-independent part of cg exactly when 128 +
+        // zero is a power of two (an all-zero row gives exactly 0)
+        constexpr int SXC = kFold ? 2 : 1;
+        float acc[NT8][4], cg[2][NT8][4], sx[SXC][NT8][4];
 #pragma unroll
         for (int nt = 0; nt < NT8; ++nt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[nt][e] = cg[0][nt][e] = cg[1][nt][e] = 0.0f;
-        uint32_t sub0 = 0x43004300u, sub1 = 0x43004300u;
-        float sf0 = 1.0f, sf1 = 1.0f;
-
-        const int nbx = (nkb + SUB - 1) / SUB;
-        const int nfull = nkb / SUB;                      // boxes whose SUB k-blocks all belong to the segment
-        // one box of k-blocks; the per-k-block bounds test is compiled only
-        // into the copy used for a partial last box (it costs ~15% of the loop)
-        auto run_box = [&](auto partial_tag, int bx, uint32_t w) {
-            constexpr bool kPartial = decltype(partial_tag)::value;
-            const uint32_t base = wrow + w * kWBox;
+            for (int e = 0; e < 4; ++e) {
+                acc[nt][e] = cg[0][nt][e] = cg[1][nt][e] = 0.0f;
+#pragma unroll
+                for (int ch = 0; ch < SXC; ++ch) sx[ch][nt][e] = 0.0f;
+            }
+        for (int kbs = sg.ka; kbs < sg.kb; kbs += SUB, ++c) {
+            // the next box's constants into the other slot
+            if (kbs + SUB < sg.kb) {
+                gv_fetch_consts<KIND>(P, cslot0 + ((c + 1) & 1) * cslot_bytes, p.cstride, tile, kbs + SUB,
+                                      min(SUB, sg.kb - kbs - SUB), warp, lane);
+            } else if (si + 1 < sh.nseg) {
+                const GvSeg sn = gv_segment(sh, si + 1);
+                gv_fetch_consts<KIND>(P, cslot0 + ((c + 1) & 1) * cslot_bytes, p.cstride, sn.tile, sn.ka,
+                                      min(SUB, sn.kb - sn.ka), warp, lane);
+            }
+            cp_async_commit();
+            cp_async_wait_1();                               // this box's constants (this lane's copies)
+            __syncwarp();                                    // ... and the other lanes'
+            const int w = c % p.ws;
+            // warp-uniform: the warp's later shuffles and MMAs need all 32 lanes
+            const bool got = live && mbar_wait(&xready[w], (c / p.ws) & 1, s_abort);
+            live = __all_sync(0xFFFFFFFFu, got);
+            if (!live) continue;
+            const int nk = min(SUB, sg.kb - kbs);
+            const uint32_t stage = smem_u32(ring + w * p.stage_bytes);
+            const uint32_t wrow = stage + rl0 * 128;
+            const uint32_t cs = cslot0 + (c & 1) * cslot_bytes;
+            const uint32_t ca0 = cs + lr0 * p.cstride, ca1 = cs + (lr0 + 8) * p.cstride;
+            // entry parity of the rows' first constant word (MinMax)
+            int par0 = 0, par1 = 0;
+            if (KIND != kCode4) {
+                const int g0 = kbs / GB;
+                par0 = static_cast<int>((gr0 * P.ngroups + g0) & 1);
+                par1 = static_cast<int>((gr1 * P.ngroups + g0) & 1);
+            }
+            uint32_t sub0 = 0x43004300u, sub1 = 0x43004300u;
+            float sf0 = 1.0f, sf1 = 1.0f, zf0 = 0.0f, zf1 = 0.0f;
+            bool far = false;
 #pragma unroll
             for (int s = 0; s < SUB; ++s) {
-                const int i = bx * SUB + s;                 // k-block within the segment
-                if (!kPartial || i < nkb) {
-                    const int lk = lk0 + i;                 // k-block within the CTA's slice (>= 0)
-                    // this k-block's codes of the thread's two rows
-                    uint32_t r0[2 * TW], r1[2 * TW];
-                    if (TW == 2) {
-                        const uint2 v0 = gemv_lds64(base + offs[s]);
-                        const uint2 v1 = gemv_lds64(base + 1024 + offs[s]);
-                        r0[0] = v0.x;
-                        r0[1] = v0.y;
-                        r1[0] = v1.x;
-                        r1[1] = v1.y;
-                    } else {
-                        r0[0] = gemv_lds32(base + offs[s]);
-                        r1[0] = gemv_lds32(base + 1024 + offs[s]);
-                    }
+                if (s < nk) {
                     if (s % GB == 0) {
-                        // this group's constants from the table
-                        const uint32_t ta = trow + static_cast<uint32_t>(lk) / GB * TE;
-                        const uint32_t e0 = gemv_lds32(ta), e1 = gemv_lds32(ta + 8 * tstride * TE);
                         if (KIND != kCode4) {
-                            sub0 = __byte_perm(e0, 0u, 0x1010);
-                            sub1 = __byte_perm(e1, 0u, 0x1010);
-                            sf0 = f16_bits_to_f32(static_cast<uint16_t>(e0 >> 16));
-                            sf1 = f16_bits_to_f32(static_cast<uint16_t>(e1 >> 16));
+                            const int gi = s / GB;
+                            sf0 = f16_bits_to_f32(gv_lds16(ca0 + 2 * (gi + par0)));
+                            sf1 = f16_bits_to_f32(gv_lds16(ca1 + 2 * (gi + par1)));
+                            zf0 = f16_bits_to_f32(gv_lds16(ca0 + zoff + 2 * (gi + par0)));
+                            zf1 = f16_bits_to_f32(gv_lds16(ca1 + zoff + 2 * (gi + par1)));
+                            if (kFold) {
+                                // A = 128 + code: the fold takes (128 + zero) * sum(x) off
+                                zf0 += 128.0f;
+                                zf1 += 128.0f;
+                                far = true;
+                            } else {
+                                far = __any_sync(0xFFFFFFFFu, (fabsf(zf0) > 128.0f) || (fabsf(zf1) > 128.0f));
+                            }
+                            if (kFold) {
+                            } else if (far) {
+                                // A = code (exact); zero * sum(x) is taken off at the fold
+                                sub0 = sub1 = 0x43004300u;
+                            } else {
+                                // (128 + code) - (128 + zero) = code - zero exactly
+                                sub0 = pack_bf16x2_rn(128.0f + zf0, 128.0f + zf0);
+                                sub1 = pack_bf16x2_rn(128.0f + zf1, 128.0f + zf1);
+                            }
+                        } else if (P.q8 == nullptr) {
+                            sf0 = __uint_as_float(gv_lds32(ca0 + 4 * s));
+                            sf1 = __uint_as_float(gv_lds32(ca1 + 4 * s));
                         } else {
-                            sf0 = __uint_as_float(e0);
-                            sf1 = __uint_as_float(e1);
+                            // absmax' = fp32(fp32(q8 / 127) * s2) + offset
+                            const int64_t e0a = gr0 * P.kbt + kbs, e0b = gr1 * P.kbt + kbs;
+                            const int ia = static_cast<int>((e0a & 3) + s), ib = static_cast<int>((e0b & 3) + s);
+                            const uint32_t qa = gv_lds32(ca0 + (ia & ~3)), qb = gv_lds32(ca1 + (ib & ~3));
+                            const uint32_t q8a = (qa >> (8 * (ia & 3))) & 0xFFu, q8b = (qb >> (8 * (ib & 3))) & 0xFFu;
+                            const float s2a = __uint_as_float(gv_lds32(ca0 + zoff + (((e0a + s) >> 8) != (e0a >> 8) ? 4 : 0)));
+                            const float s2b = __uint_as_float(gv_lds32(ca1 + zoff + (((e0b + s) >> 8) != (e0b >> 8) ? 4 : 0)));
+                            sf0 = __fadd_rn(__fmul_rn(s_q8lut[q8a], s2a), dq_off);
+                            sf1 = __fadd_rn(__fmul_rn(s_q8lut[q8b], s2b), dq_off);
                         }
                     }
-                    // A fragments: 8 code pairs of each row as bf16x2
+                    // this k-block's codes of the thread's two rows, as bf16x2 pairs
                     uint32_t f0[8], f1[8];
                     if (KIND == kInt4) {
-                        int4_pairs(r0[0], mg, f0);
-                        int4_pairs(r0[TW - 1], mg, f0 + 4);
-                        int4_pairs(r1[0], mg, f1);
-                        int4_pairs(r1[TW - 1], mg, f1 + 4);
+                        const uint2 v0 = gv_lds64(wrow + offs[s]);
+                        const uint2 v1 = gv_lds64(wrow + 1024 + offs[s]);
+                        int4_pairs(v0.x, mg, f0);
+                        int4_pairs(v0.y, mg, f0 + 4);
+                        int4_pairs(v1.x, mg, f1);
+                        int4_pairs(v1.y, mg, f1 + 4);
                     } else if (KIND == kInt2) {
-                        int2_pairs(r0[0], mg, f0);
-                        int2_pairs(r1[0], mg, f1);
+                        int2_pairs(gv_lds32(wrow + offs[s]), mg, f0);
+                        int2_pairs(gv_lds32(wrow + 1024 + offs[s]), mg, f1);
                     } else {
+                        const uint2 v0 = gv_lds64(wrow + offs[s]);
+                        const uint2 v1 = gv_lds64(wrow + 1024 + offs[s]);
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
-                            f0[q] = s_lut[__byte_perm(r0[0], 0u, 0x4440 + q)];
-                            f0[4 + q] = s_lut[__byte_perm(r0[TW - 1], 0u, 0x4440 + q)];
-                            f1[q] = s_lut[__byte_perm(r1[0], 0u, 0x4440 + q)];
-                            f1[4 + q] = s_lut[__byte_perm(r1[TW - 1], 0u, 0x4440 + q)];
+                            f0[q] = s_lut[__byte_perm(v0.x, 0u, 0x4440 + q)];
+                            f0[4 + q] = s_lut[__byte_perm(v0.y, 0u, 0x4440 + q)];
+                            f1[q] = s_lut[__byte_perm(v1.x, 0u, 0x4440 + q)];
+                            f1[4 + q] = s_lut[__byte_perm(v1.y, 0u, 0x4440 + q)];
                         }
                     }
-                    if (KIND != kCode4) {
+                    if (KIND != kCode4 && !kFold) {
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
                             f0[q] = sub_bf16x2(f0[q], sub0);
                             f1[q] = sub_bf16x2(f1[q], sub1);
                         }
                     }
-                    // B fragments (permuted activations) and four MMA steps
-                    const uint32_t xoff = static_cast<uint32_t>(lk) * 128;
-                    uint2 bxf[4][NT8];
+                    // B fragments: the 16 activations of the thread's quarter
+                    // (steps 0, 1 from the first 16 bytes, 2, 3 from the next)
+                    uint32_t xb[NT8][8];
 #pragma unroll
-                    for (int tau = 0; tau < 4; ++tau)
-#pragma unroll
-                        for (int nt = 0; nt < NT8; ++nt)
-                            bxf[tau][nt] = gemv_lds64(xthr[nt] + xoff + 8 * tau);
+                    for (int nt = 0; nt < NT8; ++nt) {
+                        const uint32_t xa = stage + xoff[nt] + s * MPAD * 128;
+                        const uint4 lo = gv_lds128(xa);
+                        const uint4 hi = gv_lds128(xa ^ 16u);
+                        xb[nt][0] = lo.x;
+                        xb[nt][1] = lo.y;
+                        xb[nt][2] = lo.z;
+                        xb[nt][3] = lo.w;
+                        xb[nt][4] = hi.x;
+                        xb[nt][5] = hi.y;
+                        xb[nt][6] = hi.z;
+                        xb[nt][7] = hi.w;
+                    }
 #pragma unroll
                     for (int tau = 0; tau < 4; ++tau)
 #pragma unroll
                         for (int nt = 0; nt < NT8; ++nt) {
                             if (s % GB == 0 && tau < 2)
                                 mma_m16n8k16_bf16_first(cg[tau & 1][nt], f0[2 * tau], f1[2 * tau], f0[2 * tau + 1],
-                                                        f1[2 * tau + 1], bxf[tau][nt].x, bxf[tau][nt].y);
+                                                        f1[2 * tau + 1], xb[nt][2 * tau], xb[nt][2 * tau + 1]);
                             else
                                 mma_m16n8k16_bf16(cg[tau & 1][nt], f0[2 * tau], f1[2 * tau], f0[2 * tau + 1],
-                                                  f1[2 * tau + 1], bxf[tau][nt].x, bxf[tau][nt].y);
+                                                  f1[2 * tau + 1], xb[nt][2 * tau], xb[nt][2 * tau + 1]);
                         }
-                    // end of a scale group: fold the group partial
-                    if (s % GB == GB - 1) {
+                    if (KIND != kCode4 && far) {
+                        // per-token sums of the group's activations (every row alike)
 #pragma unroll
-                        for (int nt = 0; nt < NT8; ++nt) {
-                            acc[nt][0] = fmaf(sf0, cg[0][nt][0] + cg[1][nt][0], acc[nt][0]);
-                            acc[nt][1] = fmaf(sf0, cg[0][nt][1] + cg[1][nt][1], acc[nt][1]);
-                            acc[nt][2] = fmaf(sf1, cg[0][nt][2] + cg[1][nt][2], acc[nt][2]);
-                            acc[nt][3] = fmaf(sf1, cg[0][nt][3] + cg[1][nt][3], acc[nt][3]);
+                        for (int tau = 0; tau < 4; ++tau)
+#pragma unroll
+                            for (int nt = 0; nt < NT8; ++nt) {
+                                if (s % GB == 0 && tau < SXC)
+                                    mma_m16n8k16_bf16_first(sx[tau % SXC][nt], ones, ones, ones, ones, xb[nt][2 * tau],
+                                                            xb[nt][2 * tau + 1]);
+                                else
+                                    mma_m16n8k16_bf16(sx[tau % SXC][nt], ones, ones, ones, ones, xb[nt][2 * tau],
+                                                      xb[nt][2 * tau + 1]);
+                            }
+                    }
+                    // end of a scale group: fold the group partial
+                    if (s % GB == GB - 1 || s == nk - 1) {
+                        if (KIND != kCode4 && far) {
+#pragma unroll
+                            for (int nt = 0; nt < NT8; ++nt) {
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const float sxe = SXC == 2 ? sx[0][nt][e] + sx[SXC - 1][nt][e] : sx[0][nt][e];
+                                    const float cge = cg[0][nt][e] + cg[1][nt][e];
+                                    acc[nt][e] = fmaf(e < 2 ? sf0 : sf1, fmaf(e < 2 ? -zf0 : -zf1, sxe, cge), acc[nt][e]);
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int nt = 0; nt < NT8; ++nt) {
+                                acc[nt][0] = fmaf(sf0, cg[0][nt][0] + cg[1][nt][0], acc[nt][0]);
+                                acc[nt][1] = fmaf(sf0, cg[0][nt][1] + cg[1][nt][1], acc[nt][1]);
+                                acc[nt][2] = fmaf(sf1, cg[0][nt][2] + cg[1][nt][2], acc[nt][2]);
+                                acc[nt][3] = fmaf(sf1, cg[0][nt][3] + cg[1][nt][3], acc[nt][3]);
+                            }
                         }
                     }
                 }
             }
-        };
-        for (int bx = 0; bx < nbx; ++bx, ++c) {
-            const uint32_t w = c % WS;
-            if (!mbar_wait(&full[w], (c / WS) & 1u, s_abort)) break;
-            if (bx < nfull)
-                run_box(std::false_type{}, bx, w);
-            else
-                run_box(std::true_type{}, bx, w);
-            // release the slot only after every loaded word has been used: an
-            // arrive issued right behind the shared loads let the next TMA
-            // write land before some of those loads had read the slot
+            // release the slot only after every loaded word has been used
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[w]);
         }
-        if (KIND != kCode4 && far) {
-            // groups stored with |zero| > 128 ran as (q - 0); add their
-            // scale * (-zero) * (sum of x over the group) here
-            for (int lg = lk0 / GB; lg < (lk0 + nkb) / GB; ++lg) {
-                const int64_t gi = kb0 / GB + (lg - lk0 / GB);      // group within the row
-                float k0 = 0.0f, k1 = 0.0f;
-                if (ok0) {
-                    const float z = f16_bits_to_f32(__ldg(p.zero + gr0 * p.ngroups + gi));
-                    if (fabsf(z) > 128.0f) k0 = f16_bits_to_f32(__ldg(p.scale + gr0 * p.ngroups + gi)) * -z;
-                }
-                if (ok1) {
-                    const float z = f16_bits_to_f32(__ldg(p.zero + gr1 * p.ngroups + gi));
-                    if (fabsf(z) > 128.0f) k1 = f16_bits_to_f32(__ldg(p.scale + gr1 * p.ngroups + gi)) * -z;
-                }
-                if (k0 == 0.0f && k1 == 0.0f) continue;
-#pragma unroll
-                for (int nt = 0; nt < NT8; ++nt) {
-                    const int tA = nt * 8 + 2 * j;
-                    float sx0 = 0.0f, sx1 = 0.0f;
-                    for (int kk = lg * GB * 64; kk < (lg + 1) * GB * 64; ++kk) {
-                        if (tA < p.m) sx0 += bf16_bits_to_f32(sX[tA * xstride + kk]);
-                        if (tA + 1 < p.m) sx1 += bf16_bits_to_f32(sX[(tA + 1) * xstride + kk]);
-                    }
-                    acc[nt][0] = fmaf(k0, sx0, acc[nt][0]);
-                    acc[nt][1] = fmaf(k0, sx1, acc[nt][1]);
-                    acc[nt][2] = fmaf(k1, sx0, acc[nt][2]);
-                    acc[nt][3] = fmaf(k1, sx1, acc[nt][3]);
-                }
-            }
-        }
         // -------------------------------------------------------------- segment epilogue
         auto lora = [&](int t, int oc) -> float {
-            if (p.rank == 0) return 0.0f;
+            if (P.rank == 0) return 0.0f;
             float d = 0.0f;
-            for (int u = 0; u < p.rank; ++u)
-                d = fmaf(p.T[static_cast<int64_t>(t) * p.rank + u],
-                         bf16_bits_to_f32(__ldg(p.B + static_cast<int64_t>(oc) * p.rank + u)), d);
-            return p.s * d;
+            for (int u = 0; u < P.rank; ++u)
+                d = fmaf(P.T[static_cast<int64_t>(t) * P.rank + u],
+                         bf16_bits_to_f32(__ldg(P.B + static_cast<int64_t>(oc) * P.rank + u)), d);
+            return P.s * d;
         };
-        if (kb0 == 0 && nkb == p.kbt) {
+        if (sg.ka == 0 && sg.kb == P.kbt) {
             // this CTA covered the whole tile
 #pragma unroll
             for (int nt = 0; nt < NT8; ++nt)
@@ -650,40 +677,40 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
                     const int t = nt * 8 + 2 * j + (e & 1);
                     const bool ok = (e < 2) ? ok0 : ok1;
                     const int64_t r = (e < 2) ? gr0 : gr1;
-                    if (ok && t < p.m) {
-                        const int oc = p.perm ? p.perm[r] : static_cast<int>(r);
-                        p.Y[static_cast<int64_t>(t) * p.ldy + oc] = acc[nt][e] + lora(t, oc);
+                    if (ok && t < m) {
+                        const int oc = P.perm ? P.perm[r] : static_cast<int>(r);
+                        P.Y[static_cast<int64_t>(t) * P.ldy + oc] = acc[nt][e] + lora(t, oc);
                     }
                 }
             continue;
         }
         // split tile.  Partial slot of (CTA b, tile t) is b + t: CTAs cover the
         // work in order, so no two (CTA, tile) pairs share a slot.
-        const int cta_lo = static_cast<int>((static_cast<int64_t>(tile) * p.kbt) / p.share);
-        const int cta_hi = static_cast<int>((static_cast<int64_t>(tile + 1) * p.kbt - 1) / p.share);
-        if (kb0 + nkb < p.kbt) {
+        const int cta_lo = static_cast<int>((static_cast<int64_t>(tile) * P.kbt) / P.share);
+        const int cta_hi = static_cast<int>((static_cast<int64_t>(tile + 1) * P.kbt - 1) / P.share);
+        if (sg.kb < P.kbt) {
             // contributor (the tile's last k-block belongs to a later CTA)
-            float* slot = p.partial + (static_cast<int64_t>(blockIdx.x) + tile) * p.m * 128;
+            float* slot = P.partial + (static_cast<int64_t>(b) + tile) * m * 128;
 #pragma unroll
             for (int nt = 0; nt < NT8; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int t = nt * 8 + 2 * j + (e & 1);
-                    if (t < p.m) slot[t * 128 + rl0 + ((e < 2) ? 0 : 8)] = acc[nt][e];
+                    if (t < m) slot[t * 128 + rl0 + ((e < 2) ? 0 : 8)] = acc[nt][e];
                 }
             asm volatile("bar.sync 1, 256;" ::: "memory");
-            if (tid == 0) flag_publish(p.counters + tile);
+            if (tid == 0) flag_publish(P.counters + tile);
             continue;
         }
         // this CTA finishes the tile: wait for the cta_hi - cta_lo contributors
         if (tid == 0) {
-            if (!flag_wait_geq(p.counters + tile, static_cast<uint32_t>(cta_hi - cta_lo))) *s_abort = 1;
-            p.counters[tile] = 0u;                     // left at zero for the next call
+            if (!flag_wait_geq(P.counters + tile, static_cast<uint32_t>(cta_hi - cta_lo))) *s_abort = 1;
+            P.counters[tile] = 0u;                          // left at zero for the next call
         }
         asm volatile("bar.sync 1, 256;" ::: "memory");
         // the contributors' partials in CTA order (QB CTAs' loads in flight
         // together), then this CTA's own sums
-        constexpr int QB = NT8 == 1 ? 8 : 2;
+        constexpr int QB = NT8 == 1 ? 8 : 4;
         float v[NT8][4];
 #pragma unroll
         for (int nt = 0; nt < NT8; ++nt)
@@ -698,8 +725,8 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int t = nt * 8 + 2 * j + (e & 1);
-                        part[q][nt][e] = (b0 + q < cta_hi && t < p.m)
-                                             ? __ldcg(p.partial + ((static_cast<int64_t>(b0 + q) + tile) * p.m + t) * 128 +
+                        part[q][nt][e] = (b0 + q < cta_hi && t < m)
+                                             ? __ldcg(P.partial + ((static_cast<int64_t>(b0 + q) + tile) * m + t) * 128 +
                                                       rl0 + ((e < 2) ? 0 : 8))
                                              : 0.0f;
                     }
@@ -717,12 +744,92 @@ dqgemv_kernel(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
                 const int t = nt * 8 + 2 * j + (e & 1);
                 const bool ok = (e < 2) ? ok0 : ok1;
                 const int64_t r = (e < 2) ? gr0 : gr1;
-                if (ok && t < p.m) {
-                    const int oc = p.perm ? p.perm[r] : static_cast<int>(r);
-                    p.Y[static_cast<int64_t>(t) * p.ldy + oc] = (v[nt][e] + acc[nt][e]) + lora(t, oc);
+                if (ok && t < m) {
+                    const int oc = P.perm ? P.perm[r] : static_cast<int>(r);
+                    P.Y[static_cast<int64_t>(t) * P.ldy + oc] = (v[nt][e] + acc[nt][e]) + lora(t, oc);
                 }
             }
     }
+    cp_async_wait_all();                                     // no copy into the buffer outlives the CTA
+}
+
+template <int NT8>
+__global__ void __launch_bounds__(kGvThreads, 2) dqgemv_grouped_kernel(const __grid_constant__ GvParams p) {
+    // let the next kernel on the stream be scheduled as soon as our CTAs leave
+    griddep_launch_dependents();
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // this CTA's matrix and its index among that matrix's CTAs; its
+    // descriptor goes to shared memory once
+    int pi = 0;
+    for (int i = 1; i < p.nprob; ++i)
+        if (static_cast<int>(blockIdx.x) >= p.prob[i].cta0) pi = i;
+    __shared__ GvProblem s_prob;
+    {
+        static_assert(sizeof(GvProblem) % 4 == 0, "descriptor copied in words");
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(&p.prob[pi]);
+        uint32_t* dst = reinterpret_cast<uint32_t*>(&s_prob);
+        for (int i = tid; i < static_cast<int>(sizeof(GvProblem) / 4); i += kGvThreads) dst[i] = src[i];
+    }
+    __syncthreads();
+    const GvProblem& P = s_prob;
+    const int b = static_cast<int>(blockIdx.x) - P.cta0;
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte alignment for the swizzled boxes, by pointer arithmetic on the
+    // shared array so that every access below stays a shared-memory access
+    uint8_t* ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t* cbuf = ring + p.ws * p.stage_bytes;                              // [warp][slot][array][16 rows]
+    uint64_t* full = reinterpret_cast<uint64_t*>(cbuf + kGvComputeWarps * 2 * 32 * p.cstride);
+    uint64_t* xready = full + kGvMaxStages;
+    uint64_t* empty = xready + kGvMaxStages;
+    volatile int* s_abort = reinterpret_cast<volatile int*>(empty + kGvMaxStages);
+    uint32_t* s_lut = reinterpret_cast<uint32_t*>(empty + kGvMaxStages) + 4;   // codebook pairs [256]
+    float* s_q8lut = reinterpret_cast<float*>(s_lut + 256);                  // q8 / 127 [256]
+
+    // the share: units [u0, u1) of (tile, k-block), in tile-major order
+    GvShare sh;
+    sh.kbt = P.kbt;
+    sh.u0 = static_cast<int64_t>(b) * P.share;
+    sh.u1 = min(sh.u0 + P.share, P.total);
+    sh.tA = static_cast<int>(sh.u0 / P.kbt);
+    sh.tB = sh.u0 < sh.u1 ? static_cast<int>((sh.u1 - 1) / P.kbt) : sh.tA - 1;
+    sh.nseg = sh.tB - sh.tA + 1;
+
+    if (tid == kGvComputeWarps * 32) {
+        tma_prefetch_desc(&p.tmW[pi]);
+        tma_prefetch_desc(&p.tmX[pi]);
+        for (int i = 0; i < p.ws; ++i) {
+            mbar_init(&full[i], 1);                      // the producer's arrival + the boxes' bytes
+            mbar_init(&xready[i], 1);                    // activations in the pairs' order
+            mbar_init(&empty[i], kGvComputeWarps);
+        }
+        *s_abort = 0;
+        fence_mbar_init();
+    }
+    if (P.kind == kCode4) {
+        for (int e = tid; e < 256; e += kGvThreads) {
+            // byte e = (first code << 4) | second code -> (codebook[first], codebook[second])
+            s_lut[e] = pack_bf16x2_rn(__ldg(P.codebook + (e >> 4)), __ldg(P.codebook + (e & 15)));
+            s_q8lut[e] = __fdiv_rn(static_cast<float>(static_cast<int8_t>(static_cast<uint8_t>(e))), 127.0f);
+        }
+    }
+    __syncthreads();
+    if (sh.nseg <= 0) return;
+
+    auto run = [&](auto kind_tag) {
+        constexpr int KIND = decltype(kind_tag)::value;
+        if (warp == kGvComputeWarps)
+            gv_produce<KIND>(p, &p.tmW[pi], &p.tmX[pi], P.xbytes, sh, ring, full, xready, empty, s_abort, lane);
+        else
+            gv_compute<KIND, NT8>(p, P, sh, b, ring, xready, empty, s_abort, cbuf, s_lut, s_q8lut);
+    };
+    if (P.kind == kInt4)
+        run(std::integral_constant<int, kInt4>{});
+    else if (P.kind == kInt2)
+        run(std::integral_constant<int, kInt2>{});
+    else
+        run(std::integral_constant<int, kCode4>{});
 }
 
 }  // namespace lbq

@@ -1,145 +1,226 @@
-// dqgemv_host.cuh -- host side of the decode GEMV: shared-memory budget,
-// stream-K plan (shares, grid, weight-ring depth) and the launch.  Included by
-// lbq.cu inside its file-local namespace, after the plan type, workspace
-// layout and stream bookkeeping it uses.
+// dqgemv_host.cuh -- host side of the grouped decode GEMV: shared-memory
+// layout, shares and grid, workspace layout and the launch.  Included by
+// lbq.cu inside its file-local namespace, after the helpers it uses (tensor
+// maps, descriptor checks, workspace header, stream bookkeeping).
 #pragma once
 
-// Decode-sized batches (m <= 16) run the stream-K GEMV: every CTA gets an
-// equal share of the (row tile, k-block) work, a whole number of scale
-// groups and as many k-blocks as its shared memory holds (weight ring,
-// activation slice, constant table) with two CTAs per SM, and the grid fills
-// whole waves of two CTAs per SM.  The weight ring holds four boxes, or
-// three when that lets the whole grid run in one wave (wide token tiles,
-// whose activation slice takes most of the shared memory).
+// Decode-sized batches (m <= 16) run the grouped GEMV: one launch for up to
+// kGvMaxProblems matrices, one wave of two CTAs per SM, every CTA an equal
+// share in bytes of one matrix's (row tile, k-block) work.
 constexpr int kGemvMaxM = 16;
-constexpr size_t kGemvSmemBudget = 113 * 1024;     // two CTAs per SM
+constexpr size_t kGemvSmemBudget = 115712 - 1024;   // two CTAs per SM (228 KB; 1 KB reserved and 1 KB static per CTA)
 
-size_t gemv_smem_bytes(int m, int share, int kind, int stages) {
-    const int gb = kind == kInt4 ? 2 : 1;
-    const int nt = m <= 8 ? 8 : 16;
-    const size_t xrows = static_cast<size_t>(m < nt ? m + 1 : m);      // + a zero row for padded lanes
-    return 1024 + static_cast<size_t>(stages) * 128 * 128 + xrows * (share * 64 + 4) * 2 +
-           static_cast<size_t>((share / gb) | 1) * 128 * 4 + (kind == kCode4 ? 1024 : 0) + 2 * stages * 8 + 16;
+// One forward of a group: activations, weight, adapter, output.
+struct GvJob {
+    const void* X;
+    const lbq_qweight* q;
+    const void* B;
+    int rank;
+    float s;
+    const float* T;
+    float* Y;
+    int64_t ldy;
+    const int32_t* perm;
+};
+
+struct GvPlan {
+    int count = 0;
+    int ctas = 0;                   // grid
+    int ws = 0;                     // ring stages
+    int stage_bytes = 0, xbox_max = 0, cstride = 0;
+    size_t smem = 0;                // dynamic shared memory per CTA
+    size_t workspace = 0;           // 0 when no tile is split
+    int share[kGvMaxProblems] = {}, pctas[kGvMaxProblems] = {}, cta0[kGvMaxProblems] = {};
+    int tiles[kGvMaxProblems] = {};
+    int cnt_off[kGvMaxProblems] = {};
+    size_t part_off[kGvMaxProblems] = {};
+};
+
+// Algorithmic bytes of one (128-row tile, k-block) unit: packed codes plus
+// the per-row constants of the k-block.
+double gv_unit_bytes(const lbq_qweight* q) {
+    const double codes = 128.0 * 64 * q->bits / 8;
+    if (q->scheme == LBQ_MINMAX_ASYM) return codes + 128.0 * 4 * 64 / q->group;
+    return codes + 128.0 * (q->double_quant ? 1 : 4);
 }
 
-Plan plan_gemv(int m, const lbq_qweight* q, int sms) {
-    Plan pl;
-    pl.nt = m <= 8 ? 8 : 16;
-    const int kind = kind_of(q);
-    const int64_t kbt = q->k / 64;
-    const int gb = kind == kInt4 ? 2 : 1;
-    pl.tiles = static_cast<int>(cdiv(q->n, 128));
-    const int64_t total = static_cast<int64_t>(pl.tiles) * kbt;
-    const int64_t slots = 2LL * sms;
-    auto max_share = [&](int stages) {
-        int64_t smax = gb;
-        while (smax + gb <= kbt && (smax + gb) / gb <= kGemvMaxTabGroups &&
-               gemv_smem_bytes(m, static_cast<int>(smax + gb), kind, stages) <= kGemvSmemBudget)
-            smax += gb;
-        return smax;
-    };
-    int64_t smax = max_share(kGemvMaxWStages);
-    int64_t waves = cdiv(total, slots * smax);
-    pl.stages = kGemvMaxWStages;
-    if (waves > 1) {
-        const int64_t smax3 = max_share(kGemvMaxWStages - 1);
-        if (cdiv(total, slots * smax3) < waves) {
-            smax = smax3;
-            waves = cdiv(total, slots * smax3);
-            pl.stages = kGemvMaxWStages - 1;
+// Bytes per row of one constant array that a weight box needs: the 4-byte
+// words covering its groups (MinMax: 2 groups for INT4, 8 for INT2, starting
+// at any entry), 4 absmax values, or 2 words of q8 and 2 of s2.
+int gv_const_stride(const lbq_qweight* q) {
+    if (q->scheme == LBQ_CODEBOOK4) return q->double_quant ? 8 : 16;
+    const int gpb = q->bits == 2 ? 8 : 2;                               // groups per box
+    return 4 * (gpb / 2 + 1);
+}
+
+// Token rows of an activation box: the real ones padded to the MMA's token
+// tile (8 or 16).
+int gv_mpad(int m) { return m <= 8 ? 8 : 16; }
+
+lbq_status gv_plan(int m, const lbq_qweight* const* qs, int count, int sms, GvPlan* pl) {
+    if (m < 1 || m > kGemvMaxM || count < 1 || count > kGvMaxProblems) return LBQ_EINVAL;
+    *pl = GvPlan();
+    pl->count = count;
+    bool any_int2 = false, any_code = false;
+    int cstride = 4;
+    double total_bytes = 0.0;
+    int tiles_sum = 0;
+    for (int i = 0; i < count; ++i) {
+        const lbq_qweight* q = qs[i];
+        const int64_t kbt = q->k / 64, tiles = cdiv(q->n, 128);
+        if (tiles * kbt >= (int64_t(1) << 31)) return LBQ_EUNSUPPORTED;
+        any_int2 |= (q->scheme == LBQ_MINMAX_ASYM && q->bits == 2);
+        any_code |= q->scheme == LBQ_CODEBOOK4;
+        cstride = std::max(cstride, gv_const_stride(q));
+        total_bytes += gv_unit_bytes(q) * static_cast<double>(tiles * kbt);
+        pl->tiles[i] = static_cast<int>(tiles);
+        pl->cnt_off[i] = tiles_sum;
+        tiles_sum += static_cast<int>(tiles);
+    }
+    if (tiles_sum > kMaxSplitTiles) return LBQ_EUNSUPPORTED;
+    // stage layout: weight box, activation box; then one constant buffer of
+    // two slots per compute warp
+    const int sub_max = any_int2 ? 8 : 4;
+    pl->xbox_max = sub_max * gv_mpad(m) * 128;
+    pl->cstride = cstride;
+    pl->stage_bytes = kGvWBox + pl->xbox_max;
+    const size_t cbuf = static_cast<size_t>(kGvComputeWarps) * 2 * 32 * cstride;
+    (void)any_code;
+    pl->ws = 0;
+    for (int ws = kGvMaxStages; ws >= 2; --ws) {
+        const size_t smem = 1024 + static_cast<size_t>(ws) * pl->stage_bytes + cbuf + kGvExtraSmem;
+        if (smem <= kGemvSmemBudget) {
+            pl->ws = ws;
+            pl->smem = smem;
+            break;
         }
     }
-    int64_t share = cdiv(cdiv(total, waves * slots), gb) * gb;
-    // at least an eighth of a row per CTA, so that the CTA finishing a tile
-    // sums a handful of partials (small layers then use fewer CTAs)
-    share = std::max(share, std::min(cdiv(cdiv(kbt, 8), gb) * gb, smax));
-    share = std::max<int64_t>(gb, std::min(share, smax));
-    pl.per_split = static_cast<int>(share);                      // k-blocks per CTA
-    pl.nsplit = static_cast<int>(cdiv(total, share));            // CTAs
-    pl.partial_bytes = round_up(static_cast<size_t>(pl.nsplit + pl.tiles) * m * 128 * sizeof(float), 256);
-    return pl;
+    if (pl->ws == 0) return LBQ_EUNSUPPORTED;
+    // shares: every CTA about the same bytes; at most one wave of two CTAs
+    // per SM (each matrix rounds its CTA count up by less than one)
+    const int slots = 2 * sms;
+    const double target = total_bytes / std::max(1, slots - count);
+    bool split = false;
+    size_t part = 0;
+    int cta = 0;
+    for (int i = 0; i < count; ++i) {
+        const lbq_qweight* q = qs[i];
+        const int64_t kbt = q->k / 64, units = static_cast<int64_t>(pl->tiles[i]) * kbt;
+        const int gb = (q->scheme == LBQ_MINMAX_ASYM && q->bits == 4) ? 2 : 1;
+        int64_t share = cdiv(static_cast<int64_t>(std::ceil(target / gv_unit_bytes(q))), gb) * gb;
+        // at least an eighth of a row per CTA, so that the CTA finishing a
+        // tile sums a handful of partials (small matrices use fewer CTAs)
+        share = std::max(share, std::min<int64_t>(kbt, cdiv(cdiv(kbt, 8), gb) * gb));
+        share = std::max<int64_t>(share, gb);
+        const int64_t ctas = cdiv(units, share);
+        pl->share[i] = static_cast<int>(share);
+        pl->pctas[i] = static_cast<int>(ctas);
+        pl->cta0[i] = cta;
+        cta += static_cast<int>(ctas);
+        if (share % kbt != 0) split = true;
+        pl->part_off[i] = part;
+        part += round_up(static_cast<size_t>(ctas + pl->tiles[i]) * m * 128 * sizeof(float), 256);
+    }
+    pl->ctas = cta;
+    pl->workspace = split ? kCounterHeader + part : 0;
+    return LBQ_OK;
 }
 
-template <int KIND, int NTOK, int WS>
-lbq_status launch_gemv_kind(const GemvParams& p, const uint8_t* packed, int grid, cudaStream_t st) {
-    auto kern = dqgemv_kernel<KIND, NTOK, WS>;
-    const size_t smem = gemv_smem_bytes(p.m, p.share, KIND, WS);
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
-        return LBQ_ECUDA;
-    CUtensorMap tmW;
-    if (!make_map_2d(&tmW, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.n, static_cast<int64_t>(p.k) * (KIND == kInt2 ? 2 : 4) / 8,
-                     128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+template <int NT8>
+lbq_status gv_launch(const GvParams& prm, const GvPlan& pl, cudaStream_t st) {
+    auto kern = dqgemv_grouped_kernel<NT8>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(pl.smem)) != cudaSuccess)
         return LBQ_ECUDA;
     // programmatic dependent launch: the kernel may start during the previous
     // kernel's tail and waits for it (griddepcontrol.wait) before reading
     // anything that kernel can have written
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
-    cfg.blockDim = dim3(kGemvThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.ctas), 1, 1);
+    cfg.blockDim = dim3(kGvThreads, 1, 1);
+    cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, tmW, p) != cudaSuccess) return LBQ_ECUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, prm) != cudaSuccess) return LBQ_ECUDA;
     return last_launch();
 }
 
-template <int WS>
-lbq_status launch_gemv_tile(const GemvParams& p, const lbq_qweight* q, const Plan& pl, cudaStream_t st) {
-    if (WS != pl.stages) {
-        if constexpr (WS > kGemvMaxWStages - 1) return launch_gemv_tile<WS - 1>(p, q, pl, st);
-        return LBQ_EUNSUPPORTED;
+// One grouped launch (count <= kGvMaxProblems) of the decode GEMV.
+lbq_status run_gemv_group(int m, const GvJob* jobs, int count, void* ws, size_t ws_bytes, int sms, cudaStream_t st) {
+    const lbq_qweight* qs[kGvMaxProblems];
+    for (int i = 0; i < count; ++i) qs[i] = jobs[i].q;
+    GvPlan pl;
+    lbq_status s = gv_plan(m, qs, count, sms, &pl);
+    if (s != LBQ_OK) return s;
+    if (pl.workspace > 0 && (!ws || ws_bytes < pl.workspace)) return LBQ_EWORKSPACE;
+    GvParams prm;                                // passed by value at launch
+    memset(&prm, 0, sizeof(prm));
+    prm.nprob = count;
+    prm.m = m;
+    prm.ws = pl.ws;
+    prm.stage_bytes = pl.stage_bytes;
+    prm.cstride = pl.cstride;
+    prm.w_early = weights_stable(st) ? 1 : 0;
+    for (int i = 0; i < count; ++i) {
+        const lbq_qweight* q = jobs[i].q;
+        GvProblem& P = prm.prob[i];
+        const int sub = (q->scheme == LBQ_MINMAX_ASYM && q->bits == 2) ? 8 : 4;
+        if (!make_map_2d(&prm.tmW[i], q->packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q->n,
+                         static_cast<int64_t>(q->k) * q->bits / 8, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+            return LBQ_ECUDA;
+        if (!make_map_x3d(&prm.tmX[i], jobs[i].X, m, q->k, gv_mpad(m), sub)) return LBQ_ECUDA;
+        P.xbytes = sub * gv_mpad(m) * 128;
+        P.X = static_cast<const uint16_t*>(jobs[i].X);
+        P.Y = jobs[i].Y;
+        P.perm = jobs[i].perm;
+        P.scale = q->scale;
+        P.zero = q->zero;
+        P.absmax = q->absmax;
+        P.q8 = (q->scheme == LBQ_CODEBOOK4 && q->double_quant) ? q->absmax_q8 : nullptr;
+        P.s2 = q->absmax_s2;
+        P.offset = q->absmax_offset;
+        P.codebook = q->codebook;
+        P.T = jobs[i].T;
+        P.B = static_cast<const uint16_t*>(jobs[i].B);
+        P.rank = jobs[i].rank;
+        P.s = jobs[i].s;
+        P.ldy = jobs[i].ldy;
+        P.n = q->n;
+        P.k = q->k;
+        P.kind = kind_of(q);
+        P.ngroups = q->scheme == LBQ_MINMAX_ASYM ? q->k / q->group : 0;
+        P.kbt = q->k / 64;
+        P.tiles = pl.tiles[i];
+        P.total = static_cast<int64_t>(pl.tiles[i]) * P.kbt;
+        P.share = pl.share[i];
+        P.cta0 = pl.cta0[i];
+        if (pl.workspace > 0) {
+            P.counters = ws_counters(ws) + pl.cnt_off[i];
+            P.partial = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws_partials(ws)) + pl.part_off[i]);
+        }
     }
-    const bool n8 = pl.nt == 8;
-    switch (kind_of(q)) {
-        case kInt4: return n8 ? launch_gemv_kind<kInt4, 8, WS>(p, q->packed, pl.nsplit, st)
-                              : launch_gemv_kind<kInt4, 16, WS>(p, q->packed, pl.nsplit, st);
-        case kInt2: return n8 ? launch_gemv_kind<kInt2, 8, WS>(p, q->packed, pl.nsplit, st)
-                              : launch_gemv_kind<kInt2, 16, WS>(p, q->packed, pl.nsplit, st);
-        default: return n8 ? launch_gemv_kind<kCode4, 8, WS>(p, q->packed, pl.nsplit, st)
-                           : launch_gemv_kind<kCode4, 16, WS>(p, q->packed, pl.nsplit, st);
-    }
+    return m <= 8 ? gv_launch<1>(prm, pl, st) : gv_launch<2>(prm, pl, st);
 }
 
-// One fused dequantize-GEMM over one stored weight (or one half of a
-// channel-mix weight).  `perm` maps its stored rows to output columns.
-lbq_status run_gemv(const void* X, int m, const lbq_qweight* q, const void* B, int rank, float s, const float* T,
-                    float* Y, int64_t ldy, const int32_t* perm, void* ws, int sms, cudaStream_t st) {
-    const Plan pl = plan_gemv(m, q, sms);
-    GemvParams p{};
-    p.m = m;
-    p.n = q->n;
-    p.k = q->k;
-    p.ngroups = q->scheme == LBQ_MINMAX_ASYM ? q->k / q->group : 0;
-    p.scale = q->scale;
-    p.zero = q->zero;
-    p.absmax = q->absmax;
-    p.q8 = (q->scheme == LBQ_CODEBOOK4 && q->double_quant) ? q->absmax_q8 : nullptr;
-    p.s2 = q->absmax_s2;
-    p.offset = q->absmax_offset;
-    p.codebook = q->codebook;
-    p.X = static_cast<const uint16_t*>(X);
-    p.rank = rank;
-    p.s = s;
-    p.T = T;
-    p.B = static_cast<const uint16_t*>(B);
-    p.Y = Y;
-    p.ldy = ldy;
-    p.perm = perm;
-    p.kbt = q->k / 64;
-    p.tiles = pl.tiles;
-    p.share = pl.per_split;
-    p.total = static_cast<int64_t>(pl.tiles) * p.kbt;
-    p.w_early = weights_stable(st) ? 1 : 0;
-    if (p.total >= (int64_t(1) << 31)) return LBQ_EUNSUPPORTED;
-    if (pl.workspace() > 0) {
-        if (!ws) return LBQ_EWORKSPACE;
-        if (pl.tiles > kMaxSplitTiles) return LBQ_EUNSUPPORTED;
-        p.partial = ws_partials(ws);
-        p.counters = ws_counters(ws);
+// Any number of matrices: groups of kGvMaxProblems, one launch each, in order.
+lbq_status run_gemv_jobs(int m, const GvJob* jobs, int count, void* ws, size_t ws_bytes, int sms, cudaStream_t st) {
+    for (int i = 0; i < count; i += kGvMaxProblems) {
+        const lbq_status s = run_gemv_group(m, jobs + i, std::min(kGvMaxProblems, count - i), ws, ws_bytes, sms, st);
+        if (s != LBQ_OK) return s;
     }
-    return launch_gemv_tile<4>(p, q, pl, st);
+    return LBQ_OK;
+}
+
+// Workspace of run_gemv_jobs: the largest of its launches'.
+size_t gemv_jobs_workspace(int m, const lbq_qweight* const* qs, int count, int sms) {
+    size_t need = 0;
+    for (int i = 0; i < count; i += kGvMaxProblems) {
+        GvPlan pl;
+        if (gv_plan(m, qs + i, std::min(kGvMaxProblems, count - i), sms, &pl) == LBQ_OK)
+            need = std::max(need, pl.workspace);
+    }
+    return need;
 }

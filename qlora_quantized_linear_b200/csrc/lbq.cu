@@ -1,8 +1,11 @@
 // lbq.cu -- the C ABI (include/lbq.h): argument validation, tensor-map setup,
 // tile and split selection, and kernel launches.  One translation unit holds
 // every kernel so that the device status word is a single object.
+#include <cmath>
+#include <cstring>
 #include <mutex>
 #include <unordered_set>
+#include <vector>
 
 #include "dqgemm.cuh"
 #include "dqgemm_bwd.cuh"
@@ -10,6 +13,8 @@
 #include "lora.cuh"
 #include "merge.cuh"
 #include "quantize.cuh"
+#include "select.cuh"
+#include "selftest.cuh"
 
 using namespace lbq;
 
@@ -138,7 +143,6 @@ struct Plan {
     int tiles;       // output tiles (rows x token tiles)
     int nsplit;      // K splits
     int per_split;   // reduction blocks per split
-    int stages = 4;  // decode GEMV: weight boxes in flight
     size_t partial_bytes;
     size_t workspace() const { return nsplit > 1 ? kCounterHeader + partial_bytes : 0; }
 };
@@ -178,10 +182,16 @@ bool weights_stable(cudaStream_t st) {
 
 #include "dqgemv_host.cuh"
 
-// Forward plan: splits start on a whole weight chunk (128 bytes of a row).
+// Forward plan of the tensor-core GEMM (m > 16): splits start on a whole
+// weight chunk (128 bytes of a row).
 Plan plan_fwd(int m, const lbq_qweight* q, int sms) {
-    if (m <= kGemvMaxM) return plan_gemv(m, q, sms);
     return plan_gemm(m, q->n, q->k / 64, sms, 256, q->bits == 2 ? 8 : 4);
+}
+
+// Workspace of one forward call (either path).
+size_t fwd_workspace(int m, const lbq_qweight* q, int sms) {
+    if (m <= kGemvMaxM) return gemv_jobs_workspace(m, &q, 1, sms);
+    return plan_fwd(m, q, sms).workspace();
 }
 
 template <int NT, int KIND>
@@ -190,7 +200,7 @@ lbq_status launch_fwd_nt(const FwdParams& p, const void* X, int m, int64_t k, co
     using C = FwdCfg<NT>;
     using L = FwdSmem<NT, C::kXStages, C::kXBlocks, C::kWStages, C::kAStages>;
     auto kern = dqgemm_fwd_kernel<NT, KIND, C::kXStages, C::kXBlocks, C::kWStages, C::kAStages, C::kMinBlocks>;
-    const size_t smem = L::total(p.rank_pad);
+    const size_t smem = L::total(p.rank);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
         return LBQ_ECUDA;
     CUtensorMap tmX, tmW;
@@ -216,9 +226,12 @@ lbq_status launch_fwd_kind(int nt, const FwdParams& p, const void* X, int m, int
 }
 
 lbq_status run_fwd_gemm(const void* X, int m, const lbq_qweight* q, const void* B, int rank, float s,
-                        const float* T, float* Y, int64_t ldy, const int32_t* perm, void* ws, int sms,
-                        cudaStream_t st) {
-    if (m <= kGemvMaxM) return run_gemv(X, m, q, B, rank, s, T, Y, ldy, perm, ws, sms, st);
+                        const float* T, float* Y, int64_t ldy, const int32_t* perm, void* ws, size_t ws_bytes,
+                        int sms, cudaStream_t st) {
+    if (m <= kGemvMaxM) {
+        const GvJob job{X, q, B, rank, s, T, Y, ldy, perm};
+        return run_gemv_jobs(m, &job, 1, ws, ws_bytes, sms, st);
+    }
     const Plan pl = plan_fwd(m, q, sms);
     FwdParams p{};
     p.m = m;
@@ -266,11 +279,12 @@ lbq_status check_lora(int rank, const void* A, const void* B, const void* saved)
 // ---------------------------------------------------------------------------
 // backward GEMM
 // ---------------------------------------------------------------------------
-template <int NT, int BITS>
+template <int NT, int KIND>
 lbq_status launch_bwd_nt(const BwdParams& p, const void* dY, const uint8_t* packed, cudaStream_t st) {
+    constexpr int BITS = KIND == kInt2 ? 2 : 4;
     using C = BwdCfg<NT>;
     using L = BwdSmem<NT, BITS, C::kXStages, C::kWStages, C::kAStages>;
-    auto kern = dqgemm_bwd_kernel<NT, BITS, C::kXStages, C::kWStages, C::kAStages, C::kMinBlocks>;
+    auto kern = dqgemm_bwd_kernel<NT, KIND, C::kXStages, C::kWStages, C::kAStages, C::kMinBlocks>;
     const size_t smem = L::total(p.rank_pad);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
         return LBQ_ECUDA;
@@ -286,14 +300,14 @@ lbq_status launch_bwd_nt(const BwdParams& p, const void* dY, const uint8_t* pack
     return last_launch();
 }
 
-template <int BITS>
-lbq_status launch_bwd_bits(int nt, const BwdParams& p, const void* dY, const uint8_t* packed, cudaStream_t st) {
+template <int KIND>
+lbq_status launch_bwd_kind(int nt, const BwdParams& p, const void* dY, const uint8_t* packed, cudaStream_t st) {
     switch (nt) {
-        case 16: return launch_bwd_nt<16, BITS>(p, dY, packed, st);
-        case 32: return launch_bwd_nt<32, BITS>(p, dY, packed, st);
-        case 64: return launch_bwd_nt<64, BITS>(p, dY, packed, st);
-        case 128: return launch_bwd_nt<128, BITS>(p, dY, packed, st);
-        default: return launch_bwd_nt<256, BITS>(p, dY, packed, st);
+        case 16: return launch_bwd_nt<16, KIND>(p, dY, packed, st);
+        case 32: return launch_bwd_nt<32, KIND>(p, dY, packed, st);
+        case 64: return launch_bwd_nt<64, KIND>(p, dY, packed, st);
+        case 128: return launch_bwd_nt<128, KIND>(p, dY, packed, st);
+        default: return launch_bwd_nt<256, KIND>(p, dY, packed, st);
     }
 }
 
@@ -302,29 +316,23 @@ lbq_status launch_bwd_bits(int nt, const BwdParams& p, const void* dY, const uin
 // ---------------------------------------------------------------------------
 // Fixed scratch of lbq_linear_fwd_noalloc.  Every device that loads this
 // library holds one copy until the process exits.  In host code the name
-// below is only a stand-in for the symbol; the device address of each
-// device's copy comes from cudaGetSymbolAddress, taken once per device with
-// that device current, on the first call made on it.
+// below is only a stand-in for the symbol; the device address of the current
+// device's copy comes from cudaGetSymbolAddress, with that device current, on
+// every call.  Both split-K paths of the forward (the decode GEMV and the
+// tensor-core GEMM) use it as their workspace.
 // ---------------------------------------------------------------------------
 static constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {
-constexpr int kNoAllocMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
-
+// The device address of the current device's copy of the array, looked up on
+// every call (a host-side lookup: no allocation, no synchronization once the
+// library's module is loaded on the device), so that a reloaded module after
+// a context teardown is never addressed through a stale pointer.
 lbq_status noalloc_scratch_address(void** out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return LBQ_ECUDA;
-    if (dev < 0 || dev >= kNoAllocMaxDevices) return LBQ_EUNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return LBQ_ECUDA;
-        g_noalloc_ptr[dev] = p;
-    }
-    *out = g_noalloc_ptr[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return LBQ_ECUDA;
+    *out = p;
     return LBQ_OK;
 }
 }  // namespace
@@ -553,19 +561,34 @@ lbq_status lbq_unmerge_lora(const void* W, int n, int k, const void* A, const vo
 size_t lbq_linear_fwd_workspace_size(int m, const lbq_qweight* q, int rank) {
     (void)rank;
     if (m < 1 || check_qweight(q, false) != LBQ_OK) return 0;
-    return plan_fwd(m, q, sm_count()).workspace();
+    return fwd_workspace(m, q, sm_count());
 }
 
-lbq_status lbq_gemv_plan(int m, const lbq_qweight* q, int sms, int64_t* plan) {
-    if (m < 1 || m > kGemvMaxM || !plan || check_qweight(q, false) != LBQ_OK) return LBQ_EINVAL;
+lbq_status lbq_gemv_plan(int m, const lbq_qweight* const* qs, int count, int sms, int64_t* plan,
+                         int64_t* per_problem) {
+    if (m < 1 || m > kGemvMaxM || !qs || !plan || count < 1 || count > kGvMaxProblems) return LBQ_EINVAL;
+    for (int i = 0; i < count; ++i)
+        if (check_qweight(qs[i], false) != LBQ_OK) return LBQ_EINVAL;
     if (sms <= 0) sms = sm_count();
-    const Plan pl = plan_gemv(m, q, sms);
-    plan[0] = pl.nsplit;
-    plan[1] = pl.per_split;
-    plan[2] = pl.tiles;
-    plan[3] = pl.stages;
-    plan[4] = static_cast<int64_t>(gemv_smem_bytes(m, pl.per_split, kind_of(q), pl.stages));
+    GvPlan pl;
+    const lbq_status st = gv_plan(m, qs, count, sms, &pl);
+    if (st != LBQ_OK) return st;
+    plan[0] = pl.ctas;
+    plan[1] = pl.ws;
+    plan[2] = pl.stage_bytes;
+    plan[3] = static_cast<int64_t>(pl.smem);
+    plan[4] = static_cast<int64_t>(pl.workspace);
     plan[5] = sms;
+    plan[6] = pl.xbox_max;
+    plan[7] = pl.cstride;
+    if (per_problem) {
+        for (int i = 0; i < count; ++i) {
+            per_problem[4 * i + 0] = pl.share[i];
+            per_problem[4 * i + 1] = pl.pctas[i];
+            per_problem[4 * i + 2] = pl.cta0[i];
+            per_problem[4 * i + 3] = pl.tiles[i];
+        }
+    }
     return LBQ_OK;
 }
 
@@ -578,14 +601,14 @@ lbq_status lbq_linear_fwd(const void* X, int m, const lbq_qweight* q, const void
     if (!aligned16(X) || !aligned16(Y)) return LBQ_EALIGN;
     if ((st = check_lora(rank, A, B, T_save)) != LBQ_OK) return st;
     const int sms = sm_count();
-    const size_t need = plan_fwd(m, q, sms).workspace();
+    const size_t need = fwd_workspace(m, q, sms);
     if (need > 0 && (!workspace || workspace_bytes < need)) return LBQ_EWORKSPACE;
     if (need > 0 && !aligned16(workspace)) return LBQ_EALIGN;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     if (rank > 0) {
         if ((st = launch_lora_rows<false>(X, m, q->k, A, rank, T_save, cs)) != LBQ_OK) return st;
     }
-    return run_fwd_gemm(X, m, q, B, rank, s, T_save, Y, q->n, nullptr, workspace, sms, cs);
+    return run_fwd_gemm(X, m, q, B, rank, s, T_save, Y, q->n, nullptr, workspace, workspace_bytes, sms, cs);
 }
 
 lbq_status lbq_linear_fwd_noalloc(const void* X, int m, const lbq_qweight* q, const void* A, const void* B, int rank,
@@ -596,7 +619,7 @@ lbq_status lbq_linear_fwd_noalloc(const void* X, int m, const lbq_qweight* q, co
     if (!aligned16(X) || !aligned16(Y)) return LBQ_EALIGN;
     if ((st = check_lora(rank, A, B, T_save)) != LBQ_OK) return st;
     const int sms = sm_count();
-    const size_t need = plan_fwd(m, q, sms).workspace();
+    const size_t need = fwd_workspace(m, q, sms);
     if (need > kNoAllocScratchBytes) return LBQ_EWORKSPACE;  // this call's scratch does not fit
     void* scratch = nullptr;
     if (need > 0 && (st = noalloc_scratch_address(&scratch)) != LBQ_OK) return st;
@@ -604,15 +627,82 @@ lbq_status lbq_linear_fwd_noalloc(const void* X, int m, const lbq_qweight* q, co
     if (rank > 0) {
         if ((st = launch_lora_rows<false>(X, m, q->k, A, rank, T_save, cs)) != LBQ_OK) return st;
     }
-    return run_fwd_gemm(X, m, q, B, rank, s, T_save, Y, q->n, nullptr, scratch, sms, cs);
+    return run_fwd_gemm(X, m, q, B, rank, s, T_save, Y, q->n, nullptr, scratch, kNoAllocScratchBytes, sms, cs);
+}
+
+size_t lbq_linear_fwd_grouped_workspace_size(int m, const lbq_fwd_problem* probs, int count) {
+    if (m < 1 || !probs || count < 1) return 0;
+    const int sms = sm_count();
+    if (m <= kGemvMaxM) {
+        std::vector<const lbq_qweight*> qs(count);
+        for (int i = 0; i < count; ++i) {
+            if (check_qweight(probs[i].q, false) != LBQ_OK) return 0;
+            qs[i] = probs[i].q;
+        }
+        return gemv_jobs_workspace(m, qs.data(), count, sms);
+    }
+    size_t need = 0;
+    for (int i = 0; i < count; ++i) {
+        if (check_qweight(probs[i].q, false) != LBQ_OK) return 0;
+        need = std::max(need, plan_fwd(m, probs[i].q, sms).workspace());
+    }
+    return need;
+}
+
+lbq_status lbq_linear_fwd_grouped(int m, const lbq_fwd_problem* probs, int count, void* workspace,
+                                  size_t workspace_bytes, lbq_stream_t stream) {
+    if (m < 1 || !probs || count < 1) return LBQ_EINVAL;
+    lbq_status st;
+    for (int i = 0; i < count; ++i) {
+        const lbq_fwd_problem& pr = probs[i];
+        if ((st = check_qweight(pr.q, true)) != LBQ_OK) return st;
+        if (!pr.X || !pr.Y) return LBQ_EINVAL;
+        if (!aligned16(pr.X) || !aligned16(pr.Y)) return LBQ_EALIGN;
+        if ((st = check_lora(pr.rank, pr.A, pr.B, pr.T_save)) != LBQ_OK) return st;
+    }
+    const size_t need = lbq_linear_fwd_grouped_workspace_size(m, probs, count);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return LBQ_EWORKSPACE;
+    if (need > 0 && !aligned16(workspace)) return LBQ_EALIGN;
+    const int sms = sm_count();
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    for (int i = 0; i < count; ++i) {
+        const lbq_fwd_problem& pr = probs[i];
+        if (pr.rank > 0 && (st = launch_lora_rows<false>(pr.X, m, pr.q->k, pr.A, pr.rank, pr.T_save, cs)) != LBQ_OK)
+            return st;
+    }
+    if (m > kGemvMaxM) {
+        // large batches: one tensor-core GEMM per matrix, in order, sharing the workspace
+        for (int i = 0; i < count; ++i) {
+            const lbq_fwd_problem& pr = probs[i];
+            if ((st = run_fwd_gemm(pr.X, m, pr.q, pr.B, pr.rank, pr.s, pr.T_save, pr.Y, pr.q->n, nullptr, workspace,
+                                   workspace_bytes, sms, cs)) != LBQ_OK)
+                return st;
+        }
+        return LBQ_OK;
+    }
+    std::vector<GvJob> jobs(count);
+    for (int i = 0; i < count; ++i) {
+        const lbq_fwd_problem& pr = probs[i];
+        jobs[i] = GvJob{pr.X, pr.q, pr.B, pr.rank, pr.s, pr.T_save, pr.Y, pr.q->n, nullptr};
+    }
+    return run_gemv_jobs(m, jobs.data(), count, workspace, workspace_bytes, sms, cs);
+}
+
+// Channel-mix: the two halves in one grouped launch (m <= 16) or one GEMM
+// each (m > 16), writing their rows' output columns through perm.
+size_t mix_workspace(int m, const lbq_qweight_mix* q, int sms) {
+    if (m <= kGemvMaxM) {
+        const lbq_qweight* qs[2] = {&q->hi, &q->lo};
+        return gemv_jobs_workspace(m, qs, 2, sms);
+    }
+    return std::max(plan_fwd(m, &q->hi, sms).workspace(), plan_fwd(m, &q->lo, sms).workspace());
 }
 
 size_t lbq_linear_fwd_mix_workspace_size(int m, const lbq_qweight_mix* q, int rank) {
     (void)rank;
     if (!q || m < 1) return 0;
     if (check_qweight(&q->hi, false) != LBQ_OK || check_qweight(&q->lo, false) != LBQ_OK) return 0;
-    const int sms = sm_count();
-    return std::max(plan_fwd(m, &q->hi, sms).workspace(), plan_fwd(m, &q->lo, sms).workspace());
+    return mix_workspace(m, q, sm_count());
 }
 
 lbq_status lbq_linear_fwd_mix(const void* X, int m, const lbq_qweight_mix* q, const void* A, const void* B, int rank,
@@ -628,8 +718,7 @@ lbq_status lbq_linear_fwd_mix(const void* X, int m, const lbq_qweight_mix* q, co
     if (!aligned16(X) || !aligned16(Y) || !aligned16(q->perm)) return LBQ_EALIGN;
     if ((st = check_lora(rank, A, B, T_save)) != LBQ_OK) return st;
     const int sms = sm_count();
-    // the two halves run one after the other on `stream` and share the workspace
-    const size_t need = std::max(plan_fwd(m, &q->hi, sms).workspace(), plan_fwd(m, &q->lo, sms).workspace());
+    const size_t need = mix_workspace(m, q, sms);
     if (need > 0 && (!workspace || workspace_bytes < need)) return LBQ_EWORKSPACE;
     if (need > 0 && !aligned16(workspace)) return LBQ_EALIGN;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
@@ -637,9 +726,16 @@ lbq_status lbq_linear_fwd_mix(const void* X, int m, const lbq_qweight_mix* q, co
     if (rank > 0) {
         if ((st = launch_lora_rows<false>(X, m, q->hi.k, A, rank, T_save, cs)) != LBQ_OK) return st;
     }
-    if ((st = run_fwd_gemm(X, m, &q->hi, B, rank, s, T_save, Y, n_total, q->perm, workspace, sms, cs)) != LBQ_OK)
+    if (m <= kGemvMaxM) {
+        const GvJob jobs[2] = {GvJob{X, &q->hi, B, rank, s, T_save, Y, n_total, q->perm},
+                               GvJob{X, &q->lo, B, rank, s, T_save, Y, n_total, q->perm + q->hi.n}};
+        return run_gemv_jobs(m, jobs, 2, workspace, workspace_bytes, sms, cs);
+    }
+    if ((st = run_fwd_gemm(X, m, &q->hi, B, rank, s, T_save, Y, n_total, q->perm, workspace, workspace_bytes, sms,
+                           cs)) != LBQ_OK)
         return st;
-    return run_fwd_gemm(X, m, &q->lo, B, rank, s, T_save, Y, n_total, q->perm + q->hi.n, workspace, sms, cs);
+    return run_fwd_gemm(X, m, &q->lo, B, rank, s, T_save, Y, n_total, q->perm + q->hi.n, workspace, workspace_bytes,
+                        sms, cs);
 }
 
 size_t lbq_linear_bwd_workspace_size(int m, const lbq_qweight* q, int rank) {
@@ -653,7 +749,6 @@ lbq_status lbq_linear_bwd(const void* dY, int m, const lbq_qweight* q, const voi
                           lbq_stream_t stream) {
     lbq_status st = check_qweight(q, true);
     if (st != LBQ_OK) return st;
-    if (q->scheme != LBQ_MINMAX_ASYM) return LBQ_EUNSUPPORTED;
     if (m < 1 || !dY || !dX || q->n % 8 != 0) return LBQ_EINVAL;
     if (!aligned16(dY) || !aligned16(dX)) return LBQ_EALIGN;
     if ((st = check_lora(rank, A, B, U_save)) != LBQ_OK) return st;
@@ -674,6 +769,11 @@ lbq_status lbq_linear_bwd(const void* dY, int m, const lbq_qweight* q, const voi
     p.group = q->group;
     p.scale = q->scale;
     p.zero = q->zero;
+    p.absmax = q->absmax;
+    p.q8 = (q->scheme == LBQ_CODEBOOK4 && q->double_quant) ? q->absmax_q8 : nullptr;
+    p.s2 = q->absmax_s2;
+    p.offset = q->absmax_offset;
+    p.codebook = q->codebook;
     p.rank = rank;
     p.rank_pad = rank > 0 ? (rank + 15) / 16 * 16 : 16;
     p.s = s;
@@ -687,8 +787,11 @@ lbq_status lbq_linear_bwd(const void* dY, int m, const lbq_qweight* q, const voi
         p.partial = ws_partials(workspace);
         p.counters = ws_counters(workspace);
     }
-    if (q->bits == 4) return launch_bwd_bits<4>(pl.nt, p, dY, q->packed, cs);
-    return launch_bwd_bits<2>(pl.nt, p, dY, q->packed, cs);
+    switch (kind_of(q)) {
+        case kInt4: return launch_bwd_kind<kInt4>(pl.nt, p, dY, q->packed, cs);
+        case kInt2: return launch_bwd_kind<kInt2>(pl.nt, p, dY, q->packed, cs);
+        default: return launch_bwd_kind<kCode4>(pl.nt, p, dY, q->packed, cs);
+    }
 }
 
 lbq_status lbq_lora_grads(const void* X, const void* dY, int m, int n, int k, const float* T, const float* U,
@@ -713,6 +816,67 @@ int lbq_trace_read(long long* host, int n) {
     return total;
 }
 #endif
+
+size_t lbq_channel_mix_select_workspace_size(int n, int k) {
+    if (n < 1 || k < 128) return 0;
+    return round_up(static_cast<size_t>(k) * sizeof(double), 256) + round_up(static_cast<size_t>(n) * sizeof(double), 256) +
+           round_up(static_cast<size_t>(n), 256);
+}
+
+lbq_status lbq_channel_mix_select(const void* W_bf16, int n, int k, const void* X_bf16, int t, int n4, double* score,
+                                  int32_t* perm, void* workspace, size_t workspace_bytes, lbq_stream_t stream) {
+    if (!W_bf16 || !X_bf16 || !perm || n < 1 || k < 128 || k % 128 != 0 || t < 1 || n4 < 0 || n4 > n)
+        return LBQ_EINVAL;
+    if (!aligned16(W_bf16) || !aligned16(X_bf16) || !aligned16(perm) || (score && !aligned16(score)))
+        return LBQ_EALIGN;
+    const size_t need = lbq_channel_mix_select_workspace_size(n, k);
+    if (!workspace || workspace_bytes < need) return LBQ_EWORKSPACE;
+    if (!aligned16(workspace)) return LBQ_EALIGN;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    double* m2 = reinterpret_cast<double*>(ws);
+    double* sc = reinterpret_cast<double*>(ws + round_up(static_cast<size_t>(k) * sizeof(double), 256));
+    uint8_t* sel = ws + round_up(static_cast<size_t>(k) * sizeof(double), 256) +
+                   round_up(static_cast<size_t>(n) * sizeof(double), 256);
+    if (score) sc = score;
+    second_moment_kernel<<<static_cast<unsigned>(cdiv(k, 256)), 256, 0, cs>>>(static_cast<const uint16_t*>(X_bf16), t,
+                                                                             k, m2);
+    lbq_status st = last_launch();
+    if (st != LBQ_OK) return st;
+    channel_score_kernel<<<static_cast<unsigned>(cdiv(n, 8)), 256, 0, cs>>>(static_cast<const uint16_t*>(W_bf16), n, k,
+                                                                          m2, sc);
+    if ((st = last_launch()) != LBQ_OK) return st;
+    channel_rank_kernel<<<static_cast<unsigned>(cdiv(n, 256)), 256, 0, cs>>>(sc, n, n4, sel);
+    if ((st = last_launch()) != LBQ_OK) return st;
+    channel_perm_kernel<<<1, 1024, 0, cs>>>(sel, n, n4, perm);
+    return last_launch();
+}
+
+lbq_status lbq_gather_rows(const void* W_bf16, int n, int k, const int32_t* rows, int count, void* out,
+                           lbq_stream_t stream) {
+    if (!W_bf16 || !rows || !out || n < 1 || k < 8 || k % 8 != 0 || count < 1) return LBQ_EINVAL;
+    if (!aligned16(W_bf16) || !aligned16(out)) return LBQ_EALIGN;
+    const int64_t total = static_cast<int64_t>(count) * (k / 8);
+    const int grid = static_cast<int>(std::min<int64_t>(cdiv(total, 256), 16LL * sm_count()));
+    gather_rows_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4*>(W_bf16), k / 8, rows, count, static_cast<uint4*>(out));
+    return last_launch();
+}
+
+lbq_status lbq_linear_fwd_noalloc_reset(lbq_stream_t stream) {
+    void* scratch = nullptr;
+    lbq_status st = noalloc_scratch_address(&scratch);
+    if (st != LBQ_OK) return st;
+    return cudaMemsetAsync(scratch, 0, kCounterHeader, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? LBQ_OK
+               : LBQ_ECUDA;
+}
+
+lbq_status lbq_selftest_wait_timeout(uint32_t limit_us, lbq_stream_t stream) {
+    if (limit_us < 1 || limit_us > 1000000u) return LBQ_EINVAL;
+    wait_timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(uint64_t(limit_us) * 1000u);
+    return last_launch();
+}
 
 lbq_status lbq_device_status(uint32_t* flags) {
     if (!flags) return LBQ_EINVAL;

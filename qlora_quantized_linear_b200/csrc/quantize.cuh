@@ -36,76 +36,94 @@ __device__ __forceinline__ float rint_div(float w, float d, float rs) {
 
 // ---------------------------------------------------------------------------
 // MinMax quantize + pack.  Group = 128 (4 bit) or 64 (2 bit); one group is
-// covered by GROUP/8 consecutive lanes.
+// covered by GROUP/8 consecutive lanes.  Each warp first issues the 16-byte
+// loads of kQuantUnroll chunks of 32 lanes (a grid stride apart), then
+// processes them, so that several loads per lane are in flight.
 // ---------------------------------------------------------------------------
+constexpr int kQuantUnroll = 4;
+
+template <int BITS>
+__device__ __forceinline__ void minmax_quantize_chunk(uint4 raw, int64_t chunk, bool valid, int lane,
+                                                      uint8_t* __restrict__ packed, uint16_t* __restrict__ scale,
+                                                      uint16_t* __restrict__ zero) {
+    constexpr int GROUP = (BITS == 4) ? 128 : 64;
+    constexpr int LPG = GROUP / 8;  // lanes per group
+    constexpr float Q = static_cast<float>((1 << BITS) - 1);
+    const uint32_t words[4] = {raw.x, raw.y, raw.z, raw.w};
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = bf16_bits_to_f32(words[i] & 0xFFFFu);
+        v[2 * i + 1] = bf16_bits_to_f32(words[i] >> 16);
+    }
+    float mn = v[0], mx = v[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) {
+        mn = fminf(mn, v[i]);
+        mx = fmaxf(mx, v[i]);
+    }
+#pragma unroll
+    for (int off = LPG / 2; off > 0; off >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
+        mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+    }
+    if (!valid) return;  // whole groups are either valid or not
+    // -0 and +0 compare equal; adding +0 makes both extremes +0.
+    mn = __fadd_rn(mn, 0.0f);
+    mx = __fadd_rn(mx, 0.0f);
+    const float r = __fsub_rn(mx, mn);
+    uint16_t s16 = f32_to_f16_bits(__fdiv_rn(r, Q));
+    if (r == 0.0f || (s16 & 0x7FFFu) == 0) s16 = 0x3C00u;  // 1.0
+    const float sf = f16_bits_to_f32(s16);
+    const uint16_t z16 = f32_to_f16_bits(rintf(__fdiv_rn(-mn, sf)));
+    const float zf = f16_bits_to_f32(z16);
+    uint32_t q[8];
+    const float rs = __frcp_rn(sf);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float t = rint_div(v[i], sf, rs);
+        t = __fadd_rn(t, zf);
+        t = fminf(fmaxf(t, 0.0f), Q);
+        q[i] = static_cast<uint32_t>(t);
+    }
+    if (BITS == 4) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) word |= ((q[2 * j] << 4) | q[2 * j + 1]) << (8 * j);
+        reinterpret_cast<uint32_t*>(packed)[chunk] = word;
+    } else {
+        uint32_t half = 0;
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+            half |= ((q[4 * j] << 6) | (q[4 * j + 1] << 4) | (q[4 * j + 2] << 2) | q[4 * j + 3]) << (8 * j);
+        reinterpret_cast<uint16_t*>(packed)[chunk] = static_cast<uint16_t>(half);
+    }
+    if ((lane & (LPG - 1)) == 0) {
+        const int64_t g = chunk / LPG;
+        scale[g] = s16;
+        zero[g] = z16;
+    }
+}
+
 template <int BITS>
 __global__ void __launch_bounds__(256) minmax_quantize_kernel(const uint4* __restrict__ W, int64_t nchunks,
                                                               uint8_t* __restrict__ packed,
                                                               uint16_t* __restrict__ scale,
                                                               uint16_t* __restrict__ zero) {
-    constexpr int GROUP = (BITS == 4) ? 128 : 64;
-    constexpr int LPG = GROUP / 8;  // lanes per group
-    constexpr float Q = static_cast<float>((1 << BITS) - 1);
     const int lane = threadIdx.x & 31;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31u); base < nchunks;
-         base += stride) {
-        const int64_t chunk = base + lane;
-        const bool valid = chunk < nchunks;
-        uint4 raw = valid ? __ldg(W + chunk) : make_uint4(0, 0, 0, 0);
-        const uint32_t words[4] = {raw.x, raw.y, raw.z, raw.w};
-        float v[8];
+         base += kQuantUnroll * stride) {
+        uint4 raw[kQuantUnroll];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            v[2 * i] = bf16_bits_to_f32(words[i] & 0xFFFFu);
-            v[2 * i + 1] = bf16_bits_to_f32(words[i] >> 16);
-        }
-        float mn = v[0], mx = v[0];
-#pragma unroll
-        for (int i = 1; i < 8; ++i) {
-            mn = fminf(mn, v[i]);
-            mx = fmaxf(mx, v[i]);
+        for (int u = 0; u < kQuantUnroll; ++u) {
+            const int64_t chunk = base + u * stride + lane;
+            raw[u] = chunk < nchunks ? __ldg(W + chunk) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
-        for (int off = LPG / 2; off > 0; off >>= 1) {
-            mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
-            mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
-        }
-        if (!valid) continue;  // whole groups are either valid or not
-        // -0 and +0 compare equal; adding +0 makes both extremes +0.
-        mn = __fadd_rn(mn, 0.0f);
-        mx = __fadd_rn(mx, 0.0f);
-        const float r = __fsub_rn(mx, mn);
-        uint16_t s16 = f32_to_f16_bits(__fdiv_rn(r, Q));
-        if (r == 0.0f || (s16 & 0x7FFFu) == 0) s16 = 0x3C00u;  // 1.0
-        const float sf = f16_bits_to_f32(s16);
-        const uint16_t z16 = f32_to_f16_bits(rintf(__fdiv_rn(-mn, sf)));
-        const float zf = f16_bits_to_f32(z16);
-        uint32_t q[8];
-        const float rs = __frcp_rn(sf);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            float t = rint_div(v[i], sf, rs);
-            t = __fadd_rn(t, zf);
-            t = fminf(fmaxf(t, 0.0f), Q);
-            q[i] = static_cast<uint32_t>(t);
-        }
-        if (BITS == 4) {
-            uint32_t word = 0;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) word |= ((q[2 * j] << 4) | q[2 * j + 1]) << (8 * j);
-            reinterpret_cast<uint32_t*>(packed)[chunk] = word;
-        } else {
-            uint32_t half = 0;
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-                half |= ((q[4 * j] << 6) | (q[4 * j + 1] << 4) | (q[4 * j + 2] << 2) | q[4 * j + 3]) << (8 * j);
-            reinterpret_cast<uint16_t*>(packed)[chunk] = static_cast<uint16_t>(half);
-        }
-        if ((lane & (LPG - 1)) == 0) {
-            const int64_t g = chunk / LPG;
-            scale[g] = s16;
-            zero[g] = z16;
+        for (int u = 0; u < kQuantUnroll; ++u) {
+            const int64_t chunk = base + u * stride + lane;
+            minmax_quantize_chunk<BITS>(raw[u], chunk, chunk < nchunks, lane, packed, scale, zero);
         }
     }
 }
@@ -115,32 +133,55 @@ __global__ void __launch_bounds__(256) minmax_quantize_kernel(const uint4* __res
 // Also accumulates, per CTA, the fp64 sum of the block absmax values (used by
 // double quantization; exact under the documented range condition).
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ bool codebook_ok(const float* c) {
+// The table in code order c[0..15] (any order; equal entries allowed, such
+// as the +0 and -0 of the FP4 table) as a search table: its distinct values
+// in increasing order u[0..nu-1] (+inf after them), and for each the lowest
+// code that holds it.  Returns false when the table breaks the preconditions:
+// entries in [-1, 1], a zero among them, distinct values at least 2^-20
+// apart (then the nearest-value search below equals the exhaustive
+// search with its lower-index tie rule).  One thread builds it.
+__device__ __forceinline__ bool codebook_search_table(const float* c, float* u, uint32_t* rep) {
     bool ok = true, has_zero = false;
-#pragma unroll
+    int nu = 0;
     for (int j = 0; j < 16; ++j) {
         has_zero |= (c[j] == 0.0f);
         ok &= (c[j] >= -1.0f) && (c[j] <= 1.0f);
-        // strictly increasing with gaps of at least 2^-20: the nearest-entry
-        // search below then equals the exhaustive search with its tie rule
-        if (j > 0) ok &= (c[j] - c[j - 1]) >= 9.5367431640625e-07f;
+        // insert value c[j] (code j) unless an equal value is already there
+        // (codes are visited in increasing order, so the first code stays)
+        int pos = 0;
+        while (pos < nu && u[pos] < c[j]) ++pos;
+        if (pos < nu && u[pos] == c[j]) continue;
+        for (int i = nu; i > pos; --i) {
+            u[i] = u[i - 1];
+            rep[i] = rep[i - 1];
+        }
+        u[pos] = c[j];
+        rep[pos] = static_cast<uint32_t>(j);
+        ++nu;
+    }
+    for (int i = 1; i < nu; ++i) ok &= (u[i] - u[i - 1]) >= 9.5367431640625e-07f;
+    for (int i = nu; i < 16; ++i) {
+        u[i] = __int_as_float(0x7f800000);   // +inf: never below x, never nearest
+        rep[i] = 15u;
     }
     return ok && has_zero;
 }
 
-// Index of the entry nearest to x, the lower index on a tie.  The table is
-// sorted, so the nearest entry is one of the two that bracket x.
-__device__ __forceinline__ uint32_t nearest_code(const float* c, float x) {
+// Code of the entry nearest to x, the lower code on a tie.  The search
+// table is sorted, so the nearest value is one of the two that bracket x.
+__device__ __forceinline__ uint32_t nearest_code(const float* u, const uint32_t* rep, float x) {
     int j = -1;
-    if (c[j + 8] <= x) j += 8;
-    if (c[j + 4] <= x) j += 4;
-    if (c[j + 2] <= x) j += 2;
-    if (c[j + 1] <= x) j += 1;
-    if (j < 0) return 0;
-    if (j == 15) return 15;
-    const float d0 = fabsf(__fsub_rn(x, c[j]));
-    const float d1 = fabsf(__fsub_rn(x, c[j + 1]));
-    return (d1 < d0) ? static_cast<uint32_t>(j + 1) : static_cast<uint32_t>(j);
+    if (u[j + 8] <= x) j += 8;
+    if (u[j + 4] <= x) j += 4;
+    if (u[j + 2] <= x) j += 2;
+    if (u[j + 1] <= x) j += 1;
+    if (j < 0) return rep[0];
+    if (j == 15) return rep[15];
+    const float d0 = fabsf(__fsub_rn(x, u[j]));
+    const float d1 = fabsf(__fsub_rn(x, u[j + 1]));
+    if (d1 < d0) return rep[j + 1];
+    if (d0 < d1) return rep[j];
+    return min(rep[j], rep[j + 1]);
 }
 
 __global__ void __launch_bounds__(256) codebook_quantize_kernel(const uint4* __restrict__ W, int64_t nchunks,
@@ -149,18 +190,20 @@ __global__ void __launch_bounds__(256) codebook_quantize_kernel(const uint4* __r
                                                                 float* __restrict__ absmax,
                                                                 double* __restrict__ cta_sums) {
     __shared__ float s_cb[16];
+    __shared__ float s_u[16];
+    __shared__ uint32_t s_rep[16];
     __shared__ double s_sum[8];
     if (threadIdx.x < 16) s_cb[threadIdx.x] = codebook[threadIdx.x];
     __syncthreads();
-    if (threadIdx.x == 0 && blockIdx.x == 0 && !codebook_ok(s_cb)) record_status(kStatusBadTable);
+    if (threadIdx.x == 0) {
+        const bool ok = codebook_search_table(s_cb, s_u, s_rep);
+        if (blockIdx.x == 0 && !ok) record_status(kStatusBadTable);
+    }
+    __syncthreads();
     const int lane = threadIdx.x & 31;
     double my_sum = 0.0;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31u); base < nchunks;
-         base += stride) {
-        const int64_t chunk = base + lane;
-        const bool valid = chunk < nchunks;
-        uint4 raw = valid ? __ldg(W + chunk) : make_uint4(0, 0, 0, 0);
+    auto process = [&](uint4 raw, int64_t chunk, bool valid) {
         const uint32_t words[4] = {raw.x, raw.y, raw.z, raw.w};
         float v[8];
         float a = 0.0f;
@@ -172,18 +215,32 @@ __global__ void __launch_bounds__(256) codebook_quantize_kernel(const uint4* __r
         }
 #pragma unroll
         for (int off = 4; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
-        if (!valid) continue;
+        if (!valid) return;
         uint32_t word = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const float x0 = (a == 0.0f) ? 0.0f : __fdiv_rn(v[2 * j], a);
             const float x1 = (a == 0.0f) ? 0.0f : __fdiv_rn(v[2 * j + 1], a);
-            word |= ((nearest_code(s_cb, x0) << 4) | nearest_code(s_cb, x1)) << (8 * j);
+            word |= ((nearest_code(s_u, s_rep, x0) << 4) | nearest_code(s_u, s_rep, x1)) << (8 * j);
         }
         reinterpret_cast<uint32_t*>(packed)[chunk] = word;
         if ((lane & 7) == 0) {
             absmax[chunk >> 3] = a;
             my_sum += static_cast<double>(a);
+        }
+    };
+    for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31u); base < nchunks;
+         base += kQuantUnroll * stride) {
+        uint4 raw[kQuantUnroll];
+#pragma unroll
+        for (int u = 0; u < kQuantUnroll; ++u) {
+            const int64_t chunk = base + u * stride + lane;
+            raw[u] = chunk < nchunks ? __ldg(W + chunk) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kQuantUnroll; ++u) {
+            const int64_t chunk = base + u * stride + lane;
+            process(raw[u], chunk, chunk < nchunks);
         }
     }
     if (cta_sums != nullptr) {

@@ -47,8 +47,15 @@ class lbq_qweight_mix(ctypes.Structure):
     _fields_ = [("hi", lbq_qweight), ("lo", lbq_qweight), ("perm", ctypes.c_void_p)]
 
 
+class lbq_fwd_problem(ctypes.Structure):
+    _fields_ = [("X", ctypes.c_void_p), ("q", ctypes.POINTER(lbq_qweight)), ("A", ctypes.c_void_p),
+                ("B", ctypes.c_void_p), ("rank", ctypes.c_int32), ("s", ctypes.c_float),
+                ("Y", ctypes.c_void_p), ("T_save", ctypes.c_void_p)]
+
+
 _vp, _int, _f32, _sz, _u32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.POINTER(ctypes.c_uint32)
 _QP, _MP = ctypes.POINTER(lbq_qweight), ctypes.POINTER(lbq_qweight_mix)
+_PP, _QPP, _I64P = ctypes.POINTER(lbq_fwd_problem), ctypes.POINTER(ctypes.POINTER(lbq_qweight)), ctypes.POINTER(ctypes.c_int64)
 _SIGS = {
     "lbq_status_string": (ctypes.c_char_p, [_int]),
     "lbq_quantize_workspace_size": (_sz, [_QP]),
@@ -64,8 +71,15 @@ _SIGS = {
     "lbq_lora_grads": (_int, [_vp, _vp, _int, _int, _int, _vp, _vp, _int, _f32, _vp, _vp, _vp]),
     "lbq_device_status": (_int, [_u32p]),
     "lbq_merge_lora": (_int, [_QP, _vp, _vp, _int, _f32, _vp, _vp]),
-    "lbq_gemv_plan": (_int, [_int, _QP, _int, ctypes.POINTER(ctypes.c_int64)]),
+    "lbq_gemv_plan": (_int, [_int, _QPP, _int, _int, _I64P, _I64P]),
+    "lbq_linear_fwd_grouped_workspace_size": (_sz, [_int, _PP, _int]),
+    "lbq_linear_fwd_grouped": (_int, [_int, _PP, _int, _vp, _sz, _vp]),
     "lbq_unmerge_lora": (_int, [_vp, _int, _int, _vp, _vp, _int, _f32, _vp, _vp]),
+    "lbq_linear_fwd_noalloc_reset": (_int, [_vp]),
+    "lbq_channel_mix_select_workspace_size": (_sz, [_int, _int]),
+    "lbq_channel_mix_select": (_int, [_vp, _int, _int, _vp, _int, _int, _vp, _vp, _vp, _sz, _vp]),
+    "lbq_gather_rows": (_int, [_vp, _int, _int, _vp, _int, _vp, _vp]),
+    "lbq_selftest_wait_timeout": (_int, [ctypes.c_uint32, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_L, _name)
@@ -94,7 +108,14 @@ lbq_lora_grads = _L.lbq_lora_grads
 lbq_device_status = _L.lbq_device_status
 lbq_merge_lora = _L.lbq_merge_lora
 lbq_gemv_plan = _L.lbq_gemv_plan
+lbq_linear_fwd_grouped_workspace_size = _L.lbq_linear_fwd_grouped_workspace_size
+lbq_linear_fwd_grouped = _L.lbq_linear_fwd_grouped
 lbq_unmerge_lora = _L.lbq_unmerge_lora
+lbq_linear_fwd_noalloc_reset = _L.lbq_linear_fwd_noalloc_reset
+lbq_channel_mix_select_workspace_size = _L.lbq_channel_mix_select_workspace_size
+lbq_channel_mix_select = _L.lbq_channel_mix_select
+lbq_gather_rows = _L.lbq_gather_rows
+lbq_selftest_wait_timeout = _L.lbq_selftest_wait_timeout
 
 
 class LbqError(RuntimeError):
@@ -207,6 +228,44 @@ class ChannelMixWeight:
         self.struct = lbq_qweight_mix(hi=hi.struct, lo=lo.struct, perm=self.perm.data_ptr())
 
 
+def channel_mix_select(W, X_calib, n4: int, stream=None):
+    """(perm int32 [n], score fp64 [n]) on the device: the n4 channels of W
+    whose INT4 -> INT2 error rise, weighted by the calibration activations'
+    second moments, is largest come first (lbq_channel_mix_select)."""
+    torch = _torch()
+    W, X_calib = _bf16_2d(W, "W"), _bf16_2d(X_calib, "X_calib")
+    n, k = W.shape
+    perm = torch.empty(n, dtype=torch.int32, device=W.device)
+    score = torch.empty(n, dtype=torch.float64, device=W.device)
+    nws = lbq_channel_mix_select_workspace_size(n, k)
+    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=W.device)
+    _check(lbq_channel_mix_select(W.data_ptr(), n, k, X_calib.data_ptr(), X_calib.shape[0], int(n4), score.data_ptr(),
+                                  perm.data_ptr(), ws.data_ptr(), nws, _stream(stream)), "lbq_channel_mix_select")
+    return perm, score
+
+
+def gather_rows(W, rows, stream=None):
+    """W[rows] (bf16 rows gathered on the device by lbq_gather_rows)."""
+    torch = _torch()
+    W = _bf16_2d(W, "W")
+    rows = torch.as_tensor(rows, dtype=torch.int32, device=W.device).contiguous()
+    out = torch.empty((rows.numel(), W.shape[1]), dtype=torch.bfloat16, device=W.device)
+    _check(lbq_gather_rows(W.data_ptr(), W.shape[0], W.shape[1], rows.data_ptr(), rows.numel(), out.data_ptr(),
+                           _stream(stream)), "lbq_gather_rows")
+    return out
+
+
+def channel_mix_weight(W, X_calib, frac_int4: float = 0.25, stream=None):
+    """A ChannelMixWeight of W: the round(frac_int4 * n) most sensitive channels
+    (lbq_channel_mix_select) as INT4 g128 rows, the others as INT2 g64 rows."""
+    n, k = W.shape
+    n4 = int(round(frac_int4 * n))
+    perm, _ = channel_mix_select(W, X_calib, n4, stream=stream)
+    hi = QuantizedWeight(n4, k, "minmax", 4).quantize(gather_rows(W, perm[:n4], stream=stream), stream=stream)
+    lo = QuantizedWeight(n - n4, k, "minmax", 2).quantize(gather_rows(W, perm[n4:], stream=stream), stream=stream)
+    return ChannelMixWeight(hi, lo, perm)
+
+
 def _workspace(nbytes: int, device):
     torch = _torch()
     # zero-filled once: the library leaves its counters at zero after every call
@@ -232,6 +291,35 @@ def linear_fwd(X, qw, A=None, B=None, s: float = 0.0, Y=None, T=None, workspace=
     _check(fn(X.data_ptr(), m, ctypes.byref(qw.struct), _ptr(A), _ptr(B), rank, float(s), Y.data_ptr(), _ptr(T),
               _ptr(workspace), nws, _stream(stream)), fn.__name__)
     return Y, T
+
+
+def linear_fwd_grouped(problems, workspace=None, stream=None):
+    """Several forwards with the same token count in one call.  `problems` is a
+    list of (X, qw) or (X, qw, A, B, s) tuples; returns the list of Y (and T
+    when an adapter is given) as linear_fwd would."""
+    torch = _torch()
+    arr = (lbq_fwd_problem * len(problems))()
+    outs, keep = [], []
+    m = None
+    for i, pr in enumerate(problems):
+        X, qw = _bf16_2d(pr[0], "X"), pr[1]
+        A, B, s = (pr[2], pr[3], pr[4]) if len(pr) > 2 else (None, None, 0.0)
+        m = X.shape[0] if m is None else m
+        if X.shape[0] != m:
+            raise ValueError("all problems of a grouped call have the same token count")
+        rank = 0 if A is None else int(A.shape[0])
+        Y = torch.empty((m, qw.n), dtype=torch.float32, device=X.device)
+        T = torch.empty((m, rank), dtype=torch.float32, device=X.device) if rank else None
+        arr[i] = lbq_fwd_problem(X=X.data_ptr(), q=ctypes.pointer(qw.struct), A=_ptr(A), B=_ptr(B), rank=rank,
+                                 s=float(s), Y=Y.data_ptr(), T_save=_ptr(T))
+        outs.append((Y, T))
+        keep.append((X, A, B))
+    nws = lbq_linear_fwd_grouped_workspace_size(m, arr, len(problems))
+    if workspace is None:
+        workspace = _workspace(nws, problems[0][0].device)
+    _check(lbq_linear_fwd_grouped(m, arr, len(problems), _ptr(workspace), nws, _stream(stream)),
+           "lbq_linear_fwd_grouped")
+    return outs
 
 
 def linear_bwd(dY, qw, A=None, B=None, s: float = 0.0, dX=None, U=None, workspace=None, stream=None):

@@ -106,15 +106,31 @@ def codebook_normal16(p_max: float = 0.97) -> np.ndarray:
     return out
 
 
+def codebook_fp4_e2m1() -> np.ndarray:
+    """The 16 FP4 (E2M1) values in code order, divided by the largest (6),
+    as fp32: code = sign (bit 3), exponent (bits 2..1), mantissa (bit 0);
+    exponent 0 is subnormal (0 or 0.5), otherwise (1 + m/2) * 2^(e - 1).
+    Codes 0 and 8 are +0 and -0.  Computed exactly, rounded to fp32 once."""
+    from fractions import Fraction
+    vals = []
+    for c in range(16):
+        s, e, m = c >> 3, (c >> 1) & 3, c & 1
+        mag = Fraction(m, 2) if e == 0 else (1 + Fraction(m, 2)) * Fraction(2) ** (e - 1)
+        v = mag / 6
+        vals.append(-float(v) if s else float(v))
+    out = np.array(vals, dtype=np.float32)
+    out[8] = np.float32(-0.0)
+    return out
+
+
 def channel_mix_perm(n: int, frac_int4: float, seed: int):
     """Seeded channel-mix split of the n output channels.
 
     Returns (perm int32 [n], n4): perm lists the INT4 channels first and then
     the INT2 channels, each group in ascending original order; n4 is the count
-    of INT4 channels (round(frac_int4 * n), rounded down to a multiple of 128
-    so that each half is a whole number of 128-row tiles).
+    of INT4 channels, round(frac_int4 * n).
     """
-    n4 = int(round(frac_int4 * n)) // 128 * 128
+    n4 = int(round(frac_int4 * n))
     order = torch.randperm(n, generator=_gen(seed + 104729))
     int4 = torch.sort(order[:n4]).values
     int2 = torch.sort(order[n4:]).values

@@ -58,8 +58,13 @@ def test_linear_fwd_rejects_bad_arguments():
 def test_bwd_and_grads_reject_bad_arguments():
     q = _qw()
     bwd = lbq.lbq_linear_bwd
-    cb = _qw(scheme=lbq.LBQ_CODEBOOK4, group=64, absmax=0x9000, codebook=0xA000)
-    assert bwd(0x4000, 4, ctypes.byref(cb), None, None, 0, 0.0, 0x5000, None, None, 0, None) == lbq.LBQ_EUNSUPPORTED
+    # codebook weights take the backward too; their arguments are checked the same way
+    cb = _qw(scheme=lbq.LBQ_CODEBOOK4, group=64, absmax=0x9000, codebook=0xA000, n=250)
+    assert bwd(0x4000, 4, ctypes.byref(cb), None, None, 0, 0.0, 0x5000, None, None, 0, None) == lbq.LBQ_EINVAL
+    cb = _qw(scheme=lbq.LBQ_CODEBOOK4, group=64, absmax=0x9008, codebook=0xA000)
+    assert bwd(0x4000, 4, ctypes.byref(cb), None, None, 0, 0.0, 0x5000, None, None, 0, None) == lbq.LBQ_EALIGN
+    cb = _qw(scheme=lbq.LBQ_CODEBOOK4, group=64, absmax=0x9000, codebook=None)
+    assert bwd(0x4000, 4, ctypes.byref(cb), None, None, 0, 0.0, 0x5000, None, None, 0, None) == lbq.LBQ_EINVAL
     q2 = _qw(n=250)
     assert bwd(0x4000, 4, ctypes.byref(q2), None, None, 0, 0.0, 0x5000, None, None, 0, None) == lbq.LBQ_EINVAL
     g = lbq.lbq_lora_grads

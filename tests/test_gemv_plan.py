@@ -1,145 +1,199 @@
-"""Host logic of the decode GEMV's stream-K plan (no GPU needed).
+"""Host logic of the grouped decode GEMV's plan (no GPU needed).
 
-lbq_gemv_plan returns the plan that lbq_linear_fwd launches for m <= 16.
-These tests rebuild every CTA's work from it with the decomposition that the
-kernel uses (equal contiguous shares of the row-tile x k-block units; a share
-is split at a tile boundary into at most two segments) and check what the
-kernel relies on:
+lbq_gemv_plan returns the plan that the forward launches for m <= 16 over a
+group of up to 8 weights.  These tests rebuild every CTA's work from it with
+the decomposition the kernel uses (equal contiguous shares of one weight's
+row-tile x k-block units, cut at tile boundaries into segments, processed
+last tile first, then the whole tiles, then the first tile) and check what
+the kernel relies on:
 
-* every unit is covered exactly once;
+* the launch is one wave of two CTAs per SM, and its shared memory (ring of
+  stages plus the fixed tail) fits two CTAs per SM;
+* every unit of every weight is covered exactly once, and CTAs of one weight
+  are contiguous in the grid;
 * a split tile is finished by the CTA that covers its last k-block, which is
-  the highest CTA index of the tile, and its contributors are the CTAs just
-  below it;
-* a CTA processes its tile-starting segment (where it is a contributor) first,
-  so no CTA waits before it has published, and no chain of waits forms;
-* partial-sum slots (CTA + tile) are distinct, and the workspace holds them;
-* shared memory fits two CTAs per SM, the constant table fits, and the
-  benchmark's layer shapes run in one wave.
+  the highest CTA index of the tile; that CTA processes it last, and every
+  contributor processes its contribution first (so no CTA waits before it has
+  published, and no chain of waits forms);
+* partial-sum slots (CTA + tile) are distinct and inside the weight's
+  partial region; the workspace holds the counter header and all regions and
+  is zero exactly when no tile is split;
+* boxes start on whole scale groups, the activation rows and constant rows
+  of a stage hold what a box needs, and every CTA gets about the same bytes.
 """
 import ctypes
-import itertools
 
 import pytest
 
 from qlora_quantized_linear_b200 import lbq
 
 SMS = 148
+BUDGET = 115712 - 1024           # dynamic shared memory per CTA at two CTAs per SM (beside 1 KB static)
+EXTRA = 3 * 4 * 8 + 16 + 2 * 256 * 4
+HEADER = 64 * 1024
+SHAPES_8B = [(4096, 4096), (1024, 4096), (1024, 4096), (4096, 4096), (14336, 4096), (14336, 4096), (4096, 14336)]
 
 
-def qweight(n, k, scheme="minmax", bits=4):
+def qweight(n, k, scheme="minmax", bits=4, dq=False):
     if scheme == "minmax":
         return lbq.lbq_qweight(n=n, k=k, bits=bits, group=128 if bits == 4 else 64, scheme=lbq.LBQ_MINMAX_ASYM)
-    return lbq.lbq_qweight(n=n, k=k, bits=4, group=64, scheme=lbq.LBQ_CODEBOOK4)
+    return lbq.lbq_qweight(n=n, k=k, bits=4, group=64, scheme=lbq.LBQ_CODEBOOK4, double_quant=int(dq))
 
 
-def plan(m, n, k, scheme="minmax", bits=4, sms=SMS):
-    q = qweight(n, k, scheme, bits)
-    out = (ctypes.c_int64 * 6)()
-    assert lbq.lbq_gemv_plan(m, ctypes.byref(q), sms, out) == lbq.LBQ_OK
-    return dict(grid=out[0], share=out[1], tiles=out[2], stages=out[3], smem=out[4], sms=out[5],
-                kbt=k // 64, gb=2 if (scheme == "minmax" and bits == 4) else 1, q=q)
+def plan(m, qs, sms=SMS):
+    arr = (ctypes.POINTER(lbq.lbq_qweight) * len(qs))(*[ctypes.pointer(q) for q in qs])
+    out = (ctypes.c_int64 * 8)()
+    per = (ctypes.c_int64 * (4 * len(qs)))()
+    rc = lbq.lbq_gemv_plan(m, arr, len(qs), sms, out, per)
+    assert rc == lbq.LBQ_OK, rc
+    P = dict(ctas=out[0], ws=out[1], stage=out[2], smem=out[3], workspace=out[4], sms=out[5], xbox=out[6],
+             cstride=out[7], probs=[])
+    for i, q in enumerate(qs):
+        kind = 2 if q.scheme == lbq.LBQ_CODEBOOK4 else (0 if q.bits == 4 else 1)
+        P["probs"].append(dict(share=per[4 * i], ctas=per[4 * i + 1], cta0=per[4 * i + 2], tiles=per[4 * i + 3],
+                               kbt=q.k // 64, n=q.n, k=q.k, kind=kind, dq=bool(q.double_quant),
+                               gb=2 if kind == 0 else 1, sub=8 if kind == 1 else 4, bits=q.bits))
+    return P
 
 
-def segments(b, P):
-    """(tile, first k-block, k-blocks) of CTA b, in the order the kernel
-    processes them (the segment that starts a tile first)."""
-    kbt, share = P["kbt"], P["share"]
-    total = P["tiles"] * kbt
+def segments(b, pr):
+    """(tile, ka, kb) of CTA b of one weight, in processing order."""
+    kbt, share = pr["kbt"], pr["share"]
+    total = pr["tiles"] * kbt
     u0 = b * share
     u1 = min(u0 + share, total)
     if u0 >= u1:
         return []
-    t0 = u0 // kbt
-    a0 = u0 - t0 * kbt
-    n0 = min(u1 - u0, kbt - a0)
-    n1 = (u1 - u0) - n0
-    segs = [(t0, a0, n0)]
-    if n1:
-        segs.append((t0 + 1, 0, n1))
-    return list(reversed(segs))
+    tA, tB = u0 // kbt, (u1 - 1) // kbt
+    nseg = tB - tA + 1
+    out = []
+    for si in range(nseg):
+        t = tA if nseg == 1 else (tB if si == 0 else (tA if si == nseg - 1 else tA + si))
+        ka = u0 - tA * kbt if t == tA else 0
+        kb = u1 - tB * kbt if t == tB else kbt
+        out.append((t, ka, kb))
+    return out
 
 
-def check_plan(m, n, k, scheme="minmax", bits=4):
-    P = plan(m, n, k, scheme, bits)
-    kbt, share, tiles, gb = P["kbt"], P["share"], P["tiles"], P["gb"]
-    assert P["sms"] == SMS and tiles == -(-n // 128)
-    assert share % gb == 0 and gb <= share <= kbt
-    assert share // gb <= 32                                   # constant-table groups per CTA
-    assert P["grid"] == -(-(tiles * kbt) // share)
-    assert P["stages"] in (3, 4)
-    assert P["smem"] <= 113 * 1024                            # two CTAs per SM
-    owner_of, ctas_of, covered, slots = {}, {}, set(), set()
-    for b in range(P["grid"]):
-        segs = segments(b, P)
-        assert 1 <= len(segs) <= 2
-        seen_owner = False
-        for (t, a, cnt) in segs:
-            assert 0 <= t < tiles and 0 <= a and cnt > 0 and a + cnt <= kbt
-            assert a % gb == 0 and cnt % gb == 0                # whole scale groups
-            for u in range(a, a + cnt):
-                assert (t, u) not in covered
-                covered.add((t, u))
-            ctas_of.setdefault(t, []).append(b)
-            full = a == 0 and cnt == kbt
-            if full:
-                continue
-            slots.add(b + t)
-            if a + cnt == kbt:
-                assert t not in owner_of
-                owner_of[t] = b
-                seen_owner = True
-            else:
-                assert not seen_owner, f"CTA {b} would publish after waiting"
-    assert len(covered) == tiles * kbt
-    for t, bs in ctas_of.items():
-        assert bs == list(range(bs[0], bs[-1] + 1))            # contiguous CTA range
-        if len(bs) > 1:
-            assert owner_of[t] == bs[-1]                         # the highest index finishes
-    assert len(slots) == len({(b, t) for t, bs in ctas_of.items() if len(bs) > 1 for b in bs})
-    assert all(s < P["grid"] + tiles for s in slots)
-    ws = lbq.lbq_linear_fwd_workspace_size(m, ctypes.byref(P["q"]), 0)
-    if P["grid"] > 1:
-        assert ws >= 64 * 1024 + (P["grid"] + tiles) * m * 128 * 4
-    return P
+def unit_bytes(pr):
+    codes = 128 * 64 * pr["bits"] / 8
+    if pr["kind"] != 2:
+        return codes + 128 * 4 * 64 / (128 if pr["bits"] == 4 else 64)
+    return codes + 128 * (1 if pr["dq"] else 4)
 
 
-SHAPES_8B = [(4096, 4096), (1024, 4096), (14336, 4096), (4096, 14336)]
-SHAPES_70B = [(8192, 8192), (28672, 8192), (8192, 28672)]
+def check(m, qs):
+    P = plan(m, qs)
+    assert P["sms"] == SMS
+    assert P["ctas"] <= 2 * SMS, "more than one wave"
+    assert 2 <= P["ws"] <= 4
+    assert P["stage"] % 1024 == 0
+    # stage: weight box, activation box (k-blocks of the box x tokens padded to
+    # the MMA's 8 or 16 x 128 bytes); then two constant slots per compute warp
+    sub_max = max(pr["sub"] for pr in P["probs"])
+    mpad = 8 if m <= 8 else 16
+    assert P["xbox"] == sub_max * mpad * 128 and P["stage"] == 16384 + P["xbox"]
+    cbuf = 8 * 2 * 32 * P["cstride"]
+    assert P["smem"] == 1024 + P["ws"] * P["stage"] + cbuf + EXTRA and P["smem"] <= BUDGET
+    cta = 0
+    any_split = False
+    part_total = 0
+    per_cta_bytes = []
+    for pr in P["probs"]:
+        assert pr["cta0"] == cta
+        kbt, share, tiles, gb = pr["kbt"], pr["share"], pr["tiles"], pr["gb"]
+        assert tiles == -(-pr["n"] // 128)
+        assert share % gb == 0 and share >= gb
+        assert pr["ctas"] == -(-(tiles * kbt) // share)
+        cta += pr["ctas"]
+        covered = set()
+        slots = set()
+        first_of, last_of = {}, {}
+        for b in range(pr["ctas"]):
+            segs = segments(b, pr)
+            assert segs
+            per_cta_bytes.append(sum(kb - ka for (_, ka, kb) in segs) * unit_bytes(pr))
+            for i, (t, ka, kb) in enumerate(segs):
+                assert 0 <= t < tiles and 0 <= ka < kb <= kbt
+                assert ka % gb == 0 and kb % gb == 0              # whole scale groups
+                for kbs in range(ka, kb, pr["sub"]):
+                    nk = min(pr["sub"], kb - kbs)
+                    assert kbs % gb == 0 and nk >= 1
+                    # constant words a box needs, for the worst row parity
+                    if pr["kind"] != 2:
+                        ng = -(-nk // gb)
+                        assert 4 * (ng // 2 + 1) <= P["cstride"]
+                    else:
+                        assert 4 * nk <= P["cstride"] or (pr["dq"] and 8 <= P["cstride"])
+                for u in range(ka, kb):
+                    assert (t, u) not in covered
+                    covered.add((t, u))
+                first_of.setdefault(t, b)
+                last_of[t] = b
+                full = ka == 0 and kb == kbt
+                if full:
+                    continue
+                any_split = True
+                if kb < kbt:
+                    # contributor: its first-processed segment, and it is not the tile's last CTA
+                    assert i == 0
+                    slot = b + t
+                    assert slot not in slots and slot < pr["ctas"] + tiles
+                    slots.add(slot)
+                else:
+                    # finisher: processed last
+                    assert i == len(segs) - 1
+        assert len(covered) == tiles * kbt
+        for t in range(tiles):
+            lo = (t * kbt) // share
+            hi = ((t + 1) * kbt - 1) // share
+            assert first_of[t] == lo and last_of[t] == hi
+        part_total += -(-((pr["ctas"] + tiles) * m * 128 * 4) // 256) * 256
+    assert P["ctas"] == cta
+    if any_split:
+        assert P["workspace"] == HEADER + part_total
+    else:
+        assert P["workspace"] == 0
+    mean = sum(per_cta_bytes) / len(per_cta_bytes)
+    return P, max(per_cta_bytes) / mean
 
 
-@pytest.mark.parametrize("m", [1, 8, 9, 16])
-@pytest.mark.parametrize("n,k", SHAPES_8B + SHAPES_70B)
-@pytest.mark.parametrize("scheme,bits", [("minmax", 4), ("minmax", 2), ("codebook", 4)])
-def test_plan_layer_shapes(m, n, k, scheme, bits):
-    check_plan(m, n, k, scheme, bits)
-
-
-@pytest.mark.parametrize("m,n,k", list(itertools.product([1, 7, 16], [128, 200, 384, 1000, 2000], [128, 640, 3200])))
-def test_plan_ragged_shapes(m, n, k):
-    check_plan(m, n, k, "minmax", 4)
-    check_plan(m, n, k, "codebook", 4)
+@pytest.mark.parametrize("m", [1, 4, 8, 9, 16])
+def test_8b_layer_set_one_launch(m):
+    P, imbalance = check(m, [qweight(n, k) for (n, k) in SHAPES_8B])
+    # the whole set in one wave with about equal bytes per CTA
+    assert P["ctas"] >= 0.9 * 2 * SMS
+    assert imbalance < 1.15
 
 
 @pytest.mark.parametrize("m", [1, 16])
-def test_8b_layer_set_runs_in_one_wave(m):
-    for n, k in SHAPES_8B:
-        P = check_plan(m, n, k)
-        assert P["grid"] <= 2 * SMS, (n, k, P)
+def test_8b_layer_mix(m):
+    bits = [2, 2, 2, 2, 4, 2, 2]
+    check(m, [qweight(n, k, bits=b) for (n, k), b in zip(SHAPES_8B, bits)])
 
 
-def test_wide_token_tile_takes_three_boxes_for_one_wave():
-    # at m = 16 the activation slice crowds the shared memory: the MLP shapes
-    # drop to a three-box ring so that the grid still fits one wave
-    for n, k in [(14336, 4096), (4096, 14336)]:
-        assert plan(16, n, k)["stages"] == 3
-    assert plan(1, 14336, 4096)["stages"] == 4
+@pytest.mark.parametrize("m", [1, 16])
+def test_channel_mix_halves(m):
+    check(m, [qweight(3584, 4096, bits=4), qweight(10752, 4096, bits=2)])
+    check(m, [qweight(250, 1024, bits=4), qweight(750, 1024, bits=2)])
+
+
+@pytest.mark.parametrize("m,n,k,scheme,bits,dq", [
+    (1, 256, 512, "minmax", 4, False), (16, 200, 640, "minmax", 4, False), (1, 14336, 4096, "minmax", 4, False),
+    (8, 4096, 4096, "minmax", 2, False), (12, 2000, 3200, "codebook", 4, True), (16, 4096, 14336, "minmax", 4, False),
+    (1, 8192, 8192, "codebook", 4, True), (16, 28672, 8192, "codebook", 4, True), (16, 8192, 28672, "codebook", 4, False),
+    (3, 1, 128, "minmax", 4, False), (1, 1000, 64 * 3, "minmax", 2, False), (5, 130, 384, "minmax", 4, False),
+])
+def test_single_weight(m, n, k, scheme, bits, dq):
+    check(m, [qweight(n, k, scheme, bits, dq)])
 
 
 def test_plan_rejects_bad_arguments():
     q = qweight(256, 512)
-    out = (ctypes.c_int64 * 6)()
-    assert lbq.lbq_gemv_plan(0, ctypes.byref(q), SMS, out) == lbq.LBQ_EINVAL
-    assert lbq.lbq_gemv_plan(17, ctypes.byref(q), SMS, out) == lbq.LBQ_EINVAL
-    assert lbq.lbq_gemv_plan(1, ctypes.byref(q), SMS, None) == lbq.LBQ_EINVAL
-    bad = qweight(256, 500)
-    assert lbq.lbq_gemv_plan(1, ctypes.byref(bad), SMS, out) == lbq.LBQ_EINVAL
+    arr = (ctypes.POINTER(lbq.lbq_qweight) * 9)(*[ctypes.pointer(q)] * 9)
+    out = (ctypes.c_int64 * 8)()
+    assert lbq.lbq_gemv_plan(0, arr, 1, SMS, out, None) == lbq.LBQ_EINVAL
+    assert lbq.lbq_gemv_plan(17, arr, 1, SMS, out, None) == lbq.LBQ_EINVAL
+    assert lbq.lbq_gemv_plan(1, arr, 0, SMS, out, None) == lbq.LBQ_EINVAL
+    assert lbq.lbq_gemv_plan(1, arr, 9, SMS, out, None) == lbq.LBQ_EINVAL
+    assert lbq.lbq_gemv_plan(1, arr, 1, SMS, None, None) == lbq.LBQ_EINVAL

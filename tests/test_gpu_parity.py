@@ -541,3 +541,475 @@ def test_merge_full_size_gate(lbq, train_problem):
     ref = oracle.lora_merge(What, syn.bits_u16(P["A"]), syn.bits_u16(P["B"]), P["s"], 1)
     assert np.array_equal(u16(out), ref)
     assert_status_clean(lbq)
+
+
+# --------------------------------------------------------------------------- rounding ties on the GPU
+@pytest.mark.parametrize("bits", [4, 2])
+def test_minmax_quantize_ties_bit_exact(lbq, bits):
+    """Groups where many w / scale land exactly on k + 1/2 (and zero points
+    exactly half-way): the GPU quantizer's codes, scales and zeros equal the
+    oracle's and the exact-rational expectation (half to even) bit for bit."""
+    from tie_inputs import tie_weight
+    group = 128 if bits == 4 else 64
+    n, k = 256, 8 * group
+    w, codes_exp, zeros_exp, scales_exp = tie_weight(n, k, bits, seed=10 + bits)
+    W = torch.from_numpy(w).to(torch.bfloat16)
+    qw = lbq.QuantizedWeight(n, k, "minmax", bits).quantize(W.cuda())
+    torch.cuda.synchronize()
+    codes, scale, zero = oracle.minmax_quantize(syn.bits_u16(W), bits, group)
+    assert np.array_equal(codes.astype(np.int64), codes_exp)
+    assert np.array_equal(qw.packed.cpu().numpy(), oracle.pack(codes, bits)), "packed codes differ"
+    assert np.array_equal(u16(qw.scale), scale), "scales differ"
+    assert np.array_equal(u16(qw.zero), zero), "zeros differ"
+    assert np.array_equal(qw.scale.cpu().numpy().astype(np.float64), scales_exp)
+    assert np.array_equal(qw.zero.cpu().numpy().astype(np.float64), zeros_exp)
+    assert_status_clean(lbq)
+
+
+# --------------------------------------------------------------------------- channel-mix
+def _channel_mix(lbq, W, frac, seed):
+    """ChannelMixWeight of W (bf16 CPU [n, k]) with the oracle's quantization
+    of both halves; returns (mix, perm, n4, (packed, scale, zero) of hi and lo)."""
+    n, k = W.shape
+    perm, n4 = syn.channel_mix_perm(n, frac, seed=seed)
+    Wp = W[torch.from_numpy(perm.astype(np.int64))]
+    halves = []
+    for rows, bits in ((slice(0, n4), 4), (slice(n4, n), 2)):
+        Wh = Wp[rows].contiguous()
+        codes, scale, zero = oracle.minmax_quantize(syn.bits_u16(Wh), bits, 128 if bits == 4 else 64)
+        halves.append((oracle.pack(codes, bits), scale, zero))
+    qws = []
+    for (packed, scale, zero), nn, bits in ((halves[0], n4, 4), (halves[1], n - n4, 2)):
+        qw = lbq.QuantizedWeight(nn, k, "minmax", bits)
+        qw.packed.copy_(torch.from_numpy(packed))
+        qw.scale.copy_(torch.from_numpy(scale.view(np.float16)))
+        qw.zero.copy_(torch.from_numpy(zero.view(np.float16)))
+        qws.append(qw)
+    torch.cuda.synchronize()
+    return lbq.ChannelMixWeight(qws[0], qws[1], perm), perm, n4, halves
+
+
+def _channel_mix_sampled_ref(X, perm, n4, halves, k, tok, col, A, B, s):
+    """Oracle Y and bound at (tok[i], col[i]) (original output columns) of a
+    channel-mix weight: each sample goes to the half that stores its column,
+    with the adapter rows of B taken in stored order."""
+    n = perm.size
+    inv = np.empty(n, np.int64)
+    inv[perm] = np.arange(n)
+    ref = np.empty(tok.size)
+    bound = np.empty(tok.size)
+    Bb = None if B is None else syn.bits_u16(B)
+    for lo_, hi_, (packed, scale, zero), bits in ((0, n4, halves[0], 4), (n4, n, halves[1], 2)):
+        sel = (inv[col] >= lo_) & (inv[col] < hi_)
+        if not sel.any():
+            continue
+        stored = inv[col[sel]] - lo_
+        Bh = None if Bb is None else np.ascontiguousarray(Bb[perm[lo_:hi_]])
+        r, b = oracle.linear_fwd_sampled_minmax(syn.bits_u16(X), packed, scale, zero, hi_ - lo_, k, bits,
+                                                128 if bits == 4 else 64, tok[sel], stored,
+                                                None if A is None else syn.bits_u16(A), Bh, s)
+        ref[sel], bound[sel] = r, b
+    return ref, bound
+
+
+def test_channel_mix_fwd_full_gate_m512(lbq):
+    """Channel-mix 25 % INT4 g128 / 75 % INT2 g64 on the 8B gate matrix
+    (14336 x 4096) at M = 512 with a rank-16 adapter: the tensor-core path
+    with the stored permutation applied in its epilogue; 4096 seeded
+    elements plus one full row and one full column against the oracle."""
+    m, n, k, r, s = 512, 14336, 4096, 16, 2.0
+    W = syn.weight_bf16(n, k, 0.02, seed=301, outlier_frac=0.001)
+    X = syn.normal_bf16((m, k), 1.0, seed=302)
+    A = syn.normal_bf16((r, k), 0.01, seed=303)
+    B = syn.normal_bf16((n, r), 0.01, seed=304)
+    mix, perm, n4, halves = _channel_mix(lbq, W, 0.25, seed=5)
+    Y, _ = lbq.linear_fwd(X.cuda(), mix, A.cuda(), B.cuda(), s)
+    torch.cuda.synchronize()
+    tok, col = _sample_pairs(m, n, 4096, seed=8)
+    ref, bound = _channel_mix_sampled_ref(X, perm, n4, halves, k, tok, col, A, B, s)
+    assert_within(Y.cpu().numpy()[tok, col], ref, bound, "Y (channel-mix, M=512)")
+    assert_status_clean(lbq)
+
+
+@pytest.mark.parametrize("m", [16, 512])
+def test_channel_mix_ragged_halves(lbq, m):
+    """Halves that are not whole 128-row tiles (250 INT4 rows, 750 INT2 rows),
+    every output element against the oracle."""
+    n, k, r, s = 1000, 1024, 8, 2.0
+    W = mixed_weight(n, k, seed=n + m)
+    X = syn.normal_bf16((m, k), 1.0, seed=m + 5)
+    A = syn.normal_bf16((r, k), 0.01, seed=6)
+    B = syn.normal_bf16((n, r), 0.01, seed=7)
+    mix, perm, n4, halves = _channel_mix(lbq, W, 0.25, seed=3)
+    assert n4 % 128 != 0 and (n - n4) % 128 != 0
+    Y, _ = lbq.linear_fwd(X.cuda(), mix, A.cuda(), B.cuda(), s)
+    torch.cuda.synchronize()
+    What = np.zeros((n, k), np.float32)
+    for (packed, scale, zero), rows, bits in ((halves[0], perm[:n4], 4), (halves[1], perm[n4:], 2)):
+        What[rows] = oracle.minmax_dequantize(packed, scale, zero, k, bits, 128 if bits == 4 else 64)
+    Yr, _, Yb = oracle.linear_fwd(syn.bits_u16(X), What, syn.bits_u16(A), syn.bits_u16(B), s)
+    assert_within(Y.cpu().numpy(), Yr, Yb, f"Y (channel-mix, ragged halves, M={m})")
+    assert_status_clean(lbq)
+
+
+# --------------------------------------------------------------------------- INT2 on the tensor cores at full size
+@pytest.mark.parametrize("name", ["gate", "down"])
+def test_int2_fwd_full_size_m512(lbq, name):
+    """Layer-mix INT2 g64 on the full 8B gate (14336 x 4096) and down
+    (4096 x 14336) matrices at M = 512 through the tensor-core GEMM: 4096
+    seeded elements plus a full row and a full column."""
+    m = 512
+    n, k = syn.LLAMA3_8B_SHAPES[name]
+    W = syn.weight_bf16(n, k, 0.02, seed=311 + n, outlier_frac=0.001)
+    X = syn.normal_bf16((m, k), 1.0, seed=312)
+    codes, scale, zero = oracle.minmax_quantize(syn.bits_u16(W), 2, 64)
+    packed = oracle.pack(codes, 2)
+    qw = lbq.QuantizedWeight(n, k, "minmax", 2)
+    qw.packed.copy_(torch.from_numpy(packed))
+    qw.scale.copy_(torch.from_numpy(scale.view(np.float16)))
+    qw.zero.copy_(torch.from_numpy(zero.view(np.float16)))
+    Y, _ = lbq.linear_fwd(X.cuda(), qw)
+    torch.cuda.synchronize()
+    tok, col = _sample_pairs(m, n, 4096, seed=9)
+    ref, bound = oracle.linear_fwd_sampled_minmax(syn.bits_u16(X), packed, scale, zero, n, k, 2, 64, tok, col)
+    assert_within(Y.cpu().numpy()[tok, col], ref, bound, f"Y (INT2 {name}, M=512)")
+    assert_status_clean(lbq)
+
+
+# --------------------------------------------------------------------------- 70B codebook MLP matrices at full size
+@pytest.mark.parametrize("name", ["gate", "down"])
+def test_codebook70b_mlp_full_size(lbq, name):
+    """The 70B gate (28672 x 8192) and down (8192 x 28672) matrices in the
+    4-bit codebook format with double quantization, quantized on the GPU:
+    codes, q8, s2 and offset bit-exact against the oracle; M = 1 every output;
+    M = 2048 on 2048 seeded elements plus a full row and a full column."""
+    n, k = syn.LLAMA3_70B_SHAPES[name]
+    cb = syn.codebook_normal16()
+    W = syn.weight_bf16(n, k, 0.015, seed=321 + n)
+    qw = lbq.QuantizedWeight(n, k, "codebook", double_quant=True, codebook=cb).quantize(W.cuda())
+    torch.cuda.synchronize()
+    codes, absmax = oracle.codebook_quantize(syn.bits_u16(W), cb)
+    del W
+    packed = oracle.pack(codes, 4)
+    del codes
+    q8, s2, off, exact = oracle.double_quant(absmax)
+    assert exact
+    assert np.array_equal(qw.packed.cpu().numpy(), packed)
+    assert np.array_equal(qw.q8.cpu().numpy(), q8)
+    assert np.array_equal(qw.s2.cpu().numpy().view(np.uint32), s2.view(np.uint32))
+    assert np.float32(qw.offset[0].item()).view(np.uint32) == np.float32(off).view(np.uint32)
+    What = oracle.codebook_dequantize(packed, oracle.double_dequant(q8, s2, off), cb, n, k)
+    del packed
+    for m, seed in ((1, 322), (2048, 323)):
+        X = syn.normal_bf16((m, k), 1.0, seed=seed)
+        Y, _ = lbq.linear_fwd(X.cuda(), qw)
+        torch.cuda.synchronize()
+        Yc = Y.cpu().numpy()
+        x = oracle.bf16_to_f32(syn.bits_u16(X))
+        if m == 1:
+            xr = x[0].astype(np.float64)
+            ref = np.empty(n)
+            bound = np.empty(n)
+            for i in range(0, n, 2048):
+                wc = What[i:i + 2048].astype(np.float64)
+                ref[i:i + 2048] = wc @ xr
+                bound[i:i + 2048] = np.abs(wc) @ np.abs(xr)
+            assert_within(Yc[0], ref, bound, f"Y (70B {name}, M=1)")
+        else:
+            rows, cols = _sample_pairs(m, n, 2048, seed=seed)
+            ref = np.empty(rows.size)
+            bound = np.empty(rows.size)
+            for i in range(0, rows.size, 512):
+                xr = x[rows[i:i + 512]].astype(np.float64)
+                wc = What[cols[i:i + 512]].astype(np.float64)
+                ref[i:i + 512] = np.einsum("ij,ij->i", xr, wc)
+                bound[i:i + 512] = np.einsum("ij,ij->i", np.abs(xr), np.abs(wc))
+            assert_within(Yc[rows, cols], ref, bound, f"Y (70B {name}, M=2048)")
+        del X, Y
+    assert_status_clean(lbq)
+
+
+# --------------------------------------------------------------------------- bounded waits
+def test_bounded_wait_times_out_and_context_survives(lbq):
+    """A kernel whose waits can never be satisfied gives up after the short
+    limit, records the timeout in the status word and returns; the device
+    stays usable: a forward with a freshly zeroed workspace afterwards matches
+    the oracle and leaves the status clean."""
+    import ctypes
+    stream = torch.cuda.current_stream().cuda_stream
+    assert lbq.lbq_selftest_wait_timeout(0, stream) == lbq.LBQ_EINVAL
+    assert lbq.lbq_selftest_wait_timeout(2000, stream) == lbq.LBQ_OK
+    assert lbq.device_status() & lbq.STATUS_TIMEOUT
+    assert lbq.device_status() == 0                    # read-and-clear
+    m, n, k = 4, 1024, 4096
+    X, W, _, _ = fwd_problem(m, n, k, 0, seed=12)
+    qw = device_qweight(lbq, W, "minmax", 4, False, None)
+    ws = lbq._workspace(lbq.lbq_linear_fwd_workspace_size(m, ctypes.byref(qw.struct), 0), "cuda")
+    Y, _ = lbq.linear_fwd(X.cuda(), qw, workspace=ws)
+    torch.cuda.synchronize()
+    Yr, _, Yb = oracle.linear_fwd(syn.bits_u16(X), oracle_weight(W, "minmax", 4, False, None))
+    assert_within(Y.cpu().numpy(), Yr, Yb, "Y after a timed-out wait")
+    assert_status_clean(lbq)
+
+
+# --------------------------------------------------------------------------- grouped forward (one launch per layer set)
+@pytest.fixture(scope="module")
+def layer_set_8b(lbq):
+    """The seven LLaMA-3-8B layers (q, k, v, o, gate, up, down), INT4 g128
+    with the oracle's quantization, as the decode benchmark runs them."""
+    out = {}
+    for i, (name, (n, k)) in enumerate(syn.LLAMA3_8B_SHAPES.items()):
+        W = syn.weight_bf16(n, k, 0.02, seed=400 + i, outlier_frac=0.001)
+        codes, scale, zero = oracle.minmax_quantize(syn.bits_u16(W), 4, 128)
+        packed = oracle.pack(codes, 4)
+        qw = lbq.QuantizedWeight(n, k, "minmax", 4)
+        qw.packed.copy_(torch.from_numpy(packed))
+        qw.scale.copy_(torch.from_numpy(scale.view(np.float16)))
+        qw.zero.copy_(torch.from_numpy(zero.view(np.float16)))
+        out[name] = (qw, packed, scale, zero)
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("m", [1, 16])
+def test_grouped_fwd_8b_layer_set_full(lbq, layer_set_8b, m):
+    """One grouped call over the whole 8B layer set (one launch of the decode
+    GEMV): every output element of every layer against the oracle."""
+    Xs = {k: syn.normal_bf16((m, k), 1.0, seed=410 + k + m) for k in (4096, 14336)}
+    Xd = {k: x.cuda() for k, x in Xs.items()}
+    names = list(syn.LLAMA3_8B_SHAPES)
+    outs = lbq.linear_fwd_grouped([(Xd[layer_set_8b[nm][0].k], layer_set_8b[nm][0]) for nm in names])
+    torch.cuda.synchronize()
+    for nm, (Y, _) in zip(names, outs):
+        qw, packed, scale, zero = layer_set_8b[nm]
+        tok = np.repeat(np.arange(m), qw.n)
+        col = np.tile(np.arange(qw.n), m)
+        ref, bound = oracle.linear_fwd_sampled_minmax(syn.bits_u16(Xs[qw.k]), packed, scale, zero, qw.n, qw.k, 4, 128,
+                                                      tok, col)
+        assert_within(Y.cpu().numpy().reshape(-1), ref, bound, f"Y ({nm}, M={m}, grouped)")
+    assert_status_clean(lbq)
+
+
+GROUP_CASES = [
+    # n, k, scheme, bits, dq, rank
+    (256, 512, "minmax", 4, False, 8),
+    (300, 1024, "minmax", 2, False, 0),
+    (200, 640, "codebook", 4, True, 16),
+    (128, 192, "codebook", 4, False, 0),
+    (130, 384, "minmax", 4, False, 4),      # ragged rows, far zero points (mixed_weight)
+    (1000, 2048, "minmax", 4, False, 0),
+]
+
+
+@pytest.mark.parametrize("m", [1, 5, 16])
+def test_grouped_fwd_mixed_kinds(lbq, m):
+    """INT4, INT2 and codebook weights (with and without double
+    quantization), ragged shapes and adapters in one grouped launch; each
+    output against the oracle."""
+    cb = syn.codebook_normal16()
+    probs, refs = [], []
+    for i, (n, k, scheme, bits, dq, rank) in enumerate(GROUP_CASES):
+        X, W, A, B = fwd_problem(m, n, k, rank, seed=500 + 17 * i + m, scheme=scheme, bits=bits)
+        qw = device_qweight(lbq, W, scheme, bits, dq, cb)
+        s = 1.5
+        probs.append((X.cuda(), qw, None if A is None else A.cuda(), None if B is None else B.cuda(), s))
+        Yr, Tr, Yb = oracle.linear_fwd(syn.bits_u16(X), oracle_weight(W, scheme, bits, dq, cb),
+                                       None if A is None else syn.bits_u16(A), None if B is None else syn.bits_u16(B), s)
+        refs.append((Yr, Yb))
+    outs = lbq.linear_fwd_grouped(probs)
+    torch.cuda.synchronize()
+    for i, ((Y, _), (Yr, Yb)) in enumerate(zip(outs, refs)):
+        assert_within(Y.cpu().numpy(), Yr, Yb, f"Y (problem {i}, M={m})")
+    assert_status_clean(lbq)
+
+
+@pytest.mark.parametrize("m", [3, 40])
+def test_grouped_fwd_more_than_one_launch(lbq, m):
+    """Ten weights: two launches of the decode GEMV (m <= 16), or ten
+    tensor-core GEMMs one after the other (m > 16), sharing one workspace."""
+    probs, refs = [], []
+    for i in range(10):
+        n, k = 128 * (1 + i % 3), 256 * (1 + i % 2)
+        X, W, _, _ = fwd_problem(m, n, k, 0, seed=600 + i)
+        qw = device_qweight(lbq, W, "minmax", 4 if i % 2 == 0 else 2, False, None)
+        probs.append((X.cuda(), qw))
+        Yr, _, Yb = oracle.linear_fwd(syn.bits_u16(X), oracle_weight(W, "minmax", 4 if i % 2 == 0 else 2, False, None))
+        refs.append((Yr, Yb))
+    outs = lbq.linear_fwd_grouped(probs)
+    torch.cuda.synchronize()
+    for i, ((Y, _), (Yr, Yb)) in enumerate(zip(outs, refs)):
+        assert_within(Y.cpu().numpy(), Yr, Yb, f"Y (problem {i}, M={m})")
+    assert_status_clean(lbq)
+
+
+# --------------------------------------------------------------------------- backward through codebook weights
+CB_BWD_CASES = [
+    # m, n, k, rank, dq
+    (8, 256, 512, 8, False),
+    (1, 128, 1024, 0, True),
+    (70, 200, 640, 16, True),      # ragged features and channels
+    (300, 264, 1024, 4, False),
+    (130, 512, 192, 0, True),      # k = 3 codebook blocks
+]
+
+
+@pytest.mark.parametrize("m,n,k,rank,dq", CB_BWD_CASES)
+def test_linear_bwd_codebook_parity(lbq, m, n, k, rank, dq):
+    """Gradients through the frozen 4-bit codebook weight (QLoRA explainer,
+    QLoRA技术原理): dX and U against the oracle on codebook (and double
+    quantized) weights."""
+    s = 2.0
+    cb = syn.codebook_normal16()
+    X, W, A, B = fwd_problem(m, n, k, rank, seed=m + 3 * n + k, scheme="codebook")
+    dY = syn.normal_bf16((m, n), 0.1, seed=m + n + 7)
+    qw = device_qweight(lbq, W, "codebook", 4, dq, cb)
+    dX, U = lbq.linear_bwd(dY.cuda(), qw, None if A is None else A.cuda(), None if B is None else B.cuda(), s)
+    torch.cuda.synchronize()
+    What = oracle_weight(W, "codebook", 4, dq, cb)
+    dXr, Ur, dXb = oracle.linear_bwd(syn.bits_u16(dY), What, None if A is None else syn.bits_u16(A),
+                                     None if B is None else syn.bits_u16(B), s)
+    assert_within(dX.cpu().numpy(), dXr, dXb, "dX (codebook)")
+    if rank:
+        Ub = np.abs(oracle.bf16_to_f32(syn.bits_u16(dY))).astype(np.float64) @ \
+            np.abs(oracle.bf16_to_f32(syn.bits_u16(B))).astype(np.float64)
+        assert_within(U.cpu().numpy(), Ur, Ub, "U (codebook)")
+    assert_status_clean(lbq)
+
+
+def test_codebook70b_backward_full_size_sampled(lbq, codebook70b):
+    """dX = dY W_hat through the 70B attention projection (8192 x 8192,
+    codebook + double quantization) at M = 2048: 2048 seeded elements plus a
+    full row and a full column against the oracle."""
+    C = codebook70b
+    m = 2048
+    dY = syn.normal_bf16((m, C["n"]), 0.1, seed=75)
+    dX, _ = lbq.linear_bwd(dY.cuda(), C["qw"])
+    torch.cuda.synchronize()
+    rows, cols = _sample_pairs(m, C["k"], 2048, seed=11)
+    g = oracle.bf16_to_f32(syn.bits_u16(dY))
+    w = C["What"]
+    ref = np.empty(rows.size)
+    bound = np.empty(rows.size)
+    for i in range(0, rows.size, 512):
+        gr = g[rows[i:i + 512]].astype(np.float64)              # [b, n]
+        wc = w[:, cols[i:i + 512]].T.astype(np.float64)         # [b, n]
+        ref[i:i + 512] = np.einsum("ij,ij->i", gr, wc)
+        bound[i:i + 512] = np.einsum("ij,ij->i", np.abs(gr), np.abs(wc))
+    assert_within(dX.cpu().numpy()[rows, cols], ref, bound, "dX (70B codebook, M=2048)")
+    assert_status_clean(lbq)
+
+
+# --------------------------------------------------------------------------- FP4 (E2M1) table
+def _fp4_weight(n, k, seed):
+    Wt = syn.weight_bf16(n, k, 0.015, seed=seed, outlier_frac=0.005).float()
+    Wt[0, :64] = 0.0                               # a zero block
+    Wt[1, 64:128] = -Wt[1, 64:128].abs()           # negative values only
+    return Wt.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("double_quant", [False, True])
+@pytest.mark.parametrize("shape", [(256, 512), (1000, 1024)])
+def test_fp4_quantize_bit_exact(lbq, double_quant, shape):
+    """The FP4 (E2M1) table in code order (bitsandbytes guide, nf4与fp4), with
+    +0 at code 0 and -0 at code 8: GPU codes, absmax and double-quantized
+    constants equal the oracle's bit for bit, and dequantization too."""
+    n, k = shape
+    cb = syn.codebook_fp4_e2m1()
+    W = _fp4_weight(n, k, seed=n + k)
+    qw = lbq.QuantizedWeight(n, k, "codebook", double_quant=double_quant, codebook=cb).quantize(W.cuda())
+    torch.cuda.synchronize()
+    codes, absmax = oracle.codebook_quantize(syn.bits_u16(W), cb)
+    assert not np.any(codes == 8)
+    packed = oracle.pack(codes, 4)
+    assert np.array_equal(qw.packed.cpu().numpy(), packed)
+    assert np.array_equal(qw.absmax.cpu().numpy().view(np.uint32), absmax.view(np.uint32))
+    a_used = absmax
+    if double_quant:
+        q8, s2, off, exact = oracle.double_quant(absmax)
+        assert exact
+        assert np.array_equal(qw.q8.cpu().numpy(), q8)
+        assert np.array_equal(qw.s2.cpu().numpy().view(np.uint32), s2.view(np.uint32))
+        a_used = oracle.double_dequant(q8, s2, off)
+    What = qw.dequantize().cpu().numpy()
+    assert np.array_equal(What.view(np.uint32), oracle.codebook_dequantize(packed, a_used, cb, n, k).view(np.uint32))
+    assert_status_clean(lbq)
+
+
+@pytest.mark.parametrize("m", [1, 16, 100])
+def test_fp4_forward_backward_merge(lbq, m):
+    """Forward (decode GEMV and tensor-core GEMM), backward and adapter merge
+    on an FP4-coded weight with double quantization, against the oracle."""
+    n, k, r, s = 384, 1024, 8, 2.0
+    cb = syn.codebook_fp4_e2m1()
+    W = _fp4_weight(n, k, seed=77 + m)
+    X = syn.normal_bf16((m, k), 1.0, seed=78)
+    A = syn.normal_bf16((r, k), 0.01, seed=79)
+    B = syn.normal_bf16((n, r), 0.01, seed=80)
+    dY = syn.normal_bf16((m, n), 0.1, seed=81)
+    qw = device_qweight(lbq, W, "codebook", 4, True, cb)
+    What = oracle_weight(W, "codebook", 4, True, cb)
+    Y, _ = lbq.linear_fwd(X.cuda(), qw, A.cuda(), B.cuda(), s)
+    dX, _ = lbq.linear_bwd(dY.cuda(), qw, A.cuda(), B.cuda(), s)
+    merged = lbq.merge_lora(qw, A.cuda(), B.cuda(), s)
+    torch.cuda.synchronize()
+    Yr, _, Yb = oracle.linear_fwd(syn.bits_u16(X), What, syn.bits_u16(A), syn.bits_u16(B), s)
+    dXr, _, dXb = oracle.linear_bwd(syn.bits_u16(dY), What, syn.bits_u16(A), syn.bits_u16(B), s)
+    assert_within(Y.cpu().numpy(), Yr, Yb, "Y (FP4)")
+    assert_within(dX.cpu().numpy(), dXr, dXb, "dX (FP4)")
+    assert np.array_equal(u16(merged), oracle.lora_merge(What, syn.bits_u16(A), syn.bits_u16(B), s, 1))
+    assert_status_clean(lbq)
+
+
+# --------------------------------------------------------------------------- channel-mix selection by sensitivity
+@pytest.mark.parametrize("n,k,t", [(1000, 1024, 64), (14336, 4096, 128)])
+def test_channel_mix_select_matches_oracle(lbq, n, k, t):
+    """Scores within fp64 rounding of the oracle's (the GPU sums in another
+    order), the selection valid against the oracle's threshold (only channels
+    whose scores are within that rounding of it may differ), the permutation
+    the INT4 channels then the others, each ascending."""
+    W = syn.weight_bf16(n, k, 0.02, seed=n + 1, outlier_frac=0.001)
+    X = syn.normal_bf16((t, k), 1.0, seed=k + 2)
+    n4 = int(round(0.25 * n))
+    perm, score = lbq.channel_mix_select(W.cuda(), X.cuda(), n4)
+    torch.cuda.synchronize()
+    ref, bound = oracle.channel_score(syn.bits_u16(W), syn.bits_u16(X))
+    got = score.cpu().numpy()
+    tol = 2.0 ** -40 * bound + 1e-300
+    assert np.all(np.abs(got - ref) <= tol)
+    perm = perm.cpu().numpy()
+    sel = np.zeros(n, bool)
+    sel[perm[:n4]] = True
+    assert np.array_equal(np.sort(perm), np.arange(n))
+    assert np.all(np.diff(perm[:n4]) > 0) and np.all(np.diff(perm[n4:]) > 0)
+    ref_perm = oracle.channel_mix_select(ref, n4)
+    thr = np.sort(ref)[::-1][n4 - 1]
+    differ = sel != np.isin(np.arange(n), ref_perm[:n4])
+    assert np.all(np.abs(ref[differ] - thr) <= 2 * tol[differ] + 2.0 ** -40 * np.abs(thr))
+    assert differ.sum() <= 2
+    assert_status_clean(lbq)
+
+
+@pytest.mark.parametrize("m", [16, 512])
+def test_channel_mix_weight_from_selection(lbq, m):
+    """The channel-mix weight built on the device from the selection (rows
+    gathered by the permutation, then quantized) computes the forward of the
+    oracle's channel-mix weight for that permutation."""
+    n, k, r, s = 768, 1024, 8, 2.0
+    W = syn.weight_bf16(n, k, 0.02, seed=91, outlier_frac=0.005)
+    Xc = syn.normal_bf16((64, k), 1.0, seed=92)
+    X = syn.normal_bf16((m, k), 1.0, seed=93)
+    A = syn.normal_bf16((r, k), 0.01, seed=94)
+    B = syn.normal_bf16((n, r), 0.01, seed=95)
+    mix = lbq.channel_mix_weight(W.cuda(), Xc.cuda(), 0.25)
+    Y, _ = lbq.linear_fwd(X.cuda(), mix, A.cuda(), B.cuda(), s)
+    torch.cuda.synchronize()
+    perm = mix.perm.cpu().numpy()
+    n4 = mix.hi.n
+    What = np.zeros((n, k), np.float32)
+    for rows, bits in ((perm[:n4], 4), (perm[n4:], 2)):
+        Wh = syn.bits_u16(W[torch.from_numpy(rows.astype(np.int64))].contiguous())
+        codes, scale, zero = oracle.minmax_quantize(Wh, bits, 128 if bits == 4 else 64)
+        What[rows] = oracle.minmax_dequantize(oracle.pack(codes, bits), scale, zero, k, bits, 128 if bits == 4 else 64)
+    Yr, _, Yb = oracle.linear_fwd(syn.bits_u16(X), What, syn.bits_u16(A), syn.bits_u16(B), s)
+    assert_within(Y.cpu().numpy(), Yr, Yb, f"Y (selected channel-mix, M={m})")
+    assert_status_clean(lbq)

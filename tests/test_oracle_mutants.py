@@ -18,6 +18,8 @@ SRC = os.path.join(ROOT, "oracle", "oracle.c")
 MUTANTS = {
     "zero_sign": ("float z32 = rintf(-mn / sf);", "float z32 = rintf(mn / sf);"),
     "floor_not_rint": ("float qf = rintf(t) + zf;", "float qf = floorf(t) + zf;"),
+    "codes_ties_away": ("float qf = rintf(t) + zf;", "float qf = roundf(t) + zf;"),
+    "zero_ties_away": ("float z32 = rintf(-mn / sf);", "float z32 = roundf(-mn / sf);"),
     "scale_denominator": ("float s32 = r / Q;", "float s32 = r / (Q + 1.0f);"),
     "group_row_index": ("const uint16_t* w = W + row * k + g * group;", "const uint16_t* w = W + g * group;"),
     "pack_low_first": ("byte |= (q & ((1u << bits) - 1)) << (8 - bits * (t + 1));",
@@ -43,6 +45,9 @@ MUTANTS = {
     "merge_A_transposed": ("oracle_bf16_to_f32(A[(int64_t)u * k + col])", "oracle_bf16_to_f32(A[col * r + u])"),
     "merge_truncates": ("if (lo > 0x8000u || (lo == 0x8000u && (hi & 1u))) hi += 1u;", "(void)lo;"),
     "merge_ties_away": ("if (lo > 0x8000u || (lo == 0x8000u && (hi & 1u))) hi += 1u;", "if (lo >= 0x8000u) hi += 1u;"),
+    "score_sign": ("sc += m2[j] * (e2 * e2 - e4 * e4);", "sc += m2[j] * (e4 * e4 - e2 * e2);"),
+    "score_first_moment": ("acc += x * x;", "acc += x;"),
+    "select_ties_upper": ("(score[d] == score[c] && d < c)", "(score[d] == score[c] && d > c)"),
     "merge_reordered_sum": ("for (int u = 0; u < r; ++u)\n                d = fmaf(", "for (int u = r - 1; u >= 0; --u)\n                d = fmaf("),
 }
 

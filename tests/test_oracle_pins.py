@@ -204,6 +204,29 @@ def test_minmax_grid_values_roundtrip_exactly(bits):
     assert np.array_equal(What.astype(np.float64), w.reshape(n, k))
 
 
+@pytest.mark.parametrize("bits", [4, 2])
+def test_minmax_ties_round_half_to_even(bits):
+    """Elements exactly half-way between two grid points, and zero points
+    exactly half-way between two integers, take the even neighbour (rint),
+    not the one away from zero: expected codes from exact rationals and
+    Python's round() (tests/tie_inputs.py)."""
+    from tie_inputs import tie_weight
+    group = 128 if bits == 4 else 64
+    n, k = 24, 4 * group
+    w, codes, zeros, scales = tie_weight(n, k, bits, seed=bits)
+    W = _bf16(w)
+    assert np.array_equal(oracle.bf16_to_f32(W), w)
+    got, scale, zero = oracle.minmax_quantize(W, bits, group)
+    assert np.array_equal(np.array([oracle.f16_to_f32(int(h)) for h in scale.ravel()]), scales.ravel())
+    assert np.array_equal(np.array([oracle.f16_to_f32(int(h)) for h in zero.ravel()]), zeros.ravel())
+    assert np.array_equal(got.astype(np.int64), codes)
+    # the case has teeth: half-away-from-zero rounding gives other codes
+    Q = (1 << bits) - 1
+    t = w.reshape(n, k // group, group) / scales[:, :, None]
+    away = np.clip(np.sign(t) * np.floor(np.abs(t) + 0.5) + zeros[:, :, None], 0, Q).reshape(n, k)
+    assert int((away != codes).sum()) > k // 4
+
+
 def test_minmax_constant_and_zero_groups():
     n, k = 2, 128
     w = np.zeros((n, k), np.float32)
@@ -286,12 +309,84 @@ def test_codebook_error_bound_and_zero_block():
 def test_codebook_rejects_bad_tables():
     W = syn.bits_u16(syn.normal_bf16((1, 64), 1.0, 0))
     cb = syn.codebook_normal16()
-    with pytest.raises(ValueError):
-        oracle.codebook_quantize(W, cb[::-1].copy())          # not sorted
     bad = cb.copy()
-    bad[7] = 1e-3                                             # no exact zero
+    bad[7] = 1e-3                                             # no zero entry
     with pytest.raises(ValueError):
         oracle.codebook_quantize(W, bad)
+    bad = cb.copy()
+    bad[15] = 1.5                                             # outside [-1, 1]
+    with pytest.raises(ValueError):
+        oracle.codebook_quantize(W, bad)
+    bad[15] = np.nan
+    with pytest.raises(ValueError):
+        oracle.codebook_quantize(W, bad)
+    # a table in another order is a valid table with other codes
+    codes, _ = oracle.codebook_quantize(W, cb[::-1].copy())
+    codes2, _ = oracle.codebook_quantize(W, cb)
+    assert np.array_equal(codes, 15 - codes2)
+
+
+# --------------------------------------------------------------------------
+# FP4 (E2M1) table ([BNB] nf4与fp4): code order, +0 and -0
+# --------------------------------------------------------------------------
+def test_fp4_table_is_e2m1():
+    """The E2M1 magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 (over 6), positive for
+    codes 0..7 and negative for 8..15, both zeros present."""
+    cb = syn.codebook_fp4_e2m1()
+    mags = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6]) / 6
+    assert np.array_equal(cb[:8].astype(np.float64), mags.astype(np.float32).astype(np.float64))
+    assert np.array_equal(cb[8:], -cb[:8])
+    assert np.signbit(cb[8]) and not np.signbit(cb[0]) and cb[8] == 0.0
+    assert cb.max() == 1.0 and cb.min() == -1.0
+
+
+def test_fp4_entries_map_to_themselves_and_zero_to_code0():
+    """Idempotence on c_j * a for the 14 nonzero codes; a zero (either sign)
+    is code 0, the lower index of the two zeros."""
+    cb = syn.codebook_fp4_e2m1()
+    rng = np.random.default_rng(23)
+    nb = 64
+    j = rng.integers(0, 16, (nb, 64))
+    j[:, 0] = 7                                   # |c| = 1 in every block: absmax = a
+    a = 2.0 ** rng.integers(-8, -2, (nb, 1))
+    w = (cb[j].astype(np.float64) * a).astype(np.float32)
+    W = _bf16(w.reshape(16, 256))
+    # c_j * a survives the bf16 rounding exactly for about half the entries;
+    # the others move by at most 2^-9 of their value, far less than half a
+    # gap of the table (1/24 of a), so every entry still maps to its code
+    exact = oracle.bf16_to_f32(W).reshape(nb, 64) == w
+    codes, absmax = oracle.codebook_quantize(W, cb)
+    codes = codes.reshape(nb, 64)
+    expect = np.where(j == 8, 0, j)
+    assert exact.mean() > 0.3
+    assert np.array_equal(absmax, a.ravel().astype(np.float32))
+    assert np.array_equal(codes, expect.astype(np.uint8))
+
+
+def test_fp4_sign_symmetry():
+    """Negating the weights flips the sign bit of every nonzero code (E2M1 is
+    sign-magnitude and the table is symmetric in code order); values
+    quantized to zero stay code 0."""
+    cb = syn.codebook_fp4_e2m1()
+    W = syn.normal_bf16((32, 512), 0.015, 29)
+    c_pos, a_pos = oracle.codebook_quantize(syn.bits_u16(W), cb)
+    c_neg, a_neg = oracle.codebook_quantize(syn.bits_u16(-W), cb)
+    assert np.array_equal(a_pos, a_neg)
+    expect = np.where(c_pos == 0, 0, c_pos ^ 8)
+    assert np.array_equal(c_neg, expect)
+    assert not np.any(c_pos == 8)                 # -0 is never chosen
+
+
+def test_fp4_error_bound():
+    cb = syn.codebook_fp4_e2m1()
+    n, k = 32, 256
+    W = syn.bits_u16(syn.weight_bf16(n, k, 0.015, 31, outlier_frac=0.01))
+    codes, absmax = oracle.codebook_quantize(W, cb)
+    What = oracle.codebook_dequantize(oracle.pack(codes, 4), absmax, cb, n, k)
+    w = oracle.bf16_to_f32(W).astype(np.float64)
+    maxgap = np.diff(np.sort(cb.astype(np.float64))).max()       # 1/3 (4/6 to 6/6)
+    a = np.repeat(absmax.astype(np.float64), 64).reshape(n, k)
+    assert np.all(np.abs(w - What) <= a * (maxgap / 2) * (1 + 1e-6) + 1e-30)
 
 
 # --------------------------------------------------------------------------
@@ -500,3 +595,59 @@ def test_unmerge_inverts_an_exact_merge():
     merged = oracle.lora_merge(W, A, B, 0.5, 1)
     back = oracle.lora_merge(_as_f32(merged), A, B, 0.5, -1)
     assert np.array_equal(_as_f32(back), W)
+
+
+# --------------------------------------------------------------------------
+# channel-mix selection by sensitivity ([GB] 模型量化 (1))
+# --------------------------------------------------------------------------
+def test_channel_score_is_the_output_error_rise_for_one_hot_calibration():
+    """With one-hot calibration tokens x_t = a_t e_t (t = k), the weighted
+    squared errors are exactly the output error energies: score[c] =
+    (|X (w2_c - w_c)|^2 - |X (w4_c - w_c)|^2) / t, computed here with a
+    numpy matmul on the oracle's (pinned) dequantized weights."""
+    n, k = 12, 256
+    W = syn.bits_u16(syn.weight_bf16(n, k, 0.02, 41, outlier_frac=0.02))
+    rng = np.random.default_rng(3)
+    amp = (rng.integers(1, 8, k) * 2.0 ** rng.integers(-3, 3, k)).astype(np.float32)
+    X = _bf16(np.diag(amp))
+    score, bound = oracle.channel_score(W, X)
+    w = oracle.bf16_to_f32(W).astype(np.float64)
+    c4, s4, z4 = oracle.minmax_quantize(W, 4, 128)
+    c2, s2, z2 = oracle.minmax_quantize(W, 2, 64)
+    w4 = oracle.minmax_dequantize(oracle.pack(c4, 4), s4, z4, k, 4, 128).astype(np.float64)
+    w2 = oracle.minmax_dequantize(oracle.pack(c2, 2), s2, z2, k, 2, 64).astype(np.float64)
+    x = oracle.bf16_to_f32(X).astype(np.float64)
+    e2 = ((w2 - w) @ x.T) ** 2
+    e4 = ((w4 - w) @ x.T) ** 2
+    expect = (e2.sum(axis=1) - e4.sum(axis=1)) / k
+    assert np.allclose(score, expect, rtol=1e-12, atol=0)
+    assert np.allclose(bound, (e2.sum(axis=1) + e4.sum(axis=1)) / k, rtol=1e-12, atol=0)
+
+
+def test_channel_score_sign_cases():
+    """A channel exact on its INT4 grid has score = bound > 0 (only INT2
+    errs); a constant integer channel is exact in both (score = bound = 0);
+    a constant 0.25 channel errs equally in both (the degenerate scale 1)."""
+    rng = np.random.default_rng(9)
+    k = 256
+    q = rng.integers(0, 16, (1, k))
+    q[0, 0], q[0, 1], q[0, 128], q[0, 129] = 0, 15, 0, 15
+    z = rng.integers(0, 16, (1, 2))
+    sf = 2.0 ** -7
+    w_grid = ((q.reshape(1, 2, 128) - z[:, :, None]) * sf).reshape(1, k)
+    w = np.vstack([w_grid, np.full((1, k), 2.0), np.full((1, k), 0.25)]).astype(np.float32)
+    W = _bf16(w)
+    X = syn.bits_u16(syn.normal_bf16((32, k), 1.0, 5))
+    score, bound = oracle.channel_score(W, X)
+    assert score[0] > 0 and score[0] == bound[0]
+    assert score[1] == 0 and bound[1] == 0
+    assert score[2] == 0 and bound[2] > 0
+
+
+def test_channel_mix_select_top_scores_lower_index_on_ties():
+    score = np.array([0.5, 2.0, 1.0, 2.0, -1.0, 1.0, 0.0, 1.0])
+    perm = oracle.channel_mix_select(score, 4)
+    # highest: 1, 3 (2.0), then 2, 5 among the three equal 1.0 (2 < 5 < 7)
+    assert perm.tolist() == [1, 2, 3, 5, 0, 4, 6, 7]
+    assert oracle.channel_mix_select(score, 0).tolist() == list(range(8))
+    assert oracle.channel_mix_select(score, 8).tolist() == list(range(8))
