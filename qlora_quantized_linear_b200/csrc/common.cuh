@@ -139,6 +139,30 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
     return false;
 }
 
+// A producer's bounded wait for "nothing could be issued": call with
+// progress = whether anything was issued this round; returns false (and sets
+// *abort and the timeout status) once no progress was made for kWaitLimitNs
+// or another warp gave up.
+struct ProgressGuard {
+    uint64_t t0 = 0;
+    __device__ __forceinline__ bool step(bool progress, volatile int* abort) {
+        if (progress) {
+            t0 = 0;
+            return true;
+        }
+        if (*abort) return false;
+        const uint64_t now = globaltimer_ns();
+        if (t0 == 0) {
+            t0 = now;
+        } else if (now - t0 > kWaitLimitNs) {
+            *abort = 1;
+            record_status(kStatusTimeout);
+            return false;
+        }
+        return true;
+    }
+};
+
 // Split-tile flags: a contributor publishes its partial sums (stored by all
 // threads of the CTA before the barrier that precedes this call) and counts
 // itself; the finishing CTA waits for the count with acquire semantics.

@@ -13,8 +13,9 @@
 //               INT4 or 512 INT2 codes per row, 128-byte swizzle) into a
 //               second ring -- wide boxes keep the TMA engine efficient.
 //   warp 1      allocates tensor memory; lane 0 issues tcgen05.mma.
-//   warps 2..9  dequantize: output channel i is TMEM lane i; the two warps
-//               of a lane quarter each take half of a k-block.  A thread
+//   warps 2..   dequantize (16 warps for the 256-token tile, else 8): output
+//               channel i is TMEM lane i; the warps of a lane quarter each
+//               take one part (a quarter or a half) of a k-block.  A thread
 //               unpacks its row's codes from smem, forms bf16 W_hat values and
 //               stores them with tcgen05.st straight into the MMA's A operand
 //               in tensor memory (an ASTAGES-deep ring), so dequantized
@@ -102,6 +103,11 @@ struct GemmSmem {
     static constexpr size_t kLoraT = kTab + size_t(TABBYTES);
     static size_t total(int rank_pad) { return kLoraT + size_t(NT) * rank_pad * 4 + 1024; }
 };
+
+// bar.sync on barrier `id` for `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -210,23 +216,36 @@ __device__ __forceinline__ PreConst preload_const(const FwdParams& p, int64_t gr
     return c;
 }
 
-// Dequantize half of this thread's row of one k-block (32 codes) into 16
+// Dequantize part of this thread's row of one k-block (2 NV codes) into NV
 // bf16x2 words (first code of each pair in the low half).  `wrow` is the row's
 // 128-byte line of the weight chunk, stored by TMA with the 128-byte swizzle
 // (16-byte unit u of row r sits at unit u ^ (r & 7)); `byte0` is the offset of
-// this half k-block's codes within the line.
-template <int KIND>
-__device__ __forceinline__ void dequant_half_kblock(const uint8_t* wrow, int row, int byte0, PreConst pc,
+// the part's codes within the line.
+template <int KIND, int NV>
+__device__ __forceinline__ void dequant_part_kblock(const uint8_t* wrow, int row, int byte0, PreConst pc,
                                                     float dq_offset, bool has_dq, const float* s_cb,
-                                                    uint32_t (&out)[16]) {
-    const int unit = (byte0 >> 4) ^ (row & 7);
+                                                    uint32_t (&out)[NV]) {
+    constexpr int NW = (KIND == kInt2) ? NV / 8 : NV / 4;   // 32-bit words of codes
+    const uint8_t* src = wrow + 16 * ((byte0 >> 4) ^ (row & 7)) + (byte0 & 15);
+    uint32_t w[NW];
+    if (NW == 4) {
+        const uint4 c = *reinterpret_cast<const uint4*>(src);
+        w[0] = c.x;
+        w[1 % NW] = c.y;
+        w[2 % NW] = c.z;
+        w[3 % NW] = c.w;
+    } else if (NW == 2) {
+        const uint2 c = *reinterpret_cast<const uint2*>(src);
+        w[0] = c.x;
+        w[1 % NW] = c.y;
+    } else {
+        w[0] = *reinterpret_cast<const uint32_t*>(src);
+    }
     if (KIND == kInt4) {
-        const uint4 c4 = *reinterpret_cast<const uint4*>(wrow + 16 * unit);
-        const uint32_t w[4] = {c4.x, c4.y, c4.z, c4.w};
         const MinMaxConst c = minmax_const(static_cast<uint16_t>(pc.a), static_cast<uint16_t>(pc.b));
         if (c.fast) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < NW; ++i) {
                 uint32_t o[4];
                 unpack_int4_word(w[i], o);
 #pragma unroll
@@ -234,18 +253,16 @@ __device__ __forceinline__ void dequant_half_kblock(const uint8_t* wrow, int row
             }
         } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < NW; ++i)
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     out[4 * i + j] = minmax_pair_exact((w[i] >> (8 * j + 4)) & 15u, (w[i] >> (8 * j)) & 15u, c);
         }
     } else if (KIND == kInt2) {
-        const uint2 c2 = *reinterpret_cast<const uint2*>(wrow + 16 * unit + (byte0 & 15));
-        const uint32_t w[2] = {c2.x, c2.y};
         const MinMaxConst c = minmax_const(static_cast<uint16_t>(pc.a), static_cast<uint16_t>(pc.b));
         if (c.fast) {
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
+            for (int i = 0; i < NW; ++i) {
                 uint32_t o[8];
                 unpack_int2_word(w[i], o);
 #pragma unroll
@@ -253,7 +270,7 @@ __device__ __forceinline__ void dequant_half_kblock(const uint8_t* wrow, int row
             }
         } else {
 #pragma unroll
-            for (int i = 0; i < 2; ++i)
+            for (int i = 0; i < NW; ++i)
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -263,14 +280,12 @@ __device__ __forceinline__ void dequant_half_kblock(const uint8_t* wrow, int row
         }
     } else {
         // codebook: W_hat = bf16(fp32(codebook[code] * absmax')), absmax per 64
-        const uint4 c4 = *reinterpret_cast<const uint4*>(wrow + 16 * unit);
-        const uint32_t w[4] = {c4.x, c4.y, c4.z, c4.w};
         const float a = has_dq ? __fadd_rn(__fmul_rn(__fdiv_rn(static_cast<float>(static_cast<int32_t>(pc.a)), 127.0f),
                                                      __uint_as_float(pc.b)),
                                            dq_offset)
                                : __uint_as_float(pc.a);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < NW; ++i)
 #pragma unroll
             for (int j = 0; j < 4; ++j)
                 out[4 * i + j] = pack_bf16x2_rn(__fmul_rn(s_cb[(w[i] >> (8 * j + 4)) & 15u], a),
@@ -304,20 +319,53 @@ __device__ __forceinline__ void lora_add16(float (&acc)[16], const float* sT, in
     }
 }
 
+// Row tt of the adapter operand tile: bf16(s * T[t0 + tt, u]) for u <
+// rank_pad in a 128-byte-swizzled K-major tile of 128-byte rows (16-byte
+// unit c of row tt at unit c ^ (tt & 7)), zero beyond the rank and beyond the
+// mt real tokens.  One token row per thread, its loads all in flight
+// together (the tile is staged before the main loop, on its critical path).
+__device__ __forceinline__ void stage_scaled_rows(uint8_t* tile, const float* T, int64_t t0, int mt, int nrows,
+                                                  int rank, int rank_pad, float s, int tid, int nthreads) {
+    for (int tt = tid; tt < nrows; tt += nthreads) {
+        const float* row = T + (t0 + tt) * rank;
+        const bool tok = tt < mt;
+        for (int u0 = 0; u0 < rank_pad; u0 += 16) {
+            float v[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) v[q] = (tok && u0 + q < rank) ? __ldg(row + u0 + q) : 0.0f;
+            uint32_t w[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) w[q] = pack_bf16x2_rn(__fmul_rn(s, v[2 * q]), __fmul_rn(s, v[2 * q + 1]));
+            const int c0 = u0 >> 3;
+            *reinterpret_cast<uint4*>(tile + tt * 128 + ((c0 ^ (tt & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(tile + tt * 128 + (((c0 + 1) ^ (tt & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
+        }
+    }
+}
+
 // Launch shape of the forward kernel: warp 0 = TMA producer, warp 1 = TMEM
-// allocator + MMA issuer, warps 2..9 = dequantize + epilogue.  Two dequant
-// warps share each TMEM lane quarter (warp & 3); warp group h = (warp-2)/4
-// takes half h of every k-block and, in the epilogue, half h of the tokens.
-constexpr int kFwdThreads = 320;
-constexpr int kDqWarps = 8;
+// allocator + MMA issuer, then DQW dequantize + epilogue warps.  DQW / 4
+// dequant warps share each TMEM lane quarter (warp & 3); part p = (warp-2)/4
+// takes part p of every k-block and, in the epilogue, part p of the tokens.
+// The 256-token tile (one CTA per SM) runs 16 dequant warps, so that each
+// warp's share of a k-block is short and the slowest warp, which gates the
+// MMAs, is never far behind; smaller tiles (two CTAs per SM) run 8.
+__host__ __device__ constexpr int fwd_threads(int dqw) { return 64 + 32 * dqw; }
+
+__device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
 
 template <int NT>
 struct FwdCfg {
     static constexpr int kXBlocks = NT <= 16 ? 8 : NT <= 32 ? 4 : NT <= 64 ? 2 : 1;   // k-blocks per X box
     static constexpr int kXStages = NT <= 32 ? 2 : NT <= 128 ? 3 : 4;
-    static constexpr int kWStages = NT <= 32 ? 4 : NT <= 64 ? 3 : 2;
+    static constexpr int kWStages = NT <= 32 ? 4 : NT <= 64 ? 3 : NT <= 128 ? 2 : 4;
     static constexpr int kAStages = NT <= 32 ? 6 : 4;
     static constexpr int kMinBlocks = NT >= 256 ? 1 : 2;   // CTAs per SM
+    static constexpr int kDqWarps = NT >= 256 ? 16 : 8;
 };
 
 __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
@@ -329,11 +377,13 @@ __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_
         : "memory");
 }
 
-template <int NT, int KIND, int XS, int XB, int WS, int AS, int MINB>
-__global__ void __launch_bounds__(kFwdThreads, MINB)
+template <int NT, int KIND, int XS, int XB, int WS, int AS, int MINB, int DQW>
+__global__ void __launch_bounds__(fwd_threads(DQW), MINB)
 dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                   const FwdParams p) {
     constexpr int WB = WeightTile<KIND>::kRowBytes;
+    constexpr int PARTS = DQW / 4;                     // dequant warps per TMEM lane quarter
+    constexpr int NV = 32 / PARTS;                     // bf16x2 words of a warp's part of a k-block row
     constexpr int SUB = WeightTile<KIND>::kSub;        // k-blocks per weight chunk
     using L = FwdSmem<NT, XS, XB, WS, AS>;
     constexpr int kACols = 32;                         // one k-block of 64 bf16 = 32 columns
@@ -382,10 +432,10 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         }
         for (int i = 0; i < WS; ++i) {
             mbar_init(&fullW[i], 1);
-            mbar_init(&emptyW[i], kDqWarps);
+            mbar_init(&emptyW[i], DQW);
         }
         for (int i = 0; i < AS; ++i) {
-            mbar_init(&afull[i], kDqWarps);
+            mbar_init(&afull[i], DQW);
             mbar_init(&aempty[i], 1);
         }
         mbar_init(dfull, 1);
@@ -409,28 +459,34 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        // Weight chunks run ahead of the activation tiles: chunk c is issued
-        // before the first k-block that needs it.
+        // The weight chunks and the activation tiles are two independent
+        // streams: each is issued as soon as its own ring has a free slot
+        // (weights: released by the dequantize warps; activations: by the
+        // MMAs), so that neither waits behind the other.
         if (lane == 0) {
-            int xi = 0, wi = 0;
+            const int nxb = (nkb + XB - 1) / XB;           // activation boxes
+            int xi = 0, wi = 0;                            // next box / chunk to issue
+            ProgressGuard guard;
             bool ok = true;
-            for (int i = 0; i < nkb && ok; ++i) {
-                if (i % SUB == 0) {
-                    const int c = i / SUB, w = c % WS;
-                    if (c >= WS && !mbar_wait(&emptyW[w], ((c / WS) - 1) & 1, s_abort)) { ok = false; break; }
+            while (ok && (wi < nch || xi < nxb)) {
+                bool prog = false;
+                if (wi < nch && (wi < WS || mbar_try_wait(&emptyW[wi % WS], ((wi / WS) - 1) & 1))) {
+                    const int w = wi % WS;
                     mbar_arrive_expect_tx(&fullW[w], L::kWBytes);
-                    tma_load_2d(sW + w * L::kWBytes, &tmW, &fullW[w], (kb0 + i) * WB, n0);
-                    wi = c + 1;
+                    tma_load_2d(sW + w * L::kWBytes, &tmW, &fullW[w], (kb0 + wi * SUB) * WB, n0);
+                    ++wi;
+                    prog = true;
                 }
-                if (i % XB == 0) {
-                    const int j = i / XB, x = j % XS;
-                    if (j >= XS && !mbar_wait(&emptyX[x], ((j / XS) - 1) & 1, s_abort)) { ok = false; break; }
-                    LBQ_TRACE_EVENT(6, i);
+                if (xi < nxb && (xi < XS || mbar_try_wait(&emptyX[xi % XS], ((xi / XS) - 1) & 1))) {
+                    const int x = xi % XS;
+                    LBQ_TRACE_EVENT(6, xi * XB);
                     mbar_arrive_expect_tx(&fullX[x], L::kXBytes);
-                    tma_load_3d(sX + x * L::kXBytes, &tmX, &fullX[x], 0, t0, kb0 + i);
-                    LBQ_TRACE_EVENT(1, i);
-                    xi = j + 1;
+                    tma_load_3d(sX + x * L::kXBytes, &tmX, &fullX[x], 0, t0, kb0 + xi * XB);
+                    LBQ_TRACE_EVENT(1, xi * XB);
+                    ++xi;
+                    prog = true;
                 }
+                ok = guard.step(prog, s_abort);
             }
             // never leave with a copy in flight (matters only after an abort)
             for (int j = max(0, xi - XS); j < xi; ++j) mbar_wait_drain(&fullX[j % XS], (j / XS) & 1);
@@ -472,7 +528,7 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     } else {
         // ------------------------------------------------------------ dequantize
         const int q = warp & 3;              // TMEM lane quarter of this warp
-        const int half = (warp - 2) >> 2;    // k-block half (and token half in the epilogue)
+        const int part = (warp - 2) >> 2;    // k-block part (and token part in the epilogue)
         const int row = q * 32 + lane;       // output channel within the tile
         const int64_t grow = n0 + row;       // stored weight row
         const bool row_ok = grow < p.n;
@@ -483,30 +539,21 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         const int mt = min(NT, p.m - t0);                  // tokens in this tile
         if (lora) {
             // A operand (ring slot 0): this row's adapter coefficients
-            // B[out_col, 32 half .. 32 half + 31] (bf16, zero beyond the rank)
-            uint32_t bv[16];
+            // B[out_col, 2 NV part .. 2 NV part + 2 NV - 1] (bf16, zero beyond the rank)
+            uint32_t bv[NV];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int u = 32 * half + 2 * i;
+            for (int i = 0; i < NV; ++i) {
+                const int u = 2 * NV * part + 2 * i;
                 const uint32_t lo = (row_ok && u < p.rank) ? __ldg(p.B + static_cast<int64_t>(out_col) * p.rank + u) : 0u;
                 const uint32_t hi = (row_ok && u + 1 < p.rank) ? __ldg(p.B + static_cast<int64_t>(out_col) * p.rank + u + 1) : 0u;
                 bv[i] = lo | (hi << 16);
             }
-            tmem_st_32x32b_x16(tmem + lane_base + kACol0 + 16 * half, bv);
-            // B operand: bf16(s * T[t0 + tt, u]) at row tt, 16-byte unit u / 8 of its
-            // 128-byte line, swizzled with the row (zero beyond the tokens and the rank)
-            const int tid = threadIdx.x - 64;
-            for (int e = tid; e < NT * 32; e += 32 * kDqWarps) {
-                const int tt = e >> 5, u = 2 * (e & 31);
-                float v0 = 0.0f, v1 = 0.0f;
-                if (tt < mt) {
-                    const float* trow = p.T + static_cast<int64_t>(t0 + tt) * p.rank;
-                    if (u < p.rank) v0 = __fmul_rn(p.s, trow[u]);
-                    if (u + 1 < p.rank) v1 = __fmul_rn(p.s, trow[u + 1]);
-                }
-                *reinterpret_cast<uint32_t*>(sTop + tt * 128 + (((u >> 3) ^ (tt & 7)) << 4) + (u & 7) * 2) =
-                    pack_bf16x2_rn(v0, v1);
-            }
+            if (NV == 16)
+                tmem_st_32x32b_x16(tmem + lane_base + kACol0 + NV * part, reinterpret_cast<const uint32_t(&)[16]>(bv));
+            else
+                tmem_st_32x32b_x8(tmem + lane_base + kACol0 + NV * part, reinterpret_cast<const uint32_t(&)[8]>(bv));
+            // B operand: the tile of bf16(s * T) rows
+            stage_scaled_rows(sTop, p.T, t0, mt, NT, p.rank, p.rank_pad, p.s, threadIdx.x - 64, 32 * DQW);
             fence_proxy_async_smem();
             tmem_st_wait();
             tc_fence_before();
@@ -514,6 +561,18 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             if (lane == 0) mbar_arrive(&afull[0]);
         }
         PreConst nxt = preload_const<KIND>(p, grow, kb0, row_ok && nkb > 0);
+        // A k-block's tensor-memory store completes while the next k-block is
+        // dequantized: its arrival on afull comes one k-block later, off the
+        // warp's critical path (the A ring keeps the MMAs fed meanwhile).
+        int pend = -1;                                     // A slot whose store is in flight
+        auto release_pending = [&]() {
+            if (pend < 0) return;
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&afull[pend]);
+            pend = -1;
+        };
         for (int i = 0; i < nkb; ++i) {
             const int c = i / SUB, sub = i - c * SUB, w = c % WS, ia = i + a_off, a = ia % AS;
             const PreConst cur = nxt;
@@ -521,37 +580,43 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             if (sub == 0 && !mbar_wait(&fullW[w], (c / WS) & 1, s_abort)) break;
             if (ia >= AS && !mbar_wait(&aempty[a], ((ia / AS) - 1) & 1, s_abort)) break;
             tc_fence_after();
-            if (lane == 0) LBQ_TRACE_EVENT(2, i * 8 + (warp - 2));
-            uint32_t vals[16];
+            if (lane == 0) LBQ_TRACE_EVENT(2, i * DQW + (warp - 2));
+            uint32_t vals[NV];
             if (row_ok) {
-                dequant_half_kblock<KIND>(sW + w * L::kWBytes + row * 128, row, sub * WB + half * (WB / 2), cur,
-                                          dq_offset, has_dq, s_cb, vals);
+                dequant_part_kblock<KIND, NV>(sW + w * L::kWBytes + row * 128, row, sub * WB + part * (WB / PARTS), cur,
+                                              dq_offset, has_dq, s_cb, vals);
             } else {
 #pragma unroll
-                for (int j = 0; j < 16; ++j) vals[j] = 0u;
+                for (int j = 0; j < NV; ++j) vals[j] = 0u;
             }
-            tmem_st_32x32b_x16(tmem + lane_base + kACol0 + a * kACols + 16 * half, vals);
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&afull[a]);
-                if (sub == SUB - 1 || i == nkb - 1) mbar_arrive(&emptyW[w]);
+            // the warp's last read of this weight chunk
+            if (sub == SUB - 1 || i == nkb - 1) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&emptyW[w]);
             }
-            if (lane == 0) LBQ_TRACE_EVENT(3, i * 8 + (warp - 2));
+            release_pending();
+            if (NV == 16)
+                tmem_st_32x32b_x16(tmem + lane_base + kACol0 + a * kACols + NV * part,
+                                   reinterpret_cast<const uint32_t(&)[16]>(vals));
+            else
+                tmem_st_32x32b_x8(tmem + lane_base + kACol0 + a * kACols + NV * part,
+                                  reinterpret_cast<const uint32_t(&)[8]>(vals));
+            pend = a;
+            if (lane == 0) LBQ_TRACE_EVENT(3, i * DQW + (warp - 2));
         }
+        release_pending();
         (void)nch;
 
         // ------------------------------------------------------------ epilogue
         // (the adapter term is already in the accumulator)
-        asm volatile("bar.sync 1, 256;" ::: "memory");
+        named_barrier_sync(1, 32 * DQW);
         const bool got = mbar_wait(dfull, 0, s_abort);
         tc_fence_after();
         if (threadIdx.x == 64) LBQ_TRACE_EVENT(0, 1);
         const bool splitk = p.nsplit > 1;
-        constexpr int kHalfCols = NT >= 32 ? NT / 2 : 16;  // token columns per warp group
-        const int c_begin = half * kHalfCols;
-        const int c_end = min(NT, c_begin + kHalfCols);
+        constexpr int kPartCols = NT / PARTS >= 16 ? NT / PARTS : 16;   // token columns per warp part
+        const int c_begin = part * kPartCols;
+        const int c_end = min(NT, c_begin + kPartCols);
         for (int jj = c_begin; jj < c_end; jj += 16) {
             uint32_t raw[16];
             tmem_ld_32x32b_x16(tmem + lane_base + kDCol + jj, raw);
@@ -573,7 +638,7 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         if (splitk) {
             // the last CTA of this output tile sums the partials in split order
             __threadfence();
-            asm volatile("bar.sync 1, 256;" ::: "memory");
+            named_barrier_sync(1, 32 * DQW);
             if (threadIdx.x == 64) {
                 const uint32_t tile = blockIdx.y * gridDim.x + blockIdx.x;
                 const uint32_t prev = atomicAdd(p.counters + tile, 1u);
@@ -581,7 +646,7 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 if (last) p.counters[tile] = 0u;
                 *s_last = last;
             }
-            asm volatile("bar.sync 1, 256;" ::: "memory");
+            named_barrier_sync(1, 32 * DQW);
             if (*s_last && row_ok && got) {
                 __threadfence();
                 for (int jj = c_begin; jj < min(c_end, mt); jj += 16) {

@@ -19,8 +19,8 @@
 //    two bytes apart), so within every 8 (INT4) or 16 (INT2) features the A
 //    tile holds the features in a fixed permuted order; the epilogue writes
 //    each tensor-memory lane back to its own feature.
-//  * Roles: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, warps 2..9
-//    dequantize and run the epilogue.  Rings, bounded waits and the split-K
+//  * Roles: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, then 16
+//    (256-token tile) or 8 warps dequantize and run the epilogue.  Rings, bounded waits and the split-K
 //    reduction (the last CTA of a tile sums the partials in split order) follow
 //    the forward kernel.
 #pragma once
@@ -61,15 +61,14 @@ struct BwdParams {
     uint32_t* counters;
 };
 
-constexpr int kBwdThreads = 320;
-constexpr int kBwdDqWarps = 8;
 
 template <int NT>
 struct BwdCfg {
-    static constexpr int kXStages = NT <= 64 ? 4 : NT <= 128 ? 2 : 3;
+    static constexpr int kXStages = NT <= 64 ? 4 : NT <= 128 ? 2 : 4;   // dY tiles in flight (see the forward)
     static constexpr int kWStages = 4;
     static constexpr int kAStages = NT <= 64 ? 3 : 2;
     static constexpr int kMinBlocks = NT >= 256 ? 1 : 2;   // CTAs per SM
+    static constexpr int kDqWarps = NT >= 256 ? 16 : 8;     // dequantize + epilogue warps
 };
 
 template <int NT, int BITS, int XS, int WS, int AS>
@@ -121,15 +120,17 @@ __device__ __forceinline__ uint32_t bwd_a_offset(int c, int fu) {
     return static_cast<uint32_t>((c >> 3) * 2048 + (fu >> 3) * 1024 + row * 128 + ((uu ^ row) << 4));
 }
 
-template <int NT, int KIND, int XS, int WS, int AS, int MINB>
-__global__ void __launch_bounds__(kBwdThreads, MINB)
+template <int NT, int KIND, int XS, int WS, int AS, int MINB, int DQW>
+__global__ void __launch_bounds__(fwd_threads(DQW), MINB)
 dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constant__ CUtensorMap tmW,
                   const BwdParams p) {
     constexpr int BITS = KIND == kInt2 ? 2 : 4;
     using L = BwdSmem<NT, BITS, XS, WS, AS>;
     constexpr int KTB = L::kKTB;
     constexpr int PG = BITS == 4 ? 8 : 16;                 // features per pairing group
-    constexpr int SLOTS = BITS == 4 ? 4 : 2;               // (channel, word) units per thread and block
+    constexpr int WPR = BITS == 4 ? 16 : 8;                // 32-bit code words per channel row of a block
+    constexpr int SLOTS = 64 * WPR / (32 * DQW);           // (channel, word) units per thread and block
+    constexpr int PARTS = DQW / 4;                         // epilogue warps per TMEM lane quarter
     constexpr uint32_t kTmemCols = tmem_cols_for(NT);
     constexpr uint32_t kIdesc = idesc_bf16_f32(128, NT) | (1u << 15);   // A is MN-major
 
@@ -172,10 +173,10 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
         }
         for (int i = 0; i < WS; ++i) {
             mbar_init(&fullW[i], 1);
-            mbar_init(&emptyW[i], kBwdDqWarps);
+            mbar_init(&emptyW[i], DQW);
         }
         for (int i = 0; i < AS; ++i) {
-            mbar_init(&afull[i], kBwdDqWarps);
+            mbar_init(&afull[i], DQW);
             mbar_init(&aempty[i], 1);
         }
         mbar_init(dfull, 1);
@@ -199,18 +200,29 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
+            // two independent streams, each issued as soon as its ring has a
+            // free slot (weights: released by the dequantize warps; dY: by
+            // the MMAs)
             int wi = 0, xi = 0;
-            for (int i = 0; i < ncb; ++i) {
-                const int w = i % WS, x = i % XS;
-                const int c0 = (cb0 + i) * 64;
-                if (i >= WS && !mbar_wait(&emptyW[w], ((i / WS) - 1) & 1, s_abort)) break;
-                mbar_arrive_expect_tx(&fullW[w], L::kWBytes);
-                tma_load_2d(sW + w * L::kWBytes, &tmW, &fullW[w], k0 * BITS / 8, c0);
-                wi = i + 1;
-                if (i >= XS && !mbar_wait(&emptyX[x], ((i / XS) - 1) & 1, s_abort)) break;
-                mbar_arrive_expect_tx(&fullX[x], L::kXBytes);
-                tma_load_2d(sX + x * L::kXBytes, &tmDY, &fullX[x], c0, t0);
-                xi = i + 1;
+            ProgressGuard guard;
+            bool ok = true;
+            while (ok && (wi < ncb || xi < ncb)) {
+                bool prog = false;
+                if (wi < ncb && (wi < WS || mbar_try_wait(&emptyW[wi % WS], ((wi / WS) - 1) & 1))) {
+                    const int w = wi % WS;
+                    mbar_arrive_expect_tx(&fullW[w], L::kWBytes);
+                    tma_load_2d(sW + w * L::kWBytes, &tmW, &fullW[w], k0 * BITS / 8, (cb0 + wi) * 64);
+                    ++wi;
+                    prog = true;
+                }
+                if (xi < ncb && (xi < XS || mbar_try_wait(&emptyX[xi % XS], ((xi / XS) - 1) & 1))) {
+                    const int x = xi % XS;
+                    mbar_arrive_expect_tx(&fullX[x], L::kXBytes);
+                    tma_load_2d(sX + x * L::kXBytes, &tmDY, &fullX[x], (cb0 + xi) * 64, t0);
+                    ++xi;
+                    prog = true;
+                }
+                ok = guard.step(prog, s_abort);
             }
             for (int i = max(0, xi - XS); i < xi; ++i) mbar_wait_drain(&fullX[i % XS], (i / XS) & 1);
             for (int i = max(0, wi - WS); i < wi; ++i) mbar_wait_drain(&fullW[i % WS], (i / WS) & 1);
@@ -249,11 +261,11 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
         }
     } else {
         // ------------------------------------------------------------ dequantize
-        const int tid = threadIdx.x - 64;                  // 0..255
+        const int tid = threadIdx.x - 64;                  // 0 .. 32 DQW - 1
         // unit slot u: channel row cl(u) of the block and word fw of that row
-        const int fw = BITS == 4 ? (tid & 15) : (tid & 7);
-        const int crow0 = BITS == 4 ? (tid >> 4) : (tid >> 3);
-        const int cstep = BITS == 4 ? 16 : 32;
+        const int fw = tid % WPR;
+        const int crow0 = tid / WPR;
+        constexpr int cstep = 32 * DQW / WPR;
         const int gsub = BITS == 4 ? 0 : (fw >> 2);        // 64-feature group of this word (INT2 g64)
         const int gcol = KIND == kCode4 ? 0 : k0 / p.group + gsub;
         const int64_t kbt = p.k / 64;
@@ -287,7 +299,7 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
             // A operand (ring slot 0): K row u = A[u, k0 + feature], features in
             // the tile's pairing order (zero beyond the rank and beyond k)
             const int nunits = p.rank_pad * 16;            // 16-byte units: 8 features of one row
-            for (int e = tid; e < nunits; e += 32 * kBwdDqWarps) {
+            for (int e = tid; e < nunits; e += 32 * DQW) {
                 const int u = e >> 4, fu = e & 15;
                 uint32_t wv[4];
 #pragma unroll
@@ -304,20 +316,8 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
                 }
                 *reinterpret_cast<uint4*>(sA + bwd_a_offset(u, fu)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
-            // B operand: bf16(s * U[t0 + tt, u]) at row tt, 16-byte unit u / 8,
-            // swizzled with the row (zero beyond the tokens and the rank)
-            const int mt0 = min(NT, p.m - t0);
-            for (int e = tid; e < NT * 32; e += 32 * kBwdDqWarps) {
-                const int tt = e >> 5, u = 2 * (e & 31);
-                float v0 = 0.0f, v1 = 0.0f;
-                if (tt < mt0) {
-                    const float* urow = p.U + static_cast<int64_t>(t0 + tt) * p.rank;
-                    if (u < p.rank) v0 = __fmul_rn(p.s, urow[u]);
-                    if (u + 1 < p.rank) v1 = __fmul_rn(p.s, urow[u + 1]);
-                }
-                *reinterpret_cast<uint32_t*>(sUop + tt * 128 + (((u >> 3) ^ (tt & 7)) << 4) + (u & 7) * 2) =
-                    pack_bf16x2_rn(v0, v1);
-            }
+            // B operand: the tile of bf16(s * U) rows
+            stage_scaled_rows(sUop, p.U, t0, min(NT, p.m - t0), NT, p.rank, p.rank_pad, p.s, tid, 32 * DQW);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&afull[0]);
@@ -389,7 +389,7 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
 
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;                            // TMEM lane quarter of this warp
-        const int half = (warp - 2) >> 2;                  // token half
+        const int part = (warp - 2) >> 2;                  // token part
         const int lrow = q * 32 + lane;                    // A-tile row = TMEM lane
         // feature of this lane: the pairing order of its group of PG features
         const int feat = (lrow & ~(PG - 1)) + bwd_xperm(KIND, lrow & (PG - 1));
@@ -398,13 +398,13 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         const int mt = min(NT, p.m - t0);
         // (the adapter term is already in the accumulator)
-        asm volatile("bar.sync 1, 256;" ::: "memory");
+        named_barrier_sync(1, 32 * DQW);
         const bool got = mbar_wait(dfull, 0, s_abort);
         tc_fence_after();
         const bool splitk = p.nsplit > 1;
-        constexpr int kHalfCols = NT >= 32 ? NT / 2 : 16;
-        const int c_begin = half * kHalfCols;
-        const int c_end = min(NT, c_begin + kHalfCols);
+        constexpr int kPartCols = NT / PARTS >= 16 ? NT / PARTS : 16;
+        const int c_begin = part * kPartCols;
+        const int c_end = min(NT, c_begin + kPartCols);
         for (int jj = c_begin; jj < c_end; jj += 16) {
             uint32_t raw[16];
             tmem_ld_32x32b_x16(tmem + lane_base + jj, raw);
@@ -425,7 +425,7 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
         }
         if (splitk) {
             __threadfence();
-            asm volatile("bar.sync 1, 256;" ::: "memory");
+            named_barrier_sync(1, 32 * DQW);
             if (threadIdx.x == 64) {
                 const uint32_t tile = blockIdx.y * gridDim.x + blockIdx.x;
                 const uint32_t prev = atomicAdd(p.counters + tile, 1u);
@@ -433,7 +433,7 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
                 if (last) p.counters[tile] = 0u;   // left at zero for the next call
                 *s_last = last;
             }
-            asm volatile("bar.sync 1, 256;" ::: "memory");
+            named_barrier_sync(1, 32 * DQW);
             if (*s_last && col_ok && got) {
                 __threadfence();
                 for (int jj = c_begin; jj < min(c_end, mt); jj += 16) {

@@ -27,7 +27,7 @@ struct GvPlan {
     int count = 0;
     int ctas = 0;                   // grid
     int ws = 0;                     // ring stages
-    int stage_bytes = 0, xbox_max = 0, cstride = 0;
+    int stage_bytes = 0, xbox_max = 0, cslot_bytes = 0, cstride = 0;
     size_t smem = 0;                // dynamic shared memory per CTA
     size_t workspace = 0;           // 0 when no tile is split
     int share[kGvMaxProblems] = {}, pctas[kGvMaxProblems] = {}, cta0[kGvMaxProblems] = {};
@@ -46,7 +46,8 @@ double gv_unit_bytes(const lbq_qweight* q) {
 
 // Bytes per row of one constant array that a weight box needs: the 4-byte
 // words covering its groups (MinMax: 2 groups for INT4, 8 for INT2, starting
-// at any entry), 4 absmax values, or 2 words of q8 and 2 of s2.
+// at any entry), 4 absmax values, or 2 words of q8 (and of s2 in the second
+// array).
 int gv_const_stride(const lbq_qweight* q) {
     if (q->scheme == LBQ_CODEBOOK4) return q->double_quant ? 8 : 16;
     const int gpb = q->bits == 2 ? 8 : 2;                               // groups per box
@@ -78,17 +79,20 @@ lbq_status gv_plan(int m, const lbq_qweight* const* qs, int count, int sms, GvPl
         tiles_sum += static_cast<int>(tiles);
     }
     if (tiles_sum > kMaxSplitTiles) return LBQ_EUNSUPPORTED;
-    // stage layout: weight box, activation box; then one constant buffer of
-    // two slots per compute warp
+    // stage layout: weight box, activation box; after the ring the constant
+    // ring (ws + kGvConstAhead slots of [2 arrays][128 rows][cstride]) and the
+    // buffer in which the compute warps add the two k-halves of their rows
     const int sub_max = any_int2 ? 8 : 4;
     pl->xbox_max = sub_max * gv_mpad(m) * 128;
     pl->cstride = cstride;
+    pl->cslot_bytes = 256 * cstride;
     pl->stage_bytes = kGvWBox + pl->xbox_max;
-    const size_t cbuf = static_cast<size_t>(kGvComputeWarps) * 2 * 32 * cstride;
+    const size_t xchg = m <= 8 ? kGvXchgBytes : 0;
     (void)any_code;
     pl->ws = 0;
     for (int ws = kGvMaxStages; ws >= 2; --ws) {
-        const size_t smem = 1024 + static_cast<size_t>(ws) * pl->stage_bytes + cbuf + kGvExtraSmem;
+        const size_t smem = 1024 + static_cast<size_t>(ws) * pl->stage_bytes +
+                            static_cast<size_t>(ws + kGvConstAhead) * pl->cslot_bytes + xchg + kGvExtraSmem;
         if (smem <= kGemvSmemBudget) {
             pl->ws = ws;
             pl->smem = smem;
@@ -162,6 +166,7 @@ lbq_status run_gemv_group(int m, const GvJob* jobs, int count, void* ws, size_t 
     prm.m = m;
     prm.ws = pl.ws;
     prm.stage_bytes = pl.stage_bytes;
+    prm.cslot_bytes = pl.cslot_bytes;
     prm.cstride = pl.cstride;
     prm.w_early = weights_stable(st) ? 1 : 0;
     for (int i = 0; i < count; ++i) {

@@ -199,7 +199,8 @@ lbq_status launch_fwd_nt(const FwdParams& p, const void* X, int m, int64_t k, co
                          int nsplit, cudaStream_t st) {
     using C = FwdCfg<NT>;
     using L = FwdSmem<NT, C::kXStages, C::kXBlocks, C::kWStages, C::kAStages>;
-    auto kern = dqgemm_fwd_kernel<NT, KIND, C::kXStages, C::kXBlocks, C::kWStages, C::kAStages, C::kMinBlocks>;
+    auto kern = dqgemm_fwd_kernel<NT, KIND, C::kXStages, C::kXBlocks, C::kWStages, C::kAStages, C::kMinBlocks,
+                                  C::kDqWarps>;
     const size_t smem = L::total(p.rank);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
         return LBQ_ECUDA;
@@ -209,7 +210,7 @@ lbq_status launch_fwd_nt(const FwdParams& p, const void* X, int m, int64_t k, co
                      CU_TENSOR_MAP_SWIZZLE_128B))
         return LBQ_ECUDA;
     dim3 grid(static_cast<unsigned>(cdiv(nrows, 128)), static_cast<unsigned>(cdiv(m, NT)), static_cast<unsigned>(nsplit));
-    kern<<<grid, kFwdThreads, smem, st>>>(tmX, tmW, p);
+    kern<<<grid, fwd_threads(C::kDqWarps), smem, st>>>(tmX, tmW, p);
     return last_launch();
 }
 
@@ -284,7 +285,7 @@ lbq_status launch_bwd_nt(const BwdParams& p, const void* dY, const uint8_t* pack
     constexpr int BITS = KIND == kInt2 ? 2 : 4;
     using C = BwdCfg<NT>;
     using L = BwdSmem<NT, BITS, C::kXStages, C::kWStages, C::kAStages>;
-    auto kern = dqgemm_bwd_kernel<NT, KIND, C::kXStages, C::kWStages, C::kAStages, C::kMinBlocks>;
+    auto kern = dqgemm_bwd_kernel<NT, KIND, C::kXStages, C::kWStages, C::kAStages, C::kMinBlocks, C::kDqWarps>;
     const size_t smem = L::total(p.rank_pad);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
         return LBQ_ECUDA;
@@ -296,7 +297,7 @@ lbq_status launch_bwd_nt(const BwdParams& p, const void* dY, const uint8_t* pack
         return LBQ_ECUDA;
     dim3 grid(static_cast<unsigned>(cdiv(p.k, 128)), static_cast<unsigned>(cdiv(p.m, NT)),
               static_cast<unsigned>(p.nsplit));
-    kern<<<grid, kBwdThreads, smem, st>>>(tmDY, tmW, p);
+    kern<<<grid, fwd_threads(C::kDqWarps), smem, st>>>(tmDY, tmW, p);
     return last_launch();
 }
 

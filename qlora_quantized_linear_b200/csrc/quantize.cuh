@@ -36,11 +36,12 @@ __device__ __forceinline__ float rint_div(float w, float d, float rs) {
 
 // ---------------------------------------------------------------------------
 // MinMax quantize + pack.  Group = 128 (4 bit) or 64 (2 bit); one group is
-// covered by GROUP/8 consecutive lanes.  Each warp first issues the 16-byte
-// loads of kQuantUnroll chunks of 32 lanes (a grid stride apart), then
-// processes them, so that several loads per lane are in flight.
+// covered by GROUP/8 consecutive lanes.  The kernel is bound by its
+// arithmetic (exact IEEE steps per element), not by its loads: issuing
+// several chunks' loads ahead (kQuantUnroll > 1) measured slower, as the
+// registers it takes lower the occupancy.
 // ---------------------------------------------------------------------------
-constexpr int kQuantUnroll = 4;
+constexpr int kQuantUnroll = 1;
 
 template <int BITS>
 __device__ __forceinline__ void minmax_quantize_chunk(uint4 raw, int64_t chunk, bool valid, int lane,
