@@ -50,7 +50,8 @@ def parse_args():
     ap.add_argument("--case", default=None,
                     help="run one kernel configuration `reps` times and exit (for ncu captures): "
                          "decode_<matrix>_m<M> | layerset_8b_m<M> | train_<matrix>_{fwd,bwd,grads} | "
-                         "codebook70b_<matrix>_m<M> | quantize_<matrix>")
+                         "codebook70b_<matrix>_m<M> | quantize_<matrix>_{int4,codebook} | merge_<matrix>_r16 | "
+                         "select_<matrix>_q")
     ap.add_argument("--reps", type=int, default=3)
     return ap.parse_args()
 
@@ -596,9 +597,20 @@ def row_mixed(lbq, syn, torch, peaks, stream):
             if rc != 0:
                 raise RuntimeError(f"lbq_linear_fwd_grouped returned {rc}")
 
+        # channel-mix: the seven layers' halves in one grouped call (two
+        # launches of the decode GEMV at M = 16; one GEMM per half at M = 512)
+        mprobs = (lbq.lbq_mix_problem * len(shapes))()
+        for i, (nm, (n, k)) in enumerate(shapes.items()):
+            mprobs[i] = lbq.lbq_mix_problem(X=Xs[k].data_ptr(), q=ctypes.pointer(mixw[nm].struct), A=None, B=None,
+                                            rank=0, s=0.0, Y=Ys[nm].data_ptr(), T_save=None)
+        mws_bytes = lbq.lbq_linear_fwd_mix_grouped_workspace_size(m, mprobs, len(shapes))
+        mws = lbq._workspace(mws_bytes, "cuda")
+
         def channel_mix_step():
-            for nm, (n, k) in shapes.items():
-                lbq.linear_fwd(Xs[k], mixw[nm], Y=Ys[nm], stream=stream)
+            rc = lbq.lbq_linear_fwd_mix_grouped(m, mprobs, len(shapes), None if mws is None else mws.data_ptr(),
+                                                mws_bytes, stream.cuda_stream)
+            if rc != 0:
+                raise RuntimeError(f"lbq_linear_fwd_mix_grouped returned {rc}")
         for label, step, bytes_of in (
                 ("layer_mix", layer_mix_step,
                  lambda nm, n, k: gemm_bytes(m, n, k, bits=bits[nm], group=128 if bits[nm] == 4 else 64)),
@@ -822,6 +834,20 @@ def run_case(args):
         m = int(arg[1:])
         X = syn.normal_bf16((m, k), 1.0, seed=2, device="cuda")
         fn = lambda: lbq.linear_fwd(X, qw)
+    elif kind == "merge":
+        # merging a rank-16 adapter into one 8B matrix (INT4 g128 -> bf16)
+        n, k = syn.LLAMA3_8B_SHAPES[name]
+        W = syn.weight_bf16(n, k, 0.02, seed=1, device="cuda")
+        qw = lbq.QuantizedWeight(n, k, "minmax", 4).quantize(W)
+        A = syn.normal_bf16((16, k), 0.01, seed=3, device="cuda")
+        B = syn.normal_bf16((n, 16), 0.01, seed=4, device="cuda")
+        fn = lambda: lbq.merge_lora(qw, A, B, 2.0, out=W)
+    elif kind == "select":
+        # choosing the INT4 quarter of one 8B matrix's channels (128 calibration tokens)
+        n, k = syn.LLAMA3_8B_SHAPES[name]
+        W = syn.weight_bf16(n, k, 0.02, seed=1, device="cuda")
+        Xc = syn.normal_bf16((128, k), 1.0, seed=2, device="cuda")
+        fn = lambda: lbq.channel_mix_select(W, Xc, n // 4)
     elif kind == "quantize":
         n, k = (syn.LLAMA3_8B_SHAPES.get(name) or syn.LLAMA3_70B_SHAPES[name])
         W = syn.weight_bf16(n, k, 0.02, seed=1, device="cuda")

@@ -313,6 +313,39 @@ lbq_status lbq_linear_fwd_mix(const void* X, int m, const lbq_qweight_mix* q,
                               size_t workspace_bytes, lbq_stream_t stream);
 
 /*
+ * Several channel-mix forwards with the same token count m in one call (the
+ * layers of a channel-mix model at decode time; GreenBit.AI article, 模型量化
+ * (1): a bit width per output channel).  Each problem is one
+ * lbq_linear_fwd_mix with its own activations, channel-mix weight (`q` is a
+ * host pointer to the descriptor), adapter and outputs, under the same layout,
+ * rank and alignment rules.  For m <= 16 both halves of every problem run as
+ * decode GEMV launches of up to 8 weights each (after one adapter launch per
+ * problem with rank > 0); for larger m the problems run one after the other
+ * on `stream`.  The workspace (lbq_linear_fwd_mix_grouped_workspace_size
+ * bytes, zero-filled before its first use, same reuse rules as
+ * lbq_linear_fwd's) serves all of them.  Each Y_i is within the forward's
+ * stated bound, in the original channel order, and deterministic.
+ * Errors: LBQ_EINVAL (count < 1, m < 1, a NULL pointer, halves that are not
+ * MinMax or differ in k), LBQ_EALIGN, LBQ_EWORKSPACE, as lbq_linear_fwd_mix.
+ */
+typedef struct {
+    const void* X;              /* bf16 [m, k], device */
+    const lbq_qweight_mix* q;   /* host pointer to the channel-mix descriptor */
+    const void* A;              /* bf16 [rank, k], device, or NULL when rank == 0 */
+    const void* B;              /* bf16 [n, rank] by original channel, or NULL */
+    int32_t rank;               /* 0 .. 64 */
+    float s;                    /* adapter scale */
+    float* Y;                   /* fp32 [m, n] in the original channel order, device */
+    float* T_save;              /* fp32 [m, rank], device, or NULL when rank == 0 */
+} lbq_mix_problem;
+
+size_t lbq_linear_fwd_mix_grouped_workspace_size(int m, const lbq_mix_problem* probs,
+                                                 int count);
+lbq_status lbq_linear_fwd_mix_grouped(int m, const lbq_mix_problem* probs, int count,
+                                      void* workspace, size_t workspace_bytes,
+                                      lbq_stream_t stream);
+
+/*
  * Input gradient (QLoRA explainer, QLoRA技术原理: gradients pass through the
  * frozen quantized weight):
  *   U  = dY B  [m, rank]                         (fp32, written to U_save)

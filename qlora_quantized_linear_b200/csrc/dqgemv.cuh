@@ -12,14 +12,16 @@
 //    (in bytes) of the (128-row tile, 64-wide k-block) work of ONE matrix of
 //    the group, contiguous in (tile, k-block) order, so a share may span
 //    several tiles;
-//  * one producer warp fills a ring of stages.  A stage holds one weight box
+//  * one producer lane fills a ring of stages.  A stage holds one weight box
 //    (128 rows x 128 bytes, 128-byte swizzle, by TMA) and the matching
 //    activation slice (a 3-D TMA box of (64 k) x (tokens padded to 8 or 16)
 //    x (k-blocks of the weight box), 128-byte swizzle, rows beyond the real
-//    tokens read as zeros).  The boxes' per-row constants (scale and zero, or
-//    absmax) go to a separate ring with two more slots, which the producer's
-//    32 lanes fill with cp.async two boxes further ahead than the weights, so
-//    that their scattered small reads never hold up a stage;
+//    tokens read as zeros);
+//  * each compute warp copies the per-row constants (scale and zero, or
+//    absmax) of its own rows and its part of the box one box ahead with a few
+//    cp.async into a double buffer of its own: spread over the eight warps
+//    these scattered small reads keep up with the weights, where one producer
+//    warp issuing them all for the CTA held the stages back;
 //  * eight compute warps.  With up to 8 tokens warp w owns 32 rows (two
 //    16-row MMA tiles) and one half of the k-blocks of every box (warps 0-3
 //    the first half, 4-7 the second), so a warp's activation fragments and
@@ -66,8 +68,7 @@ constexpr int kGvThreads = 32 * (kGvComputeWarps + 1);        // + one producer 
 constexpr int kGvMaxProblems = 8;                             // matrices per launch
 constexpr int kGvMaxStages = 4;
 constexpr int kGvWBox = 128 * 128;                            // weight box bytes
-constexpr int kGvConstAhead = 2;                              // constant slots beyond the ring's stages
-constexpr int kGvExtraSmem = (3 * kGvMaxStages + kGvConstAhead) * 8 + 16 + 2 * 256 * 4;   // barriers, flags, tables
+constexpr int kGvExtraSmem = 2 * kGvMaxStages * 8 + 16 + 2 * 256 * 4;   // barriers, flags, codebook tables
 constexpr int kGvXchgBytes = 4 * 32 * 4 * 4;                  // half the warps' 16x8 fp32 tiles (up to 8 tokens)
 
 // One matrix of a grouped launch (everything but its tensor maps).  Each CTA
@@ -104,8 +105,7 @@ struct GvParams {
     int m;                            // tokens, 1..16
     int ws;                           // ring stages (2..4)
     int stage_bytes;                  // a multiple of 1024: weight box, then the activation box
-    int cslot_bytes;                  // one box's constants: [2 arrays][128 rows][cstride]
-    int cstride;                      // bytes per row of one constant array
+    int cstride;                      // bytes per row of one constant array in a warp's buffer
     int w_early;                      // weights and constants may be read before the previous kernel ends
 };
 
@@ -254,23 +254,23 @@ struct GvBoxCursor {
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// The constants of one box (k-blocks [kbs, kbs + nk) of row tile `tile`)
-// into the stage's constant block [2 arrays][128 rows][cstride]: lane l
-// copies rows l, l + 32, l + 64, l + 96, each as the 4-byte words that cover
-// the row's entries (MinMax: scale and zero of the box's groups; codebook:
-// the box's absmax values, or its q8 bytes and s2 values).  A row's entries
-// may start at an odd 2-byte (or 1-byte) position in its first word; the
-// readers account for it.
+// The constants of one box (k-blocks [kbs, kbs + nk) of row tile `tile`) for
+// rows [row0, row0 + nrows) of the tile into a buffer [2 arrays][nrows]
+// [cstride]: lane l copies rows l, l + 32, ..., each as the 4-byte words that
+// cover the row's entries (MinMax: scale and zero of the box's groups;
+// codebook: the box's absmax values, or its q8 bytes and s2 values).  A row's
+// entries may start at an odd 2-byte (or 1-byte) position in its first word;
+// the readers account for it.
 template <int KIND>
-__device__ __forceinline__ void gv_fetch_consts(const GvProblem& P, uint32_t cslot, int cstride, int tile, int kbs,
-                                                int nk, int lane) {
+__device__ __forceinline__ void gv_fetch_consts(const GvProblem& P, uint32_t slot, int cstride, int tile, int kbs,
+                                                int nk, int row0, int nrows, int lane) {
     constexpr int GB = GvKind<KIND>::kGroupBlocks;
-    const uint32_t arr1 = 128u * cstride;                    // second array
+    const uint32_t arr1 = static_cast<uint32_t>(nrows * cstride);   // second array
 #pragma unroll 1
-    for (int r = lane; r < 128; r += 32) {
-        const int64_t grow = static_cast<int64_t>(tile) * 128 + r;
+    for (int r = lane; r < nrows; r += 32) {
+        const int64_t grow = static_cast<int64_t>(tile) * 128 + row0 + r;
         if (grow >= P.n) break;                              // rows ascend with r
-        const uint32_t d = cslot + r * cstride;
+        const uint32_t d = slot + r * cstride;
         if (KIND != kCode4) {
             const int64_t e0 = grow * P.ngroups + kbs / GB;
             const int nw = static_cast<int>(((e0 + (nk + GB - 1) / GB - 1) >> 1) - (e0 >> 1)) + 1;
@@ -294,73 +294,51 @@ __device__ __forceinline__ void gv_fetch_consts(const GvProblem& P, uint32_t csl
     }
 }
 
-// The producer warp: lane 0 issues the TMA copies, every lane the constant
-// copies.  The stage ring runs ws boxes ahead of the compute warps, the
-// constant ring (ws + kGvConstAhead slots, one arrival per lane and box on
-// cfull) kGvConstAhead boxes further.
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// The producer lane issues the TMA copies; the ring runs ws boxes ahead of
+// the compute warps.
 template <int KIND>
 __device__ __forceinline__ void gv_produce(const GvParams& p, const GvProblem& P, const CUtensorMap* tmW,
-                                           const CUtensorMap* tmX, const GvShare& sh, uint8_t* ring, uint8_t* cring,
-                                           uint64_t* full, uint64_t* cfull, uint64_t* empty, volatile int* s_abort,
-                                           int lane) {
+                                           const CUtensorMap* tmX, const GvShare& sh, uint8_t* ring, uint64_t* full,
+                                           uint64_t* empty, volatile int* s_abort) {
     constexpr int SUB = GvKind<KIND>::kSub;
-    const int ws = p.ws, ncs = p.ws + kGvConstAhead;
-    GvBoxCursor cc;                                          // next box whose constants to fetch
-    cc.start(sh, SUB);
-    int cslot = 0;
-    auto consts_next = [&]() {
-        gv_fetch_consts<KIND>(P, smem_u32(cring + cslot * p.cslot_bytes), p.cstride, cc.sg.tile, cc.kbs,
-                              min(SUB, cc.sg.kb - cc.kbs), lane);
-        cp_async_mbar_arrive_noinc(&cfull[cslot]);
-        cc.next();
-        if (++cslot == ncs) cslot = 0;
-    };
+    const int ws = p.ws;
     GvBoxCursor ic;                                          // next box to issue
     ic.start(sh, SUB);
     int nissued = 0;
     if (p.w_early) {
-        // the first boxes' weights and constants before the previous kernel
-        // on the stream has finished; the activations only after it has
+        // the first boxes' weights before the previous kernel on the stream
+        // has finished; the activations only after it has
         GvBoxCursor pre = ic;
         for (int c = 0; pre.valid && c < ws; ++c, pre.next())
-            if (lane == 0) gv_issue_weights<KIND>(tmW, P.xbytes, ring + c * p.stage_bytes, &full[c], pre.sg.tile, pre.kbs);
-        for (int c = 0; cc.valid && c < ncs; ++c) consts_next();
+            gv_issue_weights<KIND>(tmW, P.xbytes, ring + c * p.stage_bytes, &full[c], pre.sg.tile, pre.kbs);
         griddep_wait();
         for (; ic.valid && nissued < ws; ++nissued, ic.next())
-            if (lane == 0) gv_issue_acts(tmX, ring + nissued * p.stage_bytes, &full[nissued], ic.kbs);
+            gv_issue_acts(tmX, ring + nissued * p.stage_bytes, &full[nissued], ic.kbs);
     } else {
         griddep_wait();
         for (; ic.valid && nissued < ws; ++nissued, ic.next()) {
-            if (lane == 0) {
-                gv_issue_weights<KIND>(tmW, P.xbytes, ring + nissued * p.stage_bytes, &full[nissued], ic.sg.tile, ic.kbs);
-                gv_issue_acts(tmX, ring + nissued * p.stage_bytes, &full[nissued], ic.kbs);
-            }
+            gv_issue_weights<KIND>(tmW, P.xbytes, ring + nissued * p.stage_bytes, &full[nissued], ic.sg.tile, ic.kbs);
+            gv_issue_acts(tmX, ring + nissued * p.stage_bytes, &full[nissued], ic.kbs);
         }
-        for (int c = 0; cc.valid && c < ncs; ++c) consts_next();
     }
-    // box j goes into slot j % ws once the compute warps have released box
-    // j - ws, and with it the constants of box j + kGvConstAhead into the
-    // constant slot of box j - ws
+    // box j goes into slot j % ws once the compute warps have released box j - ws
     int slot = 0;
     uint32_t ph = 0;
     for (; ic.valid; ++nissued, ic.next()) {
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[slot], ph, s_abort))) break;
+        if (!mbar_wait(&empty[slot], ph, s_abort)) break;
         uint8_t* stage = ring + slot * p.stage_bytes;
-        if (lane == 0) {
-            gv_issue_weights<KIND>(tmW, P.xbytes, stage, &full[slot], ic.sg.tile, ic.kbs);
-            gv_issue_acts(tmX, stage, &full[slot], ic.kbs);
-        }
-        if (cc.valid) consts_next();
+        gv_issue_weights<KIND>(tmW, P.xbytes, stage, &full[slot], ic.sg.tile, ic.kbs);
+        gv_issue_acts(tmX, stage, &full[slot], ic.kbs);
         if (++slot == ws) {
             slot = 0;
             ph ^= 1u;
         }
     }
     // never leave with a copy in flight (matters only after an abort)
-    cp_async_wait_all();
-    if (lane == 0)
-        for (int i = max(0, nissued - ws); i < nissued; ++i) mbar_wait_drain(&full[i % ws], (i / ws) & 1);
-    __syncwarp();
+    for (int i = max(0, nissued - ws); i < nissued; ++i) mbar_wait_drain(&full[i % ws], (i / ws) & 1);
 }
 
 // ----------------------------------------------------------------------------
@@ -376,8 +354,8 @@ __device__ __forceinline__ uint32_t gv_exact_pair(uint32_t v, float zf, float sf
 
 template <int KIND, int NT8>
 __device__ __forceinline__ void gv_compute(const GvParams& p, const GvProblem& P, const GvShare& sh, int b,
-                                           uint8_t* ring, uint8_t* cring, uint64_t* full, uint64_t* cfull,
-                                           uint64_t* empty, volatile int* s_abort, float* xchg, const uint32_t* s_lut,
+                                           uint8_t* ring, uint8_t* cbuf, uint64_t* full, uint64_t* empty,
+                                           volatile int* s_abort, float* xchg, const uint32_t* s_lut,
                                            const float* s_q8lut) {
     using G = GvKind<KIND>;
     constexpr int SUB = G::kSub, RB = G::kRowBytes, GB = G::kGroupBlocks;
@@ -427,16 +405,32 @@ __device__ __forceinline__ void gv_compute(const GvParams& p, const GvProblem& P
     uint32_t mg = 0x43004300u;                               // bf16x2 (128, 128), kept in a register
     asm volatile("" : "+r"(mg));
     const uint32_t cstride = static_cast<uint32_t>(p.cstride);
-    const uint32_t arr1 = 128u * cstride;
-    // nothing global is written before the previous kernel on the stream has finished
-    griddep_wait();
+    // this warp's constant double buffer: [slot][2 arrays][its rows][cstride]
+    constexpr int NRW = 16 * TILES;                    // the warp's rows
+    const int row0 = (warp % WPK) * NRW;
+    const uint32_t arr1 = NRW * cstride;
+    const uint32_t cslot_bytes = 2 * NRW * cstride;
+    const uint32_t cslot0 = smem_u32(cbuf) + warp * 2 * cslot_bytes;
+    // the constants of the warp's part of a box (k-blocks [kbs + kh HALF,
+    // kbs + min(nk, (kh + 1) HALF))), for its own rows
+    auto fetch_part = [&](uint32_t slot, int tile, int kbs, int nk) {
+        const int lo = kh * HALF;
+        if (lo < nk) gv_fetch_consts<KIND>(P, slot, p.cstride, tile, kbs + lo, min(nk, lo + HALF) - lo, row0, NRW, lane);
+    };
+    // the first box's constants; nothing global is written before the
+    // previous kernel on the stream has finished
+    {
+        const GvSeg s0 = gv_segment(sh, 0);
+        if (!p.w_early) griddep_wait();
+        fetch_part(cslot0, s0.tile, s0.ka, min(SUB, s0.kb - s0.ka));
+        cp_async_commit();
+        if (p.w_early) griddep_wait();
+    }
 
     bool live = true;                                        // false after a timed-out wait
     int w = 0;                                               // ring slot of the box (matches the producer)
     uint32_t ph = 0;                                         // ... and its phase parity
-    int cw = 0;                                              // constant slot of the box
-    uint32_t cph = 0;                                        // ... and its phase parity
-    const int ncs = p.ws + kGvConstAhead;
+    uint32_t cbit = 0;                                       // constant slot of the box
     // (after a timed-out wait every warp still runs every segment's barriers)
     for (int si = 0; si < sh.nseg; ++si) {
         const GvSeg sg = gv_segment(sh, si);
@@ -449,17 +443,28 @@ __device__ __forceinline__ void gv_compute(const GvParams& p, const GvProblem& P
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[t2][nt][e] = 0.0f;
         for (int kbs = sg.ka; kbs < sg.kb; kbs += SUB) {
+            // the next box's constants into the other slot
+            if (kbs + SUB < sg.kb) {
+                fetch_part(cslot0 + (cbit ^ 1u) * cslot_bytes, tile, kbs + SUB, min(SUB, sg.kb - kbs - SUB));
+            } else if (si + 1 < sh.nseg) {
+                const GvSeg sn = gv_segment(sh, si + 1);
+                fetch_part(cslot0 + (cbit ^ 1u) * cslot_bytes, sn.tile, sn.ka, min(SUB, sn.kb - sn.ka));
+            }
+            cp_async_commit();
+            cp_async_wait_1();                               // this box's constants (this lane's copies)
+            __syncwarp();                                    // ... and the other lanes'
             // warp-uniform: the warp's later shuffles and MMAs need all 32 lanes
-            const bool got = live && mbar_wait(&cfull[cw], cph, s_abort) && mbar_wait(&full[w], ph, s_abort);
+            const bool got = live && mbar_wait(&full[w], ph, s_abort);
             live = __all_sync(0xFFFFFFFFu, got);
             const int nk = min(SUB, sg.kb - kbs);
             if (live && kh * HALF < nk) {
                 const uint32_t stage = smem_u32(ring + w * p.stage_bytes);
-                const uint32_t crow = smem_u32(cring + cw * p.cslot_bytes) + rq * cstride;   // row rq, array 0
+                const uint32_t crow = cslot0 + cbit * cslot_bytes + (rq - row0) * cstride;   // row rq, array 0
                 // entry parity of the rows' first constant word (MinMax): the
                 // parity of row * groups + first group (the four rows have the
                 // parity of rq, as a tile starts on an even row)
-                const int par = ((rq & P.ngroups) + kbs / GB) & 1;
+                const int s_lo = kh * HALF;                  // the warp's first k-block of the box
+                const int par = ((rq & P.ngroups) + (kbs + s_lo) / GB) & 1;
                 float sf[NR], zf[NR];
 #pragma unroll
                 for (int i = 0; i < NR; ++i) {
@@ -475,7 +480,7 @@ __device__ __forceinline__ void gv_compute(const GvParams& p, const GvProblem& P
                         if (s % GB == 0) {
                             // the group's (or k-block's) constants of the thread's rows
                             if (KIND != kCode4) {
-                                const uint32_t ce = crow + 2 * (s / GB + par);
+                                const uint32_t ce = crow + 2 * ((s - s_lo) / GB + par);
 #pragma unroll
                                 for (int i = 0; i < NR; ++i) {
                                     sf[i] = f16_bits_to_f32(gv_lds16(ce + 8 * i * cstride));
@@ -492,17 +497,18 @@ __device__ __forceinline__ void gv_compute(const GvParams& p, const GvProblem& P
                                 }
                             } else if (P.q8 == nullptr) {
 #pragma unroll
-                                for (int i = 0; i < NR; ++i) sf[i] = __uint_as_float(gv_lds32(crow + 8 * i * cstride + 4 * s));
+                                for (int i = 0; i < NR; ++i)
+                                    sf[i] = __uint_as_float(gv_lds32(crow + 8 * i * cstride + 4 * (s - s_lo)));
                             } else {
                                 // absmax' = fp32(fp32(q8 / 127) * s2) + offset
 #pragma unroll
                                 for (int i = 0; i < NR; ++i) {
-                                    const int64_t e0 = (static_cast<int64_t>(tile) * 128 + rq + 8 * i) * P.kbt + kbs;
-                                    const int ia = static_cast<int>((e0 & 3) + s);
+                                    const int64_t e0 = (static_cast<int64_t>(tile) * 128 + rq + 8 * i) * P.kbt + kbs + s_lo;
+                                    const int ia = static_cast<int>((e0 & 3) + (s - s_lo));
                                     const uint32_t qa = gv_lds32(crow + 8 * i * cstride + (ia & ~3));
                                     const uint32_t q8 = (qa >> (8 * (ia & 3))) & 0xFFu;
                                     const float s2 = __uint_as_float(
-                                        gv_lds32(crow + 8 * i * cstride + arr1 + (((e0 + s) >> 8) != (e0 >> 8) ? 4 : 0)));
+                                        gv_lds32(crow + 8 * i * cstride + arr1 + (((e0 + s - s_lo) >> 8) != (e0 >> 8) ? 4 : 0)));
                                     sf[i] = __fadd_rn(__fmul_rn(s_q8lut[q8], s2), dq_off);
                                 }
                             }
@@ -647,10 +653,7 @@ __device__ __forceinline__ void gv_compute(const GvParams& p, const GvProblem& P
                 w = 0;
                 ph ^= 1u;
             }
-            if (++cw == ncs) {
-                cw = 0;
-                cph ^= 1u;
-            }
+            cbit ^= 1u;
         }
         // -------------------------------------------------------------- segment epilogue
         // With two k-parts: warps 0-3 finish tile 0 of their 32 rows, warps
@@ -785,6 +788,7 @@ __device__ __forceinline__ void gv_compute(const GvParams& p, const GvProblem& P
                 }
             }
     }
+    cp_async_wait_all();                                     // no copy into the buffer outlives the CTA
 }
 
 template <int NT8>
@@ -813,11 +817,10 @@ __global__ void __launch_bounds__(kGvThreads, 2) dqgemv_grouped_kernel(const __g
     // 1024-byte alignment for the swizzled boxes, by pointer arithmetic on the
     // shared array so that every access below stays a shared-memory access
     uint8_t* ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint8_t* cring = ring + p.ws * p.stage_bytes;                              // [ws + 2][2][128][cstride]
-    float* xchg = reinterpret_cast<float*>(cring + (p.ws + kGvConstAhead) * p.cslot_bytes);   // [4][4][32] (8 tokens)
+    uint8_t* cbuf = ring + p.ws * p.stage_bytes;                               // [warp][2][2][rows][cstride]
+    float* xchg = reinterpret_cast<float*>(cbuf + kGvComputeWarps * 2 * 2 * (16 * (3 - NT8)) * p.cstride);   // [4][4][32]
     uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(xchg) + (NT8 == 1 ? kGvXchgBytes : 0));
-    uint64_t* cfull = full + kGvMaxStages;
-    uint64_t* empty = cfull + kGvMaxStages + kGvConstAhead;
+    uint64_t* empty = full + kGvMaxStages;
     volatile int* s_abort = reinterpret_cast<volatile int*>(empty + kGvMaxStages);
     uint32_t* s_lut = reinterpret_cast<uint32_t*>(empty + kGvMaxStages) + 4;   // codebook pairs [256]
     float* s_q8lut = reinterpret_cast<float*>(s_lut + 256);                  // q8 / 127 [256]
@@ -838,8 +841,6 @@ __global__ void __launch_bounds__(kGvThreads, 2) dqgemv_grouped_kernel(const __g
             mbar_init(&full[i], 1);                      // the producer's TMA arrival + the boxes' bytes
             mbar_init(&empty[i], kGvComputeWarps);
         }
-        for (int i = 0; i < p.ws + kGvConstAhead; ++i)
-            mbar_init(&cfull[i], 32);                    // one per producer lane once its copies have landed
         *s_abort = 0;
         fence_mbar_init();
     }
@@ -855,10 +856,11 @@ __global__ void __launch_bounds__(kGvThreads, 2) dqgemv_grouped_kernel(const __g
 
     auto run = [&](auto kind_tag) {
         constexpr int KIND = decltype(kind_tag)::value;
-        if (warp == kGvComputeWarps)
-            gv_produce<KIND>(p, P, &p.tmW[pi], &p.tmX[pi], sh, ring, cring, full, cfull, empty, s_abort, lane);
-        else
-            gv_compute<KIND, NT8>(p, P, sh, b, ring, cring, full, cfull, empty, s_abort, xchg, s_lut, s_q8lut);
+        if (warp == kGvComputeWarps) {
+            if (lane == 0) gv_produce<KIND>(p, P, &p.tmW[pi], &p.tmX[pi], sh, ring, full, empty, s_abort);
+        } else {
+            gv_compute<KIND, NT8>(p, P, sh, b, ring, cbuf, full, empty, s_abort, xchg, s_lut, s_q8lut);
+        }
     };
     if (P.kind == kInt4)
         run(std::integral_constant<int, kInt4>{});

@@ -27,7 +27,7 @@ struct GvPlan {
     int count = 0;
     int ctas = 0;                   // grid
     int ws = 0;                     // ring stages
-    int stage_bytes = 0, xbox_max = 0, cslot_bytes = 0, cstride = 0;
+    int stage_bytes = 0, xbox_max = 0, cstride = 0;
     size_t smem = 0;                // dynamic shared memory per CTA
     size_t workspace = 0;           // 0 when no tile is split
     int share[kGvMaxProblems] = {}, pctas[kGvMaxProblems] = {}, cta0[kGvMaxProblems] = {};
@@ -44,14 +44,16 @@ double gv_unit_bytes(const lbq_qweight* q) {
     return codes + 128.0 * (q->double_quant ? 1 : 4);
 }
 
-// Bytes per row of one constant array that a weight box needs: the 4-byte
-// words covering its groups (MinMax: 2 groups for INT4, 8 for INT2, starting
-// at any entry), 4 absmax values, or 2 words of q8 (and of s2 in the second
-// array).
-int gv_const_stride(const lbq_qweight* q) {
-    if (q->scheme == LBQ_CODEBOOK4) return q->double_quant ? 8 : 16;
-    const int gpb = q->bits == 2 ? 8 : 2;                               // groups per box
-    return 4 * (gpb / 2 + 1);
+// Bytes per row of one constant array that a compute warp's part of a weight
+// box needs (half the box's k-blocks with up to 8 tokens, all of them with
+// more): the 4-byte words covering its groups (MinMax, starting at any
+// entry), its absmax values, or 2 words of q8 (and of s2 in the second array).
+int gv_const_stride(const lbq_qweight* q, int m) {
+    const int parts = m <= 8 ? 2 : 1;
+    const int kpp = (q->scheme == LBQ_MINMAX_ASYM && q->bits == 2 ? 8 : 4) / parts;   // k-blocks per part
+    if (q->scheme == LBQ_CODEBOOK4) return q->double_quant ? 8 : 4 * kpp;
+    const int gpp = q->bits == 2 ? kpp : kpp / 2;                                    // groups per part
+    return 4 * (gpp / 2 + 1);
 }
 
 // Token rows of an activation box: the real ones padded to the MMA's token
@@ -72,27 +74,27 @@ lbq_status gv_plan(int m, const lbq_qweight* const* qs, int count, int sms, GvPl
         if (tiles * kbt >= (int64_t(1) << 31)) return LBQ_EUNSUPPORTED;
         any_int2 |= (q->scheme == LBQ_MINMAX_ASYM && q->bits == 2);
         any_code |= q->scheme == LBQ_CODEBOOK4;
-        cstride = std::max(cstride, gv_const_stride(q));
+        cstride = std::max(cstride, gv_const_stride(q, m));
         total_bytes += gv_unit_bytes(q) * static_cast<double>(tiles * kbt);
         pl->tiles[i] = static_cast<int>(tiles);
         pl->cnt_off[i] = tiles_sum;
         tiles_sum += static_cast<int>(tiles);
     }
     if (tiles_sum > kMaxSplitTiles) return LBQ_EUNSUPPORTED;
-    // stage layout: weight box, activation box; after the ring the constant
-    // ring (ws + kGvConstAhead slots of [2 arrays][128 rows][cstride]) and the
-    // buffer in which the compute warps add the two k-halves of their rows
+    // stage layout: weight box, activation box; after the ring each compute
+    // warp's constant double buffer ([2 slots][2 arrays][its 32 or 16 rows]
+    // [cstride]) and the buffer in which the compute warps add the two
+    // k-halves of their rows
     const int sub_max = any_int2 ? 8 : 4;
     pl->xbox_max = sub_max * gv_mpad(m) * 128;
     pl->cstride = cstride;
-    pl->cslot_bytes = 256 * cstride;
     pl->stage_bytes = kGvWBox + pl->xbox_max;
+    const size_t cbuf = static_cast<size_t>(kGvComputeWarps) * 2 * 2 * (m <= 8 ? 32 : 16) * cstride;
     const size_t xchg = m <= 8 ? kGvXchgBytes : 0;
     (void)any_code;
     pl->ws = 0;
     for (int ws = kGvMaxStages; ws >= 2; --ws) {
-        const size_t smem = 1024 + static_cast<size_t>(ws) * pl->stage_bytes +
-                            static_cast<size_t>(ws + kGvConstAhead) * pl->cslot_bytes + xchg + kGvExtraSmem;
+        const size_t smem = 1024 + static_cast<size_t>(ws) * pl->stage_bytes + cbuf + xchg + kGvExtraSmem;
         if (smem <= kGemvSmemBudget) {
             pl->ws = ws;
             pl->smem = smem;
@@ -166,7 +168,6 @@ lbq_status run_gemv_group(int m, const GvJob* jobs, int count, void* ws, size_t 
     prm.m = m;
     prm.ws = pl.ws;
     prm.stage_bytes = pl.stage_bytes;
-    prm.cslot_bytes = pl.cslot_bytes;
     prm.cstride = pl.cstride;
     prm.w_early = weights_stable(st) ? 1 : 0;
     for (int i = 0; i < count; ++i) {

@@ -415,6 +415,31 @@ lbq_status launch_lora_colgrad(const void* in, int64_t m, int64_t ncols, const f
     return last_launch();
 }
 
+namespace {
+
+// The workspace of a channel-mix forward (both halves).
+size_t mix_workspace(int m, const lbq_qweight_mix* q, int sms) {
+    if (m <= kGemvMaxM) {
+        const lbq_qweight* qs[2] = {&q->hi, &q->lo};
+        return gemv_jobs_workspace(m, qs, 2, sms);
+    }
+    return std::max(plan_fwd(m, &q->hi, sms).workspace(), plan_fwd(m, &q->lo, sms).workspace());
+}
+
+// Validation of one channel-mix problem's descriptor, activations and outputs.
+lbq_status check_mix(const lbq_qweight_mix* q, int m, const void* X, const float* Y) {
+    if (!q || !q->perm) return LBQ_EINVAL;
+    lbq_status st;
+    if ((st = check_qweight(&q->hi, true)) != LBQ_OK) return st;
+    if ((st = check_qweight(&q->lo, true)) != LBQ_OK) return st;
+    if (q->hi.scheme != LBQ_MINMAX_ASYM || q->lo.scheme != LBQ_MINMAX_ASYM || q->hi.k != q->lo.k) return LBQ_EINVAL;
+    if (m < 1 || !X || !Y) return LBQ_EINVAL;
+    if (!aligned16(X) || !aligned16(Y) || !aligned16(q->perm)) return LBQ_EALIGN;
+    return LBQ_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* lbq_status_string(lbq_status s) {
@@ -691,14 +716,6 @@ lbq_status lbq_linear_fwd_grouped(int m, const lbq_fwd_problem* probs, int count
 
 // Channel-mix: the two halves in one grouped launch (m <= 16) or one GEMM
 // each (m > 16), writing their rows' output columns through perm.
-size_t mix_workspace(int m, const lbq_qweight_mix* q, int sms) {
-    if (m <= kGemvMaxM) {
-        const lbq_qweight* qs[2] = {&q->hi, &q->lo};
-        return gemv_jobs_workspace(m, qs, 2, sms);
-    }
-    return std::max(plan_fwd(m, &q->hi, sms).workspace(), plan_fwd(m, &q->lo, sms).workspace());
-}
-
 size_t lbq_linear_fwd_mix_workspace_size(int m, const lbq_qweight_mix* q, int rank) {
     (void)rank;
     if (!q || m < 1) return 0;
@@ -709,14 +726,8 @@ size_t lbq_linear_fwd_mix_workspace_size(int m, const lbq_qweight_mix* q, int ra
 lbq_status lbq_linear_fwd_mix(const void* X, int m, const lbq_qweight_mix* q, const void* A, const void* B, int rank,
                               float s, float* Y, float* T_save, void* workspace, size_t workspace_bytes,
                               lbq_stream_t stream) {
-    if (!q || !q->perm) return LBQ_EINVAL;
     lbq_status st;
-    if ((st = check_qweight(&q->hi, true)) != LBQ_OK) return st;
-    if ((st = check_qweight(&q->lo, true)) != LBQ_OK) return st;
-    if (q->hi.scheme != LBQ_MINMAX_ASYM || q->lo.scheme != LBQ_MINMAX_ASYM || q->hi.k != q->lo.k)
-        return LBQ_EINVAL;
-    if (m < 1 || !X || !Y) return LBQ_EINVAL;
-    if (!aligned16(X) || !aligned16(Y) || !aligned16(q->perm)) return LBQ_EALIGN;
+    if ((st = check_mix(q, m, X, Y)) != LBQ_OK) return st;
     if ((st = check_lora(rank, A, B, T_save)) != LBQ_OK) return st;
     const int sms = sm_count();
     const size_t need = mix_workspace(m, q, sms);
@@ -737,6 +748,70 @@ lbq_status lbq_linear_fwd_mix(const void* X, int m, const lbq_qweight_mix* q, co
         return st;
     return run_fwd_gemm(X, m, &q->lo, B, rank, s, T_save, Y, n_total, q->perm + q->hi.n, workspace, workspace_bytes,
                         sms, cs);
+}
+
+size_t lbq_linear_fwd_mix_grouped_workspace_size(int m, const lbq_mix_problem* probs, int count) {
+    if (m < 1 || !probs || count < 1) return 0;
+    const int sms = sm_count();
+    if (m <= kGemvMaxM) {
+        std::vector<const lbq_qweight*> qs;
+        for (int i = 0; i < count; ++i) {
+            const lbq_qweight_mix* q = probs[i].q;
+            if (!q || check_qweight(&q->hi, false) != LBQ_OK || check_qweight(&q->lo, false) != LBQ_OK) return 0;
+            qs.push_back(&q->hi);
+            qs.push_back(&q->lo);
+        }
+        return gemv_jobs_workspace(m, qs.data(), static_cast<int>(qs.size()), sms);
+    }
+    size_t need = 0;
+    for (int i = 0; i < count; ++i) {
+        const lbq_qweight_mix* q = probs[i].q;
+        if (!q || check_qweight(&q->hi, false) != LBQ_OK || check_qweight(&q->lo, false) != LBQ_OK) return 0;
+        need = std::max(need, mix_workspace(m, q, sms));
+    }
+    return need;
+}
+
+lbq_status lbq_linear_fwd_mix_grouped(int m, const lbq_mix_problem* probs, int count, void* workspace,
+                                      size_t workspace_bytes, lbq_stream_t stream) {
+    if (m < 1 || !probs || count < 1) return LBQ_EINVAL;
+    lbq_status st;
+    for (int i = 0; i < count; ++i) {
+        const lbq_mix_problem& pr = probs[i];
+        if ((st = check_mix(pr.q, m, pr.X, pr.Y)) != LBQ_OK) return st;
+        if ((st = check_lora(pr.rank, pr.A, pr.B, pr.T_save)) != LBQ_OK) return st;
+    }
+    const size_t need = lbq_linear_fwd_mix_grouped_workspace_size(m, probs, count);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return LBQ_EWORKSPACE;
+    if (need > 0 && !aligned16(workspace)) return LBQ_EALIGN;
+    const int sms = sm_count();
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    for (int i = 0; i < count; ++i) {
+        const lbq_mix_problem& pr = probs[i];
+        if (pr.rank > 0 && (st = launch_lora_rows<false>(pr.X, m, pr.q->hi.k, pr.A, pr.rank, pr.T_save, cs)) != LBQ_OK)
+            return st;
+    }
+    if (m > kGemvMaxM) {
+        for (int i = 0; i < count; ++i) {
+            const lbq_mix_problem& pr = probs[i];
+            const int64_t n_total = static_cast<int64_t>(pr.q->hi.n) + pr.q->lo.n;
+            if ((st = run_fwd_gemm(pr.X, m, &pr.q->hi, pr.B, pr.rank, pr.s, pr.T_save, pr.Y, n_total, pr.q->perm,
+                                   workspace, workspace_bytes, sms, cs)) != LBQ_OK)
+                return st;
+            if ((st = run_fwd_gemm(pr.X, m, &pr.q->lo, pr.B, pr.rank, pr.s, pr.T_save, pr.Y, n_total,
+                                   pr.q->perm + pr.q->hi.n, workspace, workspace_bytes, sms, cs)) != LBQ_OK)
+                return st;
+        }
+        return LBQ_OK;
+    }
+    std::vector<GvJob> jobs;
+    for (int i = 0; i < count; ++i) {
+        const lbq_mix_problem& pr = probs[i];
+        const int64_t n_total = static_cast<int64_t>(pr.q->hi.n) + pr.q->lo.n;
+        jobs.push_back(GvJob{pr.X, &pr.q->hi, pr.B, pr.rank, pr.s, pr.T_save, pr.Y, n_total, pr.q->perm});
+        jobs.push_back(GvJob{pr.X, &pr.q->lo, pr.B, pr.rank, pr.s, pr.T_save, pr.Y, n_total, pr.q->perm + pr.q->hi.n});
+    }
+    return run_gemv_jobs(m, jobs.data(), static_cast<int>(jobs.size()), workspace, workspace_bytes, sms, cs);
 }
 
 size_t lbq_linear_bwd_workspace_size(int m, const lbq_qweight* q, int rank) {

@@ -53,9 +53,16 @@ class lbq_fwd_problem(ctypes.Structure):
                 ("Y", ctypes.c_void_p), ("T_save", ctypes.c_void_p)]
 
 
+class lbq_mix_problem(ctypes.Structure):
+    _fields_ = [("X", ctypes.c_void_p), ("q", ctypes.POINTER(lbq_qweight_mix)), ("A", ctypes.c_void_p),
+                ("B", ctypes.c_void_p), ("rank", ctypes.c_int32), ("s", ctypes.c_float),
+                ("Y", ctypes.c_void_p), ("T_save", ctypes.c_void_p)]
+
+
 _vp, _int, _f32, _sz, _u32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.POINTER(ctypes.c_uint32)
 _QP, _MP = ctypes.POINTER(lbq_qweight), ctypes.POINTER(lbq_qweight_mix)
 _PP, _QPP, _I64P = ctypes.POINTER(lbq_fwd_problem), ctypes.POINTER(ctypes.POINTER(lbq_qweight)), ctypes.POINTER(ctypes.c_int64)
+_MPP = ctypes.POINTER(lbq_mix_problem)
 _SIGS = {
     "lbq_status_string": (ctypes.c_char_p, [_int]),
     "lbq_quantize_workspace_size": (_sz, [_QP]),
@@ -80,6 +87,8 @@ _SIGS = {
     "lbq_channel_mix_select": (_int, [_vp, _int, _int, _vp, _int, _int, _vp, _vp, _vp, _sz, _vp]),
     "lbq_gather_rows": (_int, [_vp, _int, _int, _vp, _int, _vp, _vp]),
     "lbq_selftest_wait_timeout": (_int, [ctypes.c_uint32, _vp]),
+    "lbq_linear_fwd_mix_grouped_workspace_size": (_sz, [_int, _MPP, _int]),
+    "lbq_linear_fwd_mix_grouped": (_int, [_int, _MPP, _int, _vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_L, _name)
@@ -116,6 +125,8 @@ lbq_channel_mix_select_workspace_size = _L.lbq_channel_mix_select_workspace_size
 lbq_channel_mix_select = _L.lbq_channel_mix_select
 lbq_gather_rows = _L.lbq_gather_rows
 lbq_selftest_wait_timeout = _L.lbq_selftest_wait_timeout
+lbq_linear_fwd_mix_grouped_workspace_size = _L.lbq_linear_fwd_mix_grouped_workspace_size
+lbq_linear_fwd_mix_grouped = _L.lbq_linear_fwd_mix_grouped
 
 
 class LbqError(RuntimeError):
@@ -319,6 +330,35 @@ def linear_fwd_grouped(problems, workspace=None, stream=None):
         workspace = _workspace(nws, problems[0][0].device)
     _check(lbq_linear_fwd_grouped(m, arr, len(problems), _ptr(workspace), nws, _stream(stream)),
            "lbq_linear_fwd_grouped")
+    return outs
+
+
+def linear_fwd_mix_grouped(problems, workspace=None, stream=None):
+    """Several channel-mix forwards with the same token count in one call.
+    `problems` is a list of (X, ChannelMixWeight) or (X, ChannelMixWeight, A,
+    B, s) tuples; returns the list of (Y, T) as linear_fwd would."""
+    torch = _torch()
+    arr = (lbq_mix_problem * len(problems))()
+    outs, keep = [], []
+    m = None
+    for i, pr in enumerate(problems):
+        X, mw = _bf16_2d(pr[0], "X"), pr[1]
+        A, B, s = (pr[2], pr[3], pr[4]) if len(pr) > 2 else (None, None, 0.0)
+        m = X.shape[0] if m is None else m
+        if X.shape[0] != m:
+            raise ValueError("all problems of a grouped call have the same token count")
+        rank = 0 if A is None else int(A.shape[0])
+        Y = torch.empty((m, mw.n), dtype=torch.float32, device=X.device)
+        T = torch.empty((m, rank), dtype=torch.float32, device=X.device) if rank else None
+        arr[i] = lbq_mix_problem(X=X.data_ptr(), q=ctypes.pointer(mw.struct), A=_ptr(A), B=_ptr(B), rank=rank,
+                                 s=float(s), Y=Y.data_ptr(), T_save=_ptr(T))
+        outs.append((Y, T))
+        keep.append((X, A, B))
+    nws = lbq_linear_fwd_mix_grouped_workspace_size(m, arr, len(problems))
+    if workspace is None:
+        workspace = _workspace(nws, problems[0][0].device)
+    _check(lbq_linear_fwd_mix_grouped(m, arr, len(problems), _ptr(workspace), nws, _stream(stream)),
+           "lbq_linear_fwd_mix_grouped")
     return outs
 
 

@@ -8,8 +8,8 @@ last tile first, then the whole tiles, then the first tile) and check what
 the kernel relies on:
 
 * the launch is one wave of two CTAs per SM, and its shared memory (ring of
-  stages, each a weight box and an activation box, the constant ring and the
-  fixed tail) fits two CTAs per SM;
+  stages, each a weight box and an activation box, the compute warps'
+  constant buffers and the fixed tail) fits two CTAs per SM;
 * every unit of every weight is covered exactly once, and CTAs of one weight
   are contiguous in the grid;
 * a split tile is finished by the CTA that covers its last k-block, which is
@@ -30,7 +30,7 @@ from qlora_quantized_linear_b200 import lbq
 
 SMS = 148
 BUDGET = 115712 - 1024           # dynamic shared memory per CTA at two CTAs per SM (beside 1 KB static)
-EXTRA = (3 * 4 + 2) * 8 + 16 + 2 * 256 * 4
+EXTRA = 2 * 4 * 8 + 16 + 2 * 256 * 4
 XCHG = 4 * 32 * 4 * 4                 # the two k-halves' exchange buffer (up to 8 tokens)
 HEADER = 64 * 1024
 SHAPES_8B = [(4096, 4096), (1024, 4096), (1024, 4096), (4096, 4096), (14336, 4096), (14336, 4096), (4096, 14336)]
@@ -91,14 +91,14 @@ def check(m, qs):
     assert 2 <= P["ws"] <= 4
     assert P["stage"] % 1024 == 0
     # stage: weight box, activation box (k-blocks of the box x tokens padded to
-    # the MMA's 8 or 16 x 128 bytes); then a constant ring of ws + 2 slots
-    # (2 arrays x 128 rows each)
+    # the MMA's 8 or 16 x 128 bytes); then every compute warp's constant
+    # double buffer (2 slots x 2 arrays x its 32 or 16 rows)
     sub_max = max(pr["sub"] for pr in P["probs"])
     mpad = 8 if m <= 8 else 16
     assert P["xbox"] == sub_max * mpad * 128 and P["stage"] == 16384 + P["xbox"]
     xchg = XCHG if m <= 8 else 0
-    cring = (P["ws"] + 2) * 256 * P["cstride"]
-    assert P["smem"] == 1024 + P["ws"] * P["stage"] + cring + xchg + EXTRA and P["smem"] <= BUDGET
+    cbuf = 8 * 2 * 2 * (32 if m <= 8 else 16) * P["cstride"]
+    assert P["smem"] == 1024 + P["ws"] * P["stage"] + cbuf + xchg + EXTRA and P["smem"] <= BUDGET
     cta = 0
     any_split = False
     part_total = 0
@@ -120,15 +120,23 @@ def check(m, qs):
             for i, (t, ka, kb) in enumerate(segs):
                 assert 0 <= t < tiles and 0 <= ka < kb <= kbt
                 assert ka % gb == 0 and kb % gb == 0              # whole scale groups
+                parts = 2 if m <= 8 else 1                        # a compute warp's share of a box
+                half = pr["sub"] // parts
                 for kbs in range(ka, kb, pr["sub"]):
                     nk = min(pr["sub"], kb - kbs)
                     assert kbs % gb == 0 and nk >= 1
-                    # constant words a box needs, for the worst row parity
-                    if pr["kind"] != 2:
-                        ng = -(-nk // gb)
-                        assert 4 * (ng // 2 + 1) <= P["cstride"]
-                    else:
-                        assert 4 * nk <= P["cstride"] or (pr["dq"] and 8 <= P["cstride"])
+                    for part in range(parts):
+                        lo = part * half
+                        if lo >= nk:
+                            continue
+                        nkp = min(nk, lo + half) - lo
+                        assert (kbs + lo) % gb == 0                   # a part starts on a whole group
+                        # constant words the part needs, for the worst row parity
+                        if pr["kind"] != 2:
+                            ng = -(-nkp // gb)
+                            assert 4 * (ng // 2 + 1) <= P["cstride"]
+                        else:
+                            assert 4 * nkp <= P["cstride"] or (pr["dq"] and 8 <= P["cstride"])
                 for u in range(ka, kb):
                     assert (t, u) not in covered
                     covered.add((t, u))

@@ -631,6 +631,38 @@ def test_channel_mix_fwd_full_gate_m512(lbq):
     assert_status_clean(lbq)
 
 
+@pytest.mark.parametrize("m", [1, 16, 40])
+def test_channel_mix_grouped_layer_set(lbq, m):
+    """Four channel-mix layers (8B q, k and gate shapes, plus ragged halves of
+    1000 rows) in one grouped call, with a rank-8 adapter on two of them:
+    every output element of every layer against the oracle (m <= 16 runs the
+    halves as grouped decode launches, m = 40 the tensor-core GEMMs)."""
+    k, r, s = 4096, 8, 2.0
+    shapes = [(4096, 0), (1024, r), (14336, 0), (1000, r)]
+    X = syn.normal_bf16((m, k), 1.0, seed=900 + m)
+    probs, refs = [], []
+    for i, (n, rank) in enumerate(shapes):
+        W = mixed_weight(n, k, seed=910 + i) if n == 1000 else syn.weight_bf16(n, k, 0.02, seed=910 + i,
+                                                                                 outlier_frac=0.001)
+        mix, perm, n4, halves = _channel_mix(lbq, W, 0.25, seed=920 + i)
+        What = np.zeros((n, k), np.float32)
+        for (packed, scale, zero), rows, bits in ((halves[0], perm[:n4], 4), (halves[1], perm[n4:], 2)):
+            What[rows] = oracle.minmax_dequantize(packed, scale, zero, k, bits, 128 if bits == 4 else 64)
+        if rank:
+            A = syn.normal_bf16((rank, k), 0.01, seed=930 + i)
+            B = syn.normal_bf16((n, rank), 0.01, seed=940 + i)
+            probs.append((X.cuda(), mix, A.cuda(), B.cuda(), s))
+            refs.append(oracle.linear_fwd(syn.bits_u16(X), What, syn.bits_u16(A), syn.bits_u16(B), s))
+        else:
+            probs.append((X.cuda(), mix))
+            refs.append(oracle.linear_fwd(syn.bits_u16(X), What))
+    outs = lbq.linear_fwd_mix_grouped(probs)
+    torch.cuda.synchronize()
+    for (Y, _), (Yr, _, Yb), (n, _) in zip(outs, refs, shapes):
+        assert_within(Y.cpu().numpy(), Yr, Yb, f"Y (grouped channel-mix, n={n}, M={m})")
+    assert_status_clean(lbq)
+
+
 @pytest.mark.parametrize("m", [16, 512])
 def test_channel_mix_ragged_halves(lbq, m):
     """Halves that are not whole 128-row tiles (250 INT4 rows, 750 INT2 rows),
