@@ -223,8 +223,8 @@ __device__ __forceinline__ PreConst preload_const(const FwdParams& p, int64_t gr
 // the part's codes within the line.
 template <int KIND, int NV>
 __device__ __forceinline__ void dequant_part_kblock(const uint8_t* wrow, int row, int byte0, PreConst pc,
-                                                    float dq_offset, bool has_dq, const float* s_cb,
-                                                    uint32_t (&out)[NV]) {
+                                                    const MinMaxConst& c, float dq_offset, bool has_dq,
+                                                    const float* s_cb, uint32_t (&out)[NV]) {
     constexpr int NW = (KIND == kInt2) ? NV / 8 : NV / 4;   // 32-bit words of codes
     const uint8_t* src = wrow + 16 * ((byte0 >> 4) ^ (row & 7)) + (byte0 & 15);
     uint32_t w[NW];
@@ -242,7 +242,6 @@ __device__ __forceinline__ void dequant_part_kblock(const uint8_t* wrow, int row
         w[0] = *reinterpret_cast<const uint32_t*>(src);
     }
     if (KIND == kInt4) {
-        const MinMaxConst c = minmax_const(static_cast<uint16_t>(pc.a), static_cast<uint16_t>(pc.b));
         if (c.fast) {
 #pragma unroll
             for (int i = 0; i < NW; ++i) {
@@ -259,7 +258,6 @@ __device__ __forceinline__ void dequant_part_kblock(const uint8_t* wrow, int row
                     out[4 * i + j] = minmax_pair_exact((w[i] >> (8 * j + 4)) & 15u, (w[i] >> (8 * j)) & 15u, c);
         }
     } else if (KIND == kInt2) {
-        const MinMaxConst c = minmax_const(static_cast<uint16_t>(pc.a), static_cast<uint16_t>(pc.b));
         if (c.fast) {
 #pragma unroll
             for (int i = 0; i < NW; ++i) {
@@ -363,7 +361,10 @@ struct FwdCfg {
     static constexpr int kXBlocks = NT <= 16 ? 8 : NT <= 32 ? 4 : NT <= 64 ? 2 : 1;   // k-blocks per X box
     static constexpr int kXStages = NT <= 32 ? 2 : NT <= 128 ? 3 : 4;
     static constexpr int kWStages = NT <= 32 ? 4 : NT <= 64 ? 3 : NT <= 128 ? 2 : 4;
-    static constexpr int kAStages = NT <= 32 ? 6 : 4;
+    // dequantized A slots in tensor memory: the 256-token tile has room for
+    // eight beside its accumulator, so the dequantize warps can run further
+    // ahead of the MMAs
+    static constexpr int kAStages = NT <= 32 ? 6 : NT >= 256 ? 8 : 4;
     static constexpr int kMinBlocks = NT >= 256 ? 1 : 2;   // CTAs per SM
     static constexpr int kDqWarps = NT >= 256 ? 16 : 8;
 };
@@ -560,7 +561,12 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             __syncwarp();
             if (lane == 0) mbar_arrive(&afull[0]);
         }
+        // scale and zero (MinMax) change once per group of GB k-blocks, the
+        // absmax (codebook) every k-block; loaded one group ahead
+        constexpr int GB = (KIND == kInt4) ? 2 : 1;
         PreConst nxt = preload_const<KIND>(p, grow, kb0, row_ok && nkb > 0);
+        PreConst cur{0u, 0u};
+        MinMaxConst mc{};
         // A k-block's tensor-memory store completes while the next k-block is
         // dequantized: its arrival on afull comes one k-block later, off the
         // warp's critical path (the A ring keeps the MMAs fed meanwhile).
@@ -575,8 +581,11 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         };
         for (int i = 0; i < nkb; ++i) {
             const int c = i / SUB, sub = i - c * SUB, w = c % WS, ia = i + a_off, a = ia % AS;
-            const PreConst cur = nxt;
-            if (i + 1 < nkb) nxt = preload_const<KIND>(p, grow, kb0 + i + 1, row_ok);
+            if (i % GB == 0) {
+                cur = nxt;
+                if (i + GB < nkb) nxt = preload_const<KIND>(p, grow, kb0 + i + GB, row_ok);
+                if (KIND != kCode4) mc = minmax_const(static_cast<uint16_t>(cur.a), static_cast<uint16_t>(cur.b));
+            }
             if (sub == 0 && !mbar_wait(&fullW[w], (c / WS) & 1, s_abort)) break;
             if (ia >= AS && !mbar_wait(&aempty[a], ((ia / AS) - 1) & 1, s_abort)) break;
             tc_fence_after();
@@ -584,7 +593,7 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             uint32_t vals[NV];
             if (row_ok) {
                 dequant_part_kblock<KIND, NV>(sW + w * L::kWBytes + row * 128, row, sub * WB + part * (WB / PARTS), cur,
-                                              dq_offset, has_dq, s_cb, vals);
+                                              mc, dq_offset, has_dq, s_cb, vals);
             } else {
 #pragma unroll
                 for (int j = 0; j < NV; ++j) vals[j] = 0u;

@@ -66,7 +66,7 @@ template <int NT>
 struct BwdCfg {
     static constexpr int kXStages = NT <= 64 ? 4 : NT <= 128 ? 2 : 4;   // dY tiles in flight (see the forward)
     static constexpr int kWStages = 4;
-    static constexpr int kAStages = NT <= 64 ? 3 : 2;
+    static constexpr int kAStages = NT <= 64 ? 3 : NT >= 256 ? 3 : 2;
     static constexpr int kMinBlocks = NT >= 256 ? 1 : 2;   // CTAs per SM
     static constexpr int kDqWarps = NT >= 256 ? 16 : 8;     // dequantize + epilogue warps
 };
