@@ -93,3 +93,46 @@ def test_merge_entry_points_reject_bad_arguments():
     assert unmerge(0x4000, 16, 12, None, None, 0, 1.0, 0x5000, None) == lbq.LBQ_EINVAL     # k % 8 != 0
     assert unmerge(0x4000, 0, 16, None, None, 0, 1.0, 0x5000, None) == lbq.LBQ_EINVAL
     assert unmerge(0x4002, 16, 16, None, None, 0, 1.0, 0x5000, None) == lbq.LBQ_EALIGN
+
+
+def test_grouped_entry_points_reject_bad_arguments():
+    q = _qw()
+    P = (lbq.lbq_fwd_problem * 2)()
+    for i in range(2):
+        P[i] = lbq.lbq_fwd_problem(X=0x4000, q=ctypes.pointer(q), A=None, B=None, rank=0, s=0.0, Y=0x5000, T_save=None)
+    g = lbq.lbq_linear_fwd_grouped
+    assert g(4, P, 0, None, 0, None) == lbq.LBQ_EINVAL
+    assert g(4, None, 2, None, 0, None) == lbq.LBQ_EINVAL
+    assert g(0, P, 2, None, 0, None) == lbq.LBQ_EINVAL
+    P[1].Y = 0x5004
+    assert g(4, P, 2, None, 0, None) == lbq.LBQ_EALIGN
+    P[1].Y = 0x5000
+    P[1].rank = 8                                              # rank > 0 needs A, B and T_save
+    assert g(4, P, 2, None, 0, None) == lbq.LBQ_EINVAL
+
+    hi, lo = _qw(n=64), _qw(n=192, bits=2, group=64)
+    mix = lbq.lbq_qweight_mix(hi=hi, lo=lo, perm=0xB000)
+    M = (lbq.lbq_mix_problem * 2)()
+    for i in range(2):
+        M[i] = lbq.lbq_mix_problem(X=0x4000, q=ctypes.pointer(mix), A=None, B=None, rank=0, s=0.0, Y=0x5000,
+                                   T_save=None)
+    gm = lbq.lbq_linear_fwd_mix_grouped
+    assert gm(4, M, 0, None, 0, None) == lbq.LBQ_EINVAL
+    assert gm(4, None, 2, None, 0, None) == lbq.LBQ_EINVAL
+    M[1].Y = 0x5008
+    assert gm(4, M, 2, None, 0, None) == lbq.LBQ_EALIGN
+    M[1].Y = 0x5000
+    bad = lbq.lbq_qweight_mix(hi=hi, lo=_qw(n=192, k=1024, bits=2, group=64), perm=0xB000)   # halves differ in k
+    M[1].q = ctypes.pointer(bad)
+    assert gm(4, M, 2, None, 0, None) == lbq.LBQ_EINVAL
+    cbm = lbq.lbq_qweight_mix(hi=hi, lo=_qw(n=192, scheme=lbq.LBQ_CODEBOOK4, group=64, absmax=0x9000, codebook=0xA000),
+                              perm=0xB000)                      # halves are MinMax only
+    M[1].q = ctypes.pointer(cbm)
+    assert gm(4, M, 2, None, 0, None) == lbq.LBQ_EINVAL
+    nop = lbq.lbq_qweight_mix(hi=hi, lo=lo, perm=None)
+    M[1].q = ctypes.pointer(nop)
+    assert gm(4, M, 2, None, 0, None) == lbq.LBQ_EINVAL
+    # the workspace queries are host-only and cover both halves of every problem
+    M[1].q = ctypes.pointer(mix)
+    assert lbq.lbq_linear_fwd_mix_grouped_workspace_size(0, M, 2) == 0
+    assert lbq.lbq_linear_fwd_mix_grouped_workspace_size(4, M, 2) % 256 == 0
