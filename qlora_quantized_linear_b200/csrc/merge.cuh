@@ -16,7 +16,8 @@
 // registers.  The thread's weight words go out first; meanwhile the adapter
 // is staged in shared memory as fp32 (A as 16-byte loads along the columns, B
 // as 16-byte loads along each row when the rank is a multiple of 8), so that
-// one 16-byte load of A and two broadcast loads of B feed 16 paired FMAs.
+// one 16-byte load of A and two broadcast loads of B feed 16 packed fp32 FMAs
+// (fma.rn.f32x2 on pairs of rows).
 #pragma once
 
 #include "quantize.cuh"
@@ -51,14 +52,21 @@ struct MergeParams {
 
 __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) { return pack_bf16x2_rn(lo, hi); }
 
-// (d0, d1) = fma((a0, a1), (b, b), (d0, d1)): two IEEE fused multiply-adds in
-// one instruction, each rounded once exactly as fmaf
-__device__ __forceinline__ void fma_x2(float& d0, float& d1, float a0, float a1, float b) {
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\tmov.b64 rd, {%0, %1};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rd;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "+f"(d0), "+f"(d1)
-        : "f"(a0), "f"(a1), "f"(b));
+// Two fp32 values in one 64-bit register pair, for the packed fp32 FMA.
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void unpack_f32x2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+// d = fma(a, b, d) on both halves: two IEEE fused multiply-adds in one
+// instruction, each rounded once exactly as fmaf.
+__device__ __forceinline__ void fma_x2(uint64_t& d, uint64_t a, uint64_t b) {
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
 }
 
 // The weight inputs of one thread for one row tile (loaded a tile ahead).
@@ -115,11 +123,14 @@ __global__ void __launch_bounds__(kMergeThreads, 3) lora_merge_kernel(const Merg
     MergeIn in;
     merge_load<MODE>(p, row0, col0, in);
 
-    float d[8][4];
+    // the partial sums as pairs of rows (2 ip, 2 ip + 1) per column c, so that
+    // the B values of two rows (adjacent in shared memory) form one operand and
+    // only the A value of a column is duplicated into a pair
+    uint64_t dp[4][4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int ip = 0; ip < 4; ++ip)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) d[i][c] = 0.0f;
+        for (int c = 0; c < 4; ++c) dp[ip][c] = 0ull;
 
     for (int u0 = 0; u0 < p.rank; u0 += kMergeRankChunk) {
         const int ur = min(kMergeRankChunk, p.rank - u0);
@@ -164,16 +175,23 @@ __global__ void __launch_bounds__(kMergeThreads, 3) lora_merge_kernel(const Merg
             const float4 a = *reinterpret_cast<const float4*>(&sA[u][lane * 4]);
             const float4 b0 = *reinterpret_cast<const float4*>(&sB[u][warp * 8]);
             const float4 b1 = *reinterpret_cast<const float4*>(&sB[u][warp * 8 + 4]);
-            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            const uint64_t bp[4] = {pack_f32x2(b0.x, b0.y), pack_f32x2(b0.z, b0.w), pack_f32x2(b1.x, b1.y),
+                                    pack_f32x2(b1.z, b1.w)};
+            const uint64_t ap[4] = {pack_f32x2(a.x, a.x), pack_f32x2(a.y, a.y), pack_f32x2(a.z, a.z),
+                                    pack_f32x2(a.w, a.w)};
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                fma_x2(d[i][0], d[i][1], a.x, a.y, bv[i]);
-                fma_x2(d[i][2], d[i][3], a.z, a.w, bv[i]);
-            }
+            for (int ip = 0; ip < 4; ++ip)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) fma_x2(dp[ip][c], bp[ip], ap[c]);
         }
     }
     if (MODE == kMergeCode4 && p.rank == 0) __syncthreads();  // the codebook copy (else done by the chunk barrier)
     if (col0 >= p.k) return;                                  // k % 8 == 0: a thread's 4 columns are all in or out
+    float d[8][4];
+#pragma unroll
+    for (int ip = 0; ip < 4; ++ip)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) unpack_f32x2(dp[ip][c], d[2 * ip][c], d[2 * ip + 1][c]);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int64_t row = row0 + i;

@@ -23,14 +23,15 @@ namespace lbq {
 // rint(fl(w / d)), the IEEE quotient rounded half-to-even to an integer, for
 // finite w and a positive normal d with rs = fl(1 / d).  t = fl(w * rs) is
 // within 2 ulp of w / d and fl(w / d) within half an ulp, so rint(t) is the
-// answer whenever t is more than 3 ulp away from the nearest half-integer;
-// only those rare elements pay for the correctly rounded division.
+// answer whenever t is more than 3 ulp away from the nearest half-integer.
+// For |t| < 2^11 an ulp is at most 2^-13, so a fixed margin of 2^-10 covers
+// the 3 ulp; only elements inside the margin (or with |t| >= 2^11) pay for
+// the correctly rounded division.
 __device__ __forceinline__ float rint_div(float w, float d, float rs) {
     const float t = __fmul_rn(w, rs);
     const float n = rintf(t);
-    const float gap = 0.5f - fabsf(__fsub_rn(t, n));                 // distance to the half-integer
-    const float ulp3 = fmaxf(fabsf(t), 1.0f) * 3.5762786865234375e-07f;  // 3 * 2^-23 * max(|t|, 1)
-    if (gap > ulp3) return n;
+    const float h = __fsub_rn(t, n);                                 // exact (Sterbenz): |h| <= 0.5
+    if (fabsf(h) < 0.4990234375f && fabsf(t) < 2048.0f) return n;   // 0.5 - 2^-10
     return rintf(__fdiv_rn(w, d));
 }
 
@@ -57,12 +58,16 @@ __device__ __forceinline__ void minmax_quantize_chunk(uint4 raw, int64_t chunk, 
         v[2 * i] = bf16_bits_to_f32(words[i] & 0xFFFFu);
         v[2 * i + 1] = bf16_bits_to_f32(words[i] >> 16);
     }
-    float mn = v[0], mx = v[0];
+    // the lane's extremes on bf16 pairs (exact: a minimum of bf16 values is one of them)
+    __nv_bfloat162 mn2 = *reinterpret_cast<const __nv_bfloat162*>(&words[0]), mx2 = mn2;
 #pragma unroll
-    for (int i = 1; i < 8; ++i) {
-        mn = fminf(mn, v[i]);
-        mx = fmaxf(mx, v[i]);
+    for (int i = 1; i < 4; ++i) {
+        const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&words[i]);
+        mn2 = __hmin2(mn2, x);
+        mx2 = __hmax2(mx2, x);
     }
+    float mn = fminf(__low2float(mn2), __high2float(mn2));
+    float mx = fmaxf(__low2float(mx2), __high2float(mx2));
 #pragma unroll
     for (int off = LPG / 2; off > 0; off >>= 1) {
         mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
