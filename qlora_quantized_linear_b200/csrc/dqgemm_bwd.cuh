@@ -274,10 +274,13 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
         const float dq_off = has_dq ? __ldg(p.offset) : 0.0f;
         uint32_t mg = 0x43004300u;
         asm volatile("" : "+r"(mg));
-        // constants of the next block's channels, loaded one block ahead:
-        // MinMax scale and zero; codebook absmax, or q8 and s2
-        uint32_t ns[SLOTS], nz[SLOTS];
-        auto load_const = [&](int i) {
+        // constants of a block's channels (MinMax scale and zero; codebook
+        // absmax, or q8 and s2), loaded two blocks ahead into one of two
+        // register sets that the loop below uses in turn (the blocks are
+        // processed in pairs, so no register is copied while its load is in
+        // flight)
+        uint32_t s0[SLOTS], z0[SLOTS], s1[SLOTS], z1[SLOTS];
+        auto load_const = [&](int i, uint32_t (&ns)[SLOTS], uint32_t (&nz)[SLOTS]) {
 #pragma unroll
             for (int u = 0; u < SLOTS; ++u) {
                 const int64_t c = static_cast<int64_t>(cb0 + i) * 64 + crow0 + u * cstep;
@@ -294,7 +297,8 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
                 }
             }
         };
-        if (ncb > 0) load_const(0);
+        if (ncb > 0) load_const(0, s0, z0);
+        if (ncb > 1) load_const(1, s1, z1);
         if (lora) {
             // A operand (ring slot 0): K row u = A[u, k0 + feature], features in
             // the tile's pairing order (zero beyond the rank and beyond k)
@@ -322,17 +326,11 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
             __syncwarp();
             if (lane == 0) mbar_arrive(&afull[0]);
         }
-        for (int i = 0; i < ncb; ++i) {
+        // block i with its constants cs, cz; false after a timed-out wait
+        auto block = [&](int i, const uint32_t (&cs)[SLOTS], const uint32_t (&cz)[SLOTS]) -> bool {
             const int w = i % WS, ia = i + a_off, a = ia % AS;
-            uint32_t cs[SLOTS], cz[SLOTS];
-#pragma unroll
-            for (int u = 0; u < SLOTS; ++u) {
-                cs[u] = ns[u];
-                cz[u] = nz[u];
-            }
-            if (i + 1 < ncb) load_const(i + 1);
-            if (!mbar_wait(&fullW[w], (i / WS) & 1, s_abort)) break;
-            if (ia >= AS && !mbar_wait(&aempty[a], ((ia / AS) - 1) & 1, s_abort)) break;
+            if (!mbar_wait(&fullW[w], (i / WS) & 1, s_abort)) return false;
+            if (ia >= AS && !mbar_wait(&aempty[a], ((ia / AS) - 1) & 1, s_abort)) return false;
             uint32_t words[SLOTS];
 #pragma unroll
             for (int u = 0; u < SLOTS; ++u)
@@ -385,6 +383,14 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
                 mbar_arrive(&afull[a]);
                 mbar_arrive(&emptyW[w]);
             }
+            return true;
+        };
+        for (int i = 0; i < ncb; i += 2) {
+            if (!block(i, s0, z0)) break;
+            if (i + 2 < ncb) load_const(i + 2, s0, z0);
+            if (i + 1 >= ncb) break;
+            if (!block(i + 1, s1, z1)) break;
+            if (i + 3 < ncb) load_const(i + 3, s1, z1);
         }
 
         // ------------------------------------------------------------ epilogue
