@@ -397,57 +397,82 @@ def run_decode(args, dist, lbq, syn, torch, peaks):
 
 
 def run_decode_e2e(args, dist, wl, lbq, torch, stream):
-    """The decode step end to end through the C ABI: every step copies that
-    step's activations from pinned host memory to the device (one copy of the
-    four distinct X of the layer set), makes the two grouped forward calls
-    (seven layers each), and
-    reads all 14 outputs back to pinned host memory (one copy).  Wall clock
-    from the host, synchronised at both ends, between barriers; with several
-    ranks, the units of all ranks over the slowest rank's time."""
+    """The decode step end to end through the C ABI, as a serving loop runs
+    it: every step copies that step's activations from pinned host memory to
+    the device (one copy of the four distinct X of the layer set), makes the
+    two grouped forward calls (seven layers each) and reads all 14 outputs
+    back to pinned host memory (one copy).  The copies run on their own
+    streams (host to device, device to host) with the host and device buffers
+    doubled, so step i's outputs travel back and step i + 1's inputs travel
+    in while step i + 1 (or i) computes; events order each buffer's reuse.
+    Wall clock from the host, synchronised at both ends, between barriers;
+    with several ranks, the units of all ranks over the slowest rank's
+    time."""
     import ctypes
     xkeys = sorted(wl.X)                                      # (m, k): the distinct activations
     ykeys = [(m, name) for m in DECODE_M for name in wl.shapes]
     xn = {key: wl.X[key].numel() for key in xkeys}
     yn = {key: wl.Y[key].numel() for key in ykeys}
-    xh = torch.empty(sum(xn.values()), dtype=torch.bfloat16).pin_memory()
-    yh = torch.empty(sum(yn.values()), dtype=torch.float32).pin_memory()
-    xd = torch.empty_like(xh, device="cuda")
-    yd = torch.empty_like(yh, device="cuda")
-    xview, yview, off = {}, {}, 0
-    for key in xkeys:                                         # host copy of the inputs, views on the device
-        xh[off:off + xn[key]].copy_(wl.X[key].reshape(-1).cpu())
-        xview[key] = xd[off:off + xn[key]]
-        off += xn[key]
-    off = 0
-    for key in ykeys:
-        yview[key] = yd[off:off + yn[key]]
-        off += yn[key]
-    import ctypes
+    nb = 2                                                    # buffers in flight
+    xh = [torch.empty(sum(xn.values()), dtype=torch.bfloat16).pin_memory() for _ in range(nb)]
+    yh = [torch.empty(sum(yn.values()), dtype=torch.float32).pin_memory() for _ in range(nb)]
+    xd = [torch.empty_like(xh[0], device="cuda") for _ in range(nb)]
+    yd = [torch.empty_like(yh[0], device="cuda") for _ in range(nb)]
+    xview = [{} for _ in range(nb)]
+    yview = [{} for _ in range(nb)]
+    for b in range(nb):
+        off = 0
+        for key in xkeys:                                     # host copy of the inputs, views on the device
+            xh[b][off:off + xn[key]].copy_(wl.X[key].reshape(-1).cpu())
+            xview[b][key] = xd[b][off:off + xn[key]]
+            off += xn[key]
+        off = 0
+        for key in ykeys:
+            yview[b][key] = yd[b][off:off + yn[key]]
+            off += yn[key]
     sh = stream.cuda_stream
-    calls = []                                                # one grouped call per decode size and copy
+    calls = []                                                # [phase][buffer]: one grouped call per decode size
     for phase in range(COPIES):
-        row = []
-        for j, m in enumerate(DECODE_M):
-            copy = (2 * phase + j) % COPIES
-            arr = (lbq.lbq_fwd_problem * len(wl.shapes))()
-            for i, (name, (n, k)) in enumerate(wl.shapes.items()):
-                arr[i] = lbq.lbq_fwd_problem(X=xview[(m, k)].data_ptr(), q=ctypes.pointer(wl.qw[copy][name].struct),
-                                             A=None, B=None, rank=0, s=0.0, Y=yview[(m, name)].data_ptr(), T_save=None)
-            row.append((m, arr, len(wl.shapes), wl.ws.data_ptr(), wl.ws_bytes, sh))
-        calls.append(row)
+        per_buf = []
+        for b in range(nb):
+            row = []
+            for j, m in enumerate(DECODE_M):
+                copy = (2 * phase + j) % COPIES
+                arr = (lbq.lbq_fwd_problem * len(wl.shapes))()
+                for i, (name, (n, k)) in enumerate(wl.shapes.items()):
+                    arr[i] = lbq.lbq_fwd_problem(X=xview[b][(m, k)].data_ptr(),
+                                                 q=ctypes.pointer(wl.qw[copy][name].struct), A=None, B=None, rank=0,
+                                                 s=0.0, Y=yview[b][(m, name)].data_ptr(), T_save=None)
+                row.append((m, arr, len(wl.shapes), wl.ws.data_ptr(), wl.ws_bytes, sh))
+            per_buf.append(row)
+        calls.append(per_buf)
     fwd = lbq.lbq_linear_fwd_grouped
-    h2d = xh.numel() * xh.element_size()
-    d2h = yh.numel() * yh.element_size()
+    h2d = xh[0].numel() * xh[0].element_size()
+    d2h = yh[0].numel() * yh[0].element_size()
     steps = max(3, min(args.steps, 50))
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    x_ready = [torch.cuda.Event() for _ in range(nb)]         # inputs of buffer b on the device
+    y_ready = [torch.cuda.Event() for _ in range(nb)]         # outputs of buffer b written (inputs read)
+    y_read = [torch.cuda.Event() for _ in range(nb)]          # outputs of buffer b copied to the host
 
     def one_step(i):
+        b = i % nb
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(y_ready[b])                       # step i - nb has read these inputs
+            xd[b].copy_(xh[b], non_blocking=True)
+            x_ready[b].record(s_in)
         with torch.cuda.stream(stream):
-            xd.copy_(xh, non_blocking=True)
-            for a in calls[i % COPIES]:
+            stream.wait_event(x_ready[b])
+            stream.wait_event(y_read[b])                      # step i - nb's outputs are on the host
+            for a in calls[i % COPIES][b]:
                 rc = fwd(*a)
                 if rc != 0:
                     raise RuntimeError(f"lbq_linear_fwd_grouped returned {rc}")
-            yh.copy_(yd, non_blocking=True)
+            y_ready[b].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(y_ready[b])
+            yh[b].copy_(yd[b], non_blocking=True)
+            y_read[b].record(s_out)
 
     for i in range(3):
         one_step(i)
@@ -456,7 +481,7 @@ def run_decode_e2e(args, dist, wl, lbq, torch, stream):
     t0 = time.perf_counter()
     for i in range(steps):
         one_step(i)
-    stream.synchronize()
+    torch.cuda.synchronize()                                  # every step's outputs are on the host
     dt = time.perf_counter() - t0
     dist.barrier()
     dt_max = dist.max(dt)
@@ -465,7 +490,8 @@ def run_decode_e2e(args, dist, wl, lbq, torch, stream):
             "d2h_bytes_per_step": d2h, "steps": steps,
             "note": "lbq_linear_fwd_grouped through the C ABI, one call per decode size (7 layers each); per step "
                     "and rank one pinned host->device copy of the four distinct activations and one device->host "
-                    "copy of the 14 outputs"}
+                    "copy of the 14 outputs, on their own streams with double buffers, overlapping the "
+                    "neighbouring steps' calls"}
 
 
 # ----------------------------------------------------------------------------- extra rows
