@@ -160,6 +160,12 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
     const int cb_total = (p.n + 63) / 64;
     const int cb0 = split * p.cb_per_split;
     const int ncb = min(p.cb_per_split, cb_total - cb0);
+    // The CTAs of a wave start their walk over the channel blocks at
+    // different blocks (a fixed rotation per CTA), so that a block's scales
+    // and zeros and its dY tile are not first requested by all of them at
+    // once; the order of the sum over blocks is then fixed per CTA.
+    const int rot = ncb > 0 ? static_cast<int>((static_cast<int64_t>(blockIdx.y * gridDim.x + blockIdx.x) * 37) % ncb) : 0;
+    auto blk = [&](int i) { return cb0 + (i + rot < ncb ? i + rot : i + rot - ncb); };
     // the adapter term s * U A enters the accumulator through rank/16 MMAs
     // before the main loop, in the first split only; its A operand (the rows
     // of A) takes the first slot of the A ring, as a block before the first
@@ -211,14 +217,14 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
                 if (wi < ncb && (wi < WS || mbar_try_wait(&emptyW[wi % WS], ((wi / WS) - 1) & 1))) {
                     const int w = wi % WS;
                     mbar_arrive_expect_tx(&fullW[w], L::kWBytes);
-                    tma_load_2d(sW + w * L::kWBytes, &tmW, &fullW[w], k0 * BITS / 8, (cb0 + wi) * 64);
+                    tma_load_2d(sW + w * L::kWBytes, &tmW, &fullW[w], k0 * BITS / 8, blk(wi) * 64);
                     ++wi;
                     prog = true;
                 }
                 if (xi < ncb && (xi < XS || mbar_try_wait(&emptyX[xi % XS], ((xi / XS) - 1) & 1))) {
                     const int x = xi % XS;
                     mbar_arrive_expect_tx(&fullX[x], L::kXBytes);
-                    tma_load_2d(sX + x * L::kXBytes, &tmDY, &fullX[x], (cb0 + xi) * 64, t0);
+                    tma_load_2d(sX + x * L::kXBytes, &tmDY, &fullX[x], blk(xi) * 64, t0);
                     ++xi;
                     prog = true;
                 }
@@ -283,7 +289,7 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
         auto load_const = [&](int i, uint32_t (&ns)[SLOTS], uint32_t (&nz)[SLOTS]) {
 #pragma unroll
             for (int u = 0; u < SLOTS; ++u) {
-                const int64_t c = static_cast<int64_t>(cb0 + i) * 64 + crow0 + u * cstep;
+                const int64_t c = static_cast<int64_t>(blk(i)) * 64 + crow0 + u * cstep;
                 if (KIND != kCode4) {
                     ns[u] = c < p.n ? __ldg(p.scale + c * p.ngroups + gcol) : 0u;
                     nz[u] = c < p.n ? __ldg(p.zero + c * p.ngroups + gcol) : 0u;
