@@ -420,6 +420,19 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     const int kb0 = split * p.kb_per_split;            // a multiple of SUB
     const int nkb = min(p.kb_per_split, kb_total - kb0);
     const int nch = (nkb + SUB - 1) / SUB;              // weight chunks of this CTA
+    // On long walks (at least 192 k-blocks, K >= 12288) the CTAs of a wave
+    // start at different places (a fixed rotation per CTA, in whole weight
+    // chunks and activation boxes), so that an activation tile is not first
+    // requested by all of them at once; the order of the sum is then fixed
+    // per CTA.  (Measured: the 8B down projection at M = 4096 580 -> 545 us;
+    // the gate projection, 64 k-blocks, ran slower rotated.)  k-block i of
+    // the walk is k-block kbat(i).
+    constexpr int RU = SUB > XB ? SUB : XB;
+    const int nru = nkb / RU;
+    const int rotk = (nkb >= 192 && nkb % RU == 0 && nru > 1)
+                         ? static_cast<int>((static_cast<int64_t>(blockIdx.y * gridDim.x + blockIdx.x) * 37) % nru) * RU
+                         : 0;
+    auto kbat = [&](int i) { return kb0 + (i + rotk < nkb ? i + rotk : i + rotk - nkb); };
     // the adapter term s * T B^T enters the accumulator through rank/16 MMAs
     // before the main loop, in the first K split only: its A operand (the B
     // rows) takes the first slot of the A ring, as a k-block before the first
@@ -474,7 +487,7 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 if (wi < nch && (wi < WS || mbar_try_wait(&emptyW[wi % WS], ((wi / WS) - 1) & 1))) {
                     const int w = wi % WS;
                     mbar_arrive_expect_tx(&fullW[w], L::kWBytes);
-                    tma_load_2d(sW + w * L::kWBytes, &tmW, &fullW[w], (kb0 + wi * SUB) * WB, n0);
+                    tma_load_2d(sW + w * L::kWBytes, &tmW, &fullW[w], kbat(wi * SUB) * WB, n0);
                     ++wi;
                     prog = true;
                 }
@@ -482,7 +495,7 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     const int x = xi % XS;
                     LBQ_TRACE_EVENT(6, xi * XB);
                     mbar_arrive_expect_tx(&fullX[x], L::kXBytes);
-                    tma_load_3d(sX + x * L::kXBytes, &tmX, &fullX[x], 0, t0, kb0 + xi * XB);
+                    tma_load_3d(sX + x * L::kXBytes, &tmX, &fullX[x], 0, t0, kbat(xi * XB));
                     LBQ_TRACE_EVENT(1, xi * XB);
                     ++xi;
                     prog = true;
@@ -564,7 +577,7 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         // scale and zero (MinMax) change once per group of GB k-blocks, the
         // absmax (codebook) every k-block; loaded one group ahead
         constexpr int GB = (KIND == kInt4) ? 2 : 1;
-        PreConst nxt = preload_const<KIND>(p, grow, kb0, row_ok && nkb > 0);
+        PreConst nxt = preload_const<KIND>(p, grow, kbat(0), row_ok && nkb > 0);
         PreConst cur{0u, 0u};
         MinMaxConst mc{};
         // A k-block's tensor-memory store completes while the next k-block is
@@ -583,7 +596,7 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             const int c = i / SUB, sub = i - c * SUB, w = c % WS, ia = i + a_off, a = ia % AS;
             if (i % GB == 0) {
                 cur = nxt;
-                if (i + GB < nkb) nxt = preload_const<KIND>(p, grow, kb0 + i + GB, row_ok);
+                if (i + GB < nkb) nxt = preload_const<KIND>(p, grow, kbat(i + GB), row_ok);
                 if (KIND != kCode4) mc = minmax_const(static_cast<uint16_t>(cur.a), static_cast<uint16_t>(cur.b));
             }
             if (sub == 0 && !mbar_wait(&fullW[w], (c / WS) & 1, s_abort)) break;
