@@ -278,8 +278,11 @@ lbq_status lbq_linear_fwd_noalloc_reset(lbq_stream_t stream);
  * outputs (same layouts, rank and alignment rules; `q` is a host pointer to
  * the descriptor).  For m <= 16 the problems run as one launch of the decode
  * GEMV per group of up to 8 weights (after one adapter launch per problem with
- * rank > 0), so the fixed costs of a launch are paid once per group; for
- * larger m they run one after the other on `stream`.  The workspace
+ * rank > 0), so the fixed costs of a launch are paid once per group.  For
+ * larger m, when the problems' 128-row x token tiles together fill the
+ * GPU's CTA slots, they run as grouped tensor-core launches of up to 8
+ * problems each, without K splits; otherwise one after the other on
+ * `stream`, each with its own K split.  The workspace
  * (lbq_linear_fwd_grouped_workspace_size bytes, zero-filled before its first
  * use, same reuse rules as lbq_linear_fwd's) serves all of them.  Results are
  * bit for bit those of separate lbq_linear_fwd calls on the same inputs when

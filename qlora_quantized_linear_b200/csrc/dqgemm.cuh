@@ -378,10 +378,20 @@ __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_
         : "memory");
 }
 
-template <int NT, int KIND, int XS, int XB, int WS, int AS, int MINB, int DQW>
-__global__ void __launch_bounds__(fwd_threads(DQW), MINB)
-dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                  const FwdParams p) {
+// The output tile a CTA computes: rows n0 .. n0 + 127 of the weight, tokens
+// t0 .. t0 + NT - 1, K split `split`; `tile` numbers the tile within its
+// GEMM (the split-K counters), `cta` the CTA within the launch (the rotation
+// of long k-walks).
+struct FwdTile {
+    int n0, t0, split;
+    uint32_t tile, cta;
+};
+
+// One CTA of the forward GEMM (see the top of this file); tmX and tmW are
+// the tensor maps of its activations and packed weight.
+template <int NT, int KIND, int XS, int XB, int WS, int AS, int DQW>
+__device__ __forceinline__ void fwd_tile(const CUtensorMap* tmX, const CUtensorMap* tmW, const FwdParams& p,
+                                         const FwdTile tl) {
     constexpr int WB = WeightTile<KIND>::kRowBytes;
     constexpr int PARTS = DQW / 4;                     // dequant warps per TMEM lane quarter
     constexpr int NV = 32 / PARTS;                     // bf16x2 words of a warp's part of a k-block row
@@ -413,9 +423,9 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     uint8_t* sTop = smem + L::kLoraT;                  // s*T operand tile [NT x 128 B]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * 128;
-    const int t0 = blockIdx.y * NT;
-    const int split = blockIdx.z;
+    const int n0 = tl.n0;
+    const int t0 = tl.t0;
+    const int split = tl.split;
     const int kb_total = p.k / 64;
     const int kb0 = split * p.kb_per_split;            // a multiple of SUB
     const int nkb = min(p.kb_per_split, kb_total - kb0);
@@ -430,7 +440,7 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     constexpr int RU = SUB > XB ? SUB : XB;
     const int nru = nkb / RU;
     const int rotk = (nkb >= 192 && nkb % RU == 0 && nru > 1)
-                         ? static_cast<int>((static_cast<int64_t>(blockIdx.y * gridDim.x + blockIdx.x) * 37) % nru) * RU
+                         ? static_cast<int>((static_cast<int64_t>(tl.cta) * 37) % nru) * RU
                          : 0;
     auto kbat = [&](int i) { return kb0 + (i + rotk < nkb ? i + rotk : i + rotk - nkb); };
     // the adapter term s * T B^T enters the accumulator through rank/16 MMAs
@@ -458,8 +468,8 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
     }
     if (KIND == kCode4 && threadIdx.x < 16) s_cb[threadIdx.x] = p.codebook[threadIdx.x];
     if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmX);
-        tma_prefetch_desc(&tmW);
+        tma_prefetch_desc(tmX);
+        tma_prefetch_desc(tmW);
     }
     if (warp == 1) {
         tmem_alloc(s_tmem, kTmemCols);
@@ -487,7 +497,7 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                 if (wi < nch && (wi < WS || mbar_try_wait(&emptyW[wi % WS], ((wi / WS) - 1) & 1))) {
                     const int w = wi % WS;
                     mbar_arrive_expect_tx(&fullW[w], L::kWBytes);
-                    tma_load_2d(sW + w * L::kWBytes, &tmW, &fullW[w], kbat(wi * SUB) * WB, n0);
+                    tma_load_2d(sW + w * L::kWBytes, tmW, &fullW[w], kbat(wi * SUB) * WB, n0);
                     ++wi;
                     prog = true;
                 }
@@ -495,7 +505,7 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
                     const int x = xi % XS;
                     LBQ_TRACE_EVENT(6, xi * XB);
                     mbar_arrive_expect_tx(&fullX[x], L::kXBytes);
-                    tma_load_3d(sX + x * L::kXBytes, &tmX, &fullX[x], 0, t0, kbat(xi * XB));
+                    tma_load_3d(sX + x * L::kXBytes, tmX, &fullX[x], 0, t0, kbat(xi * XB));
                     LBQ_TRACE_EVENT(1, xi * XB);
                     ++xi;
                     prog = true;
@@ -662,7 +672,7 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
             __threadfence();
             named_barrier_sync(1, 32 * DQW);
             if (threadIdx.x == 64) {
-                const uint32_t tile = blockIdx.y * gridDim.x + blockIdx.x;
+                const uint32_t tile = tl.tile;
                 const uint32_t prev = atomicAdd(p.counters + tile, 1u);
                 const int last = (prev == static_cast<uint32_t>(p.nsplit - 1)) ? 1 : 0;
                 if (last) p.counters[tile] = 0u;
@@ -698,6 +708,49 @@ dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+}
+
+template <int NT, int KIND, int XS, int XB, int WS, int AS, int MINB, int DQW>
+__global__ void __launch_bounds__(fwd_threads(DQW), MINB)
+dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                  const FwdParams p) {
+    const uint32_t id = blockIdx.y * gridDim.x + blockIdx.x;
+    fwd_tile<NT, KIND, XS, XB, WS, AS, DQW>(&tmX, &tmW, p, FwdTile{static_cast<int>(blockIdx.x) * 128,
+                                                                  static_cast<int>(blockIdx.y) * NT,
+                                                                  static_cast<int>(blockIdx.z), id, id});
+}
+
+// A group of forward GEMMs with the same token count in one launch (several
+// matrices of a layer, or the two halves of a channel-mix weight): problem i
+// owns CTAs cta0[i] .. cta0[i+1]-1, row tiles fastest, then token tiles, and
+// no K split.  Every CTA runs the kernel above for its problem's weight kind.
+constexpr int kFwdMaxGroup = 8;
+
+struct FwdGroupParams {
+    CUtensorMap tmX[kFwdMaxGroup];   // activations of problem i (as for dqgemm_fwd_kernel)
+    CUtensorMap tmW[kFwdMaxGroup];   // packed weight of problem i
+    FwdParams p[kFwdMaxGroup];
+    int kind[kFwdMaxGroup];
+    int rtiles[kFwdMaxGroup];        // 128-row tiles of problem i
+    int cta0[kFwdMaxGroup + 1];      // first CTA of problem i; cta0[count] = the grid
+    int count;
+};
+
+template <int NT, int XS, int XB, int WS, int AS, int MINB, int DQW>
+__global__ void __launch_bounds__(fwd_threads(DQW), MINB)
+dqgemm_fwd_grouped_kernel(const __grid_constant__ FwdGroupParams g) {
+    int i = 0;
+    for (int j = 1; j < g.count; ++j)
+        if (static_cast<int>(blockIdx.x) >= g.cta0[j]) i = j;
+    const int local = static_cast<int>(blockIdx.x) - g.cta0[i];
+    const FwdTile tl{(local % g.rtiles[i]) * 128, (local / g.rtiles[i]) * NT, 0, static_cast<uint32_t>(local),
+                     blockIdx.x};
+    if (g.kind[i] == kInt4)
+        fwd_tile<NT, kInt4, XS, XB, WS, AS, DQW>(&g.tmX[i], &g.tmW[i], g.p[i], tl);
+    else if (g.kind[i] == kInt2)
+        fwd_tile<NT, kInt2, XS, XB, WS, AS, DQW>(&g.tmX[i], &g.tmW[i], g.p[i], tl);
+    else
+        fwd_tile<NT, kCode4, XS, XB, WS, AS, DQW>(&g.tmX[i], &g.tmW[i], g.p[i], tl);
 }
 
 }  // namespace lbq

@@ -226,14 +226,9 @@ lbq_status launch_fwd_kind(int nt, const FwdParams& p, const void* X, int m, int
     }
 }
 
-lbq_status run_fwd_gemm(const void* X, int m, const lbq_qweight* q, const void* B, int rank, float s,
-                        const float* T, float* Y, int64_t ldy, const int32_t* perm, void* ws, size_t ws_bytes,
-                        int sms, cudaStream_t st) {
-    if (m <= kGemvMaxM) {
-        const GvJob job{X, q, B, rank, s, T, Y, ldy, perm};
-        return run_gemv_jobs(m, &job, 1, ws, ws_bytes, sms, st);
-    }
-    const Plan pl = plan_fwd(m, q, sms);
+// The kernel arguments of one forward GEMM, without a K split.
+FwdParams fwd_params(int m, const lbq_qweight* q, const void* B, int rank, float s, const float* T, float* Y,
+                     int64_t ldy, const int32_t* perm) {
     FwdParams p{};
     p.m = m;
     p.n = q->n;
@@ -254,6 +249,20 @@ lbq_status run_fwd_gemm(const void* X, int m, const lbq_qweight* q, const void* 
     p.Y = Y;
     p.ldy = ldy;
     p.perm = perm;
+    p.kb_per_split = q->k / 64;
+    p.nsplit = 1;
+    return p;
+}
+
+lbq_status run_fwd_gemm(const void* X, int m, const lbq_qweight* q, const void* B, int rank, float s,
+                        const float* T, float* Y, int64_t ldy, const int32_t* perm, void* ws, size_t ws_bytes,
+                        int sms, cudaStream_t st) {
+    if (m <= kGemvMaxM) {
+        const GvJob job{X, q, B, rank, s, T, Y, ldy, perm};
+        return run_gemv_jobs(m, &job, 1, ws, ws_bytes, sms, st);
+    }
+    const Plan pl = plan_fwd(m, q, sms);
+    FwdParams p = fwd_params(m, q, B, rank, s, T, Y, ldy, perm);
     p.kb_per_split = pl.per_split;
     p.nsplit = pl.nsplit;
     if (pl.nsplit > 1) {
@@ -267,6 +276,76 @@ lbq_status run_fwd_gemm(const void* X, int m, const lbq_qweight* q, const void* 
         case kInt2: return launch_fwd_kind<kInt2>(pl.nt, p, X, m, q->k, q->packed, q->n, pl.nsplit, st);
         default: return launch_fwd_kind<kCode4>(pl.nt, p, X, m, q->k, q->packed, q->n, pl.nsplit, st);
     }
+}
+
+// One grouped launch of the forward GEMM over g.count problems.
+template <int NT>
+lbq_status launch_fwd_group_nt(const FwdGroupParams& g, bool any_rank, cudaStream_t st) {
+    using C = FwdCfg<NT>;
+    using L = FwdSmem<NT, C::kXStages, C::kXBlocks, C::kWStages, C::kAStages>;
+    auto kern = dqgemm_fwd_grouped_kernel<NT, C::kXStages, C::kXBlocks, C::kWStages, C::kAStages, C::kMinBlocks,
+                                          C::kDqWarps>;
+    const size_t smem = L::total(any_rank ? 1 : 0);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+        return LBQ_ECUDA;
+    kern<<<static_cast<unsigned>(g.cta0[g.count]), fwd_threads(C::kDqWarps), smem, st>>>(g);
+    return last_launch();
+}
+
+template <int NT>
+lbq_status run_fwd_group_nt(int m, const GvJob* jobs, int count, cudaStream_t st) {
+    using C = FwdCfg<NT>;
+    FwdGroupParams g;                                    // passed by value at launch
+    memset(&g, 0, sizeof(g));
+    g.count = count;
+    bool any_rank = false;
+    int cta = 0;
+    for (int i = 0; i < count; ++i) {
+        const GvJob& j = jobs[i];
+        const lbq_qweight* q = j.q;
+        if (!make_map_x3d(&g.tmX[i], j.X, m, q->k, NT, C::kXBlocks)) return LBQ_ECUDA;
+        if (!make_map_2d(&g.tmW[i], q->packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q->n,
+                         static_cast<int64_t>(q->k) * q->bits / 8, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+            return LBQ_ECUDA;
+        g.p[i] = fwd_params(m, q, j.B, j.rank, j.s, j.T, j.Y, j.ldy, j.perm);
+        g.kind[i] = kind_of(q);
+        g.rtiles[i] = static_cast<int>(cdiv(q->n, 128));
+        g.cta0[i] = cta;
+        cta += g.rtiles[i] * static_cast<int>(cdiv(m, NT));
+        any_rank |= j.rank > 0;
+    }
+    g.cta0[count] = cta;
+    return launch_fwd_group_nt<NT>(g, any_rank, st);
+}
+
+// Forward GEMMs with one token count m > 16 (several matrices, or the two
+// halves of channel-mix weights).  When their output tiles together fill the
+// machine's CTA slots they run as grouped launches of up to kFwdMaxGroup
+// problems, without K splits; otherwise one launch each, with the split that
+// fills the machine.
+lbq_status run_fwd_jobs(int m, const GvJob* jobs, int count, void* ws, size_t ws_bytes, int sms, cudaStream_t st) {
+    const int nt = std::min(token_tile(m), 256);
+    const int slots = (nt >= 256 ? 1 : 2) * sms;
+    int64_t tiles = 0;
+    for (int i = 0; i < count; ++i) tiles += cdiv(jobs[i].q->n, 128) * cdiv(m, nt);
+    lbq_status s = LBQ_OK;
+    if (count < 2 || tiles < slots) {
+        for (int i = 0; i < count && s == LBQ_OK; ++i) {
+            const GvJob& j = jobs[i];
+            s = run_fwd_gemm(j.X, m, j.q, j.B, j.rank, j.s, j.T, j.Y, j.ldy, j.perm, ws, ws_bytes, sms, st);
+        }
+        return s;
+    }
+    for (int i = 0; i < count && s == LBQ_OK; i += kFwdMaxGroup) {
+        const int c = std::min(kFwdMaxGroup, count - i);
+        switch (nt) {
+            case 32: s = run_fwd_group_nt<32>(m, jobs + i, c, st); break;
+            case 64: s = run_fwd_group_nt<64>(m, jobs + i, c, st); break;
+            case 128: s = run_fwd_group_nt<128>(m, jobs + i, c, st); break;
+            default: s = run_fwd_group_nt<256>(m, jobs + i, c, st); break;
+        }
+    }
+    return s;
 }
 
 lbq_status check_lora(int rank, const void* A, const void* B, const void* saved) {
@@ -696,26 +775,18 @@ lbq_status lbq_linear_fwd_grouped(int m, const lbq_fwd_problem* probs, int count
         if (pr.rank > 0 && (st = launch_lora_rows<false>(pr.X, m, pr.q->k, pr.A, pr.rank, pr.T_save, cs)) != LBQ_OK)
             return st;
     }
-    if (m > kGemvMaxM) {
-        // large batches: one tensor-core GEMM per matrix, in order, sharing the workspace
-        for (int i = 0; i < count; ++i) {
-            const lbq_fwd_problem& pr = probs[i];
-            if ((st = run_fwd_gemm(pr.X, m, pr.q, pr.B, pr.rank, pr.s, pr.T_save, pr.Y, pr.q->n, nullptr, workspace,
-                                   workspace_bytes, sms, cs)) != LBQ_OK)
-                return st;
-        }
-        return LBQ_OK;
-    }
     std::vector<GvJob> jobs(count);
     for (int i = 0; i < count; ++i) {
         const lbq_fwd_problem& pr = probs[i];
         jobs[i] = GvJob{pr.X, pr.q, pr.B, pr.rank, pr.s, pr.T_save, pr.Y, pr.q->n, nullptr};
     }
+    if (m > kGemvMaxM) return run_fwd_jobs(m, jobs.data(), count, workspace, workspace_bytes, sms, cs);
     return run_gemv_jobs(m, jobs.data(), count, workspace, workspace_bytes, sms, cs);
 }
 
-// Channel-mix: the two halves in one grouped launch (m <= 16) or one GEMM
-// each (m > 16), writing their rows' output columns through perm.
+// Channel-mix: the two halves in one grouped decode launch (m <= 16) or as
+// two tensor-core GEMM jobs (m > 16, grouped when their tiles fill the
+// machine), writing their rows' output columns through perm.
 size_t lbq_linear_fwd_mix_workspace_size(int m, const lbq_qweight_mix* q, int rank) {
     (void)rank;
     if (!q || m < 1) return 0;
@@ -738,16 +809,10 @@ lbq_status lbq_linear_fwd_mix(const void* X, int m, const lbq_qweight_mix* q, co
     if (rank > 0) {
         if ((st = launch_lora_rows<false>(X, m, q->hi.k, A, rank, T_save, cs)) != LBQ_OK) return st;
     }
-    if (m <= kGemvMaxM) {
-        const GvJob jobs[2] = {GvJob{X, &q->hi, B, rank, s, T_save, Y, n_total, q->perm},
-                               GvJob{X, &q->lo, B, rank, s, T_save, Y, n_total, q->perm + q->hi.n}};
-        return run_gemv_jobs(m, jobs, 2, workspace, workspace_bytes, sms, cs);
-    }
-    if ((st = run_fwd_gemm(X, m, &q->hi, B, rank, s, T_save, Y, n_total, q->perm, workspace, workspace_bytes, sms,
-                           cs)) != LBQ_OK)
-        return st;
-    return run_fwd_gemm(X, m, &q->lo, B, rank, s, T_save, Y, n_total, q->perm + q->hi.n, workspace, workspace_bytes,
-                        sms, cs);
+    const GvJob jobs[2] = {GvJob{X, &q->hi, B, rank, s, T_save, Y, n_total, q->perm},
+                           GvJob{X, &q->lo, B, rank, s, T_save, Y, n_total, q->perm + q->hi.n}};
+    if (m <= kGemvMaxM) return run_gemv_jobs(m, jobs, 2, workspace, workspace_bytes, sms, cs);
+    return run_fwd_jobs(m, jobs, 2, workspace, workspace_bytes, sms, cs);
 }
 
 size_t lbq_linear_fwd_mix_grouped_workspace_size(int m, const lbq_mix_problem* probs, int count) {
@@ -791,19 +856,6 @@ lbq_status lbq_linear_fwd_mix_grouped(int m, const lbq_mix_problem* probs, int c
         if (pr.rank > 0 && (st = launch_lora_rows<false>(pr.X, m, pr.q->hi.k, pr.A, pr.rank, pr.T_save, cs)) != LBQ_OK)
             return st;
     }
-    if (m > kGemvMaxM) {
-        for (int i = 0; i < count; ++i) {
-            const lbq_mix_problem& pr = probs[i];
-            const int64_t n_total = static_cast<int64_t>(pr.q->hi.n) + pr.q->lo.n;
-            if ((st = run_fwd_gemm(pr.X, m, &pr.q->hi, pr.B, pr.rank, pr.s, pr.T_save, pr.Y, n_total, pr.q->perm,
-                                   workspace, workspace_bytes, sms, cs)) != LBQ_OK)
-                return st;
-            if ((st = run_fwd_gemm(pr.X, m, &pr.q->lo, pr.B, pr.rank, pr.s, pr.T_save, pr.Y, n_total,
-                                   pr.q->perm + pr.q->hi.n, workspace, workspace_bytes, sms, cs)) != LBQ_OK)
-                return st;
-        }
-        return LBQ_OK;
-    }
     std::vector<GvJob> jobs;
     for (int i = 0; i < count; ++i) {
         const lbq_mix_problem& pr = probs[i];
@@ -811,6 +863,7 @@ lbq_status lbq_linear_fwd_mix_grouped(int m, const lbq_mix_problem* probs, int c
         jobs.push_back(GvJob{pr.X, &pr.q->hi, pr.B, pr.rank, pr.s, pr.T_save, pr.Y, n_total, pr.q->perm});
         jobs.push_back(GvJob{pr.X, &pr.q->lo, pr.B, pr.rank, pr.s, pr.T_save, pr.Y, n_total, pr.q->perm + pr.q->hi.n});
     }
+    if (m > kGemvMaxM) return run_fwd_jobs(m, jobs.data(), static_cast<int>(jobs.size()), workspace, workspace_bytes, sms, cs);
     return run_gemv_jobs(m, jobs.data(), static_cast<int>(jobs.size()), workspace, workspace_bytes, sms, cs);
 }
 

@@ -855,6 +855,44 @@ def test_grouped_fwd_mixed_kinds(lbq, m):
     assert_status_clean(lbq)
 
 
+# Tall weights for the grouped tensor-core launch: together their 128-row
+# tiles fill the B200's CTA slots (296 at the 64-token tile, 148 at 256), so
+# the problems run in one grouped launch instead of one launch each.
+GROUP_TC_CASES = [
+    # n, k, scheme, bits, dq, rank
+    (8704, 256, "minmax", 4, False, 8),
+    (10000, 512, "minmax", 2, False, 0),     # ragged rows
+    (6144, 384, "codebook", 4, True, 16),
+    (4100, 256, "codebook", 4, False, 0),    # ragged rows
+    (9000, 256, "minmax", 4, False, 4),      # far zero points (mixed_weight)
+]
+
+
+@pytest.mark.parametrize("m", [40, 300])
+def test_grouped_fwd_tensor_core_launch(lbq, m):
+    """m > 16 with INT4, INT2 and codebook weights, adapters and ragged row
+    counts in one grouped tensor-core launch (every CTA picks its problem and
+    weight kind); each output against the oracle."""
+    cb = syn.codebook_normal16()
+    tile = 64 if m <= 64 else 256
+    tiles = sum(-(-n // 128) * -(-m // tile) for (n, *_) in GROUP_TC_CASES)
+    assert tiles >= (2 if tile < 256 else 1) * 148          # the grouped path
+    probs, refs = [], []
+    for i, (n, k, scheme, bits, dq, rank) in enumerate(GROUP_TC_CASES):
+        X, W, A, B = fwd_problem(m, n, k, rank, seed=700 + 13 * i + m, scheme=scheme, bits=bits)
+        qw = device_qweight(lbq, W, scheme, bits, dq, cb)
+        s = 2.0
+        probs.append((X.cuda(), qw, None if A is None else A.cuda(), None if B is None else B.cuda(), s))
+        Yr, Tr, Yb = oracle.linear_fwd(syn.bits_u16(X), oracle_weight(W, scheme, bits, dq, cb),
+                                       None if A is None else syn.bits_u16(A), None if B is None else syn.bits_u16(B), s)
+        refs.append((Yr, Yb))
+    outs = lbq.linear_fwd_grouped(probs)
+    torch.cuda.synchronize()
+    for i, ((Y, _), (Yr, Yb)) in enumerate(zip(outs, refs)):
+        assert_within(Y.cpu().numpy(), Yr, Yb, f"Y (problem {i}, M={m})")
+    assert_status_clean(lbq)
+
+
 @pytest.mark.parametrize("m", [3, 40])
 def test_grouped_fwd_more_than_one_launch(lbq, m):
     """Ten weights: two launches of the decode GEMV (m <= 16), or ten
