@@ -522,6 +522,7 @@ def row_training(lbq, syn, torch, peaks, stream):
     m, r, s = 4096, 16, 2.0
     out = {}
     tot_flops = tot_ms = 0.0
+    keep, per = {}, {}
     for i, name in enumerate(("gate", "up", "down")):
         n, k = syn.LLAMA3_8B_SHAPES[name]
         W = syn.weight_bf16(n, k, 0.02, seed=500 + i, device="cuda")
@@ -550,11 +551,30 @@ def row_training(lbq, syn, torch, peaks, stream):
                      "bwd_frac_of_bf16_peak": round(b_fl / b_ms / 1e9 / peaks["bf16_tflops"], 3)}
         tot_flops += f_fl + b_fl + g_fl
         tot_ms += f_ms + b_ms + g_ms
+        per[name] = (f_ms, b_ms, g_ms, f_fl)
+        if name != "down":
+            keep[name] = (qw, X, A, B, dY)
         del qw, X, A, B, dY, Y, T, dX, U, dA, dB
         torch.cuda.empty_cache()
     out["step_TFLOP/s"] = round(tot_flops / tot_ms / 1e9, 1)
     out["step_ms"] = round(tot_ms, 3)
+    # gate and up (the same shape) as one grouped launch for the forward and
+    # one for the backward, as an MLP block runs them
+    fwd_probs = [(keep[nm][1], keep[nm][0], keep[nm][2], keep[nm][3], s) for nm in ("gate", "up")]
+    bwd_probs = [(keep[nm][4], keep[nm][0], keep[nm][2], keep[nm][3], s) for nm in ("gate", "up")]
+    gf_ms = time_graph(torch, lambda: lbq.linear_fwd_grouped(fwd_probs, stream=stream), stream)
+    gb_ms = time_graph(torch, lambda: lbq.linear_bwd_grouped(bwd_probs, stream=stream), stream)
+    fl2 = per["gate"][3] + per["up"][3]
+    out["gate_up_grouped"] = {"fwd_ms": round(gf_ms, 3), "fwd_TFLOP/s": round(fl2 / gf_ms / 1e9, 1),
+                              "fwd_frac_of_bf16_peak": round(fl2 / gf_ms / 1e9 / peaks["bf16_tflops"], 3),
+                              "bwd_ms": round(gb_ms, 3), "bwd_TFLOP/s": round(fl2 / gb_ms / 1e9, 1),
+                              "bwd_frac_of_bf16_peak": round(fl2 / gb_ms / 1e9 / peaks["bf16_tflops"], 3)}
+    step_g = gf_ms + gb_ms + per["down"][0] + per["down"][1] + sum(per[nm][2] for nm in per)
+    out["step_grouped_ms"] = round(step_g, 3)
+    out["step_grouped_TFLOP/s"] = round(tot_flops / step_g / 1e9, 1)
     out["peak_bf16_tflops"] = peaks["bf16_tflops"]
+    del keep, fwd_probs, bwd_probs
+    torch.cuda.empty_cache()
     return out
 
 

@@ -366,6 +366,42 @@ lbq_status lbq_linear_bwd(const void* dY, int m, const lbq_qweight* q,
                           size_t workspace_bytes, lbq_stream_t stream);
 
 /*
+ * Several backward passes with the same token count m in one call (for
+ * example the gate and up projections of an MLP block).  Each problem is one
+ * lbq_linear_bwd: dX_i = dY_i W_i + s_i (dY_i B_i) A_i, with U_i = dY_i B_i
+ * saved when rank_i > 0, with its own gradient, weight, adapter and outputs
+ * (same layouts, rank and alignment rules; `q` is a host pointer to the
+ * descriptor).  After one adapter launch per problem with rank > 0, when the
+ * problems' 128-feature x token tiles together fill the GPU's CTA slots they
+ * run as grouped tensor-core launches of up to 8 problems each, without
+ * channel splits and needing no workspace; otherwise one after the other on
+ * `stream`, each with the split its size calls for, sharing the workspace
+ * (lbq_linear_bwd_grouped_workspace_size bytes, the largest of the
+ * problems' lbq_linear_bwd_workspace_size; zero-filled before its first use,
+ * same reuse rules).  Each dX_i is within the backward's stated bound and
+ * deterministic.  Errors: those of lbq_linear_bwd for any problem, checked
+ * before anything is launched; LBQ_EINVAL for m < 1, count < 1 or a NULL
+ * probs.  (The pages' backward, QLoRA explainer, QLoRA技术原理, applied to a
+ * set of layers.)
+ */
+typedef struct {
+    const void* dY;           /* bf16 [m, q->n], device */
+    const lbq_qweight* q;     /* host pointer to the weight descriptor */
+    const void* A;            /* bf16 [rank, q->k], device, or NULL when rank == 0 */
+    const void* B;            /* bf16 [q->n, rank], device, or NULL when rank == 0 */
+    int32_t rank;             /* 0 .. 64 */
+    float s;                  /* adapter scale */
+    float* dX;                /* fp32 [m, q->k], device */
+    float* U_save;            /* fp32 [m, rank], device, or NULL when rank == 0 */
+} lbq_bwd_problem;
+
+size_t lbq_linear_bwd_grouped_workspace_size(int m, const lbq_bwd_problem* probs,
+                                             int count);
+lbq_status lbq_linear_bwd_grouped(int m, const lbq_bwd_problem* probs, int count,
+                                  void* workspace, size_t workspace_bytes,
+                                  lbq_stream_t stream);
+
+/*
  * Adapter gradients (the only trainable parameters; QLoRA explainer,
  * QLoRA技术原理):
  *   dA = s U^T X  [rank, k]       dB = s dY^T T  [n, rank]      (fp32)

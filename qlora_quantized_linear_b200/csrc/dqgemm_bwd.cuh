@@ -120,10 +120,20 @@ __device__ __forceinline__ uint32_t bwd_a_offset(int c, int fu) {
     return static_cast<uint32_t>((c >> 3) * 2048 + (fu >> 3) * 1024 + row * 128 + ((uu ^ row) << 4));
 }
 
-template <int NT, int KIND, int XS, int WS, int AS, int MINB, int DQW>
-__global__ void __launch_bounds__(fwd_threads(DQW), MINB)
-dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constant__ CUtensorMap tmW,
-                  const BwdParams p) {
+// The output tile a CTA computes: features k0 .. k0 + 127, tokens t0 ..
+// t0 + NT - 1, channel split `split`; `tile` numbers the tile within its
+// GEMM (the split counters), `cta` the CTA within the launch (the rotation of
+// the channel-block walk).
+struct BwdTile {
+    int k0, t0, split;
+    uint32_t tile, cta;
+};
+
+// One CTA of the backward GEMM; tmDY and tmW are the tensor maps of dY and
+// of the packed weight.
+template <int NT, int KIND, int XS, int WS, int AS, int DQW>
+__device__ __forceinline__ void bwd_tile(const CUtensorMap* tmDY, const CUtensorMap* tmW, const BwdParams& p,
+                                         const BwdTile tl) {
     constexpr int BITS = KIND == kInt2 ? 2 : 4;
     using L = BwdSmem<NT, BITS, XS, WS, AS>;
     constexpr int KTB = L::kKTB;
@@ -154,9 +164,9 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
     uint8_t* sUop = smem + L::kLoraT;                  // s*U operand tile [NT x 128 B] (bf16, K-major, SW128)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int k0 = blockIdx.x * 128;
-    const int t0 = blockIdx.y * NT;
-    const int split = blockIdx.z;
+    const int k0 = tl.k0;
+    const int t0 = tl.t0;
+    const int split = tl.split;
     const int cb_total = (p.n + 63) / 64;
     const int cb0 = split * p.cb_per_split;
     const int ncb = min(p.cb_per_split, cb_total - cb0);
@@ -164,7 +174,7 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
     // different blocks (a fixed rotation per CTA), so that a block's scales
     // and zeros and its dY tile are not first requested by all of them at
     // once; the order of the sum over blocks is then fixed per CTA.
-    const int rot = ncb > 0 ? static_cast<int>((static_cast<int64_t>(blockIdx.y * gridDim.x + blockIdx.x) * 37) % ncb) : 0;
+    const int rot = ncb > 0 ? static_cast<int>((static_cast<int64_t>(tl.cta) * 37) % ncb) : 0;
     auto blk = [&](int i) { return cb0 + (i + rot < ncb ? i + rot : i + rot - ncb); };
     // the adapter term s * U A enters the accumulator through rank/16 MMAs
     // before the main loop, in the first split only; its A operand (the rows
@@ -191,8 +201,8 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
     }
     if (KIND == kCode4 && threadIdx.x < 16) s_cb[threadIdx.x] = p.codebook[threadIdx.x];
     if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmDY);
-        tma_prefetch_desc(&tmW);
+        tma_prefetch_desc(tmDY);
+        tma_prefetch_desc(tmW);
     }
     if (warp == 1) {
         tmem_alloc(s_tmem, kTmemCols);
@@ -217,14 +227,14 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
                 if (wi < ncb && (wi < WS || mbar_try_wait(&emptyW[wi % WS], ((wi / WS) - 1) & 1))) {
                     const int w = wi % WS;
                     mbar_arrive_expect_tx(&fullW[w], L::kWBytes);
-                    tma_load_2d(sW + w * L::kWBytes, &tmW, &fullW[w], k0 * BITS / 8, blk(wi) * 64);
+                    tma_load_2d(sW + w * L::kWBytes, tmW, &fullW[w], k0 * BITS / 8, blk(wi) * 64);
                     ++wi;
                     prog = true;
                 }
                 if (xi < ncb && (xi < XS || mbar_try_wait(&emptyX[xi % XS], ((xi / XS) - 1) & 1))) {
                     const int x = xi % XS;
                     mbar_arrive_expect_tx(&fullX[x], L::kXBytes);
-                    tma_load_2d(sX + x * L::kXBytes, &tmDY, &fullX[x], blk(xi) * 64, t0);
+                    tma_load_2d(sX + x * L::kXBytes, tmDY, &fullX[x], blk(xi) * 64, t0);
                     ++xi;
                     prog = true;
                 }
@@ -439,7 +449,7 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
             __threadfence();
             named_barrier_sync(1, 32 * DQW);
             if (threadIdx.x == 64) {
-                const uint32_t tile = blockIdx.y * gridDim.x + blockIdx.x;
+                const uint32_t tile = tl.tile;
                 const uint32_t prev = atomicAdd(p.counters + tile, 1u);
                 const int last = (prev == static_cast<uint32_t>(p.nsplit - 1)) ? 1 : 0;
                 if (last) p.counters[tile] = 0u;   // left at zero for the next call
@@ -476,6 +486,50 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+}
+
+template <int NT, int KIND, int XS, int WS, int AS, int MINB, int DQW>
+__global__ void __launch_bounds__(fwd_threads(DQW), MINB)
+dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constant__ CUtensorMap tmW,
+                  const BwdParams p) {
+    const uint32_t id = blockIdx.y * gridDim.x + blockIdx.x;
+    bwd_tile<NT, KIND, XS, WS, AS, DQW>(&tmDY, &tmW, p, BwdTile{static_cast<int>(blockIdx.x) * 128,
+                                                               static_cast<int>(blockIdx.y) * NT,
+                                                               static_cast<int>(blockIdx.z), id, id});
+}
+
+// A group of backward GEMMs with the same token count in one launch (for
+// example the gate and up projections of an MLP): problem i owns CTAs
+// cta0[i] .. cta0[i+1]-1, feature tiles fastest, then token tiles, and no
+// channel split.  Every CTA runs the kernel above for its problem's weight
+// kind (the launch's shared memory fits the largest kind's layout).
+constexpr int kBwdMaxGroup = 8;
+
+struct BwdGroupParams {
+    CUtensorMap tmDY[kBwdMaxGroup];  // dY of problem i (as for dqgemm_bwd_kernel)
+    CUtensorMap tmW[kBwdMaxGroup];   // packed weight of problem i
+    BwdParams p[kBwdMaxGroup];
+    int kind[kBwdMaxGroup];
+    int ftiles[kBwdMaxGroup];        // 128-feature tiles of problem i
+    int cta0[kBwdMaxGroup + 1];      // first CTA of problem i; cta0[count] = the grid
+    int count;
+};
+
+template <int NT, int XS, int WS, int AS, int MINB, int DQW>
+__global__ void __launch_bounds__(fwd_threads(DQW), MINB)
+dqgemm_bwd_grouped_kernel(const __grid_constant__ BwdGroupParams g) {
+    int i = 0;
+    for (int j = 1; j < g.count; ++j)
+        if (static_cast<int>(blockIdx.x) >= g.cta0[j]) i = j;
+    const int local = static_cast<int>(blockIdx.x) - g.cta0[i];
+    const BwdTile tl{(local % g.ftiles[i]) * 128, (local / g.ftiles[i]) * NT, 0, static_cast<uint32_t>(local),
+                     blockIdx.x};
+    if (g.kind[i] == kInt4)
+        bwd_tile<NT, kInt4, XS, WS, AS, DQW>(&g.tmDY[i], &g.tmW[i], g.p[i], tl);
+    else if (g.kind[i] == kInt2)
+        bwd_tile<NT, kInt2, XS, WS, AS, DQW>(&g.tmDY[i], &g.tmW[i], g.p[i], tl);
+    else
+        bwd_tile<NT, kCode4, XS, WS, AS, DQW>(&g.tmDY[i], &g.tmW[i], g.p[i], tl);
 }
 
 }  // namespace lbq

@@ -391,6 +391,100 @@ lbq_status launch_bwd_kind(int nt, const BwdParams& p, const void* dY, const uin
     }
 }
 
+// The kernel arguments of one backward GEMM, without a channel split.
+BwdParams bwd_params(int m, const lbq_qweight* q, const void* A, int rank, float s, const float* U, float* dX) {
+    BwdParams p{};
+    p.m = m;
+    p.n = q->n;
+    p.k = q->k;
+    p.bits = q->bits;
+    p.ngroups = q->k / q->group;
+    p.group = q->group;
+    p.scale = q->scale;
+    p.zero = q->zero;
+    p.absmax = q->absmax;
+    p.q8 = (q->scheme == LBQ_CODEBOOK4 && q->double_quant) ? q->absmax_q8 : nullptr;
+    p.s2 = q->absmax_s2;
+    p.offset = q->absmax_offset;
+    p.codebook = q->codebook;
+    p.rank = rank;
+    p.rank_pad = rank > 0 ? (rank + 15) / 16 * 16 : 16;
+    p.s = s;
+    p.U = U;
+    p.A = static_cast<const uint16_t*>(A);
+    p.dX = dX;
+    p.cb_per_split = static_cast<int>(cdiv(q->n, 64));
+    p.nsplit = 1;
+    return p;
+}
+
+// One backward GEMM (the adapter's U already computed), with the channel
+// split its plan gives.
+lbq_status run_bwd_gemm(const void* dY, int m, const lbq_qweight* q, const void* A, int rank, float s, const float* U,
+                        float* dX, void* ws, int sms, cudaStream_t st) {
+    const Plan pl = plan_gemm(m, q->k, cdiv(q->n, 64), sms, 256);
+    BwdParams p = bwd_params(m, q, A, rank, s, U, dX);
+    p.cb_per_split = pl.per_split;
+    p.nsplit = pl.nsplit;
+    if (pl.nsplit > 1) {
+        if (!ws) return LBQ_EWORKSPACE;
+        if (pl.tiles > kMaxSplitTiles) return LBQ_EUNSUPPORTED;
+        p.partial = ws_partials(ws);
+        p.counters = ws_counters(ws);
+    }
+    switch (kind_of(q)) {
+        case kInt4: return launch_bwd_kind<kInt4>(pl.nt, p, dY, q->packed, st);
+        case kInt2: return launch_bwd_kind<kInt2>(pl.nt, p, dY, q->packed, st);
+        default: return launch_bwd_kind<kCode4>(pl.nt, p, dY, q->packed, st);
+    }
+}
+
+// One grouped launch of the backward GEMM over `count` problems.
+template <int NT>
+lbq_status run_bwd_group_nt(int m, const lbq_bwd_problem* probs, int count, cudaStream_t st) {
+    using C = BwdCfg<NT>;
+    BwdGroupParams g;                                    // passed by value at launch
+    memset(&g, 0, sizeof(g));
+    g.count = count;
+    size_t smem = 0;
+    int cta = 0;
+    for (int i = 0; i < count; ++i) {
+        const lbq_bwd_problem& pr = probs[i];
+        const lbq_qweight* q = pr.q;
+        const bool int2 = kind_of(q) == kInt2;
+        const int ktb = 128 * (int2 ? 2 : 4) / 8;        // packed bytes of a channel row across a feature tile
+        if (!make_map_2d(&g.tmDY[i], pr.dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, m, q->n, NT, 64,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
+            return LBQ_ECUDA;
+        if (!make_map_2d(&g.tmW[i], q->packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q->n,
+                         static_cast<int64_t>(q->k) * (int2 ? 2 : 4) / 8, 64, ktb, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return LBQ_ECUDA;
+        g.p[i] = bwd_params(m, q, pr.A, pr.rank, pr.s, pr.U_save, pr.dX);
+        g.kind[i] = kind_of(q);
+        g.ftiles[i] = static_cast<int>(cdiv(q->k, 128));
+        g.cta0[i] = cta;
+        cta += g.ftiles[i] * static_cast<int>(cdiv(m, NT));
+        smem = std::max(smem, int2 ? BwdSmem<NT, 2, C::kXStages, C::kWStages, C::kAStages>::total(g.p[i].rank_pad)
+                                   : BwdSmem<NT, 4, C::kXStages, C::kWStages, C::kAStages>::total(g.p[i].rank_pad));
+    }
+    g.cta0[count] = cta;
+    auto kern = dqgemm_bwd_grouped_kernel<NT, C::kXStages, C::kWStages, C::kAStages, C::kMinBlocks, C::kDqWarps>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+        return LBQ_ECUDA;
+    kern<<<static_cast<unsigned>(cta), fwd_threads(C::kDqWarps), smem, st>>>(g);
+    return last_launch();
+}
+
+// Checks of one backward problem (as lbq_linear_bwd's).
+lbq_status check_bwd(const void* dY, int m, const lbq_qweight* q, const void* A, const void* B, int rank,
+                     const float* dX, const float* U_save) {
+    lbq_status st = check_qweight(q, true);
+    if (st != LBQ_OK) return st;
+    if (m < 1 || !dY || !dX || q->n % 8 != 0) return LBQ_EINVAL;
+    if (!aligned16(dY) || !aligned16(dX)) return LBQ_EALIGN;
+    return check_lora(rank, A, B, U_save);
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -876,51 +970,74 @@ size_t lbq_linear_bwd_workspace_size(int m, const lbq_qweight* q, int rank) {
 lbq_status lbq_linear_bwd(const void* dY, int m, const lbq_qweight* q, const void* A, const void* B, int rank,
                           float s, float* dX, float* U_save, void* workspace, size_t workspace_bytes,
                           lbq_stream_t stream) {
-    lbq_status st = check_qweight(q, true);
+    lbq_status st = check_bwd(dY, m, q, A, B, rank, dX, U_save);
     if (st != LBQ_OK) return st;
-    if (m < 1 || !dY || !dX || q->n % 8 != 0) return LBQ_EINVAL;
-    if (!aligned16(dY) || !aligned16(dX)) return LBQ_EALIGN;
-    if ((st = check_lora(rank, A, B, U_save)) != LBQ_OK) return st;
     const int sms = sm_count();
-    const Plan pl = plan_gemm(m, q->k, cdiv(q->n, 64), sms, 256);
-    if (pl.workspace() > 0 && (!workspace || workspace_bytes < pl.workspace())) return LBQ_EWORKSPACE;
-    if (pl.workspace() > 0 && !aligned16(workspace)) return LBQ_EALIGN;
+    const size_t need = plan_gemm(m, q->k, cdiv(q->n, 64), sms, 256).workspace();
+    if (need > 0 && (!workspace || workspace_bytes < need)) return LBQ_EWORKSPACE;
+    if (need > 0 && !aligned16(workspace)) return LBQ_EALIGN;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     if (rank > 0) {
         if ((st = launch_lora_rows<true>(dY, m, q->n, B, rank, U_save, cs)) != LBQ_OK) return st;
     }
-    BwdParams p{};
-    p.m = m;
-    p.n = q->n;
-    p.k = q->k;
-    p.bits = q->bits;
-    p.ngroups = q->k / q->group;
-    p.group = q->group;
-    p.scale = q->scale;
-    p.zero = q->zero;
-    p.absmax = q->absmax;
-    p.q8 = (q->scheme == LBQ_CODEBOOK4 && q->double_quant) ? q->absmax_q8 : nullptr;
-    p.s2 = q->absmax_s2;
-    p.offset = q->absmax_offset;
-    p.codebook = q->codebook;
-    p.rank = rank;
-    p.rank_pad = rank > 0 ? (rank + 15) / 16 * 16 : 16;
-    p.s = s;
-    p.U = U_save;
-    p.A = static_cast<const uint16_t*>(A);
-    p.dX = dX;
-    p.cb_per_split = pl.per_split;
-    p.nsplit = pl.nsplit;
-    if (pl.nsplit > 1) {
-        if (pl.tiles > kMaxSplitTiles) return LBQ_EUNSUPPORTED;
-        p.partial = ws_partials(workspace);
-        p.counters = ws_counters(workspace);
+    return run_bwd_gemm(dY, m, q, A, rank, s, U_save, dX, workspace, sms, cs);
+}
+
+size_t lbq_linear_bwd_grouped_workspace_size(int m, const lbq_bwd_problem* probs, int count) {
+    if (m < 1 || !probs || count < 1) return 0;
+    const int sms = sm_count();
+    size_t need = 0;
+    for (int i = 0; i < count; ++i) {
+        if (check_qweight(probs[i].q, false) != LBQ_OK) return 0;
+        need = std::max(need, plan_gemm(m, probs[i].q->k, cdiv(probs[i].q->n, 64), sms, 256).workspace());
     }
-    switch (kind_of(q)) {
-        case kInt4: return launch_bwd_kind<kInt4>(pl.nt, p, dY, q->packed, cs);
-        case kInt2: return launch_bwd_kind<kInt2>(pl.nt, p, dY, q->packed, cs);
-        default: return launch_bwd_kind<kCode4>(pl.nt, p, dY, q->packed, cs);
+    return need;
+}
+
+lbq_status lbq_linear_bwd_grouped(int m, const lbq_bwd_problem* probs, int count, void* workspace,
+                                  size_t workspace_bytes, lbq_stream_t stream) {
+    if (m < 1 || !probs || count < 1) return LBQ_EINVAL;
+    lbq_status st;
+    for (int i = 0; i < count; ++i) {
+        const lbq_bwd_problem& pr = probs[i];
+        if ((st = check_bwd(pr.dY, m, pr.q, pr.A, pr.B, pr.rank, pr.dX, pr.U_save)) != LBQ_OK) return st;
     }
+    const int sms = sm_count();
+    const int nt = std::min(token_tile(m), 256);
+    const int slots = (nt >= 256 ? 1 : 2) * sms;
+    int64_t tiles = 0;
+    for (int i = 0; i < count; ++i) tiles += cdiv(probs[i].q->k, 128) * cdiv(m, nt);
+    const bool grouped = count >= 2 && tiles >= slots;
+    const size_t need = grouped ? 0 : lbq_linear_bwd_grouped_workspace_size(m, probs, count);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return LBQ_EWORKSPACE;
+    if (need > 0 && !aligned16(workspace)) return LBQ_EALIGN;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    for (int i = 0; i < count; ++i) {
+        const lbq_bwd_problem& pr = probs[i];
+        if (pr.rank > 0 && (st = launch_lora_rows<true>(pr.dY, m, pr.q->n, pr.B, pr.rank, pr.U_save, cs)) != LBQ_OK)
+            return st;
+    }
+    if (!grouped) {
+        // too few tiles to fill the GPU together: one launch each, with its split
+        for (int i = 0; i < count; ++i) {
+            const lbq_bwd_problem& pr = probs[i];
+            if ((st = run_bwd_gemm(pr.dY, m, pr.q, pr.A, pr.rank, pr.s, pr.U_save, pr.dX, workspace, sms, cs)) != LBQ_OK)
+                return st;
+        }
+        return LBQ_OK;
+    }
+    for (int i = 0; i < count; i += kBwdMaxGroup) {
+        const int c = std::min(kBwdMaxGroup, count - i);
+        switch (nt) {
+            case 16: st = run_bwd_group_nt<16>(m, probs + i, c, cs); break;
+            case 32: st = run_bwd_group_nt<32>(m, probs + i, c, cs); break;
+            case 64: st = run_bwd_group_nt<64>(m, probs + i, c, cs); break;
+            case 128: st = run_bwd_group_nt<128>(m, probs + i, c, cs); break;
+            default: st = run_bwd_group_nt<256>(m, probs + i, c, cs); break;
+        }
+        if (st != LBQ_OK) return st;
+    }
+    return LBQ_OK;
 }
 
 lbq_status lbq_lora_grads(const void* X, const void* dY, int m, int n, int k, const float* T, const float* U,

@@ -53,6 +53,12 @@ class lbq_fwd_problem(ctypes.Structure):
                 ("Y", ctypes.c_void_p), ("T_save", ctypes.c_void_p)]
 
 
+class lbq_bwd_problem(ctypes.Structure):
+    _fields_ = [("dY", ctypes.c_void_p), ("q", ctypes.POINTER(lbq_qweight)), ("A", ctypes.c_void_p),
+                ("B", ctypes.c_void_p), ("rank", ctypes.c_int32), ("s", ctypes.c_float),
+                ("dX", ctypes.c_void_p), ("U_save", ctypes.c_void_p)]
+
+
 class lbq_mix_problem(ctypes.Structure):
     _fields_ = [("X", ctypes.c_void_p), ("q", ctypes.POINTER(lbq_qweight_mix)), ("A", ctypes.c_void_p),
                 ("B", ctypes.c_void_p), ("rank", ctypes.c_int32), ("s", ctypes.c_float),
@@ -62,6 +68,7 @@ class lbq_mix_problem(ctypes.Structure):
 _vp, _int, _f32, _sz, _u32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.POINTER(ctypes.c_uint32)
 _QP, _MP = ctypes.POINTER(lbq_qweight), ctypes.POINTER(lbq_qweight_mix)
 _PP, _QPP, _I64P = ctypes.POINTER(lbq_fwd_problem), ctypes.POINTER(ctypes.POINTER(lbq_qweight)), ctypes.POINTER(ctypes.c_int64)
+_BPP = ctypes.POINTER(lbq_bwd_problem)
 _MPP = ctypes.POINTER(lbq_mix_problem)
 _SIGS = {
     "lbq_status_string": (ctypes.c_char_p, [_int]),
@@ -81,6 +88,8 @@ _SIGS = {
     "lbq_gemv_plan": (_int, [_int, _QPP, _int, _int, _I64P, _I64P]),
     "lbq_linear_fwd_grouped_workspace_size": (_sz, [_int, _PP, _int]),
     "lbq_linear_fwd_grouped": (_int, [_int, _PP, _int, _vp, _sz, _vp]),
+    "lbq_linear_bwd_grouped_workspace_size": (_sz, [_int, _BPP, _int]),
+    "lbq_linear_bwd_grouped": (_int, [_int, _BPP, _int, _vp, _sz, _vp]),
     "lbq_unmerge_lora": (_int, [_vp, _int, _int, _vp, _vp, _int, _f32, _vp, _vp]),
     "lbq_linear_fwd_noalloc_reset": (_int, [_vp]),
     "lbq_channel_mix_select_workspace_size": (_sz, [_int, _int]),
@@ -119,6 +128,8 @@ lbq_merge_lora = _L.lbq_merge_lora
 lbq_gemv_plan = _L.lbq_gemv_plan
 lbq_linear_fwd_grouped_workspace_size = _L.lbq_linear_fwd_grouped_workspace_size
 lbq_linear_fwd_grouped = _L.lbq_linear_fwd_grouped
+lbq_linear_bwd_grouped_workspace_size = _L.lbq_linear_bwd_grouped_workspace_size
+lbq_linear_bwd_grouped = _L.lbq_linear_bwd_grouped
 lbq_unmerge_lora = _L.lbq_unmerge_lora
 lbq_linear_fwd_noalloc_reset = _L.lbq_linear_fwd_noalloc_reset
 lbq_channel_mix_select_workspace_size = _L.lbq_channel_mix_select_workspace_size
@@ -378,6 +389,35 @@ def linear_bwd(dY, qw, A=None, B=None, s: float = 0.0, dX=None, U=None, workspac
     _check(lbq_linear_bwd(dY.data_ptr(), m, ctypes.byref(qw.struct), _ptr(A), _ptr(B), rank, float(s), dX.data_ptr(),
                           _ptr(U), _ptr(workspace), nws, _stream(stream)), "lbq_linear_bwd")
     return dX, U
+
+
+def linear_bwd_grouped(problems, workspace=None, stream=None):
+    """Several backward passes with the same token count in one call.
+    `problems` is a list of (dY, qw) or (dY, qw, A, B, s) tuples; returns the
+    list of (dX, U) as linear_bwd would."""
+    torch = _torch()
+    arr = (lbq_bwd_problem * len(problems))()
+    outs, keep = [], []
+    m = None
+    for i, pr in enumerate(problems):
+        dY, qw = _bf16_2d(pr[0], "dY"), pr[1]
+        A, B, s = (pr[2], pr[3], pr[4]) if len(pr) > 2 else (None, None, 0.0)
+        m = dY.shape[0] if m is None else m
+        if dY.shape[0] != m:
+            raise ValueError("all problems of a grouped call have the same token count")
+        rank = 0 if A is None else int(A.shape[0])
+        dX = torch.empty((m, qw.k), dtype=torch.float32, device=dY.device)
+        U = torch.empty((m, rank), dtype=torch.float32, device=dY.device) if rank else None
+        arr[i] = lbq_bwd_problem(dY=dY.data_ptr(), q=ctypes.pointer(qw.struct), A=_ptr(A), B=_ptr(B), rank=rank,
+                                 s=float(s), dX=dX.data_ptr(), U_save=_ptr(U))
+        outs.append((dX, U))
+        keep.append((dY, A, B))
+    nws = lbq_linear_bwd_grouped_workspace_size(m, arr, len(problems))
+    if workspace is None:
+        workspace = _workspace(nws, problems[0][0].device)
+    _check(lbq_linear_bwd_grouped(m, arr, len(problems), _ptr(workspace), nws, _stream(stream)),
+           "lbq_linear_bwd_grouped")
+    return outs
 
 
 def lora_grads(X, dY, T, U, s: float, dA=None, dB=None, stream=None):

@@ -132,6 +132,26 @@ def test_grouped_entry_points_reject_bad_arguments():
     nop = lbq.lbq_qweight_mix(hi=hi, lo=lo, perm=None)
     M[1].q = ctypes.pointer(nop)
     assert gm(4, M, 2, None, 0, None) == lbq.LBQ_EINVAL
+    # the grouped backward: the same checks as lbq_linear_bwd, before any launch
+    D = (lbq.lbq_bwd_problem * 2)()
+    for i in range(2):
+        D[i] = lbq.lbq_bwd_problem(dY=0x4000, q=ctypes.pointer(q), A=None, B=None, rank=0, s=0.0, dX=0x5000,
+                                   U_save=None)
+    gb = lbq.lbq_linear_bwd_grouped
+    assert gb(4, D, 0, None, 0, None) == lbq.LBQ_EINVAL
+    assert gb(4, None, 2, None, 0, None) == lbq.LBQ_EINVAL
+    assert gb(0, D, 2, None, 0, None) == lbq.LBQ_EINVAL
+    D[1].dX = 0x5004
+    assert gb(4, D, 2, None, 0, None) == lbq.LBQ_EALIGN
+    D[1].dX = 0x5000
+    D[1].rank = 8                                              # rank > 0 needs A, B and U_save
+    assert gb(4, D, 2, None, 0, None) == lbq.LBQ_EINVAL
+    D[1].rank = 0
+    odd = _qw(n=100)                                           # n must be a multiple of 8
+    D[1].q = ctypes.pointer(odd)
+    assert gb(4, D, 2, None, 0, None) == lbq.LBQ_EINVAL
+    D[1].q = ctypes.pointer(q)
+    assert lbq.lbq_linear_bwd_grouped_workspace_size(0, D, 2) == 0
     # the workspace queries are host-only and cover both halves of every problem
     M[1].q = ctypes.pointer(mix)
     assert lbq.lbq_linear_fwd_mix_grouped_workspace_size(0, M, 2) == 0

@@ -946,6 +946,49 @@ def test_linear_bwd_codebook_parity(lbq, m, n, k, rank, dq):
     assert_status_clean(lbq)
 
 
+# Wide weights for the grouped backward: at M = 300 (two 256-token tiles)
+# their 128-feature tiles fill the B200's 148 CTA slots together.
+GROUP_BWD_CASES = [
+    # n, k, scheme, bits, dq, rank
+    (512, 4096, "minmax", 4, False, 16),
+    (264, 3072, "minmax", 2, False, 0),
+    (256, 2048, "codebook", 4, True, 8),
+    (136, 1536, "minmax", 4, False, 0),      # far zero points (mixed_weight)
+]
+
+
+@pytest.mark.parametrize("m", [40, 300])
+def test_grouped_bwd(lbq, m):
+    """Several backward passes in one call: at M = 300 one grouped tensor-core
+    launch (every CTA picks its problem and weight kind), at M = 40 (too few
+    tiles) one launch each; dX and U against the oracle."""
+    cb = syn.codebook_normal16()
+    tiles = sum(-(-k // 128) for (_, k, *_) in GROUP_BWD_CASES) * -(-m // 256)
+    assert (tiles >= 148) == (m == 300)                        # which path each case takes
+    probs, refs = [], []
+    for i, (n, k, scheme, bits, dq, rank) in enumerate(GROUP_BWD_CASES):
+        X, W, A, B = fwd_problem(m, n, k, rank, seed=800 + 11 * i + m, scheme=scheme, bits=bits)
+        dY = syn.normal_bf16((m, n), 0.1, seed=900 + i + m)
+        qw = device_qweight(lbq, W, scheme, bits, dq, cb)
+        s = 2.0
+        probs.append((dY.cuda(), qw, None if A is None else A.cuda(), None if B is None else B.cuda(), s))
+        What = oracle_weight(W, scheme, bits, dq, cb)
+        dXr, Ur, dXb = oracle.linear_bwd(syn.bits_u16(dY), What, None if A is None else syn.bits_u16(A),
+                                         None if B is None else syn.bits_u16(B), s)
+        Ub = None
+        if rank:
+            Ub = np.abs(oracle.bf16_to_f32(syn.bits_u16(dY))).astype(np.float64) @ \
+                np.abs(oracle.bf16_to_f32(syn.bits_u16(B))).astype(np.float64)
+        refs.append((dXr, dXb, Ur, Ub))
+    outs = lbq.linear_bwd_grouped(probs)
+    torch.cuda.synchronize()
+    for i, ((dX, U), (dXr, dXb, Ur, Ub)) in enumerate(zip(outs, refs)):
+        assert_within(dX.cpu().numpy(), dXr, dXb, f"dX (problem {i}, M={m})")
+        if Ub is not None:
+            assert_within(U.cpu().numpy(), Ur, Ub, f"U (problem {i}, M={m})")
+    assert_status_clean(lbq)
+
+
 def test_codebook70b_backward_full_size_sampled(lbq, codebook70b):
     """dX = dY W_hat through the 70B attention projection (8192 x 8192,
     codebook + double quantization) at M = 2048: 2048 seeded elements plus a
