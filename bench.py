@@ -50,6 +50,7 @@ def parse_args():
     ap.add_argument("--case", default=None,
                     help="run one kernel configuration `reps` times and exit (for ncu captures): "
                          "decode_<matrix>_m<M> | layerset_8b_m<M> | train_<matrix>_{fwd,bwd,grads} | "
+                         "traingrp_gateup_{fwd,bwd} | "
                          "codebook70b_<matrix>_m<M> | quantize_<matrix>_{int4,codebook} | merge_<matrix>_r16 | "
                          "select_<matrix>_q")
     ap.add_argument("--reps", type=int, default=3)
@@ -872,6 +873,22 @@ def run_case(args):
             fn = {"fwd": lambda: lbq.linear_fwd(X, qw, A, B, s),
                   "bwd": lambda: lbq.linear_bwd(dY, qw, A, B, s),
                   "grads": lambda: lbq.lora_grads(X, dY, T, U, s)}[arg]
+    elif kind == "traingrp":
+        # gate and up at M = 4096, rank 16, as one grouped call (arg: fwd or bwd)
+        m, r, s = 4096, 16, 2.0
+        fwd_p, bwd_p = [], []
+        for i, nm in enumerate(("gate", "up")):
+            n, k = syn.LLAMA3_8B_SHAPES[nm]
+            W = syn.weight_bf16(n, k, 0.02, seed=1 + i, outlier_frac=0.001, device="cuda")
+            qw = lbq.QuantizedWeight(n, k, "minmax", 4).quantize(W)
+            del W
+            X = syn.normal_bf16((m, k), 1.0, seed=2 + i, device="cuda")
+            A = syn.normal_bf16((r, k), 0.01, seed=3 + i, device="cuda")
+            B = syn.normal_bf16((n, r), 0.01, seed=4 + i, device="cuda")
+            dY = syn.normal_bf16((m, n), 0.1, seed=5 + i, device="cuda")
+            fwd_p.append((X, qw, A, B, s))
+            bwd_p.append((dY, qw, A, B, s))
+        fn = {"fwd": lambda: lbq.linear_fwd_grouped(fwd_p), "bwd": lambda: lbq.linear_bwd_grouped(bwd_p)}[arg]
     elif kind == "codebook70b":
         n, k = syn.LLAMA3_70B_SHAPES[name]
         W = syn.weight_bf16(n, k, 0.015, seed=1, device="cuda")
