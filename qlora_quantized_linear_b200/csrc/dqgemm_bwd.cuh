@@ -122,11 +122,10 @@ __device__ __forceinline__ uint32_t bwd_a_offset(int c, int fu) {
 
 // The output tile a CTA computes: features k0 .. k0 + 127, tokens t0 ..
 // t0 + NT - 1, channel split `split`; `tile` numbers the tile within its
-// GEMM (the split counters), `cta` the CTA within the launch (the rotation of
-// the channel-block walk).
+// GEMM (the split counters).
 struct BwdTile {
     int k0, t0, split;
-    uint32_t tile, cta;
+    uint32_t tile;
 };
 
 // One CTA of the backward GEMM; tmDY and tmW are the tensor maps of dY and
@@ -170,11 +169,12 @@ __device__ __forceinline__ void bwd_tile(const CUtensorMap* tmDY, const CUtensor
     const int cb_total = (p.n + 63) / 64;
     const int cb0 = split * p.cb_per_split;
     const int ncb = min(p.cb_per_split, cb_total - cb0);
-    // The CTAs of a wave start their walk over the channel blocks at
-    // different blocks (a fixed rotation per CTA), so that a block's scales
-    // and zeros and its dY tile are not first requested by all of them at
-    // once; the order of the sum over blocks is then fixed per CTA.
-    const int rot = ncb > 0 ? static_cast<int>((static_cast<int64_t>(tl.cta) * 37) % ncb) : 0;
+    // The token tiles start their walk over the channel blocks at different
+    // blocks (a fixed rotation per token tile), so that a block's scales and
+    // zeros are not first requested by all CTAs of a wave at once, while the
+    // CTAs of one token tile, which read the same dY tiles, walk together;
+    // the order of the sum over blocks is then fixed per tile.
+    const int rot = ncb > 0 ? static_cast<int>((static_cast<int64_t>(t0 / NT) * 37) % ncb) : 0;
     auto blk = [&](int i) { return cb0 + (i + rot < ncb ? i + rot : i + rot - ncb); };
     // the adapter term s * U A enters the accumulator through rank/16 MMAs
     // before the main loop, in the first split only; its A operand (the rows
@@ -495,7 +495,7 @@ dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constan
     const uint32_t id = blockIdx.y * gridDim.x + blockIdx.x;
     bwd_tile<NT, KIND, XS, WS, AS, DQW>(&tmDY, &tmW, p, BwdTile{static_cast<int>(blockIdx.x) * 128,
                                                                static_cast<int>(blockIdx.y) * NT,
-                                                               static_cast<int>(blockIdx.z), id, id});
+                                                               static_cast<int>(blockIdx.z), id});
 }
 
 // A group of backward GEMMs with the same token count in one launch (for
@@ -522,8 +522,7 @@ dqgemm_bwd_grouped_kernel(const __grid_constant__ BwdGroupParams g) {
     for (int j = 1; j < g.count; ++j)
         if (static_cast<int>(blockIdx.x) >= g.cta0[j]) i = j;
     const int local = static_cast<int>(blockIdx.x) - g.cta0[i];
-    const BwdTile tl{(local % g.ftiles[i]) * 128, (local / g.ftiles[i]) * NT, 0, static_cast<uint32_t>(local),
-                     blockIdx.x};
+    const BwdTile tl{(local % g.ftiles[i]) * 128, (local / g.ftiles[i]) * NT, 0, static_cast<uint32_t>(local)};
     if (g.kind[i] == kInt4)
         bwd_tile<NT, kInt4, XS, WS, AS, DQW>(&g.tmDY[i], &g.tmW[i], g.p[i], tl);
     else if (g.kind[i] == kInt2)
