@@ -55,8 +55,10 @@ struct FwdParams {
     int64_t ldy;
     const int32_t* perm;         // stored row -> output column (NULL = identity)
     int kb_per_split;            // k-blocks of 64 per split
-    int nsplit;
-    float* partial;              // [nsplit, m, n] fp32 (nsplit > 1)
+    int nsplit;                  // splits of every tile of this launch
+    int tile0;                   // first tile of this launch (tiles numbered row tile fastest)
+    int rtiles;                  // 128-row tiles of the GEMM
+    float* partial;              // [tile - tile0][nsplit][NT tokens][128 rows] fp32 (nsplit > 1)
     uint32_t* counters;          // [tiles] (nsplit > 1), zero between calls
 };
 
@@ -658,9 +660,10 @@ __device__ __forceinline__ void fwd_tile(const CUtensorMap* tmX, const CUtensorM
 #pragma unroll
             for (int j = 0; j < 16; ++j) acc[j] = __uint_as_float(raw[j]);
             if (splitk) {
+                float* dst = p.partial + ((static_cast<int64_t>(tl.tile - p.tile0) * p.nsplit + split) * NT + jj) * 128 + row;
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
-                    if (jj + j < mt) p.partial[(static_cast<int64_t>(split) * p.m + t0 + jj + j) * p.n + grow] = acc[j];
+                    if (jj + j < mt) dst[j * 128] = acc[j];
                 continue;
             }
 #pragma unroll
@@ -686,10 +689,11 @@ __device__ __forceinline__ void fwd_tile(const CUtensorMap* tmX, const CUtensorM
 #pragma unroll
                     for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
                     for (int sp = 0; sp < p.nsplit; ++sp) {
-                        const float* src = p.partial + (static_cast<int64_t>(sp) * p.m + t0 + jj) * p.n + grow;
+                        const float* src =
+                            p.partial + ((static_cast<int64_t>(tl.tile - p.tile0) * p.nsplit + sp) * NT + jj) * 128 + row;
                         float part[16];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) part[j] = (jj + j < mt) ? __ldcg(src + static_cast<int64_t>(j) * p.n) : 0.0f;
+                        for (int j = 0; j < 16; ++j) part[j] = (jj + j < mt) ? __ldcg(src + j * 128) : 0.0f;
 #pragma unroll
                         for (int j = 0; j < 16; ++j) acc[j] += part[j];
                     }
@@ -714,10 +718,13 @@ template <int NT, int KIND, int XS, int XB, int WS, int AS, int MINB, int DQW>
 __global__ void __launch_bounds__(fwd_threads(DQW), MINB)
 dqgemm_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                   const FwdParams p) {
-    const uint32_t id = blockIdx.y * gridDim.x + blockIdx.x;
-    fwd_tile<NT, KIND, XS, XB, WS, AS, DQW>(&tmX, &tmW, p, FwdTile{static_cast<int>(blockIdx.x) * 128,
-                                                                  static_cast<int>(blockIdx.y) * NT,
-                                                                  static_cast<int>(blockIdx.z), id, id});
+    // a one-dimensional grid: nsplit consecutive CTAs per tile, tiles from
+    // tile0 on, row tile fastest
+    const int lin = p.tile0 + static_cast<int>(blockIdx.x) / p.nsplit;
+    const int split = static_cast<int>(blockIdx.x) % p.nsplit;
+    fwd_tile<NT, KIND, XS, XB, WS, AS, DQW>(&tmX, &tmW, p,
+                                            FwdTile{(lin % p.rtiles) * 128, (lin / p.rtiles) * NT, split,
+                                                    static_cast<uint32_t>(lin), static_cast<uint32_t>(lin)});
 }
 
 // A group of forward GEMMs with the same token count in one launch (several

@@ -56,8 +56,10 @@ struct BwdParams {
     const uint16_t* A;           // [rank, k] bf16
     float* dX;                   // [m, k]
     int cb_per_split;            // blocks of 64 output channels per split
-    int nsplit;
-    float* partial;              // [nsplit, m, k]
+    int nsplit;                  // splits of every tile of this launch
+    int tile0;                   // first tile of this launch (tiles numbered feature tile fastest)
+    int ftiles;                  // 128-feature tiles of the GEMM
+    float* partial;              // [tile - tile0][nsplit][NT tokens][128 lanes] fp32 (nsplit > 1)
     uint32_t* counters;
 };
 
@@ -436,9 +438,10 @@ __device__ __forceinline__ void bwd_tile(const CUtensorMap* tmDY, const CUtensor
 #pragma unroll
             for (int j = 0; j < 16; ++j) acc[j] = __uint_as_float(raw[j]);
             if (splitk) {
+                float* dst = p.partial + ((static_cast<int64_t>(tl.tile - p.tile0) * p.nsplit + split) * NT + jj) * 128 + lrow;
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
-                    if (jj + j < mt) p.partial[(static_cast<int64_t>(split) * p.m + t0 + jj + j) * p.k + kcol] = acc[j];
+                    if (jj + j < mt) dst[j * 128] = acc[j];
                 continue;
             }
 #pragma unroll
@@ -463,12 +466,11 @@ __device__ __forceinline__ void bwd_tile(const CUtensorMap* tmDY, const CUtensor
 #pragma unroll
                     for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
                     for (int sp = 0; sp < p.nsplit; ++sp) {
+                        const float* src =
+                            p.partial + ((static_cast<int64_t>(tl.tile - p.tile0) * p.nsplit + sp) * NT + jj) * 128 + lrow;
                         float part[16];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            part[j] = (jj + j < mt)
-                                          ? __ldcg(p.partial + (static_cast<int64_t>(sp) * p.m + t0 + jj + j) * p.k + kcol)
-                                          : 0.0f;
+                        for (int j = 0; j < 16; ++j) part[j] = (jj + j < mt) ? __ldcg(src + j * 128) : 0.0f;
 #pragma unroll
                         for (int j = 0; j < 16; ++j) acc[j] += part[j];
                     }
@@ -492,10 +494,13 @@ template <int NT, int KIND, int XS, int WS, int AS, int MINB, int DQW>
 __global__ void __launch_bounds__(fwd_threads(DQW), MINB)
 dqgemm_bwd_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constant__ CUtensorMap tmW,
                   const BwdParams p) {
-    const uint32_t id = blockIdx.y * gridDim.x + blockIdx.x;
-    bwd_tile<NT, KIND, XS, WS, AS, DQW>(&tmDY, &tmW, p, BwdTile{static_cast<int>(blockIdx.x) * 128,
-                                                               static_cast<int>(blockIdx.y) * NT,
-                                                               static_cast<int>(blockIdx.z), id});
+    // a one-dimensional grid: nsplit consecutive CTAs per tile, tiles from
+    // tile0 on, feature tile fastest
+    const int lin = p.tile0 + static_cast<int>(blockIdx.x) / p.nsplit;
+    const int split = static_cast<int>(blockIdx.x) % p.nsplit;
+    bwd_tile<NT, KIND, XS, WS, AS, DQW>(&tmDY, &tmW, p,
+                                        BwdTile{(lin % p.ftiles) * 128, (lin / p.ftiles) * NT, split,
+                                                static_cast<uint32_t>(lin)});
 }
 
 // A group of backward GEMMs with the same token count in one launch (for

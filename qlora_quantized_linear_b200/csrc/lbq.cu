@@ -138,31 +138,6 @@ constexpr int kMaxSplitTiles = static_cast<int>(kCounterHeader / sizeof(uint32_t
 inline uint32_t* ws_counters(void* ws) { return static_cast<uint32_t*>(ws); }
 inline float* ws_partials(void* ws) { return reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kCounterHeader); }
 
-struct Plan {
-    int nt;          // token tile
-    int tiles;       // output tiles (rows x token tiles)
-    int nsplit;      // K splits
-    int per_split;   // reduction blocks per split
-    size_t partial_bytes;
-    size_t workspace() const { return nsplit > 1 ? kCounterHeader + partial_bytes : 0; }
-};
-
-// Token tile, output tiles and K splits of one GEMM.  When the output tiles
-// alone cannot fill the CTA slots of the machine (decode sizes), the
-// reduction is split so that all CTAs fit in one wave.
-Plan plan_gemm(int m, int64_t out_rows, int64_t red_blocks, int sms, int max_nt = 256, int align = 1) {
-    Plan pl;
-    pl.nt = std::min(token_tile(m), max_nt);
-    pl.tiles = static_cast<int>(cdiv(out_rows, 128) * cdiv(m, pl.nt));
-    const int slots = (pl.nt >= 256 ? 1 : 2) * sms;
-    pl.nsplit = 1;
-    if (pl.tiles < slots) pl.nsplit = static_cast<int>(std::min<int64_t>(red_blocks, std::max(1, slots / pl.tiles)));
-    pl.per_split = static_cast<int>(cdiv(cdiv(red_blocks, pl.nsplit), align) * align);
-    pl.nsplit = static_cast<int>(cdiv(red_blocks, pl.per_split));
-    pl.partial_bytes = round_up(static_cast<size_t>(pl.nsplit) * m * out_rows * sizeof(float), 256);
-    return pl;
-}
-
 // Streams on which the last library call was a quantization: the forward
 // that follows on such a stream reads the weight only after that kernel has
 // finished.  Any other forward may stream the packed weight while the kernel
@@ -182,21 +157,76 @@ bool weights_stable(cudaStream_t st) {
 
 #include "dqgemv_host.cuh"
 
-// Forward plan of the tensor-core GEMM (m > 16): splits start on a whole
-// weight chunk (128 bytes of a row).
-Plan plan_fwd(int m, const lbq_qweight* q, int sms) {
-    return plan_gemm(m, q->n, q->k / 64, sms, 256, q->bits == 2 ? 8 : 4);
+// Plan of a tensor-core GEMM (forward: 128-row output tiles, reduction over
+// k/64 blocks; backward: 128-feature tiles, reduction over n/64 channel
+// blocks), m > 16 or the backward at any m.  Tiles are numbered output tile
+// fastest, then token tile.  When the tiles alone cannot fill the CTA slots, every tile's
+// reduction is split so that all CTAs fit in one wave (required).  When they
+// fill several waves and the last holds a quarter to a half of the slots,
+// the full waves run unsplit and the tiles of the last wave are split over
+// the idle slots in a second launch, if their partial sums fit `ws_budget`
+// bytes of workspace (optional: 512 tiles on 148 slots take 3.5 waves
+// instead of 4; a last wave of a few tiles split many ways measured slower,
+// as the fixed cost of each CTA and the partial sums outweigh the gain).
+// Splits start on a multiple of `align` blocks (the forward's weight chunk);
+// the partial sums are [tile - first split tile][split][NT tokens][128] fp32.
+struct TilePlan {
+    int nt = 0, tiles = 0, rtiles = 0;
+    int nsplit = 1, per_split = 0;       // splits of every tile
+    int tail0 = 0, tail_split = 1, tail_per = 0;   // tiles tail0 .. tiles - 1, split tail_split ways
+    size_t partial_bytes = 0;
+    bool split() const { return nsplit > 1 || tail_split > 1; }
+    size_t workspace() const { return split() ? kCounterHeader + partial_bytes : 0; }
+};
+
+TilePlan plan_tiles(int m, int64_t out_rows, int64_t red, int align, int sms, size_t ws_budget) {
+    TilePlan pl;
+    pl.nt = std::min(token_tile(m), 256);
+    pl.rtiles = static_cast<int>(cdiv(out_rows, 128));
+    pl.tiles = static_cast<int>(pl.rtiles * cdiv(m, pl.nt));
+    pl.per_split = static_cast<int>(red);
+    const int slots = (pl.nt >= 256 ? 1 : 2) * sms;
+    auto per_for = [&](int64_t ns) { return static_cast<int>(cdiv(cdiv(red, ns), align) * align); };
+    auto bytes_for = [&](int64_t tiles, int ns) {
+        return round_up(static_cast<size_t>(tiles) * ns * pl.nt * 128 * sizeof(float), 256);
+    };
+    if (pl.tiles < slots) {
+        pl.per_split = per_for(std::min<int64_t>(red, std::max(1, slots / pl.tiles)));
+        pl.nsplit = static_cast<int>(cdiv(red, pl.per_split));
+        if (pl.nsplit > 1) pl.partial_bytes = bytes_for(pl.tiles, pl.nsplit);
+        return pl;
+    }
+    const int full = pl.tiles / slots * slots, tail = pl.tiles - full;
+    if (2 * tail > slots || 4 * tail < slots || pl.tiles > kMaxSplitTiles) return pl;
+    const int per = per_for(slots / tail);
+    const int ns = static_cast<int>(cdiv(red, per));
+    if (ns < 2 || kCounterHeader + bytes_for(tail, ns) > ws_budget) return pl;
+    pl.tail0 = full;
+    pl.tail_split = ns;
+    pl.tail_per = per;
+    pl.partial_bytes = bytes_for(tail, ns);
+    return pl;
 }
 
-// Workspace of one forward call (either path).
-size_t fwd_workspace(int m, const lbq_qweight* q, int sms) {
+TilePlan plan_fwd(int m, const lbq_qweight* q, int sms, size_t ws_budget = ~size_t(0)) {
+    return plan_tiles(m, q->n, q->k / 64, q->bits == 2 ? 8 : 4, sms, ws_budget);
+}
+
+TilePlan plan_bwd(int m, const lbq_qweight* q, int sms, size_t ws_budget = ~size_t(0)) {
+    return plan_tiles(m, q->k, cdiv(q->n, 64), 1, sms, ws_budget);
+}
+
+// Workspace of one forward call (either path): with ws_budget = 0 the part
+// that a call requires, unbounded the size that also lets it split the tiles
+// of its last wave (what the size queries report).
+size_t fwd_workspace(int m, const lbq_qweight* q, int sms, size_t ws_budget = ~size_t(0)) {
     if (m <= kGemvMaxM) return gemv_jobs_workspace(m, &q, 1, sms);
-    return plan_fwd(m, q, sms).workspace();
+    return plan_fwd(m, q, sms, ws_budget).workspace();
 }
 
 template <int NT, int KIND>
 lbq_status launch_fwd_nt(const FwdParams& p, const void* X, int m, int64_t k, const uint8_t* packed, int nrows,
-                         int nsplit, cudaStream_t st) {
+                         int nctas, cudaStream_t st) {
     using C = FwdCfg<NT>;
     using L = FwdSmem<NT, C::kXStages, C::kXBlocks, C::kWStages, C::kAStages>;
     auto kern = dqgemm_fwd_kernel<NT, KIND, C::kXStages, C::kXBlocks, C::kWStages, C::kAStages, C::kMinBlocks,
@@ -209,20 +239,20 @@ lbq_status launch_fwd_nt(const FwdParams& p, const void* X, int m, int64_t k, co
     if (!make_map_2d(&tmW, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, nrows, k * (KIND == kInt2 ? 2 : 4) / 8, 128, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B))
         return LBQ_ECUDA;
-    dim3 grid(static_cast<unsigned>(cdiv(nrows, 128)), static_cast<unsigned>(cdiv(m, NT)), static_cast<unsigned>(nsplit));
-    kern<<<grid, fwd_threads(C::kDqWarps), smem, st>>>(tmX, tmW, p);
+    (void)m;
+    kern<<<static_cast<unsigned>(nctas), fwd_threads(C::kDqWarps), smem, st>>>(tmX, tmW, p);
     return last_launch();
 }
 
 template <int KIND>
 lbq_status launch_fwd_kind(int nt, const FwdParams& p, const void* X, int m, int64_t k, const uint8_t* packed,
-                           int nrows, int nsplit, cudaStream_t st) {
+                           int nrows, int nctas, cudaStream_t st) {
     switch (nt) {
-        case 16: return launch_fwd_nt<16, KIND>(p, X, m, k, packed, nrows, nsplit, st);
-        case 32: return launch_fwd_nt<32, KIND>(p, X, m, k, packed, nrows, nsplit, st);
-        case 64: return launch_fwd_nt<64, KIND>(p, X, m, k, packed, nrows, nsplit, st);
-        case 128: return launch_fwd_nt<128, KIND>(p, X, m, k, packed, nrows, nsplit, st);
-        default: return launch_fwd_nt<256, KIND>(p, X, m, k, packed, nrows, nsplit, st);
+        case 16: return launch_fwd_nt<16, KIND>(p, X, m, k, packed, nrows, nctas, st);
+        case 32: return launch_fwd_nt<32, KIND>(p, X, m, k, packed, nrows, nctas, st);
+        case 64: return launch_fwd_nt<64, KIND>(p, X, m, k, packed, nrows, nctas, st);
+        case 128: return launch_fwd_nt<128, KIND>(p, X, m, k, packed, nrows, nctas, st);
+        default: return launch_fwd_nt<256, KIND>(p, X, m, k, packed, nrows, nctas, st);
     }
 }
 
@@ -261,21 +291,33 @@ lbq_status run_fwd_gemm(const void* X, int m, const lbq_qweight* q, const void* 
         const GvJob job{X, q, B, rank, s, T, Y, ldy, perm};
         return run_gemv_jobs(m, &job, 1, ws, ws_bytes, sms, st);
     }
-    const Plan pl = plan_fwd(m, q, sms);
+    const TilePlan pl = plan_fwd(m, q, sms, ws && aligned16(ws) ? ws_bytes : 0);
     FwdParams p = fwd_params(m, q, B, rank, s, T, Y, ldy, perm);
-    p.kb_per_split = pl.per_split;
-    p.nsplit = pl.nsplit;
-    if (pl.nsplit > 1) {
+    p.rtiles = pl.rtiles;
+    if (pl.split()) {
         if (!ws) return LBQ_EWORKSPACE;
         if (pl.tiles > kMaxSplitTiles) return LBQ_EUNSUPPORTED;
         p.partial = ws_partials(ws);
         p.counters = ws_counters(ws);
     }
-    switch (kind_of(q)) {
-        case kInt4: return launch_fwd_kind<kInt4>(pl.nt, p, X, m, q->k, q->packed, q->n, pl.nsplit, st);
-        case kInt2: return launch_fwd_kind<kInt2>(pl.nt, p, X, m, q->k, q->packed, q->n, pl.nsplit, st);
-        default: return launch_fwd_kind<kCode4>(pl.nt, p, X, m, q->k, q->packed, q->n, pl.nsplit, st);
-    }
+    auto launch = [&](const FwdParams& lp, int nctas) {
+        switch (kind_of(q)) {
+            case kInt4: return launch_fwd_kind<kInt4>(pl.nt, lp, X, m, q->k, q->packed, q->n, nctas, st);
+            case kInt2: return launch_fwd_kind<kInt2>(pl.nt, lp, X, m, q->k, q->packed, q->n, nctas, st);
+            default: return launch_fwd_kind<kCode4>(pl.nt, lp, X, m, q->k, q->packed, q->n, nctas, st);
+        }
+    };
+    p.kb_per_split = pl.per_split;
+    p.nsplit = pl.nsplit;
+    if (pl.tail_split <= 1) return launch(p, pl.tiles * pl.nsplit);
+    // the full waves unsplit, then the last wave's tiles split over the slots
+    lbq_status r = launch(p, pl.tail0);
+    if (r != LBQ_OK) return r;
+    FwdParams t = p;
+    t.tile0 = pl.tail0;
+    t.nsplit = pl.tail_split;
+    t.kb_per_split = pl.tail_per;
+    return launch(t, (pl.tiles - pl.tail0) * pl.tail_split);
 }
 
 // One grouped launch of the forward GEMM over g.count problems.
@@ -360,7 +402,7 @@ lbq_status check_lora(int rank, const void* A, const void* B, const void* saved)
 // backward GEMM
 // ---------------------------------------------------------------------------
 template <int NT, int KIND>
-lbq_status launch_bwd_nt(const BwdParams& p, const void* dY, const uint8_t* packed, cudaStream_t st) {
+lbq_status launch_bwd_nt(const BwdParams& p, const void* dY, const uint8_t* packed, int nctas, cudaStream_t st) {
     constexpr int BITS = KIND == kInt2 ? 2 : 4;
     using C = BwdCfg<NT>;
     using L = BwdSmem<NT, BITS, C::kXStages, C::kWStages, C::kAStages>;
@@ -374,20 +416,19 @@ lbq_status launch_bwd_nt(const BwdParams& p, const void* dY, const uint8_t* pack
     if (!make_map_2d(&tmW, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, p.n, static_cast<int64_t>(p.k) * BITS / 8, 64,
                      L::kKTB, CU_TENSOR_MAP_SWIZZLE_NONE))
         return LBQ_ECUDA;
-    dim3 grid(static_cast<unsigned>(cdiv(p.k, 128)), static_cast<unsigned>(cdiv(p.m, NT)),
-              static_cast<unsigned>(p.nsplit));
-    kern<<<grid, fwd_threads(C::kDqWarps), smem, st>>>(tmDY, tmW, p);
+    kern<<<static_cast<unsigned>(nctas), fwd_threads(C::kDqWarps), smem, st>>>(tmDY, tmW, p);
     return last_launch();
 }
 
 template <int KIND>
-lbq_status launch_bwd_kind(int nt, const BwdParams& p, const void* dY, const uint8_t* packed, cudaStream_t st) {
+lbq_status launch_bwd_kind(int nt, const BwdParams& p, const void* dY, const uint8_t* packed, int nctas,
+                           cudaStream_t st) {
     switch (nt) {
-        case 16: return launch_bwd_nt<16, KIND>(p, dY, packed, st);
-        case 32: return launch_bwd_nt<32, KIND>(p, dY, packed, st);
-        case 64: return launch_bwd_nt<64, KIND>(p, dY, packed, st);
-        case 128: return launch_bwd_nt<128, KIND>(p, dY, packed, st);
-        default: return launch_bwd_nt<256, KIND>(p, dY, packed, st);
+        case 16: return launch_bwd_nt<16, KIND>(p, dY, packed, nctas, st);
+        case 32: return launch_bwd_nt<32, KIND>(p, dY, packed, nctas, st);
+        case 64: return launch_bwd_nt<64, KIND>(p, dY, packed, nctas, st);
+        case 128: return launch_bwd_nt<128, KIND>(p, dY, packed, nctas, st);
+        default: return launch_bwd_nt<256, KIND>(p, dY, packed, nctas, st);
     }
 }
 
@@ -421,22 +462,34 @@ BwdParams bwd_params(int m, const lbq_qweight* q, const void* A, int rank, float
 // One backward GEMM (the adapter's U already computed), with the channel
 // split its plan gives.
 lbq_status run_bwd_gemm(const void* dY, int m, const lbq_qweight* q, const void* A, int rank, float s, const float* U,
-                        float* dX, void* ws, int sms, cudaStream_t st) {
-    const Plan pl = plan_gemm(m, q->k, cdiv(q->n, 64), sms, 256);
+                        float* dX, void* ws, size_t ws_bytes, int sms, cudaStream_t st) {
+    const TilePlan pl = plan_bwd(m, q, sms, ws && aligned16(ws) ? ws_bytes : 0);
     BwdParams p = bwd_params(m, q, A, rank, s, U, dX);
-    p.cb_per_split = pl.per_split;
-    p.nsplit = pl.nsplit;
-    if (pl.nsplit > 1) {
+    p.ftiles = pl.rtiles;
+    if (pl.split()) {
         if (!ws) return LBQ_EWORKSPACE;
         if (pl.tiles > kMaxSplitTiles) return LBQ_EUNSUPPORTED;
         p.partial = ws_partials(ws);
         p.counters = ws_counters(ws);
     }
-    switch (kind_of(q)) {
-        case kInt4: return launch_bwd_kind<kInt4>(pl.nt, p, dY, q->packed, st);
-        case kInt2: return launch_bwd_kind<kInt2>(pl.nt, p, dY, q->packed, st);
-        default: return launch_bwd_kind<kCode4>(pl.nt, p, dY, q->packed, st);
-    }
+    auto launch = [&](const BwdParams& lp, int nctas) {
+        switch (kind_of(q)) {
+            case kInt4: return launch_bwd_kind<kInt4>(pl.nt, lp, dY, q->packed, nctas, st);
+            case kInt2: return launch_bwd_kind<kInt2>(pl.nt, lp, dY, q->packed, nctas, st);
+            default: return launch_bwd_kind<kCode4>(pl.nt, lp, dY, q->packed, nctas, st);
+        }
+    };
+    p.cb_per_split = pl.per_split;
+    p.nsplit = pl.nsplit;
+    if (pl.tail_split <= 1) return launch(p, pl.tiles * pl.nsplit);
+    // the full waves unsplit, then the last wave's tiles split over the slots
+    lbq_status r = launch(p, pl.tail0);
+    if (r != LBQ_OK) return r;
+    BwdParams t = p;
+    t.tile0 = pl.tail0;
+    t.nsplit = pl.tail_split;
+    t.cb_per_split = pl.tail_per;
+    return launch(t, (pl.tiles - pl.tail0) * pl.tail_split);
 }
 
 // One grouped launch of the backward GEMM over `count` problems.
@@ -590,13 +643,14 @@ lbq_status launch_lora_colgrad(const void* in, int64_t m, int64_t ncols, const f
 
 namespace {
 
-// The workspace of a channel-mix forward (both halves).
-size_t mix_workspace(int m, const lbq_qweight_mix* q, int sms) {
+// The workspace of a channel-mix forward (both halves); ws_budget as for
+// fwd_workspace.
+size_t mix_workspace(int m, const lbq_qweight_mix* q, int sms, size_t ws_budget = ~size_t(0)) {
     if (m <= kGemvMaxM) {
         const lbq_qweight* qs[2] = {&q->hi, &q->lo};
         return gemv_jobs_workspace(m, qs, 2, sms);
     }
-    return std::max(plan_fwd(m, &q->hi, sms).workspace(), plan_fwd(m, &q->lo, sms).workspace());
+    return std::max(plan_fwd(m, &q->hi, sms, ws_budget).workspace(), plan_fwd(m, &q->lo, sms, ws_budget).workspace());
 }
 
 // Validation of one channel-mix problem's descriptor, activations and outputs.
@@ -800,7 +854,7 @@ lbq_status lbq_linear_fwd(const void* X, int m, const lbq_qweight* q, const void
     if (!aligned16(X) || !aligned16(Y)) return LBQ_EALIGN;
     if ((st = check_lora(rank, A, B, T_save)) != LBQ_OK) return st;
     const int sms = sm_count();
-    const size_t need = fwd_workspace(m, q, sms);
+    const size_t need = fwd_workspace(m, q, sms, 0);
     if (need > 0 && (!workspace || workspace_bytes < need)) return LBQ_EWORKSPACE;
     if (need > 0 && !aligned16(workspace)) return LBQ_EALIGN;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
@@ -818,10 +872,10 @@ lbq_status lbq_linear_fwd_noalloc(const void* X, int m, const lbq_qweight* q, co
     if (!aligned16(X) || !aligned16(Y)) return LBQ_EALIGN;
     if ((st = check_lora(rank, A, B, T_save)) != LBQ_OK) return st;
     const int sms = sm_count();
-    const size_t need = fwd_workspace(m, q, sms);
+    const size_t need = fwd_workspace(m, q, sms, 0);
     if (need > kNoAllocScratchBytes) return LBQ_EWORKSPACE;  // this call's scratch does not fit
     void* scratch = nullptr;
-    if (need > 0 && (st = noalloc_scratch_address(&scratch)) != LBQ_OK) return st;
+    if ((st = noalloc_scratch_address(&scratch)) != LBQ_OK) return st;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     if (rank > 0) {
         if ((st = launch_lora_rows<false>(X, m, q->k, A, rank, T_save, cs)) != LBQ_OK) return st;
@@ -829,7 +883,8 @@ lbq_status lbq_linear_fwd_noalloc(const void* X, int m, const lbq_qweight* q, co
     return run_fwd_gemm(X, m, q, B, rank, s, T_save, Y, q->n, nullptr, scratch, kNoAllocScratchBytes, sms, cs);
 }
 
-size_t lbq_linear_fwd_grouped_workspace_size(int m, const lbq_fwd_problem* probs, int count) {
+// Workspace of a grouped forward; ws_budget as for fwd_workspace.
+static size_t grouped_fwd_workspace(int m, const lbq_fwd_problem* probs, int count, size_t ws_budget) {
     if (m < 1 || !probs || count < 1) return 0;
     const int sms = sm_count();
     if (m <= kGemvMaxM) {
@@ -843,9 +898,13 @@ size_t lbq_linear_fwd_grouped_workspace_size(int m, const lbq_fwd_problem* probs
     size_t need = 0;
     for (int i = 0; i < count; ++i) {
         if (check_qweight(probs[i].q, false) != LBQ_OK) return 0;
-        need = std::max(need, plan_fwd(m, probs[i].q, sms).workspace());
+        need = std::max(need, plan_fwd(m, probs[i].q, sms, ws_budget).workspace());
     }
     return need;
+}
+
+size_t lbq_linear_fwd_grouped_workspace_size(int m, const lbq_fwd_problem* probs, int count) {
+    return grouped_fwd_workspace(m, probs, count, ~size_t(0));
 }
 
 lbq_status lbq_linear_fwd_grouped(int m, const lbq_fwd_problem* probs, int count, void* workspace,
@@ -859,7 +918,7 @@ lbq_status lbq_linear_fwd_grouped(int m, const lbq_fwd_problem* probs, int count
         if (!aligned16(pr.X) || !aligned16(pr.Y)) return LBQ_EALIGN;
         if ((st = check_lora(pr.rank, pr.A, pr.B, pr.T_save)) != LBQ_OK) return st;
     }
-    const size_t need = lbq_linear_fwd_grouped_workspace_size(m, probs, count);
+    const size_t need = grouped_fwd_workspace(m, probs, count, 0);
     if (need > 0 && (!workspace || workspace_bytes < need)) return LBQ_EWORKSPACE;
     if (need > 0 && !aligned16(workspace)) return LBQ_EALIGN;
     const int sms = sm_count();
@@ -895,7 +954,7 @@ lbq_status lbq_linear_fwd_mix(const void* X, int m, const lbq_qweight_mix* q, co
     if ((st = check_mix(q, m, X, Y)) != LBQ_OK) return st;
     if ((st = check_lora(rank, A, B, T_save)) != LBQ_OK) return st;
     const int sms = sm_count();
-    const size_t need = mix_workspace(m, q, sms);
+    const size_t need = mix_workspace(m, q, sms, 0);
     if (need > 0 && (!workspace || workspace_bytes < need)) return LBQ_EWORKSPACE;
     if (need > 0 && !aligned16(workspace)) return LBQ_EALIGN;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
@@ -909,7 +968,8 @@ lbq_status lbq_linear_fwd_mix(const void* X, int m, const lbq_qweight_mix* q, co
     return run_fwd_jobs(m, jobs, 2, workspace, workspace_bytes, sms, cs);
 }
 
-size_t lbq_linear_fwd_mix_grouped_workspace_size(int m, const lbq_mix_problem* probs, int count) {
+// Workspace of a grouped channel-mix forward; ws_budget as for fwd_workspace.
+static size_t mix_grouped_workspace(int m, const lbq_mix_problem* probs, int count, size_t ws_budget) {
     if (m < 1 || !probs || count < 1) return 0;
     const int sms = sm_count();
     if (m <= kGemvMaxM) {
@@ -926,9 +986,13 @@ size_t lbq_linear_fwd_mix_grouped_workspace_size(int m, const lbq_mix_problem* p
     for (int i = 0; i < count; ++i) {
         const lbq_qweight_mix* q = probs[i].q;
         if (!q || check_qweight(&q->hi, false) != LBQ_OK || check_qweight(&q->lo, false) != LBQ_OK) return 0;
-        need = std::max(need, mix_workspace(m, q, sms));
+        need = std::max(need, mix_workspace(m, q, sms, ws_budget));
     }
     return need;
+}
+
+size_t lbq_linear_fwd_mix_grouped_workspace_size(int m, const lbq_mix_problem* probs, int count) {
+    return mix_grouped_workspace(m, probs, count, ~size_t(0));
 }
 
 lbq_status lbq_linear_fwd_mix_grouped(int m, const lbq_mix_problem* probs, int count, void* workspace,
@@ -940,7 +1004,7 @@ lbq_status lbq_linear_fwd_mix_grouped(int m, const lbq_mix_problem* probs, int c
         if ((st = check_mix(pr.q, m, pr.X, pr.Y)) != LBQ_OK) return st;
         if ((st = check_lora(pr.rank, pr.A, pr.B, pr.T_save)) != LBQ_OK) return st;
     }
-    const size_t need = lbq_linear_fwd_mix_grouped_workspace_size(m, probs, count);
+    const size_t need = mix_grouped_workspace(m, probs, count, 0);
     if (need > 0 && (!workspace || workspace_bytes < need)) return LBQ_EWORKSPACE;
     if (need > 0 && !aligned16(workspace)) return LBQ_EALIGN;
     const int sms = sm_count();
@@ -964,7 +1028,7 @@ lbq_status lbq_linear_fwd_mix_grouped(int m, const lbq_mix_problem* probs, int c
 size_t lbq_linear_bwd_workspace_size(int m, const lbq_qweight* q, int rank) {
     (void)rank;
     if (m < 1 || check_qweight(q, false) != LBQ_OK) return 0;
-    return plan_gemm(m, q->k, cdiv(q->n, 64), sm_count(), 256).workspace();
+    return plan_bwd(m, q, sm_count()).workspace();
 }
 
 lbq_status lbq_linear_bwd(const void* dY, int m, const lbq_qweight* q, const void* A, const void* B, int rank,
@@ -973,14 +1037,14 @@ lbq_status lbq_linear_bwd(const void* dY, int m, const lbq_qweight* q, const voi
     lbq_status st = check_bwd(dY, m, q, A, B, rank, dX, U_save);
     if (st != LBQ_OK) return st;
     const int sms = sm_count();
-    const size_t need = plan_gemm(m, q->k, cdiv(q->n, 64), sms, 256).workspace();
+    const size_t need = plan_bwd(m, q, sms, 0).workspace();
     if (need > 0 && (!workspace || workspace_bytes < need)) return LBQ_EWORKSPACE;
     if (need > 0 && !aligned16(workspace)) return LBQ_EALIGN;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     if (rank > 0) {
         if ((st = launch_lora_rows<true>(dY, m, q->n, B, rank, U_save, cs)) != LBQ_OK) return st;
     }
-    return run_bwd_gemm(dY, m, q, A, rank, s, U_save, dX, workspace, sms, cs);
+    return run_bwd_gemm(dY, m, q, A, rank, s, U_save, dX, workspace, workspace_bytes, sms, cs);
 }
 
 size_t lbq_linear_bwd_grouped_workspace_size(int m, const lbq_bwd_problem* probs, int count) {
@@ -989,7 +1053,7 @@ size_t lbq_linear_bwd_grouped_workspace_size(int m, const lbq_bwd_problem* probs
     size_t need = 0;
     for (int i = 0; i < count; ++i) {
         if (check_qweight(probs[i].q, false) != LBQ_OK) return 0;
-        need = std::max(need, plan_gemm(m, probs[i].q->k, cdiv(probs[i].q->n, 64), sms, 256).workspace());
+        need = std::max(need, plan_bwd(m, probs[i].q, sms).workspace());
     }
     return need;
 }
@@ -1008,7 +1072,8 @@ lbq_status lbq_linear_bwd_grouped(int m, const lbq_bwd_problem* probs, int count
     int64_t tiles = 0;
     for (int i = 0; i < count; ++i) tiles += cdiv(probs[i].q->k, 128) * cdiv(m, nt);
     const bool grouped = count >= 2 && tiles >= slots;
-    const size_t need = grouped ? 0 : lbq_linear_bwd_grouped_workspace_size(m, probs, count);
+    size_t need = 0;                                     // what the launches one by one require
+    for (int i = 0; !grouped && i < count; ++i) need = std::max(need, plan_bwd(m, probs[i].q, sms, 0).workspace());
     if (need > 0 && (!workspace || workspace_bytes < need)) return LBQ_EWORKSPACE;
     if (need > 0 && !aligned16(workspace)) return LBQ_EALIGN;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
@@ -1021,7 +1086,8 @@ lbq_status lbq_linear_bwd_grouped(int m, const lbq_bwd_problem* probs, int count
         // too few tiles to fill the GPU together: one launch each, with its split
         for (int i = 0; i < count; ++i) {
             const lbq_bwd_problem& pr = probs[i];
-            if ((st = run_bwd_gemm(pr.dY, m, pr.q, pr.A, pr.rank, pr.s, pr.U_save, pr.dX, workspace, sms, cs)) != LBQ_OK)
+            if ((st = run_bwd_gemm(pr.dY, m, pr.q, pr.A, pr.rank, pr.s, pr.U_save, pr.dX, workspace, workspace_bytes, sms,
+                                   cs)) != LBQ_OK)
                 return st;
         }
         return LBQ_OK;
