@@ -188,7 +188,11 @@ lbq_status lbq_unmerge_lora(const void* W, int n, int k, const void* A,
  * (the compute dtype) inside the kernel and products accumulate in fp32.
  * workspace: lbq_linear_fwd_workspace_size(m, q, rank) bytes of device memory,
  * zero-filled before the first call that uses it; NULL is accepted when that
- * size is 0.  It holds split-K partial sums and per-tile arrival counters;
+ * size is 0.  It holds split-K partial sums and per-tile arrival counters.
+ * For m > 16 the size includes the partial sums of an optional split of the
+ * GEMM's last wave of tiles: a smaller workspace is accepted as long as it
+ * holds what the call requires (the last wave then runs unsplit, with the
+ * same results within the stated bound);
  * every call leaves the counters at zero again, so one zero-fill at
  * allocation serves any number of later calls of any shape.  After a call
  * whose kernels timed out (LBQ_ETIMEOUT from lbq_device_status), zero it
@@ -243,10 +247,11 @@ lbq_status lbq_linear_fwd(const void* X, int m, const lbq_qweight* q,
  * (The source pages have no counterpart of this entry point.)
  *
  * Arguments, layouts, results and errors are those of lbq_linear_fwd, plus:
- *  - LBQ_EWORKSPACE when this call's scratch (lbq_linear_fwd_workspace_size)
- *    is larger than the 8 MiB array; nothing is launched then.  Shapes whose
- *    split-K scratch exceeds the array (large n or k with many token tiles)
- *    are refused this way; lbq_linear_fwd_workspace_size tells in advance.
+ *  - LBQ_EWORKSPACE when the scratch this call requires is larger than the
+ *    8 MiB array; nothing is launched then (for m <= 16 it is
+ *    lbq_linear_fwd_workspace_size, which tells in advance; for m > 16 that
+ *    query may report more, for an optional split of the last wave of tiles
+ *    that the call then leaves out when it does not fit).
  *  - Every call looks up the array's device address with the current device
  *    current; the first call on a device may load the library's module, so
  *    make it before any stream capture.
