@@ -5,6 +5,8 @@ dequantized weights.  GEMM outputs: within the stated bound
 |dY| <= 2^-7 * sum_k |x_k| |w_eff,k| + 1e-6 (w_eff = W_hat plus the adapter
 term), computed by the oracle for every element.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -986,6 +988,38 @@ def test_grouped_bwd(lbq, m):
         assert_within(dX.cpu().numpy(), dXr, dXb, f"dX (problem {i}, M={m})")
         if Ub is not None:
             assert_within(U.cpu().numpy(), Ur, Ub, f"U (problem {i}, M={m})")
+    assert_status_clean(lbq)
+
+
+@pytest.mark.parametrize("scheme,bits", [("minmax", 4), ("minmax", 2), ("codebook", 4)])
+def test_last_wave_split(lbq, scheme, bits):
+    """The GEMMs' split of the last wave: at M = 300 (two 256-token tiles)
+    93 output (or feature) tiles make 186 tiles, 148 in a full wave and 38 in
+    the last, which a second launch splits over the idle SMs; every element of
+    Y and dX against the oracle."""
+    m, r, s = 300, 16, 2.0
+    cb = syn.codebook_normal16()
+    # forward: 93 row tiles (k = 1024 so that INT2, split on 8-block chunks, splits too)
+    n, k = 93 * 128, 1024
+    X, W, A, B = fwd_problem(m, n, k, r, seed=31 + bits, scheme=scheme, bits=bits)
+    qw = device_qweight(lbq, W, scheme, bits, scheme == "codebook", cb)
+    assert lbq.lbq_linear_fwd_workspace_size(m, ctypes.byref(qw.struct), r) > 0     # the split is planned
+    Y, _ = lbq.linear_fwd(X.cuda(), qw, A.cuda(), B.cuda(), s)
+    torch.cuda.synchronize()
+    What = oracle_weight(W, scheme, bits, scheme == "codebook", cb)
+    Yr, _, Yb = oracle.linear_fwd(syn.bits_u16(X), What, syn.bits_u16(A), syn.bits_u16(B), s)
+    assert_within(Y.cpu().numpy(), Yr, Yb, f"Y ({scheme} {bits}-bit, last wave split)")
+    # backward: 93 feature tiles
+    n, k = 256, 93 * 128
+    X, W, A, B = fwd_problem(m, n, k, r, seed=41 + bits, scheme=scheme, bits=bits)
+    dY = syn.normal_bf16((m, n), 0.1, seed=51 + bits)
+    qw = device_qweight(lbq, W, scheme, bits, scheme == "codebook", cb)
+    assert lbq.lbq_linear_bwd_workspace_size(m, ctypes.byref(qw.struct), r) > 0
+    dX, _ = lbq.linear_bwd(dY.cuda(), qw, A.cuda(), B.cuda(), s)
+    torch.cuda.synchronize()
+    What = oracle_weight(W, scheme, bits, scheme == "codebook", cb)
+    dXr, _, dXb = oracle.linear_bwd(syn.bits_u16(dY), What, syn.bits_u16(A), syn.bits_u16(B), s)
+    assert_within(dX.cpu().numpy(), dXr, dXb, f"dX ({scheme} {bits}-bit, last wave split)")
     assert_status_clean(lbq)
 
 
